@@ -1,0 +1,184 @@
+/*
+ * psispec.h -- C ABI of the B200 (sm_100a) Psi-Spec verification library, libpsispec.so.
+ *
+ * The operation is the lossless rejection-correction step of Uno's Psi-Spec sampler,
+ * "Unlocking Lossless Speedups in LLMs via Discrete Diffusion" (arXiv 2609.04010). The
+ * long-form review page (vibe-research.pages.dev, 2026-09-09) states it in section 3.3: the
+ * diffusion path drafts a token block; the AR (target) path scores every drafted position;
+ * draft token i is accepted with probability min(1, p_AR(x_i) / p_draft(x_i)); the longest
+ * prefix before the first rejection is kept; a rejected position is resampled from the
+ * normalised residual [p_AR - p_draft]_+; when the whole block is accepted, one extra token is
+ * drawn from the last verifier row. Section 3.4 names the linear sampler (one candidate per
+ * position) and the tree sampler (several candidate prefixes verified together). The
+ * project README's inference example lists the sampling controls --temperature and --top-p.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - Pointers named *_logits, u_*, temperature, top_p, draft_tokens, node_*, parent, tokens,
+ *    out_*, row_stats and workspace are DEVICE pointers owned by the caller. The library
+ *    allocates no memory and keeps no state between calls; it only enqueues kernels on
+ *    `stream` (a cudaStream_t; NULL selects the legacy default stream). Calls are
+ *    asynchronous: outputs are valid once the stream reaches that point.
+ *  - Logit rows are contiguous: row r of a [rows, V] tensor starts at element r * V. dtype is
+ *    PSISPEC_F32 or PSISPEC_BF16. Any V >= 1 is accepted; V up to 2^24.
+ *  - Temperature T (per request): T == 0 means greedy (a point mass on the lowest-index
+ *    maximum); T > 0 divides the logits by T before the softmax over the whole vocabulary.
+ *    T < 0, NaN or inf is a per-request data error.
+ *  - top_p (per request): in (0, 1); values >= 1 switch the filter off. The kept set is every
+ *    token whose logit is >= tau, where tau is the largest logit value whose tie-inclusive
+ *    upper-tail probability is >= top_p; the distribution is renormalised over the kept set.
+ *    It is applied after the temperature, to the verifier row and to the draft row
+ *    separately, and it is a no-op at T == 0. (The pages leave top-p's definition open.)
+ *  - Uniforms u are floats in [0, 1) supplied by the caller; the library draws no random
+ *    numbers. An inverse-CDF draw with uniform u over weights r returns the first index v, in
+ *    vocabulary order, with C(v) > u * Z (C inclusive prefix sum, Z = sum of r), so a token of
+ *    zero probability is never returned.
+ *  - The accept test for a draft token x is u * q(x) < p(x); with q(x) > 0 this is
+ *    u < p(x)/q(x), i.e. acceptance with probability min(1, p/q).
+ *  - Data errors found on the device (a NaN or +inf logit, a row with no finite logit, a draft
+ *    token outside [0, V), a malformed trie, a bad temperature) affect only the request they
+ *    occur in: its accept length is written as -1 and its token outputs as -1.
+ *  - Host-side argument errors are returned as a status before anything is enqueued.
+ *  - workspace: device scratch of at least psispec_workspace_size(...) bytes, 256-byte
+ *    aligned. Its contents need no initialisation and are not meaningful after the call. Two
+ *    calls in flight at the same time must not share one workspace.
+ */
+#ifndef PSISPEC_H
+#define PSISPEC_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  PSISPEC_OK = 0,
+  PSISPEC_ERR_INVALID_ARG = 1, /* null pointer, bad size, bad dtype, misaligned pointer */
+  PSISPEC_ERR_UNSUPPORTED = 2, /* a size beyond the documented limits */
+  PSISPEC_ERR_CUDA = 3,        /* a kernel launch failed (cudaGetLastError after the launch) */
+  PSISPEC_ERR_WORKSPACE = 4    /* workspace null, too small or not 256-byte aligned */
+} psispec_status;
+
+typedef enum { PSISPEC_F32 = 0, PSISPEC_BF16 = 1 } psispec_dtype;
+
+typedef enum {
+  PSISPEC_OP_SAMPLE_DRAFT = 0,
+  PSISPEC_OP_VERIFY_LINEAR = 1,
+  PSISPEC_OP_VERIFY_TREE = 2
+} psispec_op;
+
+/* Bytes of one per-row statistics record written by psispec_sample_draft (out_row_stats). */
+#define PSISPEC_ROW_STATS_BYTES 32
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* psispec_status_string(int status);
+
+/* Library ABI version: 100 * major + minor. */
+int psispec_version(void);
+
+/* Workspace bytes needed by one call of `op` with these sizes (an upper bound).
+ *   SAMPLE_DRAFT:  a = B, b = K (rows = B*K), c = V
+ *   VERIFY_LINEAR: a = B, b = K, c = V
+ *   VERIFY_TREE:   a = B, b = N (total nodes), c = V
+ * Returns 0 for invalid sizes. */
+size_t psispec_workspace_size(int op, int64_t a, int64_t b, int64_t c);
+
+/*
+ * psispec_sample_draft -- draw each drafted token from its draft distribution q.
+ * Section 3.3 of the review page: the drafted block is a sample of the diffusion path's
+ * distribution, after the sampling controls (temperature, top-p).
+ *
+ *   draft_logits  [B, K, V] dtype   draft (diffusion-path) logits, row i of request b at
+ *                                   element (b*K + i) * V
+ *   temperature   [B] float, top_p [B] float
+ *   u             [B, K] float in [0, 1)     one uniform per drafted position
+ *   out_tokens    [B, K] int32      drawn token (-1 on a data error in that row)
+ *   out_q         [B, K] float      q(token) after temperature/top-p; may be NULL
+ *   out_row_stats [B, K] records of PSISPEC_ROW_STATS_BYTES; may be NULL. When given, they
+ *                 can be passed to psispec_verify_linear (draft_row_stats) for the same
+ *                 draft logits, temperature and top-p, so that the verifier does not re-read
+ *                 the whole draft tensor.
+ * Limits: B, K >= 1, B*K <= 2^26, V <= 2^24.
+ */
+psispec_status psispec_sample_draft(const void* draft_logits, int dtype, int32_t B, int32_t K, int32_t V,
+                                    const float* temperature, const float* top_p, const float* u,
+                                    int32_t* out_tokens, float* out_q, void* out_row_stats,
+                                    void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * psispec_verify_linear -- Psi-Spec linear verification (review page, section 3.3; linear
+ * sampler of section 3.4).
+ *
+ * For request b and drafted position i < K: p_i = verifier distribution of target row i,
+ * q_i = draft distribution of draft row i (both after temperature/top-p); x_i =
+ * draft_tokens[b, i]. Position i is accepted iff u_accept[b, i] * q_i(x_i) < p_i(x_i). With j
+ * the first rejected position (j = K if none), the call emits x_0 .. x_{j-1} and then one
+ * more token y: for j < K, y is drawn with u_resid[b, j] from max(0, p_j - q_j) (from p_j if
+ * that residual is zero everywhere); for j = K it is the bonus token drawn with
+ * u_resid[b, K] from p_K. At T == 0 this reduces to exact argmax matching.
+ *
+ *   target_logits   [B, K+1, V] dtype    verifier rows (row K is the bonus row)
+ *   draft_logits    [B, K, V] dtype      draft rows (only the rejected row is read in full
+ *                                        when draft_row_stats is given)
+ *   draft_tokens    [B, K] int32
+ *   draft_row_stats [B, K] records from psispec_sample_draft over the same draft logits and
+ *                   controls, or NULL to recompute them here
+ *   u_accept [B, K] float, u_resid [B, K+1] float, temperature [B] float, top_p [B] float
+ *   out_tokens      [B, K+1] int32    accepted prefix, then y, then -1 padding
+ *   out_accept_len  [B] int32         j, or -1 on a data error
+ *   out_p, out_q    [B, K] float      p_i(x_i) and q_i(x_i) for every position; may be NULL
+ * Limits: B >= 1, 1 <= K <= 64, B*(K+1) <= 2^26, V <= 2^24.
+ */
+psispec_status psispec_verify_linear(const void* target_logits, const void* draft_logits, int dtype,
+                                     int32_t B, int32_t K, int32_t V, const int32_t* draft_tokens,
+                                     const void* draft_row_stats, const float* u_accept,
+                                     const float* u_resid, const float* temperature, const float* top_p,
+                                     int32_t* out_tokens, int32_t* out_accept_len, float* out_p,
+                                     float* out_q, void* workspace, size_t workspace_bytes,
+                                     void* stream);
+
+/*
+ * psispec_verify_tree -- Psi-Spec tree verification (tree sampler of the review page's
+ * section 3.4; the pages give no acceptance rule for it, so this is the plainest lossless
+ * reading: recursive rejection sampling without replacement over each node's children).
+ *
+ * Request b owns nodes node_offsets[b] .. node_offsets[b+1]-1; the first one is its root.
+ * Every node n has a verifier row target[n] and a draft row draft[n], both distributions of
+ * the token that follows the prefix ending at n. The children of n (nodes whose parent is n)
+ * carry distinct tokens drawn without replacement from n's draft distribution. The walk
+ * starts at the root with r = p_root and q~ = q_root and tries the children in increasing
+ * node order: child c with token t is accepted iff u_accept[c] * q~(t) < r(t); then the walk
+ * moves to c. On rejection r <- normalise(max(0, r - q~)) (unchanged if that is zero) and
+ * q~ <- q~ with t removed, renormalised (when no draft mass is left the remaining children
+ * are skipped). When no child is accepted the final token is drawn from r with
+ * u_resid[current node]. At T == 0 the child whose token is the verifier's argmax is
+ * accepted and the final token is that argmax. With one child per node this is exactly
+ * psispec_verify_linear.
+ *
+ *   target_logits, draft_logits  [N, V] dtype
+ *   node_offsets [B+1] int32 (node_offsets[0] = 0, node_offsets[B] = N)
+ *   parent       [N] int32   request-local index of the parent, -1 at the root, otherwise
+ *                            smaller than the node's own local index
+ *   tokens       [N] int32   token appended by each node (ignored at the root)
+ *   u_accept [N] float, u_resid [N] float, temperature [B] float, top_p [B] float
+ *   max_depth    path-length limit; a trie deeper than this is a data error
+ *   out_path       [B, max_depth] int32   local node ids of the accepted path, -1 padded
+ *   out_tokens     [B, max_depth+1] int32 accepted tokens, then the final token, -1 padded
+ *   out_accept_len [B] int32              number of accepted nodes, -1 on a data error
+ * Limits: B >= 1, N >= B, N <= 2^26, 1 <= max_depth <= 64, at most 1024 nodes per request,
+ * V <= 2^24.
+ */
+psispec_status psispec_verify_tree(const void* target_logits, const void* draft_logits, int dtype,
+                                   int32_t B, int32_t N, int32_t V, const int32_t* node_offsets,
+                                   const int32_t* parent, const int32_t* tokens, const float* u_accept,
+                                   const float* u_resid, const float* temperature, const float* top_p,
+                                   int32_t max_depth, int32_t* out_path, int32_t* out_tokens,
+                                   int32_t* out_accept_len, void* workspace, size_t workspace_bytes,
+                                   void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* PSISPEC_H */

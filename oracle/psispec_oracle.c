@@ -1,0 +1,309 @@
+/*
+ * psispec_oracle.c -- plain fp64 CPU oracle of the Psi-Spec verification step.
+ *
+ * TEST INFRASTRUCTURE ONLY: loaded by the tests, the smoke check and the benchmark's
+ * CPU-baseline leg, never by the product path. It shares no code with the CUDA library.
+ *
+ * The method is the rejection-correction step of "Unlocking Lossless Speedups in LLMs via
+ * Discrete Diffusion" (arXiv 2609.04010), as stated on the long-form review page
+ * (vibe-research.pages.dev, 2026-09-09), section 3.3 "Psi-Spec": accept draft token i with
+ * probability min(1, p_AR(x_i)/p_draft(x_i)), keep the longest prefix before the first
+ * rejection, resample the rejected position from the normalised residual [p_AR - p_draft]_+,
+ * and draw one extra token from the last verifier row when the whole block is accepted.
+ * Temperature and top-p are the sampling controls listed by the project's README (inference
+ * example, "--temperature --top-p"). Section 3.4 names the tree sampler; its acceptance rule
+ * is not printed on the pages, and the reading implemented here is recursive rejection
+ * sampling without replacement over the children of a node, in index order.
+ *
+ * Readings where the pages are silent (each listed in the design notes):
+ *   - top-p keeps every token whose logit is >= tau, where tau is the largest logit value
+ *     whose tie-inclusive upper-tail probability reaches top_p; it is applied after the
+ *     temperature, to the verifier row and to the draft row separately;
+ *   - temperature 0 is greedy: a point mass on the lowest-index maximum;
+ *   - an inverse-CDF draw walks the vocabulary in index order and returns the first v with
+ *     C(v) > u * Z (strict, inclusive prefix), so a zero-mass token is never drawn;
+ *   - "accept with probability min(1, p/q)" is the test u * q < p with u in [0, 1);
+ *   - an all-zero residual (reachable only by rounding) leaves the previous distribution.
+ *
+ * Everything below is straight fp64 loops over the vocabulary; no blocking or reordering.
+ */
+#include "psispec_oracle.h"
+
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+
+static double dmin(double a, double b) { return a < b ? a : b; }
+
+static int cmp_desc(const void* a, const void* b) {
+  double x = *(const double*)a, y = *(const double*)b;
+  return (x < y) - (x > y);
+}
+
+int oracle_row_dist(const double* l, int V, double T, double top_p, double* out, double* band) {
+  *band = INFINITY;
+  if (V <= 0 || !(T >= 0)) return -1;
+  int any_finite = 0;
+  for (int v = 0; v < V; ++v) {
+    if (isnan(l[v]) || l[v] == INFINITY) return -1;
+    if (isfinite(l[v])) any_finite = 1;
+  }
+  if (!any_finite) return -1;
+
+  /* row maximum, lowest index on ties */
+  double m = -INFINITY;
+  int amax = -1;
+  for (int v = 0; v < V; ++v)
+    if (l[v] > m) { m = l[v]; amax = v; }
+
+  if (T == 0.0) {
+    for (int v = 0; v < V; ++v) out[v] = 0.0;
+    out[amax] = 1.0;
+    return 0;
+  }
+
+  /* softmax(l / T) numerator and total, in vocabulary order */
+  double S = 0.0;
+  for (int v = 0; v < V; ++v) {
+    out[v] = exp((l[v] - m) / T);
+    S += out[v];
+  }
+
+  double tau = -INFINITY, S_kept = S;
+  if (top_p < 1.0) {
+    /* walk the distinct logit values from the top; stop at the first value whose
+       tie-inclusive tail mass reaches top_p of the total */
+    double* vals = (double*)malloc(sizeof(double) * (size_t)V);
+    memcpy(vals, l, sizeof(double) * (size_t)V);
+    qsort(vals, (size_t)V, sizeof(double), cmp_desc);
+    double tail = 0.0;
+    int found = 0;
+    for (int i = 0; i < V;) {
+      double t = vals[i], group = 0.0;
+      int j = i;
+      while (j < V && vals[j] == t) { group += exp((t - m) / T); ++j; }
+      double above = tail;
+      tail += group;
+      if (tail >= top_p * S) {
+        tau = t;
+        S_kept = tail;
+        *band = dmin(fabs(tail / S - top_p), fabs(above / S - top_p));
+        found = 1;
+        break;
+      }
+      i = j;
+    }
+    free(vals);
+    if (!found) { tau = -INFINITY; S_kept = S; *band = 0.0; }
+  }
+  for (int v = 0; v < V; ++v) out[v] = (l[v] >= tau) ? out[v] / S_kept : 0.0;
+  return 0;
+}
+
+int oracle_inverse_cdf(const double* r, int V, double u, double* band) {
+  double Z = 0.0;
+  for (int v = 0; v < V; ++v) Z += r[v];
+  if (!(Z > 0.0)) { *band = 0.0; return -1; }
+  double target = u * Z, C = 0.0;
+  int last = -1;
+  for (int v = 0; v < V; ++v) {
+    double before = C;
+    C += r[v];
+    if (r[v] > 0.0) last = v;
+    if (C > target) {
+      *band = dmin(fabs(before / Z - u), fabs(C / Z - u));
+      return v;
+    }
+  }
+  *band = 0.0;
+  return last;
+}
+
+int oracle_sample_draft(const double* draft, int rows, int V, const int* row_req,
+                        const double* temperature, const double* top_p, const double* u,
+                        int* tokens, double* q_at, double* band) {
+  if (rows < 0 || V <= 0) return ORACLE_BAD_ARG;
+  double* q = (double*)malloc(sizeof(double) * (size_t)V);
+  for (int i = 0; i < rows; ++i) {
+    int b = row_req[i];
+    double b3 = INFINITY, b2 = INFINITY;
+    tokens[i] = -1;
+    q_at[i] = -1.0;
+    band[i] = INFINITY;
+    if (oracle_row_dist(draft + (size_t)i * V, V, temperature[b], top_p[b], q, &b3) != 0) continue;
+    int y = oracle_inverse_cdf(q, V, u[i], &b2);
+    tokens[i] = y;
+    q_at[i] = y >= 0 ? q[y] : -1.0;
+    band[i] = dmin(b2, b3);
+  }
+  free(q);
+  return ORACLE_OK;
+}
+
+int oracle_verify_linear(const double* target, const double* draft, int B, int K, int V,
+                         const int* draft_tokens, const double* u_accept, const double* u_resid,
+                         const double* temperature, const double* top_p,
+                         int* out_tokens, int* accept_len, double* out_p, double* out_q,
+                         double* band, double* pq_band) {
+  if (B < 0 || K < 0 || V <= 0) return ORACLE_BAD_ARG;
+  double* p = (double*)malloc(sizeof(double) * (size_t)V);
+  double* q = (double*)malloc(sizeof(double) * (size_t)V);
+  double* res = (double*)malloc(sizeof(double) * (size_t)V);
+  for (int b = 0; b < B; ++b) {
+    const double T = temperature[b], tp = top_p[b];
+    const double* tgt = target + (size_t)b * (K + 1) * V;
+    const double* drf = draft + (size_t)b * K * V;
+    int* toks = out_tokens + (size_t)b * (K + 1);
+    int bad = 0, j = K, y = -1;
+    double path_band = INFINITY;
+    for (int i = 0; i <= K; ++i) toks[i] = -1;
+    for (int i = 0; i < K; ++i) pq_band[(size_t)b * K + i] = INFINITY;
+
+    for (int i = 0; i < K && !bad; ++i) {
+      double bp = INFINITY, bq = INFINITY;
+      int x = draft_tokens[(size_t)b * K + i];
+      if (x < 0 || x >= V) { bad = 1; break; }
+      if (oracle_row_dist(tgt + (size_t)i * V, V, T, tp, p, &bp) != 0) { bad = 1; break; }
+      if (oracle_row_dist(drf + (size_t)i * V, V, T, tp, q, &bq) != 0) { bad = 1; break; }
+      out_p[(size_t)b * K + i] = p[x];
+      out_q[(size_t)b * K + i] = q[x];
+      pq_band[(size_t)b * K + i] = dmin(bp, bq);
+      if (i > j) continue; /* past the first rejection: probabilities only */
+      double u = u_accept[(size_t)b * K + i];
+      path_band = dmin(path_band, dmin(bp, bq));
+      if (q[x] > 0.0) path_band = dmin(path_band, fabs(u - p[x] / q[x]));
+      if (u * q[x] < p[x]) continue; /* accepted */
+      /* first rejection: draw from the normalised residual [p - q]_+ */
+      j = i;
+      double Z = 0.0;
+      for (int v = 0; v < V; ++v) {
+        res[v] = p[v] > q[v] ? p[v] - q[v] : 0.0;
+        Z += res[v];
+      }
+      double b2 = INFINITY;
+      y = oracle_inverse_cdf(Z > 0.0 ? res : p, V, u_resid[(size_t)b * (K + 1) + i], &b2);
+      path_band = dmin(path_band, b2);
+    }
+    if (!bad) {
+      double bp = INFINITY;
+      if (oracle_row_dist(tgt + (size_t)K * V, V, T, tp, p, &bp) != 0) bad = 1;
+      if (!bad && j == K) { /* whole block accepted: bonus draw from the last verifier row */
+        double b2 = INFINITY;
+        y = oracle_inverse_cdf(p, V, u_resid[(size_t)b * (K + 1) + K], &b2);
+        path_band = dmin(path_band, dmin(bp, b2));
+      }
+    }
+    if (bad) {
+      accept_len[b] = -1;
+      for (int i = 0; i < K; ++i) { out_p[(size_t)b * K + i] = -1.0; out_q[(size_t)b * K + i] = -1.0; }
+      band[b] = INFINITY;
+      continue;
+    }
+    accept_len[b] = j;
+    for (int i = 0; i < j; ++i) toks[i] = draft_tokens[(size_t)b * K + i];
+    toks[j] = y;
+    band[b] = path_band;
+  }
+  free(p);
+  free(q);
+  free(res);
+  return ORACLE_OK;
+}
+
+int oracle_verify_tree(const double* target, const double* draft, int B, int V,
+                       const int* node_offsets, const int* parent, const int* tokens,
+                       const double* u_accept, const double* u_resid,
+                       const double* temperature, const double* top_p, int max_depth,
+                       int* out_path, int* out_tokens, int* accept_len, double* band) {
+  if (B < 0 || V <= 0 || max_depth < 0) return ORACLE_BAD_ARG;
+  double* r = (double*)malloc(sizeof(double) * (size_t)V);
+  double* qt = (double*)malloc(sizeof(double) * (size_t)V);
+  double* res = (double*)malloc(sizeof(double) * (size_t)V);
+  for (int b = 0; b < B; ++b) {
+    const int n0 = node_offsets[b], n = node_offsets[b + 1] - node_offsets[b];
+    const double T = temperature[b], tp = top_p[b];
+    int* path = out_path + (size_t)b * max_depth;
+    int* toks = out_tokens + (size_t)b * (max_depth + 1);
+    for (int i = 0; i < max_depth; ++i) path[i] = -1;
+    for (int i = 0; i <= max_depth; ++i) toks[i] = -1;
+    accept_len[b] = -1;
+    band[b] = INFINITY;
+
+    /* structure checks: root first, parents precede children, depth within max_depth */
+    int bad = n <= 0 || parent[n0] != -1;
+    int* depth = (int*)calloc((size_t)(n > 0 ? n : 1), sizeof(int));
+    for (int c = 1; c < n && !bad; ++c) {
+      int pa = parent[n0 + c], t = tokens[n0 + c];
+      if (pa < 0 || pa >= c || t < 0 || t >= V) { bad = 1; break; }
+      depth[c] = depth[pa] + 1;
+      if (depth[c] > max_depth) bad = 1;
+    }
+    free(depth);
+    if (bad) continue;
+
+    double path_band = INFINITY;
+    int cur = 0, len = 0, y = -1;
+    for (;;) {
+      double b3 = INFINITY;
+      if (oracle_row_dist(target + (size_t)(n0 + cur) * V, V, T, tp, r, &b3) != 0) { bad = 1; break; }
+      path_band = dmin(path_band, b3);
+      int has_child = 0;
+      for (int c = cur + 1; c < n; ++c) has_child |= parent[n0 + c] == cur;
+      if (has_child && T > 0.0) {
+        if (oracle_row_dist(draft + (size_t)(n0 + cur) * V, V, T, tp, qt, &b3) != 0) { bad = 1; break; }
+        path_band = dmin(path_band, b3);
+      }
+      int next = -1;
+      for (int c = cur + 1; c < n && next < 0; ++c) {
+        if (parent[n0 + c] != cur) continue;
+        int t = tokens[n0 + c];
+        if (T == 0.0) { /* greedy: the child carrying the verifier's argmax is accepted */
+          if (r[t] > 0.0) next = c;
+          continue;
+        }
+        double qmass = 0.0;
+        for (int v = 0; v < V; ++v) qmass += qt[v];
+        if (!(qmass > 0.0)) break; /* draft mass exhausted: remaining siblings skipped */
+        double u = u_accept[n0 + c];
+        if (qt[t] > 0.0) path_band = dmin(path_band, fabs(u - r[t] / qt[t]));
+        if (u * qt[t] < r[t]) { next = c; break; }
+        /* rejected: r <- norm([r - qt]_+), then remove t from the draft and renormalise */
+        double Z = 0.0;
+        for (int v = 0; v < V; ++v) {
+          res[v] = r[v] > qt[v] ? r[v] - qt[v] : 0.0;
+          Z += res[v];
+        }
+        if (Z > 0.0)
+          for (int v = 0; v < V; ++v) r[v] = res[v] / Z;
+        qt[t] = 0.0;
+        double Zq = 0.0;
+        for (int v = 0; v < V; ++v) Zq += qt[v];
+        if (Zq > 0.0)
+          for (int v = 0; v < V; ++v) qt[v] /= Zq;
+      }
+      if (next >= 0) {
+        path[len] = next;
+        toks[len] = tokens[n0 + next];
+        ++len;
+        cur = next;
+        continue;
+      }
+      double b2 = INFINITY;
+      y = oracle_inverse_cdf(r, V, u_resid[n0 + cur], &b2);
+      path_band = dmin(path_band, b2);
+      break;
+    }
+    if (bad) {
+      for (int i = 0; i < max_depth; ++i) path[i] = -1;
+      for (int i = 0; i <= max_depth; ++i) toks[i] = -1;
+      continue;
+    }
+    toks[len] = y;
+    accept_len[b] = len;
+    band[b] = path_band;
+  }
+  free(r);
+  free(qt);
+  free(res);
+  return ORACLE_OK;
+}

@@ -1,0 +1,89 @@
+/*
+ * psispec_oracle.h -- plain, slow fp64 CPU oracle of the Psi-Spec verification step.
+ *
+ * TEST INFRASTRUCTURE ONLY. Only the tests, the smoke check and the benchmark's CPU-baseline
+ * leg may load this library. It shares no code, header, table or constant with the CUDA
+ * library; neither side includes or links the other.
+ *
+ * Source of the method: "Unlocking Lossless Speedups in LLMs via Discrete Diffusion"
+ * (arXiv 2609.04010), long-form review page (vibe-research.pages.dev, silicon-writer,
+ * 2026-09-09), section 3.3 "Psi-Spec": draft block sampled from the diffusion path; accept
+ * draft token i with probability min(1, p_AR(x_i)/p_draft(x_i)); keep the longest prefix
+ * before the first rejection; on rejection resample from the normalised residual
+ * [p_AR - p_draft]_+; if the whole block is accepted, draw one more token from the last
+ * verifier row. Section 3.4 names the linear and tree samplers (the tree rule itself is not
+ * stated on the pages; the reading used here is recursive rejection without replacement
+ * over the sibling candidates).
+ *
+ * All randomness is an explicit input: every uniform u is a double in [0, 1).
+ * Logits are passed as doubles (bf16 and fp32 inputs convert to double exactly).
+ *
+ * "band" outputs: for every request (or draft row) the smallest distance, over the decisions
+ * on the oracle's own path, between a uniform and the quantity it is compared against:
+ *   E1 |u - p/q|               for each accept test (q > 0),
+ *   E2 |C(y-1)/Z - u|, |C(y)/Z - u|   for each inverse-CDF draw,
+ *   E3 |tail(tau)/S - top_p|, |tail(tau+)/S - top_p|   for each top-p threshold used.
+ * A comparison whose band is below the agreed tolerance may legitimately differ between
+ * two correct implementations with different rounding.
+ */
+#ifndef PSISPEC_ORACLE_H
+#define PSISPEC_ORACLE_H
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Return codes. Per-request data errors are reported through accept_len = -1 instead. */
+#define ORACLE_OK 0
+#define ORACLE_BAD_ARG 1
+
+/* One row's distribution after temperature T and top-p.
+ * l[V] logits; T == 0 means greedy (a point mass on the lowest-index maximum).
+ * top_p >= 1 disables the filter. out[V] receives probabilities (sum 1).
+ * *band receives the E3 margin (+inf when the filter is off).
+ * Returns 0, or -1 for a bad row (NaN or +inf logit, or no finite logit). */
+int oracle_row_dist(const double* l, int V, double T, double top_p, double* out, double* band);
+
+/* Inverse-CDF draw in vocabulary order: y = min{v : C(v) > u * Z}, C inclusive.
+ * r[V] >= 0 need not be normalised. If no index qualifies (rounding), y is the last v with
+ * r[v] > 0. Returns y, or -1 when Z == 0. *band receives the E2 margin. */
+int oracle_inverse_cdf(const double* r, int V, double u, double* band);
+
+/* Draft sampling, one draw per row.
+ * draft[rows*V]; row_req[rows] maps a row to its request for temperature[]/top_p[];
+ * u[rows]. Outputs: tokens[rows] (-1 on a bad row), q_at[rows] = q(token), band[rows]. */
+int oracle_sample_draft(const double* draft, int rows, int V, const int* row_req,
+                        const double* temperature, const double* top_p, const double* u,
+                        int* tokens, double* q_at, double* band);
+
+/* Linear verification.
+ * target[B*(K+1)*V], draft[B*K*V], draft_tokens[B*K], u_accept[B*K], u_resid[B*(K+1)],
+ * temperature[B], top_p[B].
+ * Outputs: out_tokens[B*(K+1)] (accepted prefix, then the resampled or bonus token, then -1),
+ * accept_len[B] (-1 on a data error), out_p[B*K] = p_i(x_i), out_q[B*K] = q_i(x_i),
+ * band[B] = smallest E1/E2/E3 margin on the request's path,
+ * pq_band[B*K] = E3 margin of the two rows behind out_p/out_q at that position. */
+int oracle_verify_linear(const double* target, const double* draft, int B, int K, int V,
+                         const int* draft_tokens, const double* u_accept, const double* u_resid,
+                         const double* temperature, const double* top_p,
+                         int* out_tokens, int* accept_len, double* out_p, double* out_q,
+                         double* band, double* pq_band);
+
+/* Tree verification (recursive rejection without replacement over siblings).
+ * node_offsets[B+1]: request b owns nodes [node_offsets[b], node_offsets[b+1]); the first is
+ * its root. parent[N]: local index of the parent (-1 at the root, otherwise < own local
+ * index). tokens[N]: token that node appends (root's ignored). target[N*V], draft[N*V]:
+ * the next-token rows at each node. u_accept[N] is consumed when a node is tested as a
+ * candidate child; u_resid[N] when the final draw happens at that node.
+ * Outputs: out_path[B*max_depth] local node ids of the accepted path (-1 padded),
+ * out_tokens[B*(max_depth+1)], accept_len[B] (-1 on a data error), band[B]. */
+int oracle_verify_tree(const double* target, const double* draft, int B, int V,
+                       const int* node_offsets, const int* parent, const int* tokens,
+                       const double* u_accept, const double* u_resid,
+                       const double* temperature, const double* top_p, int max_depth,
+                       int* out_path, int* out_tokens, int* accept_len, double* band);
+
+#ifdef __cplusplus
+}
+#endif
+#endif

@@ -1,0 +1,51 @@
+"""The oracle's pins catch plausible mistakes (no GPU).
+
+Each mutation below plants one small error in a copy of oracle/psispec_oracle.c (a swapped
+operand, a wrong sign or index, a dropped update, a changed comparison), builds it under a
+temporary directory, and reruns the pin suites against it with ORACLE_LIB. Every mutant must
+fail at least one pin; the unmodified source passes them (the other test files).
+"""
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle", "psispec_oracle.c")
+
+MUTATIONS = {
+    "accept_operands_swapped": ("if (u * q[x] < p[x]) continue;", "if (u * p[x] < q[x]) continue;"),
+    "accept_not_strict": ("if (u * q[x] < p[x]) continue;", "if (u * q[x] <= p[x]) continue;"),
+    "residual_sign": ("res[v] = p[v] > q[v] ? p[v] - q[v] : 0.0;", "res[v] = q[v] > p[v] ? q[v] - p[v] : 0.0;"),
+    "residual_not_clipped": ("res[v] = p[v] > q[v] ? p[v] - q[v] : 0.0;", "res[v] = p[v];"),
+    "cdf_not_strict": ("if (C > target) {", "if (C >= target) {"),
+    "bonus_wrong_row": ("oracle_row_dist(tgt + (size_t)K * V, V, T, tp, p, &bp)",
+                        "oracle_row_dist(tgt + (size_t)(K - 1) * V, V, T, tp, p, &bp)"),
+    "resid_uniform_index": ("u_resid[(size_t)b * (K + 1) + i], &b2);", "u_resid[(size_t)b * (K + 1) + i + 1], &b2);"),
+    "temperature_multiplied": ("out[v] = exp((l[v] - m) / T);", "out[v] = exp((l[v] - m) * T);"),
+    "topp_drops_ties": ("out[v] = (l[v] >= tau) ? out[v] / S_kept : 0.0;", "out[v] = (l[v] > tau) ? out[v] / S_kept : 0.0;"),
+    "topp_not_renormalised": ("out[v] = (l[v] >= tau) ? out[v] / S_kept : 0.0;", "out[v] = (l[v] >= tau) ? out[v] / S : 0.0;"),
+    "greedy_highest_index": ("if (l[v] > m) { m = l[v]; amax = v; }", "if (l[v] >= m) { m = l[v]; amax = v; }"),
+    "tree_no_removal": ("qt[t] = 0.0;", "(void)t;"),
+    "tree_no_residual_update": ("for (int v = 0; v < V; ++v) r[v] = res[v] / Z;", "(void)Z;"),
+    "tree_wrong_uniform": ("double u = u_accept[n0 + c];", "double u = u_accept[n0 + cur];"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_mutant_is_caught(name, tmp_path):
+    old, new = MUTATIONS[name]
+    src = open(SRC).read()
+    assert src.count(old) == 1, name
+    mut = tmp_path / "mutant.c"
+    mut.write_text(src.replace(old, new))
+    lib = tmp_path / "libmutant.so"
+    subprocess.check_call(["gcc", "-O2", "-std=c99", "-shared", "-fPIC", "-I", os.path.dirname(SRC),
+                           "-o", str(lib), str(mut), "-lm"])
+    env = dict(os.environ, ORACLE_LIB=str(lib))
+    r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
+                        os.path.join(ROOT, "tests", "test_oracle_pins.py"),
+                        os.path.join(ROOT, "tests", "test_oracle_lossless.py")],
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode != 0, "mutation %s survived the pins" % name
