@@ -1,0 +1,212 @@
+// common.cuh -- device helpers shared by the Psi-Spec kernels (sm_100a).
+//
+// Arithmetic conventions of the CUDA path:
+//   * a logit l of a row with statistics (m, c) has weight w = 2^((l - m) * c), c = log2(e)/T,
+//     evaluated with the hardware ex2.approx instruction (ftz); m is the row maximum, so
+//     every weight is in [0, 1];
+//   * per-thread sums are fp32, block and cross-slice combinations of probability mass that
+//     feed an inverse-CDF draw are fp64;
+//   * top-p thresholds are compared on order-preserving 32-bit keys of the logit values, so
+//     ties are kept or dropped together.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace psi {
+
+constexpr int kThreads = 256;       // threads per CTA of the streaming kernels
+constexpr int kSliceElems = 16384;  // vocabulary elements per slice (work unit of a CTA)
+
+// Per-row statistics record (32 bytes; also the public row-stats record).
+struct RowStat {
+  float m;         // row maximum
+  float c;         // log2(e) / T; 0 means greedy
+  float s;         // sum over the row of 2^((l - m) c)
+  float s_kept;    // the same sum restricted to the top-p kept set
+  uint32_t tau;    // kept <=> key(l) >= tau (0 keeps every token)
+  int32_t amax;    // lowest index of the maximum (greedy rows)
+  int32_t status;  // 0 ok, 1 data error in this row
+  int32_t pad;
+};
+static_assert(sizeof(RowStat) == 32, "row stats record is 32 bytes");
+
+// Partial statistics of one (row, slice) work unit.
+struct Partial {
+  float m;
+  float s;  // relative to this slice's own maximum
+  int32_t amax;
+  int32_t pad;
+};
+
+// Inverse-CDF job: draw from row a of tensor A (mode kSample) or from max(0, pA - qB)
+// (mode kResidual), with uniform u; the result goes to out_tokens[out_index].
+enum JobMode : int32_t { kNone = 0, kSample = 2, kResidual = 3 };
+struct Job {
+  int32_t mode;
+  int32_t row_a;
+  int32_t row_b;
+  int32_t out_index;
+  float u;
+  int32_t aux;  // index for a probability output (sample_draft's out_q), -1 if none
+  int32_t pad[2];
+};
+static_assert(sizeof(Job) == 32, "job record is 32 bytes");
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// maximum that propagates NaN (so a NaN logit poisons the row statistics)
+__device__ __forceinline__ float fmax_nan(float a, float b) {
+  float y;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(y) : "f"(a), "f"(b));
+  return y;
+}
+
+// order-preserving key of a float; -0 and +0 share one key
+__device__ __forceinline__ uint32_t fkey(float x) {
+  uint32_t b = __float_as_uint(x);
+  if (b == 0x80000000u) b = 0u;
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+__device__ __forceinline__ bool is_finite(float x) { return fabsf(x) <= 3.402823466e38f; }
+
+__device__ __forceinline__ float load_elem(const float* p) { return __ldg(p); }
+__device__ __forceinline__ float load_elem(const __nv_bfloat16* p) {
+  unsigned short h = __ldg(reinterpret_cast<const unsigned short*>(p));
+  return __uint_as_float(static_cast<uint32_t>(h) << 16);
+}
+
+// 16-byte vector of elements
+template <typename T>
+struct Vec;
+template <>
+struct Vec<float> {
+  static constexpr int N = 4;
+  __device__ __forceinline__ static void load(const float* p, float (&f)[8]) {
+    float4 v = __ldg(reinterpret_cast<const float4*>(p));
+    f[0] = v.x; f[1] = v.y; f[2] = v.z; f[3] = v.w;
+  }
+};
+template <>
+struct Vec<__nv_bfloat16> {
+  static constexpr int N = 8;
+  __device__ __forceinline__ static void load(const __nv_bfloat16* p, float (&f)[8]) {
+    uint4 v = __ldg(reinterpret_cast<const uint4*>(p));
+    uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      f[2 * k] = __uint_as_float(w[k] << 16);
+      f[2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
+    }
+  }
+};
+
+// The aligned vector range of [v0, v1) within a row: [a0, a1) with a0 - v0 < N elements.
+template <typename T>
+__device__ __forceinline__ void vec_range(const T* row, int v0, int v1, int& a0, int& a1) {
+  constexpr int N = Vec<T>::N;
+  uintptr_t addr = reinterpret_cast<uintptr_t>(row + v0);
+  int head = static_cast<int>(((16u - (addr & 15u)) & 15u) / sizeof(T));
+  a0 = min(v1, v0 + head);
+  a1 = a0 + ((v1 - a0) / N) * N;
+}
+
+// Weight of logit l under row statistics st (kept set applied); greedy rows are handled by
+// the callers.
+__device__ __forceinline__ float kept_weight(const RowStat& st, float l) {
+  return fkey(l) >= st.tau ? ex2((l - st.m) * st.c) : 0.0f;
+}
+
+// Probability of token v with logit l under st.
+__device__ __forceinline__ float prob_of(const RowStat& st, float l, int v) {
+  if (st.c == 0.0f) return v == st.amax ? 1.0f : 0.0f;
+  return kept_weight(st, l) / st.s_kept;
+}
+
+__device__ __forceinline__ float warp_max(float x) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) x = fmax_nan(x, __shfl_xor_sync(0xffffffffu, x, o));
+  return x;
+}
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+  return x;
+}
+__device__ __forceinline__ double warp_sum(double x) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+  return x;
+}
+
+// Block-wide reductions (blockDim.x a multiple of 32, at most 1024); the result is returned
+// to every thread. `scratch` holds at least 32 elements and is reused after a barrier.
+__device__ __forceinline__ float block_max(float x, float* scratch) {
+  int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  x = warp_max(x);
+  __syncthreads();
+  if (lane == 0) scratch[warp] = x;
+  __syncthreads();
+  x = lane < nw ? scratch[lane] : -INFINITY;
+  return warp_max(x);
+}
+__device__ __forceinline__ float block_sum(float x, float* scratch) {
+  int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  x = warp_sum(x);
+  __syncthreads();
+  if (lane == 0) scratch[warp] = x;
+  __syncthreads();
+  x = lane < nw ? scratch[lane] : 0.0f;
+  return warp_sum(x);
+}
+__device__ __forceinline__ double block_sum(double x, double* scratch) {
+  int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  x = warp_sum(x);
+  __syncthreads();
+  if (lane == 0) scratch[warp] = x;
+  __syncthreads();
+  x = lane < nw ? scratch[lane] : 0.0;
+  return warp_sum(x);
+}
+
+// Exclusive prefix sum of one double per thread, in thread order (deterministic).
+// `scratch` holds at least 33 doubles; *total receives the block total.
+__device__ __forceinline__ double block_exclusive_scan(double x, double* scratch, double* total) {
+  int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  double incl = x;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    double y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  double excl = __shfl_up_sync(0xffffffffu, incl, 1);
+  if (lane == 0) excl = 0.0;
+  __syncthreads();
+  if (lane == 31) scratch[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    double w = lane < nw ? scratch[lane] : 0.0;
+    double wi = w;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      double y = __shfl_up_sync(0xffffffffu, wi, o);
+      if (lane >= o) wi += y;
+    }
+    double we = __shfl_up_sync(0xffffffffu, wi, 1);
+    if (lane == 0) we = 0.0;
+    if (lane < nw) scratch[lane] = we;
+    if (lane == nw - 1) scratch[32] = wi;
+  }
+  __syncthreads();
+  double r = scratch[warp] + excl;
+  *total = scratch[32];
+  return r;
+}
+
+}  // namespace psi

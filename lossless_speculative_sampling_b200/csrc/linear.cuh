@@ -1,0 +1,97 @@
+// linear.cuh -- accept test, first-rejection scan and output assembly of the linear sampler.
+//
+// Review page of arXiv 2609.04010, section 3.3: draft token x_i is accepted with probability
+// min(1, p(x_i)/q(x_i)), the longest prefix before the first rejection is kept, the rejected
+// position is resampled from the normalised residual [p - q]_+, and a fully accepted block
+// earns a bonus token from the last verifier row. Section 3.4: the linear sampler proposes
+// one candidate per position.
+//
+// One warp per request: lane i tests position i (and i + 32), a ballot gives the first
+// rejection j, and lane 0 writes the residual (or bonus) draw job that cdf_partial/cdf_pick
+// complete. Greedy requests (T == 0) need no draw: the verifier argmax is written directly.
+#pragma once
+
+#include "common.cuh"
+
+namespace psi {
+
+// u * q(x) < p(x), evaluated as u < 2^(((lp - lq) + (mq - mp)) c) * sq / sp so that tiny
+// probabilities do not underflow before the comparison.
+__device__ __forceinline__ bool accept_test(float u, const RowStat& sp, float lp, const RowStat& sq, float lq, int x) {
+  if (sp.c == 0.0f) return x == sp.amax;
+  const bool p_pos = fkey(lp) >= sp.tau && lp > -INFINITY;
+  const bool q_pos = fkey(lq) >= sq.tau && lq > -INFINITY;
+  if (!p_pos) return false;
+  if (!q_pos) return true;
+  const float e = ((lp - lq) + (sq.m - sp.m)) * sp.c;
+  const float ratio = ex2(e) * (sq.s_kept / sp.s_kept);
+  return u < ratio;
+}
+
+template <typename T>
+__global__ void linear_decide_kernel(const T* __restrict__ tgt, const T* __restrict__ drf, int B, int K, int V,
+                                     const int32_t* __restrict__ tokens, const RowStat* __restrict__ ts,
+                                     const RowStat* __restrict__ ds, const float* __restrict__ u_acc,
+                                     const float* __restrict__ u_res, int32_t* __restrict__ out_tokens,
+                                     int32_t* __restrict__ out_len, float* __restrict__ out_p,
+                                     float* __restrict__ out_q, Job* __restrict__ jobs) {
+  const int lane = threadIdx.x & 31;
+  const int b = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (b >= B) return;
+  const size_t trow0 = static_cast<size_t>(b) * (K + 1), drow0 = static_cast<size_t>(b) * K;
+  bool bad = false;
+  uint32_t rej_lo = 0u, rej_hi = 0u;
+  int x_mine[3] = {-1, -1, -1};
+  float p_mine[2] = {-1.0f, -1.0f}, q_mine[2] = {-1.0f, -1.0f};
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int i = lane + 32 * h;
+    if (i >= K) break;
+    const int x = tokens[drow0 + i];
+    const RowStat sp = ts[trow0 + i], sq = ds[drow0 + i];
+    const bool rowbad = sp.status != 0 || sq.status != 0 || x < 0 || x >= V;
+    bool acc = false;
+    if (!rowbad) {
+      const float lp = load_elem(tgt + (trow0 + i) * V + x);
+      const float lq = load_elem(drf + (drow0 + i) * V + x);
+      p_mine[h] = prob_of(sp, lp, x);
+      q_mine[h] = prob_of(sq, lq, x);
+      acc = accept_test(u_acc[drow0 + i], sp, lp, sq, lq, x);
+    }
+    x_mine[h] = x;
+    bad |= rowbad;
+    if (!acc) (h ? rej_hi : rej_lo) |= 1u << lane;
+  }
+  const RowStat bonus = ts[trow0 + K];
+  bad = __any_sync(0xffffffffu, bad) || bonus.status != 0;
+  rej_lo = __reduce_or_sync(0xffffffffu, rej_lo);
+  rej_hi = __reduce_or_sync(0xffffffffu, rej_hi);
+  const int j = rej_lo ? __ffs(rej_lo) - 1 : (rej_hi ? 32 + __ffs(rej_hi) - 1 : K);
+  const RowStat sj = ts[trow0 + j];  // verifier row of the draw (row K for the bonus)
+
+#pragma unroll
+  for (int h = 0; h < 3; ++h) {  // K + 1 <= 65 token slots
+    const int i = lane + 32 * h;
+    if (i < K && h < 2) {
+      if (out_p) out_p[drow0 + i] = bad ? -1.0f : p_mine[h];
+      if (out_q) out_q[drow0 + i] = bad ? -1.0f : q_mine[h];
+    }
+    if (i <= K) {
+      int t = -1;
+      if (!bad) {
+        if (i < j) t = x_mine[h];
+        else if (i == j && sj.c == 0.0f) t = sj.amax;  // greedy: the verifier argmax
+      }
+      out_tokens[trow0 + i] = t;
+    }
+  }
+  if (lane == 0) {
+    out_len[b] = bad ? -1 : j;
+    Job jb{kNone, static_cast<int32_t>(trow0 + j), static_cast<int32_t>(drow0 + j), static_cast<int32_t>(trow0 + j),
+           u_res[trow0 + j], -1, {0, 0}};
+    if (!bad && sj.c != 0.0f) jb.mode = j < K ? kResidual : kSample;
+    jobs[b] = jb;
+  }
+}
+
+}  // namespace psi

@@ -1,0 +1,239 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 oracle, on a B200.
+
+Integer results must be identical except on requests the oracle marks in-band (see
+tests/parity.py); probabilities agree to 1e-5. Draft tokens fed to verification come from the
+oracle's own sampler (or from the input generator for rows the oracle does not check), never
+from the CUDA path. Small cases span several 16384-element slices and a ragged tail; the
+full-size workloads run in the benchmark's launch configuration and are checked on sampled
+requests.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from goldens import load, nums, rows
+from parity import compare_linear, compare_sample, compare_tree
+from lossless_speculative_sampling_b200 import psispec, synth
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda:0"
+
+
+def _cuda(x, dtype=None):
+    t = torch.as_tensor(np.asarray(x)) if not isinstance(x, torch.Tensor) else x
+    return t.to(DEV, dtype=dtype).contiguous()
+
+
+def _rand_logits(g, shape, dtype, std=2.0, neg_inf_frac=0.0):
+    x = torch.randn(shape, generator=g) * std
+    if neg_inf_frac:
+        x[torch.rand(shape, generator=g) < neg_inf_frac] = -float("inf")
+    return x.to(dtype)
+
+
+# ------------------------------------------------------------------ worked examples
+
+
+@pytest.mark.parametrize("case", load("linear.txt"), ids=lambda c: c["name"])
+def test_golden_linear_gpu(case):
+    tgt, drf = rows(case["target"]), rows(case["draft"])
+    K, V = drf.shape
+    out = psispec.verify_linear(_cuda(tgt[None], torch.float32), _cuda(drf[None], torch.float32),
+                                _cuda(np.array(nums(case["tokens"]), np.int32)[None]),
+                                _cuda(nums(case["u_accept"]), torch.float32), _cuda(nums(case["u_resid"]), torch.float32),
+                                _cuda([nums(case["T"])[0]], torch.float32), _cuda([nums(case["top_p"])[0]], torch.float32))
+    assert int(out["accept_len"][0]) == int(nums(case["expect_len"])[0])
+    assert out["tokens"][0].tolist() == [int(x) for x in nums(case["expect_tokens"])]
+    np.testing.assert_allclose(out["p"][0].cpu().numpy(), nums(case["expect_p"]), atol=1e-6)
+    np.testing.assert_allclose(out["q"][0].cpu().numpy(), nums(case["expect_q"]), atol=1e-6)
+
+
+@pytest.mark.parametrize("case", load("tree.txt"), ids=lambda c: c["name"])
+def test_golden_tree_gpu(case):
+    tgt, drf = rows(case["target"]), rows(case["draft"])
+    n = tgt.shape[0]
+    md = int(case["max_depth"])
+    out = psispec.verify_tree(_cuda(tgt, torch.float32), _cuda(drf, torch.float32), _cuda(np.array([0, n], np.int32)),
+                              _cuda(np.array(nums(case["parent"]), np.int32)), _cuda(np.array(nums(case["tokens"]), np.int32)),
+                              _cuda(nums(case["u_accept"]), torch.float32), _cuda(nums(case["u_resid"]), torch.float32),
+                              _cuda([nums(case["T"])[0]], torch.float32), _cuda([nums(case["top_p"])[0]], torch.float32), md)
+    assert int(out["accept_len"][0]) == int(nums(case["expect_len"])[0])
+    assert out["path"][0].tolist() == [int(x) for x in nums(case["expect_path"])]
+    assert out["tokens"][0].tolist() == [int(x) for x in nums(case["expect_tokens"])]
+
+
+# ------------------------------------------------------------------ random small cases
+
+GRID = [
+    # B, K, V, dtype, T, top_p, draft noise
+    (3, 4, 1, torch.float32, 1.0, 1.0, 0.5),
+    (4, 3, 7, torch.float32, 0.7, 1.0, 0.5),
+    (5, 4, 1024, torch.float32, 1.0, 1.0, 0.5),
+    (4, 5, 16384 * 2 + 37, torch.bfloat16, 1.0, 1.0, 1.0),
+    (4, 5, 16384 * 2 + 37, torch.bfloat16, 0.7, 0.9, 0.5),
+    (3, 6, 50001, torch.bfloat16, 1.0, 0.5, 2.0),
+    (3, 4, 40000, torch.float32, 1.3, 0.95, 1.0),
+    (4, 4, 20000, torch.bfloat16, 0.0, 0.9, 0.5),
+    (2, 64, 3000, torch.bfloat16, 1.0, 1.0, 0.05),
+    (1, 1, 151936, torch.bfloat16, 1.0, 0.95, 1.0),
+]
+
+
+def _linear_inputs(B, K, V, dtype, T, top_p, noise, seed, neg_inf_frac=0.0):
+    g = torch.Generator().manual_seed(seed)
+    tgt = _rand_logits(g, (B, K + 1, V), torch.float32, 2.0, neg_inf_frac)
+    drf = (tgt[:, :K].float() + torch.randn((B, K, V), generator=g) * noise).to(dtype)
+    tgt = tgt.to(dtype)
+    ud, ua, ur = synth.uniforms((B, K), seed + 1), synth.uniforms((B, K), seed + 2), synth.uniforms((B, K + 1), seed + 3)
+    Ts, Ps = torch.full((B,), T), torch.full((B,), top_p)
+    return tgt, drf, ud, ua, ur, Ts, Ps
+
+
+@pytest.mark.parametrize("B,K,V,dtype,T,top_p,noise", GRID)
+def test_sample_draft_parity(B, K, V, dtype, T, top_p, noise):
+    tgt, drf, ud, ua, ur, Ts, Ps = _linear_inputs(B, K, V, dtype, T, top_p, noise, seed=V + K)
+    tok, q, _ = psispec.sample_draft(_cuda(drf), _cuda(Ts), _cuda(Ps), _cuda(ud))
+    ora = oracle.sample_draft(drf.reshape(B * K, V), Ts.numpy(), Ps.numpy(), ud.reshape(-1), row_req=np.arange(B * K) // K)
+    compare_sample(tok, q, ora)
+
+
+@pytest.mark.parametrize("use_stats", [False, True])
+@pytest.mark.parametrize("B,K,V,dtype,T,top_p,noise", GRID)
+def test_verify_linear_parity(B, K, V, dtype, T, top_p, noise, use_stats):
+    tgt, drf, ud, ua, ur, Ts, Ps = _linear_inputs(B, K, V, dtype, T, top_p, noise, seed=V + 3 * K)
+    o_s = oracle.sample_draft(drf.reshape(B * K, V), Ts.numpy(), Ps.numpy(), ud.reshape(-1), row_req=np.arange(B * K) // K)
+    x = torch.from_numpy(o_s["tokens"].reshape(B, K).astype(np.int32))
+    stats = None
+    if use_stats:
+        _, _, stats = psispec.sample_draft(_cuda(drf), _cuda(Ts), _cuda(Ps), _cuda(ud))
+    out = psispec.verify_linear(_cuda(tgt), _cuda(drf), _cuda(x), _cuda(ua), _cuda(ur), _cuda(Ts), _cuda(Ps),
+                                draft_row_stats=stats)
+    ora = oracle.verify_linear(tgt, drf, x.numpy(), ua, ur, Ts.numpy(), Ps.numpy())
+    compare_linear(out, ora)
+
+
+def test_verify_linear_mixed_requests_and_data_errors():
+    """Per-request temperature/top-p, -inf logits, and data errors confined to their request."""
+    B, K, V = 8, 5, 9000
+    tgt, drf, ud, ua, ur, _, _ = _linear_inputs(B, K, V, torch.bfloat16, 1.0, 1.0, 0.7, seed=77, neg_inf_frac=0.2)
+    Ts = torch.tensor([1.0, 0.0, 0.5, 2.0, 1.0, 1.0, 0.8, 1.0])
+    Ps = torch.tensor([1.0, 0.9, 0.8, 0.3, 1.0, 0.99, 1.0, 1e-6])
+    o_s = oracle.sample_draft(drf.reshape(B * K, V), Ts.numpy(), Ps.numpy(), ud.reshape(-1), row_req=np.arange(B * K) // K)
+    x = o_s["tokens"].reshape(B, K).astype(np.int32)
+    x[4, 2] = V  # out-of-range token: request 4 is a data error
+    tgt[5, 3, 17] = float("nan")  # NaN logit: request 5 is a data error
+    drf[6, 1, :] = -float("inf")  # draft row without a finite logit: request 6
+    out = psispec.verify_linear(_cuda(tgt), _cuda(drf), _cuda(x), _cuda(ua), _cuda(ur), _cuda(Ts), _cuda(Ps))
+    ora = oracle.verify_linear(tgt, drf, x, ua, ur, Ts.numpy(), Ps.numpy())
+    assert ora["accept_len"][4] == ora["accept_len"][5] == ora["accept_len"][6] == -1
+    compare_linear(out, ora)
+
+
+def test_q_equals_p_accepts_all_on_gpu():
+    B, K, V = 16, 8, 30000
+    g = torch.Generator().manual_seed(5)
+    tgt = _rand_logits(g, (B, K + 1, V), torch.bfloat16)
+    drf = tgt[:, :K].clone()
+    x = torch.randint(0, V, (B, K), generator=g, dtype=torch.int32)
+    ua = synth.uniforms((B, K), 9)
+    ur = synth.uniforms((B, K + 1), 10)
+    out = psispec.verify_linear(_cuda(tgt), _cuda(drf), _cuda(x), _cuda(ua), _cuda(ur), _cuda(torch.ones(B)),
+                                _cuda(torch.ones(B)))
+    assert (out["accept_len"] == K).all()
+    assert torch.equal(out["p"], out["q"])  # the p and q pipelines are bit-identical
+
+
+def _tree_inputs(B, nodes, V, dtype, T, top_p, seed):
+    trie = synth.trie_topology(B, nodes, 6, 3, seed)
+    g = torch.Generator().manual_seed(seed)
+    tgt = _rand_logits(g, (trie.N, V), torch.float32, 2.0)
+    drf = (tgt + torch.randn((trie.N, V), generator=g) * 0.7).to(dtype)
+    tgt = tgt.to(dtype)
+    toks = torch.zeros(trie.N, dtype=torch.int32)
+    for n in range(trie.N):
+        if trie.children[n]:
+            picks = synth.gumbel_tokens(drf[n:n + 1], max(T, 1e-3), seed + n, k=len(trie.children[n]))[0]
+            for k, c in enumerate(trie.children[n]):
+                toks[c] = int(picks[k])
+    ua, ur = synth.uniforms((trie.N,), seed + 1), synth.uniforms((trie.N,), seed + 2)
+    return trie, tgt, drf, toks, ua, ur
+
+
+@pytest.mark.parametrize("V,dtype,T,top_p", [(5, torch.float32, 1.0, 1.0), (1000, torch.float32, 0.8, 0.9),
+                                             (20000, torch.bfloat16, 1.0, 1.0), (33000, torch.bfloat16, 0.7, 0.8),
+                                             (4000, torch.bfloat16, 0.0, 1.0)])
+def test_verify_tree_parity(V, dtype, T, top_p):
+    B, nodes = 6, 24
+    trie, tgt, drf, toks, ua, ur = _tree_inputs(B, nodes, V, dtype, T, top_p, seed=V)
+    Ts, Ps = torch.full((B,), T), torch.full((B,), top_p)
+    out = psispec.verify_tree(_cuda(tgt), _cuda(drf), _cuda(trie.node_offsets), _cuda(trie.parent), _cuda(toks),
+                              _cuda(ua), _cuda(ur), _cuda(Ts), _cuda(Ps), 6)
+    ora = oracle.verify_tree(tgt, drf, trie.node_offsets.numpy(), trie.parent.numpy(), toks.numpy(), ua, ur,
+                             Ts.numpy(), Ps.numpy(), 6)
+    compare_tree(out, ora)
+
+
+def test_branching_one_tree_equals_linear_gpu():
+    B, K, V = 6, 5, 12000
+    tgt, drf, ud, ua, ur, Ts, Ps = _linear_inputs(B, K, V, torch.bfloat16, 0.9, 0.95, 0.6, seed=31)
+    x, _, _ = psispec.sample_draft(_cuda(drf), _cuda(Ts), _cuda(Ps), _cuda(ud))
+    lin = psispec.verify_linear(_cuda(tgt), _cuda(drf), x, _cuda(ua), _cuda(ur), _cuda(Ts), _cuda(Ps))
+    N = B * (K + 1)
+    d_rows = torch.cat([drf, torch.zeros((B, 1, V), dtype=drf.dtype)], dim=1).reshape(N, V)
+    parent = torch.arange(-1, K, dtype=torch.int32).repeat(B)
+    tok = torch.zeros((B, K + 1), dtype=torch.int32)
+    tok[:, 1:] = x.cpu()
+    uacc = torch.zeros((B, K + 1))
+    uacc[:, 1:] = ua
+    tr = psispec.verify_tree(_cuda(tgt.reshape(N, V)), _cuda(d_rows), _cuda(torch.arange(0, N + 1, K + 1, dtype=torch.int32)),
+                             _cuda(parent), _cuda(tok.reshape(-1)), _cuda(uacc.reshape(-1)), _cuda(ur.reshape(-1)),
+                             _cuda(Ts), _cuda(Ps), K)
+    assert torch.equal(lin["accept_len"], tr["accept_len"])
+    assert torch.equal(lin["tokens"], tr["tokens"])
+
+
+# ------------------------------------------------------------------ full-size workloads
+
+
+def _sampled(B, n):
+    return np.unique(np.linspace(0, B - 1, n).astype(int))
+
+
+@pytest.mark.parametrize("name", ["mid", "max", "sweep_b32_t0", "sweep_b32_t0.7", "sweep_b1_t1"])
+def test_full_size_linear_sampled(name):
+    case = synth.linear_cases()[name]
+    B, K, V = case.B, case.K, case.V
+    tgt, drf = synth.linear_logits(case, device=DEV)
+    ud, ua, ur = synth.linear_uniforms(case)
+    Ts, Ps = torch.full((B,), case.temperature), torch.full((B,), case.top_p)
+    x, q, stats = psispec.sample_draft(drf, _cuda(Ts), _cuda(Ps), _cuda(ud))
+    pick = _sampled(B, 4 if B >= 256 else 6)
+    idx = torch.as_tensor(pick, device=DEV)
+    d_host = drf[idx].cpu()
+    o_s = oracle.sample_draft(d_host.reshape(-1, V), Ts[pick].numpy(), Ps[pick].numpy(), ud[pick].reshape(-1),
+                              row_req=np.arange(len(pick) * K) // K)
+    compare_sample(x[idx], q[idx], o_s)
+    # the oracle's draft tokens replace the sampled requests' rows
+    x_in = x.clone()
+    x_in[idx] = torch.from_numpy(o_s["tokens"].reshape(len(pick), K)).to(DEV)
+    out = psispec.verify_linear(tgt, drf, x_in, _cuda(ua), _cuda(ur), _cuda(Ts), _cuda(Ps), draft_row_stats=stats)
+    ora = oracle.verify_linear(tgt[idx].cpu(), d_host, o_s["tokens"].reshape(len(pick), K), ua[pick], ur[pick],
+                               Ts[pick].numpy(), Ps[pick].numpy())
+    sub = {k: v[idx] for k, v in out.items()}
+    stats_report = compare_linear(sub, ora)
+    lens = out["accept_len"].cpu().numpy()
+    assert (lens >= 0).all() and (lens <= K).all()
+    print(name, stats_report, "gpu mean accept", lens.mean())
+
+
+def test_full_size_tree():
+    case = synth.tree_cases()["tree"]
+    trie, tgt, drf, toks, ua, ur = synth.tree_inputs(case, device=DEV)
+    B = case.B
+    Ts, Ps = torch.full((B,), case.temperature), torch.full((B,), case.top_p)
+    out = psispec.verify_tree(tgt, drf, _cuda(trie.node_offsets), _cuda(trie.parent), _cuda(toks), _cuda(ua), _cuda(ur),
+                              _cuda(Ts), _cuda(Ps), case.max_depth)
+    ora = oracle.verify_tree(tgt.cpu(), drf.cpu(), trie.node_offsets.numpy(), trie.parent.numpy(), toks.numpy(), ua, ur,
+                             Ts.numpy(), Ps.numpy(), case.max_depth)
+    print("tree", compare_tree(out, ora), "accept", out["accept_len"].tolist())
