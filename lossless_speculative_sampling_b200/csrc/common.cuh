@@ -4,8 +4,10 @@
 //   * a logit l of a row with statistics (m, c) has weight w = 2^((l - m) * c), c = log2(e)/T,
 //     evaluated with the hardware ex2.approx instruction (ftz); m is the row maximum, so
 //     every weight is in [0, 1];
-//   * per-thread sums are fp32, block and cross-slice combinations of probability mass that
-//     feed an inverse-CDF draw are fp64;
+//   * weights are summed in fp32 over one 16-byte vector (at most 8 terms) and accumulated in
+//     fp64 from there on (per thread, across threads, across slices, in top-p histograms), so
+//     normalisers and CDF totals carry about the ex2 error (~1e-7 relative), not the
+//     accumulation error of long fp32 sums;
 //   * top-p thresholds are compared on order-preserving 32-bit keys of the logit values, so
 //     ties are kept or dropped together.
 #pragma once
@@ -34,9 +36,10 @@ static_assert(sizeof(RowStat) == 32, "row stats record is 32 bytes");
 
 // Partial statistics of one (row, slice) work unit.
 struct Partial {
+  double s;  // sum of 2^((l - m) c) over the slice, relative to this slice's own maximum m
   float m;
-  float s;  // relative to this slice's own maximum
   int32_t amax;
+  int32_t bad;
   int32_t pad;
 };
 

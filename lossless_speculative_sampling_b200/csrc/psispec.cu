@@ -122,7 +122,7 @@ psispec_status sample_draft_impl(const T* draft, int B, int K, int V, const floa
                                                                               ns, w.cdf);
   if ((s = launched()) != PSISPEC_OK) return s;
   cdf_pick_kernel<T><<<static_cast<unsigned>(rows), kThreads, 0, st>>>(draft, draft, stats, stats, w.jobs, V, ns,
-                                                                       w.cdf, out_tokens, out_q);
+                                                                       w.st.parts, w.cdf, out_tokens, out_q);
   return launched();
 }
 
@@ -151,7 +151,8 @@ psispec_status verify_linear_impl(const T* tgt, const T* drf, int B, int K, int 
   cdf_partial_kernel<T><<<static_cast<unsigned>(int64_t(B) * ns), kThreads, 0, st>>>(tgt, drf, w.t.stats, ds, w.jobs,
                                                                                      V, ns, w.cdf);
   if ((s = launched()) != PSISPEC_OK) return s;
-  cdf_pick_kernel<T><<<B, kThreads, 0, st>>>(tgt, drf, w.t.stats, ds, w.jobs, V, ns, w.cdf, out_tokens, nullptr);
+  cdf_pick_kernel<T><<<B, kThreads, 0, st>>>(tgt, drf, w.t.stats, ds, w.jobs, V, ns, w.t.parts, w.cdf, out_tokens,
+                                              nullptr);
   return launched();
 }
 

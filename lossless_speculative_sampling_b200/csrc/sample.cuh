@@ -6,16 +6,19 @@
 // section 3.3): a row's own distribution (drafting, and the bonus token after a fully
 // accepted block) and the residual max(0, p - q) of a rejected position.
 //
-//   cdf_partial_kernel  one CTA per (job, slice): the slice's total weight (fp64), plus the
-//                       total of p for the fallback when the residual is zero everywhere;
-//   cdf_pick_kernel     one CTA per job: locates the slice holding u * Z from the slice
-//                       totals, splits it into one contiguous run per thread, scans the run
-//                       totals (fp64, thread order) and lets the owning thread walk its run.
+// The draw is hierarchical. Slice totals (kSliceElems elements each) locate the slice that
+// holds u * Z; they come from the row-statistics partials when the row's own distribution
+// has no top-p cut, and from cdf_partial_kernel otherwise (a residual, or a kept set). Then
+// one CTA scans that slice: each warp totals a contiguous kWarpSpan sub-range with coalesced
+// 16-byte loads, a block scan picks the owning warp, which walks its sub-range 256 elements
+// at a time with warp scans; the owning lane walks its 8 elements. All prefix sums are fp64.
 #pragma once
 
 #include "common.cuh"
 
 namespace psi {
+
+constexpr int kWarpSpan = kSliceElems / (kThreads / 32);  // elements per warp in a slice scan
 
 struct ResidCtx {
   RowStat a, b;
@@ -29,15 +32,57 @@ __device__ __forceinline__ void resid_weight(const ResidCtx& r, float xa, float 
   res = fmaxf(pa - qb, 0.0f);
 }
 
-// Weight of element v for a job; `use_p` selects p_a for a residual job whose residual is 0.
+// 8 consecutive elements starting at e (elements at or past `end` read as -inf)
 template <typename T>
-__device__ __forceinline__ float job_weight(int mode, bool use_p, const ResidCtx& r, const T* ra, const T* rb, int v) {
-  float xa = load_elem(ra + v);
-  if (mode == kSample) return kept_weight(r.a, xa);
-  float res, pa;
-  resid_weight(r, xa, load_elem(rb + v), res, pa);
-  return use_p ? pa : res;
+__device__ __forceinline__ void load8(const T* __restrict__ row, int e, int end, bool aligned, float (&x)[8]) {
+  if (aligned && e + 8 <= end) {
+    if (sizeof(T) == 2) {
+      Vec<T>::load(row + e, x);
+    } else {
+      float lo[8], hi[8];
+      Vec<T>::load(row + e, lo);
+      Vec<T>::load(row + e + 4, hi);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) { x[k] = lo[k]; x[k + 4] = hi[k]; }
+    }
+  } else {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) x[k] = e + k < end ? load_elem(row + e + k) : -INFINITY;
+  }
 }
+
+template <typename T>
+struct JobRows {
+  int mode;
+  bool use_p;
+  ResidCtx r;
+  const T* ra;
+  const T* rb;
+  bool al_a, al_b;
+  int end;
+
+  // weights of elements e .. e+7; returns their fp32 sum
+  __device__ __forceinline__ float weights8(int e, float (&w)[8]) const {
+    float xa[8];
+    load8(ra, e, end, al_a, xa);
+    float sum = 0.0f;
+    if (mode == kSample) {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) { w[k] = kept_weight(r.a, xa[k]); sum += w[k]; }
+    } else {
+      float xb[8];
+      load8(rb, e, end, al_b, xb);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        float res, pa;
+        resid_weight(r, xa[k], xb[k], res, pa);
+        w[k] = use_p ? pa : res;
+        sum += w[k];
+      }
+    }
+    return sum;
+  }
+};
 
 template <typename T>
 __global__ void __launch_bounds__(kThreads) cdf_partial_kernel(const T* __restrict__ A, const T* __restrict__ Bt,
@@ -50,12 +95,13 @@ __global__ void __launch_bounds__(kThreads) cdf_partial_kernel(const T* __restri
   const int job = unit / nslices, slice = unit - job * nslices;
   const Job jb = jobs[job];
   if (jb.mode < kSample) return;
-  const int v0 = slice * kSliceElems, v1 = min(V, v0 + kSliceElems);
   ResidCtx r;
   r.a = sa[jb.row_a];
+  if (jb.mode == kSample && r.a.tau == 0u) return;  // slice totals come from the row statistics
+  const int v0 = slice * kSliceElems, v1 = min(V, v0 + kSliceElems);
   r.ia = 1.0f / r.a.s_kept;
   const T* ra = A + static_cast<size_t>(jb.row_a) * V;
-  float sr = 0.0f, sp = 0.0f;
+  double sr = 0.0, sp = 0.0;
   constexpr int N = Vec<T>::N;
   if (jb.mode == kSample) {
     int a0, a1;
@@ -63,10 +109,11 @@ __global__ void __launch_bounds__(kThreads) cdf_partial_kernel(const T* __restri
     for (int v = v0 + threadIdx.x; v < a0; v += blockDim.x) sr += kept_weight(r.a, load_elem(ra + v));
     for (int v = a1 + threadIdx.x; v < v1; v += blockDim.x) sr += kept_weight(r.a, load_elem(ra + v));
     for (int v = a0 + threadIdx.x * N; v < a1; v += blockDim.x * N) {
-      float x[8];
+      float x[8], acc = 0.0f;
       Vec<T>::load(ra + v, x);
 #pragma unroll
-      for (int k = 0; k < N; ++k) sr += kept_weight(r.a, x[k]);
+      for (int k = 0; k < N; ++k) acc += kept_weight(r.a, x[k]);
+      sr += static_cast<double>(acc);
     }
   } else {
     r.b = sb[jb.row_b];
@@ -76,54 +123,70 @@ __global__ void __launch_bounds__(kThreads) cdf_partial_kernel(const T* __restri
     vec_range(ra, v0, v1, a0, a1);
     vec_range(rb, v0, v1, b0, b1);
     if (a0 != b0) { a0 = v1; a1 = v1; }  // rows aligned differently: scalar path
-    auto one = [&](float xa, float xb) {
+    auto one = [&](float xa, float xb, float& ar, float& ap) {
       float res, pa;
       resid_weight(r, xa, xb, res, pa);
-      sr += res;
-      sp += pa;
+      ar += res;
+      ap += pa;
     };
-    for (int v = v0 + threadIdx.x; v < a0; v += blockDim.x) one(load_elem(ra + v), load_elem(rb + v));
-    for (int v = a1 + threadIdx.x; v < v1; v += blockDim.x) one(load_elem(ra + v), load_elem(rb + v));
+    float ar = 0.0f, ap = 0.0f;
+    for (int v = v0 + threadIdx.x; v < a0; v += blockDim.x) one(load_elem(ra + v), load_elem(rb + v), ar, ap);
+    for (int v = a1 + threadIdx.x; v < v1; v += blockDim.x) one(load_elem(ra + v), load_elem(rb + v), ar, ap);
+    sr += ar;
+    sp += ap;
     for (int v = a0 + threadIdx.x * N; v < a1; v += blockDim.x * N) {
       float xa[8], xb[8];
       Vec<T>::load(ra + v, xa);
       Vec<T>::load(rb + v, xb);
+      ar = 0.0f;
+      ap = 0.0f;
 #pragma unroll
-      for (int k = 0; k < N; ++k) one(xa[k], xb[k]);
+      for (int k = 0; k < N; ++k) one(xa[k], xb[k], ar, ap);
+      sr += static_cast<double>(ar);
+      sp += static_cast<double>(ap);
     }
   }
-  double tr = block_sum(static_cast<double>(sr), red);
-  double tp = block_sum(static_cast<double>(sp), red);
+  double tr = block_sum(sr, red);
+  double tp = block_sum(sp, red);
   if (threadIdx.x == 0) out[unit] = make_double2(tr, tp);
 }
 
+// parts_a: row-statistics partials of tensor A (used for sample jobs without a top-p cut)
 template <typename T>
 __global__ void __launch_bounds__(kThreads) cdf_pick_kernel(const T* __restrict__ A, const T* __restrict__ Bt,
                                                             const RowStat* __restrict__ sa,
                                                             const RowStat* __restrict__ sb, const Job* __restrict__ jobs,
-                                                            int V, int nslices, const double2* __restrict__ parts,
-                                                            int32_t* __restrict__ out_tokens, float* __restrict__ out_q) {
-  __shared__ double red[33];
-  __shared__ int sh_slice, sh_use_p, sh_y, sh_last;
-  __shared__ double sh_base, sh_target;
+                                                            int V, int nslices, const Partial* __restrict__ parts_a,
+                                                            const double2* __restrict__ parts, int32_t* __restrict__ out_tokens,
+                                                            float* __restrict__ out_q) {
+  __shared__ double wtot[kThreads / 32];
+  __shared__ int sh_slice, sh_use_p, sh_y, sh_last, sh_owner;
+  __shared__ double sh_base, sh_target, sh_c0;
   const Job jb = jobs[blockIdx.x];
   if (jb.mode < kSample) return;
-  const double2* pp = parts + static_cast<size_t>(blockIdx.x) * nslices;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const RowStat sta = sa[jb.row_a];
+  const bool from_stats = jb.mode == kSample && sta.tau == 0u;
   if (threadIdx.x == 0) {
+    const double2* pp = parts + static_cast<size_t>(blockIdx.x) * nslices;
+    const Partial* ps = parts_a + static_cast<size_t>(jb.row_a) * nslices;
+    auto total = [&](int s, int use_p) -> double {
+      if (from_stats) return ps[s].m > -INFINITY ? ps[s].s * static_cast<double>(ex2((ps[s].m - sta.m) * sta.c)) : 0.0;
+      return use_p ? pp[s].y : pp[s].x;
+    };
     double Z = 0.0;
-    for (int s = 0; s < nslices; ++s) Z += pp[s].x;
+    for (int s = 0; s < nslices; ++s) Z += total(s, 0);
     int use_p = 0;
     if (jb.mode == kResidual && !(Z > 0.0)) {  // zero residual: draw from p instead
       use_p = 1;
       Z = 0.0;
-      for (int s = 0; s < nslices; ++s) Z += pp[s].y;
+      for (int s = 0; s < nslices; ++s) Z += total(s, 1);
     }
     const double target = static_cast<double>(jb.u) * Z;
-    double C = 0.0;
+    double C = 0.0, base = 0.0;
     int sel = -1;
-    double base = 0.0;
     for (int s = 0; s < nslices; ++s) {
-      double w = use_p ? pp[s].y : pp[s].x;
+      const double w = total(s, use_p);
       if (w > 0.0) { sel = s; base = C; }
       if (C + w > target && w > 0.0) break;
       C += w;
@@ -134,6 +197,7 @@ __global__ void __launch_bounds__(kThreads) cdf_pick_kernel(const T* __restrict_
     sh_target = target;
     sh_y = 0x7fffffff;
     sh_last = -1;
+    sh_owner = -1;
   }
   __syncthreads();
   const int sel = sh_slice;
@@ -144,46 +208,100 @@ __global__ void __launch_bounds__(kThreads) cdf_pick_kernel(const T* __restrict_
     }
     return;
   }
-  ResidCtx r;
-  r.a = sa[jb.row_a];
-  r.ia = 1.0f / r.a.s_kept;
-  const T* ra = A + static_cast<size_t>(jb.row_a) * V;
-  const T* rb = nullptr;
+  JobRows<T> J;
+  J.mode = jb.mode;
+  J.use_p = sh_use_p != 0;
+  J.r.a = sta;
+  J.r.ia = 1.0f / sta.s_kept;
+  J.ra = A + static_cast<size_t>(jb.row_a) * V;
+  J.rb = nullptr;
+  J.al_a = (reinterpret_cast<uintptr_t>(J.ra) & 15u) == 0;
+  J.al_b = false;
   if (jb.mode == kResidual) {
-    r.b = sb[jb.row_b];
-    r.ib = 1.0f / r.b.s_kept;
-    rb = Bt + static_cast<size_t>(jb.row_b) * V;
+    J.r.b = sb[jb.row_b];
+    J.r.ib = 1.0f / J.r.b.s_kept;
+    J.rb = Bt + static_cast<size_t>(jb.row_b) * V;
+    J.al_b = (reinterpret_cast<uintptr_t>(J.rb) & 15u) == 0;
   }
-  const bool use_p = sh_use_p != 0;
   const int v0 = sel * kSliceElems, v1 = min(V, v0 + kSliceElems);
-  const int run = (v1 - v0 + blockDim.x - 1) / blockDim.x;
-  const int r0 = min(v1, v0 + threadIdx.x * run), r1 = min(v1, r0 + run);
+  const int w0 = v0 + warp * kWarpSpan, w1 = min(v1, w0 + kWarpSpan);
+  J.end = w1;
+  const double target = sh_target;
+
+  // phase 1: per-warp totals of contiguous sub-ranges
   double mine = 0.0;
   int last = -1;
-  for (int v = r0; v < r1; ++v) {
-    float w = job_weight<T>(jb.mode, use_p, r, ra, rb, v);
-    mine += static_cast<double>(w);
-    if (w > 0.0f) last = v;
+  for (int e = w0 + lane * 8; e < w1; e += 256) {
+    float w[8];
+    mine += static_cast<double>(J.weights8(e, w));
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      if (w[k] > 0.0f) last = e + k;
   }
-  double total;
-  const double C0 = sh_base + block_exclusive_scan(mine, red, &total);
-  if (last >= 0) atomicMax(&sh_last, last);
-  const double target = sh_target;
-  if (C0 <= target && target < C0 + mine) {
-    double C = C0;
-    for (int v = r0; v < r1; ++v) {
-      C += static_cast<double>(job_weight<T>(jb.mode, use_p, r, ra, rb, v));
-      if (C > target) {
-        atomicMin(&sh_y, v);
-        break;
-      }
-    }
+  mine = warp_sum(mine);
+  last = __reduce_max_sync(0xffffffffu, last);
+  if (lane == 0) {
+    wtot[warp] = mine;
+    if (last >= 0) atomicMax(&sh_last, last);
   }
   __syncthreads();
   if (threadIdx.x == 0) {
-    int y = sh_y != 0x7fffffff ? sh_y : sh_last;  // rounding at a run edge: last positive entry
+    double C = sh_base;
+    for (int i = 0; i < kThreads / 32; ++i) {
+      if (C <= target && target < C + wtot[i]) { sh_owner = i; sh_c0 = C; break; }
+      C += wtot[i];
+    }
+  }
+  __syncthreads();
+
+  // phase 2: the owning warp walks its sub-range, 256 elements per step (vector sums in fp64
+  // so that the lane walk below retraces the scanned totals)
+  if (warp == sh_owner) {
+    double Cb = sh_c0;
+    int wlast = -1;
+    for (int e = w0 + lane * 8; e - lane * 8 < w1; e += 256) {
+      float w[8];
+      J.weights8(e, w);
+      double vs = 0.0;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        vs += static_cast<double>(w[k]);
+        if (w[k] > 0.0f) wlast = e + k;
+      }
+      double incl = vs;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const double y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      double excl = __shfl_up_sync(0xffffffffu, incl, 1);
+      if (lane == 0) excl = 0.0;
+      const unsigned hit = __ballot_sync(0xffffffffu, Cb + incl > target);
+      if (hit) {
+        if (lane == __ffs(hit) - 1) {
+          double C = Cb + excl;
+          int y = -1, lastpos = -1;
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            C += static_cast<double>(w[k]);
+            if (w[k] > 0.0f) lastpos = e + k;
+            if (y < 0 && C > target) y = e + k;
+          }
+          sh_y = y >= 0 ? y : lastpos;  // rounding at the group's end: its last positive entry
+        }
+        break;
+      }
+      Cb += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    // no crossing found (rounding against the phase-1 total): the warp's last positive entry
+    wlast = __reduce_max_sync(0xffffffffu, wlast);
+    if (lane == 0 && sh_y == 0x7fffffff && wlast >= 0) sh_y = wlast;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const int y = sh_y != 0x7fffffff ? sh_y : sh_last;  // rounding at a sub-range edge: last positive entry
     out_tokens[jb.out_index] = y;
-    if (out_q && jb.aux >= 0) out_q[jb.aux] = kept_weight(r.a, load_elem(ra + y)) / r.a.s_kept;
+    if (out_q && jb.aux >= 0) out_q[jb.aux] = kept_weight(sta, load_elem(J.ra + y)) / sta.s_kept;
   }
 }
 

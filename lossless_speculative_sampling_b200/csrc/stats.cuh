@@ -18,51 +18,77 @@
 
 namespace psi {
 
-// Online max/sum over [v0, v1) of one row, per thread. Returns via references.
+// Online max/sum over [v0, v1) of one row, per thread. The vector body batches kBatch
+// 16-byte loads before using them (memory-level parallelism) and sums weights per vector in
+// fp32, accumulating vector sums with a compensated (Kahan) fp32 sum: ~1 ulp overall without
+// fp64 work in the loop.
+constexpr int kBatch = 4;
+
 template <typename T, bool GREEDY>
 __device__ __forceinline__ void thread_slice_stats(const T* __restrict__ row, int v0, int v1, float c, float& m,
-                                                   float& s, int& amax, bool& bad) {
+                                                   double& s_out, int& amax, bool& bad) {
   constexpr int N = Vec<T>::N;
   int a0, a1;
   vec_range(row, v0, v1, a0, a1);
+  float s = 0.0f, comp = 0.0f;
+  auto add = [&](float y) {  // compensated s += y
+    y -= comp;
+    const float t = s + y;
+    comp = (t - s) - y;
+    s = t;
+  };
+  auto rescale = [&](float nm) {
+    const float f = ex2((m - nm) * c);
+    s *= f;
+    comp *= f;
+    m = nm;
+  };
   auto scalar = [&](int v) {
     float x = load_elem(row + v);
     bad |= !(x < INFINITY);
     if (GREEDY) {
       if (x > m) { m = x; amax = v; }
     } else {
-      if (x > m) { s *= ex2((m - x) * c); m = x; }
-      if (m > -INFINITY) s += ex2((x - m) * c);
+      if (x > m) rescale(x);
+      if (m > -INFINITY) add(ex2((x - m) * c));
     }
   };
   // head and tail elements (fewer than N each), then the aligned body
   for (int v = v0 + threadIdx.x; v < a0; v += blockDim.x) scalar(v);
   for (int v = a1 + threadIdx.x; v < v1; v += blockDim.x) scalar(v);
-#pragma unroll 2
-  for (int v = a0 + threadIdx.x * N; v < a1; v += blockDim.x * N) {
-    float f[8];
-    Vec<T>::load(row + v, f);
-    float vmax = f[0];
+  const int stride = blockDim.x * N;
+  for (int vb = a0 + threadIdx.x * N; vb < a1; vb += kBatch * stride) {
+    float f[kBatch][8];
 #pragma unroll
-    for (int k = 1; k < N; ++k) vmax = fmax_nan(vmax, f[k]);
-    bad |= !(vmax < INFINITY);
-    if (GREEDY) {
-      if (vmax > m) {
+    for (int u = 0; u < kBatch; ++u)
+      if (vb + u * stride < a1) Vec<T>::load(row + vb + u * stride, f[u]);
 #pragma unroll
-        for (int k = N - 1; k >= 0; --k)
-          if (f[k] == vmax) amax = v + k;
-        m = vmax;
-      }
-    } else {
-      if (vmax > m) { s *= ex2((m - vmax) * c); m = vmax; }
-      if (m > -INFINITY) {
-        float acc = 0.0f;
+    for (int u = 0; u < kBatch; ++u) {
+      const int v = vb + u * stride;
+      if (v >= a1) break;
+      float vmax = f[u][0];
 #pragma unroll
-        for (int k = 0; k < N; ++k) acc += ex2((f[k] - m) * c);
-        s += acc;
+      for (int k = 1; k < N; ++k) vmax = fmax_nan(vmax, f[u][k]);
+      bad |= !(vmax < INFINITY);
+      if (GREEDY) {
+        if (vmax > m) {
+#pragma unroll
+          for (int k = N - 1; k >= 0; --k)
+            if (f[u][k] == vmax) amax = v + k;
+          m = vmax;
+        }
+      } else {
+        if (vmax > m) rescale(vmax);
+        if (m > -INFINITY) {
+          float acc = 0.0f;
+#pragma unroll
+          for (int k = 0; k < N; ++k) acc += ex2((f[u][k] - m) * c);
+          add(acc);
+        }
       }
     }
   }
+  s_out = static_cast<double>(s) - static_cast<double>(comp);
 }
 
 __device__ __forceinline__ float temp_scale(float T) {
@@ -80,13 +106,15 @@ __global__ void __launch_bounds__(kThreads) row_partial_kernel(const T* __restri
                                                                 int nslices, const float* __restrict__ temperature,
                                                                 Partial* __restrict__ out) {
   __shared__ float red[32];
+  __shared__ double dred[33];
   __shared__ int ired[32];
   const int unit = blockIdx.x;
   const int row = unit / nslices, slice = unit - row * nslices;
   const float c = temp_scale(temperature[row_request(row, rows_per_req, row_req)]);
   const T* rp = base + static_cast<size_t>(row) * V;
   const int v0 = slice * kSliceElems, v1 = min(V, v0 + kSliceElems);
-  float m = -INFINITY, s = 0.0f;
+  float m = -INFINITY;
+  double s = 0.0;
   int amax = 0x7fffffff;
   bool bad = false;
   if (c == 0.0f) {
@@ -104,14 +132,14 @@ __global__ void __launch_bounds__(kThreads) row_partial_kernel(const T* __restri
       if (threadIdx.x == 0) ired[0] = x;
     }
     bad = __syncthreads_or(bad);
-    if (threadIdx.x == 0) out[unit] = Partial{M, 0.0f, ired[0], bad ? 1 : 0};
+    if (threadIdx.x == 0) out[unit] = Partial{0.0, M, ired[0], bad ? 1 : 0, 0};
   } else {
     thread_slice_stats<T, false>(rp, v0, v1, c, m, s, amax, bad);
     float M = block_max(m, red);
-    float mine = (m > -INFINITY) ? s * ex2((m - M) * c) : 0.0f;
-    float S = block_sum(mine, red);
+    double mine = (m > -INFINITY) ? s * static_cast<double>(ex2((m - M) * c)) : 0.0;
+    double S = block_sum(mine, dred);
     bad = __syncthreads_or(bad);
-    if (threadIdx.x == 0) out[unit] = Partial{M, S, 0, bad ? 1 : 0};
+    if (threadIdx.x == 0) out[unit] = Partial{S, M, 0, bad ? 1 : 0, 0};
   }
 }
 
@@ -140,7 +168,7 @@ __global__ void __launch_bounds__(kThreads) row_finalize_kernel(
     RowStat* __restrict__ stats,
     const float* __restrict__ u, Job* __restrict__ jobs, int32_t* __restrict__ out_tokens,
     float* __restrict__ out_q) {
-  __shared__ float hmass[256];
+  __shared__ double hmass[256];
   __shared__ int hcnt[256];
   __shared__ RowStat st;
   __shared__ uint32_t sh_prefix;
@@ -156,15 +184,15 @@ __global__ void __launch_bounds__(kThreads) row_finalize_kernel(
     bool bad = !(Tv >= 0.0f && Tv < INFINITY);
     for (int i = lane; i < nslices; i += 32) {
       M = fmax_nan(M, pp[i].m);
-      bad |= pp[i].pad != 0;
+      bad |= pp[i].bad != 0;
     }
     M = warp_max(M);
-    float S = 0.0f;
+    double S = 0.0;
     int amax = 0x7fffffff;
     for (int i = lane; i < nslices; i += 32) {
       Partial q = pp[i];
       if (c != 0.0f) {
-        if (q.m > -INFINITY) S += q.s * ex2((q.m - M) * c);
+        if (q.m > -INFINITY) S += q.s * static_cast<double>(ex2((q.m - M) * c));
       } else if (q.m == M) {
         amax = min(amax, q.amax);
       }
@@ -175,7 +203,7 @@ __global__ void __launch_bounds__(kThreads) row_finalize_kernel(
     if (lane == 0) {
       st.m = M;
       st.c = c;
-      st.s = c != 0.0f ? S : 1.0f;
+      st.s = c != 0.0f ? static_cast<float>(S) : 1.0f;
       st.s_kept = st.s;
       st.tau = 0u;
       st.amax = c != 0.0f ? -1 : amax;
@@ -191,19 +219,19 @@ __global__ void __launch_bounds__(kThreads) row_finalize_kernel(
     // bf16 rows the two top digits already separate every distinct value.
     const T* rp = base + static_cast<size_t>(row) * V;
     const float M = st.m;
-    const float target = tp * st.s;
+    const double target = static_cast<double>(tp) * static_cast<double>(st.s);
     const int levels = sizeof(T) == 2 ? 2 : 4;
     if (threadIdx.x == 0) { sh_prefix = 0u; sh_above = 0.0; sh_bucket = 0.0; }
     for (int lv = 0; lv < levels; ++lv) {
       const int shift = 24 - 8 * lv;
-      for (int d = threadIdx.x; d < 256; d += blockDim.x) { hmass[d] = 0.0f; hcnt[d] = 0; }
+      for (int d = threadIdx.x; d < 256; d += blockDim.x) { hmass[d] = 0.0; hcnt[d] = 0; }
       __syncthreads();
       const uint32_t prefix = sh_prefix;
       for_each_elem(rp, V, [&](float x) {
         uint32_t k = fkey(x);
         if (lv == 0 || (k >> (shift + 8)) == (prefix >> (shift + 8))) {
           int d = (k >> shift) & 255;
-          atomicAdd(&hmass[d], ex2((x - M) * c));
+          atomicAdd(&hmass[d], static_cast<double>(ex2((x - M) * c)));
           atomicAdd(&hcnt[d], 1);
         }
       });
