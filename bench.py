@@ -29,10 +29,10 @@ sys.path.insert(0, ROOT)
 
 METRIC = "verified draft positions/sec and logits HBM GB/s vs B200 peak (Ψ-Spec verify)"
 UNIT = "positions/s"
-# kernel launches per call (see csrc/psispec.cu): sample_draft = stats partial + finalize +
-# cdf partial + cdf pick; verify_linear with draft statistics = stats partial + finalize +
-# decide + cdf partial + cdf pick
-LAUNCHES_PER_STEP = 4 + 5
+# kernel launches per call (see csrc/psispec.cu): sample_draft = stream + finish + top-p;
+# verify_linear = stream + finish + top-p + clustered draw (the per-request
+# arrival counters are cleared with a memset, which is not a kernel of this library)
+LAUNCHES_PER_STEP = 3 + 4
 
 
 def _peaks():
@@ -216,9 +216,34 @@ def run_ours(args):
         psispec.verify_linear(t_in, d_in, x, ua, ur, Ts, Ps, draft_row_stats=stats, out_tokens=o_tok,
                               out_accept_len=o_len, out_p=o_p, out_q=o_q, ws=ws_v)
 
+    def call_sample():
+        psispec.sample_draft(drf, Ts, Ps, ud, out_tokens=x, out_q=q, row_stats=stats, ws=ws_s)
+
+    def call_verify():
+        psispec.verify_linear(tgt, drf, x, ua, ur, Ts, Ps, draft_row_stats=stats, out_tokens=o_tok,
+                              out_accept_len=o_len, out_p=o_p, out_q=o_q, ws=ws_v)
+
     for _ in range(args.warmup):
         step(tgt, drf)
     torch.cuda.synchronize()
+    if not args.no_graph:
+        # each call is captured once and replayed: the launch sequence a serving loop would use
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(side):
+            call_sample()
+            call_verify()
+        torch.cuda.current_stream(dev).wait_stream(side)
+        g_s, g_v = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_s):
+            call_sample()
+        with torch.cuda.graph(g_v):
+            call_verify()
+        call_sample, call_verify = g_s.replay, g_v.replay
+        for _ in range(args.warmup):
+            call_sample()
+            call_verify()
+        torch.cuda.synchronize()
     _barrier(dist)
 
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(3 * args.steps)]
@@ -229,10 +254,9 @@ def run_ours(args):
         start.record()
         for k in range(args.steps):
             ev[3 * k].record()
-            psispec.sample_draft(drf, Ts, Ps, ud, out_tokens=x, out_q=q, row_stats=stats, ws=ws_s)
+            call_sample()
             ev[3 * k + 1].record()
-            psispec.verify_linear(tgt, drf, x, ua, ur, Ts, Ps, draft_row_stats=stats, out_tokens=o_tok,
-                                  out_accept_len=o_len, out_p=o_p, out_q=o_q, ws=ws_v)
+            call_verify()
             ev[3 * k + 2].record()
         end.record()
         torch.cuda.synchronize()
@@ -299,7 +323,8 @@ def run_ours(args):
             "config": {"workload": "%s: linear verify B=%d K=%d V=%d %s, T=%g, top-p %g" % (
                 args.workload, B, K, V, "bf16" if esz == 2 else "fp32", case.temperature, case.top_p),
                 "global_batch": B * world, "block": K, "vocab": V, "parallelism": "replicas x%d" % world,
-                "l2": "inputs %.0f MB > 126 MB L2, no flush" % (bytes_step / 1e6)},
+                "l2": "inputs %.0f MB > 126 MB L2, no flush" % (bytes_step / 1e6),
+                "cuda_graph": not args.no_graph},
             "roofline": {"bound": "hbm", "kernel": "psispec_verify_linear", "achieved": gbs_verify, "peak": peak,
                          "unit": "GB/s", "frac": gbs_verify / peak, "peak_kind": peak_kind,
                          "traffic": _traffic(args.workload)},
@@ -326,6 +351,7 @@ def main():
     ap.add_argument("--workload", default="mid")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="launch calls directly instead of replaying CUDA graphs")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-requests", type=int, default=2)
     args = ap.parse_args()

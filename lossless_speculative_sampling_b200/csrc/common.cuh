@@ -18,8 +18,12 @@
 
 namespace psi {
 
-constexpr int kThreads = 256;       // threads per CTA of the streaming kernels
-constexpr int kSliceElems = 16384;  // vocabulary elements per slice (work unit of a CTA)
+constexpr int kThreads = 256;                               // threads per CTA of the streaming kernels
+constexpr int kChunkElems = 2048;                           // contiguous elements per warp (one partial)
+constexpr int kSliceElems = kChunkElems * (kThreads / 32);  // elements per CTA work unit
+
+__host__ __device__ inline int nchunks_for(int64_t V) { return static_cast<int>((V + kChunkElems - 1) / kChunkElems); }
+__host__ __device__ inline int nslices_for(int64_t V) { return static_cast<int>((V + kSliceElems - 1) / kSliceElems); }
 
 // Per-row statistics record (32 bytes; also the public row-stats record).
 struct RowStat {
@@ -34,14 +38,15 @@ struct RowStat {
 };
 static_assert(sizeof(RowStat) == 32, "row stats record is 32 bytes");
 
-// Partial statistics of one (row, slice) work unit.
+// Partial statistics of one (row, chunk): a warp's contiguous kChunkElems elements.
 struct Partial {
-  double s;  // sum of 2^((l - m) c) over the slice, relative to this slice's own maximum m
+  double s;  // sum of 2^((l - m) c) over the chunk, relative to the chunk's own maximum m
   float m;
   int32_t amax;
   int32_t bad;
   int32_t pad;
 };
+static_assert(sizeof(Partial) == 24 && offsetof(Partial, m) == 8 && offsetof(Partial, bad) == 16, "partial layout");
 
 // Inverse-CDF job: draw from row a of tensor A (mode kSample) or from max(0, pA - qB)
 // (mode kResidual), with uniform u; the result goes to out_tokens[out_index].
@@ -91,22 +96,31 @@ struct Vec;
 template <>
 struct Vec<float> {
   static constexpr int N = 4;
+  __device__ __forceinline__ static void unpack(const uint4& v, float (&f)[8]) {
+    f[0] = __uint_as_float(v.x);
+    f[1] = __uint_as_float(v.y);
+    f[2] = __uint_as_float(v.z);
+    f[3] = __uint_as_float(v.w);
+  }
   __device__ __forceinline__ static void load(const float* p, float (&f)[8]) {
-    float4 v = __ldg(reinterpret_cast<const float4*>(p));
-    f[0] = v.x; f[1] = v.y; f[2] = v.z; f[3] = v.w;
+    unpack(__ldg(reinterpret_cast<const uint4*>(p)), f);
   }
 };
 template <>
 struct Vec<__nv_bfloat16> {
   static constexpr int N = 8;
+  __device__ __forceinline__ static void unpack(const uint4& v, float (&f)[8]) {
+    f[0] = __uint_as_float(v.x << 16);
+    f[1] = __uint_as_float(v.x & 0xFFFF0000u);
+    f[2] = __uint_as_float(v.y << 16);
+    f[3] = __uint_as_float(v.y & 0xFFFF0000u);
+    f[4] = __uint_as_float(v.z << 16);
+    f[5] = __uint_as_float(v.z & 0xFFFF0000u);
+    f[6] = __uint_as_float(v.w << 16);
+    f[7] = __uint_as_float(v.w & 0xFFFF0000u);
+  }
   __device__ __forceinline__ static void load(const __nv_bfloat16* p, float (&f)[8]) {
-    uint4 v = __ldg(reinterpret_cast<const uint4*>(p));
-    uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      f[2 * k] = __uint_as_float(w[k] << 16);
-      f[2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
-    }
+    unpack(__ldg(reinterpret_cast<const uint4*>(p)), f);
   }
 };
 
@@ -123,7 +137,8 @@ __device__ __forceinline__ void vec_range(const T* row, int v0, int v1, int& a0,
 // Weight of logit l under row statistics st (kept set applied); greedy rows are handled by
 // the callers.
 __device__ __forceinline__ float kept_weight(const RowStat& st, float l) {
-  return fkey(l) >= st.tau ? ex2((l - st.m) * st.c) : 0.0f;
+  const float w = ex2((l - st.m) * st.c);
+  return (st.tau == 0u || fkey(l) >= st.tau) ? w : 0.0f;
 }
 
 // Probability of token v with logit l under st.

@@ -7,8 +7,8 @@
 // one candidate per position.
 //
 // One warp per request: lane i tests position i (and i + 32), a ballot gives the first
-// rejection j, and lane 0 writes the residual (or bonus) draw job that cdf_partial/cdf_pick
-// complete. Greedy requests (T == 0) need no draw: the verifier argmax is written directly.
+// rejection j, and lane 0 writes the residual (or bonus) draw job. Greedy requests (T == 0)
+// need no draw: the verifier argmax is written directly.
 #pragma once
 
 #include "common.cuh"
@@ -28,16 +28,30 @@ __device__ __forceinline__ bool accept_test(float u, const RowStat& sp, float lp
   return u < ratio;
 }
 
+// a row-statistics record written by another CTA of the running kernel (read through L2)
+__device__ __forceinline__ RowStat load_stat_cg(const RowStat* p) {
+  const int4* q = reinterpret_cast<const int4*>(p);
+  const int4 a = __ldcg(q), b = __ldcg(q + 1);
+  RowStat s;
+  s.m = __int_as_float(a.x);
+  s.c = __int_as_float(a.y);
+  s.s = __int_as_float(a.z);
+  s.s_kept = __int_as_float(a.w);
+  s.tau = static_cast<uint32_t>(b.x);
+  s.amax = b.y;
+  s.status = b.z;
+  s.pad = b.w;
+  return s;
+}
+
+// Called by one full warp for request b. ts: verifier rows [B*(K+1)], ds: draft rows [B*K].
 template <typename T>
-__global__ void linear_decide_kernel(const T* __restrict__ tgt, const T* __restrict__ drf, int B, int K, int V,
-                                     const int32_t* __restrict__ tokens, const RowStat* __restrict__ ts,
-                                     const RowStat* __restrict__ ds, const float* __restrict__ u_acc,
-                                     const float* __restrict__ u_res, int32_t* __restrict__ out_tokens,
-                                     int32_t* __restrict__ out_len, float* __restrict__ out_p,
-                                     float* __restrict__ out_q, Job* __restrict__ jobs) {
+__device__ void warp_decide_request(int b, const T* __restrict__ tgt, const T* __restrict__ drf, int K, int V,
+                                    const int32_t* __restrict__ tokens, const RowStat* ts, const RowStat* ds,
+                                    const float* __restrict__ u_acc, const float* __restrict__ u_res,
+                                    int32_t* __restrict__ out_tokens, int32_t* __restrict__ out_len,
+                                    float* __restrict__ out_p, float* __restrict__ out_q, Job* __restrict__ jobs) {
   const int lane = threadIdx.x & 31;
-  const int b = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (b >= B) return;
   const size_t trow0 = static_cast<size_t>(b) * (K + 1), drow0 = static_cast<size_t>(b) * K;
   bool bad = false;
   uint32_t rej_lo = 0u, rej_hi = 0u;
@@ -48,7 +62,7 @@ __global__ void linear_decide_kernel(const T* __restrict__ tgt, const T* __restr
     const int i = lane + 32 * h;
     if (i >= K) break;
     const int x = tokens[drow0 + i];
-    const RowStat sp = ts[trow0 + i], sq = ds[drow0 + i];
+    const RowStat sp = load_stat_cg(ts + trow0 + i), sq = load_stat_cg(ds + drow0 + i);
     const bool rowbad = sp.status != 0 || sq.status != 0 || x < 0 || x >= V;
     bool acc = false;
     if (!rowbad) {
@@ -62,12 +76,12 @@ __global__ void linear_decide_kernel(const T* __restrict__ tgt, const T* __restr
     bad |= rowbad;
     if (!acc) (h ? rej_hi : rej_lo) |= 1u << lane;
   }
-  const RowStat bonus = ts[trow0 + K];
+  const RowStat bonus = load_stat_cg(ts + trow0 + K);
   bad = __any_sync(0xffffffffu, bad) || bonus.status != 0;
   rej_lo = __reduce_or_sync(0xffffffffu, rej_lo);
   rej_hi = __reduce_or_sync(0xffffffffu, rej_hi);
   const int j = rej_lo ? __ffs(rej_lo) - 1 : (rej_hi ? 32 + __ffs(rej_hi) - 1 : K);
-  const RowStat sj = ts[trow0 + j];  // verifier row of the draw (row K for the bonus)
+  const RowStat sj = load_stat_cg(ts + trow0 + j);  // verifier row of the draw (row K for the bonus)
 
 #pragma unroll
   for (int h = 0; h < 3; ++h) {  // K + 1 <= 65 token slots

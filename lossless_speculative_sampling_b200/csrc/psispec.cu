@@ -3,6 +3,7 @@
 #include "psispec.h"
 
 #include "common.cuh"
+#include "finish.cuh"
 #include "linear.cuh"
 #include "sample.cuh"
 #include "stats.cuh"
@@ -16,7 +17,6 @@ constexpr int64_t kMaxV = int64_t(1) << 24;
 constexpr int64_t kMaxGrid = 0x7fffffff;
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
-inline int nslices_for(int64_t V) { return static_cast<int>((V + kSliceElems - 1) / kSliceElems); }
 
 // Carves a workspace into 256-byte aligned regions; with base == nullptr it only measures.
 struct Carver {
@@ -35,32 +35,33 @@ struct StatsWs {
   Partial* parts;
   RowStat* stats;
 };
-StatsWs carve_stats(Carver& c, int64_t rows, int ns) { return StatsWs{c.take<Partial>(rows * ns), c.take<RowStat>(rows)}; }
+StatsWs carve_stats(Carver& c, int64_t rows, int nch) {
+  return StatsWs{c.take<Partial>(rows * nch), c.take<RowStat>(rows)};
+}
 
 struct SampleWs {
   StatsWs st;
-  Job* jobs;
-  double2* cdf;
 };
-SampleWs carve_sample(Carver& c, int64_t rows, int ns) {
+SampleWs carve_sample(Carver& c, int64_t rows, int64_t V) {
   SampleWs w;
-  w.st = carve_stats(c, rows, ns);
-  w.jobs = c.take<Job>(rows);
-  w.cdf = c.take<double2>(rows * ns);
+  w.st = carve_stats(c, rows, nchunks_for(V));
   return w;
 }
 
 struct LinearWs {
   StatsWs t, d;
   Job* jobs;
-  double2* cdf;
+  int32_t* cnt;      // arrival counters: one per request (top-p), one per draw job
+  double2* draw_tot;  // per (draw job, chunk) weight totals
 };
-LinearWs carve_linear(Carver& c, int64_t B, int64_t K, int ns) {
+LinearWs carve_linear(Carver& c, int64_t B, int64_t K, int64_t V) {
+  const int ns = nchunks_for(V);
   LinearWs w;
   w.t = carve_stats(c, B * (K + 1), ns);
   w.d = carve_stats(c, B * K, ns);
   w.jobs = c.take<Job>(B);
-  w.cdf = c.take<double2>(B * ns);
+  w.cnt = c.take<int32_t>(2 * B);
+  w.draw_tot = c.take<double2>(B * ns);
   return w;
 }
 
@@ -68,7 +69,8 @@ struct TreeWs {
   StatsWs t, d;
   int32_t* row_req;
 };
-TreeWs carve_tree(Carver& c, int64_t N, int ns) {
+TreeWs carve_tree(Carver& c, int64_t N, int64_t V) {
+  const int ns = nchunks_for(V);
   TreeWs w;
   w.t = carve_stats(c, N, ns);
   w.d = carve_stats(c, N, ns);
@@ -92,17 +94,37 @@ __global__ void node_request_kernel(const int32_t* __restrict__ offs, int B, int
   for (int n = lo + threadIdx.x; n < hi; n += blockDim.x) row_req[n] = b;
 }
 
-// Row statistics of a [rows, V] tensor (and, for draft sampling, the draw jobs).
+// Persistent grid for a warp-granular streaming kernel: one CTA per resident slot, fewer
+// when there is less work than that.
+template <typename Kern>
+unsigned persistent_grid(Kern kernel, int64_t work_warps) {
+  int dev = 0, sms = 148, occ = 1;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, kThreads, 0);
+  const int64_t want = (work_warps + (kThreads / 32) - 1) / (kThreads / 32);
+  const int64_t slots = static_cast<int64_t>(sms) * (occ > 0 ? occ : 1);
+  return static_cast<unsigned>(want < 1 ? 1 : (want < slots ? want : slots));
+}
+
+// The streaming pass over a [rows, V] tensor: one partial per chunk.
 template <typename T>
-psispec_status launch_stats(const T* base, int64_t rows, int rows_per_req, const int32_t* row_req, int V, int ns,
-                            const float* temperature, const float* top_p, StatsWs ws, RowStat* stats_out,
-                            const float* u, Job* jobs, int32_t* out_tokens, float* out_q, cudaStream_t st) {
-  row_partial_kernel<T><<<static_cast<unsigned>(rows * ns), kThreads, 0, st>>>(base, rows_per_req, row_req, V, ns,
-                                                                              temperature, ws.parts);
-  psispec_status s = launched();
+psispec_status launch_stream(const T* base, int64_t rows, int rows_per_req, const int32_t* row_req, int V,
+                             const float* temperature, Partial* parts, cudaStream_t st) {
+  const int64_t chunks = rows * nchunks_for(V);
+  stream_partials_kernel<T><<<persistent_grid(stream_partials_kernel<T>, chunks), kThreads, 0, st>>>(
+      base, rows_per_req, row_req, V, chunks, temperature, parts);
+  return launched();
+}
+
+// Row statistics of a [rows, V] tensor (the tree's statistics pass).
+template <typename T>
+psispec_status launch_stats(const T* base, int64_t rows, int rows_per_req, const int32_t* row_req, int V,
+                            const float* temperature, const float* top_p, StatsWs ws, cudaStream_t st) {
+  psispec_status s = launch_stream<T>(base, rows, rows_per_req, row_req, V, temperature, ws.parts, st);
   if (s != PSISPEC_OK) return s;
-  row_finalize_kernel<T><<<static_cast<unsigned>(rows), kThreads, 0, st>>>(
-      base, rows_per_req, row_req, V, ns, temperature, top_p, ws.parts, stats_out, u, jobs, out_tokens, out_q);
+  row_finalize_kernel<T><<<static_cast<unsigned>(rows), kThreads, 0, st>>>(base, rows_per_req, row_req, V,
+                                                                            temperature, top_p, ws.parts, ws.stats);
   return launched();
 }
 
@@ -111,18 +133,16 @@ psispec_status sample_draft_impl(const T* draft, int B, int K, int V, const floa
                                  const float* u, int32_t* out_tokens, float* out_q, RowStat* out_stats, void* ws,
                                  cudaStream_t st) {
   const int64_t rows = int64_t(B) * K;
-  const int ns = nslices_for(V);
   Carver c(ws);
-  SampleWs w = carve_sample(c, rows, ns);
+  SampleWs w = carve_sample(c, rows, V);
   RowStat* stats = out_stats ? out_stats : w.st.stats;
-  psispec_status s = launch_stats<T>(draft, rows, K, nullptr, V, ns, temperature, top_p, w.st, stats, u, w.jobs,
-                                     out_tokens, out_q, st);
+  psispec_status s = launch_stream<T>(draft, rows, K, nullptr, V, temperature, w.st.parts, st);
   if (s != PSISPEC_OK) return s;
-  cdf_partial_kernel<T><<<static_cast<unsigned>(rows * ns), kThreads, 0, st>>>(draft, draft, stats, stats, w.jobs, V,
-                                                                              ns, w.cdf);
+  sample_finish_kernel<T><<<static_cast<unsigned>((rows + 7) / 8), kThreads, 0, st>>>(
+      draft, K, V, static_cast<int>(rows), temperature, top_p, u, w.st.parts, stats, out_tokens, out_q);
   if ((s = launched()) != PSISPEC_OK) return s;
-  cdf_pick_kernel<T><<<static_cast<unsigned>(rows), kThreads, 0, st>>>(draft, draft, stats, stats, w.jobs, V, ns,
-                                                                       w.st.parts, w.cdf, out_tokens, out_q);
+  sample_topp_kernel<T><<<static_cast<unsigned>(rows), kThreads, 0, st>>>(draft, K, V, top_p, u, stats, out_tokens,
+                                                                          out_q);
   return launched();
 }
 
@@ -131,28 +151,43 @@ psispec_status verify_linear_impl(const T* tgt, const T* drf, int B, int K, int 
                                   const RowStat* draft_stats, const float* u_acc, const float* u_res,
                                   const float* temperature, const float* top_p, int32_t* out_tokens,
                                   int32_t* out_len, float* out_p, float* out_q, void* ws, cudaStream_t st) {
-  const int ns = nslices_for(V);
   Carver c(ws);
-  LinearWs w = carve_linear(c, B, K, ns);
-  psispec_status s = launch_stats<T>(tgt, int64_t(B) * (K + 1), K + 1, nullptr, V, ns, temperature, top_p, w.t,
-                                     w.t.stats, nullptr, nullptr, nullptr, nullptr, st);
+  LinearWs w = carve_linear(c, B, K, V);
+  const int64_t rows_t = int64_t(B) * (K + 1), rows_d = draft_stats ? 0 : int64_t(B) * K;
+  if (cudaMemsetAsync(w.cnt, 0, sizeof(int32_t) * 2 * B, st) != cudaSuccess) return PSISPEC_ERR_CUDA;
+  VerifyArgs a;
+  a.B = B;
+  a.K = K;
+  a.V = V;
+  a.stream_draft = draft_stats ? 0 : 1;
+  a.temperature = temperature;
+  a.top_p = top_p;
+  a.tokens = tokens;
+  a.dstats_in = draft_stats;
+  a.u_acc = u_acc;
+  a.u_res = u_res;
+  a.parts_t = w.t.parts;
+  a.parts_d = w.d.parts;
+  a.stats_t = w.t.stats;
+  a.stats_d = w.d.stats;
+  a.cnt = w.cnt;
+  a.out_tokens = out_tokens;
+  a.out_len = out_len;
+  a.out_p = out_p;
+  a.out_q = out_q;
+  a.jobs = w.jobs;
+  psispec_status s = launch_stream<T>(tgt, rows_t, K + 1, nullptr, V, temperature, w.t.parts, st);
   if (s != PSISPEC_OK) return s;
-  const RowStat* ds = draft_stats;
-  if (ds == nullptr) {
-    s = launch_stats<T>(drf, int64_t(B) * K, K, nullptr, V, ns, temperature, top_p, w.d, w.d.stats, nullptr, nullptr,
-                        nullptr, nullptr, st);
-    if (s != PSISPEC_OK) return s;
-    ds = w.d.stats;
-  }
-  constexpr int kWarps = 8;
-  linear_decide_kernel<T><<<(B + kWarps - 1) / kWarps, 32 * kWarps, 0, st>>>(
-      tgt, drf, B, K, V, tokens, w.t.stats, ds, u_acc, u_res, out_tokens, out_len, out_p, out_q, w.jobs);
+  if (rows_d > 0 && (s = launch_stream<T>(drf, rows_d, K, nullptr, V, temperature, w.d.parts, st)) != PSISPEC_OK)
+    return s;
+  verify_finish_kernel<T><<<static_cast<unsigned>(B), kThreads, 0, st>>>(tgt, drf, a);
   if ((s = launched()) != PSISPEC_OK) return s;
-  cdf_partial_kernel<T><<<static_cast<unsigned>(int64_t(B) * ns), kThreads, 0, st>>>(tgt, drf, w.t.stats, ds, w.jobs,
-                                                                                     V, ns, w.cdf);
+  verify_topp_kernel<T><<<static_cast<unsigned>(rows_t + rows_d), kThreads, 0, st>>>(tgt, drf, a);
   if ((s = launched()) != PSISPEC_OK) return s;
-  cdf_pick_kernel<T><<<B, kThreads, 0, st>>>(tgt, drf, w.t.stats, ds, w.jobs, V, ns, w.t.parts, w.cdf, out_tokens,
-                                              nullptr);
+  const RowStat* ds = draft_stats ? draft_stats : w.d.stats;
+  const int64_t draw_warps = int64_t(B) * nchunks_for(V);
+  draw_jobs_kernel<T><<<static_cast<unsigned>((draw_warps + 7) / 8), kThreads, 0, st>>>(
+      tgt, drf, V, B, w.t.stats, ds, w.t.parts, w.jobs, w.draw_tot, w.cnt + B, out_tokens);
   return launched();
 }
 
@@ -163,15 +198,13 @@ psispec_status verify_tree_impl(const T* tgt, const T* drf, int B, int N, int V,
                                 int32_t* out_tokens, int32_t* out_len, void* ws, cudaStream_t st) {
   const int ns = nslices_for(V);
   Carver c(ws);
-  TreeWs w = carve_tree(c, N, ns);
+  TreeWs w = carve_tree(c, N, V);
   node_request_kernel<<<B, 128, 0, st>>>(offs, B, N, w.row_req);
   psispec_status s = launched();
   if (s != PSISPEC_OK) return s;
-  s = launch_stats<T>(tgt, N, 1, w.row_req, V, ns, temperature, top_p, w.t, w.t.stats, nullptr, nullptr, nullptr,
-                      nullptr, st);
+  s = launch_stats<T>(tgt, N, 1, w.row_req, V, temperature, top_p, w.t, st);
   if (s != PSISPEC_OK) return s;
-  s = launch_stats<T>(drf, N, 1, w.row_req, V, ns, temperature, top_p, w.d, w.d.stats, nullptr, nullptr, nullptr,
-                      nullptr, st);
+  s = launch_stats<T>(drf, N, 1, w.row_req, V, temperature, top_p, w.d, st);
   if (s != PSISPEC_OK) return s;
   tree_walk_kernel<T><<<B, kTreeThreads, 0, st>>>(tgt, drf, V, offs, parent, tokens, w.t.stats, w.d.stats, u_acc,
                                                   u_res, max_depth, out_path, out_tokens, out_len);
@@ -203,12 +236,11 @@ int psispec_version(void) { return 100; }
 
 size_t psispec_workspace_size(int op, int64_t a, int64_t b, int64_t c) {
   if (a <= 0 || b <= 0 || c <= 0 || c > kMaxV) return 0;
-  const int ns = nslices_for(c);
   Carver m(nullptr);
   switch (op) {
-    case PSISPEC_OP_SAMPLE_DRAFT: carve_sample(m, a * b, ns); break;
-    case PSISPEC_OP_VERIFY_LINEAR: carve_linear(m, a, b, ns); break;
-    case PSISPEC_OP_VERIFY_TREE: carve_tree(m, b, ns); break;
+    case PSISPEC_OP_SAMPLE_DRAFT: carve_sample(m, a * b, c); break;
+    case PSISPEC_OP_VERIFY_LINEAR: carve_linear(m, a, b, c); break;
+    case PSISPEC_OP_VERIFY_TREE: carve_tree(m, b, c); break;
     default: return 0;
   }
   return m.used;

@@ -1,4 +1,4 @@
-// sample.cuh -- inverse-CDF draws in vocabulary order.
+// sample.cuh -- inverse-CDF draws in vocabulary order (warp- and block-level building blocks).
 //
 // A draw with uniform u over non-negative weights r returns the first index v with
 // C(v) > u * Z, C the inclusive prefix sum and Z the total (so a zero-weight token is never
@@ -6,31 +6,25 @@
 // section 3.3): a row's own distribution (drafting, and the bonus token after a fully
 // accepted block) and the residual max(0, p - q) of a rejected position.
 //
-// The draw is hierarchical. Slice totals (kSliceElems elements each) locate the slice that
-// holds u * Z; they come from the row-statistics partials when the row's own distribution
-// has no top-p cut, and from cdf_partial_kernel otherwise (a residual, or a kept set). Then
-// one CTA scans that slice: each warp totals a contiguous kWarpSpan sub-range with coalesced
-// 16-byte loads, a block scan picks the owning warp, which walks its sub-range 256 elements
-// at a time with warp scans; the owning lane walks its 8 elements. All prefix sums are fp64.
+// Ranges are walked by warps in groups of 256 elements (8 consecutive elements per lane,
+// coalesced), with kBatch groups loaded before any is used. warp_draw_range scans a range
+// with warp-wide fp64 prefix sums and lets the lane that crosses u * Z walk its 8 elements;
+// block_draw_range first totals one contiguous sub-range per warp and hands the crossing to
+// the owning warp. Per-element weights are fp32, every prefix sum is fp64.
 #pragma once
 
 #include "common.cuh"
 
 namespace psi {
 
-constexpr int kWarpSpan = kSliceElems / (kThreads / 32);  // elements per warp in a slice scan
+constexpr int kGroup = 256;     // elements per warp step (8 per lane)
+template <bool RESID>
+constexpr int kDrawBatch = 4;  // groups in flight per lane
 
 struct ResidCtx {
   RowStat a, b;
   float ia, ib;  // 1 / s_kept of rows a and b
 };
-
-// residual weight max(0, p_a(v) - q_b(v)) and p_a(v)
-__device__ __forceinline__ void resid_weight(const ResidCtx& r, float xa, float xb, float& res, float& pa) {
-  pa = kept_weight(r.a, xa) * r.ia;
-  float qb = kept_weight(r.b, xb) * r.ib;
-  res = fmaxf(pa - qb, 0.0f);
-}
 
 // 8 consecutive elements starting at e (elements at or past `end` read as -inf)
 template <typename T>
@@ -51,217 +45,151 @@ __device__ __forceinline__ void load8(const T* __restrict__ row, int e, int end,
   }
 }
 
+// The raw bits of 8 consecutive elements (one 16-byte word for bf16, two for fp32), kept
+// packed while loads are in flight. Elements at or past `end` read as -inf.
 template <typename T>
+struct Raw8x {
+  uint4 w[sizeof(T) == 2 ? 1 : 2];
+  __device__ __forceinline__ void load(const T* __restrict__ row, int e, int end, bool aligned) {
+    if (aligned && e + 8 <= end) {
+      w[0] = __ldg(reinterpret_cast<const uint4*>(row + e));
+      if constexpr (sizeof(T) == 4) w[1] = __ldg(reinterpret_cast<const uint4*>(row + e + 4));
+    } else {
+      float x[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) x[k] = e + k < end ? load_elem(row + e + k) : -INFINITY;
+      pack(x);
+    }
+  }
+  __device__ __forceinline__ void pack(const float (&x)[8]) {
+    if constexpr (sizeof(T) == 2) {  // every value here is an exact bf16 (or -inf)
+      w[0] = make_uint4((__float_as_uint(x[0]) >> 16) | (__float_as_uint(x[1]) & 0xFFFF0000u),
+                        (__float_as_uint(x[2]) >> 16) | (__float_as_uint(x[3]) & 0xFFFF0000u),
+                        (__float_as_uint(x[4]) >> 16) | (__float_as_uint(x[5]) & 0xFFFF0000u),
+                        (__float_as_uint(x[6]) >> 16) | (__float_as_uint(x[7]) & 0xFFFF0000u));
+    } else {
+      w[0] = make_uint4(__float_as_uint(x[0]), __float_as_uint(x[1]), __float_as_uint(x[2]), __float_as_uint(x[3]));
+      w[1] = make_uint4(__float_as_uint(x[4]), __float_as_uint(x[5]), __float_as_uint(x[6]), __float_as_uint(x[7]));
+    }
+  }
+  __device__ __forceinline__ void unpack(float (&x)[8]) const {
+    if constexpr (sizeof(T) == 2) {
+      Vec<T>::unpack(w[0], x);
+    } else {
+      float lo[8], hi[8];
+      Vec<T>::unpack(w[0], lo);
+      Vec<T>::unpack(w[1], hi);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) { x[k] = lo[k]; x[k + 4] = hi[k]; }
+    }
+  }
+};
+
+// Raw logits of one 8-element group (row a, and row b for a residual).
+template <typename T, bool RESID>
+struct Raw8 {
+  Raw8x<T> a;
+  Raw8x<T> b[RESID ? 1 : 0 + 1];
+};
+
+// The weights a draw runs over: row a's kept distribution (RESID = false), or the residual
+// max(0, p_a - q_b) (RESID = true), or, with use_p, p_a normalised (the fallback when the
+// residual is zero everywhere).
+template <typename T, bool RESID>
 struct JobRows {
-  int mode;
+  static constexpr bool kResid = RESID;
   bool use_p;
   ResidCtx r;
   const T* ra;
   const T* rb;
   bool al_a, al_b;
-  int end;
 
-  // weights of elements e .. e+7; returns their fp32 sum
-  __device__ __forceinline__ float weights8(int e, float (&w)[8]) const {
+  __device__ __forceinline__ void init(const T* rowa, const RowStat& sa, const T* rowb, const RowStat& sb) {
+    use_p = false;
+    r.a = sa;
+    r.ia = 1.0f / sa.s_kept;
+    ra = rowa;
+    al_a = (reinterpret_cast<uintptr_t>(rowa) & 15u) == 0;
+    rb = rowb;
+    r.b = sb;
+    r.ib = RESID ? 1.0f / sb.s_kept : 0.0f;
+    al_b = RESID && (reinterpret_cast<uintptr_t>(rowb) & 15u) == 0;
+  }
+  __device__ __forceinline__ void load(int e, int end, Raw8<T, RESID>& x) const {
+    x.a.load(ra, e, end, al_a);
+    if constexpr (RESID) x.b[0].load(rb, e, end, al_b);
+  }
+  // weights (and p_a, for residual totals) of a loaded group
+  __device__ __forceinline__ void weights(const Raw8<T, RESID>& x, float (&w)[8], float (&pw)[8]) const {
     float xa[8];
-    load8(ra, e, end, al_a, xa);
-    float sum = 0.0f;
-    if (mode == kSample) {
-#pragma unroll
-      for (int k = 0; k < 8; ++k) { w[k] = kept_weight(r.a, xa[k]); sum += w[k]; }
-    } else {
+    x.a.unpack(xa);
+    if constexpr (RESID) {
       float xb[8];
-      load8(rb, e, end, al_b, xb);
+      x.b[0].unpack(xb);
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
-        float res, pa;
-        resid_weight(r, xa[k], xb[k], res, pa);
-        w[k] = use_p ? pa : res;
-        sum += w[k];
+        const float pa = kept_weight(r.a, xa[k]) * r.ia;
+        const float qb = kept_weight(r.b, xb[k]) * r.ib;
+        w[k] = use_p ? pa : fmaxf(pa - qb, 0.0f);
+        pw[k] = pa;
+      }
+    } else {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        w[k] = kept_weight(r.a, xa[k]);
+        pw[k] = w[k];
       }
     }
-    return sum;
   }
 };
 
-template <typename T>
-__global__ void __launch_bounds__(kThreads) cdf_partial_kernel(const T* __restrict__ A, const T* __restrict__ Bt,
-                                                               const RowStat* __restrict__ sa,
-                                                               const RowStat* __restrict__ sb,
-                                                               const Job* __restrict__ jobs, int V, int nslices,
-                                                               double2* __restrict__ out) {
-  __shared__ double red[33];
-  const int unit = blockIdx.x;
-  const int job = unit / nslices, slice = unit - job * nslices;
-  const Job jb = jobs[job];
-  if (jb.mode < kSample) return;
-  ResidCtx r;
-  r.a = sa[jb.row_a];
-  if (jb.mode == kSample && r.a.tau == 0u) return;  // slice totals come from the row statistics
-  const int v0 = slice * kSliceElems, v1 = min(V, v0 + kSliceElems);
-  r.ia = 1.0f / r.a.s_kept;
-  const T* ra = A + static_cast<size_t>(jb.row_a) * V;
+// Warp-level totals over [lo, hi) of the job weights (.x) and of p_a (.y), and the last
+// index with positive weight; every lane gets them.
+template <typename T, bool RESID>
+__device__ double2 warp_range_totals(const JobRows<T, RESID>& J, int lo, int hi, int* last_pos) {
+  const int lane = threadIdx.x & 31;
   double sr = 0.0, sp = 0.0;
-  constexpr int N = Vec<T>::N;
-  if (jb.mode == kSample) {
-    int a0, a1;
-    vec_range(ra, v0, v1, a0, a1);
-    for (int v = v0 + threadIdx.x; v < a0; v += blockDim.x) sr += kept_weight(r.a, load_elem(ra + v));
-    for (int v = a1 + threadIdx.x; v < v1; v += blockDim.x) sr += kept_weight(r.a, load_elem(ra + v));
-    for (int v = a0 + threadIdx.x * N; v < a1; v += blockDim.x * N) {
-      float x[8], acc = 0.0f;
-      Vec<T>::load(ra + v, x);
+  int last = -1;
+  for (int g = lo; g < hi; g += kDrawBatch<RESID> * kGroup) {
+    Raw8<T, RESID> x[kDrawBatch<RESID>];
 #pragma unroll
-      for (int k = 0; k < N; ++k) acc += kept_weight(r.a, x[k]);
-      sr += static_cast<double>(acc);
-    }
-  } else {
-    r.b = sb[jb.row_b];
-    r.ib = 1.0f / r.b.s_kept;
-    const T* rb = Bt + static_cast<size_t>(jb.row_b) * V;
-    int a0, a1, b0, b1;
-    vec_range(ra, v0, v1, a0, a1);
-    vec_range(rb, v0, v1, b0, b1);
-    if (a0 != b0) { a0 = v1; a1 = v1; }  // rows aligned differently: scalar path
-    auto one = [&](float xa, float xb, float& ar, float& ap) {
-      float res, pa;
-      resid_weight(r, xa, xb, res, pa);
-      ar += res;
-      ap += pa;
-    };
-    float ar = 0.0f, ap = 0.0f;
-    for (int v = v0 + threadIdx.x; v < a0; v += blockDim.x) one(load_elem(ra + v), load_elem(rb + v), ar, ap);
-    for (int v = a1 + threadIdx.x; v < v1; v += blockDim.x) one(load_elem(ra + v), load_elem(rb + v), ar, ap);
-    sr += ar;
-    sp += ap;
-    for (int v = a0 + threadIdx.x * N; v < a1; v += blockDim.x * N) {
-      float xa[8], xb[8];
-      Vec<T>::load(ra + v, xa);
-      Vec<T>::load(rb + v, xb);
-      ar = 0.0f;
-      ap = 0.0f;
+    for (int b = 0; b < kDrawBatch<RESID>; ++b) J.load(g + b * kGroup + lane * 8, hi, x[b]);
 #pragma unroll
-      for (int k = 0; k < N; ++k) one(xa[k], xb[k], ar, ap);
+    for (int b = 0; b < kDrawBatch<RESID>; ++b) {
+      float w[8], pw[8];
+      J.weights(x[b], w, pw);
+      float ar = 0.0f, ap = 0.0f;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        ar += w[k];
+        ap += pw[k];
+        if (w[k] > 0.0f) last = g + b * kGroup + lane * 8 + k;
+      }
       sr += static_cast<double>(ar);
       sp += static_cast<double>(ap);
     }
   }
-  double tr = block_sum(sr, red);
-  double tp = block_sum(sp, red);
-  if (threadIdx.x == 0) out[unit] = make_double2(tr, tp);
+  *last_pos = __reduce_max_sync(0xffffffffu, last);
+  return make_double2(warp_sum(sr), warp_sum(sp));
 }
 
-// parts_a: row-statistics partials of tensor A (used for sample jobs without a top-p cut)
-template <typename T>
-__global__ void __launch_bounds__(kThreads) cdf_pick_kernel(const T* __restrict__ A, const T* __restrict__ Bt,
-                                                            const RowStat* __restrict__ sa,
-                                                            const RowStat* __restrict__ sb, const Job* __restrict__ jobs,
-                                                            int V, int nslices, const Partial* __restrict__ parts_a,
-                                                            const double2* __restrict__ parts, int32_t* __restrict__ out_tokens,
-                                                            float* __restrict__ out_q) {
-  __shared__ double wtot[kThreads / 32];
-  __shared__ int sh_slice, sh_use_p, sh_y, sh_last, sh_owner;
-  __shared__ double sh_base, sh_target, sh_c0;
-  const Job jb = jobs[blockIdx.x];
-  if (jb.mode < kSample) return;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const RowStat sta = sa[jb.row_a];
-  const bool from_stats = jb.mode == kSample && sta.tau == 0u;
-  if (threadIdx.x == 0) {
-    const double2* pp = parts + static_cast<size_t>(blockIdx.x) * nslices;
-    const Partial* ps = parts_a + static_cast<size_t>(jb.row_a) * nslices;
-    auto total = [&](int s, int use_p) -> double {
-      if (from_stats) return ps[s].m > -INFINITY ? ps[s].s * static_cast<double>(ex2((ps[s].m - sta.m) * sta.c)) : 0.0;
-      return use_p ? pp[s].y : pp[s].x;
-    };
-    double Z = 0.0;
-    for (int s = 0; s < nslices; ++s) Z += total(s, 0);
-    int use_p = 0;
-    if (jb.mode == kResidual && !(Z > 0.0)) {  // zero residual: draw from p instead
-      use_p = 1;
-      Z = 0.0;
-      for (int s = 0; s < nslices; ++s) Z += total(s, 1);
-    }
-    const double target = static_cast<double>(jb.u) * Z;
-    double C = 0.0, base = 0.0;
-    int sel = -1;
-    for (int s = 0; s < nslices; ++s) {
-      const double w = total(s, use_p);
-      if (w > 0.0) { sel = s; base = C; }
-      if (C + w > target && w > 0.0) break;
-      C += w;
-    }
-    sh_slice = sel;
-    sh_use_p = use_p;
-    sh_base = base;
-    sh_target = target;
-    sh_y = 0x7fffffff;
-    sh_last = -1;
-    sh_owner = -1;
-  }
-  __syncthreads();
-  const int sel = sh_slice;
-  if (sel < 0) {  // no mass anywhere (cannot happen for a valid row): report a data error
-    if (threadIdx.x == 0) {
-      out_tokens[jb.out_index] = -1;
-      if (out_q && jb.aux >= 0) out_q[jb.aux] = -1.0f;
-    }
-    return;
-  }
-  JobRows<T> J;
-  J.mode = jb.mode;
-  J.use_p = sh_use_p != 0;
-  J.r.a = sta;
-  J.r.ia = 1.0f / sta.s_kept;
-  J.ra = A + static_cast<size_t>(jb.row_a) * V;
-  J.rb = nullptr;
-  J.al_a = (reinterpret_cast<uintptr_t>(J.ra) & 15u) == 0;
-  J.al_b = false;
-  if (jb.mode == kResidual) {
-    J.r.b = sb[jb.row_b];
-    J.r.ib = 1.0f / J.r.b.s_kept;
-    J.rb = Bt + static_cast<size_t>(jb.row_b) * V;
-    J.al_b = (reinterpret_cast<uintptr_t>(J.rb) & 15u) == 0;
-  }
-  const int v0 = sel * kSliceElems, v1 = min(V, v0 + kSliceElems);
-  const int w0 = v0 + warp * kWarpSpan, w1 = min(v1, w0 + kWarpSpan);
-  J.end = w1;
-  const double target = sh_target;
-
-  // phase 1: per-warp totals of contiguous sub-ranges
-  double mine = 0.0;
-  int last = -1;
-  for (int e = w0 + lane * 8; e < w1; e += 256) {
-    float w[8];
-    mine += static_cast<double>(J.weights8(e, w));
+// Warp-level draw inside [lo, hi): `base` is the weight before lo, `target` = u * Z.
+// Returns the first index whose inclusive prefix exceeds target, or the last index with
+// positive weight when rounding leaves none (-1 if the range has no positive weight).
+template <typename T, bool RESID, int NB = kDrawBatch<RESID>>
+__device__ int warp_draw_range(const JobRows<T, RESID>& J, int lo, int hi, double base, double target) {
+  const int lane = threadIdx.x & 31;
+  double Cb = base;
+  int wlast = -1;
+  for (int g = lo; g < hi; g += NB * kGroup) {
+    Raw8<T, RESID> x[NB];
 #pragma unroll
-    for (int k = 0; k < 8; ++k)
-      if (w[k] > 0.0f) last = e + k;
-  }
-  mine = warp_sum(mine);
-  last = __reduce_max_sync(0xffffffffu, last);
-  if (lane == 0) {
-    wtot[warp] = mine;
-    if (last >= 0) atomicMax(&sh_last, last);
-  }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    double C = sh_base;
-    for (int i = 0; i < kThreads / 32; ++i) {
-      if (C <= target && target < C + wtot[i]) { sh_owner = i; sh_c0 = C; break; }
-      C += wtot[i];
-    }
-  }
-  __syncthreads();
-
-  // phase 2: the owning warp walks its sub-range, 256 elements per step (vector sums in fp64
-  // so that the lane walk below retraces the scanned totals)
-  if (warp == sh_owner) {
-    double Cb = sh_c0;
-    int wlast = -1;
-    for (int e = w0 + lane * 8; e - lane * 8 < w1; e += 256) {
-      float w[8];
-      J.weights8(e, w);
+    for (int b = 0; b < NB; ++b) J.load(g + b * kGroup + lane * 8, hi, x[b]);
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+      const int e = g + b * kGroup + lane * 8;
+      float w[8], pw[8];
+      J.weights(x[b], w, pw);
       double vs = 0.0;
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
@@ -278,31 +206,92 @@ __global__ void __launch_bounds__(kThreads) cdf_pick_kernel(const T* __restrict_
       if (lane == 0) excl = 0.0;
       const unsigned hit = __ballot_sync(0xffffffffu, Cb + incl > target);
       if (hit) {
-        if (lane == __ffs(hit) - 1) {
+        const int src = __ffs(hit) - 1;
+        int y = -1, lastpos = -1;
+        if (lane == src) {
           double C = Cb + excl;
-          int y = -1, lastpos = -1;
 #pragma unroll
           for (int k = 0; k < 8; ++k) {
             C += static_cast<double>(w[k]);
             if (w[k] > 0.0f) lastpos = e + k;
             if (y < 0 && C > target) y = e + k;
           }
-          sh_y = y >= 0 ? y : lastpos;  // rounding at the group's end: its last positive entry
+          if (y < 0) y = lastpos;  // rounding at the group's end: its last positive entry
         }
-        break;
+        return __shfl_sync(0xffffffffu, y, src);
       }
       Cb += __shfl_sync(0xffffffffu, incl, 31);
     }
-    // no crossing found (rounding against the phase-1 total): the warp's last positive entry
-    wlast = __reduce_max_sync(0xffffffffu, wlast);
-    if (lane == 0 && sh_y == 0x7fffffff && wlast >= 0) sh_y = wlast;
+  }
+  return __reduce_max_sync(0xffffffffu, wlast);
+}
+
+// Block-level totals over [lo, hi) (.x job weights, .y p_a); every thread gets them.
+template <typename T, bool RESID>
+__device__ double2 block_range_totals(const JobRows<T, RESID>& J, int lo, int hi, double* red) {
+  const int warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  const int span = (((hi - lo + nw - 1) / nw) + 7) & ~7;
+  const int w0 = min(hi, lo + warp * span), w1 = min(hi, w0 + span);
+  int last;
+  const double2 t = warp_range_totals(J, w0, w1, &last);
+  __syncthreads();
+  if ((threadIdx.x & 31) == 0) { red[warp] = t.x; red[32 + warp] = t.y; }
+  __syncthreads();
+  double x = 0.0, y = 0.0;
+  for (int i = 0; i < nw; ++i) { x += red[i]; y += red[32 + i]; }
+  __syncthreads();
+  return make_double2(x, y);
+}
+
+struct DrawSmem {
+  double wtot[32];
+  double c0, target;
+  int owner, y, last;
+};
+
+// Block-level draw inside [lo, hi) (lo a multiple of 8). With target >= 0 the draw is
+// absolute: `base` is the weight before lo and `target` = u * Z of the whole distribution.
+// With target < 0 the range is the whole distribution: target = u * (range total). Returns
+// the drawn index to every thread (-1 if the range has no positive weight).
+template <typename T, bool RESID>
+__device__ int block_draw_range(const JobRows<T, RESID>& J, int lo, int hi, double base, double target, float u,
+                                DrawSmem& sm) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  const int span = (((hi - lo + nw - 1) / nw) + 7) & ~7;
+  const int w0 = min(hi, lo + warp * span), w1 = min(hi, w0 + span);
+  int last;
+  const double2 t = warp_range_totals(J, w0, w1, &last);
+  __syncthreads();
+  if (threadIdx.x == 0) { sm.y = -1; sm.last = -1; sm.owner = -1; }
+  __syncthreads();
+  if (lane == 0) {
+    sm.wtot[warp] = t.x;
+    if (last >= 0) atomicMax(&sm.last, last);
   }
   __syncthreads();
   if (threadIdx.x == 0) {
-    const int y = sh_y != 0x7fffffff ? sh_y : sh_last;  // rounding at a sub-range edge: last positive entry
-    out_tokens[jb.out_index] = y;
-    if (out_q && jb.aux >= 0) out_q[jb.aux] = kept_weight(sta, load_elem(J.ra + y)) / sta.s_kept;
+    double C = base, tg = target;
+    if (tg < 0.0) {
+      double Z = 0.0;
+      for (int i = 0; i < nw; ++i) Z += sm.wtot[i];
+      tg = static_cast<double>(u) * Z;
+      C = 0.0;
+    }
+    sm.target = tg;
+    for (int i = 0; i < nw; ++i) {
+      if (C <= tg && tg < C + sm.wtot[i]) { sm.owner = i; sm.c0 = C; break; }
+      C += sm.wtot[i];
+    }
   }
+  __syncthreads();
+  if (warp == sm.owner) {
+    const int y = warp_draw_range(J, w0, w1, sm.c0, sm.target);
+    if (lane == 0) sm.y = y;
+  }
+  __syncthreads();
+  const int y = sm.y >= 0 ? sm.y : sm.last;  // past every sub-range (rounding): last positive entry
+  __syncthreads();
+  return y;
 }
 
 }  // namespace psi

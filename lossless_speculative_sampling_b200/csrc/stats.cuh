@@ -6,90 +6,20 @@
 // log2(e)/T, the normaliser s = sum 2^((l - m) c), the top-p threshold key tau and the kept
 // normaliser s_kept. Any probability of the row is then one ex2 away.
 //
-// Two kernels:
-//   row_partial_kernel  one CTA per (row, slice of kSliceElems): streaming online max/sum
-//                       with 16-byte vector loads (greedy rows: max and lowest argmax);
-//   row_finalize_kernel one CTA per row: combines the slice partials and, when top-p is on,
-//                       finds tau by a most-significant-digit radix select over the keys,
-//                       accumulating probability mass per digit.
+// Streaming: a warp covers one contiguous chunk of kChunkElems elements of a row with
+// coalesced 16-byte loads (lanes take consecutive vectors, kBatch loads in flight per lane)
+// and leaves that chunk's partial (maximum and normaliser relative to it, or the lowest
+// argmax for greedy rows). Chunk partials are also the prefix totals that a draw uses to find
+// the chunk holding u * Z. warp_finalize_row combines a row's chunk partials;
+// block_topp_select finds the top-p threshold by a most-significant-digit radix select over
+// the keys with the fp64 mass of every digit.
 #pragma once
 
 #include "common.cuh"
 
 namespace psi {
 
-// Online max/sum over [v0, v1) of one row, per thread. The vector body batches kBatch
-// 16-byte loads before using them (memory-level parallelism) and sums weights per vector in
-// fp32, accumulating vector sums with a compensated (Kahan) fp32 sum: ~1 ulp overall without
-// fp64 work in the loop.
-constexpr int kBatch = 4;
-
-template <typename T, bool GREEDY>
-__device__ __forceinline__ void thread_slice_stats(const T* __restrict__ row, int v0, int v1, float c, float& m,
-                                                   double& s_out, int& amax, bool& bad) {
-  constexpr int N = Vec<T>::N;
-  int a0, a1;
-  vec_range(row, v0, v1, a0, a1);
-  float s = 0.0f, comp = 0.0f;
-  auto add = [&](float y) {  // compensated s += y
-    y -= comp;
-    const float t = s + y;
-    comp = (t - s) - y;
-    s = t;
-  };
-  auto rescale = [&](float nm) {
-    const float f = ex2((m - nm) * c);
-    s *= f;
-    comp *= f;
-    m = nm;
-  };
-  auto scalar = [&](int v) {
-    float x = load_elem(row + v);
-    bad |= !(x < INFINITY);
-    if (GREEDY) {
-      if (x > m) { m = x; amax = v; }
-    } else {
-      if (x > m) rescale(x);
-      if (m > -INFINITY) add(ex2((x - m) * c));
-    }
-  };
-  // head and tail elements (fewer than N each), then the aligned body
-  for (int v = v0 + threadIdx.x; v < a0; v += blockDim.x) scalar(v);
-  for (int v = a1 + threadIdx.x; v < v1; v += blockDim.x) scalar(v);
-  const int stride = blockDim.x * N;
-  for (int vb = a0 + threadIdx.x * N; vb < a1; vb += kBatch * stride) {
-    float f[kBatch][8];
-#pragma unroll
-    for (int u = 0; u < kBatch; ++u)
-      if (vb + u * stride < a1) Vec<T>::load(row + vb + u * stride, f[u]);
-#pragma unroll
-    for (int u = 0; u < kBatch; ++u) {
-      const int v = vb + u * stride;
-      if (v >= a1) break;
-      float vmax = f[u][0];
-#pragma unroll
-      for (int k = 1; k < N; ++k) vmax = fmax_nan(vmax, f[u][k]);
-      bad |= !(vmax < INFINITY);
-      if (GREEDY) {
-        if (vmax > m) {
-#pragma unroll
-          for (int k = N - 1; k >= 0; --k)
-            if (f[u][k] == vmax) amax = v + k;
-          m = vmax;
-        }
-      } else {
-        if (vmax > m) rescale(vmax);
-        if (m > -INFINITY) {
-          float acc = 0.0f;
-#pragma unroll
-          for (int k = 0; k < N; ++k) acc += ex2((f[u][k] - m) * c);
-          add(acc);
-        }
-      }
-    }
-  }
-  s_out = static_cast<double>(s) - static_cast<double>(comp);
-}
+constexpr int kBatch = 4;  // 16-byte loads in flight per lane
 
 __device__ __forceinline__ float temp_scale(float T) {
   return T > 0.0f && T < INFINITY ? static_cast<float>(1.4426950408889634 / static_cast<double>(T)) : 0.0f;
@@ -100,46 +30,139 @@ __device__ __forceinline__ int row_request(int row, int rows_per_req, const int3
   return row_req ? row_req[row] : row / rows_per_req;
 }
 
-template <typename T>
-__global__ void __launch_bounds__(kThreads) row_partial_kernel(const T* __restrict__ base, int rows_per_req,
-                                                                const int32_t* __restrict__ row_req, int V,
-                                                                int nslices, const float* __restrict__ temperature,
-                                                                Partial* __restrict__ out) {
-  __shared__ float red[32];
-  __shared__ double dred[33];
-  __shared__ int ired[32];
-  const int unit = blockIdx.x;
-  const int row = unit / nslices, slice = unit - row * nslices;
-  const float c = temp_scale(temperature[row_request(row, rows_per_req, row_req)]);
-  const T* rp = base + static_cast<size_t>(row) * V;
-  const int v0 = slice * kSliceElems, v1 = min(V, v0 + kSliceElems);
-  float m = -INFINITY;
-  double s = 0.0;
-  int amax = 0x7fffffff;
-  bool bad = false;
-  if (c == 0.0f) {
-    thread_slice_stats<T, true>(rp, v0, v1, c, m, s, amax, bad);
-    float M = block_max(m, red);
-    int cand = (m == M) ? amax : 0x7fffffff;
-    // lowest index attaining the maximum
-    cand = __reduce_min_sync(0xffffffffu, cand);
-    __syncthreads();
-    if ((threadIdx.x & 31) == 0) ired[threadIdx.x >> 5] = cand;
-    __syncthreads();
-    if (threadIdx.x < 32) {
-      int x = threadIdx.x < (blockDim.x >> 5) ? ired[threadIdx.x] : 0x7fffffff;
-      x = __reduce_min_sync(0xffffffffu, x);
-      if (threadIdx.x == 0) ired[0] = x;
-    }
-    bad = __syncthreads_or(bad);
-    if (threadIdx.x == 0) out[unit] = Partial{0.0, M, ired[0], bad ? 1 : 0, 0};
+// Running statistics of one lane over a chunk: maximum m and the fp32 sum s of
+// 2^((x - m) c), or (greedy rows) the maximum and its lowest index. A NaN or +inf logit
+// makes s NaN (non-greedy) or sets `bad` (greedy), which marks the row as a data error.
+struct LaneStat {
+  float m, s;
+  int amax;
+  bool bad;
+};
+
+template <bool GREEDY>
+__device__ __forceinline__ void lane_scalar(LaneStat& L, float x, int v, float c) {
+  if (GREEDY) {
+    L.bad |= !(x < INFINITY);
+    if (x > L.m) { L.m = x; L.amax = v; }
   } else {
-    thread_slice_stats<T, false>(rp, v0, v1, c, m, s, amax, bad);
-    float M = block_max(m, red);
-    double mine = (m > -INFINITY) ? s * static_cast<double>(ex2((m - M) * c)) : 0.0;
-    double S = block_sum(mine, dred);
-    bad = __syncthreads_or(bad);
-    if (threadIdx.x == 0) out[unit] = Partial{S, M, 0, bad ? 1 : 0, 0};
+    if (x > L.m) {
+      L.s *= ex2((L.m - x) * c);
+      L.m = x;
+    }
+    L.s += ex2((x - L.m) * c);
+  }
+}
+
+template <typename T, bool GREEDY>
+__device__ __forceinline__ void lane_vector(LaneStat& L, const uint4& raw, int v, float c) {
+  constexpr int N = Vec<T>::N;
+  float f[8];
+  Vec<T>::unpack(raw, f);
+  if (GREEDY) {
+    float vmax = f[0];
+#pragma unroll
+    for (int k = 1; k < N; ++k) vmax = fmax_nan(vmax, f[k]);
+    L.bad |= !(vmax < INFINITY);
+    if (vmax > L.m) {
+#pragma unroll
+      for (int k = N - 1; k >= 0; --k)
+        if (f[k] == vmax) L.amax = v + k;
+      L.m = vmax;
+    }
+  } else {
+    float vmax = f[0];
+#pragma unroll
+    for (int k = 1; k < N; ++k) vmax = fmaxf(vmax, f[k]);
+    if (vmax > L.m) {
+      L.s *= ex2((L.m - vmax) * c);
+      L.m = vmax;
+    }
+    float acc = 0.0f;
+#pragma unroll
+    for (int k = 0; k < N; ++k) acc += ex2((f[k] - L.m) * c);
+    L.s += acc;
+  }
+}
+
+// Warp-level partial of the chunk [c0, c1) of one row: per lane online statistics over
+// coalesced 16-byte vectors (kBatch loads in flight), across lanes fp64. All lanes get it.
+// The lane maximum starts at the lowest finite float so that -inf logits add exact zeros;
+// a lane that saw no finite logit ends with s == 0 and reports -inf.
+template <typename T, bool GREEDY>
+__device__ __forceinline__ Partial warp_chunk_partial(const T* __restrict__ row, int c0, int c1, float c) {
+  constexpr int N = Vec<T>::N;
+  constexpr int stride = 32 * N;
+  constexpr int kFull = kChunkElems / stride;  // vectors per lane in a full chunk
+  const int lane = threadIdx.x & 31;
+  LaneStat L{GREEDY ? -INFINITY : -3.402823466e38f, 0.0f, 0x7fffffff, false};
+  const bool full = c1 - c0 == kChunkElems && (reinterpret_cast<uintptr_t>(row + c0) & 15u) == 0;
+  if (full) {
+    static_assert(kFull % kBatch == 0, "full chunks are whole batches");
+#pragma unroll
+    for (int b = 0; b < kFull; b += kBatch) {
+      uint4 raw[kBatch];
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u)
+        raw[u] = __ldg(reinterpret_cast<const uint4*>(row + c0 + (b + u) * stride + lane * N));
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) lane_vector<T, GREEDY>(L, raw[u], c0 + (b + u) * stride + lane * N, c);
+    }
+  } else {
+    int a0, a1;
+    vec_range(row, c0, c1, a0, a1);
+    for (int v = c0 + lane; v < a0; v += 32) lane_scalar<GREEDY>(L, load_elem(row + v), v, c);
+    for (int v = a1 + lane; v < c1; v += 32) lane_scalar<GREEDY>(L, load_elem(row + v), v, c);
+#pragma unroll 1
+    for (int vb = a0 + lane * N; vb < a1; vb += kBatch * stride) {
+      uint4 raw[kBatch];
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u)
+        if (vb + u * stride < a1) raw[u] = __ldg(reinterpret_cast<const uint4*>(row + vb + u * stride));
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u)
+        if (vb + u * stride < a1) lane_vector<T, GREEDY>(L, raw[u], vb + u * stride, c);
+    }
+  }
+  if (!GREEDY && L.s == 0.0f) L.m = -INFINITY;  // no finite logit in this lane
+  const float M = warp_max(L.m);
+  Partial p{0.0, M, 0, __any_sync(0xffffffffu, L.bad) ? 1 : 0, 0};
+  if (GREEDY) {
+    p.amax = __reduce_min_sync(0xffffffffu, L.m == M ? L.amax : 0x7fffffff);
+  } else {
+    const double mine = L.m > -INFINITY ? static_cast<double>(L.s) * static_cast<double>(ex2((L.m - M) * c)) : 0.0;
+    p.s = warp_sum(mine);  // NaN when the chunk holds a NaN or +inf logit
+  }
+  return p;
+}
+
+// The streaming pass: persistent warps over every chunk of a [rows, V] tensor, each chunk
+// read once, one partial per chunk (parts[row * nchunks + chunk]).
+template <typename T>
+__global__ void __launch_bounds__(kThreads, 4) stream_partials_kernel(const T* __restrict__ base, int rows_per_req,
+                                                                    const int32_t* __restrict__ row_req, int V,
+                                                                    int64_t total_chunks,
+                                                                    const float* __restrict__ temperature,
+                                                                    Partial* __restrict__ parts) {
+  const int nch = nchunks_for(V);
+  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  int64_t g = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (g >= total_chunks) return;
+  // (row, chunk) of g, advanced by nwarps chunks per step without a division in the loop
+  int row = static_cast<int>(g / nch), chunk = static_cast<int>(g - static_cast<int64_t>(row) * nch);
+  const int drow = static_cast<int>(nwarps / nch), dchunk = static_cast<int>(nwarps - static_cast<int64_t>(drow) * nch);
+#pragma unroll 1
+  for (; g < total_chunks; g += nwarps) {
+    const float c = temp_scale(temperature[row_request(row, rows_per_req, row_req)]);
+    const T* rp = base + static_cast<size_t>(row) * V;
+    const int c0 = chunk * kChunkElems, c1 = min(V, c0 + kChunkElems);
+    const Partial p = c == 0.0f ? warp_chunk_partial<T, true>(rp, c0, c1, c) : warp_chunk_partial<T, false>(rp, c0, c1, c);
+    if ((threadIdx.x & 31) == 0) parts[g] = p;
+    row += drow;
+    chunk += dchunk;
+    if (chunk >= nch) {
+      chunk -= nch;
+      ++row;
+    }
   }
 }
 
@@ -159,126 +182,251 @@ __device__ __forceinline__ void for_each_elem(const T* __restrict__ row, int V, 
   }
 }
 
-// One CTA per row. When `jobs` is given (draft sampling), also emits this row's draw job, or
-// writes the token directly for greedy and bad rows.
-template <typename T>
-__global__ void __launch_bounds__(kThreads) row_finalize_kernel(
-    const T* __restrict__ base, int rows_per_req, const int32_t* __restrict__ row_req, int V, int nslices,
-    const float* __restrict__ temperature, const float* __restrict__ top_p, const Partial* __restrict__ parts,
-    RowStat* __restrict__ stats,
-    const float* __restrict__ u, Job* __restrict__ jobs, int32_t* __restrict__ out_tokens,
-    float* __restrict__ out_q) {
-  __shared__ double hmass[256];
-  __shared__ int hcnt[256];
-  __shared__ RowStat st;
-  __shared__ uint32_t sh_prefix;
-  __shared__ double sh_above, sh_bucket;
-  const int row = blockIdx.x, req = row_request(row, rows_per_req, row_req);
-  const float Tv = temperature[req];
-  const float c = temp_scale(Tv);
-  const Partial* pp = parts + static_cast<size_t>(row) * nslices;
+// A partial written by another warp of the running kernel, read through L2.
+__device__ __forceinline__ Partial load_partial_cg(const Partial* p) {
+  Partial q;
+  q.s = __ldcg(&p->s);
+  const int2 a = __ldcg(reinterpret_cast<const int2*>(&p->m));
+  const int2 b = __ldcg(reinterpret_cast<const int2*>(&p->bad));
+  q.m = __int_as_float(a.x);
+  q.amax = a.y;
+  q.bad = b.x;
+  q.pad = b.y;
+  return q;
+}
 
-  if (threadIdx.x < 32) {
-    const int lane = threadIdx.x;
-    float M = -INFINITY;
-    bool bad = !(Tv >= 0.0f && Tv < INFINITY);
-    for (int i = lane; i < nslices; i += 32) {
-      M = fmax_nan(M, pp[i].m);
-      bad |= pp[i].bad != 0;
-    }
-    M = warp_max(M);
-    double S = 0.0;
-    int amax = 0x7fffffff;
-    for (int i = lane; i < nslices; i += 32) {
-      Partial q = pp[i];
-      if (c != 0.0f) {
-        if (q.m > -INFINITY) S += q.s * static_cast<double>(ex2((q.m - M) * c));
-      } else if (q.m == M) {
-        amax = min(amax, q.amax);
+// Warp-level: combine the chunk partials of one row in one pass (read through L2: they may
+// come from other warps of the running kernel). Every lane gets the statistics; top-p is not
+// applied.
+__device__ __forceinline__ RowStat warp_finalize_row(const Partial* __restrict__ pp, int nchunks, float Tv) {
+  const int lane = threadIdx.x & 31;
+  const float c = temp_scale(Tv);
+  float M = -INFINITY;
+  double S = 0.0;
+  int amax = 0x7fffffff;
+  bool bad = !(Tv >= 0.0f && Tv < INFINITY);
+  for (int i = lane; i < nchunks; i += 32) {
+    const Partial q = load_partial_cg(pp + i);
+    bad |= q.bad != 0 || q.m != q.m;
+    if (c != 0.0f) {
+      if (q.m > M) {
+        if (M > -INFINITY) S *= static_cast<double>(ex2((M - q.m) * c));
+        M = q.m;
       }
-    }
-    S = warp_sum(S);
-    amax = __reduce_min_sync(0xffffffffu, amax);
-    bad = __any_sync(0xffffffffu, bad) || !(M > -INFINITY) || !(M < INFINITY);
-    if (lane == 0) {
-      st.m = M;
-      st.c = c;
-      st.s = c != 0.0f ? static_cast<float>(S) : 1.0f;
-      st.s_kept = st.s;
-      st.tau = 0u;
-      st.amax = c != 0.0f ? -1 : amax;
-      st.status = bad ? 1 : 0;
-      st.pad = 0;
+      if (q.m > -INFINITY) S += q.s * static_cast<double>(ex2((q.m - M) * c));
+    } else if (q.m > M || (q.m == M && q.amax < amax)) {
+      M = q.m;
+      amax = q.amax;
     }
   }
-  __syncthreads();
+  const float Mw = warp_max(M);
+  if (c != 0.0f) {
+    S = M > -INFINITY ? S * static_cast<double>(ex2((M - Mw) * c)) : 0.0;
+    S = warp_sum(S);
+  }
+  amax = __reduce_min_sync(0xffffffffu, M == Mw ? amax : 0x7fffffff);
+  bad = __any_sync(0xffffffffu, bad) || !(Mw > -INFINITY) || !(Mw < INFINITY) || (c != 0.0f && !(S == S));
+  RowStat st;
+  st.m = Mw;
+  st.c = c;
+  st.s = c != 0.0f ? static_cast<float>(S) : 1.0f;
+  st.s_kept = st.s;
+  st.tau = 0u;
+  st.amax = c != 0.0f ? -1 : amax;
+  st.status = bad ? 1 : 0;
+  st.pad = 0;
+  return st;
+}
 
-  const float tp = top_p[req];
-  if (st.status == 0 && st.c != 0.0f && tp < 1.0f) {
-    // Top-p threshold: radix select on the 32-bit keys, most significant digit first. For
-    // bf16 rows the two top digits already separate every distinct value.
-    const T* rp = base + static_cast<size_t>(row) * V;
-    const float M = st.m;
-    const double target = static_cast<double>(tp) * static_cast<double>(st.s);
-    const int levels = sizeof(T) == 2 ? 2 : 4;
-    if (threadIdx.x == 0) { sh_prefix = 0u; sh_above = 0.0; sh_bucket = 0.0; }
-    for (int lv = 0; lv < levels; ++lv) {
-      const int shift = 24 - 8 * lv;
-      for (int d = threadIdx.x; d < 256; d += blockDim.x) { hmass[d] = 0.0; hcnt[d] = 0; }
-      __syncthreads();
-      const uint32_t prefix = sh_prefix;
-      for_each_elem(rp, V, [&](float x) {
-        uint32_t k = fkey(x);
-        if (lv == 0 || (k >> (shift + 8)) == (prefix >> (shift + 8))) {
-          int d = (k >> shift) & 255;
-          atomicAdd(&hmass[d], static_cast<double>(ex2((x - M) * c)));
-          atomicAdd(&hcnt[d], 1);
-        }
-      });
-      __syncthreads();
-      if (threadIdx.x == 0) {
-        double running = sh_above;
-        int pick = -1;
-        for (int d = 255; d >= 0; --d) {
-          if (hcnt[d] == 0) continue;
-          if (running + hmass[d] >= target) { pick = d; break; }
-          running += hmass[d];
-        }
-        if (pick < 0) {  // rounding left the target unreached: keep the whole candidate range
-          running = sh_above;
-          for (int d = 255; d >= 0; --d)
-            if (hcnt[d] != 0) { pick = d; running += hmass[d]; }
-          running -= hmass[pick];
-        }
-        sh_prefix = prefix | (static_cast<uint32_t>(pick) << shift);
-        sh_above = running;
-        sh_bucket = hmass[pick];
-      }
-      __syncthreads();
+constexpr int kCache = 4;  // chunk partials per lane held in registers by warp_finalize_pick
+
+// Result of warp_finalize_pick.
+struct RowPick {
+  RowStat st;
+  int chunk;           // chunk holding u * Z (-1 if none / not requested)
+  double base, target;  // weight before that chunk, and u * Z
+};
+
+// Warp-level finish of one row from its chunk partials in one round trip: statistics (as
+// warp_finalize_row) and, when `pick` is set, the chunk holding u * Z of the row's own
+// distribution (no top-p cut). Lane l owns the contiguous chunks [l*q, l*q + q); for rows
+// of more than 32 * kCache chunks it falls back to two passes.
+__device__ __forceinline__ RowPick warp_finalize_pick(const Partial* __restrict__ pp, int nchunks, float Tv, float u,
+                                                      bool pick) {
+  const int lane = threadIdx.x & 31;
+  RowPick r;
+  r.chunk = -1;
+  r.base = 0.0;
+  r.target = 0.0;
+  const int q = (nchunks + 31) / 32;
+  if (q > kCache) {
+    r.st = warp_finalize_row(pp, nchunks, Tv);
+    return r;  // callers use warp_pick_chunk on this path
+  }
+  const float c = temp_scale(Tv);
+  const int i0 = min(nchunks, lane * q);
+  Partial part[kCache];
+#pragma unroll
+  for (int k = 0; k < kCache; ++k)
+    if (k < q && i0 + k < nchunks) part[k] = load_partial_cg(pp + i0 + k);
+  float M = -INFINITY;
+  int amax = 0x7fffffff;
+  bool bad = !(Tv >= 0.0f && Tv < INFINITY);
+#pragma unroll
+  for (int k = 0; k < kCache; ++k) {
+    if (!(k < q && i0 + k < nchunks)) continue;
+    bad |= part[k].bad != 0 || part[k].m != part[k].m;
+    if (part[k].m > M || (c == 0.0f && part[k].m == M && part[k].amax < amax)) {
+      M = part[k].m;
+      amax = part[k].amax;
     }
+  }
+  const float Mw = warp_max(M);
+  double t[kCache];
+  double mine = 0.0;
+#pragma unroll
+  for (int k = 0; k < kCache; ++k) {
+    t[k] = (k < q && i0 + k < nchunks && c != 0.0f && part[k].m > -INFINITY)
+               ? part[k].s * static_cast<double>(ex2((part[k].m - Mw) * c))
+               : 0.0;
+    mine += t[k];
+  }
+  double incl = mine;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const double y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  const double S = __shfl_sync(0xffffffffu, incl, 31);
+  amax = __reduce_min_sync(0xffffffffu, M == Mw ? amax : 0x7fffffff);
+  bad = __any_sync(0xffffffffu, bad) || !(Mw > -INFINITY) || !(Mw < INFINITY) || (c != 0.0f && !(S == S));
+  r.st.m = Mw;
+  r.st.c = c;
+  r.st.s = c != 0.0f ? static_cast<float>(S) : 1.0f;
+  r.st.s_kept = r.st.s;
+  r.st.tau = 0u;
+  r.st.amax = c != 0.0f ? -1 : amax;
+  r.st.status = bad ? 1 : 0;
+  r.st.pad = 0;
+  if (pick && !bad && c != 0.0f) {
+    double excl = __shfl_up_sync(0xffffffffu, incl, 1);
+    if (lane == 0) excl = 0.0;
+    const double tg = static_cast<double>(u) * S;
+    int sel = -1, last = -1;
+    double b = 0.0, C = excl;
+#pragma unroll
+    for (int k = 0; k < kCache; ++k) {
+      if (t[k] > 0.0) {
+        last = i0 + k;
+        if (sel < 0 && excl <= tg && tg < incl) {
+          if (C + t[k] > tg) { sel = i0 + k; b = C; }
+        }
+      }
+      C += t[k];
+    }
+    const unsigned who = __ballot_sync(0xffffffffu, sel >= 0);
+    if (who) {
+      const int src = __ffs(who) - 1;
+      r.chunk = __shfl_sync(0xffffffffu, sel, src);
+      r.base = __shfl_sync(0xffffffffu, b, src);
+    } else {  // rounding put u * Z past every chunk: the last chunk with positive weight
+      const int lastc = __reduce_max_sync(0xffffffffu, last);
+      const int owner = __reduce_max_sync(0xffffffffu, last == lastc ? lane : -1);
+      double bb = excl;
+#pragma unroll
+      for (int k = 0; k < kCache; ++k)
+        if (i0 + k < lastc) bb += t[k];
+      r.chunk = lastc;
+      r.base = __shfl_sync(0xffffffffu, bb, owner < 0 ? 0 : owner);
+    }
+    r.target = tg;
+  }
+  return r;
+}
+
+// Whether a row's statistics still need the top-p threshold.
+__device__ __forceinline__ bool needs_topp(const RowStat& st, float tp) {
+  return st.status == 0 && st.c != 0.0f && tp < 1.0f;
+}
+
+// Shared memory of a block-level top-p selection.
+struct ToppSmem {
+  double hmass[256];
+  int hcnt[256];
+  uint32_t prefix;
+  double above, bucket;
+};
+
+// Block-level top-p threshold of row rp under statistics st (m, c, s set): radix select on the
+// 32-bit keys, most significant digit first, with the fp64 mass of every digit. For bf16 rows
+// the two top digits already separate every distinct value. Sets st.tau and st.s_kept (in
+// every thread).
+template <typename T>
+__device__ void block_topp_select(const T* __restrict__ rp, int V, float tp, RowStat& st, ToppSmem& sm) {
+  const float M = st.m, c = st.c;
+  const double target = static_cast<double>(tp) * static_cast<double>(st.s);
+  const int levels = sizeof(T) == 2 ? 2 : 4;
+  if (threadIdx.x == 0) { sm.prefix = 0u; sm.above = 0.0; sm.bucket = 0.0; }
+  for (int lv = 0; lv < levels; ++lv) {
+    const int shift = 24 - 8 * lv;
+    for (int d = threadIdx.x; d < 256; d += blockDim.x) { sm.hmass[d] = 0.0; sm.hcnt[d] = 0; }
+    __syncthreads();
+    const uint32_t prefix = sm.prefix;
+    for_each_elem(rp, V, [&](float x) {
+      const uint32_t k = fkey(x);
+      if (lv == 0 || (k >> (shift + 8)) == (prefix >> (shift + 8))) {
+        const int d = (k >> shift) & 255;
+        atomicAdd(&sm.hmass[d], static_cast<double>(ex2((x - M) * c)));
+        atomicAdd(&sm.hcnt[d], 1);
+      }
+    });
+    __syncthreads();
     if (threadIdx.x == 0) {
-      st.tau = sh_prefix;
-      st.s_kept = static_cast<float>(sh_above + sh_bucket);
+      double running = sm.above;
+      int pick = -1;
+      for (int d = 255; d >= 0; --d) {
+        if (sm.hcnt[d] == 0) continue;
+        if (running + sm.hmass[d] >= target) { pick = d; break; }
+        running += sm.hmass[d];
+      }
+      if (pick < 0) {  // rounding left the target unreached: keep the whole candidate range
+        running = sm.above;
+        for (int d = 255; d >= 0; --d)
+          if (sm.hcnt[d] != 0) { pick = d; running += sm.hmass[d]; }
+        running -= sm.hmass[pick];
+      }
+      sm.prefix = prefix | (static_cast<uint32_t>(pick) << shift);
+      sm.above = running;
+      sm.bucket = sm.hmass[pick];
     }
     __syncthreads();
   }
+  st.tau = sm.prefix;
+  st.s_kept = static_cast<float>(sm.above + sm.bucket);
+  __syncthreads();
+}
 
-  if (threadIdx.x == 0) {
-    stats[row] = st;
-    if (jobs != nullptr) {
-      Job jb{kNone, row, -1, row, u[row], row, {0, 0}};
-      if (st.status != 0) {
-        out_tokens[row] = -1;
-        if (out_q) out_q[row] = -1.0f;
-      } else if (st.c == 0.0f) {
-        out_tokens[row] = st.amax;
-        if (out_q) out_q[row] = 1.0f;
-      } else {
-        jb.mode = kSample;
-      }
-      jobs[row] = jb;
-    }
+// One CTA per row (the tree's statistics pass).
+template <typename T>
+__global__ void __launch_bounds__(kThreads) row_finalize_kernel(const T* __restrict__ base, int rows_per_req,
+                                                                 const int32_t* __restrict__ row_req, int V,
+                                                                 const float* __restrict__ temperature,
+                                                                 const float* __restrict__ top_p,
+                                                                 const Partial* __restrict__ parts,
+                                                                 RowStat* __restrict__ stats) {
+  __shared__ ToppSmem sm;
+  __shared__ RowStat sh_st;
+  const int row = blockIdx.x, req = row_request(row, rows_per_req, row_req);
+  const int nch = nchunks_for(V);
+  if (threadIdx.x < 32) {
+    const RowStat st = warp_finalize_row(parts + static_cast<size_t>(row) * nch, nch, temperature[req]);
+    if (threadIdx.x == 0) sh_st = st;
   }
+  __syncthreads();
+  RowStat st = sh_st;
+  const float tp = top_p[req];
+  if (needs_topp(st, tp)) block_topp_select<T>(base + static_cast<size_t>(row) * V, V, tp, st, sm);
+  if (threadIdx.x == 0) stats[row] = st;
 }
 
 }  // namespace psi
