@@ -30,9 +30,9 @@ sys.path.insert(0, ROOT)
 METRIC = "verified draft positions/sec and logits HBM GB/s vs B200 peak (Ψ-Spec verify)"
 UNIT = "positions/s"
 # kernel launches per call (see csrc/psispec.cu): sample_draft = stream + finish + top-p;
-# verify_linear = stream + finish + top-p + clustered draw (the per-request
+# verify_linear = stream + finish + top-p + draw totals + draw pick (the per-request
 # arrival counters are cleared with a memset, which is not a kernel of this library)
-LAUNCHES_PER_STEP = 3 + 4
+LAUNCHES_PER_STEP = 3 + 5
 
 
 def _peaks():

@@ -75,6 +75,59 @@ __device__ __forceinline__ float fmax_nan(float a, float b) {
   return y;
 }
 
+// Two fp32 values in one 64-bit register, for the packed sm_100 fp32x2 arithmetic. The
+// packed operations round every lane exactly like their scalar counterparts.
+using f32x2 = unsigned long long;
+__device__ __forceinline__ f32x2 pack2(float a, float b) {
+  f32x2 r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void unpack2(f32x2 r, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r));
+}
+__device__ __forceinline__ f32x2 sub2(f32x2 a, f32x2 b) {
+  f32x2 d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ f32x2 mul2(f32x2 a, f32x2 b) {
+  f32x2 d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ f32x2 add2(f32x2 a, f32x2 b) {
+  f32x2 d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// 2^((x_k - m) c) for the 8 values of x, in the same arithmetic as kept_weight (x - m
+// rounded, then the product rounded, then ex2).
+__device__ __forceinline__ void exp8(const float (&x)[8], float m, float c, float (&w)[8]) {
+  const f32x2 mm = pack2(m, m), cc = pack2(c, c);
+#pragma unroll
+  for (int k = 0; k < 8; k += 2) {
+    float a, b;
+    unpack2(mul2(sub2(pack2(x[k], x[k + 1]), mm), cc), a, b);
+    w[k] = ex2(a);
+    w[k + 1] = ex2(b);
+  }
+}
+
+// Sum of 8 values as four packed pair sums then two scalar adds (a fixed association).
+__device__ __forceinline__ float sum8(const float (&w)[8]) {
+  const f32x2 s = add2(add2(pack2(w[0], w[1]), pack2(w[2], w[3])), add2(pack2(w[4], w[5]), pack2(w[6], w[7])));
+  float a, b;
+  unpack2(s, a, b);
+  return a + b;
+}
+
 // order-preserving key of a float; -0 and +0 share one key
 __device__ __forceinline__ uint32_t fkey(float x) {
   uint32_t b = __float_as_uint(x);
@@ -85,6 +138,11 @@ __device__ __forceinline__ uint32_t fkey(float x) {
 __device__ __forceinline__ bool is_finite(float x) { return fabsf(x) <= 3.402823466e38f; }
 
 __device__ __forceinline__ float load_elem(const float* p) { return __ldg(p); }
+// element load through a generic pointer (global or shared memory)
+__device__ __forceinline__ float load_elem_any(const float* p) { return *p; }
+__device__ __forceinline__ float load_elem_any(const __nv_bfloat16* p) {
+  return __uint_as_float(static_cast<uint32_t>(*reinterpret_cast<const unsigned short*>(p)) << 16);
+}
 __device__ __forceinline__ float load_elem(const __nv_bfloat16* p) {
   unsigned short h = __ldg(reinterpret_cast<const unsigned short*>(p));
   return __uint_as_float(static_cast<uint32_t>(h) << 16);

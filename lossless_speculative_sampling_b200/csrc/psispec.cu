@@ -2,6 +2,8 @@
 // The operations are specified in include/psispec.h.
 #include "psispec.h"
 
+#include <algorithm>
+
 #include "common.cuh"
 #include "finish.cuh"
 #include "linear.cuh"
@@ -107,11 +109,29 @@ unsigned persistent_grid(Kern kernel, int64_t work_warps) {
   return static_cast<unsigned>(want < 1 ? 1 : (want < slots ? want : slots));
 }
 
-// The streaming pass over a [rows, V] tensor: one partial per chunk.
+// The streaming pass over a [rows, V] tensor: one partial per chunk. Aligned tensors go
+// through the bulk-copy ring kernel, others through plain 16-byte loads.
 template <typename T>
 psispec_status launch_stream(const T* base, int64_t rows, int rows_per_req, const int32_t* row_req, int V,
-                             const float* temperature, Partial* parts, cudaStream_t st) {
+                             const float* temperature, int nreq, Partial* parts, cudaStream_t st) {
   const int64_t chunks = rows * nchunks_for(V);
+  const bool aligned = (reinterpret_cast<uintptr_t>(base) & 15u) == 0 && (int64_t(V) * sizeof(T)) % 16 == 0;
+  if (aligned) {
+    const int smem = (kThreads / 32) * kRing * kStageBytes<T>;
+    if (cudaFuncSetAttribute(stream_partials_tma_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+        cudaSuccess)
+      return PSISPEC_ERR_CUDA;
+    int dev = 0, sms = 148, occ = 1;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, stream_partials_tma_kernel<T>, kThreads, smem);
+    const int64_t want = (chunks + (kThreads / 32) - 1) / (kThreads / 32);
+    const int64_t slots = static_cast<int64_t>(sms) * (occ > 0 ? occ : 1);
+    const unsigned grid = static_cast<unsigned>(want < slots ? want : slots);
+    stream_partials_tma_kernel<T><<<grid, kThreads, smem, st>>>(base, rows_per_req, row_req, V, chunks, temperature,
+                                                                nreq, parts);
+    return launched();
+  }
   stream_partials_kernel<T><<<persistent_grid(stream_partials_kernel<T>, chunks), kThreads, 0, st>>>(
       base, rows_per_req, row_req, V, chunks, temperature, parts);
   return launched();
@@ -120,8 +140,8 @@ psispec_status launch_stream(const T* base, int64_t rows, int rows_per_req, cons
 // Row statistics of a [rows, V] tensor (the tree's statistics pass).
 template <typename T>
 psispec_status launch_stats(const T* base, int64_t rows, int rows_per_req, const int32_t* row_req, int V,
-                            const float* temperature, const float* top_p, StatsWs ws, cudaStream_t st) {
-  psispec_status s = launch_stream<T>(base, rows, rows_per_req, row_req, V, temperature, ws.parts, st);
+                            const float* temperature, int nreq, const float* top_p, StatsWs ws, cudaStream_t st) {
+  psispec_status s = launch_stream<T>(base, rows, rows_per_req, row_req, V, temperature, nreq, ws.parts, st);
   if (s != PSISPEC_OK) return s;
   row_finalize_kernel<T><<<static_cast<unsigned>(rows), kThreads, 0, st>>>(base, rows_per_req, row_req, V,
                                                                             temperature, top_p, ws.parts, ws.stats);
@@ -136,7 +156,7 @@ psispec_status sample_draft_impl(const T* draft, int B, int K, int V, const floa
   Carver c(ws);
   SampleWs w = carve_sample(c, rows, V);
   RowStat* stats = out_stats ? out_stats : w.st.stats;
-  psispec_status s = launch_stream<T>(draft, rows, K, nullptr, V, temperature, w.st.parts, st);
+  psispec_status s = launch_stream<T>(draft, rows, K, nullptr, V, temperature, B, w.st.parts, st);
   if (s != PSISPEC_OK) return s;
   sample_finish_kernel<T><<<static_cast<unsigned>((rows + 7) / 8), kThreads, 0, st>>>(
       draft, K, V, static_cast<int>(rows), temperature, top_p, u, w.st.parts, stats, out_tokens, out_q);
@@ -176,18 +196,22 @@ psispec_status verify_linear_impl(const T* tgt, const T* drf, int B, int K, int 
   a.out_p = out_p;
   a.out_q = out_q;
   a.jobs = w.jobs;
-  psispec_status s = launch_stream<T>(tgt, rows_t, K + 1, nullptr, V, temperature, w.t.parts, st);
+  psispec_status s = launch_stream<T>(tgt, rows_t, K + 1, nullptr, V, temperature, B, w.t.parts, st);
   if (s != PSISPEC_OK) return s;
-  if (rows_d > 0 && (s = launch_stream<T>(drf, rows_d, K, nullptr, V, temperature, w.d.parts, st)) != PSISPEC_OK)
+  if (rows_d > 0 && (s = launch_stream<T>(drf, rows_d, K, nullptr, V, temperature, B, w.d.parts, st)) != PSISPEC_OK)
     return s;
-  verify_finish_kernel<T><<<static_cast<unsigned>(B), kThreads, 0, st>>>(tgt, drf, a);
+  const int finish_warps = static_cast<int>(std::min<int64_t>(32, (K + 1) + (rows_d ? K : 0)));
+  verify_finish_kernel<T><<<static_cast<unsigned>(B), 32 * finish_warps, 0, st>>>(tgt, drf, a);
   if ((s = launched()) != PSISPEC_OK) return s;
   verify_topp_kernel<T><<<static_cast<unsigned>(rows_t + rows_d), kThreads, 0, st>>>(tgt, drf, a);
   if ((s = launched()) != PSISPEC_OK) return s;
   const RowStat* ds = draft_stats ? draft_stats : w.d.stats;
-  const int64_t draw_warps = int64_t(B) * nchunks_for(V);
-  draw_jobs_kernel<T><<<static_cast<unsigned>((draw_warps + 7) / 8), kThreads, 0, st>>>(
-      tgt, drf, V, B, w.t.stats, ds, w.t.parts, w.jobs, w.draw_tot, w.cnt + B, out_tokens);
+  const int64_t items = int64_t(B) * nchunks_for(V);
+  draw_totals_kernel<T><<<persistent_grid(draw_totals_kernel<T>, items), kThreads, 0, st>>>(tgt, drf, V, B, w.t.stats,
+                                                                                          ds, w.jobs, w.draw_tot);
+  if ((s = launched()) != PSISPEC_OK) return s;
+  draw_pick_kernel<T><<<static_cast<unsigned>(B), 32, 0, st>>>(tgt, drf, V, B, w.t.stats, ds, w.t.parts, w.jobs,
+                                                                 w.draw_tot, out_tokens);
   return launched();
 }
 
@@ -202,9 +226,9 @@ psispec_status verify_tree_impl(const T* tgt, const T* drf, int B, int N, int V,
   node_request_kernel<<<B, 128, 0, st>>>(offs, B, N, w.row_req);
   psispec_status s = launched();
   if (s != PSISPEC_OK) return s;
-  s = launch_stats<T>(tgt, N, 1, w.row_req, V, temperature, top_p, w.t, st);
+  s = launch_stats<T>(tgt, N, 1, w.row_req, V, temperature, B, top_p, w.t, st);
   if (s != PSISPEC_OK) return s;
-  s = launch_stats<T>(drf, N, 1, w.row_req, V, temperature, top_p, w.d, st);
+  s = launch_stats<T>(drf, N, 1, w.row_req, V, temperature, B, top_p, w.d, st);
   if (s != PSISPEC_OK) return s;
   tree_walk_kernel<T><<<B, kTreeThreads, 0, st>>>(tgt, drf, V, offs, parent, tokens, w.t.stats, w.d.stats, u_acc,
                                                   u_res, max_depth, out_path, out_tokens, out_len);

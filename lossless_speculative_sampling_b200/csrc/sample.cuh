@@ -123,22 +123,29 @@ struct JobRows {
   __device__ __forceinline__ void weights(const Raw8<T, RESID>& x, float (&w)[8], float (&pw)[8]) const {
     float xa[8];
     x.a.unpack(xa);
+    exp8(xa, r.a.m, r.a.c, pw);
+    if (r.a.tau != 0u) {
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        if (fkey(xa[k]) < r.a.tau) pw[k] = 0.0f;
+    }
     if constexpr (RESID) {
-      float xb[8];
+      float xb[8], qw[8];
       x.b[0].unpack(xb);
+      exp8(xb, r.b.m, r.b.c, qw);
+      if (r.b.tau != 0u) {
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          if (fkey(xb[k]) < r.b.tau) qw[k] = 0.0f;
+      }
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
-        const float pa = kept_weight(r.a, xa[k]) * r.ia;
-        const float qb = kept_weight(r.b, xb[k]) * r.ib;
-        w[k] = use_p ? pa : fmaxf(pa - qb, 0.0f);
-        pw[k] = pa;
+        pw[k] *= r.ia;
+        w[k] = use_p ? pw[k] : fmaxf(pw[k] - qw[k] * r.ib, 0.0f);
       }
     } else {
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        w[k] = kept_weight(r.a, xa[k]);
-        pw[k] = w[k];
-      }
+      for (int k = 0; k < 8; ++k) w[k] = pw[k];
     }
   }
 };

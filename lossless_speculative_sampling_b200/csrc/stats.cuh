@@ -70,17 +70,26 @@ __device__ __forceinline__ void lane_vector(LaneStat& L, const uint4& raw, int v
       L.m = vmax;
     }
   } else {
-    float vmax = f[0];
-#pragma unroll
-    for (int k = 1; k < N; ++k) vmax = fmaxf(vmax, f[k]);
+    float vmax;
+    if (N == 8) {
+      vmax = fmaxf(fmaxf(fmaxf(f[0], f[1]), fmaxf(f[2], f[3])), fmaxf(fmaxf(f[4], f[5]), fmaxf(f[6], f[7])));
+    } else {
+      vmax = fmaxf(fmaxf(f[0], f[1]), fmaxf(f[2], f[3]));
+    }
     if (vmax > L.m) {
       L.s *= ex2((L.m - vmax) * c);
       L.m = vmax;
     }
-    float acc = 0.0f;
+    if (N == 8) {
+      float w[8];
+      exp8(f, L.m, c, w);
+      L.s += sum8(w);
+    } else {
+      float acc = 0.0f;
 #pragma unroll
-    for (int k = 0; k < N; ++k) acc += ex2((f[k] - L.m) * c);
-    L.s += acc;
+      for (int k = 0; k < N; ++k) acc += ex2((f[k] - L.m) * c);
+      L.s += acc;
+    }
   }
 }
 
@@ -163,6 +172,160 @@ __global__ void __launch_bounds__(kThreads, 4) stream_partials_kernel(const T* _
       chunk -= nch;
       ++row;
     }
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// Bulk-copy (TMA, non-tensor) streaming pass. Every warp owns a private ring of kRing
+// shared-memory stages of one chunk each; its lane 0 keeps kRing - 1 chunks in flight with
+// cp.async.bulk (completion counted on one mbarrier per stage) while the warp reduces the
+// oldest one from shared memory. Requires 16-byte aligned rows whose byte length is a
+// multiple of 16 (then every chunk copy is aligned); other tensors use the LDG pass.
+constexpr int kRing = 2;
+template <typename T>
+constexpr int kStageBytes = kChunkElems * static_cast<int>(sizeof(T));  // one chunk
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
+}
+// Bounded wait for a stage: false if the copy has not landed after about a second.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity))
+    if (globaltimer_ns() - t0 > 1000000000ull) return false;
+  return true;
+}
+
+// Warp-level partial of one chunk held in shared memory (n elements, 16-byte vectors).
+template <typename T, bool GREEDY>
+__device__ __forceinline__ Partial warp_chunk_partial_smem(const T* __restrict__ sp, int c0, int n, float c) {
+  constexpr int N = Vec<T>::N;
+  constexpr int kFull = kChunkElems / (32 * N);  // vectors per lane in a full chunk
+  const int lane = threadIdx.x & 31;
+  LaneStat L{GREEDY ? -INFINITY : -3.402823466e38f, 0.0f, 0x7fffffff, false};
+  const uint4* v4 = reinterpret_cast<const uint4*>(sp);
+  if (n == kChunkElems) {
+    uint4 raw[kFull];
+#pragma unroll
+    for (int j = 0; j < kFull; ++j) raw[j] = v4[lane + 32 * j];
+#pragma unroll
+    for (int j = 0; j < kFull; ++j) lane_vector<T, GREEDY>(L, raw[j], c0 + (lane + 32 * j) * N, c);
+  } else {
+    const int nv = n / N;
+    for (int j = lane; j < nv; j += 32) lane_vector<T, GREEDY>(L, v4[j], c0 + j * N, c);
+  }
+  if (!GREEDY && L.s == 0.0f) L.m = -INFINITY;  // no finite logit in this lane
+  const float M = warp_max(L.m);
+  Partial p{0.0, M, 0, __any_sync(0xffffffffu, L.bad) ? 1 : 0, 0};
+  if (GREEDY) {
+    p.amax = __reduce_min_sync(0xffffffffu, L.m == M ? L.amax : 0x7fffffff);
+  } else {
+    const double mine = L.m > -INFINITY ? static_cast<double>(L.s) * static_cast<double>(ex2((L.m - M) * c)) : 0.0;
+    p.s = warp_sum(mine);
+  }
+  return p;
+}
+
+// log2(e)/T of up to kScaleTable requests, computed once per CTA into shared memory (the
+// fp64 division per chunk would otherwise cost a few percent of the streaming pass).
+constexpr int kScaleTable = 1024;
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads) stream_partials_tma_kernel(const T* __restrict__ base, int rows_per_req,
+                                                                        const int32_t* __restrict__ row_req, int V,
+                                                                        int64_t total_chunks,
+                                                                        const float* __restrict__ temperature,
+                                                                        int nreq, Partial* __restrict__ parts) {
+  extern __shared__ __align__(128) unsigned char ring_smem[];
+  __shared__ uint64_t bars[kThreads / 32][kRing];
+  __shared__ float scale[kScaleTable];
+  const bool table = nreq <= kScaleTable;
+  if (table)
+    for (int i = threadIdx.x; i < nreq; i += kThreads) scale[i] = temp_scale(temperature[i]);
+  __syncthreads();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  unsigned char* ring = ring_smem + warp * kRing * kStageBytes<T>;
+  uint64_t* bar = bars[warp];
+  const int nch = nchunks_for(V);
+  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (kThreads / 32);
+  const int64_t g0 = static_cast<int64_t>(blockIdx.x) * (kThreads / 32) + warp;
+  if (g0 >= total_chunks) return;
+  if (lane == 0) {
+    for (int s = 0; s < kRing; ++s) mbar_init(&bar[s], 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncwarp();
+  // (row, chunk) cursors advanced by nwarps chunks per step, for the copies and the reduction
+  const int drow = static_cast<int>(nwarps / nch), dchunk = static_cast<int>(nwarps - static_cast<int64_t>(drow) * nch);
+  auto advance = [&](int& row, int& chunk) {
+    row += drow;
+    chunk += dchunk;
+    if (chunk >= nch) {
+      chunk -= nch;
+      ++row;
+    }
+  };
+  int row = static_cast<int>(g0 / nch), chunk = static_cast<int>(g0 - static_cast<int64_t>(row) * nch);
+  int irow = row, ichunk = chunk;  // cursor of the next copy to issue
+  int64_t gi = g0;
+  auto issue = [&](int i) {  // copy of this warp's i-th chunk into stage i % kRing (lane 0)
+    if (gi < total_chunks) {
+      const int c0 = ichunk * kChunkElems, n = min(V - c0, kChunkElems);
+      const uint32_t bytes = static_cast<uint32_t>(n) * sizeof(T);
+      uint64_t* b = &bar[i % kRing];
+      mbar_expect_tx(b, bytes);
+      bulk_g2s(ring + (i % kRing) * kStageBytes<T>, base + static_cast<size_t>(irow) * V + c0, bytes, b);
+    }
+    gi += nwarps;
+    advance(irow, ichunk);
+  };
+  if (lane == 0)
+    for (int i = 0; i < kRing - 1; ++i) issue(i);
+  int i = 0;
+  for (int64_t g = g0; g < total_chunks; g += nwarps, ++i) {
+    __syncwarp();  // every lane is done with the stage that the next copy overwrites
+    if (lane == 0) issue(i + kRing - 1);
+    const int c0 = chunk * kChunkElems, n = min(V - c0, kChunkElems);
+    const int req = row_request(row, rows_per_req, row_req);
+    const float c = table ? scale[req] : temp_scale(temperature[req]);
+    const bool landed = mbar_wait_bounded(&bar[i % kRing], static_cast<uint32_t>((i / kRing) & 1));
+    if (!__all_sync(0xffffffffu, landed)) {
+      // a copy that never completed: report this chunk as a data error and stop streaming
+      if (lane == 0) parts[g] = Partial{0.0, NAN, 0, 1, 0};
+      return;
+    }
+    const T* sp = reinterpret_cast<const T*>(ring + (i % kRing) * kStageBytes<T>);
+    const Partial p = c == 0.0f ? warp_chunk_partial_smem<T, true>(sp, c0, n, c)
+                                : warp_chunk_partial_smem<T, false>(sp, c0, n, c);
+    if (lane == 0) parts[g] = p;
+    advance(row, chunk);
   }
 }
 
