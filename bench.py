@@ -32,7 +32,7 @@ UNIT = "positions/s"
 # kernel launches per call (see csrc/psispec.cu): sample_draft = stream + finish + top-p;
 # verify_linear = stream + finish + top-p + draw totals + draw pick (the per-request
 # arrival counters are cleared with a memset, which is not a kernel of this library)
-LAUNCHES_PER_STEP = 3 + 5
+LAUNCHES_PER_STEP = 2 + 4  # sample: stream, sample_row; verify: stream, verify_row, draw totals, draw pick
 
 
 def _peaks():

@@ -49,18 +49,20 @@ struct Partial {
 static_assert(sizeof(Partial) == 24 && offsetof(Partial, m) == 8 && offsetof(Partial, bad) == 16, "partial layout");
 
 // Inverse-CDF job: draw from row a of tensor A (mode kSample) or from max(0, pA - qB)
-// (mode kResidual), with uniform u; the result goes to out_tokens[out_index].
+// (mode kResidual), with uniform u; the result goes to out_tokens[out_index]. The job carries
+// the statistics of both rows so that a worker needs one load to start.
 enum JobMode : int32_t { kNone = 0, kSample = 2, kResidual = 3 };
-struct Job {
+struct __align__(16) Job {
   int32_t mode;
   int32_t row_a;
   int32_t row_b;
   int32_t out_index;
   float u;
-  int32_t aux;  // index for a probability output (sample_draft's out_q), -1 if none
-  int32_t pad[2];
+  int32_t pad[3];
+  RowStat sa;  // statistics of row a
+  RowStat sb;  // statistics of row b (residual jobs)
 };
-static_assert(sizeof(Job) == 32, "job record is 32 bytes");
+static_assert(sizeof(Job) == 96 && offsetof(Job, sa) == 32 && offsetof(Job, sb) == 64, "job record layout");
 
 __device__ __forceinline__ float ex2(float x) {
   float y;
@@ -126,6 +128,59 @@ __device__ __forceinline__ float sum8(const float (&w)[8]) {
   float a, b;
   unpack2(s, a, b);
   return a + b;
+}
+
+// A row-statistics record from its two 16-byte words.
+__device__ __forceinline__ RowStat stat_from(const int4& a, const int4& b) {
+  RowStat s;
+  s.m = __int_as_float(a.x);
+  s.c = __int_as_float(a.y);
+  s.s = __int_as_float(a.z);
+  s.s_kept = __int_as_float(a.w);
+  s.tau = static_cast<uint32_t>(b.x);
+  s.amax = b.y;
+  s.status = b.z;
+  s.pad = b.w;
+  return s;
+}
+
+// A row-statistics record written by another CTA of the running kernel (read through L2).
+__device__ __forceinline__ RowStat load_stat_cg(const RowStat* p) {
+  const int4* q = reinterpret_cast<const int4*>(p);
+  return stat_from(__ldcg(q), __ldcg(q + 1));
+}
+
+// A job record written by another CTA or an earlier kernel (read through L2).
+__device__ __forceinline__ Job load_job_cg(const Job* p) {
+  const int4* q = reinterpret_cast<const int4*>(p);
+  const int4 h = __ldcg(q), g = __ldcg(q + 1), a0 = __ldcg(q + 2), a1 = __ldcg(q + 3), b0 = __ldcg(q + 4),
+             b1 = __ldcg(q + 5);
+  Job j;
+  j.mode = h.x;
+  j.row_a = h.y;
+  j.row_b = h.z;
+  j.out_index = h.w;
+  j.u = __int_as_float(g.x);
+  j.pad[0] = g.y;
+  j.pad[1] = g.z;
+  j.pad[2] = g.w;
+  j.sa = stat_from(a0, a1);
+  j.sb = stat_from(b0, b1);
+  return j;
+}
+
+// Row statistics held by lane `src` of the warp, to every lane.
+__device__ __forceinline__ RowStat shfl_stat(const RowStat& s, int src) {
+  RowStat r;
+  r.m = __shfl_sync(0xffffffffu, s.m, src);
+  r.c = __shfl_sync(0xffffffffu, s.c, src);
+  r.s = __shfl_sync(0xffffffffu, s.s, src);
+  r.s_kept = __shfl_sync(0xffffffffu, s.s_kept, src);
+  r.tau = __shfl_sync(0xffffffffu, s.tau, src);
+  r.amax = __shfl_sync(0xffffffffu, s.amax, src);
+  r.status = __shfl_sync(0xffffffffu, s.status, src);
+  r.pad = __shfl_sync(0xffffffffu, s.pad, src);
+  return r;
 }
 
 // order-preserving key of a float; -0 and +0 share one key

@@ -2,20 +2,19 @@
 //
 // The streaming pass (stream_partials_kernel) reads every logits row once and leaves one
 // partial per kChunkElems-element chunk. The kernels here finish from those partials:
-//   sample_finish_kernel   one warp per draft row: row statistics, then the inverse-CDF draw
-//                          inside the one chunk that holds u * Z (chunk partials are the
-//                          prefix totals);
-//   sample_topp_kernel     one CTA per draft row with a top-p cut (returns at once for the
-//                          others): threshold by radix select, then a draw over the row;
-//   verify_finish_kernel   one CTA per request: statistics of its verifier (and draft) rows,
-//                          then, for requests without top-p, the accept tests, the first
-//                          rejection and the draw job;
-//   verify_topp_kernel     one CTA per row of a top-p request: threshold; the CTA that
-//                          completes the request decides it;
-//   draw_jobs_kernel       one warp per (draw job, chunk): chunk totals of the residual (or
-//                          kept) weights; the warp that completes a job picks the chunk that
-//                          holds u * Z and walks it.
-// Cross-warp handoffs use arrival counters (the last arrival continues); nothing waits.
+//   sample_row_kernel   one warp per draft row: row statistics and the chunk holding u * Z
+//                       (chunk partials are the prefix totals), then the draw inside that
+//                       chunk; rows with a top-p cut are finished by their CTA (threshold by
+//                       radix select, draw over the row);
+//   verify_row_kernel   one warp per verifier (and streamed draft) row: statistics (top-p
+//                       threshold by the CTA), then an arrival on the request's counter; the
+//                       warp completing a request runs the accept tests, finds the first
+//                       rejection and writes the draw job;
+//   draw_totals_*       one warp per (draw job, chunk) item over every SM: group and chunk
+//                       totals of the residual (or kept) weights;
+//   draw_pick_kernel    one warp per draw job: the chunk, then the 256-element group holding
+//                       u * Z, and the walk of that group.
+// Cross-CTA handoffs use arrival counters (the last arrival continues); nothing waits.
 #pragma once
 
 #include "common.cuh"
@@ -222,71 +221,110 @@ __device__ __forceinline__ int warp_pick_chunk(const Partial* pp, int nchunks, c
   return sel;
 }
 
-// One warp per draft row: statistics, then the draw inside the chunk that holds u * Z. Rows
-// with a top-p cut are left to sample_topp_kernel.
-template <typename T>
-__global__ void __launch_bounds__(kThreads) sample_finish_kernel(const T* __restrict__ draft, int K, int V, int rows,
-                                                                 const float* __restrict__ temperature,
-                                                                 const float* __restrict__ top_p,
-                                                                 const float* __restrict__ u,
-                                                                 const Partial* __restrict__ parts,
-                                                                 RowStat* __restrict__ stats,
-                                                                 int32_t* __restrict__ out_tokens,
-                                                                 float* __restrict__ out_q) {
+// Residual draw of a job: the chunk holding u * Z of max(0, p - q) (.x totals), or of p (.y
+// totals) when the residual is zero everywhere (*use_p tells which). Same contract as
+// warp_pick_cached.
+__device__ __forceinline__ int warp_pick_resid(const double2* tot, int nchunks, float u, double* base, double* target,
+                                               bool* use_p) {
   const int lane = threadIdx.x & 31;
-  const int row = blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5);
-  if (row >= rows) return;
-  const int b = row / K;
-  const int nch = nchunks_for(V);
-  const T* rp = draft + static_cast<size_t>(row) * V;
-  const Partial* pp = parts + static_cast<size_t>(row) * nch;
-  const float tp = top_p[b];
-  const bool no_cut = !(tp < 1.0f);
-  RowPick rp_ = warp_finalize_pick(pp, nch, temperature[b], u[row], no_cut);
-  const RowStat st = rp_.st;
-  if (lane == 0) stats[row] = st;
-  if (needs_topp(st, tp)) return;
-  if (st.status != 0 || st.c == 0.0f) {
-    if (lane == 0) {
-      out_tokens[row] = st.status != 0 ? -1 : st.amax;
-      if (out_q) out_q[row] = st.status != 0 ? -1.0f : 1.0f;
+  const int q = (nchunks + 31) / 32;
+  const int i0 = min(nchunks, lane * q);
+  if (q <= kCache) {
+    double tx[kCache], ty[kCache], z = 0.0;
+#pragma unroll
+    for (int k = 0; k < kCache; ++k) {
+      const bool ok = k < q && i0 + k < nchunks;
+      tx[k] = ok ? __ldcg(&tot[i0 + k].x) : 0.0;
+      ty[k] = ok ? __ldcg(&tot[i0 + k].y) : 0.0;
+      z += tx[k];
     }
-    return;
+    *use_p = !(warp_sum(z) > 0.0);
+    if (*use_p) {
+#pragma unroll
+      for (int k = 0; k < kCache; ++k) tx[k] = ty[k];
+    }
+    return warp_pick_cached(tx, q, i0, nchunks, u, base, target);
   }
-  JobRows<T, false> J;
-  J.init(rp, st, nullptr, st);
-  int ch = rp_.chunk;
-  double base = rp_.base, target = rp_.target;
-  if ((nch + 31) / 32 > kCache) ch = warp_pick_chunk(pp, nch, st, u[row], &base, &target);
-  const int y = ch < 0 ? -1 : warp_draw_range<T, false, 8>(J, ch * kChunkElems, min(V, (ch + 1) * kChunkElems), base, target);
-  if (lane == 0) {
-    out_tokens[row] = y;
-    if (out_q) out_q[row] = y >= 0 ? kept_weight(st, load_elem(rp + y)) / st.s_kept : -1.0f;
-  }
+  double z = 0.0;
+  for (int i = lane; i < nchunks; i += 32) z += __ldcg(&tot[i].x);
+  *use_p = !(warp_sum(z) > 0.0);
+  return warp_pick_totals(tot, nchunks, *use_p, u, base, target);
 }
 
-// Draft rows with a top-p cut: one CTA per row finds the threshold and draws over the row.
+// Draft rows, kThreads / 32 per CTA. Each warp turns its row's chunk partials into the row
+// statistics, locates the chunk holding u * Z and draws inside it. Rows with a top-p cut are
+// then finished by the whole CTA, one after another: threshold by radix select, then a draw
+// over the row.
 template <typename T>
-__global__ void __launch_bounds__(kThreads) sample_topp_kernel(const T* __restrict__ draft, int K, int V,
-                                                               const float* __restrict__ top_p,
-                                                               const float* __restrict__ u, RowStat* __restrict__ stats,
-                                                               int32_t* __restrict__ out_tokens,
-                                                               float* __restrict__ out_q) {
+__global__ void __launch_bounds__(kThreads, 2) sample_row_kernel(const T* __restrict__ draft, int K, int V, int rows,
+                                                              const float* __restrict__ temperature,
+                                                              const float* __restrict__ top_p,
+                                                              const float* __restrict__ u,
+                                                              const Partial* __restrict__ parts,
+                                                              RowStat* __restrict__ stats,
+                                                              int32_t* __restrict__ out_tokens,
+                                                              float* __restrict__ out_q) {
+  constexpr int kRowsPerCta = kThreads / 32;
   __shared__ ToppSmem tsm;
   __shared__ DrawSmem dsm;
-  const int row = blockIdx.x;
-  const float tp = top_p[row / K];
-  RowStat st = stats[row];
-  if (!needs_topp(st, tp)) return;
-  const T* rp = draft + static_cast<size_t>(row) * V;
-  block_topp_select<T>(rp, V, tp, st, tsm);
-  if (threadIdx.x == 0) stats[row] = st;
-  JobRows<T, false> J;
-  J.init(rp, st, nullptr, st);
-  const int y = block_draw_range(J, 0, V, 0.0, -1.0, u[row], dsm);
-  if (threadIdx.x == 0) {
-    out_tokens[row] = y;
-    if (out_q) out_q[row] = y >= 0 ? kept_weight(st, load_elem(rp + y)) / st.s_kept : -1.0f;
+  __shared__ RowStat cut_st[kRowsPerCta];
+  __shared__ int cut_row[kRowsPerCta];
+  __shared__ int ncut;
+  const int lane = threadIdx.x & 31;
+  const int row = blockIdx.x * kRowsPerCta + (threadIdx.x >> 5);
+  const int nch = nchunks_for(V);
+  if (threadIdx.x == 0) ncut = 0;
+  __syncthreads();
+  if (row < rows) {
+    const int b = row / K;
+    const T* rp = draft + static_cast<size_t>(row) * V;
+    const Partial* pp = parts + static_cast<size_t>(row) * nch;
+    const float tp = top_p[b], ur = u[row];
+    const bool no_cut = !(tp < 1.0f);
+    RowPick r = warp_finalize_pick(pp, nch, temperature[b], ur, no_cut);
+    const RowStat st = r.st;
+    if (needs_topp(st, tp)) {
+      if (lane == 0) {
+        const int k = atomicAdd(&ncut, 1);
+        cut_row[k] = row;
+        cut_st[k] = st;
+      }
+    } else {
+      int y = -1;
+      float q = -1.0f;
+      if (st.status == 0 && st.c == 0.0f) {
+        y = st.amax;
+        q = 1.0f;
+      } else if (st.status == 0) {
+        if ((nch + 31) / 32 > kCache) r.chunk = warp_pick_chunk(pp, nch, st, ur, &r.base, &r.target);
+        JobRows<T, false> J;
+        J.init(rp, st, nullptr, st);
+        float ly = 0.0f;
+        if (r.chunk >= 0)
+          y = warp_draw_chunk(J, r.chunk * kChunkElems, min(V, (r.chunk + 1) * kChunkElems), r.base, r.target, &ly);
+        if (y >= 0) q = kept_weight(st, ly) / st.s_kept;
+      }
+      if (lane == 0) {
+        stats[row] = st;
+        out_tokens[row] = y;
+        if (out_q) out_q[row] = q;
+      }
+    }
+  }
+  __syncthreads();
+  for (int k = 0; k < ncut; ++k) {
+    const int rw = cut_row[k];
+    RowStat st = cut_st[k];
+    const T* rp = draft + static_cast<size_t>(rw) * V;
+    block_topp_select<T>(rp, V, top_p[rw / K], st, tsm);
+    JobRows<T, false> J;
+    J.init(rp, st, nullptr, st);
+    const int y = block_draw_range(J, 0, V, 0.0, -1.0, u[rw], dsm);
+    if (threadIdx.x == 0) {
+      stats[rw] = st;
+      out_tokens[rw] = y;
+      if (out_q) out_q[rw] = y >= 0 ? kept_weight(st, load_elem(rp + y)) / st.s_kept : -1.0f;
+    }
   }
 }
 
@@ -303,7 +341,7 @@ struct VerifyArgs {
   Partial* parts_d;
   RowStat* stats_t;
   RowStat* stats_d;
-  int* cnt;  // one arrival counter per request (top-p requests)
+  int* cnt;  // arrival counters, one per request
   int32_t* out_tokens;
   int32_t* out_len;
   float* out_p;
@@ -311,133 +349,315 @@ struct VerifyArgs {
   Job* jobs;
 };
 
-// Whether request b's rows carry a top-p cut (then verify_topp_kernel finishes it).
-__device__ __forceinline__ bool request_topp(const VerifyArgs& a, int b) {
-  return a.top_p[b] < 1.0f && temp_scale(a.temperature[b]) != 0.0f;
-}
-
-// One CTA per request: statistics of its rows (warps in parallel), then the decision.
+// Verifier rows (then draft rows, when the draft tensor is streamed here), kThreads / 32 per
+// CTA. Each warp turns its row's chunk partials into the row statistics and arrives on the
+// request's counter; the warp completing a request runs its accept tests, finds the first
+// rejection and writes the draw job. Rows with a top-p cut get their threshold from the whole
+// CTA first and arrive after it.
 template <typename T>
-__global__ void __launch_bounds__(1024) verify_finish_kernel(const T* __restrict__ tgt, const T* __restrict__ drf,
-                                                                 VerifyArgs a) {
-  const int b = blockIdx.x;
-  const int K = a.K, nch = nchunks_for(a.V);
-  const int nrows = (K + 1) + (a.stream_draft ? K : 0);
-  const float Tv = a.temperature[b];
-  for (int i = threadIdx.x >> 5; i < nrows; i += blockDim.x >> 5) {
-    const bool is_draft = i > K;
-    const int row = is_draft ? b * K + (i - K - 1) : b * (K + 1) + i;
-    const Partial* pp = (is_draft ? a.parts_d : a.parts_t) + static_cast<size_t>(row) * nch;
-    const RowStat st = warp_finalize_pick(pp, nch, Tv, 0.0f, false).st;
-    if ((threadIdx.x & 31) == 0) (is_draft ? a.stats_d : a.stats_t)[row] = st;
-  }
-  if (request_topp(a, b)) return;
-  __syncthreads();
-  __threadfence_block();
-  if (threadIdx.x < 32)
-    warp_decide_request<T>(b, tgt, drf, K, a.V, a.tokens, a.stats_t, a.stream_draft ? a.stats_d : a.dstats_in, a.u_acc,
-                           a.u_res, a.out_tokens, a.out_len, a.out_p, a.out_q, a.jobs);
-}
-
-// One CTA per row of a top-p request: the threshold; the CTA that completes the request
-// decides it.
-template <typename T>
-__global__ void __launch_bounds__(kThreads) verify_topp_kernel(const T* __restrict__ tgt, const T* __restrict__ drf,
-                                                               VerifyArgs a) {
+__global__ void __launch_bounds__(kThreads) verify_row_kernel(const T* __restrict__ tgt, const T* __restrict__ drf,
+                                                              VerifyArgs a) {
+  constexpr int kRowsPerCta = kThreads / 32;
   __shared__ ToppSmem tsm;
-  __shared__ int sh_flag;
+  __shared__ RowStat cut_st[kRowsPerCta];
+  __shared__ int cut_row[kRowsPerCta];
+  __shared__ int ncut, sh_flag;
   const int K = a.K, V = a.V;
-  const int rows_t = a.B * (K + 1);
-  const bool is_draft = static_cast<int>(blockIdx.x) >= rows_t;
-  const int row = is_draft ? static_cast<int>(blockIdx.x) - rows_t : static_cast<int>(blockIdx.x);
-  const int b = is_draft ? row / K : row / (K + 1);
-  if (!request_topp(a, b)) return;
-  const float tp = a.top_p[b];
-  RowStat* sp = (is_draft ? a.stats_d : a.stats_t) + row;
-  RowStat st = *sp;
-  if (needs_topp(st, tp)) {
-    block_topp_select<T>((is_draft ? drf : tgt) + static_cast<size_t>(row) * V, V, tp, st, tsm);
-    if (threadIdx.x == 0) *sp = st;
+  const int rows_t = a.B * (K + 1), rows = rows_t + (a.stream_draft ? a.B * K : 0);
+  const int per_req = (K + 1) + (a.stream_draft ? K : 0);
+  const int nch = nchunks_for(V);
+  const int g = blockIdx.x * kRowsPerCta + (threadIdx.x >> 5);  // 0 .. rows - 1: verifier rows, then draft rows
+  auto request_of = [&](int gr) { return gr < rows_t ? gr / (K + 1) : (gr - rows_t) / K; };
+  auto stat_of = [&](int gr) -> RowStat* { return gr < rows_t ? a.stats_t + gr : a.stats_d + (gr - rows_t); };
+  if (threadIdx.x == 0) ncut = 0;
+  __syncthreads();
+  if (g < rows) {
+    const int b = request_of(g);
+    const Partial* pp = g < rows_t ? a.parts_t + static_cast<size_t>(g) * nch
+                                   : a.parts_d + static_cast<size_t>(g - rows_t) * nch;
+    const RowStat st = warp_finalize_pick(pp, nch, a.temperature[b], 0.0f, false).st;
+    if (needs_topp(st, a.top_p[b])) {
+      if ((threadIdx.x & 31) == 0) {
+        const int k = atomicAdd(&ncut, 1);
+        cut_row[k] = g;
+        cut_st[k] = st;
+      }
+    } else {
+      if ((threadIdx.x & 31) == 0) *stat_of(g) = st;
+      if (warp_arrive_last(&a.cnt[b], per_req))
+        warp_decide_request<T>(b, tgt, drf, K, V, a.tokens, a.stats_t, a.stream_draft ? a.stats_d : a.dstats_in,
+                               a.u_acc, a.u_res, a.out_tokens, a.out_len, a.out_p, a.out_q, a.jobs);
+    }
   }
-  if (!block_arrive_last(&a.cnt[b], (K + 1) + (a.stream_draft ? K : 0), &sh_flag)) return;
-  if (threadIdx.x < 32)
-    warp_decide_request<T>(b, tgt, drf, K, V, a.tokens, a.stats_t, a.stream_draft ? a.stats_d : a.dstats_in, a.u_acc,
-                           a.u_res, a.out_tokens, a.out_len, a.out_p, a.out_q, a.jobs);
+  __syncthreads();
+  for (int k = 0; k < ncut; ++k) {
+    const int gr = cut_row[k], b = request_of(gr);
+    RowStat st = cut_st[k];
+    const T* rp = gr < rows_t ? tgt + static_cast<size_t>(gr) * V : drf + static_cast<size_t>(gr - rows_t) * V;
+    block_topp_select<T>(rp, V, a.top_p[b], st, tsm);
+    if (threadIdx.x == 0) *stat_of(gr) = st;
+    if (block_arrive_last(&a.cnt[b], per_req, &sh_flag) && threadIdx.x < 32)
+      warp_decide_request<T>(b, tgt, drf, K, V, a.tokens, a.stats_t, a.stream_draft ? a.stats_d : a.dstats_in,
+                             a.u_acc, a.u_res, a.out_tokens, a.out_len, a.out_p, a.out_q, a.jobs);
+    __syncthreads();
+  }
 }
 
-// Draw jobs (a residual draw at the first rejection, or the bonus draw from a row with a
-// top-p cut) need per-chunk totals of their weights: draw_totals_kernel spreads the
-// (job, chunk) items over every SM with persistent warps (two exponentials per element pair
-// make this pass compute-heavy, so it must not sit on a few SMs). draw_pick_kernel then
-// uses one warp per job: it finds the chunk that holds u * Z (from those totals, or from the
-// row's own partials for a bonus draw without a cut) and walks it.
+// Draw jobs (the residual draw at a first rejection, or the bonus draw after a fully
+// accepted block) take two launches. The totals pass spreads (job, chunk) items over every
+// SM: each warp reduces one chunk of the job's weights (.x the residual max(0, p - q) or the
+// kept distribution, .y p) to its eight 256-element group totals and the chunk total. The
+// pick pass gives each job a warp that locates the chunk holding u * Z, then the group
+// inside it, and walks that group. A bonus draw without a top-p cut needs no totals: its
+// chunk comes from the row's own partials and is walked whole.
+
+// Whether a job's draw needs the totals pass.
+__device__ __forceinline__ bool job_needs_totals(int32_t mode, uint32_t tau_a) {
+  return mode == kResidual || (mode == kSample && tau_a != 0u);
+}
+
+// Per-lane group sums of one chunk held in shared memory (sa: row a, sb: row b; n elements).
+template <typename T, bool RESID>
+__device__ __forceinline__ void smem_chunk_sums(const JobRows<T, RESID>& J, const T* sa, const T* sb, int n,
+                                                double (&sx)[kChunkGroups], double (&sy)[kChunkGroups]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int g = 0; g < kChunkGroups; ++g) {
+    const int e = g * kGroup + lane * 8;
+    Raw8<T, RESID> x;
+    if (e + 8 <= n) {
+      x.a.w[0] = *reinterpret_cast<const uint4*>(sa + e);
+      if constexpr (sizeof(T) == 4) x.a.w[1] = *reinterpret_cast<const uint4*>(sa + e + 4);
+      if constexpr (RESID) {
+        x.b[0].w[0] = *reinterpret_cast<const uint4*>(sb + e);
+        if constexpr (sizeof(T) == 4) x.b[0].w[1] = *reinterpret_cast<const uint4*>(sb + e + 4);
+      }
+    } else {
+      float fa[8], fb[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        fa[k] = e + k < n ? load_elem_any(sa + e + k) : -INFINITY;
+        fb[k] = (RESID && e + k < n) ? load_elem_any(sb + e + k) : -INFINITY;
+      }
+      x.a.pack(fa);
+      if constexpr (RESID) x.b[0].pack(fb);
+    }
+    const double2 t = lane_group_sums(J, x);
+    sx[g] = t.x;
+    sy[g] = t.y;
+  }
+}
+
+// Totals pass through a per-warp ring of bulk copies (rows 16-byte aligned, row bytes a
+// multiple of 16): lane 0 keeps the next item's copies in flight, with the job record staged
+// in shared memory for the warp, while the warp reduces the current item.
+constexpr int kDrawRing = 2;
+constexpr int kDrawWarps = 4;  // warps per CTA of the bulk-copy totals pass
 template <typename T>
-__global__ void __launch_bounds__(kThreads) draw_totals_kernel(const T* __restrict__ A, const T* __restrict__ Bt,
-                                                               int V, int njobs, const RowStat* __restrict__ sa,
-                                                               const RowStat* __restrict__ sb,
-                                                               const Job* __restrict__ jobs,
-                                                               double2* __restrict__ tot) {
+constexpr int kDrawStageBytes = 2 * kChunkElems * static_cast<int>(sizeof(T));  // rows a and b
+
+template <typename T>
+__global__ void __launch_bounds__(kDrawWarps * 32) draw_totals_tma_kernel(const T* __restrict__ A, const T* __restrict__ Bt,
+                                                                  int V, int njobs, const Job* __restrict__ jobs,
+                                                                  double2* __restrict__ tot_c,
+                                                                  double2* __restrict__ tot_g) {
+  extern __shared__ __align__(128) unsigned char dring_smem[];
+  __shared__ uint64_t bars[kDrawWarps][kDrawRing];
+  __shared__ Job sjob[kDrawWarps][kDrawRing];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  unsigned char* ring = dring_smem + warp * kDrawRing * kDrawStageBytes<T>;
+  uint64_t* bar = bars[warp];
+  const int nch = nchunks_for(V);
+  const int64_t items = static_cast<int64_t>(njobs) * nch;
+  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * kDrawWarps;
+  const int64_t g0 = static_cast<int64_t>(blockIdx.x) * kDrawWarps + warp;
+  if (g0 >= items) return;
+  if (lane == 0) {
+    for (int s = 0; s < kDrawRing; ++s) mbar_init(&bar[s], 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncwarp();
+  const int djob = static_cast<int>(nwarps / nch), dchunk = static_cast<int>(nwarps - static_cast<int64_t>(djob) * nch);
+  int ijob = static_cast<int>(g0 / nch), ichunk = static_cast<int>(g0 - static_cast<int64_t>(ijob) * nch);
+  int64_t gi = g0;
+  // lane 0: stage the job record of this warp's i-th item and start its copies
+  auto issue = [&](int i) {
+    if (gi < items) {
+      const int st = i % kDrawRing;
+      const Job jb = load_job_cg(jobs + ijob);
+      sjob[warp][st] = jb;
+      if (job_needs_totals(jb.mode, jb.sa.tau)) {
+        const int c0 = ichunk * kChunkElems, n = min(V - c0, kChunkElems);
+        const uint32_t bytes = static_cast<uint32_t>(n) * sizeof(T);
+        const bool resid = jb.mode == kResidual;
+        unsigned char* dst = ring + st * kDrawStageBytes<T>;
+        mbar_expect_tx(&bar[st], resid ? 2 * bytes : bytes);
+        bulk_g2s(dst, A + static_cast<size_t>(jb.row_a) * V + c0, bytes, &bar[st]);
+        if (resid) bulk_g2s(dst + kChunkElems * sizeof(T), Bt + static_cast<size_t>(jb.row_b) * V + c0, bytes, &bar[st]);
+      }
+    }
+    gi += nwarps;
+    ijob += djob;
+    ichunk += dchunk;
+    if (ichunk >= nch) {
+      ichunk -= nch;
+      ++ijob;
+    }
+  };
+  if (lane == 0)
+    for (int i = 0; i < kDrawRing - 1; ++i) issue(i);
+  int jid = static_cast<int>(g0 / nch), chunk = static_cast<int>(g0 - static_cast<int64_t>(jid) * nch);
+  uint32_t phase_bits = 0u;  // parity of the next wait, per stage
+  int i = 0;
+  for (int64_t g = g0; g < items; g += nwarps, ++i) {
+    __syncwarp();  // every lane is done with the stage that the next copy overwrites
+    if (lane == 0) issue(i + kDrawRing - 1);
+    __syncwarp();
+    const int st = i % kDrawRing;
+    const Job& jb = sjob[warp][st];
+    const int32_t mode = jb.mode;
+    if (job_needs_totals(mode, jb.sa.tau)) {
+      const bool landed = mbar_wait_bounded(&bar[st], (phase_bits >> st) & 1u);
+      phase_bits ^= 1u << st;
+      double2* tc = tot_c + static_cast<size_t>(jid) * nch + chunk;
+      double2* tg = tot_g + (static_cast<size_t>(jid) * nch + chunk) * kChunkGroups;
+      if (!__all_sync(0xffffffffu, landed)) {
+        // a copy that never completed: poison the job's totals (its draw reports -1) and stop
+        if (lane == 0) *tc = make_double2(NAN, NAN);
+        return;
+      }
+      const int c0 = chunk * kChunkElems, n = min(V - c0, kChunkElems);
+      const T* sa = reinterpret_cast<const T*>(ring + st * kDrawStageBytes<T>);
+      const T* sb = sa + kChunkElems;
+      double sx[kChunkGroups], sy[kChunkGroups];
+      if (mode == kResidual) {
+        JobRows<T, true> J;
+        J.init(nullptr, jb.sa, nullptr, jb.sb);
+        smem_chunk_sums(J, sa, sb, n, sx, sy);
+      } else {
+        JobRows<T, false> J;
+        J.init(nullptr, jb.sa, nullptr, jb.sa);
+        smem_chunk_sums(J, sa, sa, n, sx, sy);
+      }
+      (void)c0;
+      emit_chunk_totals(sx, sy, tc, tg);
+    }
+    chunk += dchunk;
+    jid += djob;
+    if (chunk >= nch) {
+      chunk -= nch;
+      ++jid;
+    }
+  }
+}
+
+// Totals pass with plain vector loads (any alignment), one warp per (job, chunk) item.
+template <typename T>
+__global__ void __launch_bounds__(kThreads) draw_totals_kernel(const T* __restrict__ A, const T* __restrict__ Bt, int V,
+                                                              int njobs, const Job* __restrict__ jobs,
+                                                              double2* __restrict__ tot_c,
+                                                              double2* __restrict__ tot_g) {
   const int lane = threadIdx.x & 31;
   const int nch = nchunks_for(V);
   const int64_t items = static_cast<int64_t>(njobs) * nch;
-  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (kThreads / 32);
-  for (int64_t g = static_cast<int64_t>(blockIdx.x) * (kThreads / 32) + (threadIdx.x >> 5); g < items; g += nwarps) {
-    const int jid = static_cast<int>(g / nch), chunk = static_cast<int>(g - static_cast<int64_t>(jid) * nch);
-    const Job jb = jobs[jid];
-    if (jb.mode < kSample) continue;
-    const RowStat st_a = sa[jb.row_a];
-    if (jb.mode == kSample && st_a.tau == 0u) continue;  // totals are the row's partials
-    const T* ra = A + static_cast<size_t>(jb.row_a) * V;
+  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  for (int64_t it = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); it < items;
+       it += nwarps) {
+    const int jid = static_cast<int>(it / nch), chunk = static_cast<int>(it - static_cast<int64_t>(jid) * nch);
+    const Job jb = load_job_cg(jobs + jid);
+    if (!job_needs_totals(jb.mode, jb.sa.tau)) continue;
     const int c0 = chunk * kChunkElems, c1 = min(V, c0 + kChunkElems);
-    int last;
-    double2 t;
-    if (jb.mode == kSample) {
-      JobRows<T, false> J;
-      J.init(ra, st_a, nullptr, st_a);
-      t = warp_range_totals(J, c0, c1, &last);
-    } else {
+    double sx[kChunkGroups], sy[kChunkGroups];
+    if (jb.mode == kResidual) {
       JobRows<T, true> J;
-      J.init(ra, st_a, Bt + static_cast<size_t>(jb.row_b) * V, sb[jb.row_b]);
-      t = warp_range_totals(J, c0, c1, &last);
+      J.init(A + static_cast<size_t>(jb.row_a) * V, jb.sa, Bt + static_cast<size_t>(jb.row_b) * V, jb.sb);
+#pragma unroll
+      for (int g = 0; g < kChunkGroups; ++g) {
+        Raw8<T, true> x;
+        J.load(c0 + g * kGroup + lane * 8, c1, x);
+        const double2 t = lane_group_sums(J, x);
+        sx[g] = t.x;
+        sy[g] = t.y;
+      }
+    } else {
+      JobRows<T, false> J;
+      J.init(A + static_cast<size_t>(jb.row_a) * V, jb.sa, nullptr, jb.sa);
+#pragma unroll
+      for (int g = 0; g < kChunkGroups; ++g) {
+        Raw8<T, false> x;
+        J.load(c0 + g * kGroup + lane * 8, c1, x);
+        const double2 t = lane_group_sums(J, x);
+        sx[g] = t.x;
+        sy[g] = t.y;
+      }
     }
-    if (lane == 0) tot[g] = t;
+    emit_chunk_totals(sx, sy, tot_c + static_cast<size_t>(jid) * nch + chunk,
+                      tot_g + (static_cast<size_t>(jid) * nch + chunk) * kChunkGroups);
   }
 }
 
+// Pick pass: one warp per job.
 template <typename T>
-__global__ void __launch_bounds__(32) draw_pick_kernel(const T* __restrict__ A, const T* __restrict__ Bt, int V,
-                                                             int njobs, const RowStat* __restrict__ sa,
-                                                             const RowStat* __restrict__ sb,
-                                                             const Partial* __restrict__ parts_a,
-                                                             const Job* __restrict__ jobs,
-                                                             const double2* __restrict__ tot,
-                                                             int32_t* __restrict__ out_tokens) {
+__global__ void __launch_bounds__(kThreads, 1) draw_pick_kernel(const T* __restrict__ A, const T* __restrict__ Bt, int V,
+                                                            int njobs, const Partial* __restrict__ parts_a,
+                                                            const Job* __restrict__ jobs,
+                                                            const double2* __restrict__ tot_c,
+                                                            const double2* __restrict__ tot_g,
+                                                            int32_t* __restrict__ out_tokens) {
   const int lane = threadIdx.x & 31;
-  const int jid = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);  // one warp per job
+  const int jid = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (jid >= njobs) return;
-  const Job jb = jobs[jid];
+  const Job jb = load_job_cg(jobs + jid);
   if (jb.mode < kSample) return;
   const int nch = nchunks_for(V);
-  const RowStat st_a = sa[jb.row_a];
   const T* ra = A + static_cast<size_t>(jb.row_a) * V;
-  const double2* jt = tot + static_cast<size_t>(jid) * nch;
-  double base, target;
-  int y;
-  if (jb.mode == kSample) {
+  const T* rb = Bt + static_cast<size_t>(jb.row_b) * V;
+  float ly;
+  int y = -1;
+  if (!job_needs_totals(jb.mode, jb.sa.tau)) {  // bonus draw without a cut: the row's partials
+    double base, target;
+    const int ch = warp_pick_chunk(parts_a + static_cast<size_t>(jb.row_a) * nch, nch, jb.sa, jb.u, &base, &target);
     JobRows<T, false> J;
-    J.init(ra, st_a, nullptr, st_a);
-    const int ch = st_a.tau == 0u ? warp_pick_chunk(parts_a + static_cast<size_t>(jb.row_a) * nch, nch, st_a, jb.u, &base, &target)
-                                  : warp_pick_totals(jt, nch, false, jb.u, &base, &target);
-    y = ch < 0 ? -1 : warp_draw_range<T, false, 8>(J, ch * kChunkElems, min(V, (ch + 1) * kChunkElems), base, target);
+    J.init(ra, jb.sa, nullptr, jb.sa);
+    if (ch >= 0) y = warp_draw_chunk(J, ch * kChunkElems, min(V, (ch + 1) * kChunkElems), base, target, &ly);
   } else {
-    JobRows<T, true> J;
-    J.init(ra, st_a, Bt + static_cast<size_t>(jb.row_b) * V, sb[jb.row_b]);
-    double z = 0.0;
-#pragma unroll 4
-    for (int i = lane; i < nch; i += 32) z += __ldcg(&jt[i].x);
-    J.use_p = !(warp_sum(z) > 0.0);  // zero residual: draw from p instead
-    const int ch = warp_pick_totals(jt, nch, J.use_p, jb.u, &base, &target);
-    y = ch < 0 ? -1 : warp_draw_range<T, true, 8>(J, ch * kChunkElems, min(V, (ch + 1) * kChunkElems), base, target);
+    const double2* jc = tot_c + static_cast<size_t>(jid) * nch;
+    double base = 0.0, target = 0.0;
+    bool use_p = false;
+    const int ch = jb.mode == kSample ? warp_pick_totals(jc, nch, false, jb.u, &base, &target)
+                                      : warp_pick_resid(jc, nch, jb.u, &base, &target, &use_p);
+    if (ch >= 0) {
+      // the group of the chunk holding target: lanes 0..7 hold the group totals
+      const double2* jg = tot_g + (static_cast<size_t>(jid) * nch + ch) * kChunkGroups;
+      const double t = lane < kChunkGroups ? (use_p ? __ldcg(&jg[lane].y) : __ldcg(&jg[lane].x)) : 0.0;
+      double incl = t;
+#pragma unroll
+      for (int o = 1; o < kChunkGroups; o <<= 1) {
+        const double v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      double excl = __shfl_up_sync(0xffffffffu, incl, 1);
+      if (lane == 0) excl = 0.0;
+      const bool in = lane < kChunkGroups && t > 0.0;
+      const unsigned hit = __ballot_sync(0xffffffffu, in && base + incl > target);
+      const unsigned pos = __ballot_sync(0xffffffffu, in);
+      if (pos) {
+        // rounding can leave no group crossing: the chunk's last positive group then
+        const int G = hit ? __ffs(hit) - 1 : 31 - __clz(pos);
+        const double gb = base + __shfl_sync(0xffffffffu, excl, G);
+        const int c1 = min(V, (ch + 1) * kChunkElems);
+        if (jb.mode == kSample) {
+          JobRows<T, false> J;
+          J.init(ra, jb.sa, nullptr, jb.sa);
+          y = warp_draw_group(J, ch * kChunkElems + G * kGroup, c1, gb, target, &ly);
+        } else {
+          JobRows<T, true> J;
+          J.init(ra, jb.sa, rb, jb.sb);
+          J.use_p = use_p;
+          y = warp_draw_group(J, ch * kChunkElems + G * kGroup, c1, gb, target, &ly);
+        }
+      }
+    }
   }
   if (lane == 0) out_tokens[jb.out_index] = y;
 }

@@ -28,22 +28,6 @@ __device__ __forceinline__ bool accept_test(float u, const RowStat& sp, float lp
   return u < ratio;
 }
 
-// a row-statistics record written by another CTA of the running kernel (read through L2)
-__device__ __forceinline__ RowStat load_stat_cg(const RowStat* p) {
-  const int4* q = reinterpret_cast<const int4*>(p);
-  const int4 a = __ldcg(q), b = __ldcg(q + 1);
-  RowStat s;
-  s.m = __int_as_float(a.x);
-  s.c = __int_as_float(a.y);
-  s.s = __int_as_float(a.z);
-  s.s_kept = __int_as_float(a.w);
-  s.tau = static_cast<uint32_t>(b.x);
-  s.amax = b.y;
-  s.status = b.z;
-  s.pad = b.w;
-  return s;
-}
-
 // Called by one full warp for request b. ts: verifier rows [B*(K+1)], ds: draft rows [B*K].
 template <typename T>
 __device__ void warp_decide_request(int b, const T* __restrict__ tgt, const T* __restrict__ drf, int K, int V,
@@ -57,12 +41,15 @@ __device__ void warp_decide_request(int b, const T* __restrict__ tgt, const T* _
   uint32_t rej_lo = 0u, rej_hi = 0u;
   int x_mine[3] = {-1, -1, -1};
   float p_mine[2] = {-1.0f, -1.0f}, q_mine[2] = {-1.0f, -1.0f};
+  RowStat sq_mine[2];
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     const int i = lane + 32 * h;
-    if (i >= K) break;
+    sq_mine[h] = RowStat{0.0f, 0.0f, 1.0f, 1.0f, 0u, -1, 1, 0};
+    if (i >= K) continue;
     const int x = tokens[drow0 + i];
     const RowStat sp = load_stat_cg(ts + trow0 + i), sq = load_stat_cg(ds + drow0 + i);
+    sq_mine[h] = sq;
     const bool rowbad = sp.status != 0 || sq.status != 0 || x < 0 || x >= V;
     bool acc = false;
     if (!rowbad) {
@@ -82,6 +69,8 @@ __device__ void warp_decide_request(int b, const T* __restrict__ tgt, const T* _
   rej_hi = __reduce_or_sync(0xffffffffu, rej_hi);
   const int j = rej_lo ? __ffs(rej_lo) - 1 : (rej_hi ? 32 + __ffs(rej_hi) - 1 : K);
   const RowStat sj = load_stat_cg(ts + trow0 + j);  // verifier row of the draw (row K for the bonus)
+  // draft row of a residual draw (held by lane j % 32 of half j / 32)
+  const RowStat sqj = shfl_stat(j >= 32 ? sq_mine[1] : sq_mine[0], j & 31);
 
 #pragma unroll
   for (int h = 0; h < 3; ++h) {  // K + 1 <= 65 token slots
@@ -101,9 +90,15 @@ __device__ void warp_decide_request(int b, const T* __restrict__ tgt, const T* _
   }
   if (lane == 0) {
     out_len[b] = bad ? -1 : j;
-    Job jb{kNone, static_cast<int32_t>(trow0 + j), static_cast<int32_t>(drow0 + j), static_cast<int32_t>(trow0 + j),
-           u_res[trow0 + j], -1, {0, 0}};
-    if (!bad && sj.c != 0.0f) jb.mode = j < K ? kResidual : kSample;
+    Job jb;
+    jb.mode = (!bad && sj.c != 0.0f) ? (j < K ? kResidual : kSample) : kNone;
+    jb.row_a = static_cast<int32_t>(trow0 + j);
+    jb.row_b = static_cast<int32_t>(drow0 + j);
+    jb.out_index = static_cast<int32_t>(trow0 + j);
+    jb.u = u_res[trow0 + j];
+    jb.pad[0] = jb.pad[1] = jb.pad[2] = 0;
+    jb.sa = sj;
+    jb.sb = sqj;
     jobs[b] = jb;
   }
 }

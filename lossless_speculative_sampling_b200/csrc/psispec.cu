@@ -53,8 +53,9 @@ SampleWs carve_sample(Carver& c, int64_t rows, int64_t V) {
 struct LinearWs {
   StatsWs t, d;
   Job* jobs;
-  int32_t* cnt;      // arrival counters: one per request (top-p), one per draw job
-  double2* draw_tot;  // per (draw job, chunk) weight totals
+  int32_t* cnt;      // arrival counters, one per request
+  double2* draw_tc;   // per (draw job, chunk) weight totals
+  double2* draw_tg;   // per (draw job, chunk, group) weight totals
 };
 LinearWs carve_linear(Carver& c, int64_t B, int64_t K, int64_t V) {
   const int ns = nchunks_for(V);
@@ -62,8 +63,9 @@ LinearWs carve_linear(Carver& c, int64_t B, int64_t K, int64_t V) {
   w.t = carve_stats(c, B * (K + 1), ns);
   w.d = carve_stats(c, B * K, ns);
   w.jobs = c.take<Job>(B);
-  w.cnt = c.take<int32_t>(2 * B);
-  w.draw_tot = c.take<double2>(B * ns);
+  w.cnt = c.take<int32_t>(B);
+  w.draw_tc = c.take<double2>(B * ns);
+  w.draw_tg = c.take<double2>(B * ns * kChunkGroups);
   return w;
 }
 
@@ -148,6 +150,39 @@ psispec_status launch_stats(const T* base, int64_t rows, int rows_per_req, const
   return launched();
 }
 
+// The draw jobs of a verification call: totals pass (bulk-copy ring when the rows allow it),
+// then the pick pass.
+template <typename T>
+psispec_status launch_draws(const T* A, const T* Bt, int V, int njobs, const Partial* parts_a, const Job* jobs,
+                            double2* tc, double2* tg, int32_t* out_tokens, cudaStream_t st) {
+  const int64_t items = int64_t(njobs) * nchunks_for(V);
+  // the bulk-copy ring serves bf16 rows (fp32 stages would not fit enough warps per SM)
+  const bool ring = sizeof(T) == 2 && (reinterpret_cast<uintptr_t>(A) & 15u) == 0 &&
+                    (reinterpret_cast<uintptr_t>(Bt) & 15u) == 0 && (int64_t(V) * sizeof(T)) % 16 == 0;
+  if (ring) {
+    const int smem = kDrawWarps * kDrawRing * kDrawStageBytes<T>;
+    if (cudaFuncSetAttribute(draw_totals_tma_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+        cudaSuccess)
+      return PSISPEC_ERR_CUDA;
+    int dev = 0, sms = 148, occ = 1;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, draw_totals_tma_kernel<T>, kDrawWarps * 32, smem);
+    const int64_t want = (items + kDrawWarps - 1) / kDrawWarps;
+    const int64_t slots = static_cast<int64_t>(sms) * (occ > 0 ? occ : 1);
+    draw_totals_tma_kernel<T><<<static_cast<unsigned>(want < slots ? want : slots), kDrawWarps * 32, smem, st>>>(
+        A, Bt, V, njobs, jobs, tc, tg);
+  } else {
+    draw_totals_kernel<T><<<persistent_grid(draw_totals_kernel<T>, items), kThreads, 0, st>>>(A, Bt, V, njobs, jobs,
+                                                                                            tc, tg);
+  }
+  psispec_status s = launched();
+  if (s != PSISPEC_OK) return s;
+  draw_pick_kernel<T><<<static_cast<unsigned>((njobs + kThreads / 32 - 1) / (kThreads / 32)), kThreads, 0, st>>>(
+      A, Bt, V, njobs, parts_a, jobs, tc, tg, out_tokens);
+  return launched();
+}
+
 template <typename T>
 psispec_status sample_draft_impl(const T* draft, int B, int K, int V, const float* temperature, const float* top_p,
                                  const float* u, int32_t* out_tokens, float* out_q, RowStat* out_stats, void* ws,
@@ -158,11 +193,8 @@ psispec_status sample_draft_impl(const T* draft, int B, int K, int V, const floa
   RowStat* stats = out_stats ? out_stats : w.st.stats;
   psispec_status s = launch_stream<T>(draft, rows, K, nullptr, V, temperature, B, w.st.parts, st);
   if (s != PSISPEC_OK) return s;
-  sample_finish_kernel<T><<<static_cast<unsigned>((rows + 7) / 8), kThreads, 0, st>>>(
+  sample_row_kernel<T><<<static_cast<unsigned>((rows + kThreads / 32 - 1) / (kThreads / 32)), kThreads, 0, st>>>(
       draft, K, V, static_cast<int>(rows), temperature, top_p, u, w.st.parts, stats, out_tokens, out_q);
-  if ((s = launched()) != PSISPEC_OK) return s;
-  sample_topp_kernel<T><<<static_cast<unsigned>(rows), kThreads, 0, st>>>(draft, K, V, top_p, u, stats, out_tokens,
-                                                                          out_q);
   return launched();
 }
 
@@ -174,7 +206,7 @@ psispec_status verify_linear_impl(const T* tgt, const T* drf, int B, int K, int 
   Carver c(ws);
   LinearWs w = carve_linear(c, B, K, V);
   const int64_t rows_t = int64_t(B) * (K + 1), rows_d = draft_stats ? 0 : int64_t(B) * K;
-  if (cudaMemsetAsync(w.cnt, 0, sizeof(int32_t) * 2 * B, st) != cudaSuccess) return PSISPEC_ERR_CUDA;
+  if (cudaMemsetAsync(w.cnt, 0, sizeof(int32_t) * B, st) != cudaSuccess) return PSISPEC_ERR_CUDA;
   VerifyArgs a;
   a.B = B;
   a.K = K;
@@ -200,19 +232,10 @@ psispec_status verify_linear_impl(const T* tgt, const T* drf, int B, int K, int 
   if (s != PSISPEC_OK) return s;
   if (rows_d > 0 && (s = launch_stream<T>(drf, rows_d, K, nullptr, V, temperature, B, w.d.parts, st)) != PSISPEC_OK)
     return s;
-  const int finish_warps = static_cast<int>(std::min<int64_t>(32, (K + 1) + (rows_d ? K : 0)));
-  verify_finish_kernel<T><<<static_cast<unsigned>(B), 32 * finish_warps, 0, st>>>(tgt, drf, a);
+  verify_row_kernel<T><<<static_cast<unsigned>((rows_t + rows_d + kThreads / 32 - 1) / (kThreads / 32)), kThreads, 0,
+                         st>>>(tgt, drf, a);
   if ((s = launched()) != PSISPEC_OK) return s;
-  verify_topp_kernel<T><<<static_cast<unsigned>(rows_t + rows_d), kThreads, 0, st>>>(tgt, drf, a);
-  if ((s = launched()) != PSISPEC_OK) return s;
-  const RowStat* ds = draft_stats ? draft_stats : w.d.stats;
-  const int64_t items = int64_t(B) * nchunks_for(V);
-  draw_totals_kernel<T><<<persistent_grid(draw_totals_kernel<T>, items), kThreads, 0, st>>>(tgt, drf, V, B, w.t.stats,
-                                                                                          ds, w.jobs, w.draw_tot);
-  if ((s = launched()) != PSISPEC_OK) return s;
-  draw_pick_kernel<T><<<static_cast<unsigned>(B), 32, 0, st>>>(tgt, drf, V, B, w.t.stats, ds, w.t.parts, w.jobs,
-                                                                 w.draw_tot, out_tokens);
-  return launched();
+  return launch_draws<T>(tgt, drf, V, B, w.t.parts, w.jobs, w.draw_tc, w.draw_tg, out_tokens, st);
 }
 
 template <typename T>

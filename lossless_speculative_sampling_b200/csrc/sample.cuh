@@ -61,6 +61,11 @@ struct Raw8x {
       pack(x);
     }
   }
+  // 8 elements known to be in range, from a 16-byte aligned address
+  __device__ __forceinline__ void load_full(const T* __restrict__ row, int e) {
+    w[0] = __ldg(reinterpret_cast<const uint4*>(row + e));
+    if constexpr (sizeof(T) == 4) w[1] = __ldg(reinterpret_cast<const uint4*>(row + e + 4));
+  }
   __device__ __forceinline__ void pack(const float (&x)[8]) {
     if constexpr (sizeof(T) == 2) {  // every value here is an exact bf16 (or -inf)
       w[0] = make_uint4((__float_as_uint(x[0]) >> 16) | (__float_as_uint(x[1]) & 0xFFFF0000u),
@@ -114,6 +119,15 @@ struct JobRows {
     r.b = sb;
     r.ib = RESID ? 1.0f / sb.s_kept : 0.0f;
     al_b = RESID && (reinterpret_cast<uintptr_t>(rowb) & 15u) == 0;
+  }
+  __device__ __forceinline__ float logit_a(int v) const { return load_elem(ra + v); }
+  // whether [lo, lo + n) can be read with unconditional aligned vector loads
+  __device__ __forceinline__ bool vector_ok(int lo, int hi, int n) const {
+    return hi - lo == n && al_a && (!RESID || al_b);
+  }
+  __device__ __forceinline__ void load_full(int e, Raw8<T, RESID>& x) const {
+    x.a.load_full(ra, e);
+    if constexpr (RESID) x.b[0].load_full(rb, e);
   }
   __device__ __forceinline__ void load(int e, int end, Raw8<T, RESID>& x) const {
     x.a.load(ra, e, end, al_a);
@@ -178,6 +192,178 @@ __device__ double2 warp_range_totals(const JobRows<T, RESID>& J, int lo, int hi,
   }
   *last_pos = __reduce_max_sync(0xffffffffu, last);
   return make_double2(warp_sum(sr), warp_sum(sp));
+}
+
+// Groups of one chunk, and how many of them warp_chunk_totals and warp_draw_chunk keep in
+// flight at once (the whole chunk, except for residual fp32 rows: half of it).
+constexpr int kChunkGroups = kChunkElems / kGroup;
+template <typename T, bool RESID>
+constexpr int kChunkBatch = (sizeof(T) == 4 && RESID) ? kChunkGroups / 2 : kChunkGroups;
+
+// This lane's fp64 weight in one loaded group (8 elements), and its last positive index.
+template <typename T, bool RESID>
+__device__ __forceinline__ double lane_group_weight(const JobRows<T, RESID>& J, const Raw8<T, RESID>& x, int e,
+                                                    int* last) {
+  float w[8], pw[8];
+  J.weights(x, w, pw);
+  double v = 0.0;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    v += static_cast<double>(w[k]);
+    if (w[k] > 0.0f) *last = e + k;
+  }
+  return v;
+}
+
+// This lane's fp64 sums of the job weights (.x) and of p_a (.y) over one loaded group.
+template <typename T, bool RESID>
+__device__ __forceinline__ double2 lane_group_sums(const JobRows<T, RESID>& J, const Raw8<T, RESID>& x) {
+  float w[8], pw[8];
+  J.weights(x, w, pw);
+  double a = 0.0, b = 0.0;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    a += static_cast<double>(w[k]);
+    b += static_cast<double>(pw[k]);
+  }
+  return make_double2(a, b);
+}
+
+// Reduce-scatter of eight per-lane values: lane l ends with the warp total of value
+// (l >> 2) & 7 (halves exchanged over lane bits 4, 3, 2, then summed over bits 1, 0).
+__device__ __forceinline__ double warp_reduce_scatter8(const double (&v)[8]) {
+  const int lane = threadIdx.x & 31;
+  const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4;
+  double h[4], q[2];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const double send = b4 ? v[k] : v[k + 4], keep = b4 ? v[k + 4] : v[k];
+    h[k] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+  }
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const double send = b3 ? h[k] : h[k + 2], keep = b3 ? h[k + 2] : h[k];
+    q[k] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+  }
+  const double send = b2 ? q[0] : q[1], keep = b2 ? q[1] : q[0];
+  double r = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+  r += __shfl_xor_sync(0xffffffffu, r, 2);
+  r += __shfl_xor_sync(0xffffffffu, r, 1);
+  return r;
+}
+
+// Totals of one chunk from per-lane group sums (sx the job weights, sy p_a): writes the eight
+// group totals to tg[0..7] and the chunk total to *tc (fp64 throughout).
+__device__ __forceinline__ void emit_chunk_totals(const double (&sx)[kChunkGroups], const double (&sy)[kChunkGroups],
+                                                  double2* tc, double2* tg) {
+  static_assert(kChunkGroups == 8, "eight groups per chunk");
+  const int lane = threadIdx.x & 31;
+  double gx = warp_reduce_scatter8(sx), gy = warp_reduce_scatter8(sy);
+  if ((lane & 3) == 0) tg[lane >> 2] = make_double2(gx, gy);
+#pragma unroll
+  for (int o = 4; o < 32; o <<= 1) {
+    gx += __shfl_xor_sync(0xffffffffu, gx, o);
+    gy += __shfl_xor_sync(0xffffffffu, gy, o);
+  }
+  if (lane == 0) *tc = make_double2(gx, gy);
+}
+
+// Warp-level draw inside one group [e0, e0 + kGroup) (clipped at hi): `base` is the weight
+// before e0 and `target` = u * Z. Returns the first index whose inclusive prefix exceeds
+// target, else (rounding) the group's last index with positive weight, or -1 if it has none;
+// *la receives row a's logit at that index.
+template <typename T, bool RESID>
+__device__ int warp_draw_group(const JobRows<T, RESID>& J, int e0, int hi, double base, double target, float* la) {
+  const int lane = threadIdx.x & 31;
+  const int e = e0 + lane * 8;
+  Raw8<T, RESID> xg;
+  if (J.vector_ok(e0, min(hi, e0 + kGroup), kGroup))
+    J.load_full(e, xg);
+  else
+    J.load(e, hi, xg);
+  float w[8], pw[8], xa[8];
+  J.weights(xg, w, pw);
+  xg.a.unpack(xa);
+  double mine = 0.0;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) mine += static_cast<double>(w[k]);
+  double incl = mine;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const double t = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += t;
+  }
+  double excl = __shfl_up_sync(0xffffffffu, incl, 1);
+  if (lane == 0) excl = 0.0;
+  const unsigned hit = __ballot_sync(0xffffffffu, base + incl > target);
+  const unsigned pos = __ballot_sync(0xffffffffu, mine > 0.0);
+  if (pos == 0u) {
+    *la = 0.0f;
+    return -1;
+  }
+  // rounding can leave no lane crossing: the group's last positive element then
+  const int src = hit ? __ffs(hit) - 1 : 31 - __clz(pos);
+  int yl = -1, lp = -1;
+  float lyl = 0.0f, llp = 0.0f;
+  double Cl = base + excl;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    Cl += static_cast<double>(w[k]);
+    if (w[k] > 0.0f) { lp = k; llp = xa[k]; }
+    if (yl < 0 && w[k] > 0.0f && Cl > target) { yl = k; lyl = xa[k]; }
+  }
+  if (yl < 0) { yl = lp; lyl = llp; }
+  *la = __shfl_sync(0xffffffffu, lyl, src);
+  return __shfl_sync(0xffffffffu, e + yl, src);
+}
+
+// Warp-level draw inside one chunk [lo, hi) (hi - lo <= kChunkElems, lo a multiple of 8):
+// `base` is the weight before lo and `target` = u * Z. A whole batch of groups is in flight
+// at once; the group totals locate the 256-element group whose prefix crosses target, which
+// warp_draw_group then walks (its data comes again from L1/L2). Returns the first index
+// whose inclusive prefix exceeds target, else (rounding) the last index with positive
+// weight, or -1 if the chunk has no positive weight; *la receives row a's logit there.
+template <typename T, bool RESID>
+__device__ int warp_draw_chunk(const JobRows<T, RESID>& J, int lo, int hi, double base, double target, float* la) {
+  constexpr int NB = kChunkBatch<T, RESID>;
+  const int lane = threadIdx.x & 31;
+  const bool full = J.vector_ok(lo, hi, kChunkElems);
+  double C = base, cG = 0.0;
+  int last = -1, G = -1;
+#pragma unroll 1
+  for (int g0 = 0; g0 < kChunkGroups && G < 0; g0 += NB) {
+    double gs[NB];
+    {
+      Raw8<T, RESID> x[NB];
+      if (full) {
+#pragma unroll
+        for (int g = 0; g < NB; ++g) J.load_full(lo + (g0 + g) * kGroup + lane * 8, x[g]);
+      } else {
+#pragma unroll
+        for (int g = 0; g < NB; ++g) J.load(lo + (g0 + g) * kGroup + lane * 8, hi, x[g]);
+      }
+#pragma unroll
+      for (int g = 0; g < NB; ++g) gs[g] = lane_group_weight(J, x[g], lo + (g0 + g) * kGroup + lane * 8, &last);
+    }
+#pragma unroll
+    for (int g = 0; g < NB; ++g) gs[g] = warp_sum(gs[g]);
+    // the group whose prefix crosses target (every lane computes the same)
+#pragma unroll
+    for (int g = 0; g < NB; ++g) {
+      if (G < 0 && gs[g] > 0.0 && C + gs[g] > target) {
+        G = g0 + g;
+        cG = C;
+      }
+      C += gs[g];
+    }
+  }
+  if (G < 0) {
+    // rounding put target past the chunk's total: its last positive element
+    const int y = __reduce_max_sync(0xffffffffu, last);
+    *la = y >= 0 ? J.logit_a(y) : 0.0f;
+    return y;
+  }
+  return warp_draw_group(J, lo + G * kGroup, hi, cG, target, la);
 }
 
 // Warp-level draw inside [lo, hi): `base` is the weight before lo, `target` = u * Z.
