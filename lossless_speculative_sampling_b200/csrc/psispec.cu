@@ -88,7 +88,18 @@ psispec_status check_ws(const void* ws, size_t bytes, size_t need) {
 }
 
 inline bool aligned_to(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
-inline psispec_status launched() { return cudaGetLastError() == cudaSuccess ? PSISPEC_OK : PSISPEC_ERR_CUDA; }
+
+// One kernel launch on the caller's stream; a launch error becomes PSISPEC_ERR_CUDA.
+template <typename... KArgs, typename... Args>
+psispec_status launch(void (*kernel)(KArgs...), unsigned grid, unsigned block, size_t smem, cudaStream_t st,
+                      Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...) == cudaSuccess ? PSISPEC_OK : PSISPEC_ERR_CUDA;
+}
 
 // Request index of every node, from node_offsets (tree rows have no fixed count per request).
 __global__ void node_request_kernel(const int32_t* __restrict__ offs, int B, int N, int32_t* __restrict__ row_req) {
@@ -111,11 +122,25 @@ unsigned persistent_grid(Kern kernel, int64_t work_warps) {
   return static_cast<unsigned>(want < 1 ? 1 : (want < slots ? want : slots));
 }
 
+// Persistent grid for a warp-granular kernel with `warps` warps per CTA and dynamic shared
+// memory: one CTA per resident slot, fewer when there is less work than that.
+template <typename Kern>
+int64_t want_slots(int64_t work_warps, int warps, Kern kernel, int block, int smem) {
+  int dev = 0, sms = 148, occ = 1;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, block, smem);
+  const int64_t want = (work_warps + warps - 1) / warps;
+  const int64_t slots = static_cast<int64_t>(sms) * (occ > 0 ? occ : 1);
+  return want < 1 ? 1 : (want < slots ? want : slots);
+}
+
 // The streaming pass over a [rows, V] tensor: one partial per chunk. Aligned tensors go
 // through the bulk-copy ring kernel, others through plain 16-byte loads.
 template <typename T>
 psispec_status launch_stream(const T* base, int64_t rows, int rows_per_req, const int32_t* row_req, int V,
-                             const float* temperature, int nreq, Partial* parts, cudaStream_t st) {
+                             const float* temperature, int nreq, Partial* parts, cudaStream_t st,
+                             int32_t* zero = nullptr, int nzero = 0) {
   const int64_t chunks = rows * nchunks_for(V);
   const bool aligned = (reinterpret_cast<uintptr_t>(base) & 15u) == 0 && (int64_t(V) * sizeof(T)) % 16 == 0;
   if (aligned) {
@@ -130,13 +155,11 @@ psispec_status launch_stream(const T* base, int64_t rows, int rows_per_req, cons
     const int64_t want = (chunks + (kThreads / 32) - 1) / (kThreads / 32);
     const int64_t slots = static_cast<int64_t>(sms) * (occ > 0 ? occ : 1);
     const unsigned grid = static_cast<unsigned>(want < slots ? want : slots);
-    stream_partials_tma_kernel<T><<<grid, kThreads, smem, st>>>(base, rows_per_req, row_req, V, chunks, temperature,
-                                                                nreq, parts);
-    return launched();
+    return launch(stream_partials_tma_kernel<T>, grid, kThreads, smem, st, base, rows_per_req, row_req, V, chunks,
+                  temperature, nreq, parts, zero, nzero);
   }
-  stream_partials_kernel<T><<<persistent_grid(stream_partials_kernel<T>, chunks), kThreads, 0, st>>>(
-      base, rows_per_req, row_req, V, chunks, temperature, parts);
-  return launched();
+  return launch(stream_partials_kernel<T>, persistent_grid(stream_partials_kernel<T>, chunks), kThreads, 0, st, base,
+                rows_per_req, row_req, V, chunks, temperature, parts, zero, nzero);
 }
 
 // Row statistics of a [rows, V] tensor (the tree's statistics pass).
@@ -145,9 +168,8 @@ psispec_status launch_stats(const T* base, int64_t rows, int rows_per_req, const
                             const float* temperature, int nreq, const float* top_p, StatsWs ws, cudaStream_t st) {
   psispec_status s = launch_stream<T>(base, rows, rows_per_req, row_req, V, temperature, nreq, ws.parts, st);
   if (s != PSISPEC_OK) return s;
-  row_finalize_kernel<T><<<static_cast<unsigned>(rows), kThreads, 0, st>>>(base, rows_per_req, row_req, V,
-                                                                            temperature, top_p, ws.parts, ws.stats);
-  return launched();
+  return launch(row_finalize_kernel<T>, static_cast<unsigned>(rows), kThreads, 0, st, base, rows_per_req, row_req, V,
+                temperature, top_p, ws.parts, ws.stats);
 }
 
 // The draw jobs of a verification call: totals pass (bulk-copy ring when the rows allow it),
@@ -159,28 +181,21 @@ psispec_status launch_draws(const T* A, const T* Bt, int V, int njobs, const Par
   // the bulk-copy ring serves bf16 rows (fp32 stages would not fit enough warps per SM)
   const bool ring = sizeof(T) == 2 && (reinterpret_cast<uintptr_t>(A) & 15u) == 0 &&
                     (reinterpret_cast<uintptr_t>(Bt) & 15u) == 0 && (int64_t(V) * sizeof(T)) % 16 == 0;
-  if (ring) {
-    const int smem = kDrawWarps * kDrawRing * kDrawStageBytes<T>;
-    if (cudaFuncSetAttribute(draw_totals_tma_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-        cudaSuccess)
-      return PSISPEC_ERR_CUDA;
-    int dev = 0, sms = 148, occ = 1;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, draw_totals_tma_kernel<T>, kDrawWarps * 32, smem);
-    const int64_t want = (items + kDrawWarps - 1) / kDrawWarps;
-    const int64_t slots = static_cast<int64_t>(sms) * (occ > 0 ? occ : 1);
-    draw_totals_tma_kernel<T><<<static_cast<unsigned>(want < slots ? want : slots), kDrawWarps * 32, smem, st>>>(
-        A, Bt, V, njobs, jobs, tc, tg);
-  } else {
-    draw_totals_kernel<T><<<persistent_grid(draw_totals_kernel<T>, items), kThreads, 0, st>>>(A, Bt, V, njobs, jobs,
-                                                                                            tc, tg);
-  }
-  psispec_status s = launched();
+  const int smem = kDrawWarps * kDrawRing * kDrawStageBytes<T>;
+  if (ring && cudaFuncSetAttribute(draw_totals_tma_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+                  cudaSuccess)
+    return PSISPEC_ERR_CUDA;
+  psispec_status s;
+  if (ring)
+    s = launch(draw_totals_tma_kernel<T>, static_cast<unsigned>(want_slots(items, kDrawWarps, draw_totals_tma_kernel<T>,
+                                                                           kDrawWarps * 32, smem)),
+               kDrawWarps * 32, smem, st, A, Bt, V, njobs, jobs, tc, tg);
+  else
+    s = launch(draw_totals_kernel<T>, persistent_grid(draw_totals_kernel<T>, items), kThreads, 0, st, A, Bt, V, njobs,
+               jobs, tc, tg);
   if (s != PSISPEC_OK) return s;
-  draw_pick_kernel<T><<<static_cast<unsigned>((njobs + kThreads / 32 - 1) / (kThreads / 32)), kThreads, 0, st>>>(
-      A, Bt, V, njobs, parts_a, jobs, tc, tg, out_tokens);
-  return launched();
+  return launch(draw_pick_kernel<T>, static_cast<unsigned>((njobs + kThreads / 32 - 1) / (kThreads / 32)), kThreads, 0,
+                st, A, Bt, V, njobs, parts_a, jobs, tc, tg, out_tokens);
 }
 
 template <typename T>
@@ -193,9 +208,8 @@ psispec_status sample_draft_impl(const T* draft, int B, int K, int V, const floa
   RowStat* stats = out_stats ? out_stats : w.st.stats;
   psispec_status s = launch_stream<T>(draft, rows, K, nullptr, V, temperature, B, w.st.parts, st);
   if (s != PSISPEC_OK) return s;
-  sample_row_kernel<T><<<static_cast<unsigned>((rows + kThreads / 32 - 1) / (kThreads / 32)), kThreads, 0, st>>>(
-      draft, K, V, static_cast<int>(rows), temperature, top_p, u, w.st.parts, stats, out_tokens, out_q);
-  return launched();
+  return launch(sample_row_kernel<T>, static_cast<unsigned>((rows + kThreads / 32 - 1) / (kThreads / 32)), kThreads, 0,
+                st, draft, K, V, static_cast<int>(rows), temperature, top_p, u, w.st.parts, stats, out_tokens, out_q);
 }
 
 template <typename T>
@@ -206,7 +220,6 @@ psispec_status verify_linear_impl(const T* tgt, const T* drf, int B, int K, int 
   Carver c(ws);
   LinearWs w = carve_linear(c, B, K, V);
   const int64_t rows_t = int64_t(B) * (K + 1), rows_d = draft_stats ? 0 : int64_t(B) * K;
-  if (cudaMemsetAsync(w.cnt, 0, sizeof(int32_t) * B, st) != cudaSuccess) return PSISPEC_ERR_CUDA;
   VerifyArgs a;
   a.B = B;
   a.K = K;
@@ -228,13 +241,14 @@ psispec_status verify_linear_impl(const T* tgt, const T* drf, int B, int K, int 
   a.out_p = out_p;
   a.out_q = out_q;
   a.jobs = w.jobs;
-  psispec_status s = launch_stream<T>(tgt, rows_t, K + 1, nullptr, V, temperature, B, w.t.parts, st);
+  // the first streaming pass also clears the request arrival counters
+  psispec_status s = launch_stream<T>(tgt, rows_t, K + 1, nullptr, V, temperature, B, w.t.parts, st, w.cnt, B);
   if (s != PSISPEC_OK) return s;
   if (rows_d > 0 && (s = launch_stream<T>(drf, rows_d, K, nullptr, V, temperature, B, w.d.parts, st)) != PSISPEC_OK)
     return s;
-  verify_row_kernel<T><<<static_cast<unsigned>((rows_t + rows_d + kThreads / 32 - 1) / (kThreads / 32)), kThreads, 0,
-                         st>>>(tgt, drf, a);
-  if ((s = launched()) != PSISPEC_OK) return s;
+  s = launch(verify_row_kernel<T>, static_cast<unsigned>((rows_t + rows_d + kThreads / 32 - 1) / (kThreads / 32)),
+             kThreads, 0, st, tgt, drf, a);
+  if (s != PSISPEC_OK) return s;
   return launch_draws<T>(tgt, drf, V, B, w.t.parts, w.jobs, w.draw_tc, w.draw_tg, out_tokens, st);
 }
 
@@ -246,16 +260,14 @@ psispec_status verify_tree_impl(const T* tgt, const T* drf, int B, int N, int V,
   const int ns = nslices_for(V);
   Carver c(ws);
   TreeWs w = carve_tree(c, N, V);
-  node_request_kernel<<<B, 128, 0, st>>>(offs, B, N, w.row_req);
-  psispec_status s = launched();
+  psispec_status s = launch(node_request_kernel, static_cast<unsigned>(B), 128, 0, st, offs, B, N, w.row_req);
   if (s != PSISPEC_OK) return s;
   s = launch_stats<T>(tgt, N, 1, w.row_req, V, temperature, B, top_p, w.t, st);
   if (s != PSISPEC_OK) return s;
   s = launch_stats<T>(drf, N, 1, w.row_req, V, temperature, B, top_p, w.d, st);
   if (s != PSISPEC_OK) return s;
-  tree_walk_kernel<T><<<B, kTreeThreads, 0, st>>>(tgt, drf, V, offs, parent, tokens, w.t.stats, w.d.stats, u_acc,
-                                                  u_res, max_depth, out_path, out_tokens, out_len);
-  return launched();
+  return launch(tree_walk_kernel<T>, static_cast<unsigned>(B), kTreeThreads, 0, st, tgt, drf, V, offs, parent, tokens,
+                w.t.stats, w.d.stats, u_acc, u_res, max_depth, out_path, out_tokens, out_len);
 }
 
 bool bad_dtype(int dtype) { return dtype != PSISPEC_F32 && dtype != PSISPEC_BF16; }

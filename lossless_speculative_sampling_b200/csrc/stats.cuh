@@ -145,13 +145,17 @@ __device__ __forceinline__ Partial warp_chunk_partial(const T* __restrict__ row,
 }
 
 // The streaming pass: persistent warps over every chunk of a [rows, V] tensor, each chunk
-// read once, one partial per chunk (parts[row * nchunks + chunk]).
+// read once, one partial per chunk (parts[row * nchunks + chunk]). CTA 0 also clears the
+// nzero arrival counters at `zero` that the call's later kernels use.
 template <typename T>
 __global__ void __launch_bounds__(kThreads, 4) stream_partials_kernel(const T* __restrict__ base, int rows_per_req,
                                                                     const int32_t* __restrict__ row_req, int V,
                                                                     int64_t total_chunks,
                                                                     const float* __restrict__ temperature,
-                                                                    Partial* __restrict__ parts) {
+                                                                    Partial* __restrict__ parts,
+                                                                    int32_t* __restrict__ zero, int nzero) {
+  if (blockIdx.x == 0)
+    for (int i = threadIdx.x; i < nzero; i += blockDim.x) zero[i] = 0;
   const int nch = nchunks_for(V);
   const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
   int64_t g = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
@@ -223,14 +227,83 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
   return true;
 }
 
+// NaN-propagating maximum of two packed bf16 pairs.
+__device__ __forceinline__ uint32_t bmax2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.NaN.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+// NaN-propagating maximum of the elements of NV 16-byte vectors (bf16 pairs are compared
+// packed, before any conversion).
+template <typename T, int NV>
+__device__ __forceinline__ float lane_max_raw(const uint4 (&raw)[NV]) {
+  if constexpr (sizeof(T) == 2) {
+    uint32_t m0 = bmax2(raw[0].x, raw[0].y), m1 = bmax2(raw[0].z, raw[0].w);
+#pragma unroll
+    for (int j = 1; j < NV; ++j) {
+      m0 = bmax2(m0, bmax2(raw[j].x, raw[j].y));
+      m1 = bmax2(m1, bmax2(raw[j].z, raw[j].w));
+    }
+    const uint32_t m = bmax2(m0, m1);
+    return fmax_nan(__uint_as_float(m << 16), __uint_as_float(m & 0xFFFF0000u));
+  } else {
+    float m0 = fmax_nan(__uint_as_float(raw[0].x), __uint_as_float(raw[0].y));
+    float m1 = fmax_nan(__uint_as_float(raw[0].z), __uint_as_float(raw[0].w));
+#pragma unroll
+    for (int j = 1; j < NV; ++j) {
+      m0 = fmax_nan(m0, fmax_nan(__uint_as_float(raw[j].x), __uint_as_float(raw[j].y)));
+      m1 = fmax_nan(m1, fmax_nan(__uint_as_float(raw[j].z), __uint_as_float(raw[j].w)));
+    }
+    return fmax_nan(m0, m1);
+  }
+}
+
+// Warp-level partial of one full chunk held in registers (NV vectors per lane), in two
+// steps: the chunk maximum M first (NaN-propagating, so a NaN or +inf logit leaves s NaN),
+// then the weights 2^((x - M) c) relative to it, summed in packed fp32 pairs per lane and in
+// fp64 across lanes. A chunk of -inf logits only reports s = 0, m = -inf.
+template <typename T, int NV>
+__device__ __forceinline__ Partial warp_chunk_partial_full(const uint4 (&raw)[NV], float c) {
+  const float M = warp_max(lane_max_raw<T, NV>(raw));
+  Partial p{0.0, M, 0, 0, 0};
+  if (M == -INFINITY) return p;
+  const f32x2 mm = pack2(M, M), cc = pack2(c, c);
+  f32x2 acc0 = pack2(0.0f, 0.0f), acc1 = acc0;
+#pragma unroll
+  for (int j = 0; j < NV; ++j) {
+    float f[8];
+    Vec<T>::unpack(raw[j], f);
+#pragma unroll
+    for (int k = 0; k < Vec<T>::N; k += 4) {
+      float a, b, d, e;
+      unpack2(mul2(sub2(pack2(f[k], f[k + 1]), mm), cc), a, b);
+      unpack2(mul2(sub2(pack2(f[k + 2], f[k + 3]), mm), cc), d, e);
+      acc0 = add2(acc0, pack2(ex2(a), ex2(b)));
+      acc1 = add2(acc1, pack2(ex2(d), ex2(e)));
+    }
+  }
+  float a, b, d, e;
+  unpack2(acc0, a, b);
+  unpack2(acc1, d, e);
+  p.s = warp_sum((static_cast<double>(a) + static_cast<double>(b)) + (static_cast<double>(d) + static_cast<double>(e)));
+  return p;
+}
+
 // Warp-level partial of one chunk held in shared memory (n elements, 16-byte vectors).
 template <typename T, bool GREEDY>
 __device__ __forceinline__ Partial warp_chunk_partial_smem(const T* __restrict__ sp, int c0, int n, float c) {
   constexpr int N = Vec<T>::N;
   constexpr int kFull = kChunkElems / (32 * N);  // vectors per lane in a full chunk
   const int lane = threadIdx.x & 31;
-  LaneStat L{GREEDY ? -INFINITY : -3.402823466e38f, 0.0f, 0x7fffffff, false};
   const uint4* v4 = reinterpret_cast<const uint4*>(sp);
+  if (!GREEDY && n == kChunkElems) {
+    uint4 raw[kFull];
+#pragma unroll
+    for (int j = 0; j < kFull; ++j) raw[j] = v4[lane + 32 * j];
+    return warp_chunk_partial_full<T, kFull>(raw, c);
+  }
+  LaneStat L{GREEDY ? -INFINITY : -3.402823466e38f, 0.0f, 0x7fffffff, false};
   if (n == kChunkElems) {
     uint4 raw[kFull];
 #pragma unroll
@@ -262,7 +335,10 @@ __global__ void __launch_bounds__(kThreads) stream_partials_tma_kernel(const T* 
                                                                         const int32_t* __restrict__ row_req, int V,
                                                                         int64_t total_chunks,
                                                                         const float* __restrict__ temperature,
-                                                                        int nreq, Partial* __restrict__ parts) {
+                                                                        int nreq, Partial* __restrict__ parts,
+                                                                        int32_t* __restrict__ zero, int nzero) {
+  if (blockIdx.x == 0)
+    for (int i = threadIdx.x; i < nzero; i += blockDim.x) zero[i] = 0;
   extern __shared__ __align__(128) unsigned char ring_smem[];
   __shared__ uint64_t bars[kThreads / 32][kRing];
   __shared__ float scale[kScaleTable];
