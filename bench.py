@@ -29,10 +29,10 @@ sys.path.insert(0, ROOT)
 
 METRIC = "verified draft positions/sec and logits HBM GB/s vs B200 peak (Ψ-Spec verify)"
 UNIT = "positions/s"
-# kernel launches per call (see csrc/psispec.cu): sample_draft = stream + finish + top-p;
-# verify_linear = stream + finish + top-p + draw totals + draw pick (the per-request
-# arrival counters are cleared with a memset, which is not a kernel of this library)
-LAUNCHES_PER_STEP = 2 + 4  # sample: stream, sample_row; verify: stream, verify_row, draw totals, draw pick
+# kernel launches per step of the default workload (see csrc/psispec.cu): sample_draft =
+# streaming pass + row finisher; verify_linear = streaming pass + row finisher + draw totals +
+# draw pick
+LAUNCHES_PER_STEP = 2 + 4
 
 
 def _peaks():
@@ -162,6 +162,8 @@ def run_reference(args):
         return
     from lossless_speculative_sampling_b200 import synth
 
+    if args.workload in synth.tree_cases():
+        return _run_reference_tree(args)
     case = synth.linear_cases()[args.workload]
     # about 80 ms of oracle work per request at V = 151936: keep the whole run near two minutes
     n_req = max(1, min(args.ref_requests, int(120.0 / (0.08 * (args.steps + args.warmup)))))
@@ -176,31 +178,57 @@ def run_reference(args):
     dt = (time.perf_counter() - t0) / args.steps
     value = n_req * case.K / dt
     sample = "%d of %d requests of workload %s per step (fp64 C oracle, 1 thread)" % (n_req, case.B, args.workload)
+    _print_reference(args, value, dt, "f64", {"workload": args.workload, "requests_per_step": n_req, "block": case.K,
+                                              "vocab": case.V}, sample)
+
+
+def _run_reference_tree(args):
+    import oracle
+    from lossless_speculative_sampling_b200 import synth
+
+    case = synth.tree_cases()[args.workload]
+    trie, tgt, drf, tokens, ua, ur = synth.tree_inputs(case, device="cpu")
+    n_req = max(1, min(case.B, args.ref_requests))
+    n = int(trie.node_offsets[n_req])
+    t, d = tgt[:n].to(torch.float64).numpy(), drf[:n].to(torch.float64).numpy()
+    off, par, tok = trie.node_offsets[: n_req + 1].numpy(), trie.parent[:n].numpy(), tokens[:n].numpy()
+    a, r = ua[:n].numpy(), ur[:n].numpy()
+    T, P = np.full(n_req, case.temperature), np.full(n_req, case.top_p)
+
+    def one():
+        oracle.verify_tree(t, d, off, par, tok, a, r, T, P, case.max_depth)
+
+    for _ in range(args.warmup):
+        one()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        one()
+    dt = (time.perf_counter() - t0) / args.steps
+    sample = "%d of %d tries (%d nodes) of workload %s per step (fp64 C oracle, 1 thread)" % (n_req, case.B, n,
+                                                                                              args.workload)
+    _print_reference(args, n / dt, dt, "f64", {"workload": args.workload, "tries_per_step": n_req, "nodes": n,
+                                               "vocab": case.V}, sample)
+
+
+def _print_reference(args, value, dt, dtype, config, sample):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": args.workload, "requests_per_step": n_req, "block": case.K, "vocab": case.V},
+            "scaling": "weak", "vs_baseline": None, "dtype": dtype, "data": "synthetic", "config": config,
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
-def run_ours(args):
+def _prepare_linear(case, dev):
+    """Device inputs, outputs and the two calls of one linear step."""
     from lossless_speculative_sampling_b200 import psispec, synth
 
-    dist, rank, world, local = _dist()
-    dev = torch.device("cuda", local)
-    torch.cuda.set_device(dev)
-    case = synth.linear_cases()[args.workload]
     B, K, V = case.B, case.K, case.V
-    case.seed += 97 * rank  # each rank verifies its own batch
     tgt, drf = synth.linear_logits(case, device=dev)
     ud, ua, ur = synth.linear_uniforms(case)
     ud, ua, ur = ud.to(dev), ua.to(dev), ur.to(dev)
     Ts = torch.full((B,), case.temperature, device=dev)
     Ps = torch.full((B,), case.top_p, device=dev)
-    esz = tgt.element_size()
-
     x = torch.empty((B, K), dtype=torch.int32, device=dev)
     q = torch.empty((B, K), dtype=torch.float32, device=dev)
     stats = torch.empty((B, K, psispec.ROW_STATS_BYTES), dtype=torch.uint8, device=dev)
@@ -210,129 +238,215 @@ def run_ours(args):
     o_q = torch.empty((B, K), dtype=torch.float32, device=dev)
     ws_s = torch.empty(psispec.workspace_size(psispec.OP_SAMPLE_DRAFT, B, K, V), dtype=torch.uint8, device=dev)
     ws_v = torch.empty(psispec.workspace_size(psispec.OP_VERIFY_LINEAR, B, K, V), dtype=torch.uint8, device=dev)
+    esz = tgt.element_size()
 
-    def step(t_in, d_in):
+    def sample(t_in=tgt, d_in=drf):
         psispec.sample_draft(d_in, Ts, Ps, ud, out_tokens=x, out_q=q, row_stats=stats, ws=ws_s)
+
+    def verify(t_in=tgt, d_in=drf):
         psispec.verify_linear(t_in, d_in, x, ua, ur, Ts, Ps, draft_row_stats=stats, out_tokens=o_tok,
                               out_accept_len=o_len, out_p=o_p, out_q=o_q, ws=ws_v)
 
-    def call_sample():
-        psispec.sample_draft(drf, Ts, Ps, ud, out_tokens=x, out_q=q, row_stats=stats, ws=ws_s)
+    return {
+        "inputs": (tgt, drf), "calls": [("sample_draft", sample), ("verify_linear", verify)],
+        "outputs": (o_tok, o_len), "positions": B * K, "esz": esz,
+        # algorithmic bytes: sample_draft reads the draft tensor once; verify_linear reads the
+        # verifier tensor once plus, per request, the one draft row of the residual draw
+        "bytes": {"sample_draft": B * K * V * esz, "verify_linear": B * (K + 1) * V * esz + B * V * esz},
+        "bytes_step": (B * (K + 1) + B * K) * V * esz,
+        "describe": "linear verify B=%d K=%d V=%d %s, T=%g, top-p %g" % (
+            B, K, V, "bf16" if esz == 2 else "fp32", case.temperature, case.top_p),
+        "config": {"global_batch": B, "block": K, "vocab": V},
+        "accept": lambda: float(o_len.float().mean()),
+    }
 
-    def call_verify():
-        psispec.verify_linear(tgt, drf, x, ua, ur, Ts, Ps, draft_row_stats=stats, out_tokens=o_tok,
-                              out_accept_len=o_len, out_p=o_p, out_q=o_q, ws=ws_v)
 
-    for _ in range(args.warmup):
-        step(tgt, drf)
+def _prepare_tree(case, dev):
+    """Device inputs, outputs and the one call of a tree step."""
+    from lossless_speculative_sampling_b200 import psispec, synth
+
+    trie, tgt, drf, tokens, ua, ur = synth.tree_inputs(case, device=dev)
+    B, N, V = case.B, trie.N, case.V
+    offs, parent, tok = trie.node_offsets.to(dev), trie.parent.to(dev), tokens.to(dev)
+    ua, ur = ua.to(dev), ur.to(dev)
+    Ts = torch.full((B,), case.temperature, device=dev)
+    Ps = torch.full((B,), case.top_p, device=dev)
+    D = case.max_depth
+    o_path = torch.empty((B, D), dtype=torch.int32, device=dev)
+    o_tok = torch.empty((B, D + 1), dtype=torch.int32, device=dev)
+    o_len = torch.empty(B, dtype=torch.int32, device=dev)
+    ws = torch.empty(psispec.workspace_size(psispec.OP_VERIFY_TREE, B, N, V), dtype=torch.uint8, device=dev)
+    esz = tgt.element_size()
+
+    def verify(t_in=tgt, d_in=drf):
+        psispec.verify_tree(t_in, d_in, offs, parent, tok, ua, ur, Ts, Ps, D, out_path=o_path, out_tokens=o_tok,
+                            out_accept_len=o_len, ws=ws)
+
+    return {
+        "inputs": (tgt, drf), "calls": [("verify_tree", verify)], "outputs": (o_tok, o_len), "positions": N,
+        "esz": esz, "bytes": {"verify_tree": 2 * N * V * esz}, "bytes_step": 2 * N * V * esz,
+        "describe": "tree verify B=%d tries x %d nodes (depth <= %d, branching <= %d) V=%d %s, T=%g, top-p %g" % (
+            B, case.nodes, case.max_depth, case.max_branch, V, "bf16" if esz == 2 else "fp32", case.temperature,
+            case.top_p),
+        "config": {"global_batch": B, "nodes": N, "vocab": V},
+        "accept": lambda: float(o_len.float().mean()),
+    }
+
+
+def _prepare(name, dev, rank=0):
+    from lossless_speculative_sampling_b200 import synth
+
+    lin, tre = synth.linear_cases(), synth.tree_cases()
+    if name in lin:
+        case = lin[name]
+        case.seed += 97 * rank  # each rank verifies its own batch
+        return _prepare_linear(case, dev), case
+    case = tre[name]
+    case.seed += 97 * rank
+    return _prepare_tree(case, dev), case
+
+
+def _graphs(calls, dev, warmup):
+    """Each call captured once into a CUDA graph and replayed: the launch sequence a serving
+    loop would use."""
+    for _ in range(warmup):
+        for _, f in calls:
+            f()
     torch.cuda.synchronize()
-    if not args.no_graph:
-        # each call is captured once and replayed: the launch sequence a serving loop would use
-        side = torch.cuda.Stream(dev)
-        side.wait_stream(torch.cuda.current_stream(dev))
-        with torch.cuda.stream(side):
-            call_sample()
-            call_verify()
-        torch.cuda.current_stream(dev).wait_stream(side)
-        g_s, g_v = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g_s):
-            call_sample()
-        with torch.cuda.graph(g_v):
-            call_verify()
-        call_sample, call_verify = g_s.replay, g_v.replay
-        for _ in range(args.warmup):
-            call_sample()
-            call_verify()
-        torch.cuda.synchronize()
-    _barrier(dist)
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(side):
+        for _, f in calls:
+            f()
+    torch.cuda.current_stream(dev).wait_stream(side)
+    out = []
+    for name, f in calls:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            f()
+        out.append((name, g.replay, g))
+    for _ in range(warmup):
+        for _, r, _g in out:
+            r()
+    torch.cuda.synchronize()
+    return out
 
-    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3 * args.steps)]
+
+def _time_steps(calls, steps, dist=None):
+    """Device time of `steps` steps (CUDA events on the launching stream): (ms per step,
+    {call: mean ms})."""
+    n = len(calls)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range((n + 1) * steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    _barrier(dist)
+    start.record()
+    for k in range(steps):
+        for i, c in enumerate(calls):
+            ev[(n + 1) * k + i].record()
+            c[1]()
+        ev[(n + 1) * k + n].record()
+    end.record()
+    torch.cuda.synchronize()
+    _barrier(dist)
+    ms = _max_over_ranks(dist, start.elapsed_time(end)) / steps
+    per = {c[0]: statistics.mean(ev[(n + 1) * k + i].elapsed_time(ev[(n + 1) * k + i + 1]) for k in range(steps))
+           for i, c in enumerate(calls)}
+    return ms, per
+
+
+def _all_workloads(args, dev):
+    """One JSON line per workload (the parity configurations at full size), for the tables."""
+    from lossless_speculative_sampling_b200 import synth
+
+    peak, peak_kind = _peaks()
+    names = [n for n in synth.linear_cases() if n != "tiny"] + list(synth.tree_cases())
+    for name in names:
+        P, case = _prepare(name, dev)
+        calls = _graphs(P["calls"], dev, 3) if not args.no_graph else P["calls"]
+        steps = max(5, min(args.steps, int(2e5 / max(1.0, P["bytes_step"] / 1e6))))
+        ms, per = _time_steps(calls, steps)
+        line = {"workload": name, "describe": P["describe"], "value": P["positions"] / (ms * 1e-3), "unit": UNIT,
+                "ms_per_step": ms, "steps": steps, "step_gbs": P["bytes_step"] / (ms * 1e-3) / 1e9,
+                "calls_ms": per, "calls_gbs": {k: P["bytes"][k] / (per[k] * 1e-3) / 1e9 for k in per},
+                "peak_gbs": peak, "peak_kind": peak_kind, "mean_accept_len": P["accept"]()}
+        line["step_frac"] = line["step_gbs"] / peak
+        print(json.dumps(line), flush=True)
+        del P, calls
+        torch.cuda.empty_cache()
+
+
+def run_ours(args):
+    dist, rank, world, local = _dist()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if args.all:
+        _all_workloads(args, dev)
+        if dist is not None:
+            dist.destroy_process_group()
+        return
+    P, case = _prepare(args.workload, dev, rank)
+    calls = P["calls"] if args.no_graph else _graphs(P["calls"], dev, args.warmup)
+    if args.no_graph:
+        for _ in range(args.warmup):
+            for _, f in calls:
+                f()
+    _barrier(dist)
     with ClockSampler(dev) as clk:
-        torch.cuda.synchronize()
-        _barrier(dist)
-        start.record()
-        for k in range(args.steps):
-            ev[3 * k].record()
-            call_sample()
-            ev[3 * k + 1].record()
-            call_verify()
-            ev[3 * k + 2].record()
-        end.record()
-        torch.cuda.synchronize()
-        _barrier(dist)
-    ms_total = _max_over_ranks(dist, start.elapsed_time(end))
-    ms_step = ms_total / args.steps
-    t_sample = statistics.mean(ev[3 * k].elapsed_time(ev[3 * k + 1]) for k in range(args.steps))
-    t_verify = statistics.mean(ev[3 * k + 1].elapsed_time(ev[3 * k + 2]) for k in range(args.steps))
-    mean_accept = float(o_len.float().mean())
+        ms_step, per = _time_steps(calls, args.steps, dist)
+    mean_accept = P["accept"]()
 
     # end to end through the public API with host buffers: pinned H2D of the step's inputs,
     # the step, D2H of its result, every step inside the timed region
     e2e_steps = max(3, min(args.steps, 20))
-    tgt_h = tgt.cpu().pin_memory()
-    drf_h = drf.cpu().pin_memory()
-    tok_h = torch.empty((B, K + 1), dtype=torch.int32).pin_memory()
-    len_h = torch.empty(B, dtype=torch.int32).pin_memory()
-    t_dev, d_dev = torch.empty_like(tgt), torch.empty_like(drf)
-    step(tgt, drf)
+    hosts = [t.cpu().pin_memory() for t in P["inputs"]]
+    devs = [torch.empty_like(t) for t in P["inputs"]]
+    outs_h = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in P["outputs"]]
+    for _, f in P["calls"]:
+        f(*devs)
     torch.cuda.synchronize()
     _barrier(dist)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
     for _ in range(e2e_steps):
-        t_dev.copy_(tgt_h, non_blocking=True)
-        d_dev.copy_(drf_h, non_blocking=True)
-        step(t_dev, d_dev)
-        tok_h.copy_(o_tok, non_blocking=True)
-        len_h.copy_(o_len, non_blocking=True)
+        for d, h in zip(devs, hosts):
+            d.copy_(h, non_blocking=True)
+        for _, f in P["calls"]:
+            f(*devs)
+        for h, o in zip(outs_h, P["outputs"]):
+            h.copy_(o, non_blocking=True)
     e1.record()
     torch.cuda.synchronize()
     e2e_ms = _max_over_ranks(dist, e0.elapsed_time(e1)) / e2e_steps
-    h2d = (tgt.numel() + drf.numel()) * esz
-    d2h = tok_h.numel() * 4 + len_h.numel() * 4
+    h2d = sum(t.numel() * t.element_size() for t in P["inputs"])
+    d2h = sum(o.numel() * o.element_size() for o in P["outputs"])
+    del hosts, devs
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        tgt_c, drf_c = tgt.cpu(), drf.cpu()
-        udc, uac, urc = synth.linear_uniforms(synth.linear_cases()[args.workload])
-        n = 0
-        t0 = time.perf_counter()
-        while time.perf_counter() - t0 < args.cpu_seconds and n < B:
-            _oracle_sample(case, tgt_c, drf_c, udc, uac, urc, np.arange(n, min(B, n + 4)))
-            n = min(B, n + 4)
-        dt = time.perf_counter() - t0
-        cpu = {"value": n * K / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
-               "sample": "%d of %d requests of workload %s (sample_draft + verify_linear, fp64 C oracle, "
-                         "single thread, %.1f s)" % (n, B, args.workload, dt)}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.workload in _linear_names():
+        cpu = _cpu_baseline(args, case, P)
 
     peak, peak_kind = _peaks()
-    # algorithmic bytes: sample_draft reads the draft tensor once; verify_linear reads the
-    # verifier tensor once plus, per request, the one draft row of the residual draw
-    bytes_sample = B * K * V * esz
-    bytes_verify = B * (K + 1) * V * esz + B * V * esz
-    gbs_verify = bytes_verify / (t_verify * 1e-3) / 1e9
-    gbs_sample = bytes_sample / (t_sample * 1e-3) / 1e9
-    bytes_step = (B * (K + 1) + B * K) * V * esz
-    value = world * B * K / (ms_step * 1e-3)
+    main_call = P["calls"][-1][0]
+    gbs_main = P["bytes"][main_call] / (per[main_call] * 1e-3) / 1e9
+    value = world * P["positions"] / (ms_step * 1e-3)
+    esz = P["esz"]
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16" if esz == 2 else "f32", "data": "synthetic",
-            "config": {"workload": "%s: linear verify B=%d K=%d V=%d %s, T=%g, top-p %g" % (
-                args.workload, B, K, V, "bf16" if esz == 2 else "fp32", case.temperature, case.top_p),
-                "global_batch": B * world, "block": K, "vocab": V, "parallelism": "replicas x%d" % world,
-                "l2": "inputs %.0f MB > 126 MB L2, no flush" % (bytes_step / 1e6),
-                "cuda_graph": not args.no_graph},
-            "roofline": {"bound": "hbm", "kernel": "psispec_verify_linear", "achieved": gbs_verify, "peak": peak,
-                         "unit": "GB/s", "frac": gbs_verify / peak, "peak_kind": peak_kind,
+            "config": dict({"workload": "%s: %s" % (args.workload, P["describe"]), "parallelism": "replicas x%d" % world,
+                            "l2": "inputs %.0f MB > 126 MB L2, no flush" % (P["bytes_step"] / 1e6),
+                            "cuda_graph": not args.no_graph}, **P["config"]),
+            "roofline": {"bound": "hbm", "kernel": "psispec_" + main_call, "achieved": gbs_main, "peak": peak,
+                         "unit": "GB/s", "frac": gbs_main / peak, "peak_kind": peak_kind,
                          "traffic": _traffic(args.workload)},
-            "step_gbs": bytes_step / (ms_step * 1e-3) / 1e9,
-            "calls": {"sample_draft_ms": t_sample, "sample_draft_gbs": gbs_sample, "verify_linear_ms": t_verify,
-                      "verify_linear_gbs": gbs_verify},
+            "step_gbs": P["bytes_step"] / (ms_step * 1e-3) / 1e9,
+            "calls": dict({k + "_ms": v for k, v in per.items()},
+                          **{k + "_gbs": P["bytes"][k] / (v * 1e-3) / 1e9 for k, v in per.items()}),
             "mean_accept_len": mean_accept,
-            "e2e": {"value": world * B * K / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+            "e2e": {"value": world * P["positions"] / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
             "gpu_launches": LAUNCHES_PER_STEP * args.steps,
             "clocks": clk.summary(),
@@ -341,6 +455,30 @@ def run_ours(args):
         print(json.dumps(line), flush=True)
     if dist is not None:
         dist.destroy_process_group()
+
+
+def _linear_names():
+    from lossless_speculative_sampling_b200 import synth
+
+    return set(synth.linear_cases())
+
+
+def _cpu_baseline(args, case, P):
+    """The oracle as it stands, on a bounded sample of the same workload (host cores)."""
+    from lossless_speculative_sampling_b200 import synth
+
+    B, K = case.B, case.K
+    tgt_c, drf_c = (t.cpu() for t in P["inputs"])
+    udc, uac, urc = synth.linear_uniforms(synth.linear_cases()[args.workload])
+    n = 0
+    t0 = time.perf_counter()
+    while time.perf_counter() - t0 < args.cpu_seconds and n < B:
+        _oracle_sample(case, tgt_c, drf_c, udc, uac, urc, np.arange(n, min(B, n + 4)))
+        n = min(B, n + 4)
+    dt = time.perf_counter() - t0
+    return {"value": n * K / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": "%d of %d requests of workload %s (sample_draft + verify_linear, fp64 C oracle, "
+                      "single thread, %.1f s)" % (n, B, args.workload, dt)}
 
 
 def main():
@@ -354,6 +492,7 @@ def main():
     ap.add_argument("--no-graph", action="store_true", help="launch calls directly instead of replaying CUDA graphs")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-requests", type=int, default=2)
+    ap.add_argument("--all", action="store_true", help="one line per full-size workload instead of the bench line")
     args = ap.parse_args()
     if args.impl == "reference":
         run_reference(args)

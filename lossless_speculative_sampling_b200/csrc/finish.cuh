@@ -2,14 +2,13 @@
 //
 // The streaming pass (stream_partials_kernel) reads every logits row once and leaves one
 // partial per kChunkElems-element chunk. The kernels here finish from those partials:
-//   sample_row_kernel   one warp per draft row: row statistics and the chunk holding u * Z
-//                       (chunk partials are the prefix totals), then the draw inside that
-//                       chunk; rows with a top-p cut are finished by their CTA (threshold by
-//                       radix select, draw over the row);
-//   verify_row_kernel   one warp per verifier (and streamed draft) row: statistics (top-p
-//                       threshold by the CTA), then an arrival on the request's counter; the
-//                       warp completing a request runs the accept tests, finds the first
-//                       rejection and writes the draw job;
+//   warp_sample_row     one warp per draft row (no top-p cut): row statistics and the chunk
+//                       holding u * Z (chunk partials are the prefix totals), then the draw
+//                       inside that chunk;
+//   warp_verify_row     one warp per verifier (and streamed draft) row (no top-p cut):
+//                       statistics, then an arrival on the request's counter; the warp
+//                       completing a request runs the accept tests, finds the first rejection
+//                       and writes the draw job (both run inside the row kernels of topp.cuh);
 //   draw_totals_*       one warp per (draw job, chunk) item over every SM: group and chunk
 //                       totals of the residual (or kept) weights;
 //   draw_pick_kernel    one warp per draw job: the chunk, then the 256-element group holding
@@ -251,80 +250,40 @@ __device__ __forceinline__ int warp_pick_resid(const double2* tot, int nchunks, 
   return warp_pick_totals(tot, nchunks, *use_p, u, base, target);
 }
 
-// Draft rows, kThreads / 32 per CTA. Each warp turns its row's chunk partials into the row
-// statistics, locates the chunk holding u * Z and draws inside it. Rows with a top-p cut are
-// then finished by the whole CTA, one after another: threshold by radix select, then a draw
-// over the row.
+// Warp-level finish of one draft row without a top-p cut: statistics from the chunk
+// partials, the chunk holding u * Z (chunk partials are the prefix totals), and the draw
+// inside that chunk.
 template <typename T>
-__global__ void __launch_bounds__(kThreads, 2) sample_row_kernel(const T* __restrict__ draft, int K, int V, int rows,
-                                                              const float* __restrict__ temperature,
-                                                              const float* __restrict__ top_p,
-                                                              const float* __restrict__ u,
-                                                              const Partial* __restrict__ parts,
-                                                              RowStat* __restrict__ stats,
-                                                              int32_t* __restrict__ out_tokens,
-                                                              float* __restrict__ out_q) {
-  constexpr int kRowsPerCta = kThreads / 32;
-  __shared__ ToppSmem tsm;
-  __shared__ DrawSmem dsm;
-  __shared__ RowStat cut_st[kRowsPerCta];
-  __shared__ int cut_row[kRowsPerCta];
-  __shared__ int ncut;
+__device__ void warp_sample_row(const T* __restrict__ draft, int row, int K, int V,
+                                const float* __restrict__ temperature, const float* __restrict__ u,
+                                const Partial* __restrict__ parts, RowStat* __restrict__ stats,
+                                int32_t* __restrict__ out_tokens, float* __restrict__ out_q) {
   const int lane = threadIdx.x & 31;
-  const int row = blockIdx.x * kRowsPerCta + (threadIdx.x >> 5);
+  const int b = row / K;
   const int nch = nchunks_for(V);
-  if (threadIdx.x == 0) ncut = 0;
-  __syncthreads();
-  if (row < rows) {
-    const int b = row / K;
-    const T* rp = draft + static_cast<size_t>(row) * V;
-    const Partial* pp = parts + static_cast<size_t>(row) * nch;
-    const float tp = top_p[b], ur = u[row];
-    const bool no_cut = !(tp < 1.0f);
-    RowPick r = warp_finalize_pick(pp, nch, temperature[b], ur, no_cut);
-    const RowStat st = r.st;
-    if (needs_topp(st, tp)) {
-      if (lane == 0) {
-        const int k = atomicAdd(&ncut, 1);
-        cut_row[k] = row;
-        cut_st[k] = st;
-      }
-    } else {
-      int y = -1;
-      float q = -1.0f;
-      if (st.status == 0 && st.c == 0.0f) {
-        y = st.amax;
-        q = 1.0f;
-      } else if (st.status == 0) {
-        if ((nch + 31) / 32 > kCache) r.chunk = warp_pick_chunk(pp, nch, st, ur, &r.base, &r.target);
-        JobRows<T, false> J;
-        J.init(rp, st, nullptr, st);
-        float ly = 0.0f;
-        if (r.chunk >= 0)
-          y = warp_draw_chunk(J, r.chunk * kChunkElems, min(V, (r.chunk + 1) * kChunkElems), r.base, r.target, &ly);
-        if (y >= 0) q = kept_weight(st, ly) / st.s_kept;
-      }
-      if (lane == 0) {
-        stats[row] = st;
-        out_tokens[row] = y;
-        if (out_q) out_q[row] = q;
-      }
-    }
-  }
-  __syncthreads();
-  for (int k = 0; k < ncut; ++k) {
-    const int rw = cut_row[k];
-    RowStat st = cut_st[k];
-    const T* rp = draft + static_cast<size_t>(rw) * V;
-    block_topp_select<T>(rp, V, top_p[rw / K], st, tsm);
+  const T* rp = draft + static_cast<size_t>(row) * V;
+  const Partial* pp = parts + static_cast<size_t>(row) * nch;
+  const float ur = u[row];
+  RowPick r = warp_finalize_pick(pp, nch, temperature[b], ur, true);
+  const RowStat st = r.st;
+  int y = -1;
+  float q = -1.0f;
+  if (st.status == 0 && st.c == 0.0f) {
+    y = st.amax;
+    q = 1.0f;
+  } else if (st.status == 0) {
+    if ((nch + 31) / 32 > kCache) r.chunk = warp_pick_chunk(pp, nch, st, ur, &r.base, &r.target);
     JobRows<T, false> J;
     J.init(rp, st, nullptr, st);
-    const int y = block_draw_range(J, 0, V, 0.0, -1.0, u[rw], dsm);
-    if (threadIdx.x == 0) {
-      stats[rw] = st;
-      out_tokens[rw] = y;
-      if (out_q) out_q[rw] = y >= 0 ? kept_weight(st, load_elem(rp + y)) / st.s_kept : -1.0f;
-    }
+    float ly = 0.0f;
+    if (r.chunk >= 0)
+      y = warp_draw_chunk(J, r.chunk * kChunkElems, min(V, (r.chunk + 1) * kChunkElems), r.base, r.target, &ly);
+    if (y >= 0) q = kept_weight(st, ly) / st.s_kept;
+  }
+  if (lane == 0) {
+    stats[row] = st;
+    out_tokens[row] = y;
+    if (out_q) out_q[row] = q;
   }
 }
 
@@ -349,58 +308,25 @@ struct VerifyArgs {
   Job* jobs;
 };
 
-// Verifier rows (then draft rows, when the draft tensor is streamed here), kThreads / 32 per
-// CTA. Each warp turns its row's chunk partials into the row statistics and arrives on the
-// request's counter; the warp completing a request runs its accept tests, finds the first
-// rejection and writes the draw job. Rows with a top-p cut get their threshold from the whole
-// CTA first and arrive after it.
+// Warp-level finish of one row g (verifier rows, then streamed draft rows) of a request
+// without a top-p cut: statistics from the chunk partials, then the arrival on the request's
+// counter; the warp completing the request runs its accept tests, finds the first rejection
+// and writes the draw job.
 template <typename T>
-__global__ void __launch_bounds__(kThreads) verify_row_kernel(const T* __restrict__ tgt, const T* __restrict__ drf,
-                                                              VerifyArgs a) {
-  constexpr int kRowsPerCta = kThreads / 32;
-  __shared__ ToppSmem tsm;
-  __shared__ RowStat cut_st[kRowsPerCta];
-  __shared__ int cut_row[kRowsPerCta];
-  __shared__ int ncut, sh_flag;
-  const int K = a.K, V = a.V;
-  const int rows_t = a.B * (K + 1), rows = rows_t + (a.stream_draft ? a.B * K : 0);
+__device__ void warp_verify_row(const T* __restrict__ tgt, const T* __restrict__ drf, int g, const VerifyArgs& a) {
+  const int K = a.K;
+  const int rows_t = a.B * (K + 1);
   const int per_req = (K + 1) + (a.stream_draft ? K : 0);
-  const int nch = nchunks_for(V);
-  const int g = blockIdx.x * kRowsPerCta + (threadIdx.x >> 5);  // 0 .. rows - 1: verifier rows, then draft rows
-  auto request_of = [&](int gr) { return gr < rows_t ? gr / (K + 1) : (gr - rows_t) / K; };
-  auto stat_of = [&](int gr) -> RowStat* { return gr < rows_t ? a.stats_t + gr : a.stats_d + (gr - rows_t); };
-  if (threadIdx.x == 0) ncut = 0;
-  __syncthreads();
-  if (g < rows) {
-    const int b = request_of(g);
-    const Partial* pp = g < rows_t ? a.parts_t + static_cast<size_t>(g) * nch
-                                   : a.parts_d + static_cast<size_t>(g - rows_t) * nch;
-    const RowStat st = warp_finalize_pick(pp, nch, a.temperature[b], 0.0f, false).st;
-    if (needs_topp(st, a.top_p[b])) {
-      if ((threadIdx.x & 31) == 0) {
-        const int k = atomicAdd(&ncut, 1);
-        cut_row[k] = g;
-        cut_st[k] = st;
-      }
-    } else {
-      if ((threadIdx.x & 31) == 0) *stat_of(g) = st;
-      if (warp_arrive_last(&a.cnt[b], per_req))
-        warp_decide_request<T>(b, tgt, drf, K, V, a.tokens, a.stats_t, a.stream_draft ? a.stats_d : a.dstats_in,
-                               a.u_acc, a.u_res, a.out_tokens, a.out_len, a.out_p, a.out_q, a.jobs);
-    }
-  }
-  __syncthreads();
-  for (int k = 0; k < ncut; ++k) {
-    const int gr = cut_row[k], b = request_of(gr);
-    RowStat st = cut_st[k];
-    const T* rp = gr < rows_t ? tgt + static_cast<size_t>(gr) * V : drf + static_cast<size_t>(gr - rows_t) * V;
-    block_topp_select<T>(rp, V, a.top_p[b], st, tsm);
-    if (threadIdx.x == 0) *stat_of(gr) = st;
-    if (block_arrive_last(&a.cnt[b], per_req, &sh_flag) && threadIdx.x < 32)
-      warp_decide_request<T>(b, tgt, drf, K, V, a.tokens, a.stats_t, a.stream_draft ? a.stats_d : a.dstats_in,
-                             a.u_acc, a.u_res, a.out_tokens, a.out_len, a.out_p, a.out_q, a.jobs);
-    __syncthreads();
-  }
+  const int nch = nchunks_for(a.V);
+  const bool is_draft = g >= rows_t;
+  const int row = is_draft ? g - rows_t : g;
+  const int b = is_draft ? row / K : row / (K + 1);
+  const Partial* pp = (is_draft ? a.parts_d : a.parts_t) + static_cast<size_t>(row) * nch;
+  const RowStat st = warp_finalize_pick(pp, nch, a.temperature[b], 0.0f, false).st;
+  if ((threadIdx.x & 31) == 0) (is_draft ? a.stats_d : a.stats_t)[row] = st;
+  if (warp_arrive_last(&a.cnt[b], per_req))
+    warp_decide_request<T>(b, tgt, drf, K, a.V, a.tokens, a.stats_t, a.stream_draft ? a.stats_d : a.dstats_in,
+                           a.u_acc, a.u_res, a.out_tokens, a.out_len, a.out_p, a.out_q, a.jobs);
 }
 
 // Draw jobs (the residual draw at a first rejection, or the bonus draw after a fully

@@ -9,6 +9,7 @@
 #include "linear.cuh"
 #include "sample.cuh"
 #include "stats.cuh"
+#include "topp.cuh"
 #include "tree.cuh"
 
 namespace psi {
@@ -140,7 +141,7 @@ int64_t want_slots(int64_t work_warps, int warps, Kern kernel, int block, int sm
 template <typename T>
 psispec_status launch_stream(const T* base, int64_t rows, int rows_per_req, const int32_t* row_req, int V,
                              const float* temperature, int nreq, Partial* parts, cudaStream_t st,
-                             int32_t* zero = nullptr, int nzero = 0) {
+                             const float* skip_top_p = nullptr, int32_t* zero = nullptr, int nzero = 0) {
   const int64_t chunks = rows * nchunks_for(V);
   const bool aligned = (reinterpret_cast<uintptr_t>(base) & 15u) == 0 && (int64_t(V) * sizeof(T)) % 16 == 0;
   if (aligned) {
@@ -156,10 +157,10 @@ psispec_status launch_stream(const T* base, int64_t rows, int rows_per_req, cons
     const int64_t slots = static_cast<int64_t>(sms) * (occ > 0 ? occ : 1);
     const unsigned grid = static_cast<unsigned>(want < slots ? want : slots);
     return launch(stream_partials_tma_kernel<T>, grid, kThreads, smem, st, base, rows_per_req, row_req, V, chunks,
-                  temperature, nreq, parts, zero, nzero);
+                  temperature, skip_top_p, nreq, parts, zero, nzero);
   }
   return launch(stream_partials_kernel<T>, persistent_grid(stream_partials_kernel<T>, chunks), kThreads, 0, st, base,
-                rows_per_req, row_req, V, chunks, temperature, parts, zero, nzero);
+                rows_per_req, row_req, V, chunks, temperature, skip_top_p, parts, zero, nzero);
 }
 
 // Row statistics of a [rows, V] tensor (the tree's statistics pass).
@@ -198,6 +199,16 @@ psispec_status launch_draws(const T* A, const T* Bt, int V, int njobs, const Par
                 st, A, Bt, V, njobs, parts_a, jobs, tc, tg, out_tokens);
 }
 
+// The top-p CTAs of a row kernel: persistent (one per resident slot) over the call's rows.
+template <typename Kern>
+psispec_status prepare_topp(Kern kernel, int64_t rows, unsigned* grid) {
+  const int smem = static_cast<int>(sizeof(TpSmem));
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return PSISPEC_ERR_CUDA;
+  *grid = static_cast<unsigned>(want_slots(rows, 1, kernel, kTpThreads, smem));
+  return PSISPEC_OK;
+}
+
 template <typename T>
 psispec_status sample_draft_impl(const T* draft, int B, int K, int V, const float* temperature, const float* top_p,
                                  const float* u, int32_t* out_tokens, float* out_q, RowStat* out_stats, void* ws,
@@ -206,10 +217,15 @@ psispec_status sample_draft_impl(const T* draft, int B, int K, int V, const floa
   Carver c(ws);
   SampleWs w = carve_sample(c, rows, V);
   RowStat* stats = out_stats ? out_stats : w.st.stats;
-  psispec_status s = launch_stream<T>(draft, rows, K, nullptr, V, temperature, B, w.st.parts, st);
+  // rows of requests with a top-p cut skip the streaming pass: the row kernel's top-p CTAs
+  // read them whole
+  psispec_status s = launch_stream<T>(draft, rows, K, nullptr, V, temperature, B, w.st.parts, st, top_p);
   if (s != PSISPEC_OK) return s;
-  return launch(sample_row_kernel<T>, static_cast<unsigned>((rows + kThreads / 32 - 1) / (kThreads / 32)), kThreads, 0,
-                st, draft, K, V, static_cast<int>(rows), temperature, top_p, u, w.st.parts, stats, out_tokens, out_q);
+  unsigned tgrid = 1;
+  if ((s = prepare_topp(sample_rows_kernel<T>, rows, &tgrid)) != PSISPEC_OK) return s;
+  const int warp_ctas = static_cast<int>((rows + kTpWarps - 1) / kTpWarps);
+  return launch(sample_rows_kernel<T>, warp_ctas + tgrid, kTpThreads, sizeof(TpSmem), st, draft, K, V,
+                static_cast<int>(rows), temperature, top_p, u, w.st.parts, stats, out_tokens, out_q, warp_ctas);
 }
 
 template <typename T>
@@ -242,12 +258,17 @@ psispec_status verify_linear_impl(const T* tgt, const T* drf, int B, int K, int 
   a.out_q = out_q;
   a.jobs = w.jobs;
   // the first streaming pass also clears the request arrival counters
-  psispec_status s = launch_stream<T>(tgt, rows_t, K + 1, nullptr, V, temperature, B, w.t.parts, st, w.cnt, B);
+  psispec_status s =
+      launch_stream<T>(tgt, rows_t, K + 1, nullptr, V, temperature, B, w.t.parts, st, top_p, w.cnt, B);
   if (s != PSISPEC_OK) return s;
-  if (rows_d > 0 && (s = launch_stream<T>(drf, rows_d, K, nullptr, V, temperature, B, w.d.parts, st)) != PSISPEC_OK)
+  if (rows_d > 0 &&
+      (s = launch_stream<T>(drf, rows_d, K, nullptr, V, temperature, B, w.d.parts, st, top_p)) != PSISPEC_OK)
     return s;
-  s = launch(verify_row_kernel<T>, static_cast<unsigned>((rows_t + rows_d + kThreads / 32 - 1) / (kThreads / 32)),
-             kThreads, 0, st, tgt, drf, a);
+  // one row kernel: warps for the requests without a top-p cut, whole CTAs for the others
+  unsigned tgrid = 1;
+  if ((s = prepare_topp(verify_rows_kernel<T>, rows_t + rows_d, &tgrid)) != PSISPEC_OK) return s;
+  const int warp_ctas = static_cast<int>((rows_t + rows_d + kTpWarps - 1) / kTpWarps);
+  s = launch(verify_rows_kernel<T>, warp_ctas + tgrid, kTpThreads, sizeof(TpSmem), st, tgt, drf, a, warp_ctas);
   if (s != PSISPEC_OK) return s;
   return launch_draws<T>(tgt, drf, V, B, w.t.parts, w.jobs, w.draw_tc, w.draw_tg, out_tokens, st);
 }

@@ -229,6 +229,35 @@ __device__ __forceinline__ double2 lane_group_sums(const JobRows<T, RESID>& J, c
   return make_double2(a, b);
 }
 
+// Warp-level totals of one chunk [lo, hi) (hi - lo <= kChunkElems, lo a multiple of 8): the
+// job weights (.x) and p_a (.y), summed in fp64 per lane and across lanes, with a whole batch
+// of groups in flight at once. Every lane gets them.
+template <typename T, bool RESID>
+__device__ double2 warp_chunk_totals(const JobRows<T, RESID>& J, int lo, int hi) {
+  constexpr int NB = kChunkBatch<T, RESID>;
+  const int lane = threadIdx.x & 31;
+  const bool full = J.vector_ok(lo, hi, kChunkElems);
+  double sr = 0.0, sp = 0.0;
+#pragma unroll
+  for (int g0 = 0; g0 < kChunkGroups; g0 += NB) {
+    Raw8<T, RESID> x[NB];
+    if (full) {
+#pragma unroll
+      for (int g = 0; g < NB; ++g) J.load_full(lo + (g0 + g) * kGroup + lane * 8, x[g]);
+    } else {
+#pragma unroll
+      for (int g = 0; g < NB; ++g) J.load(lo + (g0 + g) * kGroup + lane * 8, hi, x[g]);
+    }
+#pragma unroll
+    for (int g = 0; g < NB; ++g) {
+      const double2 t = lane_group_sums(J, x[g]);
+      sr += t.x;
+      sp += t.y;
+    }
+  }
+  return make_double2(warp_sum(sr), warp_sum(sp));
+}
+
 // Reduce-scatter of eight per-lane values: lane l ends with the warp total of value
 // (l >> 2) & 7 (halves exchanged over lane bits 4, 3, 2, then summed over bits 1, 0).
 __device__ __forceinline__ double warp_reduce_scatter8(const double (&v)[8]) {

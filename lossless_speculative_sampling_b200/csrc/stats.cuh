@@ -25,6 +25,14 @@ __device__ __forceinline__ float temp_scale(float T) {
   return T > 0.0f && T < INFINITY ? static_cast<float>(1.4426950408889634 / static_cast<double>(T)) : 0.0f;
 }
 
+// Scale c of a request's rows for the streaming pass: -1 marks rows that the pass leaves to
+// the top-p row kernel (top_p given, below 1, and a positive temperature).
+__device__ __forceinline__ float stream_scale(const float* __restrict__ temperature, const float* __restrict__ top_p,
+                                              int req) {
+  const float c = temp_scale(temperature[req]);
+  return (top_p != nullptr && c != 0.0f && top_p[req] < 1.0f) ? -1.0f : c;
+}
+
 // Request of a row: rows_per_req consecutive rows per request, or an explicit table.
 __device__ __forceinline__ int row_request(int row, int rows_per_req, const int32_t* __restrict__ row_req) {
   return row_req ? row_req[row] : row / rows_per_req;
@@ -145,13 +153,15 @@ __device__ __forceinline__ Partial warp_chunk_partial(const T* __restrict__ row,
 }
 
 // The streaming pass: persistent warps over every chunk of a [rows, V] tensor, each chunk
-// read once, one partial per chunk (parts[row * nchunks + chunk]). CTA 0 also clears the
-// nzero arrival counters at `zero` that the call's later kernels use.
+// read once, one partial per chunk (parts[row * nchunks + chunk]). With skip_top_p set, the
+// rows of requests with a top-p cut are left alone (the top-p row kernel reads them). CTA 0
+// also clears the nzero arrival counters at `zero` that the call's later kernels use.
 template <typename T>
 __global__ void __launch_bounds__(kThreads, 4) stream_partials_kernel(const T* __restrict__ base, int rows_per_req,
                                                                     const int32_t* __restrict__ row_req, int V,
                                                                     int64_t total_chunks,
                                                                     const float* __restrict__ temperature,
+                                                                    const float* __restrict__ skip_top_p,
                                                                     Partial* __restrict__ parts,
                                                                     int32_t* __restrict__ zero, int nzero) {
   if (blockIdx.x == 0)
@@ -165,11 +175,14 @@ __global__ void __launch_bounds__(kThreads, 4) stream_partials_kernel(const T* _
   const int drow = static_cast<int>(nwarps / nch), dchunk = static_cast<int>(nwarps - static_cast<int64_t>(drow) * nch);
 #pragma unroll 1
   for (; g < total_chunks; g += nwarps) {
-    const float c = temp_scale(temperature[row_request(row, rows_per_req, row_req)]);
-    const T* rp = base + static_cast<size_t>(row) * V;
-    const int c0 = chunk * kChunkElems, c1 = min(V, c0 + kChunkElems);
-    const Partial p = c == 0.0f ? warp_chunk_partial<T, true>(rp, c0, c1, c) : warp_chunk_partial<T, false>(rp, c0, c1, c);
-    if ((threadIdx.x & 31) == 0) parts[g] = p;
+    const float c = stream_scale(temperature, skip_top_p, row_request(row, rows_per_req, row_req));
+    if (c >= 0.0f) {
+      const T* rp = base + static_cast<size_t>(row) * V;
+      const int c0 = chunk * kChunkElems, c1 = min(V, c0 + kChunkElems);
+      const Partial p =
+          c == 0.0f ? warp_chunk_partial<T, true>(rp, c0, c1, c) : warp_chunk_partial<T, false>(rp, c0, c1, c);
+      if ((threadIdx.x & 31) == 0) parts[g] = p;
+    }
     row += drow;
     chunk += dchunk;
     if (chunk >= nch) {
@@ -335,7 +348,8 @@ __global__ void __launch_bounds__(kThreads) stream_partials_tma_kernel(const T* 
                                                                         const int32_t* __restrict__ row_req, int V,
                                                                         int64_t total_chunks,
                                                                         const float* __restrict__ temperature,
-                                                                        int nreq, Partial* __restrict__ parts,
+                                                                        const float* __restrict__ skip_top_p, int nreq,
+                                                                        Partial* __restrict__ parts,
                                                                         int32_t* __restrict__ zero, int nzero) {
   if (blockIdx.x == 0)
     for (int i = threadIdx.x; i < nzero; i += blockDim.x) zero[i] = 0;
@@ -344,7 +358,7 @@ __global__ void __launch_bounds__(kThreads) stream_partials_tma_kernel(const T* 
   __shared__ float scale[kScaleTable];
   const bool table = nreq <= kScaleTable;
   if (table)
-    for (int i = threadIdx.x; i < nreq; i += kThreads) scale[i] = temp_scale(temperature[i]);
+    for (int i = threadIdx.x; i < nreq; i += kThreads) scale[i] = stream_scale(temperature, skip_top_p, i);
   __syncthreads();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   unsigned char* ring = ring_smem + warp * kRing * kStageBytes<T>;
@@ -371,8 +385,12 @@ __global__ void __launch_bounds__(kThreads) stream_partials_tma_kernel(const T* 
   int row = static_cast<int>(g0 / nch), chunk = static_cast<int>(g0 - static_cast<int64_t>(row) * nch);
   int irow = row, ichunk = chunk;  // cursor of the next copy to issue
   int64_t gi = g0;
+  auto scale_of = [&](int r) {
+    const int req = row_request(r, rows_per_req, row_req);
+    return table ? scale[req] : stream_scale(temperature, skip_top_p, req);
+  };
   auto issue = [&](int i) {  // copy of this warp's i-th chunk into stage i % kRing (lane 0)
-    if (gi < total_chunks) {
+    if (gi < total_chunks && scale_of(irow) >= 0.0f) {
       const int c0 = ichunk * kChunkElems, n = min(V - c0, kChunkElems);
       const uint32_t bytes = static_cast<uint32_t>(n) * sizeof(T);
       uint64_t* b = &bar[i % kRing];
@@ -385,19 +403,25 @@ __global__ void __launch_bounds__(kThreads) stream_partials_tma_kernel(const T* 
   if (lane == 0)
     for (int i = 0; i < kRing - 1; ++i) issue(i);
   int i = 0;
+  uint32_t phase_bits = 0u;  // parity of each stage's next completion (stages of skipped rows do not flip)
   for (int64_t g = g0; g < total_chunks; g += nwarps, ++i) {
     __syncwarp();  // every lane is done with the stage that the next copy overwrites
     if (lane == 0) issue(i + kRing - 1);
     const int c0 = chunk * kChunkElems, n = min(V - c0, kChunkElems);
-    const int req = row_request(row, rows_per_req, row_req);
-    const float c = table ? scale[req] : temp_scale(temperature[req]);
-    const bool landed = mbar_wait_bounded(&bar[i % kRing], static_cast<uint32_t>((i / kRing) & 1));
+    const float c = scale_of(row);
+    if (c < 0.0f) {  // a row left to the top-p row kernel
+      advance(row, chunk);
+      continue;
+    }
+    const int st = i % kRing;
+    const bool landed = mbar_wait_bounded(&bar[st], (phase_bits >> st) & 1u);
+    phase_bits ^= 1u << st;
     if (!__all_sync(0xffffffffu, landed)) {
       // a copy that never completed: report this chunk as a data error and stop streaming
       if (lane == 0) parts[g] = Partial{0.0, NAN, 0, 1, 0};
       return;
     }
-    const T* sp = reinterpret_cast<const T*>(ring + (i % kRing) * kStageBytes<T>);
+    const T* sp = reinterpret_cast<const T*>(ring + st * kStageBytes<T>);
     const Partial p = c == 0.0f ? warp_chunk_partial_smem<T, true>(sp, c0, n, c)
                                 : warp_chunk_partial_smem<T, false>(sp, c0, n, c);
     if (lane == 0) parts[g] = p;
@@ -588,20 +612,91 @@ __device__ __forceinline__ bool needs_topp(const RowStat& st, float tp) {
   return st.status == 0 && st.c != 0.0f && tp < 1.0f;
 }
 
-// Shared memory of a block-level top-p selection.
-struct ToppSmem {
+// Top-p threshold (value-threshold reading: keep every token whose logit is at least the
+// largest logit value t with mass(l >= t) >= top_p, ties kept together).
+//
+// First pass: every element of the row falls into one of kToppBins value bins, bin b holding
+// the logits whose log2 weight (x - m) c lies within 1/16 of -b/8 (the last bin collects all
+// smaller values). An element adds its weight relative to the bin's reference weight 2^(-b/8),
+// 2^((x - m) c + b/8) in [2^(-1/16), 2^(1/16)], as a fixed-point integer with 22 fractional
+// bits, to per-warp 64-bit histograms: sums are exact and independent of the order. The bin
+// holding the threshold is the first, scanning from the maximum, whose cumulative mass
+// reaches top_p of the total. Second, the bin's elements alone (no other element needs an
+// exponential) go through a most-significant-digit radix select on their order-preserving
+// keys, 8 bits per pass, with the same fixed-point masses; the key of the threshold value is
+// exact after two passes for bf16 rows (four for fp32).
+constexpr int kToppBins = 256;
+constexpr int kToppWarps = 8;  // histograms per CTA (blockDim.x <= 32 * kToppWarps)
+
+// Shared memory of the general radix select (block_topp_radix).
+struct RadixSmem {
   double hmass[256];
   int hcnt[256];
   uint32_t prefix;
   double above, bucket;
 };
 
-// Block-level top-p threshold of row rp under statistics st (m, c, s set): radix select on the
-// 32-bit keys, most significant digit first, with the fp64 mass of every digit. For bf16 rows
-// the two top digits already separate every distinct value. Sets st.tau and st.s_kept (in
-// every thread).
+struct ToppSmem {
+  unsigned long long h[kToppWarps][kToppBins];
+  double mass[kToppBins];
+  double above, total, target;
+  uint32_t prefix;
+  int bin, fallback;
+  RadixSmem radix;
+};
+
+// Value bin of logit x under (m, c) and its fixed-point mass relative to the bin's reference
+// weight; identical arithmetic in every pass.
+__device__ __forceinline__ void topp_bin(float x, float m, float c, int& b, uint32_t& u) {
+  const float d = (x - m) * c;                                // log2 weight, <= 0
+  const float t = fminf(d * -8.0f, 4096.0f);                  // -8 d, capped (also for -inf)
+  const float r = t + 12582912.0f;                            // round to an integer (1.5 * 2^23 trick)
+  b = min(__float_as_int(r) - __float_as_int(12582912.0f), kToppBins - 1);
+  const float bf = fminf(r - 12582912.0f, static_cast<float>(kToppBins - 1));
+  const float y = ex2(fmaf(bf, 0.125f, d));                   // 2^(d + b/8)
+  u = __float_as_uint(y + 2.0f) - 0x40000000u;                // y * 2^22, rounded to nearest
+}
+
+// Bin of x only (no exponential).
+__device__ __forceinline__ int topp_bin_only(float x, float m, float c) {
+  const float t = fminf((x - m) * c * -8.0f, 4096.0f);
+  return min(__float_as_int(t + 12582912.0f) - __float_as_int(12582912.0f), kToppBins - 1);
+}
+
+// 2^(-b/8) in fp64.
+__device__ __forceinline__ double topp_ref(int b) { return ldexp(exp2(-static_cast<double>(b & 7) * 0.125), -(b >> 3)); }
+
+// Visit every element of row [0, V) with f(x, v); vectorised body with kLoads 16-byte loads in
+// flight per thread, scalar edges.
+template <typename T, int kLoads, typename F>
+__device__ __forceinline__ void for_each_elem_batched(const T* __restrict__ row, int V, F&& f) {
+  constexpr int N = Vec<T>::N;
+  int a0, a1;
+  vec_range(row, 0, V, a0, a1);
+  for (int v = threadIdx.x; v < a0; v += blockDim.x) f(load_elem(row + v));
+  for (int v = a1 + threadIdx.x; v < V; v += blockDim.x) f(load_elem(row + v));
+  const int step = blockDim.x * N;
+  for (int v = a0 + threadIdx.x * N; v < a1; v += kLoads * step) {
+    uint4 raw[kLoads];
+#pragma unroll
+    for (int i = 0; i < kLoads; ++i)
+      if (v + i * step < a1) raw[i] = __ldg(reinterpret_cast<const uint4*>(row + v + i * step));
+#pragma unroll
+    for (int i = 0; i < kLoads; ++i) {
+      if (v + i * step < a1) {
+        float x[8];
+        Vec<T>::unpack(raw[i], x);
+#pragma unroll
+        for (int k = 0; k < N; ++k) f(x[k]);
+      }
+    }
+  }
+}
+
+// General top-p select (fallback when the threshold lies below the first pass's value range):
+// radix select on the 32-bit keys with fp64 atomics.
 template <typename T>
-__device__ void block_topp_select(const T* __restrict__ rp, int V, float tp, RowStat& st, ToppSmem& sm) {
+__device__ void block_topp_radix(const T* __restrict__ rp, int V, float tp, RowStat& st, RadixSmem& sm) {
   const float M = st.m, c = st.c;
   const double target = static_cast<double>(tp) * static_cast<double>(st.s);
   const int levels = sizeof(T) == 2 ? 2 : 4;
@@ -642,6 +737,121 @@ __device__ void block_topp_select(const T* __restrict__ rp, int V, float tp, Row
   }
   st.tau = sm.prefix;
   st.s_kept = static_cast<float>(sm.above + sm.bucket);
+  __syncthreads();
+}
+
+// Block-level top-p threshold of row rp under statistics st (m, c, s set); sets st.tau and
+// st.s_kept in every thread. Any block size up to 32 * kToppWarps threads.
+template <typename T>
+__device__ void block_topp_select(const T* __restrict__ rp, int V, float tp, RowStat& st, ToppSmem& sm) {
+  const float m = st.m, c = st.c;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  unsigned long long* hw = sm.h[warp];
+  for (int i = threadIdx.x; i < kToppWarps * kToppBins; i += blockDim.x) (&sm.h[0][0])[i] = 0ull;
+  __syncthreads();
+  for_each_elem_batched<T, 4>(rp, V, [&](float x) {
+    int b;
+    uint32_t u;
+    topp_bin(x, m, c, b, u);
+    if (u != 0u) atomicAdd(&hw[b], static_cast<unsigned long long>(u));
+  });
+  __syncthreads();
+  for (int b = threadIdx.x; b < kToppBins; b += blockDim.x) {
+    unsigned long long t = 0ull;
+    for (int w = 0; w < nw; ++w) t += sm.h[w][b];
+    sm.mass[b] = static_cast<double>(t) * topp_ref(b);
+  }
+  __syncthreads();
+  if (warp == 0) {
+    // bins of lane l: [8l, 8l + 8) (kToppBins == 256)
+    double mine = 0.0;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) mine += sm.mass[lane * 8 + k];
+    double incl = mine;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const double y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    double excl = __shfl_up_sync(0xffffffffu, incl, 1);
+    if (lane == 0) excl = 0.0;
+    const double total = __shfl_sync(0xffffffffu, incl, 31);
+    const double target = static_cast<double>(tp) * total;
+    const unsigned hit = __ballot_sync(0xffffffffu, incl >= target && mine > 0.0);
+    const int src = hit ? __ffs(hit) - 1 : 31 - __clz(__ballot_sync(0xffffffffu, mine > 0.0));
+    if (lane == src) {
+      double run = excl;
+      int pick = -1;
+      double before = excl;
+      for (int k = 0; k < 8; ++k) {
+        const double mk = sm.mass[lane * 8 + k];
+        if (mk > 0.0) {
+          pick = lane * 8 + k;
+          before = run;
+          if (run + mk >= target) break;
+        }
+        run += mk;
+      }
+      sm.bin = pick;
+      sm.above = before;
+      sm.total = total;
+      sm.target = target;
+      sm.prefix = 0u;
+      sm.fallback = pick == kToppBins - 1;
+    }
+  }
+  __syncthreads();
+  if (sm.fallback) {
+    block_topp_radix<T>(rp, V, tp, st, sm.radix);
+    return;
+  }
+  // radix select on the keys of bin sm.bin's elements, 8 bits per pass
+  const int bstar = sm.bin;
+  const double ref = topp_ref(bstar);
+  const int levels = sizeof(T) == 2 ? 2 : 4;
+  for (int lv = 0; lv < levels; ++lv) {
+    const int shift = 24 - 8 * lv;
+    for (int i = threadIdx.x; i < nw * 256; i += blockDim.x) (&sm.h[0][0])[(i / 256) * kToppBins + (i % 256)] = 0ull;
+    __syncthreads();
+    const uint32_t prefix = sm.prefix;
+    for_each_elem_batched<T, 4>(rp, V, [&](float x) {
+      if (topp_bin_only(x, m, c) != bstar) return;
+      const uint32_t k = fkey(x);
+      if (lv != 0 && (k >> (shift + 8)) != (prefix >> (shift + 8))) return;
+      int b;
+      uint32_t u;
+      topp_bin(x, m, c, b, u);
+      if (u != 0u) atomicAdd(&hw[(k >> shift) & 255], static_cast<unsigned long long>(u));
+    });
+    __syncthreads();
+    for (int d = threadIdx.x; d < 256; d += blockDim.x) {
+      unsigned long long t = 0ull;
+      for (int w = 0; w < nw; ++w) t += sm.h[w][d];
+      sm.mass[d] = static_cast<double>(t) * ref;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      // digits from the largest key down: the first whose cumulative mass reaches the target
+      double run = sm.above;
+      int pick = -1, last = -1;
+      double before = run;
+      for (int d = 255; d >= 0; --d) {
+        const double md = sm.mass[d];
+        if (md <= 0.0) continue;
+        last = d;
+        before = run;
+        if (run + md >= sm.target) { pick = d; break; }
+        run += md;
+      }
+      if (pick < 0) pick = last;  // rounding: the bin's smallest digit with mass
+      sm.prefix = prefix | (static_cast<uint32_t>(pick < 0 ? 0 : pick) << shift);
+      sm.above = before;
+      if (lv == levels - 1) sm.mass[0] = before + (pick < 0 ? 0.0 : sm.mass[pick]);
+    }
+    __syncthreads();
+  }
+  st.tau = sm.prefix;
+  st.s_kept = static_cast<float>(static_cast<double>(st.s) * (sm.mass[0] / sm.total));
   __syncthreads();
 }
 

@@ -1,0 +1,475 @@
+// topp.cuh -- rows of requests with a top-p cut: statistics, threshold and (draft rows) draw,
+// one CTA per row.
+//
+// The cut keeps every token whose logit is at least tau, the largest logit value t of the row
+// with mass(l >= t) >= top_p (review page of arXiv 2609.04010: the samplers take --top-p
+// with --temperature; ties are kept together), and renormalises over the kept set.
+//
+// A CTA reads its row once from HBM and then, while the row is still in L2:
+//   A  maximum m (NaN-propagating; bf16 pairs compared packed);
+//   B  value histogram: bin b holds the logits with (x - m) c within 1/4 of -b/2; every element
+//      adds its weight relative to the bin's reference weight 2^(-b/2), a number in
+//      [2^(-1/4), 2^(1/4)], as a fixed-point integer with 20 fractional bits to a
+//      thread-private 32-bit counter (conflict-free shared-memory reductions, exact and
+//      order-independent). The bin totals give the normaliser s and the bin holding tau;
+//   C  most-significant-digit select on the order-preserving keys of that bin's elements
+//      only (6 bits per pass, the same thread-private counters and fixed-point masses): tau
+//      exactly, and the kept mass;
+//   D  (draft rows) per-chunk totals of the kept weights, then the inverse-CDF draw inside the
+//      chunk holding u * Z.
+// Rows too long for exact 32-bit counters, or whose threshold lies below the histogram's
+// range, take the general radix select (block_topp_radix).
+#pragma once
+
+#include "common.cuh"
+#include "finish.cuh"
+#include "linear.cuh"
+#include "sample.cuh"
+#include "stats.cuh"
+
+namespace psi {
+
+constexpr int kTpThreads = 256;
+constexpr int kTpWarps = kTpThreads / 32;
+constexpr int kTpBins = 64;                                  // half log2 units below the maximum
+constexpr int kTpMaxV = kTpThreads * 2048;                   // counters stay below 2^32 up to this V
+constexpr int kTpMaxChunks = (kTpMaxV + kChunkElems - 1) / kChunkElems;
+
+struct TpSmem {
+  uint32_t priv[kTpBins][kTpThreads];             // thread-private bin (pass B) or digit (pass C) counters
+  double mass[kTpBins];                           // bin or digit masses
+  double ctot[kTpMaxChunks];                      // kept weight per chunk (pass D)
+  float fred[kTpWarps];
+  RowStat st;
+  double above, total, target;
+  uint32_t prefix;
+  int bin, fallback;
+  int y, flag;
+  double base, tgt;
+  int chunk;
+  RadixSmem radix;  // the general select
+  DrawSmem draw;    // the general draw
+};
+
+// Bin and fixed-point mass of logit x (identical arithmetic in passes B and C).
+__device__ __forceinline__ void tp_bin(float x, float m, float c, int& b, uint32_t& u) {
+  const float d = (x - m) * c;                               // log2 weight, <= 0
+  const float t = fminf(d * -2.0f, 4096.0f);                 // -2 d, capped (also for -inf)
+  const float r = t + 12582912.0f;                           // rounded to an integer (1.5 * 2^23)
+  b = min(__float_as_int(r) - __float_as_int(12582912.0f), kTpBins - 1);
+  const float bf = fminf(r - 12582912.0f, static_cast<float>(kTpBins - 1));
+  const float y = ex2(fmaf(bf, 0.5f, d));                    // 2^(d + b/2)
+  u = __float_as_uint(y + 8.0f) - __float_as_uint(8.0f);     // y * 2^20, rounded to nearest
+}
+
+__device__ __forceinline__ int tp_bin_only(float x, float m, float c) {
+  const float t = fminf((x - m) * c * -2.0f, 4096.0f);
+  return min(__float_as_int(t + 12582912.0f) - __float_as_int(12582912.0f), kTpBins - 1);
+}
+
+// 2^(-b/2) * 2^-20 in fp64: the weight of one fixed-point unit of bin b.
+__device__ __forceinline__ double tp_unit(int b) {
+  return ldexp((b & 1) ? 0.70710678118654752440 : 1.0, -(b >> 1) - 20);
+}
+
+// Visit the elements of row [0, V) of this thread: f(x) per element; 16-byte vector loads,
+// kLoads of them in flight.
+template <typename T, int kLoads, typename F>
+__device__ __forceinline__ void tp_for_each(const T* __restrict__ row, int V, F&& f) {
+  constexpr int N = Vec<T>::N;
+  int a0, a1;
+  vec_range(row, 0, V, a0, a1);
+  for (int v = threadIdx.x; v < a0; v += blockDim.x) f(load_elem(row + v));
+  for (int v = a1 + threadIdx.x; v < V; v += blockDim.x) f(load_elem(row + v));
+  const int step = blockDim.x * N;
+  for (int v = a0 + threadIdx.x * N; v < a1; v += kLoads * step) {
+    uint4 raw[kLoads];
+#pragma unroll
+    for (int i = 0; i < kLoads; ++i)
+      if (v + i * step < a1) raw[i] = __ldcg(reinterpret_cast<const uint4*>(row + v + i * step));
+#pragma unroll
+    for (int i = 0; i < kLoads; ++i) {
+      if (v + i * step < a1) {
+        float x[8];
+        Vec<T>::unpack(raw[i], x);
+#pragma unroll
+        for (int k = 0; k < N; ++k) f(x[k]);
+      }
+    }
+  }
+}
+
+// Pass A: NaN-propagating maximum of the row (every thread gets it).
+template <typename T>
+__device__ float tp_row_max(const T* __restrict__ row, int V, TpSmem& sm) {
+  constexpr int N = Vec<T>::N;
+  constexpr int kLoads = 4;
+  int a0, a1;
+  vec_range(row, 0, V, a0, a1);
+  float m = -INFINITY;
+  for (int v = threadIdx.x; v < a0; v += blockDim.x) m = fmax_nan(m, load_elem(row + v));
+  for (int v = a1 + threadIdx.x; v < V; v += blockDim.x) m = fmax_nan(m, load_elem(row + v));
+  const int step = blockDim.x * N;
+  uint32_t pm = 0xFF80FF80u;  // packed bf16 pair (-inf, -inf)
+  for (int v = a0 + threadIdx.x * N; v < a1; v += kLoads * step) {
+    uint4 raw[kLoads];
+#pragma unroll
+    for (int i = 0; i < kLoads; ++i)
+      if (v + i * step < a1) raw[i] = __ldg(reinterpret_cast<const uint4*>(row + v + i * step));
+#pragma unroll
+    for (int i = 0; i < kLoads; ++i) {
+      if (v + i * step < a1) {
+        if constexpr (sizeof(T) == 2) {
+          pm = bmax2(pm, bmax2(bmax2(raw[i].x, raw[i].y), bmax2(raw[i].z, raw[i].w)));
+        } else {
+          m = fmax_nan(m, fmax_nan(fmax_nan(__uint_as_float(raw[i].x), __uint_as_float(raw[i].y)),
+                                   fmax_nan(__uint_as_float(raw[i].z), __uint_as_float(raw[i].w))));
+        }
+      }
+    }
+  }
+  if constexpr (sizeof(T) == 2) m = fmax_nan(m, fmax_nan(__uint_as_float(pm << 16), __uint_as_float(pm & 0xFFFF0000u)));
+  m = warp_max(m);
+  __syncthreads();
+  if ((threadIdx.x & 31) == 0) sm.fred[threadIdx.x >> 5] = m;
+  __syncthreads();
+  float r = sm.fred[0];
+  for (int w = 1; w < kTpWarps; ++w) r = fmax_nan(r, sm.fred[w]);
+  return r;
+}
+
+// Passes A-C for one row: its statistics with the top-p threshold (every thread gets them).
+template <typename T>
+__device__ RowStat tp_row_stats(const T* __restrict__ row, int V, float Tv, float tp, TpSmem& sm) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  RowStat st;
+  st.c = temp_scale(Tv);
+  st.m = tp_row_max(row, V, sm);
+  st.s = 1.0f;
+  st.s_kept = 1.0f;
+  st.tau = 0u;
+  st.amax = -1;
+  st.pad = 0;
+  st.status = (st.m > -INFINITY && st.m < INFINITY && Tv >= 0.0f && Tv < INFINITY) ? 0 : 1;
+  if (st.status != 0) return st;
+  const float m = st.m, c = st.c;
+  if (V > kTpMaxV) {
+    // general path: normaliser by a block reduction, then the general select
+    double s = 0.0;
+    tp_for_each<T, 4>(row, V, [&](float x) { s += static_cast<double>(ex2((x - m) * c)); });
+    __syncthreads();
+    s = block_sum(s, reinterpret_cast<double*>(&sm.mass[0]));
+    st.s = static_cast<float>(s);
+    block_topp_radix<T>(row, V, tp, st, sm.radix);
+    return st;
+  }
+  // pass B: thread-private fixed-point bin masses
+#pragma unroll
+  for (int b = 0; b < kTpBins; ++b) sm.priv[b][threadIdx.x] = 0u;
+  tp_for_each<T, 4>(row, V, [&](float x) {
+    int b;
+    uint32_t u;
+    tp_bin(x, m, c, b, u);
+    atomicAdd(&sm.priv[b][threadIdx.x], u);  // a reduction (no return value): no chain through memory
+  });
+  __syncthreads();
+  // bin totals: warp w reduces bins w, w + kTpWarps, ...
+  for (int b = warp; b < kTpBins; b += kTpWarps) {
+    unsigned long long t = 0ull;
+    for (int j = lane; j < kTpThreads; j += 32) t += sm.priv[b][j];
+#pragma unroll
+    for (int o = 16; o; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+    if (lane == 0) sm.mass[b] = static_cast<double>(t) * tp_unit(b);
+  }
+  __syncthreads();
+  if (warp == 0) {
+    static_assert(kTpBins == 64, "two bins per lane");
+    const double m0 = sm.mass[2 * lane], m1 = sm.mass[2 * lane + 1];
+    const double mine = m0 + m1;
+    double incl = mine;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const double y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    double excl = __shfl_up_sync(0xffffffffu, incl, 1);
+    if (lane == 0) excl = 0.0;
+    const double total = __shfl_sync(0xffffffffu, incl, 31);
+    const double target = static_cast<double>(tp) * total;
+    const unsigned hit = __ballot_sync(0xffffffffu, incl >= target && mine > 0.0);
+    const unsigned pos = __ballot_sync(0xffffffffu, mine > 0.0);
+    const int src = hit ? __ffs(hit) - 1 : 31 - __clz(pos);
+    if (lane == src) {
+      int pick;
+      double before;
+      if (m0 > 0.0 && (excl + m0 >= target || m1 <= 0.0)) {
+        pick = 2 * lane;
+        before = excl;
+      } else {
+        pick = 2 * lane + 1;
+        before = excl + m0;
+      }
+      sm.bin = pick;
+      sm.above = before;
+      sm.total = total;
+      sm.target = target;
+      sm.prefix = 0u;
+      sm.fallback = pick == kTpBins - 1;
+    }
+  }
+  __syncthreads();
+  st.s = static_cast<float>(sm.total);
+  if (sm.fallback) {
+    block_topp_radix<T>(row, V, tp, st, sm.radix);
+    return st;
+  }
+  // pass C: inside bin b*, most-significant-digit select on the element keys, 6 bits of
+  // (key - klo) per pass, with the thread-private counters of pass B. [klo, khi] covers the
+  // bin's value range widened by a few representable values; an element of the bin outside
+  // it (which the widening rules out) sends the row to the general select.
+  const int bstar = sm.bin;
+  const double unit = tp_unit(bstar);
+  constexpr int kKeyShift = sizeof(T) == 2 ? 16 : 0;  // bf16 logits differ in the top 16 key bits only
+  const float xlo = m - (static_cast<float>(bstar) + 0.51f) / (2.0f * c);
+  const float xhi = bstar == 0 ? m : m - (static_cast<float>(bstar) - 0.51f) / (2.0f * c);
+  const uint32_t klo0 = fkey(xlo) >> kKeyShift, khi0 = fkey(xhi) >> kKeyShift;
+  const uint32_t klo = klo0 > 2u ? klo0 - 2u : 0u;
+  const uint32_t kmax = sizeof(T) == 2 ? 0xFFFFu : 0xFFFFFFFFu;
+  const uint32_t khi = khi0 < kmax - 2u ? khi0 + 2u : kmax;
+  const uint32_t span = khi - klo;  // largest offset
+  int levels = 1;
+  while (levels < 6 && (span >> (6 * levels)) != 0u) ++levels;
+  uint32_t prefix = 0u;  // digits chosen so far (offset >> (6 * remaining levels))
+  bool outside = false;
+  for (int lv = 0; lv < levels; ++lv) {
+    const int shift = 6 * (levels - 1 - lv);
+#pragma unroll
+    for (int d = 0; d < 64; ++d) sm.priv[d][threadIdx.x] = 0u;
+    tp_for_each<T, 4>(row, V, [&](float x) {
+      if (tp_bin_only(x, m, c) != bstar) return;
+      const uint32_t k = fkey(x) >> kKeyShift;
+      if (k < klo || k > khi) {
+        outside = true;
+        return;
+      }
+      const uint32_t off = k - klo;
+      if (shift + 6 < 32 && (off >> (shift + 6)) != prefix) return;
+      int b;
+      uint32_t u;
+      tp_bin(x, m, c, b, u);
+      atomicAdd(&sm.priv[(off >> shift) & 63u][threadIdx.x], u);
+    });
+    if (__syncthreads_or(outside)) {
+      if (threadIdx.x == 0) sm.fallback = 1;
+      break;
+    }
+    for (int d = warp; d < 64; d += kTpWarps) {
+      unsigned long long t = 0ull;
+      for (int j = lane; j < kTpThreads; j += 32) t += sm.priv[d][j];
+#pragma unroll
+      for (int o = 16; o; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+      if (lane == 0) sm.mass[d] = static_cast<double>(t) * unit;
+    }
+    __syncthreads();
+    if (warp == 0) {
+      // digits from the largest key down: lane l holds digits 63 - 2l and 62 - 2l
+      const double m0 = sm.mass[63 - 2 * lane], m1 = sm.mass[62 - 2 * lane];
+      const double mine = m0 + m1;
+      double incl = mine;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const double y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      double excl = __shfl_up_sync(0xffffffffu, incl, 1);
+      if (lane == 0) excl = 0.0;
+      const double above = sm.above, target = sm.target;
+      const unsigned hit = __ballot_sync(0xffffffffu, above + incl >= target && mine > 0.0);
+      const unsigned pos = __ballot_sync(0xffffffffu, mine > 0.0);
+      // rounding can leave the target unreached: the bin's smallest key with mass then
+      const int src = hit ? __ffs(hit) - 1 : 31 - __clz(pos);
+      if (lane == src) {
+        int pick;
+        double before;
+        if (m0 > 0.0 && (above + excl + m0 >= target || m1 <= 0.0)) {
+          pick = 63 - 2 * lane;
+          before = above + excl;
+        } else {
+          pick = 62 - 2 * lane;
+          before = above + excl + m0;
+        }
+        sm.bin = pick;  // the chosen digit
+        sm.above = before;
+        sm.base = before + (pick == 63 - 2 * lane ? m0 : m1);
+      }
+    }
+    __syncthreads();
+    prefix = (prefix << 6) | static_cast<uint32_t>(sm.bin);
+  }
+  if (sm.fallback) {
+    __syncthreads();
+    block_topp_radix<T>(row, V, tp, st, sm.radix);
+    return st;
+  }
+  st.tau = (klo + prefix) << kKeyShift;
+  st.s_kept = static_cast<float>(sm.base);
+  __syncthreads();
+  return st;
+}
+
+// Pass D: inverse-CDF draw with uniform u over the kept weights of the row, in vocabulary
+// order (the first index whose inclusive prefix exceeds u * Z). Returns the token to every
+// thread and, in *q, its kept probability.
+template <typename T>
+__device__ int tp_row_draw(const T* __restrict__ row, int V, const RowStat& st, float u, TpSmem& sm, float* q) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nch = nchunks_for(V);
+  JobRows<T, false> J;
+  J.init(row, st, nullptr, st);
+  if (V > kTpMaxV) {  // rows beyond the chunk table: the general block draw
+    const int y = block_draw_range(J, 0, V, 0.0, -1.0, u, sm.draw);
+    *q = y >= 0 ? kept_weight(st, load_elem(row + y)) / st.s_kept : -1.0f;
+    return y;
+  }
+  for (int ch = warp; ch < nch; ch += kTpWarps) {
+    const double2 t = warp_chunk_totals(J, ch * kChunkElems, min(V, (ch + 1) * kChunkElems));
+    if (lane == 0) sm.ctot[ch] = t.x;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    // lane l owns the contiguous chunks [l q, l q + q)
+    const int qn = (nch + 31) / 32;
+    const int i0 = min(nch, lane * qn), i1 = min(nch, i0 + qn);
+    double mine = 0.0;
+    for (int i = i0; i < i1; ++i) mine += sm.ctot[i];
+    double incl = mine;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const double y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    double excl = __shfl_up_sync(0xffffffffu, incl, 1);
+    if (lane == 0) excl = 0.0;
+    const double target = static_cast<double>(u) * __shfl_sync(0xffffffffu, incl, 31);
+    int sel = -1, last = -1;
+    double b = 0.0, C = excl, blast = 0.0;
+    bool open = excl <= target && target < incl;
+    for (int i = i0; i < i1; ++i) {
+      const double w = sm.ctot[i];
+      if (w > 0.0) {
+        last = i;
+        blast = C;
+        if (open) {
+          sel = i;
+          b = C;
+          open = !(C + w > target);
+        }
+      }
+      C += w;
+    }
+    const unsigned who = __ballot_sync(0xffffffffu, sel >= 0);
+    int ch;
+    if (who) {
+      const int src = __ffs(who) - 1;
+      ch = __shfl_sync(0xffffffffu, sel, src);
+      b = __shfl_sync(0xffffffffu, b, src);
+    } else {  // rounding put u * Z past every chunk: the last chunk with positive weight
+      ch = __reduce_max_sync(0xffffffffu, last);
+      const int owner = __reduce_max_sync(0xffffffffu, (ch >= 0 && last == ch) ? lane : -1);
+      b = __shfl_sync(0xffffffffu, blast, owner < 0 ? 0 : owner);
+    }
+    float ly = 0.0f;
+    int y = -1;
+    if (ch >= 0) y = warp_draw_chunk(J, ch * kChunkElems, min(V, (ch + 1) * kChunkElems), b, target, &ly);
+    if (lane == 0) {
+      sm.y = y;
+      sm.base = y >= 0 ? static_cast<double>(kept_weight(st, ly) / st.s_kept) : -1.0;
+    }
+  }
+  __syncthreads();
+  const int y = sm.y;
+  *q = static_cast<float>(sm.base);
+  __syncthreads();
+  return y;
+}
+
+// Whether request r's rows carry a top-p cut.
+__device__ __forceinline__ bool request_cut(const float* __restrict__ temperature, const float* __restrict__ top_p,
+                                            int r) {
+  return top_p[r] < 1.0f && temp_scale(temperature[r]) != 0.0f;
+}
+
+// The row kernel of sample_draft. CTAs [0, warp_ctas) finish the rows without a top-p cut,
+// one warp per row; the remaining CTAs take the rows of requests with a cut, one row per CTA
+// at a time (statistics, threshold, draw). One launch serves both kinds of rows.
+template <typename T>
+__global__ void __launch_bounds__(kTpThreads, 2) sample_rows_kernel(const T* __restrict__ draft, int K, int V,
+                                                                   int rows, const float* __restrict__ temperature,
+                                                                   const float* __restrict__ top_p,
+                                                                   const float* __restrict__ u,
+                                                                   const Partial* __restrict__ parts,
+                                                                   RowStat* __restrict__ stats,
+                                                                   int32_t* __restrict__ out_tokens,
+                                                                   float* __restrict__ out_q, int warp_ctas) {
+  if (static_cast<int>(blockIdx.x) < warp_ctas) {
+    const int row = blockIdx.x * kTpWarps + (threadIdx.x >> 5);
+    if (row < rows && !request_cut(temperature, top_p, row / K))
+      warp_sample_row(draft, row, K, V, temperature, u, parts, stats, out_tokens, out_q);
+    return;
+  }
+  extern __shared__ __align__(16) unsigned char tp_smem_raw[];
+  TpSmem& sm = *reinterpret_cast<TpSmem*>(tp_smem_raw);
+  const int ctas = static_cast<int>(gridDim.x) - warp_ctas;
+  for (int row = static_cast<int>(blockIdx.x) - warp_ctas; row < rows; row += ctas) {
+    const int b = row / K;
+    if (!request_cut(temperature, top_p, b)) continue;
+    const T* rp = draft + static_cast<size_t>(row) * V;
+    const RowStat st = tp_row_stats(rp, V, temperature[b], top_p[b], sm);
+    float q = -1.0f;
+    const int y = st.status == 0 ? tp_row_draw(rp, V, st, u[row], sm, &q) : -1;
+    if (threadIdx.x == 0) {
+      stats[row] = st;
+      out_tokens[row] = y;
+      if (out_q) out_q[row] = q;
+    }
+    __syncthreads();
+  }
+}
+
+// The row kernel of verify_linear. CTAs [0, warp_ctas) finish the rows of requests without a
+// top-p cut, one warp per row; the remaining CTAs take the rows of requests with a cut, one
+// row per CTA at a time (statistics and threshold). Every row then arrives on its request's
+// counter, and whoever completes a request runs its accept tests and writes the draw job.
+template <typename T>
+__global__ void __launch_bounds__(kTpThreads, 2) verify_rows_kernel(const T* __restrict__ tgt,
+                                                                   const T* __restrict__ drf, VerifyArgs a,
+                                                                   int warp_ctas) {
+  const int K = a.K, V = a.V;
+  const int rows_t = a.B * (K + 1);
+  const int rows = rows_t + (a.stream_draft ? a.B * K : 0);
+  if (static_cast<int>(blockIdx.x) < warp_ctas) {
+    const int g = blockIdx.x * kTpWarps + (threadIdx.x >> 5);
+    if (g < rows && !request_cut(a.temperature, a.top_p, g < rows_t ? g / (K + 1) : (g - rows_t) / K))
+      warp_verify_row(tgt, drf, g, a);
+    return;
+  }
+  extern __shared__ __align__(16) unsigned char tp_smem_raw[];
+  TpSmem& sm = *reinterpret_cast<TpSmem*>(tp_smem_raw);
+  const int per_req = (K + 1) + (a.stream_draft ? K : 0);
+  const int ctas = static_cast<int>(gridDim.x) - warp_ctas;
+  for (int g = static_cast<int>(blockIdx.x) - warp_ctas; g < rows; g += ctas) {
+    const bool is_draft = g >= rows_t;
+    const int row = is_draft ? g - rows_t : g;
+    const int b = is_draft ? row / K : row / (K + 1);
+    if (!request_cut(a.temperature, a.top_p, b)) continue;
+    const T* rp = (is_draft ? drf : tgt) + static_cast<size_t>(row) * V;
+    const RowStat st = tp_row_stats(rp, V, a.temperature[b], a.top_p[b], sm);
+    if (threadIdx.x == 0) (is_draft ? a.stats_d : a.stats_t)[row] = st;
+    if (block_arrive_last(&a.cnt[b], per_req, &sm.flag) && threadIdx.x < 32)
+      warp_decide_request<T>(b, tgt, drf, K, V, a.tokens, a.stats_t, a.stream_draft ? a.stats_d : a.dstats_in,
+                             a.u_acc, a.u_res, a.out_tokens, a.out_len, a.out_p, a.out_q, a.jobs);
+    __syncthreads();
+  }
+}
+
+}  // namespace psi
