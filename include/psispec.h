@@ -16,8 +16,9 @@
  * --------------------------------
  *  - Pointers named *_logits, u_*, temperature, top_p, draft_tokens, node_*, parent, tokens,
  *    out_*, row_stats and workspace are DEVICE pointers owned by the caller. The library
- *    allocates no memory and keeps no state between calls; it only enqueues kernels on
- *    `stream` (a cudaStream_t; NULL selects the legacy default stream). Calls are
+ *    allocates no memory and keeps no state between calls (psispec_verify_linear_static
+ *    excepted: it uses one library-owned scratch array per device); it only enqueues kernels
+ *    on `stream` (a cudaStream_t; NULL selects the legacy default stream). Calls are
  *    asynchronous: outputs are valid once the stream reaches that point.
  *  - Logit rows are contiguous: row r of a [rows, V] tensor starts at element r * V. dtype is
  *    PSISPEC_F32 or PSISPEC_BF16. Any V >= 1 is accepted; V up to 2^24.
@@ -177,6 +178,42 @@ psispec_status psispec_verify_tree(const void* target_logits, const void* draft_
                                    int32_t max_depth, int32_t* out_path, int32_t* out_tokens,
                                    int32_t* out_accept_len, void* workspace, size_t workspace_bytes,
                                    void* stream);
+
+/*
+ * psispec_verify_linear_static -- psispec_verify_linear without a caller workspace.
+ *
+ * The pages have no counterpart to this call: it is an integration convenience. It runs
+ * exactly psispec_verify_linear, with its scratch in one file-scope device array of
+ * PSISPEC_STATIC_WORKSPACE_BYTES bytes inside the library instead of a caller buffer. It
+ * allocates nothing: no cudaMalloc, no cudaFree. It serves callers that cannot allocate
+ * device memory on the calling path, e.g. a host program that links only this library and
+ * has no device allocator of its own, or a serving loop that must not let cudaMalloc or
+ * cudaFree synchronise the device between steps.
+ *
+ * Set-up: the first call on a device looks up the array's device address with
+ * cudaGetSymbolAddress (this may load the library's device code) and caches it for that
+ * device. Make that first call, on every device used, before any stream capture begins.
+ * Nothing in the array needs to start at zero: the call's first kernel clears the per-request
+ * arrival counters, and everything else is written before it is read.
+ *
+ * The array is shared by every call on one device: two calls whose executions overlap (on
+ * different streams, or from different threads) race on it and give undefined results. Calls
+ * on one stream run one after another and are safe.
+ *
+ * Arguments, outputs and limits as for psispec_verify_linear. In addition, a size whose
+ * psispec_workspace_size(PSISPEC_OP_VERIFY_LINEAR, B, K, V) exceeds
+ * PSISPEC_STATIC_WORKSPACE_BYTES is rejected with PSISPEC_ERR_UNSUPPORTED before anything
+ * is enqueued (e.g. B = 64, K = 8, V = 151936 needs about 3 MB; B = 512, K = 16 does not fit).
+ * If the device address cannot be obtained the call returns PSISPEC_ERR_CUDA.
+ */
+#define PSISPEC_STATIC_WORKSPACE_BYTES (16u << 20)
+
+psispec_status psispec_verify_linear_static(const void* target_logits, const void* draft_logits, int dtype,
+                                            int32_t B, int32_t K, int32_t V, const int32_t* draft_tokens,
+                                            const void* draft_row_stats, const float* u_accept,
+                                            const float* u_resid, const float* temperature,
+                                            const float* top_p, int32_t* out_tokens, int32_t* out_accept_len,
+                                            float* out_p, float* out_q, void* stream);
 
 #ifdef __cplusplus
 }

@@ -3,6 +3,7 @@
 #include "psispec.h"
 
 #include <algorithm>
+#include <atomic>
 
 #include "common.cuh"
 #include "finish.cuh"
@@ -297,6 +298,16 @@ size_t esize(int dtype) { return dtype == PSISPEC_BF16 ? 2 : 4; }
 }  // namespace
 }  // namespace psi
 
+// Scratch of psispec_verify_linear_static: one array per device, its address looked up once.
+static __device__ __align__(256) unsigned char g_static_workspace[PSISPEC_STATIC_WORKSPACE_BYTES];
+
+namespace psi {
+namespace {
+constexpr int kMaxDevices = 64;
+std::atomic<void*> g_static_workspace_ptr[kMaxDevices];
+}  // namespace
+}  // namespace psi
+
 using namespace psi;
 
 extern "C" {
@@ -400,6 +411,28 @@ psispec_status psispec_verify_tree(const void* target_logits, const void* draft_
   return verify_tree_impl(static_cast<const float*>(target_logits), static_cast<const float*>(draft_logits), B, N, V,
                           node_offsets, parent, tokens, u_accept, u_resid, temperature, top_p, max_depth, out_path,
                           out_tokens, out_accept_len, workspace, st);
+}
+
+psispec_status psispec_verify_linear_static(const void* target_logits, const void* draft_logits, int dtype,
+                                            int32_t B, int32_t K, int32_t V, const int32_t* draft_tokens,
+                                            const void* draft_row_stats, const float* u_accept,
+                                            const float* u_resid, const float* temperature,
+                                            const float* top_p, int32_t* out_tokens, int32_t* out_accept_len,
+                                            float* out_p, float* out_q, void* stream) {
+  if (B <= 0 || K <= 0 || V <= 0) return PSISPEC_ERR_INVALID_ARG;
+  const size_t need = psispec_workspace_size(PSISPEC_OP_VERIFY_LINEAR, B, K, V);
+  if (need == 0) return PSISPEC_ERR_INVALID_ARG;
+  if (need > static_cast<size_t>(PSISPEC_STATIC_WORKSPACE_BYTES)) return PSISPEC_ERR_UNSUPPORTED;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PSISPEC_ERR_CUDA;
+  void* ws = g_static_workspace_ptr[dev].load(std::memory_order_acquire);
+  if (ws == nullptr) {
+    if (cudaGetSymbolAddress(&ws, g_static_workspace) != cudaSuccess || ws == nullptr) return PSISPEC_ERR_CUDA;
+    g_static_workspace_ptr[dev].store(ws, std::memory_order_release);
+  }
+  return psispec_verify_linear(target_logits, draft_logits, dtype, B, K, V, draft_tokens, draft_row_stats, u_accept,
+                               u_resid, temperature, top_p, out_tokens, out_accept_len, out_p, out_q, ws,
+                               static_cast<size_t>(PSISPEC_STATIC_WORKSPACE_BYTES), stream);
 }
 
 }  // extern "C"

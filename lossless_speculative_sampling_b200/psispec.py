@@ -21,6 +21,7 @@ LIB_PATH = os.path.join(_HERE, "libpsispec.so")
 HEADER = os.path.join(os.path.dirname(_HERE), "include", "psispec.h")
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_WORKSPACE = 0, 1, 2, 3, 4
+STATIC_WORKSPACE_BYTES = 16 << 20  # PSISPEC_STATIC_WORKSPACE_BYTES
 F32, BF16 = 0, 1
 OP_SAMPLE_DRAFT, OP_VERIFY_LINEAR, OP_VERIFY_TREE = 0, 1, 2
 ROW_STATS_BYTES = 32
@@ -50,7 +51,9 @@ def lib():
         L.psispec_verify_linear.argtypes = [P, P, ctypes.c_int, I32, I32, I32, P, P, P, P, P, P, P, P, P, P, P, SZ, P]
         L.psispec_verify_tree.argtypes = [P, P, ctypes.c_int, I32, I32, I32, P, P, P, P, P, P, P, I32, P, P, P, P, SZ,
                                           P]
-        for f in ("psispec_sample_draft", "psispec_verify_linear", "psispec_verify_tree"):
+        L.psispec_verify_linear_static.argtypes = [P, P, ctypes.c_int, I32, I32, I32, P, P, P, P, P, P, P, P, P, P, P]
+        for f in ("psispec_sample_draft", "psispec_verify_linear", "psispec_verify_tree",
+                  "psispec_verify_linear_static"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -209,3 +212,33 @@ def verify_tree(target, draft, node_offsets, parent, tokens, u_accept, u_resid, 
                                    _stream(dev, stream))
     _check(st, "psispec_verify_tree")
     return {"path": out_path, "tokens": out_tokens, "accept_len": out_accept_len}
+
+
+def verify_linear_static(target, draft, draft_tokens, u_accept, u_resid, temperature, top_p, *, draft_row_stats=None,
+                         out_tokens=None, out_accept_len=None, out_p=None, out_q=None, want_pq=True, stream=None):
+    """verify_linear with the library-owned scratch array (psispec_verify_linear_static): no
+    workspace argument. Outputs not passed in are allocated here; pass them all to keep the
+    call free of allocations."""
+    B, K1, V = target.shape
+    K = K1 - 1
+    dev = target.device
+    _req(target, "target")
+    _req(draft, "draft", target.dtype, B * K * V, dev)
+    _req(draft_tokens, "draft_tokens", torch.int32, B * K, dev)
+    _req(u_accept, "u_accept", torch.float32, B * K, dev)
+    _req(u_resid, "u_resid", torch.float32, B * (K + 1), dev)
+    _req(temperature, "temperature", torch.float32, B, dev)
+    _req(top_p, "top_p", torch.float32, B, dev)
+    if draft_row_stats is not None:
+        _req(draft_row_stats, "draft_row_stats", torch.uint8, B * K * ROW_STATS_BYTES, dev)
+    out_tokens = torch.empty((B, K + 1), dtype=torch.int32, device=dev) if out_tokens is None else out_tokens
+    out_accept_len = torch.empty(B, dtype=torch.int32, device=dev) if out_accept_len is None else out_accept_len
+    if want_pq:
+        out_p = torch.empty((B, K), dtype=torch.float32, device=dev) if out_p is None else out_p
+        out_q = torch.empty((B, K), dtype=torch.float32, device=dev) if out_q is None else out_q
+    st = lib().psispec_verify_linear_static(_p(target), _p(draft), _dtype(target), B, K, V, _p(draft_tokens),
+                                            _p(draft_row_stats), _p(u_accept), _p(u_resid), _p(temperature),
+                                            _p(top_p), _p(out_tokens), _p(out_accept_len), _p(out_p), _p(out_q),
+                                            _stream(dev, stream))
+    _check(st, "psispec_verify_linear_static")
+    return {"tokens": out_tokens, "accept_len": out_accept_len, "p": out_p, "q": out_q}
