@@ -288,6 +288,31 @@ psispec_status verify_tree_impl(const T* tgt, const T* drf, int B, int N, int V,
   if (s != PSISPEC_OK) return s;
   s = launch_stats<T>(drf, N, 1, w.row_req, V, temperature, B, top_p, w.d, st);
   if (s != PSISPEC_OK) return s;
+  const int slice = tree_slice(V);
+  if (slice <= kTreeMaxSlice) {
+    // one cluster of kTreeCluster CTAs per trie, the node's rows staged across their smem
+    const int smem = 2 * slice * static_cast<int>(sizeof(float));
+    if (cudaFuncSetAttribute(tree_walk_cluster_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+        cudaSuccess)
+      return PSISPEC_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(B) * kTreeCluster);
+    cfg.blockDim = dim3(kTreeWalkThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = kTreeCluster;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, tree_walk_cluster_kernel<T>, tgt, drf, V, offs, parent, tokens,
+                              static_cast<const RowStat*>(w.t.stats), static_cast<const RowStat*>(w.d.stats), u_acc,
+                              u_res, max_depth, out_path, out_tokens, out_len) == cudaSuccess
+               ? PSISPEC_OK
+               : PSISPEC_ERR_CUDA;
+  }
   return launch(tree_walk_kernel<T>, static_cast<unsigned>(B), kTreeThreads, 0, st, tgt, drf, V, offs, parent, tokens,
                 w.t.stats, w.d.stats, u_acc, u_res, max_depth, out_path, out_tokens, out_len);
 }

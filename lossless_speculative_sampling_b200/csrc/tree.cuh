@@ -14,7 +14,10 @@
 // One CTA of kTreeThreads per request. Row statistics come from the stats kernels.
 #pragma once
 
+#include <cooperative_groups.h>
+
 #include "common.cuh"
+#include "sample.cuh"
 
 namespace psi {
 
@@ -218,6 +221,287 @@ __global__ void __launch_bounds__(kTreeThreads) tree_walk_kernel(
     } else {
       for (int i = len; i < max_depth; ++i) path[i] = -1;
       toks[len] = sh_y;
+      for (int i = len + 1; i <= max_depth; ++i) toks[i] = -1;
+      out_len[b] = len;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// Cluster walk. A cluster of kTreeCluster CTAs verifies one trie; CTA `rank` owns the
+// vocabulary slice [rank * slice, (rank + 1) * slice). At every visited node the slices of
+// r (unnormalised, r = r' / S) and q (normalised) are staged in shared memory as fp32, so the
+// passes a rejection needs run on chip:
+//   accept child k with token t  iff  u * q(t) * S < r'(t) * Q   (q~ = q / Q, r = r' / S);
+//   on rejection                      r' <- max(r' - (S / Q) q, 0),  S <- sum r',
+//                                     q(t) <- 0,  Q <- sum q       (r' unchanged when S = 0).
+// Sums are fp64: per CTA by a block reduction, across the cluster in rank order through
+// distributed shared memory, so every CTA computes the same value and takes the same branch
+// (the cluster barriers below are therefore reached in the same order by every CTA).
+namespace cg = cooperative_groups;
+
+constexpr int kTreeCluster = 8;
+constexpr int kTreeWalkThreads = 256;
+constexpr int kTreeMaxSlice = 26624;  // elements per CTA: r and q slices as fp32 fit in 208 KB
+
+__host__ __device__ inline int tree_slice(int V) {
+  return (((V + kTreeCluster - 1) / kTreeCluster) + 7) & ~7;  // a multiple of 8 elements
+}
+
+struct TreeWalkShared {
+  int depth[kMaxNodes];
+  int ch[kMaxChildren];
+  double red[33];
+  double slot[4];  // this CTA's contribution to a cluster reduction
+  int islot[2];
+  int bad, nch, next, y, acc;
+};
+
+// Sums of a and b over the cluster, in rank order (the same doubles in every CTA).
+__device__ __forceinline__ double2 cluster_sum2(cg::cluster_group& cl, double a, double b, TreeWalkShared& sh) {
+  if (threadIdx.x == 0) {
+    sh.slot[0] = a;
+    sh.slot[1] = b;
+  }
+  cl.sync();
+  double sa = 0.0, sb = 0.0;
+  for (int r = 0; r < kTreeCluster; ++r) {
+    const double* rs = cl.map_shared_rank(sh.slot, r);
+    sa += rs[0];
+    sb += rs[1];
+  }
+  cl.sync();
+  return make_double2(sa, sb);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kTreeWalkThreads, 1) tree_walk_cluster_kernel(
+    const T* __restrict__ tgt, const T* __restrict__ drf, int V, const int32_t* __restrict__ offs,
+    const int32_t* __restrict__ parent, const int32_t* __restrict__ tokens, const RowStat* __restrict__ ts,
+    const RowStat* __restrict__ ds, const float* __restrict__ u_acc, const float* __restrict__ u_res, int max_depth,
+    int32_t* __restrict__ out_path, int32_t* __restrict__ out_tokens, int32_t* __restrict__ out_len) {
+  cg::cluster_group cl = cg::this_cluster();
+  __shared__ TreeWalkShared sh;
+  extern __shared__ __align__(16) float tw_smem[];
+  const int rank = static_cast<int>(cl.block_rank());
+  const int slice = tree_slice(V);
+  float* rs = tw_smem;          // r' of this CTA's slice
+  float* qs = tw_smem + slice;  // q of this CTA's slice
+  const int v0 = min(V, rank * slice), v1 = min(V, v0 + slice), ns = v1 - v0;
+  const int b = blockIdx.x / kTreeCluster;
+  const int n0 = offs[b], n = offs[b + 1] - n0;
+  int32_t* path = out_path + static_cast<size_t>(b) * max_depth;
+  int32_t* toks = out_tokens + static_cast<size_t>(b) * (max_depth + 1);
+  const bool writer = rank == 0 && threadIdx.x == 0;
+
+  if (threadIdx.x == 0) {  // structure checks (every CTA, same data, same answer)
+    int bad = (n <= 0 || n > kMaxNodes) ? 1 : (parent[n0] != -1);
+    if (!bad) sh.depth[0] = 0;
+    for (int c = 1; c < n && !bad; ++c) {
+      const int pa = parent[n0 + c], t = tokens[n0 + c];
+      if (pa < 0 || pa >= c || t < 0 || t >= V) {
+        bad = 1;
+        break;
+      }
+      sh.depth[c] = sh.depth[pa] + 1;
+      if (sh.depth[c] > max_depth) bad = 1;
+    }
+    sh.bad = bad;
+    sh.y = -1;
+  }
+  __syncthreads();
+
+  int cur = 0, len = 0;
+  while (!sh.bad) {
+    const RowStat sp = ts[n0 + cur];
+    if (threadIdx.x == 0) {
+      int nch = 0;
+      for (int c = cur + 1; c < n; ++c)
+        if (parent[n0 + c] == cur) {
+          if (nch == kMaxChildren) {
+            sh.bad = 1;
+            break;
+          }
+          sh.ch[nch++] = c;
+        }
+      sh.nch = nch;
+      sh.next = -1;
+      if (sp.status != 0) sh.bad = 1;
+    }
+    __syncthreads();
+    if (sh.bad) break;
+    const int nch = sh.nch;
+    if (sp.c == 0.0f) {  // greedy: follow the child carrying the verifier argmax
+      if (threadIdx.x == 0) {
+        for (int k = 0; k < nch; ++k)
+          if (tokens[n0 + sh.ch[k]] == sp.amax) {
+            sh.next = sh.ch[k];
+            break;
+          }
+        sh.y = sp.amax;
+      }
+      __syncthreads();
+      const int next = sh.next;
+      if (next >= 0) {
+        if (writer) {
+          path[len] = next;
+          toks[len] = tokens[n0 + next];
+        }
+        cur = next;
+        ++len;
+        __syncthreads();
+        continue;
+      }
+      break;  // final token sh.y
+    }
+    RowStat sq = sp;
+    if (nch > 0) {
+      sq = ds[n0 + cur];
+      if (sq.status != 0) {
+        if (threadIdx.x == 0) sh.bad = 1;
+        __syncthreads();
+        break;
+      }
+    }
+    // stage the node's slices: r' = kept weight of p (relative to its maximum), q normalised
+    {
+      const T* rp = tgt + static_cast<size_t>(n0 + cur) * V;
+      const T* rq = drf + static_cast<size_t>(n0 + cur) * V;
+      JobRows<T, true> J;
+      J.init(rp, sp, rq, sq);
+      const float iq = nch > 0 ? 1.0f / sq.s_kept : 0.0f;
+      double sr = 0.0, sqm = 0.0;
+      for (int e = v0 + threadIdx.x * 8; e < v1; e += kTreeWalkThreads * 8) {
+        Raw8<T, true> x;
+        J.load(e, v1, x);
+        float lp[8], lq[8];
+        x.a.unpack(lp);
+        x.b[0].unpack(lq);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          if (e + k < v1) {
+            const float r = kept_weight(sp, lp[k]);
+            const float q = nch > 0 ? kept_weight(sq, lq[k]) * iq : 0.0f;
+            rs[e + k - v0] = r;
+            qs[e + k - v0] = q;
+            sr += static_cast<double>(r);
+            sqm += static_cast<double>(q);
+          }
+        }
+      }
+      sr = block_sum(sr, sh.red);
+      sqm = block_sum(sqm, sh.red);
+      __syncthreads();
+      const double2 t = cluster_sum2(cl, sr, sqm, sh);  // also publishes the staged slices
+      double S = t.x, Q = t.y;
+      for (int k = 0; k < nch; ++k) {
+        if (!(Q > 0.0)) break;  // draft mass exhausted: the remaining children are skipped
+        const int c = sh.ch[k], tok = tokens[n0 + c];
+        const int owner = tok / slice, off = tok - owner * slice;
+        if (threadIdx.x == 0) {
+          const float rt = cl.map_shared_rank(rs, owner)[off];
+          const float qt = cl.map_shared_rank(qs, owner)[off];
+          sh.acc = static_cast<double>(u_acc[n0 + c]) * static_cast<double>(qt) * S <
+                   static_cast<double>(rt) * Q;
+        }
+        cl.sync();  // every CTA has read r'(t) and q(t) before any slice changes
+        if (sh.acc) {
+          if (threadIdx.x == 0) sh.next = c;
+          __syncthreads();
+          break;
+        }
+        // rejected: totals of the residual and of the draft mass without t
+        const float scale = static_cast<float>(S / Q);
+        double zr = 0.0, zq = 0.0;
+        for (int i = threadIdx.x; i < ns; i += kTreeWalkThreads) {
+          const float q = qs[i];
+          zr += static_cast<double>(fmaxf(rs[i] - scale * q, 0.0f));
+          if (v0 + i != tok) zq += static_cast<double>(q);
+        }
+        zr = block_sum(zr, sh.red);
+        zq = block_sum(zq, sh.red);
+        __syncthreads();
+        const double2 z = cluster_sum2(cl, zr, zq, sh);
+        if (z.x > 0.0) {
+          for (int i = threadIdx.x; i < ns; i += kTreeWalkThreads) rs[i] = fmaxf(rs[i] - scale * qs[i], 0.0f);
+          S = z.x;
+        }
+        if (rank == owner && threadIdx.x == 0) qs[off] = 0.0f;
+        Q = z.y;
+        __syncthreads();
+        cl.sync();  // the updated slices are visible before the next child's test
+      }
+    }
+    const int next = sh.next;
+    if (next >= 0) {
+      if (writer) {
+        path[len] = next;
+        toks[len] = tokens[n0 + next];
+      }
+      cur = next;
+      ++len;
+      __syncthreads();
+      continue;
+    }
+    // final draw from r at this node: contiguous runs per thread, scanned in thread order
+    // inside each slice, slices in rank order
+    const int run = (ns + kTreeWalkThreads - 1) / kTreeWalkThreads;
+    const int r0 = min(ns, static_cast<int>(threadIdx.x) * run), r1 = min(ns, r0 + run);
+    double mine = 0.0;
+    int last = -1;
+    for (int i = r0; i < r1; ++i) {
+      const float w = rs[i];
+      mine += static_cast<double>(w);
+      if (w > 0.0f) last = v0 + i;
+    }
+    double total;
+    const double C0 = block_exclusive_scan(mine, sh.red, &total);
+    if (threadIdx.x == 0) {
+      sh.slot[0] = total;
+      sh.islot[0] = 0x7fffffff;  // drawn index, if it falls in this slice
+      sh.islot[1] = -1;          // last index with positive weight in this slice
+    }
+    cl.sync();
+    double base = 0.0, grand = 0.0;
+    for (int r = 0; r < kTreeCluster; ++r) {
+      const double tr = cl.map_shared_rank(sh.slot, r)[0];
+      if (r < rank) base += tr;
+      grand += tr;
+    }
+    const double target = static_cast<double>(u_res[n0 + cur]) * grand;
+    if (last >= 0) atomicMax(&sh.islot[1], last);
+    if (base + C0 <= target && target < base + C0 + mine) {
+      double C = base + C0;
+      for (int i = r0; i < r1; ++i) {
+        C += static_cast<double>(rs[i]);
+        if (C > target && rs[i] > 0.0f) {
+          atomicMin(&sh.islot[0], v0 + i);
+          break;
+        }
+      }
+    }
+    __syncthreads();
+    cl.sync();
+    if (writer) {
+      int y = 0x7fffffff, lastpos = -1;
+      for (int r = 0; r < kTreeCluster; ++r) {
+        const int* is = cl.map_shared_rank(sh.islot, r);
+        y = min(y, is[0]);
+        lastpos = max(lastpos, is[1]);
+      }
+      sh.y = y != 0x7fffffff ? y : lastpos;  // rounding past every slice: the last positive index
+    }
+    break;
+  }
+  cl.sync();  // no CTA leaves while another may still read its shared memory
+  if (writer) {
+    if (sh.bad) {
+      for (int i = 0; i < max_depth; ++i) path[i] = -1;
+      for (int i = 0; i <= max_depth; ++i) toks[i] = -1;
+      out_len[b] = -1;
+    } else {
+      for (int i = len; i < max_depth; ++i) path[i] = -1;
+      toks[len] = sh.y;
       for (int i = len + 1; i <= max_depth; ++i) toks[i] = -1;
       out_len[b] = len;
     }
