@@ -274,6 +274,46 @@ psispec_status verify_linear_impl(const T* tgt, const T* drf, int B, int K, int 
   return launch_draws<T>(tgt, drf, V, B, w.t.parts, w.jobs, w.draw_tc, w.draw_tg, out_tokens, st);
 }
 
+// The cluster tree walk with CL CTAs per trie; PSISPEC_ERR_UNSUPPORTED when V needs larger
+// slices than shared memory holds or the device cannot schedule such a cluster.
+template <typename T, int CL>
+psispec_status launch_tree_cluster(const T* tgt, const T* drf, int B, int V, const int32_t* offs,
+                                   const int32_t* parent, const int32_t* tokens, const RowStat* ts, const RowStat* ds,
+                                   const float* u_acc, const float* u_res, int max_depth, int32_t* out_path,
+                                   int32_t* out_tokens, int32_t* out_len, cudaStream_t st) {
+  const int slice = tree_slice(V, CL);
+  if (slice > kTreeMaxSlice) return PSISPEC_ERR_UNSUPPORTED;
+  const int smem = 2 * slice * static_cast<int>(sizeof(float));
+  auto kernel = tree_walk_cluster_kernel<T, CL>;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return PSISPEC_ERR_CUDA;
+  if (CL > 8 && cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
+    cudaGetLastError();
+    return PSISPEC_ERR_UNSUPPORTED;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(B) * CL);
+  cfg.blockDim = dim3(kTreeWalkThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = CL;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int clusters = 0;
+  if (cudaOccupancyMaxActiveClusters(&clusters, kernel, &cfg) != cudaSuccess || clusters < 1) {
+    cudaGetLastError();
+    return PSISPEC_ERR_UNSUPPORTED;
+  }
+  return cudaLaunchKernelEx(&cfg, kernel, tgt, drf, V, offs, parent, tokens, ts, ds, u_acc, u_res, max_depth, out_path,
+                            out_tokens, out_len) == cudaSuccess
+             ? PSISPEC_OK
+             : PSISPEC_ERR_CUDA;
+}
+
 template <typename T>
 psispec_status verify_tree_impl(const T* tgt, const T* drf, int B, int N, int V, const int32_t* offs,
                                 const int32_t* parent, const int32_t* tokens, const float* u_acc, const float* u_res,
@@ -288,31 +328,14 @@ psispec_status verify_tree_impl(const T* tgt, const T* drf, int B, int N, int V,
   if (s != PSISPEC_OK) return s;
   s = launch_stats<T>(drf, N, 1, w.row_req, V, temperature, B, top_p, w.d, st);
   if (s != PSISPEC_OK) return s;
-  const int slice = tree_slice(V);
-  if (slice <= kTreeMaxSlice) {
-    // one cluster of kTreeCluster CTAs per trie, the node's rows staged across their smem
-    const int smem = 2 * slice * static_cast<int>(sizeof(float));
-    if (cudaFuncSetAttribute(tree_walk_cluster_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-        cudaSuccess)
-      return PSISPEC_ERR_CUDA;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(B) * kTreeCluster);
-    cfg.blockDim = dim3(kTreeWalkThreads);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = kTreeCluster;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, tree_walk_cluster_kernel<T>, tgt, drf, V, offs, parent, tokens,
-                              static_cast<const RowStat*>(w.t.stats), static_cast<const RowStat*>(w.d.stats), u_acc,
-                              u_res, max_depth, out_path, out_tokens, out_len) == cudaSuccess
-               ? PSISPEC_OK
-               : PSISPEC_ERR_CUDA;
-  }
+  // one cluster per trie, the node's rows staged across its CTAs' shared memory: 16 CTAs
+  // where the device can schedule such clusters, else 8
+  psispec_status s16 = launch_tree_cluster<T, 16>(tgt, drf, B, V, offs, parent, tokens, w.t.stats, w.d.stats, u_acc,
+                                                  u_res, max_depth, out_path, out_tokens, out_len, st);
+  if (s16 != PSISPEC_ERR_UNSUPPORTED) return s16;
+  psispec_status s8 = launch_tree_cluster<T, 8>(tgt, drf, B, V, offs, parent, tokens, w.t.stats, w.d.stats, u_acc,
+                                                u_res, max_depth, out_path, out_tokens, out_len, st);
+  if (s8 != PSISPEC_ERR_UNSUPPORTED) return s8;
   return launch(tree_walk_kernel<T>, static_cast<unsigned>(B), kTreeThreads, 0, st, tgt, drf, V, offs, parent, tokens,
                 w.t.stats, w.d.stats, u_acc, u_res, max_depth, out_path, out_tokens, out_len);
 }

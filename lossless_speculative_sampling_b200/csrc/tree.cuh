@@ -228,7 +228,8 @@ __global__ void __launch_bounds__(kTreeThreads) tree_walk_kernel(
 }
 
 // ---------------------------------------------------------------------------------------
-// Cluster walk. A cluster of kTreeCluster CTAs verifies one trie; CTA `rank` owns the
+// Cluster walk. A cluster of CL CTAs (16 where the device can schedule it, else 8) verifies
+// one trie; CTA `rank` owns the
 // vocabulary slice [rank * slice, (rank + 1) * slice). At every visited node the slices of
 // r (unnormalised, r = r' / S) and q (normalised) are staged in shared memory as fp32, so the
 // passes a rejection needs run on chip:
@@ -240,12 +241,11 @@ __global__ void __launch_bounds__(kTreeThreads) tree_walk_kernel(
 // (the cluster barriers below are therefore reached in the same order by every CTA).
 namespace cg = cooperative_groups;
 
-constexpr int kTreeCluster = 8;
 constexpr int kTreeWalkThreads = 256;
 constexpr int kTreeMaxSlice = 26624;  // elements per CTA: r and q slices as fp32 fit in 208 KB
 
-__host__ __device__ inline int tree_slice(int V) {
-  return (((V + kTreeCluster - 1) / kTreeCluster) + 7) & ~7;  // a multiple of 8 elements
+__host__ __device__ inline int tree_slice(int V, int cl) {
+  return (((V + cl - 1) / cl) + 7) & ~7;  // a multiple of 8 elements
 }
 
 struct TreeWalkShared {
@@ -258,6 +258,7 @@ struct TreeWalkShared {
 };
 
 // Sums of a and b over the cluster, in rank order (the same doubles in every CTA).
+template <int CL>
 __device__ __forceinline__ double2 cluster_sum2(cg::cluster_group& cl, double a, double b, TreeWalkShared& sh) {
   if (threadIdx.x == 0) {
     sh.slot[0] = a;
@@ -265,7 +266,7 @@ __device__ __forceinline__ double2 cluster_sum2(cg::cluster_group& cl, double a,
   }
   cl.sync();
   double sa = 0.0, sb = 0.0;
-  for (int r = 0; r < kTreeCluster; ++r) {
+  for (int r = 0; r < CL; ++r) {
     const double* rs = cl.map_shared_rank(sh.slot, r);
     sa += rs[0];
     sb += rs[1];
@@ -274,7 +275,7 @@ __device__ __forceinline__ double2 cluster_sum2(cg::cluster_group& cl, double a,
   return make_double2(sa, sb);
 }
 
-template <typename T>
+template <typename T, int CL>
 __global__ void __launch_bounds__(kTreeWalkThreads, 1) tree_walk_cluster_kernel(
     const T* __restrict__ tgt, const T* __restrict__ drf, int V, const int32_t* __restrict__ offs,
     const int32_t* __restrict__ parent, const int32_t* __restrict__ tokens, const RowStat* __restrict__ ts,
@@ -284,11 +285,11 @@ __global__ void __launch_bounds__(kTreeWalkThreads, 1) tree_walk_cluster_kernel(
   __shared__ TreeWalkShared sh;
   extern __shared__ __align__(16) float tw_smem[];
   const int rank = static_cast<int>(cl.block_rank());
-  const int slice = tree_slice(V);
+  const int slice = tree_slice(V, CL);
   float* rs = tw_smem;          // r' of this CTA's slice
   float* qs = tw_smem + slice;  // q of this CTA's slice
   const int v0 = min(V, rank * slice), v1 = min(V, v0 + slice), ns = v1 - v0;
-  const int b = blockIdx.x / kTreeCluster;
+  const int b = blockIdx.x / CL;
   const int n0 = offs[b], n = offs[b + 1] - n0;
   int32_t* path = out_path + static_cast<size_t>(b) * max_depth;
   int32_t* toks = out_tokens + static_cast<size_t>(b) * (max_depth + 1);
@@ -371,28 +372,48 @@ __global__ void __launch_bounds__(kTreeWalkThreads, 1) tree_walk_cluster_kernel(
       J.init(rp, sp, rq, sq);
       const float iq = nch > 0 ? 1.0f / sq.s_kept : 0.0f;
       double sr = 0.0, sqm = 0.0;
-      for (int e = v0 + threadIdx.x * 8; e < v1; e += kTreeWalkThreads * 8) {
-        Raw8<T, true> x;
-        J.load(e, v1, x);
-        float lp[8], lq[8];
-        x.a.unpack(lp);
-        x.b[0].unpack(lq);
+      constexpr int kStageBatch = 4;  // 8-element groups of both rows in flight per thread
+      constexpr int kStep = kTreeWalkThreads * 8;
+      for (int e0 = v0 + threadIdx.x * 8; e0 < v1; e0 += kStageBatch * kStep) {
+        Raw8<T, true> x[kStageBatch];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          if (e + k < v1) {
-            const float r = kept_weight(sp, lp[k]);
-            const float q = nch > 0 ? kept_weight(sq, lq[k]) * iq : 0.0f;
-            rs[e + k - v0] = r;
-            qs[e + k - v0] = q;
-            sr += static_cast<double>(r);
-            sqm += static_cast<double>(q);
+        for (int j = 0; j < kStageBatch; ++j)
+          if (e0 + j * kStep < v1) J.load(e0 + j * kStep, v1, x[j]);
+#pragma unroll
+        for (int j = 0; j < kStageBatch; ++j) {
+          const int e = e0 + j * kStep;
+          if (e >= v1) continue;
+          float lp[8], lq[8];
+          x[j].a.unpack(lp);
+          x[j].b[0].unpack(lq);
+          float gr = 0.0f, gq = 0.0f;  // 8-term fp32 sums, then fp64
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            if (e + k < v1) {
+              const float r = kept_weight(sp, lp[k]);
+              const float q = nch > 0 ? kept_weight(sq, lq[k]) * iq : 0.0f;
+              rs[e + k - v0] = r;
+              qs[e + k - v0] = q;
+              gr += r;
+              gq += q;
+            }
           }
+          sr += static_cast<double>(gr);
+          sqm += static_cast<double>(gq);
+        }
+      }
+      // the walk continues at one of the children: bring their slices towards L2 meanwhile
+      for (int k = 0; k < nch; ++k) {
+        const size_t row = static_cast<size_t>(n0 + sh.ch[k]) * V;
+        for (int e = v0 + threadIdx.x * 64; e < v1; e += kTreeWalkThreads * 64) {
+          asm volatile("prefetch.global.L2 [%0];" ::"l"(tgt + row + e));
+          asm volatile("prefetch.global.L2 [%0];" ::"l"(drf + row + e));
         }
       }
       sr = block_sum(sr, sh.red);
       sqm = block_sum(sqm, sh.red);
       __syncthreads();
-      const double2 t = cluster_sum2(cl, sr, sqm, sh);  // also publishes the staged slices
+      const double2 t = cluster_sum2<CL>(cl, sr, sqm, sh);  // also publishes the staged slices
       double S = t.x, Q = t.y;
       for (int k = 0; k < nch; ++k) {
         if (!(Q > 0.0)) break;  // draft mass exhausted: the remaining children are skipped
@@ -410,20 +431,41 @@ __global__ void __launch_bounds__(kTreeWalkThreads, 1) tree_walk_cluster_kernel(
           __syncthreads();
           break;
         }
-        // rejected: totals of the residual and of the draft mass without t
+        // rejected: totals of the residual and of the draft mass without t (4-term fp32 sums,
+        // then fp64), over float4 vectors of the slices
         const float scale = static_cast<float>(S / Q);
+        const int tl = tok - v0;  // t's offset in this slice (outside [0, ns) elsewhere)
+        const int n4 = ns >> 2;
+        float4* r4 = reinterpret_cast<float4*>(rs);
+        const float4* q4 = reinterpret_cast<const float4*>(qs);
         double zr = 0.0, zq = 0.0;
-        for (int i = threadIdx.x; i < ns; i += kTreeWalkThreads) {
-          const float q = qs[i];
-          zr += static_cast<double>(fmaxf(rs[i] - scale * q, 0.0f));
-          if (v0 + i != tok) zq += static_cast<double>(q);
+        for (int i = threadIdx.x; i < n4; i += kTreeWalkThreads) {
+          const float4 r = r4[i], q = q4[i];
+          zr += static_cast<double>((fmaxf(r.x - scale * q.x, 0.0f) + fmaxf(r.y - scale * q.y, 0.0f)) +
+                                    (fmaxf(r.z - scale * q.z, 0.0f) + fmaxf(r.w - scale * q.w, 0.0f)));
+          const int j = tl - 4 * i;  // the removed token's lane within this vector, if any
+          zq += static_cast<double>(((j == 0 ? 0.0f : q.x) + (j == 1 ? 0.0f : q.y)) +
+                                    ((j == 2 ? 0.0f : q.z) + (j == 3 ? 0.0f : q.w)));
+        }
+        for (int i = 4 * n4 + threadIdx.x; i < ns; i += kTreeWalkThreads) {
+          zr += static_cast<double>(fmaxf(rs[i] - scale * qs[i], 0.0f));
+          if (i != tl) zq += static_cast<double>(qs[i]);
         }
         zr = block_sum(zr, sh.red);
         zq = block_sum(zq, sh.red);
         __syncthreads();
-        const double2 z = cluster_sum2(cl, zr, zq, sh);
+        const double2 z = cluster_sum2<CL>(cl, zr, zq, sh);
         if (z.x > 0.0) {
-          for (int i = threadIdx.x; i < ns; i += kTreeWalkThreads) rs[i] = fmaxf(rs[i] - scale * qs[i], 0.0f);
+          for (int i = threadIdx.x; i < n4; i += kTreeWalkThreads) {
+            float4 r = r4[i];
+            const float4 q = q4[i];
+            r.x = fmaxf(r.x - scale * q.x, 0.0f);
+            r.y = fmaxf(r.y - scale * q.y, 0.0f);
+            r.z = fmaxf(r.z - scale * q.z, 0.0f);
+            r.w = fmaxf(r.w - scale * q.w, 0.0f);
+            r4[i] = r;
+          }
+          for (int i = 4 * n4 + threadIdx.x; i < ns; i += kTreeWalkThreads) rs[i] = fmaxf(rs[i] - scale * qs[i], 0.0f);
           S = z.x;
         }
         if (rank == owner && threadIdx.x == 0) qs[off] = 0.0f;
@@ -463,7 +505,7 @@ __global__ void __launch_bounds__(kTreeWalkThreads, 1) tree_walk_cluster_kernel(
     }
     cl.sync();
     double base = 0.0, grand = 0.0;
-    for (int r = 0; r < kTreeCluster; ++r) {
+    for (int r = 0; r < CL; ++r) {
       const double tr = cl.map_shared_rank(sh.slot, r)[0];
       if (r < rank) base += tr;
       grand += tr;
@@ -484,7 +526,7 @@ __global__ void __launch_bounds__(kTreeWalkThreads, 1) tree_walk_cluster_kernel(
     cl.sync();
     if (writer) {
       int y = 0x7fffffff, lastpos = -1;
-      for (int r = 0; r < kTreeCluster; ++r) {
+      for (int r = 0; r < CL; ++r) {
         const int* is = cl.map_shared_rank(sh.islot, r);
         y = min(y, is[0]);
         lastpos = max(lastpos, is[1]);
