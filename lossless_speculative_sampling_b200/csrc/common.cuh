@@ -103,6 +103,11 @@ __device__ __forceinline__ f32x2 add2(f32x2 a, f32x2 b) {
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
 }
+__device__ __forceinline__ f32x2 fma2(f32x2 a, f32x2 b, f32x2 c) {
+  f32x2 d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
 __device__ __forceinline__ float max3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
@@ -247,11 +252,20 @@ __device__ __forceinline__ void vec_range(const T* row, int v0, int v1, int& a0,
   a1 = a0 + ((v1 - a0) / N) * N;
 }
 
+// The float whose order key is `key` (the inverse of fkey on keys of actual values).
+__device__ __forceinline__ float key_value(uint32_t key) {
+  return (key & 0x80000000u) ? __uint_as_float(key & 0x7FFFFFFFu) : __uint_as_float(~key);
+}
+
+// Smallest kept logit value of a top-p threshold key as a float bound: l is kept iff
+// l >= cut_value(tau), which equals fkey(l) >= tau for every non-NaN l (tau == 0 keeps all).
+__device__ __forceinline__ float cut_value(uint32_t tau) { return tau == 0u ? -INFINITY : key_value(tau); }
+
 // Weight of logit l under row statistics st (kept set applied); greedy rows are handled by
 // the callers.
 __device__ __forceinline__ float kept_weight(const RowStat& st, float l) {
   const float w = ex2((l - st.m) * st.c);
-  return (st.tau == 0u || fkey(l) >= st.tau) ? w : 0.0f;
+  return l >= cut_value(st.tau) ? w : 0.0f;
 }
 
 // Probability of token v with logit l under st.

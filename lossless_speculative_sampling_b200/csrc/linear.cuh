@@ -19,8 +19,8 @@ namespace psi {
 // probabilities do not underflow before the comparison.
 __device__ __forceinline__ bool accept_test(float u, const RowStat& sp, float lp, const RowStat& sq, float lq, int x) {
   if (sp.c == 0.0f) return x == sp.amax;
-  const bool p_pos = fkey(lp) >= sp.tau && lp > -INFINITY;
-  const bool q_pos = fkey(lq) >= sq.tau && lq > -INFINITY;
+  const bool p_pos = lp >= cut_value(sp.tau) && lp > -INFINITY;
+  const bool q_pos = lq >= cut_value(sq.tau) && lq > -INFINITY;
   if (!p_pos) return false;
   if (!q_pos) return true;
   const float e = ((lp - lq) + (sq.m - sp.m)) * sp.c;

@@ -24,6 +24,7 @@ constexpr int kDrawBatch = 4;  // groups in flight per lane
 struct ResidCtx {
   RowStat a, b;
   float ia, ib;  // 1 / s_kept of rows a and b
+  float ta, tb;  // smallest kept logit of rows a and b (cut_value of their thresholds)
 };
 
 // 8 consecutive elements starting at e (elements at or past `end` read as -inf)
@@ -118,6 +119,8 @@ struct JobRows {
     rb = rowb;
     r.b = sb;
     r.ib = RESID ? 1.0f / sb.s_kept : 0.0f;
+    r.ta = cut_value(sa.tau);
+    r.tb = cut_value(sb.tau);
     al_b = RESID && (reinterpret_cast<uintptr_t>(rowb) & 15u) == 0;
   }
   __device__ __forceinline__ float logit_a(int v) const { return load_elem(ra + v); }
@@ -141,7 +144,7 @@ struct JobRows {
     if (r.a.tau != 0u) {
 #pragma unroll
       for (int k = 0; k < 8; ++k)
-        if (fkey(xa[k]) < r.a.tau) pw[k] = 0.0f;
+        if (xa[k] < r.ta) pw[k] = 0.0f;
     }
     if constexpr (RESID) {
       float xb[8], qw[8];
@@ -150,7 +153,7 @@ struct JobRows {
       if (r.b.tau != 0u) {
 #pragma unroll
         for (int k = 0; k < 8; ++k)
-          if (fkey(xb[k]) < r.b.tau) qw[k] = 0.0f;
+          if (xb[k] < r.tb) qw[k] = 0.0f;
       }
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
@@ -200,33 +203,26 @@ constexpr int kChunkGroups = kChunkElems / kGroup;
 template <typename T, bool RESID>
 constexpr int kChunkBatch = (sizeof(T) == 4 && RESID) ? kChunkGroups / 2 : kChunkGroups;
 
-// This lane's fp64 weight in one loaded group (8 elements), and its last positive index.
+// This lane's weight in one loaded group (8 elements: an fp32 sum, returned as fp64), and its
+// last positive index.
 template <typename T, bool RESID>
 __device__ __forceinline__ double lane_group_weight(const JobRows<T, RESID>& J, const Raw8<T, RESID>& x, int e,
                                                     int* last) {
   float w[8], pw[8];
   J.weights(x, w, pw);
-  double v = 0.0;
 #pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    v += static_cast<double>(w[k]);
+  for (int k = 0; k < 8; ++k)
     if (w[k] > 0.0f) *last = e + k;
-  }
-  return v;
+  return static_cast<double>(sum8(w));
 }
 
-// This lane's fp64 sums of the job weights (.x) and of p_a (.y) over one loaded group.
+// This lane's sums of the job weights (.x) and of p_a (.y) over one loaded group (8-term fp32
+// sums, returned as fp64).
 template <typename T, bool RESID>
 __device__ __forceinline__ double2 lane_group_sums(const JobRows<T, RESID>& J, const Raw8<T, RESID>& x) {
   float w[8], pw[8];
   J.weights(x, w, pw);
-  double a = 0.0, b = 0.0;
-#pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    a += static_cast<double>(w[k]);
-    b += static_cast<double>(pw[k]);
-  }
-  return make_double2(a, b);
+  return make_double2(static_cast<double>(sum8(w)), RESID ? static_cast<double>(sum8(pw)) : 0.0);
 }
 
 // Warp-level totals of one chunk [lo, hi) (hi - lo <= kChunkElems, lo a multiple of 8): the
@@ -256,6 +252,34 @@ __device__ double2 warp_chunk_totals(const JobRows<T, RESID>& J, int lo, int hi)
     }
   }
   return make_double2(warp_sum(sr), warp_sum(sp));
+}
+
+// Warp-level total of the job weights of one chunk [lo, hi) (8-term fp32 sums per lane, fp64
+// beyond), with a whole batch of groups in flight at once. Every lane gets it.
+template <typename T, bool RESID>
+__device__ double warp_chunk_weight(const JobRows<T, RESID>& J, int lo, int hi) {
+  constexpr int NB = kChunkBatch<T, RESID>;
+  const int lane = threadIdx.x & 31;
+  const bool full = J.vector_ok(lo, hi, kChunkElems);
+  double s = 0.0;
+#pragma unroll
+  for (int g0 = 0; g0 < kChunkGroups; g0 += NB) {
+    Raw8<T, RESID> x[NB];
+    if (full) {
+#pragma unroll
+      for (int g = 0; g < NB; ++g) J.load_full(lo + (g0 + g) * kGroup + lane * 8, x[g]);
+    } else {
+#pragma unroll
+      for (int g = 0; g < NB; ++g) J.load(lo + (g0 + g) * kGroup + lane * 8, hi, x[g]);
+    }
+#pragma unroll
+    for (int g = 0; g < NB; ++g) {
+      float w[8], pw[8];
+      J.weights(x[g], w, pw);
+      s += static_cast<double>(sum8(w));
+    }
+  }
+  return warp_sum(s);
 }
 
 // Reduce-scatter of eight per-lane values: lane l ends with the warp total of value

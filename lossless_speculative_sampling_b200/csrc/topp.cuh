@@ -51,20 +51,67 @@ struct TpSmem {
   DrawSmem draw;    // the general draw
 };
 
-// Bin and fixed-point mass of logit x (identical arithmetic in passes B and C).
-__device__ __forceinline__ void tp_bin(float x, float m, float c, int& b, uint32_t& u) {
-  const float d = (x - m) * c;                               // log2 weight, <= 0
-  const float t = fminf(d * -2.0f, 4096.0f);                 // -2 d, capped (also for -inf)
-  const float r = t + 12582912.0f;                           // rounded to an integer (1.5 * 2^23)
-  b = min(__float_as_int(r) - __float_as_int(12582912.0f), kTpBins - 1);
-  const float bf = fminf(r - 12582912.0f, static_cast<float>(kTpBins - 1));
-  const float y = ex2(fmaf(bf, 0.5f, d));                    // 2^(d + b/2)
-  u = __float_as_uint(y + 8.0f) - __float_as_uint(8.0f);     // y * 2^20, rounded to nearest
+// Bins and fixed-point masses of a logit pair, packed (identical arithmetic in passes B and
+// C). r = -2 (x - m) c + 1.5 * 2^23 rounds to the bin index in its low mantissa bits; values
+// too far below the maximum (and -inf) land in the last bin with a zero or negligible mass.
+constexpr float kTpMagic = 12582912.0f;  // 1.5 * 2^23
+
+__device__ __forceinline__ f32x2 tp_r2(float x0, float x1, f32x2 mm, f32x2 cc, f32x2& d) {
+  d = mul2(sub2(pack2(x0, x1), mm), cc);  // log2 weights, <= 0
+  return fma2(d, pack2(-2.0f, -2.0f), pack2(kTpMagic, kTpMagic));
 }
 
-__device__ __forceinline__ int tp_bin_only(float x, float m, float c) {
-  const float t = fminf((x - m) * c * -2.0f, 4096.0f);
-  return min(__float_as_int(t + 12582912.0f) - __float_as_int(12582912.0f), kTpBins - 1);
+__device__ __forceinline__ void tp_bin2(float x0, float x1, f32x2 mm, f32x2 cc, int& b0, int& b1, uint32_t& u0,
+                                        uint32_t& u1) {
+  f32x2 d;
+  const f32x2 r = tp_r2(x0, x1, mm, cc, d);
+  float r0, r1, f0, f1, a0, a1, y0, y1;
+  unpack2(r, r0, r1);
+  b0 = min(__float_as_int(r0) - __float_as_int(kTpMagic), kTpBins - 1);
+  b1 = min(__float_as_int(r1) - __float_as_int(kTpMagic), kTpBins - 1);
+  unpack2(sub2(r, pack2(kTpMagic, kTpMagic)), f0, f1);
+  f0 = fminf(f0, static_cast<float>(kTpBins - 1));
+  f1 = fminf(f1, static_cast<float>(kTpBins - 1));
+  unpack2(fma2(pack2(f0, f1), pack2(0.5f, 0.5f), d), a0, a1);            // d + b/2
+  unpack2(add2(pack2(ex2(a0), ex2(a1)), pack2(8.0f, 8.0f)), y0, y1);      // 8 + 2^(d + b/2)
+  u0 = __float_as_uint(y0) - __float_as_uint(8.0f);                       // 2^(d + b/2) * 2^20, rounded
+  u1 = __float_as_uint(y1) - __float_as_uint(8.0f);
+}
+
+// Visit this thread's elements of row [0, V): f8(x) for every 8-element vector of the aligned
+// body (kLoads 16-byte loads in flight), f8 with -inf padding for the scalar edges.
+template <typename T, int kLoads, typename F>
+__device__ __forceinline__ void tp_for_each8(const T* __restrict__ row, int V, F&& f8) {
+  constexpr int N = Vec<T>::N;
+  int a0, a1;
+  vec_range(row, 0, V, a0, a1);
+  for (int v = threadIdx.x; v < a0; v += blockDim.x) {
+    float x[8] = {load_elem(row + v), -INFINITY, -INFINITY, -INFINITY, -INFINITY, -INFINITY, -INFINITY, -INFINITY};
+    f8(x);
+  }
+  for (int v = a1 + threadIdx.x; v < V; v += blockDim.x) {
+    float x[8] = {load_elem(row + v), -INFINITY, -INFINITY, -INFINITY, -INFINITY, -INFINITY, -INFINITY, -INFINITY};
+    f8(x);
+  }
+  const int step = blockDim.x * N;
+  for (int v = a0 + threadIdx.x * N; v < a1; v += kLoads * step) {
+    uint4 raw[kLoads];
+#pragma unroll
+    for (int i = 0; i < kLoads; ++i)
+      if (v + i * step < a1) raw[i] = __ldcg(reinterpret_cast<const uint4*>(row + v + i * step));
+#pragma unroll
+    for (int i = 0; i < kLoads; ++i) {
+      if (v + i * step < a1) {
+        float x[8];
+        Vec<T>::unpack(raw[i], x);
+        if constexpr (N == 4) {
+#pragma unroll
+          for (int k = 4; k < 8; ++k) x[k] = -INFINITY;
+        }
+        f8(x);
+      }
+    }
+  }
 }
 
 // 2^(-b/2) * 2^-20 in fp64: the weight of one fixed-point unit of bin b.
@@ -156,7 +203,12 @@ __device__ RowStat tp_row_stats(const T* __restrict__ row, int V, float Tv, floa
   if (V > kTpMaxV) {
     // general path: normaliser by a block reduction, then the general select
     double s = 0.0;
-    tp_for_each<T, 4>(row, V, [&](float x) { s += static_cast<double>(ex2((x - m) * c)); });
+    tp_for_each8<T, 4>(row, V, [&](const float (&x)[8]) {
+      float g = 0.0f;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) g += ex2((x[k] - m) * c);
+      s += static_cast<double>(g);
+    });
     __syncthreads();
     s = block_sum(s, reinterpret_cast<double*>(&sm.mass[0]));
     st.s = static_cast<float>(s);
@@ -166,11 +218,17 @@ __device__ RowStat tp_row_stats(const T* __restrict__ row, int V, float Tv, floa
   // pass B: thread-private fixed-point bin masses
 #pragma unroll
   for (int b = 0; b < kTpBins; ++b) sm.priv[b][threadIdx.x] = 0u;
-  tp_for_each<T, 4>(row, V, [&](float x) {
-    int b;
-    uint32_t u;
-    tp_bin(x, m, c, b, u);
-    atomicAdd(&sm.priv[b][threadIdx.x], u);  // a reduction (no return value): no chain through memory
+  const f32x2 mm = pack2(m, m), cc = pack2(c, c);
+  tp_for_each8<T, 4>(row, V, [&](const float (&x)[8]) {
+#pragma unroll
+    for (int k = 0; k < 8; k += 2) {
+      int b0, b1;
+      uint32_t u0, u1;
+      tp_bin2(x[k], x[k + 1], mm, cc, b0, b1, u0, u1);
+      // reductions (no return value): no dependence chain through shared memory
+      if (u0 != 0u) atomicAdd(&sm.priv[b0][threadIdx.x], u0);
+      if (u1 != 0u) atomicAdd(&sm.priv[b1][threadIdx.x], u1);
+    }
   });
   __syncthreads();
   // bin totals: warp w reduces bins w, w + kTpWarps, ...
@@ -245,19 +303,30 @@ __device__ RowStat tp_row_stats(const T* __restrict__ row, int V, float Tv, floa
     const int shift = 6 * (levels - 1 - lv);
 #pragma unroll
     for (int d = 0; d < 64; ++d) sm.priv[d][threadIdx.x] = 0u;
-    tp_for_each<T, 4>(row, V, [&](float x) {
-      if (tp_bin_only(x, m, c) != bstar) return;
-      const uint32_t k = fkey(x) >> kKeyShift;
-      if (k < klo || k > khi) {
-        outside = true;
-        return;
+    const float rstar = kTpMagic + static_cast<float>(bstar);  // r of the elements of bin b*
+    tp_for_each8<T, 4>(row, V, [&](const float (&x)[8]) {
+#pragma unroll
+      for (int k = 0; k < 8; k += 2) {
+        f32x2 d;
+        float r0, r1;
+        unpack2(tp_r2(x[k], x[k + 1], mm, cc, d), r0, r1);
+        if (r0 != rstar && r1 != rstar) continue;
+        int b0, b1;
+        uint32_t u0, u1;
+        tp_bin2(x[k], x[k + 1], mm, cc, b0, b1, u0, u1);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          if ((h ? r1 : r0) != rstar) continue;
+          const uint32_t kk = fkey(x[k + h]) >> kKeyShift;
+          if (kk < klo || kk > khi) {
+            outside = true;
+            continue;
+          }
+          const uint32_t off = kk - klo;
+          if (shift + 6 < 32 && (off >> (shift + 6)) != prefix) continue;
+          atomicAdd(&sm.priv[(off >> shift) & 63u][threadIdx.x], h ? u1 : u0);
+        }
       }
-      const uint32_t off = k - klo;
-      if (shift + 6 < 32 && (off >> (shift + 6)) != prefix) return;
-      int b;
-      uint32_t u;
-      tp_bin(x, m, c, b, u);
-      atomicAdd(&sm.priv[(off >> shift) & 63u][threadIdx.x], u);
     });
     if (__syncthreads_or(outside)) {
       if (threadIdx.x == 0) sm.fallback = 1;
@@ -332,8 +401,8 @@ __device__ int tp_row_draw(const T* __restrict__ row, int V, const RowStat& st, 
     return y;
   }
   for (int ch = warp; ch < nch; ch += kTpWarps) {
-    const double2 t = warp_chunk_totals(J, ch * kChunkElems, min(V, (ch + 1) * kChunkElems));
-    if (lane == 0) sm.ctot[ch] = t.x;
+    const double t = warp_chunk_weight(J, ch * kChunkElems, min(V, (ch + 1) * kChunkElems));
+    if (lane == 0) sm.ctot[ch] = t;
   }
   __syncthreads();
   if (warp == 0) {
