@@ -218,9 +218,9 @@ psispec_status sample_draft_impl(const T* draft, int B, int K, int V, const floa
   Carver c(ws);
   SampleWs w = carve_sample(c, rows, V);
   RowStat* stats = out_stats ? out_stats : w.st.stats;
-  // rows of requests with a top-p cut skip the streaming pass: the row kernel's top-p CTAs
-  // read them whole
-  psispec_status s = launch_stream<T>(draft, rows, K, nullptr, V, temperature, B, w.st.parts, st, top_p);
+  // every row through the streaming pass (maximum and normaliser); the row kernel's top-p
+  // CTAs then find the thresholds
+  psispec_status s = launch_stream<T>(draft, rows, K, nullptr, V, temperature, B, w.st.parts, st);
   if (s != PSISPEC_OK) return s;
   unsigned tgrid = 1;
   if ((s = prepare_topp(sample_rows_kernel<T>, rows, &tgrid)) != PSISPEC_OK) return s;
@@ -260,10 +260,10 @@ psispec_status verify_linear_impl(const T* tgt, const T* drf, int B, int K, int 
   a.jobs = w.jobs;
   // the first streaming pass also clears the request arrival counters
   psispec_status s =
-      launch_stream<T>(tgt, rows_t, K + 1, nullptr, V, temperature, B, w.t.parts, st, top_p, w.cnt, B);
+      launch_stream<T>(tgt, rows_t, K + 1, nullptr, V, temperature, B, w.t.parts, st, nullptr, w.cnt, B);
   if (s != PSISPEC_OK) return s;
   if (rows_d > 0 &&
-      (s = launch_stream<T>(drf, rows_d, K, nullptr, V, temperature, B, w.d.parts, st, top_p)) != PSISPEC_OK)
+      (s = launch_stream<T>(drf, rows_d, K, nullptr, V, temperature, B, w.d.parts, st)) != PSISPEC_OK)
     return s;
   // one row kernel: warps for the requests without a top-p cut, whole CTAs for the others
   unsigned tgrid = 1;

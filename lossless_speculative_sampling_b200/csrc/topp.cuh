@@ -40,6 +40,7 @@ struct TpSmem {
   double mass[kTpBins];                           // bin or digit masses
   double ctot[kTpMaxChunks];                      // kept weight per chunk (pass D)
   float fred[kTpWarps];
+  float stage[kTpWarps][256];  // per-warp compaction buffer of pass C
   RowStat st;
   double above, total, target;
   uint32_t prefix;
@@ -304,30 +305,87 @@ __device__ RowStat tp_row_stats(const T* __restrict__ row, int V, float Tv, floa
 #pragma unroll
     for (int d = 0; d < 64; ++d) sm.priv[d][threadIdx.x] = 0u;
     const float rstar = kTpMagic + static_cast<float>(bstar);  // r of the elements of bin b*
-    tp_for_each8<T, 4>(row, V, [&](const float (&x)[8]) {
-#pragma unroll
-      for (int k = 0; k < 8; k += 2) {
+    // an element of bin b*: its fixed-point mass goes to the counter of its digit
+    auto add = [&](float x) {
+      const uint32_t kk = fkey(x) >> kKeyShift;
+      if (kk < klo || kk > khi) {
+        outside = true;
+        return;
+      }
+      const uint32_t off = kk - klo;
+      if (shift + 6 < 32 && (off >> (shift + 6)) != prefix) return;
+      int b0, b1;
+      uint32_t u0, u1;
+      tp_bin2(x, -INFINITY, mm, cc, b0, b1, u0, u1);
+      atomicAdd(&sm.priv[(off >> shift) & 63u][threadIdx.x], u0);
+    };
+    {
+      constexpr int N = Vec<T>::N;
+      constexpr int kLoads = 4;
+      int a0, a1;
+      vec_range(row, 0, V, a0, a1);
+      for (int v = threadIdx.x; v < a0; v += blockDim.x) {  // scalar edges: few elements
+        const float x = load_elem(row + v);
         f32x2 d;
         float r0, r1;
-        unpack2(tp_r2(x[k], x[k + 1], mm, cc, d), r0, r1);
-        if (r0 != rstar && r1 != rstar) continue;
-        int b0, b1;
-        uint32_t u0, u1;
-        tp_bin2(x[k], x[k + 1], mm, cc, b0, b1, u0, u1);
+        unpack2(tp_r2(x, -INFINITY, mm, cc, d), r0, r1);
+        if (r0 == rstar) add(x);
+      }
+      for (int v = a1 + threadIdx.x; v < V; v += blockDim.x) {
+        const float x = load_elem(row + v);
+        f32x2 d;
+        float r0, r1;
+        unpack2(tp_r2(x, -INFINITY, mm, cc, d), r0, r1);
+        if (r0 == rstar) add(x);
+      }
+      // vector body in rounds every lane takes part in: the lanes flag the elements of bin b*,
+      // the warp compacts them into its staging buffer and shares the work on them evenly
+      const int nvec = (a1 - a0) / N;
+      const int rounds = (nvec + kTpThreads - 1) / kTpThreads;
+      float* stage = sm.stage[warp];
+      for (int r0i = 0; r0i < rounds; r0i += kLoads) {
+        uint4 raw[kLoads];
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          if ((h ? r1 : r0) != rstar) continue;
-          const uint32_t kk = fkey(x[k + h]) >> kKeyShift;
-          if (kk < klo || kk > khi) {
-            outside = true;
-            continue;
+        for (int i = 0; i < kLoads; ++i) {
+          const int vi = (r0i + i) * kTpThreads + threadIdx.x;
+          if (r0i + i < rounds && vi < nvec) raw[i] = __ldcg(reinterpret_cast<const uint4*>(row + a0 + vi * N));
+        }
+#pragma unroll
+        for (int i = 0; i < kLoads; ++i) {
+          if (r0i + i >= rounds) break;  // uniform: every thread runs the same rounds
+          const int vi = (r0i + i) * kTpThreads + threadIdx.x;
+          float x[8];
+          uint32_t mask = 0u;
+          if (vi < nvec) {
+            Vec<T>::unpack(raw[i], x);
+#pragma unroll
+            for (int k = 0; k < N; k += 2) {
+              f32x2 d;
+              float ra, rb;
+              unpack2(tp_r2(x[k], x[k + 1], mm, cc, d), ra, rb);
+              mask |= (ra == rstar ? 1u : 0u) << k;
+              mask |= (rb == rstar ? 1u : 0u) << (k + 1);
+            }
           }
-          const uint32_t off = kk - klo;
-          if (shift + 6 < 32 && (off >> (shift + 6)) != prefix) continue;
-          atomicAdd(&sm.priv[(off >> shift) & 63u][threadIdx.x], h ? u1 : u0);
+          const int cnt = __popc(mask);
+          int incl = cnt;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+          }
+          const int total = __shfl_sync(0xffffffffu, incl, 31);
+          if (total == 0) continue;
+          int pos = incl - cnt;
+#pragma unroll
+          for (int k = 0; k < N; ++k)
+            if (mask & (1u << k)) stage[pos++] = x[k];
+          __syncwarp();
+          for (int j = lane; j < total; j += 32) add(stage[j]);
+          __syncwarp();
         }
       }
-    });
+    }
     if (__syncthreads_or(outside)) {
       if (threadIdx.x == 0) sm.fallback = 1;
       break;
@@ -384,6 +442,115 @@ __device__ RowStat tp_row_stats(const T* __restrict__ row, int V, float Tv, floa
   st.s_kept = static_cast<float>(sm.base);
   __syncthreads();
   return st;
+}
+
+// Top-p threshold of a bf16 row whose maximum m and normaliser s are already known (from the
+// streaming pass): every element with the same logit has the same weight, so counting the
+// elements of each of the kTpWindow representable values just below m gives their masses
+// exactly (count times one weight). One pass over the row, no exponential per element; the
+// threshold is the first value, from m down, at which the cumulative mass reaches top_p * s.
+// Returns false (and leaves st alone) when the window holds less than that.
+constexpr int kTpWindow = 2048;
+
+// The logit value of a 16-bit order key of a bf16 number.
+__device__ __forceinline__ float key16_value(uint32_t k16) { return key_value(k16 << 16); }
+
+template <typename T>
+__device__ bool tp_window_select(const T* __restrict__ row, int V, float tp, RowStat& st, TpSmem& sm) {
+  static_assert(sizeof(T) == 2, "bf16 rows");
+  static_assert(kTpWarps * kTpWindow <= kTpBins * kTpThreads, "window counts reuse the private counters");
+  uint32_t* cnt = &sm.priv[0][0];  // [kTpWarps][kTpWindow]
+  const int warp = threadIdx.x >> 5;
+  for (int i = threadIdx.x; i < kTpWarps * kTpWindow; i += kTpThreads) cnt[i] = 0u;
+  __syncthreads();
+  const uint32_t km = fkey(st.m) >> 16;
+  uint32_t* mine = cnt + warp * kTpWindow;
+  tp_for_each8<T, 4>(row, V, [&](const float (&x)[8]) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const uint32_t o = km - (fkey(x[k]) >> 16);
+      if (o < static_cast<uint32_t>(kTpWindow)) atomicAdd(&mine[o], 1u);
+    }
+  });
+  __syncthreads();
+  // masses of offsets [8t, 8t + 8) in thread t, scanned in thread order
+  constexpr int kPer = kTpWindow / kTpThreads;
+  double mass[kPer];
+  double tsum = 0.0;
+#pragma unroll
+  for (int j = 0; j < kPer; ++j) {
+    const int o = threadIdx.x * kPer + j;
+    uint32_t c = 0u;
+#pragma unroll
+    for (int w = 0; w < kTpWarps; ++w) c += cnt[w * kTpWindow + o];
+    mass[j] = 0.0;
+    if (c != 0u && km >= static_cast<uint32_t>(o))
+      mass[j] = static_cast<double>(c) * static_cast<double>(ex2((key16_value(km - o) - st.m) * st.c));
+    tsum += mass[j];
+  }
+  double total;
+  const double C0 = block_exclusive_scan(tsum, sm.mass, &total);
+  const double target = static_cast<double>(tp) * static_cast<double>(st.s);
+  if (!(total >= target)) return false;  // the threshold lies below the window (uniform)
+  if (threadIdx.x == 0) sm.bin = -1;
+  __syncthreads();
+  if (C0 < target && C0 + tsum >= target) {  // the thread whose offsets cross the target
+    double run = C0;
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      if (mass[j] > 0.0 && run + mass[j] >= target) {
+        sm.bin = threadIdx.x * kPer + j;
+        sm.base = run + mass[j];
+        break;
+      }
+      run += mass[j];
+    }
+  }
+  __syncthreads();
+  int ostar = sm.bin;
+  if (ostar < 0) {
+    // a target of zero (the maximum's value alone), or rounding at a thread boundary: the
+    // first offset whose cumulative mass reaches the target, by thread 0
+    if (threadIdx.x == 0) {
+      double run = 0.0;
+      int pick = -1;
+      for (int o = 0; o < kTpWindow && pick < 0; ++o) {
+        uint32_t c = 0u;
+        for (int w = 0; w < kTpWarps; ++w) c += cnt[w * kTpWindow + o];
+        if (c == 0u || km < static_cast<uint32_t>(o)) continue;
+        run += static_cast<double>(c) * static_cast<double>(ex2((key16_value(km - o) - st.m) * st.c));
+        if (run >= target) pick = o;
+      }
+      sm.bin = pick;
+      sm.base = run;
+    }
+    __syncthreads();
+    ostar = sm.bin;
+    if (ostar < 0) return false;  // uniform
+  }
+  st.tau = (km - static_cast<uint32_t>(ostar)) << 16;
+  st.s_kept = static_cast<float>(sm.base);
+  __syncthreads();
+  return true;
+}
+
+// Statistics of a row of a request with a top-p cut: maximum and normaliser from the row's
+// chunk partials, the threshold from the value window (bf16), else passes A-C over the row.
+template <typename T>
+__device__ RowStat tp_row_stats_partials(const T* __restrict__ row, int V, float Tv, float tp,
+                                         const Partial* __restrict__ pp, TpSmem& sm) {
+  if (threadIdx.x < 32) {
+    const RowStat s0 = warp_finalize_pick(pp, nchunks_for(V), Tv, 0.0f, false).st;
+    if (threadIdx.x == 0) sm.st = s0;
+  }
+  __syncthreads();
+  RowStat st = sm.st;
+  __syncthreads();
+  if (st.status != 0) return st;
+  if constexpr (sizeof(T) == 2) {
+    if (tp_window_select<T>(row, V, tp, st, sm)) return st;
+  }
+  return tp_row_stats(row, V, Tv, tp, sm);
 }
 
 // Pass D: inverse-CDF draw with uniform u over the kept weights of the row, in vocabulary
@@ -493,7 +660,8 @@ __global__ void __launch_bounds__(kTpThreads, 2) sample_rows_kernel(const T* __r
     const int b = row / K;
     if (!request_cut(temperature, top_p, b)) continue;
     const T* rp = draft + static_cast<size_t>(row) * V;
-    const RowStat st = tp_row_stats(rp, V, temperature[b], top_p[b], sm);
+    const RowStat st =
+        tp_row_stats_partials(rp, V, temperature[b], top_p[b], parts + static_cast<size_t>(row) * nchunks_for(V), sm);
     float q = -1.0f;
     const int y = st.status == 0 ? tp_row_draw(rp, V, st, u[row], sm, &q) : -1;
     if (threadIdx.x == 0) {
@@ -532,7 +700,8 @@ __global__ void __launch_bounds__(kTpThreads, 2) verify_rows_kernel(const T* __r
     const int b = is_draft ? row / K : row / (K + 1);
     if (!request_cut(a.temperature, a.top_p, b)) continue;
     const T* rp = (is_draft ? drf : tgt) + static_cast<size_t>(row) * V;
-    const RowStat st = tp_row_stats(rp, V, a.temperature[b], a.top_p[b], sm);
+    const Partial* pp = (is_draft ? a.parts_d : a.parts_t) + static_cast<size_t>(row) * nchunks_for(V);
+    const RowStat st = tp_row_stats_partials(rp, V, a.temperature[b], a.top_p[b], pp, sm);
     if (threadIdx.x == 0) (is_draft ? a.stats_d : a.stats_t)[row] = st;
     if (block_arrive_last(&a.cnt[b], per_req, &sm.flag) && threadIdx.x < 32)
       warp_decide_request<T>(b, tgt, drf, K, V, a.tokens, a.stats_t, a.stream_draft ? a.stats_d : a.dstats_in,
