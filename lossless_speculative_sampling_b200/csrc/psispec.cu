@@ -142,7 +142,8 @@ int64_t want_slots(int64_t work_warps, int warps, Kern kernel, int block, int sm
 template <typename T>
 psispec_status launch_stream(const T* base, int64_t rows, int rows_per_req, const int32_t* row_req, int V,
                              const float* temperature, int nreq, Partial* parts, cudaStream_t st,
-                             const float* skip_top_p = nullptr, int32_t* zero = nullptr, int nzero = 0) {
+                             const float* top_p = nullptr, int skip_uncut = 0, int32_t* zero = nullptr,
+                             int nzero = 0) {
   const int64_t chunks = rows * nchunks_for(V);
   const bool aligned = (reinterpret_cast<uintptr_t>(base) & 15u) == 0 && (int64_t(V) * sizeof(T)) % 16 == 0;
   if (aligned) {
@@ -158,20 +159,23 @@ psispec_status launch_stream(const T* base, int64_t rows, int rows_per_req, cons
     const int64_t slots = static_cast<int64_t>(sms) * (occ > 0 ? occ : 1);
     const unsigned grid = static_cast<unsigned>(want < slots ? want : slots);
     return launch(stream_partials_tma_kernel<T>, grid, kThreads, smem, st, base, rows_per_req, row_req, V, chunks,
-                  temperature, skip_top_p, nreq, parts, zero, nzero);
+                  temperature, top_p, skip_uncut, nreq, parts, zero, nzero);
   }
   return launch(stream_partials_kernel<T>, persistent_grid(stream_partials_kernel<T>, chunks), kThreads, 0, st, base,
-                rows_per_req, row_req, V, chunks, temperature, skip_top_p, parts, zero, nzero);
+                rows_per_req, row_req, V, chunks, temperature, top_p, skip_uncut, parts, zero, nzero);
 }
 
-// Row statistics of a [rows, V] tensor (the tree's statistics pass).
+// Row statistics of a [rows, V] tensor (the tree's statistics pass); with skip_uncut, the rows
+// of requests with T > 0 and no top-p cut are left out.
 template <typename T>
 psispec_status launch_stats(const T* base, int64_t rows, int rows_per_req, const int32_t* row_req, int V,
-                            const float* temperature, int nreq, const float* top_p, StatsWs ws, cudaStream_t st) {
-  psispec_status s = launch_stream<T>(base, rows, rows_per_req, row_req, V, temperature, nreq, ws.parts, st);
+                            const float* temperature, int nreq, const float* top_p, int skip_uncut, StatsWs ws,
+                            cudaStream_t st) {
+  psispec_status s = launch_stream<T>(base, rows, rows_per_req, row_req, V, temperature, nreq, ws.parts, st, top_p,
+                                      skip_uncut);
   if (s != PSISPEC_OK) return s;
   return launch(row_finalize_kernel<T>, static_cast<unsigned>(rows), kThreads, 0, st, base, rows_per_req, row_req, V,
-                temperature, top_p, ws.parts, ws.stats);
+                temperature, top_p, ws.parts, ws.stats, skip_uncut);
 }
 
 // The draw jobs of a verification call: totals pass (bulk-copy ring when the rows allow it),
@@ -260,7 +264,7 @@ psispec_status verify_linear_impl(const T* tgt, const T* drf, int B, int K, int 
   a.jobs = w.jobs;
   // the first streaming pass also clears the request arrival counters
   psispec_status s =
-      launch_stream<T>(tgt, rows_t, K + 1, nullptr, V, temperature, B, w.t.parts, st, nullptr, w.cnt, B);
+      launch_stream<T>(tgt, rows_t, K + 1, nullptr, V, temperature, B, w.t.parts, st, nullptr, 0, w.cnt, B);
   if (s != PSISPEC_OK) return s;
   if (rows_d > 0 &&
       (s = launch_stream<T>(drf, rows_d, K, nullptr, V, temperature, B, w.d.parts, st)) != PSISPEC_OK)
@@ -274,29 +278,35 @@ psispec_status verify_linear_impl(const T* tgt, const T* drf, int B, int K, int 
   return launch_draws<T>(tgt, drf, V, B, w.t.parts, w.jobs, w.draw_tc, w.draw_tg, out_tokens, st);
 }
 
-// The cluster tree walk with CL CTAs per trie; PSISPEC_ERR_UNSUPPORTED when V needs larger
-// slices than shared memory holds or the device cannot schedule such a cluster.
+// Launch configuration of the cluster tree walk with CL CTAs per trie; PSISPEC_ERR_UNSUPPORTED
+// when V needs larger slices than shared memory holds or the device cannot schedule such a
+// cluster. cfg.attrs points at attr; *dbuf tells whether a second r' buffer fits.
 template <typename T, int CL>
-psispec_status launch_tree_cluster(const T* tgt, const T* drf, int B, int V, const int32_t* offs,
-                                   const int32_t* parent, const int32_t* tokens, const RowStat* ts, const RowStat* ds,
-                                   const float* u_acc, const float* u_res, int max_depth, int32_t* out_path,
-                                   int32_t* out_tokens, int32_t* out_len, cudaStream_t st) {
-  const int slice = tree_slice(V, CL);
-  if (slice > kTreeMaxSlice) return PSISPEC_ERR_UNSUPPORTED;
-  const int smem = 2 * slice * static_cast<int>(sizeof(float));
+psispec_status tree_cluster_config(int B, int V, cudaStream_t st, cudaLaunchConfig_t& cfg,
+                                   cudaLaunchAttribute (&attr)[1], int* dbuf) {
+  const size_t slice_bytes = static_cast<size_t>(tree_slice(V, CL)) * sizeof(float);
   auto kernel = tree_walk_cluster_kernel<T, CL>;
+  int dev = 0, optin = 0;
+  cudaFuncAttributes fa;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess ||
+      cudaFuncGetAttributes(&fa, kernel) != cudaSuccess)
+    return PSISPEC_ERR_CUDA;
+  const size_t room = static_cast<size_t>(optin) > fa.sharedSizeBytes ? optin - fa.sharedSizeBytes : 0;
+  if (2 * slice_bytes > room) return PSISPEC_ERR_UNSUPPORTED;
+  *dbuf = 3 * slice_bytes <= room;
+  const int smem = static_cast<int>((*dbuf ? 3 : 2) * slice_bytes);
   if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return PSISPEC_ERR_CUDA;
   if (CL > 8 && cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
     cudaGetLastError();
     return PSISPEC_ERR_UNSUPPORTED;
   }
-  cudaLaunchConfig_t cfg = {};
+  cfg = cudaLaunchConfig_t{};
   cfg.gridDim = dim3(static_cast<unsigned>(B) * CL);
   cfg.blockDim = dim3(kTreeWalkThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = CL;
   attr[0].val.clusterDim.y = 1;
@@ -308,10 +318,7 @@ psispec_status launch_tree_cluster(const T* tgt, const T* drf, int B, int V, con
     cudaGetLastError();
     return PSISPEC_ERR_UNSUPPORTED;
   }
-  return cudaLaunchKernelEx(&cfg, kernel, tgt, drf, V, offs, parent, tokens, ts, ds, u_acc, u_res, max_depth, out_path,
-                            out_tokens, out_len) == cudaSuccess
-             ? PSISPEC_OK
-             : PSISPEC_ERR_CUDA;
+  return PSISPEC_OK;
 }
 
 template <typename T>
@@ -319,25 +326,41 @@ psispec_status verify_tree_impl(const T* tgt, const T* drf, int B, int N, int V,
                                 const int32_t* parent, const int32_t* tokens, const float* u_acc, const float* u_res,
                                 const float* temperature, const float* top_p, int max_depth, int32_t* out_path,
                                 int32_t* out_tokens, int32_t* out_len, void* ws, cudaStream_t st) {
-  const int ns = nslices_for(V);
   Carver c(ws);
   TreeWs w = carve_tree(c, N, V);
-  psispec_status s = launch(node_request_kernel, static_cast<unsigned>(B), 128, 0, st, offs, B, N, w.row_req);
+  // the walk: one cluster per trie, the node's rows staged across its CTAs' shared memory (16
+  // CTAs where the device can schedule such clusters, else 8), else one CTA per trie
+  cudaLaunchConfig_t cfg;
+  cudaLaunchAttribute attr[1];
+  int CL = 16, dbuf = 0;
+  psispec_status s = tree_cluster_config<T, 16>(B, V, st, cfg, attr, &dbuf);
+  if (s == PSISPEC_ERR_UNSUPPORTED) {
+    CL = 8;
+    s = tree_cluster_config<T, 8>(B, V, st, cfg, attr, &dbuf);
+  }
+  if (s == PSISPEC_ERR_UNSUPPORTED) CL = 0;
+  else if (s != PSISPEC_OK) return s;
+  // the cluster walk finds the statistics of uncut requests' visited rows itself
+  const int lazy = CL != 0;
+  s = launch(node_request_kernel, static_cast<unsigned>(B), 128, 0, st, offs, B, N, w.row_req);
   if (s != PSISPEC_OK) return s;
-  s = launch_stats<T>(tgt, N, 1, w.row_req, V, temperature, B, top_p, w.t, st);
+  s = launch_stats<T>(tgt, N, 1, w.row_req, V, temperature, B, top_p, lazy, w.t, st);
   if (s != PSISPEC_OK) return s;
-  s = launch_stats<T>(drf, N, 1, w.row_req, V, temperature, B, top_p, w.d, st);
+  s = launch_stats<T>(drf, N, 1, w.row_req, V, temperature, B, top_p, lazy, w.d, st);
   if (s != PSISPEC_OK) return s;
-  // one cluster per trie, the node's rows staged across its CTAs' shared memory: 16 CTAs
-  // where the device can schedule such clusters, else 8
-  psispec_status s16 = launch_tree_cluster<T, 16>(tgt, drf, B, V, offs, parent, tokens, w.t.stats, w.d.stats, u_acc,
-                                                  u_res, max_depth, out_path, out_tokens, out_len, st);
-  if (s16 != PSISPEC_ERR_UNSUPPORTED) return s16;
-  psispec_status s8 = launch_tree_cluster<T, 8>(tgt, drf, B, V, offs, parent, tokens, w.t.stats, w.d.stats, u_acc,
-                                                u_res, max_depth, out_path, out_tokens, out_len, st);
-  if (s8 != PSISPEC_ERR_UNSUPPORTED) return s8;
-  return launch(tree_walk_kernel<T>, static_cast<unsigned>(B), kTreeThreads, 0, st, tgt, drf, V, offs, parent, tokens,
-                w.t.stats, w.d.stats, u_acc, u_res, max_depth, out_path, out_tokens, out_len);
+  cudaError_t e = cudaSuccess;
+  if (CL == 16)
+    e = cudaLaunchKernelEx(&cfg, tree_walk_cluster_kernel<T, 16>, tgt, drf, V, offs, parent, tokens,
+                           static_cast<const RowStat*>(w.t.stats), static_cast<const RowStat*>(w.d.stats), u_acc,
+                           u_res, temperature, top_p, lazy, dbuf, max_depth, out_path, out_tokens, out_len);
+  else if (CL == 8)
+    e = cudaLaunchKernelEx(&cfg, tree_walk_cluster_kernel<T, 8>, tgt, drf, V, offs, parent, tokens,
+                           static_cast<const RowStat*>(w.t.stats), static_cast<const RowStat*>(w.d.stats), u_acc,
+                           u_res, temperature, top_p, lazy, dbuf, max_depth, out_path, out_tokens, out_len);
+  else
+    return launch(tree_walk_kernel<T>, static_cast<unsigned>(B), kTreeThreads, 0, st, tgt, drf, V, offs, parent,
+                  tokens, w.t.stats, w.d.stats, u_acc, u_res, max_depth, out_path, out_tokens, out_len);
+  return e == cudaSuccess ? PSISPEC_OK : PSISPEC_ERR_CUDA;
 }
 
 bool bad_dtype(int dtype) { return dtype != PSISPEC_F32 && dtype != PSISPEC_BF16; }

@@ -25,12 +25,20 @@ __device__ __forceinline__ float temp_scale(float T) {
   return T > 0.0f && T < INFINITY ? static_cast<float>(1.4426950408889634 / static_cast<double>(T)) : 0.0f;
 }
 
-// Scale c of a request's rows for the streaming pass: -1 marks rows that the pass leaves to
-// the top-p row kernel (top_p given, below 1, and a positive temperature).
-__device__ __forceinline__ float stream_scale(const float* __restrict__ temperature, const float* __restrict__ top_p,
+// Whether a request samples at a positive temperature with no top-p cut: its row statistics
+// are then the maximum and the sum alone, which the cluster tree walk computes itself on the
+// rows it visits.
+__device__ __forceinline__ bool uncut_request(const float* __restrict__ temperature, const float* __restrict__ top_p,
                                               int req) {
+  return temp_scale(temperature[req]) != 0.0f && !(top_p[req] < 1.0f);
+}
+
+// Scale c of a request's rows for the streaming pass, or -1 for the rows it leaves alone: with
+// skip_uncut set, those of the requests uncut_request selects.
+__device__ __forceinline__ float stream_scale(const float* __restrict__ temperature, const float* __restrict__ top_p,
+                                              int skip_uncut, int req) {
   const float c = temp_scale(temperature[req]);
-  return (top_p != nullptr && c != 0.0f && top_p[req] < 1.0f) ? -1.0f : c;
+  return skip_uncut && c != 0.0f && !(top_p[req] < 1.0f) ? -1.0f : c;
 }
 
 // Request of a row: rows_per_req consecutive rows per request, or an explicit table.
@@ -153,15 +161,15 @@ __device__ __forceinline__ Partial warp_chunk_partial(const T* __restrict__ row,
 }
 
 // The streaming pass: persistent warps over every chunk of a [rows, V] tensor, each chunk
-// read once, one partial per chunk (parts[row * nchunks + chunk]). With skip_top_p set, the
-// rows of requests with a top-p cut are left alone (the top-p row kernel reads them). CTA 0
+// read once, one partial per chunk (parts[row * nchunks + chunk]), except the rows that
+// stream_scale marks. CTA 0
 // also clears the nzero arrival counters at `zero` that the call's later kernels use.
 template <typename T>
 __global__ void __launch_bounds__(kThreads, 4) stream_partials_kernel(const T* __restrict__ base, int rows_per_req,
                                                                     const int32_t* __restrict__ row_req, int V,
                                                                     int64_t total_chunks,
                                                                     const float* __restrict__ temperature,
-                                                                    const float* __restrict__ skip_top_p,
+                                                                    const float* __restrict__ top_p, int skip_uncut,
                                                                     Partial* __restrict__ parts,
                                                                     int32_t* __restrict__ zero, int nzero) {
   if (blockIdx.x == 0)
@@ -175,7 +183,7 @@ __global__ void __launch_bounds__(kThreads, 4) stream_partials_kernel(const T* _
   const int drow = static_cast<int>(nwarps / nch), dchunk = static_cast<int>(nwarps - static_cast<int64_t>(drow) * nch);
 #pragma unroll 1
   for (; g < total_chunks; g += nwarps) {
-    const float c = stream_scale(temperature, skip_top_p, row_request(row, rows_per_req, row_req));
+    const float c = stream_scale(temperature, top_p, skip_uncut, row_request(row, rows_per_req, row_req));
     if (c >= 0.0f) {
       const T* rp = base + static_cast<size_t>(row) * V;
       const int c0 = chunk * kChunkElems, c1 = min(V, c0 + kChunkElems);
@@ -348,7 +356,8 @@ __global__ void __launch_bounds__(kThreads) stream_partials_tma_kernel(const T* 
                                                                         const int32_t* __restrict__ row_req, int V,
                                                                         int64_t total_chunks,
                                                                         const float* __restrict__ temperature,
-                                                                        const float* __restrict__ skip_top_p, int nreq,
+                                                                        const float* __restrict__ top_p, int skip_uncut,
+                                                                        int nreq,
                                                                         Partial* __restrict__ parts,
                                                                         int32_t* __restrict__ zero, int nzero) {
   if (blockIdx.x == 0)
@@ -358,7 +367,7 @@ __global__ void __launch_bounds__(kThreads) stream_partials_tma_kernel(const T* 
   __shared__ float scale[kScaleTable];
   const bool table = nreq <= kScaleTable;
   if (table)
-    for (int i = threadIdx.x; i < nreq; i += kThreads) scale[i] = stream_scale(temperature, skip_top_p, i);
+    for (int i = threadIdx.x; i < nreq; i += kThreads) scale[i] = stream_scale(temperature, top_p, skip_uncut, i);
   __syncthreads();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   unsigned char* ring = ring_smem + warp * kRing * kStageBytes<T>;
@@ -387,7 +396,7 @@ __global__ void __launch_bounds__(kThreads) stream_partials_tma_kernel(const T* 
   int64_t gi = g0;
   auto scale_of = [&](int r) {
     const int req = row_request(r, rows_per_req, row_req);
-    return table ? scale[req] : stream_scale(temperature, skip_top_p, req);
+    return table ? scale[req] : stream_scale(temperature, top_p, skip_uncut, req);
   };
   auto issue = [&](int i) {  // copy of this warp's i-th chunk into stage i % kRing (lane 0)
     if (gi < total_chunks && scale_of(irow) >= 0.0f) {
@@ -409,7 +418,7 @@ __global__ void __launch_bounds__(kThreads) stream_partials_tma_kernel(const T* 
     if (lane == 0) issue(i + kRing - 1);
     const int c0 = chunk * kChunkElems, n = min(V - c0, kChunkElems);
     const float c = scale_of(row);
-    if (c < 0.0f) {  // a row left to the top-p row kernel
+    if (c < 0.0f) {  // a row this pass leaves alone
       advance(row, chunk);
       continue;
     }
@@ -855,18 +864,20 @@ __device__ void block_topp_select(const T* __restrict__ rp, int V, float tp, Row
   __syncthreads();
 }
 
-// One CTA per row (the tree's statistics pass).
+// One CTA per row (the tree's statistics pass); rows that stream_scale marks are skipped here
+// too.
 template <typename T>
 __global__ void __launch_bounds__(kThreads) row_finalize_kernel(const T* __restrict__ base, int rows_per_req,
                                                                  const int32_t* __restrict__ row_req, int V,
                                                                  const float* __restrict__ temperature,
                                                                  const float* __restrict__ top_p,
                                                                  const Partial* __restrict__ parts,
-                                                                 RowStat* __restrict__ stats) {
+                                                                 RowStat* __restrict__ stats, int skip_uncut) {
   __shared__ ToppSmem sm;
   __shared__ RowStat sh_st;
   const int row = blockIdx.x, req = row_request(row, rows_per_req, row_req);
   const int nch = nchunks_for(V);
+  if (stream_scale(temperature, top_p, skip_uncut, req) < 0.0f) return;
   if (threadIdx.x < 32) {
     const RowStat st = warp_finalize_row(parts + static_cast<size_t>(row) * nch, nch, temperature[req]);
     if (threadIdx.x == 0) sh_st = st;

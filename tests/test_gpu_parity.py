@@ -174,6 +174,40 @@ def test_verify_tree_parity(V, dtype, T, top_p):
     compare_tree(out, ora)
 
 
+@pytest.mark.parametrize("V,dtype", [(20011, torch.bfloat16), (3001, torch.float32), (151936, torch.bfloat16)])
+def test_verify_tree_mixed_requests_and_data_errors(V, dtype):
+    """Per-trie temperature/top-p (uncut tries take the walk's own row maxima), -inf logits,
+    unaligned rows (odd V), and data errors confined to their trie."""
+    B, nodes = 8, 24
+    trie = synth.trie_topology(B, nodes, 6, 3, 91)
+    g = torch.Generator().manual_seed(91)
+    tgt = _rand_logits(g, (trie.N, V), torch.float32, 2.0, neg_inf_frac=0.1)
+    drf = tgt + torch.randn((trie.N, V), generator=g) * 0.7
+    Ts = torch.tensor([1.0, 0.8, 0.0, 1.0, 1.0, 1.0, 0.9, 1.2])
+    Ps = torch.tensor([1.0, 1.0, 1.0, 0.9, 1.0, 1.0, 0.95, 1.0])
+    off = trie.node_offsets
+    tgt[int(off[4]), 5] = float("nan")  # visited root row with a NaN: trie 4 is a data error
+    drf[int(off[5]), 7] = float("inf")  # root draft row with +inf (the root has children): trie 5
+    tgt[int(off[6]), :] = -float("inf")  # root target row without a finite logit: trie 6
+    tgt[int(off[7 + 1]) - 1, 3] = float("nan")  # a late node of trie 7: an error only if visited
+    tgt, drf = tgt.to(dtype), drf.to(dtype)
+    toks = torch.zeros(trie.N, dtype=torch.int32)
+    for n in range(trie.N):
+        if trie.children[n]:
+            picks = synth.gumbel_tokens(drf[n:n + 1].float().nan_to_num(0.0, 0.0), 1.0, 91 + n,
+                                        k=len(trie.children[n]))[0]
+            for k, c in enumerate(trie.children[n]):
+                toks[c] = int(picks[k])
+    ua, ur = synth.uniforms((trie.N,), 92), synth.uniforms((trie.N,), 93)
+    out = psispec.verify_tree(_cuda(tgt), _cuda(drf), _cuda(off), _cuda(trie.parent), _cuda(toks), _cuda(ua),
+                              _cuda(ur), _cuda(Ts), _cuda(Ps), 6)
+    ora = oracle.verify_tree(tgt, drf, off.numpy(), trie.parent.numpy(), toks.numpy(), ua, ur, Ts.numpy(),
+                             Ps.numpy(), 6)
+    assert ora["accept_len"][4] == ora["accept_len"][5] == ora["accept_len"][6] == -1
+    assert (ora["accept_len"][[0, 1, 2, 3]] >= 0).all()
+    compare_tree(out, ora)
+
+
 def test_branching_one_tree_equals_linear_gpu():
     B, K, V = 6, 5, 12000
     tgt, drf, ud, ua, ur, Ts, Ps = _linear_inputs(B, K, V, torch.bfloat16, 0.9, 0.95, 0.6, seed=31)
