@@ -72,15 +72,11 @@ LinearWs carve_linear(Carver& c, int64_t B, int64_t K, int64_t V) {
 }
 
 struct TreeWs {
-  StatsWs t, d;
-  int32_t* row_req;
+  StatsWs st;  // rows [0, N) of the verifier tensor, then [N, 2N) of the draft tensor
 };
 TreeWs carve_tree(Carver& c, int64_t N, int64_t V) {
-  const int ns = nchunks_for(V);
   TreeWs w;
-  w.t = carve_stats(c, N, ns);
-  w.d = carve_stats(c, N, ns);
-  w.row_req = c.take<int32_t>(N);
+  w.st = carve_stats(c, 2 * N, nchunks_for(V));
   return w;
 }
 
@@ -101,14 +97,6 @@ psispec_status launch(void (*kernel)(KArgs...), unsigned grid, unsigned block, s
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...) == cudaSuccess ? PSISPEC_OK : PSISPEC_ERR_CUDA;
-}
-
-// Request index of every node, from node_offsets (tree rows have no fixed count per request).
-__global__ void node_request_kernel(const int32_t* __restrict__ offs, int B, int N, int32_t* __restrict__ row_req) {
-  const int b = blockIdx.x;
-  if (b >= B) return;
-  const int lo = max(0, min(N, offs[b])), hi = max(lo, min(N, offs[b + 1]));
-  for (int n = lo + threadIdx.x; n < hi; n += blockDim.x) row_req[n] = b;
 }
 
 // Persistent grid for a warp-granular streaming kernel: one CTA per resident slot, fewer
@@ -137,15 +125,21 @@ int64_t want_slots(int64_t work_warps, int warps, Kern kernel, int block, int sm
   return want < 1 ? 1 : (want < slots ? want : slots);
 }
 
-// The streaming pass over a [rows, V] tensor: one partial per chunk. Aligned tensors go
+// Rows [0, rows) of one tensor, rows_per_req consecutive rows per request.
+template <typename T>
+RowSet<T> one_tensor(const T* base, int64_t rows, int rows_per_req, int nreq) {
+  return RowSet<T>{base, nullptr, rows, rows_per_req, nullptr, nreq};
+}
+
+// The streaming pass over `rows` rows of a row set: one partial per chunk. Aligned tensors go
 // through the bulk-copy ring kernel, others through plain 16-byte loads.
 template <typename T>
-psispec_status launch_stream(const T* base, int64_t rows, int rows_per_req, const int32_t* row_req, int V,
-                             const float* temperature, int nreq, Partial* parts, cudaStream_t st,
-                             const float* top_p = nullptr, int skip_uncut = 0, int32_t* zero = nullptr,
-                             int nzero = 0) {
+psispec_status launch_stream(RowSet<T> set, int64_t rows, int V, const float* temperature, int nreq, Partial* parts,
+                             cudaStream_t st, const float* top_p = nullptr, int skip_uncut = 0,
+                             int32_t* zero = nullptr, int nzero = 0) {
   const int64_t chunks = rows * nchunks_for(V);
-  const bool aligned = (reinterpret_cast<uintptr_t>(base) & 15u) == 0 && (int64_t(V) * sizeof(T)) % 16 == 0;
+  const bool aligned = (reinterpret_cast<uintptr_t>(set.a) & 15u) == 0 &&
+                       (reinterpret_cast<uintptr_t>(set.b) & 15u) == 0 && (int64_t(V) * sizeof(T)) % 16 == 0;
   if (aligned) {
     const int smem = (kThreads / 32) * kRing * kStageBytes<T>;
     if (cudaFuncSetAttribute(stream_partials_tma_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
@@ -158,24 +152,22 @@ psispec_status launch_stream(const T* base, int64_t rows, int rows_per_req, cons
     const int64_t want = (chunks + (kThreads / 32) - 1) / (kThreads / 32);
     const int64_t slots = static_cast<int64_t>(sms) * (occ > 0 ? occ : 1);
     const unsigned grid = static_cast<unsigned>(want < slots ? want : slots);
-    return launch(stream_partials_tma_kernel<T>, grid, kThreads, smem, st, base, rows_per_req, row_req, V, chunks,
-                  temperature, top_p, skip_uncut, nreq, parts, zero, nzero);
+    return launch(stream_partials_tma_kernel<T>, grid, kThreads, smem, st, set, V, chunks, temperature, top_p,
+                  skip_uncut, nreq, parts, zero, nzero);
   }
-  return launch(stream_partials_kernel<T>, persistent_grid(stream_partials_kernel<T>, chunks), kThreads, 0, st, base,
-                rows_per_req, row_req, V, chunks, temperature, top_p, skip_uncut, parts, zero, nzero);
+  return launch(stream_partials_kernel<T>, persistent_grid(stream_partials_kernel<T>, chunks), kThreads, 0, st, set, V,
+                chunks, temperature, top_p, skip_uncut, parts, zero, nzero);
 }
 
-// Row statistics of a [rows, V] tensor (the tree's statistics pass); with skip_uncut, the rows
-// of requests with T > 0 and no top-p cut are left out.
+// Row statistics of `rows` rows of a row set (the tree's statistics pass); with skip_uncut,
+// the rows of requests with T > 0 and no top-p cut are left out.
 template <typename T>
-psispec_status launch_stats(const T* base, int64_t rows, int rows_per_req, const int32_t* row_req, int V,
-                            const float* temperature, int nreq, const float* top_p, int skip_uncut, StatsWs ws,
-                            cudaStream_t st) {
-  psispec_status s = launch_stream<T>(base, rows, rows_per_req, row_req, V, temperature, nreq, ws.parts, st, top_p,
-                                      skip_uncut);
+psispec_status launch_stats(RowSet<T> set, int64_t rows, int V, const float* temperature, int nreq,
+                            const float* top_p, int skip_uncut, StatsWs ws, cudaStream_t st) {
+  psispec_status s = launch_stream<T>(set, rows, V, temperature, nreq, ws.parts, st, top_p, skip_uncut);
   if (s != PSISPEC_OK) return s;
-  return launch(row_finalize_kernel<T>, static_cast<unsigned>(rows), kThreads, 0, st, base, rows_per_req, row_req, V,
-                temperature, top_p, ws.parts, ws.stats, skip_uncut);
+  return launch(row_finalize_kernel<T>, static_cast<unsigned>(rows), kThreads, 0, st, set, V, temperature, top_p,
+                ws.parts, ws.stats, skip_uncut);
 }
 
 // The draw jobs of a verification call: totals pass (bulk-copy ring when the rows allow it),
@@ -224,7 +216,7 @@ psispec_status sample_draft_impl(const T* draft, int B, int K, int V, const floa
   RowStat* stats = out_stats ? out_stats : w.st.stats;
   // every row through the streaming pass (maximum and normaliser); the row kernel's top-p
   // CTAs then find the thresholds
-  psispec_status s = launch_stream<T>(draft, rows, K, nullptr, V, temperature, B, w.st.parts, st);
+  psispec_status s = launch_stream<T>(one_tensor(draft, rows, K, B), rows, V, temperature, B, w.st.parts, st);
   if (s != PSISPEC_OK) return s;
   unsigned tgrid = 1;
   if ((s = prepare_topp(sample_rows_kernel<T>, rows, &tgrid)) != PSISPEC_OK) return s;
@@ -264,10 +256,11 @@ psispec_status verify_linear_impl(const T* tgt, const T* drf, int B, int K, int 
   a.jobs = w.jobs;
   // the first streaming pass also clears the request arrival counters
   psispec_status s =
-      launch_stream<T>(tgt, rows_t, K + 1, nullptr, V, temperature, B, w.t.parts, st, nullptr, 0, w.cnt, B);
+      launch_stream<T>(one_tensor(tgt, rows_t, K + 1, B), rows_t, V, temperature, B, w.t.parts, st, nullptr, 0, w.cnt,
+                       B);
   if (s != PSISPEC_OK) return s;
   if (rows_d > 0 &&
-      (s = launch_stream<T>(drf, rows_d, K, nullptr, V, temperature, B, w.d.parts, st)) != PSISPEC_OK)
+      (s = launch_stream<T>(one_tensor(drf, rows_d, K, B), rows_d, V, temperature, B, w.d.parts, st)) != PSISPEC_OK)
     return s;
   // one row kernel: warps for the requests without a top-p cut, whole CTAs for the others
   unsigned tgrid = 1;
@@ -342,24 +335,23 @@ psispec_status verify_tree_impl(const T* tgt, const T* drf, int B, int N, int V,
   else if (s != PSISPEC_OK) return s;
   // the cluster walk finds the statistics of uncut requests' visited rows itself
   const int lazy = CL != 0;
-  s = launch(node_request_kernel, static_cast<unsigned>(B), 128, 0, st, offs, B, N, w.row_req);
+  // one statistics pass over the rows of both tensors
+  s = launch_stats<T>(RowSet<T>{tgt, drf, N, 1, offs, B}, 2 * int64_t(N), V, temperature, B, top_p, lazy, w.st, st);
   if (s != PSISPEC_OK) return s;
-  s = launch_stats<T>(tgt, N, 1, w.row_req, V, temperature, B, top_p, lazy, w.t, st);
-  if (s != PSISPEC_OK) return s;
-  s = launch_stats<T>(drf, N, 1, w.row_req, V, temperature, B, top_p, lazy, w.d, st);
-  if (s != PSISPEC_OK) return s;
+  const RowStat* ts = w.st.stats;
+  const RowStat* ds = w.st.stats + N;
   cudaError_t e = cudaSuccess;
   if (CL == 16)
     e = cudaLaunchKernelEx(&cfg, tree_walk_cluster_kernel<T, 16>, tgt, drf, V, offs, parent, tokens,
-                           static_cast<const RowStat*>(w.t.stats), static_cast<const RowStat*>(w.d.stats), u_acc,
+                           ts, ds, u_acc,
                            u_res, temperature, top_p, lazy, dbuf, max_depth, out_path, out_tokens, out_len);
   else if (CL == 8)
     e = cudaLaunchKernelEx(&cfg, tree_walk_cluster_kernel<T, 8>, tgt, drf, V, offs, parent, tokens,
-                           static_cast<const RowStat*>(w.t.stats), static_cast<const RowStat*>(w.d.stats), u_acc,
+                           ts, ds, u_acc,
                            u_res, temperature, top_p, lazy, dbuf, max_depth, out_path, out_tokens, out_len);
   else
     return launch(tree_walk_kernel<T>, static_cast<unsigned>(B), kTreeThreads, 0, st, tgt, drf, V, offs, parent,
-                  tokens, w.t.stats, w.d.stats, u_acc, u_res, max_depth, out_path, out_tokens, out_len);
+                  tokens, ts, ds, u_acc, u_res, max_depth, out_path, out_tokens, out_len);
   return e == cudaSuccess ? PSISPEC_OK : PSISPEC_ERR_CUDA;
 }
 

@@ -41,10 +41,33 @@ __device__ __forceinline__ float stream_scale(const float* __restrict__ temperat
   return skip_uncut && c != 0.0f && !(top_p[req] < 1.0f) ? -1.0f : c;
 }
 
-// Request of a row: rows_per_req consecutive rows per request, or an explicit table.
-__device__ __forceinline__ int row_request(int row, int rows_per_req, const int32_t* __restrict__ row_req) {
-  return row_req ? row_req[row] : row / rows_per_req;
-}
+// The rows a statistics pass reads: rows [0, rows_a) of tensor a, then the rows of tensor b
+// (same V). The request of row k of either tensor is k / rows_per_req, or, with offs (the
+// node offsets of nreq tries), the j with offs[j] <= k < offs[j + 1] (a binary search that
+// stays in [0, nreq) whatever offs holds).
+template <typename T>
+struct RowSet {
+  const T* a;
+  const T* b;
+  int64_t rows_a;
+  int rows_per_req;
+  const int32_t* offs;
+  int nreq;
+  __device__ __forceinline__ const T* row(int64_t r, int V) const {
+    return r < rows_a ? a + static_cast<size_t>(r) * V : b + static_cast<size_t>(r - rows_a) * V;
+  }
+  __device__ __forceinline__ int request(int64_t r) const {
+    const int64_t k = r < rows_a ? r : r - rows_a;
+    if (offs == nullptr) return static_cast<int>(k / rows_per_req);
+    int lo = 0, hi = nreq;
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (__ldg(offs + mid) <= k) lo = mid;
+      else hi = mid;
+    }
+    return lo;
+  }
+};
 
 // Running statistics of one lane over a chunk: maximum m and the fp32 sum s of
 // 2^((x - m) c), or (greedy rows) the maximum and its lowest index. A NaN or +inf logit
@@ -165,8 +188,7 @@ __device__ __forceinline__ Partial warp_chunk_partial(const T* __restrict__ row,
 // stream_scale marks. CTA 0
 // also clears the nzero arrival counters at `zero` that the call's later kernels use.
 template <typename T>
-__global__ void __launch_bounds__(kThreads, 4) stream_partials_kernel(const T* __restrict__ base, int rows_per_req,
-                                                                    const int32_t* __restrict__ row_req, int V,
+__global__ void __launch_bounds__(kThreads, 4) stream_partials_kernel(RowSet<T> rows, int V,
                                                                     int64_t total_chunks,
                                                                     const float* __restrict__ temperature,
                                                                     const float* __restrict__ top_p, int skip_uncut,
@@ -183,9 +205,9 @@ __global__ void __launch_bounds__(kThreads, 4) stream_partials_kernel(const T* _
   const int drow = static_cast<int>(nwarps / nch), dchunk = static_cast<int>(nwarps - static_cast<int64_t>(drow) * nch);
 #pragma unroll 1
   for (; g < total_chunks; g += nwarps) {
-    const float c = stream_scale(temperature, top_p, skip_uncut, row_request(row, rows_per_req, row_req));
+    const float c = stream_scale(temperature, top_p, skip_uncut, rows.request(row));
     if (c >= 0.0f) {
-      const T* rp = base + static_cast<size_t>(row) * V;
+      const T* rp = rows.row(row, V);
       const int c0 = chunk * kChunkElems, c1 = min(V, c0 + kChunkElems);
       const Partial p =
           c == 0.0f ? warp_chunk_partial<T, true>(rp, c0, c1, c) : warp_chunk_partial<T, false>(rp, c0, c1, c);
@@ -352,8 +374,7 @@ __device__ __forceinline__ Partial warp_chunk_partial_smem(const T* __restrict__
 constexpr int kScaleTable = 1024;
 
 template <typename T>
-__global__ void __launch_bounds__(kThreads) stream_partials_tma_kernel(const T* __restrict__ base, int rows_per_req,
-                                                                        const int32_t* __restrict__ row_req, int V,
+__global__ void __launch_bounds__(kThreads) stream_partials_tma_kernel(RowSet<T> rows, int V,
                                                                         int64_t total_chunks,
                                                                         const float* __restrict__ temperature,
                                                                         const float* __restrict__ top_p, int skip_uncut,
@@ -366,9 +387,13 @@ __global__ void __launch_bounds__(kThreads) stream_partials_tma_kernel(const T* 
   __shared__ uint64_t bars[kThreads / 32][kRing];
   __shared__ float scale[kScaleTable];
   const bool table = nreq <= kScaleTable;
+  bool some = !table;  // whether any request's rows are read
   if (table)
-    for (int i = threadIdx.x; i < nreq; i += kThreads) scale[i] = stream_scale(temperature, top_p, skip_uncut, i);
-  __syncthreads();
+    for (int i = threadIdx.x; i < nreq; i += kThreads) {
+      scale[i] = stream_scale(temperature, top_p, skip_uncut, i);
+      some |= scale[i] >= 0.0f;
+    }
+  if (!__syncthreads_or(some)) return;  // every row left alone
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   unsigned char* ring = ring_smem + warp * kRing * kStageBytes<T>;
   uint64_t* bar = bars[warp];
@@ -395,7 +420,7 @@ __global__ void __launch_bounds__(kThreads) stream_partials_tma_kernel(const T* 
   int irow = row, ichunk = chunk;  // cursor of the next copy to issue
   int64_t gi = g0;
   auto scale_of = [&](int r) {
-    const int req = row_request(r, rows_per_req, row_req);
+    const int req = rows.request(r);
     return table ? scale[req] : stream_scale(temperature, top_p, skip_uncut, req);
   };
   auto issue = [&](int i) {  // copy of this warp's i-th chunk into stage i % kRing (lane 0)
@@ -404,7 +429,7 @@ __global__ void __launch_bounds__(kThreads) stream_partials_tma_kernel(const T* 
       const uint32_t bytes = static_cast<uint32_t>(n) * sizeof(T);
       uint64_t* b = &bar[i % kRing];
       mbar_expect_tx(b, bytes);
-      bulk_g2s(ring + (i % kRing) * kStageBytes<T>, base + static_cast<size_t>(irow) * V + c0, bytes, b);
+      bulk_g2s(ring + (i % kRing) * kStageBytes<T>, rows.row(irow, V) + c0, bytes, b);
     }
     gi += nwarps;
     advance(irow, ichunk);
@@ -867,15 +892,14 @@ __device__ void block_topp_select(const T* __restrict__ rp, int V, float tp, Row
 // One CTA per row (the tree's statistics pass); rows that stream_scale marks are skipped here
 // too.
 template <typename T>
-__global__ void __launch_bounds__(kThreads) row_finalize_kernel(const T* __restrict__ base, int rows_per_req,
-                                                                 const int32_t* __restrict__ row_req, int V,
+__global__ void __launch_bounds__(kThreads) row_finalize_kernel(RowSet<T> rows, int V,
                                                                  const float* __restrict__ temperature,
                                                                  const float* __restrict__ top_p,
                                                                  const Partial* __restrict__ parts,
                                                                  RowStat* __restrict__ stats, int skip_uncut) {
   __shared__ ToppSmem sm;
   __shared__ RowStat sh_st;
-  const int row = blockIdx.x, req = row_request(row, rows_per_req, row_req);
+  const int row = blockIdx.x, req = rows.request(row);
   const int nch = nchunks_for(V);
   if (stream_scale(temperature, top_p, skip_uncut, req) < 0.0f) return;
   if (threadIdx.x < 32) {
@@ -885,7 +909,7 @@ __global__ void __launch_bounds__(kThreads) row_finalize_kernel(const T* __restr
   __syncthreads();
   RowStat st = sh_st;
   const float tp = top_p[req];
-  if (needs_topp(st, tp)) block_topp_select<T>(base + static_cast<size_t>(row) * V, V, tp, st, sm);
+  if (needs_topp(st, tp)) block_topp_select<T>(rows.row(row, V), V, tp, st, sm);
   if (threadIdx.x == 0) stats[row] = st;
 }
 
