@@ -6,6 +6,7 @@
 #include <atomic>
 
 #include "common.cuh"
+#include "draw.cuh"
 #include "finish.cuh"
 #include "linear.cuh"
 #include "sample.cuh"
@@ -170,11 +171,64 @@ psispec_status launch_stats(RowSet<T> set, int64_t rows, int V, const float* tem
                 ws.parts, ws.stats, skip_uncut);
 }
 
-// The draw jobs of a verification call: totals pass (bulk-copy ring when the rows allow it),
-// then the pick pass.
+// Launch configuration of `nclusters` clusters of CL CTAs of `threads` threads; returns
+// PSISPEC_ERR_UNSUPPORTED when the device cannot schedule such a cluster. cfg.attrs points at
+// attr.
+template <typename Kern>
+psispec_status cluster_config(Kern kernel, int64_t nclusters, int CL, int threads, int smem, cudaStream_t st,
+                              cudaLaunchConfig_t& cfg, cudaLaunchAttribute (&attr)[1]) {
+  if (CL > 8 && cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
+    cudaGetLastError();
+    return PSISPEC_ERR_UNSUPPORTED;
+  }
+  cfg = cudaLaunchConfig_t{};
+  cfg.gridDim = dim3(static_cast<unsigned>(nclusters * CL));
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = CL;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int clusters = 0;
+  if (cudaOccupancyMaxActiveClusters(&clusters, kernel, &cfg) != cudaSuccess || clusters < 1) {
+    cudaGetLastError();
+    return PSISPEC_ERR_UNSUPPORTED;
+  }
+  return PSISPEC_OK;
+}
+
+// The draw jobs of a verification call: one cluster per job (16 CTAs where the device can
+// schedule such clusters, else 8), else a totals pass (bulk-copy ring when the rows allow it)
+// and a pick pass.
 template <typename T>
 psispec_status launch_draws(const T* A, const T* Bt, int V, int njobs, const Partial* parts_a, const Job* jobs,
                             double2* tc, double2* tg, int32_t* out_tokens, cudaStream_t st) {
+  {
+    // clusters of 8 CTAs where each warp's part fits the step buffer, else of 16
+    cudaLaunchConfig_t cfg;
+    cudaLaunchAttribute attr[1];
+    psispec_status s = PSISPEC_ERR_UNSUPPORTED;
+    if (draw_part(V, 8) <= kDrawMaxSteps * 256) {
+      s = cluster_config(draw_cluster_kernel<T, 8>, njobs, 8, kDrawClusterWarps * 32, 0, st, cfg, attr);
+      if (s == PSISPEC_OK)
+        return cudaLaunchKernelEx(&cfg, draw_cluster_kernel<T, 8>, A, Bt, V, parts_a, jobs, out_tokens) == cudaSuccess
+                   ? PSISPEC_OK
+                   : PSISPEC_ERR_CUDA;
+      if (s != PSISPEC_ERR_UNSUPPORTED) return s;
+    }
+    if (draw_part(V, 16) <= kDrawMaxSteps * 256) {
+      s = cluster_config(draw_cluster_kernel<T, 16>, njobs, 16, kDrawClusterWarps * 32, 0, st, cfg, attr);
+      if (s == PSISPEC_OK)
+        return cudaLaunchKernelEx(&cfg, draw_cluster_kernel<T, 16>, A, Bt, V, parts_a, jobs, out_tokens) ==
+                       cudaSuccess
+                   ? PSISPEC_OK
+                   : PSISPEC_ERR_CUDA;
+      if (s != PSISPEC_ERR_UNSUPPORTED) return s;
+    }
+  }
   const int64_t items = int64_t(njobs) * nchunks_for(V);
   // the bulk-copy ring serves bf16 rows (fp32 stages would not fit enough warps per SM)
   const bool ring = sizeof(T) == 2 && (reinterpret_cast<uintptr_t>(A) & 15u) == 0 &&
@@ -291,27 +345,7 @@ psispec_status tree_cluster_config(int B, int V, cudaStream_t st, cudaLaunchConf
   const int smem = static_cast<int>((*dbuf ? 3 : 2) * slice_bytes);
   if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return PSISPEC_ERR_CUDA;
-  if (CL > 8 && cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
-    cudaGetLastError();
-    return PSISPEC_ERR_UNSUPPORTED;
-  }
-  cfg = cudaLaunchConfig_t{};
-  cfg.gridDim = dim3(static_cast<unsigned>(B) * CL);
-  cfg.blockDim = dim3(kTreeWalkThreads);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = CL;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  int clusters = 0;
-  if (cudaOccupancyMaxActiveClusters(&clusters, kernel, &cfg) != cudaSuccess || clusters < 1) {
-    cudaGetLastError();
-    return PSISPEC_ERR_UNSUPPORTED;
-  }
-  return PSISPEC_OK;
+  return cluster_config(kernel, B, CL, kTreeWalkThreads, smem, st, cfg, attr);
 }
 
 template <typename T>
