@@ -32,7 +32,6 @@ UNIT = "positions/s"
 # kernel launches per step of the default workload (see csrc/psispec.cu): sample_draft =
 # streaming pass + row finisher; verify_linear = streaming pass + row finisher + draw totals +
 # draw pick
-LAUNCHES_PER_STEP = 2 + 4
 
 
 def _peaks():
@@ -238,6 +237,8 @@ def _prepare_linear(case, dev):
     o_q = torch.empty((B, K), dtype=torch.float32, device=dev)
     ws_s = torch.empty(psispec.workspace_size(psispec.OP_SAMPLE_DRAFT, B, K, V), dtype=torch.uint8, device=dev)
     ws_v = torch.empty(psispec.workspace_size(psispec.OP_VERIFY_LINEAR, B, K, V), dtype=torch.uint8, device=dev)
+    ws_r = torch.empty(psispec.workspace_size(psispec.OP_ROW_STATS, B, K + 1, V), dtype=torch.uint8, device=dev)
+    rec = torch.empty((B, K + 1, psispec.ROW_STATS_BYTES), dtype=torch.uint8, device=dev)
     esz = tgt.element_size()
 
     def sample(t_in=tgt, d_in=drf):
@@ -247,6 +248,9 @@ def _prepare_linear(case, dev):
         psispec.verify_linear(t_in, d_in, x, ua, ur, Ts, Ps, draft_row_stats=stats, out_tokens=o_tok,
                               out_accept_len=o_len, out_p=o_p, out_q=o_q, ws=ws_v)
 
+    def stream_leg():  # the streaming pass over the verifier tensor alone (plus its row finalize)
+        psispec.row_stats(tgt, Ts, Ps, out=rec, ws=ws_r)
+
     return {
         "inputs": (tgt, drf), "calls": [("sample_draft", sample), ("verify_linear", verify)],
         "outputs": (o_tok, o_len), "positions": B * K, "esz": esz,
@@ -254,6 +258,10 @@ def _prepare_linear(case, dev):
         # verifier tensor once plus, per request, the one draft row of the residual draw
         "bytes": {"sample_draft": B * K * V * esz, "verify_linear": B * (K + 1) * V * esz + B * V * esz},
         "bytes_step": (B * (K + 1) + B * K) * V * esz,
+        # stream + sample rows; stream + verify rows + cluster draw
+        "launches": 2 + 3,
+        "kernel_leg": ("stream_partials_tma_kernel (psispec_row_stats over the verifier tensor)", stream_leg,
+                       B * (K + 1) * V * esz),
         "describe": "linear verify B=%d K=%d V=%d %s, T=%g, top-p %g" % (
             B, K, V, "bf16" if esz == 2 else "fp32", case.temperature, case.top_p),
         "config": {"global_batch": B, "block": K, "vocab": V},
@@ -282,9 +290,16 @@ def _prepare_tree(case, dev):
         psispec.verify_tree(t_in, d_in, offs, parent, tok, ua, ur, Ts, Ps, D, out_path=o_path, out_tokens=o_tok,
                             out_accept_len=o_len, ws=ws)
 
+    def visited_bytes():
+        # the method reads the verifier and draft rows of the nodes the walk visits (the
+        # accepted path and the node where it stops): len + 1 nodes per trie
+        n = int((o_len.clamp(min=-1) + 1).sum())
+        return 2 * n * V * esz
+
     return {
         "inputs": (tgt, drf), "calls": [("verify_tree", verify)], "outputs": (o_tok, o_len), "positions": N,
         "esz": esz, "bytes": {"verify_tree": 2 * N * V * esz}, "bytes_step": 2 * N * V * esz,
+        "bytes_from_outputs": visited_bytes, "launches": 3,
         "describe": "tree verify B=%d tries x %d nodes (depth <= %d, branching <= %d) V=%d %s, T=%g, top-p %g" % (
             B, case.nodes, case.max_depth, case.max_branch, V, "bf16" if esz == 2 else "fp32", case.temperature,
             case.top_p),
@@ -332,6 +347,29 @@ def _graphs(calls, dev, warmup):
     return out
 
 
+def _set_bytes(P):
+    """Workloads whose algorithmic bytes depend on the result (the tree) set them from the
+    outputs of the warm-up steps."""
+    if "bytes_from_outputs" in P:
+        b = P["bytes_from_outputs"]()
+        P["bytes"] = {k: b for k in P["bytes"]}
+        P["bytes_step"] = b
+
+
+def _time_leg(fn, dev, steps, warmup):
+    """Mean device time (ms) of one launch sequence, captured in a CUDA graph."""
+    ((_, replay, g),) = _graphs([("leg", fn)], dev, warmup)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(steps):
+        replay()
+    e1.record()
+    torch.cuda.synchronize()
+    del g
+    return e0.elapsed_time(e1) / steps
+
+
 def _time_steps(calls, steps, dist=None):
     """Device time of `steps` steps (CUDA events on the launching stream): (ms per step,
     {call: mean ms})."""
@@ -364,6 +402,7 @@ def _all_workloads(args, dev):
     for name in names:
         P, case = _prepare(name, dev)
         calls = _graphs(P["calls"], dev, 3) if not args.no_graph else P["calls"]
+        _set_bytes(P)
         steps = max(5, min(args.steps, int(2e5 / max(1.0, P["bytes_step"] / 1e6))))
         ms, per = _time_steps(calls, steps)
         line = {"workload": name, "describe": P["describe"], "value": P["positions"] / (ms * 1e-3), "unit": UNIT,
@@ -391,9 +430,14 @@ def run_ours(args):
         for _ in range(args.warmup):
             for _, f in calls:
                 f()
+    _set_bytes(P)
     _barrier(dist)
     with ClockSampler(dev) as clk:
         ms_step, per = _time_steps(calls, args.steps, dist)
+        # the dominant kernel alone, for the roofline (same inputs, launched right after)
+        leg_ms = None
+        if "kernel_leg" in P:
+            leg_ms = _max_over_ranks(dist, _time_leg(P["kernel_leg"][1], dev, max(args.steps, 10), args.warmup))
     mean_accept = P["accept"]()
 
     # end to end through the public API with host buffers: pinned H2D of the step's inputs,
@@ -428,7 +472,12 @@ def run_ours(args):
 
     peak, peak_kind = _peaks()
     main_call = P["calls"][-1][0]
-    gbs_main = P["bytes"][main_call] / (per[main_call] * 1e-3) / 1e9
+    if leg_ms is not None:
+        kname, kbytes = P["kernel_leg"][0], P["kernel_leg"][2]
+        gbs_main = kbytes / (leg_ms * 1e-3) / 1e9
+    else:  # the call itself (the tree: the walk dominates; bytes of the visited rows)
+        kname, kbytes = "psispec_" + main_call, P["bytes"][main_call]
+        gbs_main = kbytes / (per[main_call] * 1e-3) / 1e9
     value = world * P["positions"] / (ms_step * 1e-3)
     esz = P["esz"]
     if rank == 0:
@@ -439,16 +488,17 @@ def run_ours(args):
             "config": dict({"workload": "%s: %s" % (args.workload, P["describe"]), "parallelism": "replicas x%d" % world,
                             "l2": "inputs %.0f MB > 126 MB L2, no flush" % (P["bytes_step"] / 1e6),
                             "cuda_graph": not args.no_graph}, **P["config"]),
-            "roofline": {"bound": "hbm", "kernel": "psispec_" + main_call, "achieved": gbs_main, "peak": peak,
+            "roofline": {"bound": "hbm", "kernel": kname, "achieved": gbs_main, "peak": peak,
                          "unit": "GB/s", "frac": gbs_main / peak, "peak_kind": peak_kind,
-                         "traffic": _traffic(args.workload)},
+                         "traffic": _traffic(args.workload), "bytes_per_launch": kbytes,
+                         "ms_per_launch": leg_ms if leg_ms is not None else per[main_call]},
             "step_gbs": P["bytes_step"] / (ms_step * 1e-3) / 1e9,
             "calls": dict({k + "_ms": v for k, v in per.items()},
                           **{k + "_gbs": P["bytes"][k] / (v * 1e-3) / 1e9 for k, v in per.items()}),
             "mean_accept_len": mean_accept,
             "e2e": {"value": world * P["positions"] / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
-            "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+            "gpu_launches": P["launches"] * args.steps,
             "clocks": clk.summary(),
             "cpu_baseline": cpu,
         }

@@ -67,7 +67,8 @@ typedef enum { PSISPEC_F32 = 0, PSISPEC_BF16 = 1 } psispec_dtype;
 typedef enum {
   PSISPEC_OP_SAMPLE_DRAFT = 0,
   PSISPEC_OP_VERIFY_LINEAR = 1,
-  PSISPEC_OP_VERIFY_TREE = 2
+  PSISPEC_OP_VERIFY_TREE = 2,
+  PSISPEC_OP_ROW_STATS = 3
 } psispec_op;
 
 /* Bytes of one per-row statistics record written by psispec_sample_draft (out_row_stats). */
@@ -83,6 +84,7 @@ int psispec_version(void);
  *   SAMPLE_DRAFT:  a = B, b = K (rows = B*K), c = V
  *   VERIFY_LINEAR: a = B, b = K, c = V
  *   VERIFY_TREE:   a = B, b = N (total nodes), c = V
+ *   ROW_STATS:     a = B, b = K (rows = B*K), c = V
  * Returns 0 for invalid sizes. */
 size_t psispec_workspace_size(int op, int64_t a, int64_t b, int64_t c);
 
@@ -107,6 +109,25 @@ psispec_status psispec_sample_draft(const void* draft_logits, int dtype, int32_t
                                     const float* temperature, const float* top_p, const float* u,
                                     int32_t* out_tokens, float* out_q, void* out_row_stats,
                                     void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * psispec_row_stats -- the per-row statistics of the sampling distribution softmax(l / T)
+ * after top-p over the full vocabulary (review page, section 3.3: both distributions of the
+ * rule are taken after the sampling controls): row maximum, normaliser, top-p threshold and
+ * kept mass, or the argmax of a greedy row. These are the records psispec_sample_draft
+ * writes, without the draw; psispec_verify_linear accepts them as draft_row_stats.
+ *
+ *   logits        [B, K, V] dtype   row i of request b at element (b*K + i) * V
+ *   temperature   [B] float, top_p [B] float
+ *   out_row_stats [B, K] records of PSISPEC_ROW_STATS_BYTES (16-byte aligned); a row with a
+ *                 data error (NaN/+inf logit, no finite logit, bad temperature) gets a
+ *                 record whose status field is nonzero
+ * Workspace: psispec_workspace_size(PSISPEC_OP_ROW_STATS, B, K, V) bytes.
+ * Limits: B, K >= 1, B*K <= 2^26, V <= 2^24.
+ */
+psispec_status psispec_row_stats(const void* logits, int dtype, int32_t B, int32_t K, int32_t V,
+                                 const float* temperature, const float* top_p, void* out_row_stats,
+                                 void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * psispec_verify_linear -- Psi-Spec linear verification (review page, section 3.3; linear

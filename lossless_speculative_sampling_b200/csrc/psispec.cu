@@ -72,6 +72,9 @@ LinearWs carve_linear(Carver& c, int64_t B, int64_t K, int64_t V) {
   return w;
 }
 
+// psispec_row_stats: the chunk partials (the records go to the caller's array).
+Partial* carve_row_stats(Carver& c, int64_t rows, int64_t V) { return c.take<Partial>(rows * nchunks_for(V)); }
+
 struct TreeWs {
   StatsWs st;  // rows [0, N) of the verifier tensor, then [N, 2N) of the draft tensor
 };
@@ -167,8 +170,8 @@ psispec_status launch_stats(RowSet<T> set, int64_t rows, int V, const float* tem
                             const float* top_p, int skip_uncut, StatsWs ws, cudaStream_t st) {
   psispec_status s = launch_stream<T>(set, rows, V, temperature, nreq, ws.parts, st, top_p, skip_uncut);
   if (s != PSISPEC_OK) return s;
-  return launch(row_finalize_kernel<T>, static_cast<unsigned>(rows), kThreads, 0, st, set, V, temperature, top_p,
-                ws.parts, ws.stats, skip_uncut);
+  return launch(row_finalize_kernel<T>, static_cast<unsigned>((rows + kThreads / 32 - 1) / (kThreads / 32)), kThreads,
+                0, st, set, rows, V, temperature, top_p, ws.parts, ws.stats, skip_uncut);
 }
 
 // Launch configuration of `nclusters` clusters of CL CTAs of `threads` threads; returns
@@ -389,6 +392,15 @@ psispec_status verify_tree_impl(const T* tgt, const T* drf, int B, int N, int V,
   return e == cudaSuccess ? PSISPEC_OK : PSISPEC_ERR_CUDA;
 }
 
+template <typename T>
+psispec_status row_stats_impl(const T* logits, int B, int K, int V, const float* temperature, const float* top_p,
+                              RowStat* out, void* ws, cudaStream_t st) {
+  const int64_t rows = int64_t(B) * K;
+  Carver c(ws);
+  Partial* parts = carve_row_stats(c, rows, V);
+  return launch_stats<T>(one_tensor(logits, rows, K, B), rows, V, temperature, B, top_p, 0, StatsWs{parts, out}, st);
+}
+
 bool bad_dtype(int dtype) { return dtype != PSISPEC_F32 && dtype != PSISPEC_BF16; }
 size_t esize(int dtype) { return dtype == PSISPEC_BF16 ? 2 : 4; }
 
@@ -429,6 +441,7 @@ size_t psispec_workspace_size(int op, int64_t a, int64_t b, int64_t c) {
     case PSISPEC_OP_SAMPLE_DRAFT: carve_sample(m, a * b, c); break;
     case PSISPEC_OP_VERIFY_LINEAR: carve_linear(m, a, b, c); break;
     case PSISPEC_OP_VERIFY_TREE: carve_tree(m, b, c); break;
+    case PSISPEC_OP_ROW_STATS: carve_row_stats(m, a * b, c); break;
     default: return 0;
   }
   return m.used;
@@ -508,6 +521,23 @@ psispec_status psispec_verify_tree(const void* target_logits, const void* draft_
   return verify_tree_impl(static_cast<const float*>(target_logits), static_cast<const float*>(draft_logits), B, N, V,
                           node_offsets, parent, tokens, u_accept, u_resid, temperature, top_p, max_depth, out_path,
                           out_tokens, out_accept_len, workspace, st);
+}
+
+psispec_status psispec_row_stats(const void* logits, int dtype, int32_t B, int32_t K, int32_t V,
+                                 const float* temperature, const float* top_p, void* out_row_stats,
+                                 void* workspace, size_t workspace_bytes, void* stream) {
+  if (!logits || !temperature || !top_p || !out_row_stats || bad_dtype(dtype)) return PSISPEC_ERR_INVALID_ARG;
+  if (B <= 0 || K <= 0 || V <= 0) return PSISPEC_ERR_INVALID_ARG;
+  if (!aligned_to(logits, esize(dtype)) || !aligned_to(out_row_stats, 16)) return PSISPEC_ERR_INVALID_ARG;
+  const int64_t rows = int64_t(B) * K;
+  if (rows > kMaxRows || V > kMaxV || rows * nslices_for(V) > kMaxGrid) return PSISPEC_ERR_UNSUPPORTED;
+  psispec_status s = check_ws(workspace, workspace_bytes, psispec_workspace_size(PSISPEC_OP_ROW_STATS, B, K, V));
+  if (s != PSISPEC_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  RowStat* rs = static_cast<RowStat*>(out_row_stats);
+  if (dtype == PSISPEC_BF16)
+    return row_stats_impl(static_cast<const __nv_bfloat16*>(logits), B, K, V, temperature, top_p, rs, workspace, st);
+  return row_stats_impl(static_cast<const float*>(logits), B, K, V, temperature, top_p, rs, workspace, st);
 }
 
 psispec_status psispec_verify_linear_static(const void* target_logits, const void* draft_logits, int dtype,

@@ -889,28 +889,45 @@ __device__ void block_topp_select(const T* __restrict__ rp, int V, float tp, Row
   __syncthreads();
 }
 
-// One CTA per row (the tree's statistics pass); rows that stream_scale marks are skipped here
-// too.
+// Row statistics from the chunk partials (the tree's statistics pass and psispec_row_stats):
+// kThreads / 32 rows per CTA, one warp finalizing each row; the CTA then runs the top-p
+// select for those of its rows that need one. Rows that stream_scale marks are skipped.
 template <typename T>
-__global__ void __launch_bounds__(kThreads) row_finalize_kernel(RowSet<T> rows, int V,
+__global__ void __launch_bounds__(kThreads) row_finalize_kernel(RowSet<T> rows, int64_t nrows, int V,
                                                                  const float* __restrict__ temperature,
                                                                  const float* __restrict__ top_p,
                                                                  const Partial* __restrict__ parts,
                                                                  RowStat* __restrict__ stats, int skip_uncut) {
+  constexpr int kRows = kThreads / 32;
   __shared__ ToppSmem sm;
-  __shared__ RowStat sh_st;
-  const int row = blockIdx.x, req = rows.request(row);
+  __shared__ RowStat sh_st[kRows];
+  __shared__ int sh_topp[kRows];
+  const int warp = threadIdx.x >> 5;
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * kRows + warp;
   const int nch = nchunks_for(V);
-  if (stream_scale(temperature, top_p, skip_uncut, req) < 0.0f) return;
-  if (threadIdx.x < 32) {
-    const RowStat st = warp_finalize_row(parts + static_cast<size_t>(row) * nch, nch, temperature[req]);
-    if (threadIdx.x == 0) sh_st = st;
+  if (row < nrows) {
+    const int req = rows.request(row);
+    int topp = 0;
+    if (stream_scale(temperature, top_p, skip_uncut, req) >= 0.0f) {
+      const RowStat st = warp_finalize_row(parts + static_cast<size_t>(row) * nch, nch, temperature[req]);
+      topp = needs_topp(st, top_p[req]);
+      if ((threadIdx.x & 31) == 0) {
+        sh_st[warp] = st;
+        if (!topp) stats[row] = st;
+      }
+    }
+    if ((threadIdx.x & 31) == 0) sh_topp[warp] = topp;
+  } else if ((threadIdx.x & 31) == 0) {
+    sh_topp[warp] = 0;
   }
   __syncthreads();
-  RowStat st = sh_st;
-  const float tp = top_p[req];
-  if (needs_topp(st, tp)) block_topp_select<T>(rows.row(row, V), V, tp, st, sm);
-  if (threadIdx.x == 0) stats[row] = st;
+  for (int w = 0; w < kRows; ++w) {
+    if (!sh_topp[w]) continue;  // the same branch in every thread
+    const int64_t r = static_cast<int64_t>(blockIdx.x) * kRows + w;
+    RowStat st = sh_st[w];
+    block_topp_select<T>(rows.row(r, V), V, top_p[rows.request(r)], st, sm);
+    if (threadIdx.x == 0) stats[r] = st;
+  }
 }
 
 }  // namespace psi

@@ -23,7 +23,7 @@ HEADER = os.path.join(os.path.dirname(_HERE), "include", "psispec.h")
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_WORKSPACE = 0, 1, 2, 3, 4
 STATIC_WORKSPACE_BYTES = 16 << 20  # PSISPEC_STATIC_WORKSPACE_BYTES
 F32, BF16 = 0, 1
-OP_SAMPLE_DRAFT, OP_VERIFY_LINEAR, OP_VERIFY_TREE = 0, 1, 2
+OP_SAMPLE_DRAFT, OP_VERIFY_LINEAR, OP_VERIFY_TREE, OP_ROW_STATS = 0, 1, 2, 3
 ROW_STATS_BYTES = 32
 
 _lib = None
@@ -48,11 +48,12 @@ def lib():
         L.psispec_version.argtypes, L.psispec_version.restype = [], ctypes.c_int
         L.psispec_workspace_size.argtypes, L.psispec_workspace_size.restype = [ctypes.c_int, I64, I64, I64], SZ
         L.psispec_sample_draft.argtypes = [P, ctypes.c_int, I32, I32, I32, P, P, P, P, P, P, P, SZ, P]
+        L.psispec_row_stats.argtypes = [P, ctypes.c_int, I32, I32, I32, P, P, P, P, SZ, P]
         L.psispec_verify_linear.argtypes = [P, P, ctypes.c_int, I32, I32, I32, P, P, P, P, P, P, P, P, P, P, P, SZ, P]
         L.psispec_verify_tree.argtypes = [P, P, ctypes.c_int, I32, I32, I32, P, P, P, P, P, P, P, I32, P, P, P, P, SZ,
                                           P]
         L.psispec_verify_linear_static.argtypes = [P, P, ctypes.c_int, I32, I32, I32, P, P, P, P, P, P, P, P, P, P, P]
-        for f in ("psispec_sample_draft", "psispec_verify_linear", "psispec_verify_tree",
+        for f in ("psispec_sample_draft", "psispec_row_stats", "psispec_verify_linear", "psispec_verify_tree",
                   "psispec_verify_linear_static"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
@@ -149,6 +150,26 @@ def sample_draft(draft, temperature, top_p, u, *, out_tokens=None, out_q=None, r
                                     _p(out_tokens), _p(out_q), _p(row_stats), _p(ws), ws.numel(), _stream(dev, stream))
     _check(st, "psispec_sample_draft")
     return out_tokens, out_q, row_stats
+
+
+def row_stats(logits, temperature, top_p, *, out=None, ws=None, stream=None):
+    """Per-row statistics records of softmax(logits / T) after top-p.
+
+    logits [B, K, V] bf16/fp32; temperature, top_p [B] fp32. Returns [B, K, 32] uint8 records,
+    usable as verify_linear(draft_row_stats=...) for the same logits and controls."""
+    B, K, V = logits.shape
+    dev = logits.device
+    _req(logits, "logits")
+    _req(temperature, "temperature", torch.float32, B, dev)
+    _req(top_p, "top_p", torch.float32, B, dev)
+    out = torch.empty((B, K, ROW_STATS_BYTES), dtype=torch.uint8, device=dev) if out is None else out
+    _req(out, "out", torch.uint8, B * K * ROW_STATS_BYTES, dev)
+    need = workspace_size(OP_ROW_STATS, B, K, V)
+    ws = workspace(need, dev) if ws is None else ws
+    st = lib().psispec_row_stats(_p(logits), _dtype(logits), B, K, V, _p(temperature), _p(top_p), _p(out), _p(ws),
+                                 ws.numel(), _stream(dev, stream))
+    _check(st, "psispec_row_stats")
+    return out
 
 
 def verify_linear(target, draft, draft_tokens, u_accept, u_resid, temperature, top_p, *, draft_row_stats=None,

@@ -31,7 +31,8 @@ def test_status_strings_and_version(L):
 
 def test_workspace_size(L):
     V = 151936
-    for op, a, b in ((psispec.OP_SAMPLE_DRAFT, 64, 8), (psispec.OP_VERIFY_LINEAR, 64, 8), (psispec.OP_VERIFY_TREE, 4, 256)):
+    for op, a, b in ((psispec.OP_SAMPLE_DRAFT, 64, 8), (psispec.OP_VERIFY_LINEAR, 64, 8), (psispec.OP_VERIFY_TREE, 4, 256),
+                     (psispec.OP_ROW_STATS, 64, 9)):
         n = psispec.workspace_size(op, a, b, V)
         assert n > 0 and n % 256 == 0
         assert psispec.workspace_size(op, a * 2, b, V) >= n
@@ -62,6 +63,25 @@ def test_sample_draft_host_checks(L):
     assert _sample(L, ws=None) == psispec.ERR_WORKSPACE
     assert _sample(L, ws=ctypes.c_void_p(4096 + 128)) == psispec.ERR_WORKSPACE
     assert _sample(L, wsb=16) == psispec.ERR_WORKSPACE
+
+
+def _row_stats(L, **kw):
+    a = dict(l=FAKE, dtype=psispec.BF16, B=2, K=3, V=100, T=FAKE, P=FAKE, out=FAKE, ws=FAKE, wsb=1 << 30)
+    a.update(kw)
+    return L.psispec_row_stats(a["l"], a["dtype"], a["B"], a["K"], a["V"], a["T"], a["P"], a["out"], a["ws"], a["wsb"],
+                               None)
+
+
+def test_row_stats_host_checks(L):
+    assert _row_stats(L, l=None) == psispec.ERR_INVALID_ARG
+    assert _row_stats(L, P=None) == psispec.ERR_INVALID_ARG
+    assert _row_stats(L, out=None) == psispec.ERR_INVALID_ARG
+    assert _row_stats(L, dtype=5) == psispec.ERR_INVALID_ARG
+    assert _row_stats(L, K=0) == psispec.ERR_INVALID_ARG
+    assert _row_stats(L, out=ctypes.c_void_p(4096 + 8)) == psispec.ERR_INVALID_ARG  # records are 16-byte aligned
+    assert _row_stats(L, V=(1 << 24) + 1) == psispec.ERR_UNSUPPORTED
+    assert _row_stats(L, ws=None) == psispec.ERR_WORKSPACE
+    assert _row_stats(L, wsb=16) == psispec.ERR_WORKSPACE
 
 
 def _linear(L, **kw):

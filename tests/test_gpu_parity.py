@@ -98,6 +98,60 @@ def test_sample_draft_parity(B, K, V, dtype, T, top_p, noise):
     compare_sample(tok, q, ora)
 
 
+def _decode_stats(rec):
+    """Host view of [rows, 32] uint8 row-statistics records: m, c, s, s_kept (fp32), tau (u32),
+    amax, status (int32)."""
+    r = np.ascontiguousarray(rec.reshape(-1, 32).cpu().numpy())
+    f, u, i = r.view(np.float32), r.view(np.uint32), r.view(np.int32)
+    return {"m": f[:, 0], "c": f[:, 1], "s": f[:, 2], "s_kept": f[:, 3], "tau": u[:, 4], "amax": i[:, 5],
+            "status": i[:, 6]}
+
+
+def _fkey(x):
+    """Order-preserving uint32 key of fp32 values (the threshold record's encoding)."""
+    u = np.asarray(x, np.float32).view(np.uint32)
+    return np.where(u & 0x80000000, ~u, u | 0x80000000).astype(np.uint32)
+
+
+@pytest.mark.parametrize("B,K,V,dtype,T,top_p", [(3, 4, 40000, torch.bfloat16, 1.0, 1.0),
+                                                 (3, 4, 40000, torch.bfloat16, 0.7, 0.9),
+                                                 (2, 5, 16384 * 2 + 37, torch.float32, 1.3, 0.5),
+                                                 (4, 3, 3001, torch.float32, 0.0, 1.0)])
+def test_row_stats_parity(B, K, V, dtype, T, top_p):
+    """psispec_row_stats records against the oracle's row distributions: the probability every
+    record implies for every token (kept set from the threshold key) within 1e-5, the greedy
+    argmax exactly, data errors flagged; and the records serve verification."""
+    tgt, drf, ud, ua, ur, Ts, Ps = _linear_inputs(B, K, V, dtype, T, top_p, 0.6, seed=V + 11, neg_inf_frac=0.05)
+    drf[1, 2, 9] = float("nan")  # one row with a data error
+    rec = psispec.row_stats(_cuda(drf), _cuda(Ts), _cuda(Ps))
+    st = _decode_stats(rec)
+    rows = drf.reshape(B * K, V).float().numpy().astype(np.float64)
+    for r in range(B * K):
+        if r == 1 * K + 2:
+            assert st["status"][r] != 0
+            continue
+        assert st["status"][r] == 0
+        probs, band = oracle.row_dist(rows[r], T, top_p)
+        if T == 0.0:
+            assert st["amax"][r] == int(np.argmax(rows[r]))
+            continue
+        if band < 1e-6:
+            continue  # a threshold tie within the band: the kept set is not unique
+        l = rows[r].astype(np.float32)
+        kept = (_fkey(l) >= st["tau"][r]) if st["tau"][r] != 0 else np.ones(V, bool)
+        p = np.where(kept, np.exp2((l.astype(np.float64) - st["m"][r]) * st["c"][r]) / st["s_kept"][r], 0.0)
+        assert np.abs(p - probs).max() <= 1e-5, (r, np.abs(p - probs).max())
+    # the records stand in for the draft statistics of verification
+    o_s = oracle.sample_draft(drf.reshape(B * K, V), Ts.numpy(), Ps.numpy(), ud.reshape(-1),
+                              row_req=np.arange(B * K) // K)
+    x = o_s["tokens"].reshape(B, K).astype(np.int32)
+    x[x < 0] = 0
+    out = psispec.verify_linear(_cuda(tgt), _cuda(drf), _cuda(x), _cuda(ua), _cuda(ur), _cuda(Ts), _cuda(Ps),
+                                draft_row_stats=rec)
+    ora = oracle.verify_linear(tgt, drf, x, ua, ur, Ts.numpy(), Ps.numpy())
+    compare_linear(out, ora)
+
+
 @pytest.mark.parametrize("use_stats", [False, True])
 @pytest.mark.parametrize("B,K,V,dtype,T,top_p,noise", GRID)
 def test_verify_linear_parity(B, K, V, dtype, T, top_p, noise, use_stats):
