@@ -465,13 +465,47 @@ __device__ bool tp_window_select(const T* __restrict__ row, int V, float tp, Row
   __syncthreads();
   const uint32_t km = fkey(st.m) >> 16;
   uint32_t* mine = cnt + warp * kTpWindow;
-  tp_for_each8<T, 4>(row, V, [&](const float (&x)[8]) {
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const uint32_t o = km - (fkey(x[k]) >> 16);
+  if (km >= 0x8000u + kTpWindow) {
+    // the window holds positive values only: a positive bf16 with bits h has the key
+    // h + 0x8000, so its offset is kb - h; negative values (h >= 0x8000) wrap to offsets far
+    // outside the window, so the raw bits are counted without any conversion
+    const uint32_t kb = km - 0x8000u;
+    const uint16_t* r16 = reinterpret_cast<const uint16_t*>(row);
+    auto count = [&](uint32_t h) {
+      const uint32_t o = kb - h;
       if (o < static_cast<uint32_t>(kTpWindow)) atomicAdd(&mine[o], 1u);
+    };
+    int a0, a1;
+    vec_range(row, 0, V, a0, a1);
+    for (int v = threadIdx.x; v < a0; v += kTpThreads) count(r16[v]);
+    for (int v = a1 + threadIdx.x; v < V; v += kTpThreads) count(r16[v]);
+    constexpr int kLoads = 4, kStep = kTpThreads * 8;
+    for (int v = a0 + threadIdx.x * 8; v < a1; v += kLoads * kStep) {
+      uint4 raw[kLoads];
+#pragma unroll
+      for (int i = 0; i < kLoads; ++i)
+        if (v + i * kStep < a1) raw[i] = __ldcg(reinterpret_cast<const uint4*>(row + v + i * kStep));
+#pragma unroll
+      for (int i = 0; i < kLoads; ++i) {
+        if (v + i * kStep < a1) {
+          const uint32_t w[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            count(w[k] & 0xFFFFu);
+            count(w[k] >> 16);
+          }
+        }
+      }
     }
-  });
+  } else {
+    tp_for_each8<T, 4>(row, V, [&](const float (&x)[8]) {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const uint32_t o = km - (fkey(x[k]) >> 16);
+        if (o < static_cast<uint32_t>(kTpWindow)) atomicAdd(&mine[o], 1u);
+      }
+    });
+  }
   __syncthreads();
   // masses of offsets [8t, 8t + 8) in thread t, scanned in thread order
   constexpr int kPer = kTpWindow / kTpThreads;
