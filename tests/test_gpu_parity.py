@@ -184,6 +184,32 @@ def test_verify_linear_mixed_requests_and_data_errors():
     compare_linear(out, ora)
 
 
+@pytest.mark.parametrize("V,T,top_p", [(40000, 100.0, 0.9), (40000, 30.0, 0.5), ((1 << 19) + 1000, 1.0, 0.9)])
+def test_topp_fallback_paths(V, T, top_p):
+    """bf16 top-p rows whose threshold lies below the 2048-value window under the row maximum
+    (a far outlier and a high temperature put most of the mass far below it), and rows longer
+    than the top-p counters' range (2^19): the histogram / digit select and the general radix
+    select and block draw, for sampling and verification."""
+    B, K = 2, 3
+    g = torch.Generator().manual_seed(V + int(T))
+    tgt = torch.randn((B, K + 1, V), generator=g) * 2.0
+    drf = tgt[:, :K] + torch.randn((B, K, V), generator=g) * 0.5
+    if T > 1.0:
+        tgt[..., 7] = 120.0  # an outlier far above the rest: the window covers only [~0.002, 120]
+        drf[..., 7] = 120.0
+    tgt, drf = tgt.to(torch.bfloat16), drf.to(torch.bfloat16)
+    Ts, Ps = torch.full((B,), T), torch.full((B,), top_p)
+    ud, ua, ur = synth.uniforms((B, K), 5), synth.uniforms((B, K), 6), synth.uniforms((B, K + 1), 7)
+    tok, q, _ = psispec.sample_draft(_cuda(drf), _cuda(Ts), _cuda(Ps), _cuda(ud))
+    o_s = oracle.sample_draft(drf.reshape(B * K, V), Ts.numpy(), Ps.numpy(), ud.reshape(-1),
+                              row_req=np.arange(B * K) // K)
+    compare_sample(tok, q, o_s)
+    x = o_s["tokens"].reshape(B, K).astype(np.int32)
+    out = psispec.verify_linear(_cuda(tgt), _cuda(drf), _cuda(x), _cuda(ua), _cuda(ur), _cuda(Ts), _cuda(Ps))
+    ora = oracle.verify_linear(tgt, drf, x, ua, ur, Ts.numpy(), Ps.numpy())
+    compare_linear(out, ora)
+
+
 def test_q_equals_p_accepts_all_on_gpu():
     B, K, V = 16, 8, 30000
     g = torch.Generator().manual_seed(5)
