@@ -9,10 +9,11 @@
 //                       statistics, then an arrival on the request's counter; the warp
 //                       completing a request runs the accept tests, finds the first rejection
 //                       and writes the draw job (both run inside the row kernels of topp.cuh);
-//   draw_totals_*       one warp per (draw job, chunk) item over every SM: group and chunk
-//                       totals of the residual (or kept) weights;
-//   draw_pick_kernel    one warp per draw job: the chunk, then the 256-element group holding
-//                       u * Z, and the walk of that group.
+//   draw_totals_*       (fallback of the cluster draw in draw.cuh) one warp per (draw job,
+//                       chunk) item over every SM: group and chunk totals of the residual (or
+//                       kept) weights;
+//   draw_pick_kernel    (same fallback) one warp per draw job: the chunk, then the 256-element
+//                       group holding u * Z, and the walk of that group.
 // Cross-CTA handoffs use arrival counters (the last arrival continues); nothing waits.
 #pragma once
 
@@ -329,13 +330,15 @@ __device__ void warp_verify_row(const T* __restrict__ tgt, const T* __restrict__
                            a.u_acc, a.u_res, a.out_tokens, a.out_len, a.out_p, a.out_q, a.jobs);
 }
 
-// Draw jobs (the residual draw at a first rejection, or the bonus draw after a fully
-// accepted block) take two launches. The totals pass spreads (job, chunk) items over every
-// SM: each warp reduces one chunk of the job's weights (.x the residual max(0, p - q) or the
-// kept distribution, .y p) to its eight 256-element group totals and the chunk total. The
-// pick pass gives each job a warp that locates the chunk holding u * Z, then the group
-// inside it, and walks that group. A bonus draw without a top-p cut needs no totals: its
-// chunk comes from the row's own partials and is walked whole.
+// Two-launch draw of the jobs (the residual draw at a first rejection, or the bonus draw after
+// a fully accepted block), used where the one-launch cluster draw (draw.cuh) cannot run: no
+// cluster of the needed size can be scheduled, or V is beyond its per-warp step buffer. The
+// totals pass spreads (job, chunk) items over every SM: each warp reduces one chunk of the
+// job's weights (.x the residual max(0, p - q) or the kept distribution, .y p) to its eight
+// 256-element group totals and the chunk total. The pick pass gives each job a warp that
+// locates the chunk holding u * Z, then the group inside it, and walks that group. A bonus
+// draw without a top-p cut needs no totals: its chunk comes from the row's own partials and
+// is walked whole.
 
 // Whether a job's draw needs the totals pass.
 __device__ __forceinline__ bool job_needs_totals(int32_t mode, uint32_t tau_a) {
