@@ -29,6 +29,19 @@
 
 namespace psi {
 
+// One to the shared-memory counter p[o] when o < n, as a predicated reduction (no branch;
+// p + o is not formed into an access otherwise).
+__device__ __forceinline__ void count_if_below(uint32_t* p, uint32_t o, uint32_t n) {
+  asm volatile(
+      "{\n"
+      " .reg .pred q;\n"
+      " setp.lt.u32 q, %1, %2;\n"
+      " @q red.shared.add.u32 [%0], 1;\n"
+      "}" ::"r"(smem_u32(p) + 4u * o),
+      "r"(o), "r"(n)
+      : "memory");
+}
+
 constexpr int kTpThreads = 256;
 constexpr int kTpWarps = kTpThreads / 32;
 constexpr int kTpBins = 64;                                  // half log2 units below the maximum
@@ -471,10 +484,7 @@ __device__ bool tp_window_select(const T* __restrict__ row, int V, float tp, Row
     // outside the window, so the raw bits are counted without any conversion
     const uint32_t kb = km - 0x8000u;
     const uint16_t* r16 = reinterpret_cast<const uint16_t*>(row);
-    auto count = [&](uint32_t h) {
-      const uint32_t o = kb - h;
-      if (o < static_cast<uint32_t>(kTpWindow)) atomicAdd(&mine[o], 1u);
-    };
+    auto count = [&](uint32_t h) { count_if_below(mine, kb - h, kTpWindow); };
     int a0, a1;
     vec_range(row, 0, V, a0, a1);
     for (int v = threadIdx.x; v < a0; v += kTpThreads) count(r16[v]);
@@ -500,10 +510,7 @@ __device__ bool tp_window_select(const T* __restrict__ row, int V, float tp, Row
   } else {
     tp_for_each8<T, 4>(row, V, [&](const float (&x)[8]) {
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const uint32_t o = km - (fkey(x[k]) >> 16);
-        if (o < static_cast<uint32_t>(kTpWindow)) atomicAdd(&mine[o], 1u);
-      }
+      for (int k = 0; k < 8; ++k) count_if_below(mine, km - (fkey(x[k]) >> 16), kTpWindow);
     });
   }
   __syncthreads();
