@@ -14,6 +14,7 @@ collective touches the data path (only the max-over-ranks timing reduction).
 """
 import argparse
 import hashlib
+import re
 import json
 import os
 import statistics
@@ -44,11 +45,16 @@ def _peaks():
 
 
 def _kernel_source_hash():
+    """Hash of the kernel sources with their comments removed (a comment edit leaves the
+    captured traffic valid; any code change invalidates it)."""
     h = hashlib.sha256()
     d = os.path.join(ROOT, "lossless_speculative_sampling_b200", "csrc")
     for f in sorted(os.listdir(d)):
-        with open(os.path.join(d, f), "rb") as fh:
-            h.update(f.encode() + fh.read())
+        with open(os.path.join(d, f)) as fh:
+            src = fh.read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        src = "\n".join(line.split("//")[0].rstrip() for line in src.splitlines() if line.split("//")[0].strip())
+        h.update(f.encode() + src.encode())
     return h.hexdigest()[:16]
 
 

@@ -6,12 +6,15 @@
 // distribution q. Child k with token t_k is accepted iff u * q~_k(t_k) < r_{k-1}(t_k). On a
 // rejection r_k = max(0, r_{k-1} - q~_k) / Z_k (unchanged when Z_k = 0) and t_k leaves the
 // draft: q~_{k+1}(v) = q(v) / Q_{k+1} for the tokens not yet removed, Q_{k+1} = Q_k - q(t_k).
-// Every r_k(v) is therefore a short chain of max/scale steps applied to p(v) and q(v), so the
-// kernel stores only the scalars (t_i, Q_i, Z_i) and re-evaluates the chain per element in
-// each pass over the vocabulary: one pass per rejected child (for Z_k) and one final
-// prefix-scan draw at the node where the walk stops.
 //
-// One CTA of kTreeThreads per request. Row statistics come from the stats kernels.
+// Two kernels implement it. The cluster walk (tree_walk_cluster_kernel, below) spreads each
+// trie over a cluster of CTAs that stage the node's rows in shared memory. The fallback
+// (tree_walk_kernel, one CTA of kTreeThreads per trie, for devices that cannot schedule such
+// clusters) uses that every r_k(v) is a short chain of max/scale steps applied to p(v) and
+// q(v): it stores only the scalars (t_i, Q_i, Z_i) and re-evaluates the chain per element in
+// each pass over the vocabulary, one pass per rejected child (for Z_k) and one final
+// prefix-scan draw at the node where the walk stops. Its row statistics come from the stats
+// kernels.
 #pragma once
 
 #include <cooperative_groups.h>
