@@ -189,8 +189,8 @@ psispec_status psispec_verify_linear(const void* target_logits, const void* draf
  *   out_path       [B, max_depth] int32   local node ids of the accepted path, -1 padded
  *   out_tokens     [B, max_depth+1] int32 accepted tokens, then the final token, -1 padded
  *   out_accept_len [B] int32              number of accepted nodes, -1 on a data error
- * Limits: B >= 1, N >= B, N <= 2^26, 1 <= max_depth <= 64, at most 1024 nodes per request,
- * V <= 2^24.
+ * Limits: B >= 1, N >= B, N <= 2^26, 1 <= max_depth <= 64, V <= 2^24. A request with more
+ * than 1024 nodes, or a node with more than 64 children, is reported as a data error (-1).
  */
 psispec_status psispec_verify_tree(const void* target_logits, const void* draft_logits, int dtype,
                                    int32_t B, int32_t N, int32_t V, const int32_t* node_offsets,

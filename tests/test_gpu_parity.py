@@ -288,6 +288,57 @@ def test_verify_tree_mixed_requests_and_data_errors(V, dtype):
     compare_tree(out, ora)
 
 
+def test_verify_tree_structure_errors():
+    """Malformed tries are data errors confined to their request: a parent that is not
+    earlier, a token outside [0, V), a path deeper than max_depth, a root with a parent, an
+    empty request; the well-formed tries around them (one greedy) match the oracle. A node with
+    more than 64 children exceeds the walk's documented limit and is a data error there."""
+    V, D = 3000, 6
+    rng = np.random.default_rng(5)
+    parents, toks = [], []
+
+    def add(par, tk):
+        parents.append(np.asarray(par, np.int32))
+        toks.append(np.asarray(tk, np.int32))
+
+    def good(n):
+        par = [-1] + [int(rng.integers(0, i)) for i in range(1, n)]
+        depth = [0] * n
+        for i in range(1, n):  # keep the path length within D
+            if depth[par[i]] >= D:
+                par[i] = 0
+            depth[i] = depth[par[i]] + 1
+        return par, rng.choice(V, n, replace=False)
+
+    add(*good(16))                                        # 0: well formed
+    p1, t1 = good(12); p1[3] = 5; add(p1, t1)              # 1: parent after the node
+    p2, t2 = good(12); t2[2] = V; add(p2, t2)              # 2: token out of range
+    add(list(range(-1, 8)), rng.choice(V, 9, replace=False))  # 3: a chain of depth 8 > D
+    p4, t4 = good(10); p4[0] = 0; add(p4, t4)              # 4: the root has a parent
+    add([-1] + [0] * 70, rng.choice(V, 71, replace=False))   # 5: 70 children under the root
+    add([], [])                                           # 6: an empty request
+    add(*good(14))                                        # 7: well formed, greedy
+    B = len(parents)
+    offs = np.concatenate([[0], np.cumsum([len(x) for x in parents])]).astype(np.int32)
+    parent, tokens = np.concatenate(parents), np.concatenate(toks)
+    N = int(offs[-1])
+    g = torch.Generator().manual_seed(17)
+    tgt = _rand_logits(g, (N, V), torch.float32, 2.0)
+    drf = tgt + torch.randn((N, V), generator=g) * 0.5
+    Ts = torch.tensor([1.0] * (B - 1) + [0.0])
+    Ps = torch.ones(B)
+    ua, ur = synth.uniforms((N,), 18), synth.uniforms((N,), 19)
+    out = psispec.verify_tree(_cuda(tgt), _cuda(drf), _cuda(offs), _cuda(parent), _cuda(tokens), _cuda(ua),
+                              _cuda(ur), _cuda(Ts), _cuda(Ps), D)
+    ora = oracle.verify_tree(tgt, drf, offs, parent, tokens, ua, ur, Ts.numpy(), Ps.numpy(), D)
+    g_len = out["accept_len"].cpu().numpy()
+    assert (g_len[[1, 2, 3, 4, 5, 6]] == -1).all(), g_len
+    assert (ora["accept_len"][[1, 2, 3, 4, 6]] == -1).all(), ora["accept_len"]
+    assert (g_len[[0, 7]] >= 0).all()
+    keep = [0, 1, 2, 3, 4, 6, 7]  # request 5 is beyond the walk's limit only
+    compare_tree({k: v[keep] for k, v in out.items()}, {k: np.asarray(v)[keep] for k, v in ora.items()})
+
+
 def test_branching_one_tree_equals_linear_gpu():
     B, K, V = 6, 5, 12000
     tgt, drf, ud, ua, ur, Ts, Ps = _linear_inputs(B, K, V, torch.bfloat16, 0.9, 0.95, 0.6, seed=31)
