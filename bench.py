@@ -119,7 +119,10 @@ class ClockSampler:
                 "samples": len(rows), "power_w_max": max(float(r[3]) for r in rows)}
 
 
-def _dist():
+def _dist(backend: str = "nccl"):
+    """(process group module or None, rank, world size, local rank) from the torchrun
+    environment. Ranks are independent replicas; the only collectives are the timing barrier
+    and the max over ranks. The GPU bench uses NCCL; the host-side tests use gloo."""
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     if ws > 1:
         import datetime
@@ -127,8 +130,12 @@ def _dist():
         import torch.distributed as dist
 
         local = int(os.environ.get("LOCAL_RANK", "0"))
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
+        timeout = datetime.timedelta(seconds=120)
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=timeout, device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group(backend, timeout=timeout)
         return dist, dist.get_rank(), ws, local
     return None, 0, 1, 0
 
@@ -141,9 +148,15 @@ def _barrier(dist):
 def _max_over_ranks(dist, x: float) -> float:
     if dist is None:
         return x
-    t = torch.tensor([x], device="cuda", dtype=torch.float64)
+    on_gpu = dist.get_backend() == "nccl"
+    t = torch.tensor([x], device="cuda" if on_gpu else "cpu", dtype=torch.float64)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def _rank_seed(seed: int, rank: int) -> int:
+    """Each rank verifies its own batch (weak scaling): a seed per rank."""
+    return seed + 97 * rank
 
 
 def _oracle_sample(case, tgt_h, drf_h, ud, ua, ur, reqs):
@@ -321,10 +334,10 @@ def _prepare(name, dev, rank=0):
     lin, tre = synth.linear_cases(), synth.tree_cases()
     if name in lin:
         case = lin[name]
-        case.seed += 97 * rank  # each rank verifies its own batch
+        case.seed = _rank_seed(case.seed, rank)
         return _prepare_linear(case, dev), case
     case = tre[name]
-    case.seed += 97 * rank
+    case.seed = _rank_seed(case.seed, rank)
     return _prepare_tree(case, dev), case
 
 
