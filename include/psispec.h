@@ -71,7 +71,19 @@ typedef enum {
   PSISPEC_OP_ROW_STATS = 3
 } psispec_op;
 
-/* Bytes of one per-row statistics record written by psispec_sample_draft (out_row_stats). */
+/* Bytes of one per-row statistics record (psispec_sample_draft's out_row_stats,
+ * psispec_row_stats' output, psispec_verify_linear's draft_row_stats). Layout, in order:
+ *   float m       row maximum of the logits
+ *   float c       log2(e) / T (0 for a greedy row)
+ *   float s       sum over the row of 2^((l - m) c)
+ *   float s_kept  the same sum over the top-p kept set (= s without a cut)
+ *   uint32 tau    kept <=> key(l) >= tau, key the order-preserving map of the fp32 bits b
+ *                 of l (b | 0x80000000 when the sign bit is clear, ~b when it is set, -0
+ *                 taken as +0); tau = 0 keeps every token
+ *   int32 amax    lowest index of the maximum (greedy rows), -1 otherwise
+ *   int32 status  0, or 1 for a data error in the row
+ *   int32 pad
+ * so a kept token's probability is 2^((l - m) c) / s_kept. */
 #define PSISPEC_ROW_STATS_BYTES 32
 
 /* Human-readable name of a status code (static string, never NULL). */
