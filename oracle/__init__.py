@@ -50,11 +50,12 @@ def _load():
         lib = ctypes.CDLL(os.environ.get("ORACLE_LIB") or build())
         D, I = ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int)
         lib.oracle_row_dist.argtypes = [D, ctypes.c_int, ctypes.c_double, ctypes.c_double, D, D]
+        lib.oracle_row_dist_k.argtypes = [D, ctypes.c_int, ctypes.c_double, ctypes.c_double, ctypes.c_int, D, D]
         lib.oracle_inverse_cdf.argtypes = [D, ctypes.c_int, ctypes.c_double, D]
-        lib.oracle_sample_draft.argtypes = [D, ctypes.c_int, ctypes.c_int, I, D, D, D, I, D, D]
-        lib.oracle_verify_linear.argtypes = [D, D, ctypes.c_int, ctypes.c_int, ctypes.c_int, I, D, D, D, D,
+        lib.oracle_sample_draft.argtypes = [D, ctypes.c_int, ctypes.c_int, I, D, D, I, D, I, D, D]
+        lib.oracle_verify_linear.argtypes = [D, D, ctypes.c_int, ctypes.c_int, ctypes.c_int, I, D, D, D, D, I,
                                              I, I, D, D, D, D]
-        lib.oracle_verify_tree.argtypes = [D, D, ctypes.c_int, ctypes.c_int, I, I, I, D, D, D, D,
+        lib.oracle_verify_tree.argtypes = [D, D, ctypes.c_int, ctypes.c_int, I, I, I, D, D, D, D, I,
                                            ctypes.c_int, I, I, I, D]
         _lib = lib
     return _lib
@@ -79,14 +80,24 @@ def _as_f64(x):
     return np.asarray(x, dtype=np.float64)
 
 
-def row_dist(logits, temperature: float, top_p: float = 1.0):
-    """Distribution of one row after temperature and top-p. Returns (probs, e3_band) or
-    (None, inf) for a bad row."""
+def row_dist(logits, temperature: float, top_p: float = 1.0, top_k: int = 0):
+    """Distribution of one row after temperature, top-k (0: off) and top-p. Returns
+    (probs, e3_band) or (None, inf) for a bad row."""
     l, lp = _f64(_as_f64(logits).reshape(-1))
     out, op = _f64(np.zeros_like(l))
     band, bp = _f64(np.zeros(1))
-    rc = _load().oracle_row_dist(lp, l.size, float(temperature), float(top_p), op, bp)
+    if top_k:
+        rc = _load().oracle_row_dist_k(lp, l.size, float(temperature), float(top_p), int(top_k), op, bp)
+    else:
+        rc = _load().oracle_row_dist(lp, l.size, float(temperature), float(top_p), op, bp)
     return (None, float("inf")) if rc != 0 else (out, float(band[0]))
+
+
+def _top_k(top_k, B):
+    """Per-request top-k as an int32 array and its pointer, or (None, None) when off."""
+    if top_k is None:
+        return None, None
+    return _i32(np.broadcast_to(np.asarray(top_k, dtype=np.int32), (B,)))
 
 
 def inverse_cdf(r, u: float):
@@ -97,9 +108,9 @@ def inverse_cdf(r, u: float):
     return int(y), float(band[0])
 
 
-def sample_draft(draft_logits, temperature, top_p, u, row_req=None):
-    """draft_logits [rows, V]; temperature/top_p per request; u [rows]; row_req maps rows to
-    requests (default: row i -> request i). Returns dict(tokens, q, band)."""
+def sample_draft(draft_logits, temperature, top_p, u, row_req=None, top_k=None):
+    """draft_logits [rows, V]; temperature/top_p (and top_k, None: off) per request; u [rows];
+    row_req maps rows to requests (default: row i -> request i). Returns dict(tokens, q, band)."""
     d = _as_f64(draft_logits)
     rows, V = d.shape
     rr = np.arange(rows) if row_req is None else np.asarray(row_req)
@@ -111,13 +122,14 @@ def sample_draft(draft_logits, temperature, top_p, u, row_req=None):
     tok, tokp = _i32(np.zeros(rows))
     q, qp = _f64(np.zeros(rows))
     band, bp = _f64(np.zeros(rows))
-    _load().oracle_sample_draft(dp, rows, V, rrp, Tp, Pp, up, tokp, qp, bp)
+    Kk, Kkp = _top_k(top_k, P.size)
+    _load().oracle_sample_draft(dp, rows, V, rrp, Tp, Pp, Kkp, up, tokp, qp, bp)
     return {"tokens": tok, "q": q, "band": band}
 
 
-def verify_linear(target, draft, draft_tokens, u_accept, u_resid, temperature, top_p):
+def verify_linear(target, draft, draft_tokens, u_accept, u_resid, temperature, top_p, top_k=None):
     """target [B, K+1, V], draft [B, K, V], draft_tokens [B, K], u_accept [B, K],
-    u_resid [B, K+1], temperature [B], top_p [B]. Returns dict(tokens [B, K+1],
+    u_resid [B, K+1], temperature [B], top_p [B], top_k [B] (None: off). Returns dict(tokens [B, K+1],
     accept_len [B], p [B, K], q [B, K], band [B], pq_band [B, K])."""
     t = _as_f64(target)
     B, K1, V = t.shape
@@ -135,12 +147,13 @@ def verify_linear(target, draft, draft_tokens, u_accept, u_resid, temperature, t
     q, qp = _f64(np.zeros((B, K)))
     band, bp = _f64(np.zeros(B))
     pqb, pqbp = _f64(np.zeros((B, K)))
-    _load().oracle_verify_linear(tp, dp, B, K, V, xp, uap, urp, Tp, Pp, tokp, lnp, pp, qp, bp, pqbp)
+    Kk, Kkp = _top_k(top_k, B)
+    _load().oracle_verify_linear(tp, dp, B, K, V, xp, uap, urp, Tp, Pp, Kkp, tokp, lnp, pp, qp, bp, pqbp)
     return {"tokens": tok, "accept_len": ln, "p": p, "q": q, "band": band, "pq_band": pqb}
 
 
 def verify_tree(target, draft, node_offsets, parent, tokens, u_accept, u_resid, temperature, top_p,
-                max_depth: int):
+                max_depth: int, top_k=None):
     """target/draft [N, V]; node_offsets [B+1]; parent/tokens/u_accept/u_resid [N] (parent is
     the request-local index, -1 at the root). Returns dict(path [B, max_depth],
     tokens [B, max_depth+1], accept_len [B], band [B])."""
@@ -161,6 +174,7 @@ def verify_tree(target, draft, node_offsets, parent, tokens, u_accept, u_resid, 
     otk, otkp = _i32(np.zeros((B, max_depth + 1)))
     ln, lnp = _i32(np.zeros(B))
     band, bp = _f64(np.zeros(B))
-    _load().oracle_verify_tree(tp, dp, B, V, offp, parp, tkp, uap, urp, Tp, Pp, int(max_depth), pathp, otkp,
-                               lnp, bp)
+    Kk, Kkp = _top_k(top_k, B)
+    _load().oracle_verify_tree(tp, dp, B, V, offp, parp, tkp, uap, urp, Tp, Pp, Kkp, int(max_depth), pathp,
+                               otkp, lnp, bp)
     return {"path": path, "tokens": otk, "accept_len": ln, "band": band}

@@ -19,6 +19,11 @@
  *   - top-p keeps every token whose logit is >= tau, where tau is the largest logit value
  *     whose tie-inclusive upper-tail probability reaches top_p; it is applied after the
  *     temperature, to the verifier row and to the draft row separately;
+ *   - top-k (listed among the README's common controls, "--top-k", and defined nowhere on
+ *     the pages) keeps every token whose logit is >= the k-th largest logit of the row (ties
+ *     with it kept together); it acts after the temperature and before top-p, which then
+ *     works on the renormalised top-k set; k <= 0 or k >= V is off, and it is a no-op at
+ *     temperature 0;
  *   - temperature 0 is greedy: a point mass on the lowest-index maximum;
  *   - an inverse-CDF draw walks the vocabulary in index order and returns the first v with
  *     C(v) > u * Z (strict, inclusive prefix), so a zero-mass token is never drawn;
@@ -40,7 +45,7 @@ static int cmp_desc(const void* a, const void* b) {
   return (x < y) - (x > y);
 }
 
-int oracle_row_dist(const double* l, int V, double T, double top_p, double* out, double* band) {
+int oracle_row_dist_k(const double* l, int V, double T, double top_p, int top_k, double* out, double* band) {
   *band = INFINITY;
   if (V <= 0 || !(T >= 0)) return -1;
   int any_finite = 0;
@@ -70,34 +75,49 @@ int oracle_row_dist(const double* l, int V, double T, double top_p, double* out,
   }
 
   double tau = -INFINITY, S_kept = S;
-  if (top_p < 1.0) {
-    /* walk the distinct logit values from the top; stop at the first value whose
-       tie-inclusive tail mass reaches top_p of the total */
+  const int use_k = top_k > 0 && top_k < V;
+  if (use_k || top_p < 1.0) {
     double* vals = (double*)malloc(sizeof(double) * (size_t)V);
     memcpy(vals, l, sizeof(double) * (size_t)V);
     qsort(vals, (size_t)V, sizeof(double), cmp_desc);
-    double tail = 0.0;
-    int found = 0;
-    for (int i = 0; i < V;) {
-      double t = vals[i], group = 0.0;
-      int j = i;
-      while (j < V && vals[j] == t) { group += exp((t - m) / T); ++j; }
-      double above = tail;
-      tail += group;
-      if (tail >= top_p * S) {
-        tau = t;
-        S_kept = tail;
-        *band = dmin(fabs(tail / S - top_p), fabs(above / S - top_p));
-        found = 1;
-        break;
+    if (use_k) {
+      /* top-k: the k-th largest value, every token at or above it kept */
+      tau = vals[top_k - 1];
+      S_kept = 0.0;
+      for (int v = 0; v < V; ++v)
+        if (l[v] >= tau) S_kept += out[v];
+    }
+    if (top_p < 1.0) {
+      /* walk the distinct logit values of the kept set from the top; stop at the first value
+         whose tie-inclusive tail mass reaches top_p of the kept set's total */
+      const double floor_v = tau, total = S_kept;
+      double tail = 0.0;
+      int found = 0;
+      for (int i = 0; i < V && vals[i] >= floor_v;) {
+        double t = vals[i], group = 0.0;
+        int j = i;
+        while (j < V && vals[j] == t) { group += exp((t - m) / T); ++j; }
+        double above = tail;
+        tail += group;
+        if (tail >= top_p * total) {
+          tau = t;
+          S_kept = tail;
+          *band = dmin(fabs(tail / total - top_p), fabs(above / total - top_p));
+          found = 1;
+          break;
+        }
+        i = j;
       }
-      i = j;
+      if (!found) *band = 0.0;  /* rounding only: the whole kept set stays */
     }
     free(vals);
-    if (!found) { tau = -INFINITY; S_kept = S; *band = 0.0; }
   }
   for (int v = 0; v < V; ++v) out[v] = (l[v] >= tau) ? out[v] / S_kept : 0.0;
   return 0;
+}
+
+int oracle_row_dist(const double* l, int V, double T, double top_p, double* out, double* band) {
+  return oracle_row_dist_k(l, V, T, top_p, 0, out, band);
 }
 
 int oracle_inverse_cdf(const double* r, int V, double u, double* band) {
@@ -120,7 +140,7 @@ int oracle_inverse_cdf(const double* r, int V, double u, double* band) {
 }
 
 int oracle_sample_draft(const double* draft, int rows, int V, const int* row_req,
-                        const double* temperature, const double* top_p, const double* u,
+                        const double* temperature, const double* top_p, const int* top_k, const double* u,
                         int* tokens, double* q_at, double* band) {
   if (rows < 0 || V <= 0) return ORACLE_BAD_ARG;
   double* q = (double*)malloc(sizeof(double) * (size_t)V);
@@ -130,7 +150,8 @@ int oracle_sample_draft(const double* draft, int rows, int V, const int* row_req
     tokens[i] = -1;
     q_at[i] = -1.0;
     band[i] = INFINITY;
-    if (oracle_row_dist(draft + (size_t)i * V, V, temperature[b], top_p[b], q, &b3) != 0) continue;
+    if (oracle_row_dist_k(draft + (size_t)i * V, V, temperature[b], top_p[b], top_k ? top_k[b] : 0, q, &b3) != 0)
+      continue;
     int y = oracle_inverse_cdf(q, V, u[i], &b2);
     tokens[i] = y;
     q_at[i] = y >= 0 ? q[y] : -1.0;
@@ -142,7 +163,7 @@ int oracle_sample_draft(const double* draft, int rows, int V, const int* row_req
 
 int oracle_verify_linear(const double* target, const double* draft, int B, int K, int V,
                          const int* draft_tokens, const double* u_accept, const double* u_resid,
-                         const double* temperature, const double* top_p,
+                         const double* temperature, const double* top_p, const int* top_k,
                          int* out_tokens, int* accept_len, double* out_p, double* out_q,
                          double* band, double* pq_band) {
   if (B < 0 || K < 0 || V <= 0) return ORACLE_BAD_ARG;
@@ -151,6 +172,7 @@ int oracle_verify_linear(const double* target, const double* draft, int B, int K
   double* res = (double*)malloc(sizeof(double) * (size_t)V);
   for (int b = 0; b < B; ++b) {
     const double T = temperature[b], tp = top_p[b];
+    const int tk = top_k ? top_k[b] : 0;
     const double* tgt = target + (size_t)b * (K + 1) * V;
     const double* drf = draft + (size_t)b * K * V;
     int* toks = out_tokens + (size_t)b * (K + 1);
@@ -163,8 +185,8 @@ int oracle_verify_linear(const double* target, const double* draft, int B, int K
       double bp = INFINITY, bq = INFINITY;
       int x = draft_tokens[(size_t)b * K + i];
       if (x < 0 || x >= V) { bad = 1; break; }
-      if (oracle_row_dist(tgt + (size_t)i * V, V, T, tp, p, &bp) != 0) { bad = 1; break; }
-      if (oracle_row_dist(drf + (size_t)i * V, V, T, tp, q, &bq) != 0) { bad = 1; break; }
+      if (oracle_row_dist_k(tgt + (size_t)i * V, V, T, tp, tk, p, &bp) != 0) { bad = 1; break; }
+      if (oracle_row_dist_k(drf + (size_t)i * V, V, T, tp, tk, q, &bq) != 0) { bad = 1; break; }
       out_p[(size_t)b * K + i] = p[x];
       out_q[(size_t)b * K + i] = q[x];
       pq_band[(size_t)b * K + i] = dmin(bp, bq);
@@ -186,7 +208,7 @@ int oracle_verify_linear(const double* target, const double* draft, int B, int K
     }
     if (!bad) {
       double bp = INFINITY;
-      if (oracle_row_dist(tgt + (size_t)K * V, V, T, tp, p, &bp) != 0) bad = 1;
+      if (oracle_row_dist_k(tgt + (size_t)K * V, V, T, tp, tk, p, &bp) != 0) bad = 1;
       if (!bad && j == K) { /* whole block accepted: bonus draw from the last verifier row */
         double b2 = INFINITY;
         y = oracle_inverse_cdf(p, V, u_resid[(size_t)b * (K + 1) + K], &b2);
@@ -213,7 +235,7 @@ int oracle_verify_linear(const double* target, const double* draft, int B, int K
 int oracle_verify_tree(const double* target, const double* draft, int B, int V,
                        const int* node_offsets, const int* parent, const int* tokens,
                        const double* u_accept, const double* u_resid,
-                       const double* temperature, const double* top_p, int max_depth,
+                       const double* temperature, const double* top_p, const int* top_k, int max_depth,
                        int* out_path, int* out_tokens, int* accept_len, double* band) {
   if (B < 0 || V <= 0 || max_depth < 0) return ORACLE_BAD_ARG;
   double* r = (double*)malloc(sizeof(double) * (size_t)V);
@@ -222,6 +244,7 @@ int oracle_verify_tree(const double* target, const double* draft, int B, int V,
   for (int b = 0; b < B; ++b) {
     const int n0 = node_offsets[b], n = node_offsets[b + 1] - node_offsets[b];
     const double T = temperature[b], tp = top_p[b];
+    const int tk = top_k ? top_k[b] : 0;
     int* path = out_path + (size_t)b * max_depth;
     int* toks = out_tokens + (size_t)b * (max_depth + 1);
     for (int i = 0; i < max_depth; ++i) path[i] = -1;
@@ -245,12 +268,12 @@ int oracle_verify_tree(const double* target, const double* draft, int B, int V,
     int cur = 0, len = 0, y = -1;
     for (;;) {
       double b3 = INFINITY;
-      if (oracle_row_dist(target + (size_t)(n0 + cur) * V, V, T, tp, r, &b3) != 0) { bad = 1; break; }
+      if (oracle_row_dist_k(target + (size_t)(n0 + cur) * V, V, T, tp, tk, r, &b3) != 0) { bad = 1; break; }
       path_band = dmin(path_band, b3);
       int has_child = 0;
       for (int c = cur + 1; c < n; ++c) has_child |= parent[n0 + c] == cur;
       if (has_child && T > 0.0) {
-        if (oracle_row_dist(draft + (size_t)(n0 + cur) * V, V, T, tp, qt, &b3) != 0) { bad = 1; break; }
+        if (oracle_row_dist_k(draft + (size_t)(n0 + cur) * V, V, T, tp, tk, qt, &b3) != 0) { bad = 1; break; }
         path_band = dmin(path_band, b3);
       }
       int next = -1;

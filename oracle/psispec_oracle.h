@@ -44,28 +44,34 @@ extern "C" {
  * Returns 0, or -1 for a bad row (NaN or +inf logit, or no finite logit). */
 int oracle_row_dist(const double* l, int V, double T, double top_p, double* out, double* band);
 
+/* oracle_row_dist with top-k first: the tokens whose logit is >= the k-th largest logit of the
+ * row (ties kept together) stay, then top-p acts on that renormalised set (its E3 margin
+ * relative to the set's mass). top_k <= 0 or >= V is off; a no-op at T == 0. */
+int oracle_row_dist_k(const double* l, int V, double T, double top_p, int top_k, double* out, double* band);
+
 /* Inverse-CDF draw in vocabulary order: y = min{v : C(v) > u * Z}, C inclusive.
  * r[V] >= 0 need not be normalised. If no index qualifies (rounding), y is the last v with
  * r[v] > 0. Returns y, or -1 when Z == 0. *band receives the E2 margin. */
 int oracle_inverse_cdf(const double* r, int V, double u, double* band);
 
 /* Draft sampling, one draw per row.
- * draft[rows*V]; row_req[rows] maps a row to its request for temperature[]/top_p[];
+ * draft[rows*V]; row_req[rows] maps a row to its request for temperature[]/top_p[]/top_k[]
+ * (top_k may be NULL: off for every request);
  * u[rows]. Outputs: tokens[rows] (-1 on a bad row), q_at[rows] = q(token), band[rows]. */
 int oracle_sample_draft(const double* draft, int rows, int V, const int* row_req,
-                        const double* temperature, const double* top_p, const double* u,
+                        const double* temperature, const double* top_p, const int* top_k, const double* u,
                         int* tokens, double* q_at, double* band);
 
 /* Linear verification.
  * target[B*(K+1)*V], draft[B*K*V], draft_tokens[B*K], u_accept[B*K], u_resid[B*(K+1)],
- * temperature[B], top_p[B].
+ * temperature[B], top_p[B], top_k[B] or NULL (top-k off).
  * Outputs: out_tokens[B*(K+1)] (accepted prefix, then the resampled or bonus token, then -1),
  * accept_len[B] (-1 on a data error), out_p[B*K] = p_i(x_i), out_q[B*K] = q_i(x_i),
  * band[B] = smallest E1/E2/E3 margin on the request's path,
  * pq_band[B*K] = E3 margin of the two rows behind out_p/out_q at that position. */
 int oracle_verify_linear(const double* target, const double* draft, int B, int K, int V,
                          const int* draft_tokens, const double* u_accept, const double* u_resid,
-                         const double* temperature, const double* top_p,
+                         const double* temperature, const double* top_p, const int* top_k,
                          int* out_tokens, int* accept_len, double* out_p, double* out_q,
                          double* band, double* pq_band);
 
@@ -80,7 +86,7 @@ int oracle_verify_linear(const double* target, const double* draft, int B, int K
 int oracle_verify_tree(const double* target, const double* draft, int B, int V,
                        const int* node_offsets, const int* parent, const int* tokens,
                        const double* u_accept, const double* u_resid,
-                       const double* temperature, const double* top_p, int max_depth,
+                       const double* temperature, const double* top_p, const int* top_k, int max_depth,
                        int* out_path, int* out_tokens, int* accept_len, double* band);
 
 #ifdef __cplusplus

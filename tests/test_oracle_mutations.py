@@ -20,8 +20,8 @@ MUTATIONS = {
     "residual_sign": ("res[v] = p[v] > q[v] ? p[v] - q[v] : 0.0;", "res[v] = q[v] > p[v] ? q[v] - p[v] : 0.0;"),
     "residual_not_clipped": ("res[v] = p[v] > q[v] ? p[v] - q[v] : 0.0;", "res[v] = p[v];"),
     "cdf_not_strict": ("if (C > target) {", "if (C >= target) {"),
-    "bonus_wrong_row": ("oracle_row_dist(tgt + (size_t)K * V, V, T, tp, p, &bp)",
-                        "oracle_row_dist(tgt + (size_t)(K - 1) * V, V, T, tp, p, &bp)"),
+    "bonus_wrong_row": ("oracle_row_dist_k(tgt + (size_t)K * V, V, T, tp, tk, p, &bp)",
+                        "oracle_row_dist_k(tgt + (size_t)(K - 1) * V, V, T, tp, tk, p, &bp)"),
     "resid_uniform_index": ("u_resid[(size_t)b * (K + 1) + i], &b2);", "u_resid[(size_t)b * (K + 1) + i + 1], &b2);"),
     "temperature_multiplied": ("out[v] = exp((l[v] - m) / T);", "out[v] = exp((l[v] - m) * T);"),
     "topp_drops_ties": ("out[v] = (l[v] >= tau) ? out[v] / S_kept : 0.0;", "out[v] = (l[v] > tau) ? out[v] / S_kept : 0.0;"),
@@ -30,6 +30,9 @@ MUTATIONS = {
     "tree_no_removal": ("qt[t] = 0.0;", "(void)t;"),
     "tree_no_residual_update": ("for (int v = 0; v < V; ++v) r[v] = res[v] / Z;", "(void)Z;"),
     "tree_wrong_uniform": ("double u = u_accept[n0 + c];", "double u = u_accept[n0 + cur];"),
+    "topk_off_by_one": ("tau = vals[top_k - 1];", "tau = vals[top_k];"),
+    "topk_topp_over_whole_row": ("const double floor_v = tau, total = S_kept;",
+                                 "const double floor_v = tau, total = S;"),
 }
 
 

@@ -126,6 +126,81 @@ def test_topp_one_is_identity_and_tiny_keeps_max():
     np.testing.assert_allclose(p, [0, 0, 0.5, 0.5, 0])  # both tied maxima survive
 
 
+def _topk_topp_brute(l, T, top_k, top_p):
+    """Top-k by enumeration (every token whose value is at least the k-th of the sorted row),
+    then, on that renormalised set, the largest candidate threshold whose tie-inclusive tail
+    reaches top_p (every candidate tried)."""
+    V = l.size
+    p = scipy.special.softmax(l / T)
+    if 0 < top_k < V:
+        kth = sorted(l.tolist(), reverse=True)[top_k - 1]
+        p = np.where(l >= kth, p, 0.0)
+        p = p / p.sum()
+    if top_p < 1.0:
+        best = -np.inf
+        for t in np.unique(l[p > 0]):
+            if p[l >= t].sum() >= top_p:
+                best = max(best, t)
+        p = np.where(l >= best, p, 0.0)
+        p = p / p.sum()
+    return p
+
+
+def test_topk_brute_force_with_ties():
+    """Top-k then top-p (the reading for the README's --top-k), against enumeration on tiny
+    rows with forced ties and -inf entries, over every k from off to beyond V."""
+    rng = np.random.default_rng(11)
+    checked = 0
+    for _ in range(600):
+        V = int(rng.integers(1, 9))
+        l = rng.choice([-1.0, 0.0, 0.5, 1.0, 2.0, -np.inf], size=V)
+        if not np.isfinite(l).any():
+            continue
+        T = float(rng.choice([0.5, 1.0, 3.0]))
+        k = int(rng.integers(0, V + 2))
+        top_p = float(rng.choice([1.0, 0.33, 0.6, 0.9]))
+        p, band = oracle.row_dist(l, T, top_p, k)
+        if top_p < 1.0 and band < 1e-9:  # a threshold exactly on a tail boundary
+            continue
+        np.testing.assert_allclose(p, _topk_topp_brute(l, T, k, top_p), atol=1e-12)
+        checked += 1
+    assert checked > 450
+
+
+def test_topk_special_cases_and_order():
+    l = np.array([0.3, -1.0, 2.0, 2.0, 0.0])
+    off = oracle.row_dist(l, 1.0, 0.9)[0]
+    for k in (0, -3, 5, 9):  # off, and k >= V
+        np.testing.assert_allclose(oracle.row_dist(l, 1.0, 0.9, k)[0], off)
+    np.testing.assert_allclose(oracle.row_dist(l, 1.0, 1.0, 1)[0], [0, 0, 0.5, 0.5, 0])  # tied maxima stay
+    np.testing.assert_allclose(oracle.row_dist(l, 0.0, 1.0, 3)[0], [0, 0, 1, 0, 0])  # greedy: k is a no-op
+    # the order: top-p acts on the renormalised top-k set. With logits (2, 1, 0.5, 0), k = 3
+    # and top_p = 0.85, top-k first keeps (2, 1, 0.5) with shares (0.628, 0.231, 0.140), and
+    # top-p then stops after two tokens; top-p first would keep three.
+    e = math.e
+    np.testing.assert_allclose(oracle.row_dist([2.0, 1.0, 0.5, 0.0], 1.0, 0.85, 3)[0],
+                               [e * e / (e * e + e), e / (e * e + e), 0, 0], atol=1e-15)
+
+
+def test_topk_reaches_the_samplers():
+    """sample_draft draws from the top-k distribution, and q == p still accepts every position
+    with top-k on both rows."""
+    rng = np.random.default_rng(3)
+    V, K = 40, 3
+    d = rng.normal(size=(K, V)) * 2.0
+    u = np.array([0.1, 0.5, 0.93])
+    s = oracle.sample_draft(d, [1.0] * K, [0.9] * K, u, row_req=np.arange(K), top_k=[5] * K)
+    for i in range(K):
+        r, _ = oracle.row_dist(d[i], 1.0, 0.9, 5)
+        assert s["tokens"][i] == oracle.inverse_cdf(r, u[i])[0]
+        assert abs(s["q"][i] - r[s["tokens"][i]]) < 1e-15
+    t = rng.normal(size=(1, K + 1, V))
+    x = np.array([[int(np.argmax(t[0, i])) for i in range(K)]])  # tokens inside every top-k set
+    out = oracle.verify_linear(t, t[:, :K], x, np.full((1, K), 0.999), np.full((1, K + 1), 0.5), [1.0], [1.0],
+                               top_k=[4])
+    assert out["accept_len"][0] == K
+
+
 def test_inverse_cdf_exhaustive_grid():
     """Over a fine uniform grid, the fraction of u mapped to token v equals r(v)/Z exactly
     (dyadic weights, midpoint grid)."""
