@@ -167,10 +167,11 @@ def _oracle_sample(case, tgt_h, drf_h, ud, ua, ur, reqs):
     K, V = case.K, case.V
     n = len(reqs)
     T, P = np.full(n, case.temperature), np.full(n, case.top_p)
+    Kk = np.full(n, case.top_k, dtype=np.int32) if case.top_k else None
     d = drf_h[reqs].to(torch.float64).numpy()
-    s = oracle.sample_draft(d.reshape(n * K, V), T, P, ud[reqs].reshape(-1), row_req=np.arange(n * K) // K)
+    s = oracle.sample_draft(d.reshape(n * K, V), T, P, ud[reqs].reshape(-1), row_req=np.arange(n * K) // K, top_k=Kk)
     r = oracle.verify_linear(tgt_h[reqs].to(torch.float64).numpy(), d, s["tokens"].reshape(n, K), ua[reqs], ur[reqs],
-                             T, P)
+                             T, P, top_k=Kk)
     return r
 
 
@@ -247,6 +248,7 @@ def _prepare_linear(case, dev):
     ud, ua, ur = ud.to(dev), ua.to(dev), ur.to(dev)
     Ts = torch.full((B,), case.temperature, device=dev)
     Ps = torch.full((B,), case.top_p, device=dev)
+    Ks = torch.full((B,), case.top_k, dtype=torch.int32, device=dev) if case.top_k else None
     x = torch.empty((B, K), dtype=torch.int32, device=dev)
     q = torch.empty((B, K), dtype=torch.float32, device=dev)
     stats = torch.empty((B, K, psispec.ROW_STATS_BYTES), dtype=torch.uint8, device=dev)
@@ -261,10 +263,10 @@ def _prepare_linear(case, dev):
     esz = tgt.element_size()
 
     def sample(t_in=tgt, d_in=drf):
-        psispec.sample_draft(d_in, Ts, Ps, ud, out_tokens=x, out_q=q, row_stats=stats, ws=ws_s)
+        psispec.sample_draft(d_in, Ts, Ps, ud, top_k=Ks, out_tokens=x, out_q=q, row_stats=stats, ws=ws_s)
 
     def verify(t_in=tgt, d_in=drf):
-        psispec.verify_linear(t_in, d_in, x, ua, ur, Ts, Ps, draft_row_stats=stats, out_tokens=o_tok,
+        psispec.verify_linear(t_in, d_in, x, ua, ur, Ts, Ps, top_k=Ks, draft_row_stats=stats, out_tokens=o_tok,
                               out_accept_len=o_len, out_p=o_p, out_q=o_q, ws=ws_v)
 
     def stream_leg():  # the streaming pass over the verifier tensor alone (plus its row finalize)
@@ -281,8 +283,9 @@ def _prepare_linear(case, dev):
         "launches": 2 + 3,
         "kernel_leg": ("stream_partials_tma_kernel (psispec_row_stats over the verifier tensor)", stream_leg,
                        B * (K + 1) * V * esz),
-        "describe": "linear verify B=%d K=%d V=%d %s, T=%g, top-p %g" % (
-            B, K, V, "bf16" if esz == 2 else "fp32", case.temperature, case.top_p),
+        "describe": "linear verify B=%d K=%d V=%d %s, T=%g, top-p %g%s" % (
+            B, K, V, "bf16" if esz == 2 else "fp32", case.temperature, case.top_p,
+            ", top-k %d" % case.top_k if case.top_k else ""),
         "config": {"global_batch": B, "block": K, "vocab": V},
         "accept": lambda: float(o_len.float().mean()),
     }

@@ -30,6 +30,11 @@
  *    upper-tail probability is >= top_p; the distribution is renormalised over the kept set.
  *    It is applied after the temperature, to the verifier row and to the draft row
  *    separately, and it is a no-op at T == 0. (The pages leave top-p's definition open.)
+ *  - top_k (per request, the *_k entry points only; NULL for all requests off): the project
+ *    README lists it among the common sampling controls without defining it. Read plainly:
+ *    keep every token whose logit is >= the k-th largest logit of the row (ties with it kept
+ *    together), after the temperature and before top-p, which then acts on the renormalised
+ *    top-k set. k <= 0 or k >= V switches it off; it is a no-op at T == 0.
  *  - Uniforms u are floats in [0, 1) supplied by the caller; the library draws no random
  *    numbers. An inverse-CDF draw with uniform u over weights r returns the first index v, in
  *    vocabulary order, with C(v) > u * Z (C inclusive prefix sum, Z = sum of r), so a token of
@@ -123,6 +128,17 @@ psispec_status psispec_sample_draft(const void* draft_logits, int dtype, int32_t
                                     void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * psispec_sample_draft_k -- psispec_sample_draft with a per-request top-k (see the
+ * conventions above): top_k [B] int32 device array, or NULL (off for every request). Row
+ * statistics records written here carry the top-k threshold and can be passed to
+ * psispec_verify_linear_k with the same top_k.
+ */
+psispec_status psispec_sample_draft_k(const void* draft_logits, int dtype, int32_t B, int32_t K, int32_t V,
+                                      const float* temperature, const float* top_p, const int32_t* top_k,
+                                      const float* u, int32_t* out_tokens, float* out_q, void* out_row_stats,
+                                      void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * psispec_row_stats -- the per-row statistics of the sampling distribution softmax(l / T)
  * after top-p over the full vocabulary (review page, section 3.3: both distributions of the
  * rule are taken after the sampling controls): row maximum, normaliser, top-p threshold and
@@ -172,6 +188,20 @@ psispec_status psispec_verify_linear(const void* target_logits, const void* draf
                                      int32_t* out_tokens, int32_t* out_accept_len, float* out_p,
                                      float* out_q, void* workspace, size_t workspace_bytes,
                                      void* stream);
+
+/*
+ * psispec_verify_linear_k -- psispec_verify_linear with a per-request top-k applied to the
+ * verifier rows and the draft rows alike: top_k [B] int32 device array, or NULL (off for
+ * every request). draft_row_stats, when given, must come from psispec_sample_draft_k with
+ * the same top_k. Same workspace size, limits and errors as psispec_verify_linear.
+ */
+psispec_status psispec_verify_linear_k(const void* target_logits, const void* draft_logits, int dtype,
+                                       int32_t B, int32_t K, int32_t V, const int32_t* draft_tokens,
+                                       const void* draft_row_stats, const float* u_accept,
+                                       const float* u_resid, const float* temperature, const float* top_p,
+                                       const int32_t* top_k, int32_t* out_tokens, int32_t* out_accept_len,
+                                       float* out_p, float* out_q, void* workspace, size_t workspace_bytes,
+                                       void* stream);
 
 /*
  * psispec_verify_tree -- Psi-Spec tree verification (tree sampler of the review page's

@@ -257,9 +257,11 @@ __device__ __forceinline__ float key_value(uint32_t key) {
   return (key & 0x80000000u) ? __uint_as_float(key & 0x7FFFFFFFu) : __uint_as_float(~key);
 }
 
-// Smallest kept logit value of a top-p threshold key as a float bound: l is kept iff
-// l >= cut_value(tau), which equals fkey(l) >= tau for every non-NaN l (tau == 0 keeps all).
-__device__ __forceinline__ float cut_value(uint32_t tau) { return tau == 0u ? -INFINITY : key_value(tau); }
+// Smallest kept logit value of a threshold key as a float bound: l is kept iff
+// l >= cut_value(tau), which equals fkey(l) >= tau for every non-NaN l. A key at or below the
+// key of -inf (0 included, and the 16-bit prefix 0x007F0000 a bf16 select leaves for -inf,
+// whose inverse bits would be a NaN) keeps every value.
+__device__ __forceinline__ float cut_value(uint32_t tau) { return tau <= 0x007FFFFFu ? -INFINITY : key_value(tau); }
 
 // Weight of logit l under row statistics st (kept set applied); greedy rows are handled by
 // the callers.

@@ -293,6 +293,7 @@ struct VerifyArgs {
   int B, K, V, stream_draft;
   const float* temperature;
   const float* top_p;
+  const int32_t* top_k;  // per request, or null (off)
   const int32_t* tokens;
   const RowStat* dstats_in;
   const float* u_acc;

@@ -265,7 +265,7 @@ psispec_status prepare_topp(Kern kernel, int64_t rows, unsigned* grid) {
 
 template <typename T>
 psispec_status sample_draft_impl(const T* draft, int B, int K, int V, const float* temperature, const float* top_p,
-                                 const float* u, int32_t* out_tokens, float* out_q, RowStat* out_stats, void* ws,
+                                 const int32_t* top_k, const float* u, int32_t* out_tokens, float* out_q, RowStat* out_stats, void* ws,
                                  cudaStream_t st) {
   const int64_t rows = int64_t(B) * K;
   Carver c(ws);
@@ -279,14 +279,15 @@ psispec_status sample_draft_impl(const T* draft, int B, int K, int V, const floa
   if ((s = prepare_topp(sample_rows_kernel<T>, rows, &tgrid)) != PSISPEC_OK) return s;
   const int warp_ctas = static_cast<int>((rows + kTpWarps - 1) / kTpWarps);
   return launch(sample_rows_kernel<T>, warp_ctas + tgrid, kTpThreads, sizeof(TpSmem), st, draft, K, V,
-                static_cast<int>(rows), temperature, top_p, u, w.st.parts, stats, out_tokens, out_q, warp_ctas);
+                static_cast<int>(rows), temperature, top_p, top_k, u, w.st.parts, stats, out_tokens, out_q, warp_ctas);
 }
 
 template <typename T>
 psispec_status verify_linear_impl(const T* tgt, const T* drf, int B, int K, int V, const int32_t* tokens,
                                   const RowStat* draft_stats, const float* u_acc, const float* u_res,
-                                  const float* temperature, const float* top_p, int32_t* out_tokens,
-                                  int32_t* out_len, float* out_p, float* out_q, void* ws, cudaStream_t st) {
+                                  const float* temperature, const float* top_p, const int32_t* top_k,
+                                  int32_t* out_tokens, int32_t* out_len, float* out_p, float* out_q, void* ws,
+                                  cudaStream_t st) {
   Carver c(ws);
   LinearWs w = carve_linear(c, B, K, V);
   const int64_t rows_t = int64_t(B) * (K + 1), rows_d = draft_stats ? 0 : int64_t(B) * K;
@@ -297,6 +298,7 @@ psispec_status verify_linear_impl(const T* tgt, const T* drf, int B, int K, int 
   a.stream_draft = draft_stats ? 0 : 1;
   a.temperature = temperature;
   a.top_p = top_p;
+  a.top_k = top_k;
   a.tokens = tokens;
   a.dstats_in = draft_stats;
   a.u_acc = u_acc;
@@ -319,7 +321,7 @@ psispec_status verify_linear_impl(const T* tgt, const T* drf, int B, int K, int 
   if (rows_d > 0 &&
       (s = launch_stream<T>(one_tensor(drf, rows_d, K, B), rows_d, V, temperature, B, w.d.parts, st)) != PSISPEC_OK)
     return s;
-  // one row kernel: warps for the requests without a top-p cut, whole CTAs for the others
+  // one row kernel: warps for the requests without a cut, whole CTAs for the others
   unsigned tgrid = 1;
   if ((s = prepare_topp(verify_rows_kernel<T>, rows_t + rows_d, &tgrid)) != PSISPEC_OK) return s;
   const int warp_ctas = static_cast<int>((rows_t + rows_d + kTpWarps - 1) / kTpWarps);
@@ -447,10 +449,10 @@ size_t psispec_workspace_size(int op, int64_t a, int64_t b, int64_t c) {
   return m.used;
 }
 
-psispec_status psispec_sample_draft(const void* draft_logits, int dtype, int32_t B, int32_t K, int32_t V,
-                                    const float* temperature, const float* top_p, const float* u,
-                                    int32_t* out_tokens, float* out_q, void* out_row_stats, void* workspace,
-                                    size_t workspace_bytes, void* stream) {
+psispec_status psispec_sample_draft_k(const void* draft_logits, int dtype, int32_t B, int32_t K, int32_t V,
+                                      const float* temperature, const float* top_p, const int32_t* top_k,
+                                      const float* u, int32_t* out_tokens, float* out_q, void* out_row_stats,
+                                      void* workspace, size_t workspace_bytes, void* stream) {
   if (!draft_logits || !temperature || !top_p || !u || !out_tokens || bad_dtype(dtype)) return PSISPEC_ERR_INVALID_ARG;
   if (B <= 0 || K <= 0 || V <= 0) return PSISPEC_ERR_INVALID_ARG;
   if (!aligned_to(draft_logits, esize(dtype)) || (out_row_stats && !aligned_to(out_row_stats, 16)))
@@ -462,17 +464,26 @@ psispec_status psispec_sample_draft(const void* draft_logits, int dtype, int32_t
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   RowStat* rs = static_cast<RowStat*>(out_row_stats);
   if (dtype == PSISPEC_BF16)
-    return sample_draft_impl(static_cast<const __nv_bfloat16*>(draft_logits), B, K, V, temperature, top_p, u,
+    return sample_draft_impl(static_cast<const __nv_bfloat16*>(draft_logits), B, K, V, temperature, top_p, top_k, u,
                              out_tokens, out_q, rs, workspace, st);
-  return sample_draft_impl(static_cast<const float*>(draft_logits), B, K, V, temperature, top_p, u, out_tokens, out_q,
-                           rs, workspace, st);
+  return sample_draft_impl(static_cast<const float*>(draft_logits), B, K, V, temperature, top_p, top_k, u, out_tokens,
+                           out_q, rs, workspace, st);
 }
 
-psispec_status psispec_verify_linear(const void* target_logits, const void* draft_logits, int dtype, int32_t B,
-                                     int32_t K, int32_t V, const int32_t* draft_tokens, const void* draft_row_stats,
-                                     const float* u_accept, const float* u_resid, const float* temperature,
-                                     const float* top_p, int32_t* out_tokens, int32_t* out_accept_len, float* out_p,
-                                     float* out_q, void* workspace, size_t workspace_bytes, void* stream) {
+psispec_status psispec_sample_draft(const void* draft_logits, int dtype, int32_t B, int32_t K, int32_t V,
+                                    const float* temperature, const float* top_p, const float* u,
+                                    int32_t* out_tokens, float* out_q, void* out_row_stats, void* workspace,
+                                    size_t workspace_bytes, void* stream) {
+  return psispec_sample_draft_k(draft_logits, dtype, B, K, V, temperature, top_p, nullptr, u, out_tokens, out_q,
+                                out_row_stats, workspace, workspace_bytes, stream);
+}
+
+psispec_status psispec_verify_linear_k(const void* target_logits, const void* draft_logits, int dtype, int32_t B,
+                                       int32_t K, int32_t V, const int32_t* draft_tokens, const void* draft_row_stats,
+                                       const float* u_accept, const float* u_resid, const float* temperature,
+                                       const float* top_p, const int32_t* top_k, int32_t* out_tokens,
+                                       int32_t* out_accept_len, float* out_p, float* out_q, void* workspace,
+                                       size_t workspace_bytes, void* stream) {
   if (!target_logits || !draft_logits || !draft_tokens || !u_accept || !u_resid || !temperature || !top_p ||
       !out_tokens || !out_accept_len || bad_dtype(dtype))
     return PSISPEC_ERR_INVALID_ARG;
@@ -490,10 +501,21 @@ psispec_status psispec_verify_linear(const void* target_logits, const void* draf
   if (dtype == PSISPEC_BF16)
     return verify_linear_impl(static_cast<const __nv_bfloat16*>(target_logits),
                               static_cast<const __nv_bfloat16*>(draft_logits), B, K, V, draft_tokens, ds, u_accept,
-                              u_resid, temperature, top_p, out_tokens, out_accept_len, out_p, out_q, workspace, st);
+                              u_resid, temperature, top_p, top_k, out_tokens, out_accept_len, out_p, out_q, workspace,
+                              st);
   return verify_linear_impl(static_cast<const float*>(target_logits), static_cast<const float*>(draft_logits), B, K, V,
-                            draft_tokens, ds, u_accept, u_resid, temperature, top_p, out_tokens, out_accept_len, out_p,
-                            out_q, workspace, st);
+                            draft_tokens, ds, u_accept, u_resid, temperature, top_p, top_k, out_tokens,
+                            out_accept_len, out_p, out_q, workspace, st);
+}
+
+psispec_status psispec_verify_linear(const void* target_logits, const void* draft_logits, int dtype, int32_t B,
+                                     int32_t K, int32_t V, const int32_t* draft_tokens, const void* draft_row_stats,
+                                     const float* u_accept, const float* u_resid, const float* temperature,
+                                     const float* top_p, int32_t* out_tokens, int32_t* out_accept_len, float* out_p,
+                                     float* out_q, void* workspace, size_t workspace_bytes, void* stream) {
+  return psispec_verify_linear_k(target_logits, draft_logits, dtype, B, K, V, draft_tokens, draft_row_stats, u_accept,
+                                 u_resid, temperature, top_p, nullptr, out_tokens, out_accept_len, out_p, out_q,
+                                 workspace, workspace_bytes, stream);
 }
 
 psispec_status psispec_verify_tree(const void* target_logits, const void* draft_logits, int dtype, int32_t B,

@@ -667,7 +667,7 @@ struct RadixSmem {
   double hmass[256];
   int hcnt[256];
   uint32_t prefix;
-  double above, bucket;
+  double above, bucket, cabove;
 };
 
 struct ToppSmem {
@@ -729,12 +729,19 @@ __device__ __forceinline__ void for_each_elem_batched(const T* __restrict__ row,
 
 // General top-p select (fallback when the threshold lies below the first pass's value range):
 // radix select on the 32-bit keys with fp64 atomics.
-template <typename T>
-__device__ void block_topp_radix(const T* __restrict__ rp, int V, float tp, RowStat& st, RadixSmem& sm) {
+// One most-significant-digit radix select over the order keys of row rp (8 bits a level; 2
+// levels cover a bf16 value, 4 an fp32 one), with the count and the fp64 weight of every
+// digit. BY_COUNT: the key of the goal-th largest element (ties kept together); otherwise the
+// largest key whose tie-inclusive tail weight reaches goal. Elements with a key below
+// floor_key take no part. Returns the key; *above gets the weight of the elements strictly
+// above its final digit bucket and *bucket that bucket's weight, so *above + *bucket is the
+// weight of every element with a key >= the returned one. The result is in every thread.
+template <typename T, bool BY_COUNT>
+__device__ uint32_t block_radix_pick(const T* __restrict__ rp, int V, const RowStat& st, double goal,
+                                     uint32_t floor_key, RadixSmem& sm, double* above, double* bucket) {
   const float M = st.m, c = st.c;
-  const double target = static_cast<double>(tp) * static_cast<double>(st.s);
   const int levels = sizeof(T) == 2 ? 2 : 4;
-  if (threadIdx.x == 0) { sm.prefix = 0u; sm.above = 0.0; sm.bucket = 0.0; }
+  if (threadIdx.x == 0) { sm.prefix = 0u; sm.above = 0.0; sm.bucket = 0.0; sm.cabove = 0.0; }
   for (int lv = 0; lv < levels; ++lv) {
     const int shift = 24 - 8 * lv;
     for (int d = threadIdx.x; d < 256; d += blockDim.x) { sm.hmass[d] = 0.0; sm.hcnt[d] = 0; }
@@ -742,7 +749,7 @@ __device__ void block_topp_radix(const T* __restrict__ rp, int V, float tp, RowS
     const uint32_t prefix = sm.prefix;
     for_each_elem(rp, V, [&](float x) {
       const uint32_t k = fkey(x);
-      if (lv == 0 || (k >> (shift + 8)) == (prefix >> (shift + 8))) {
+      if (k >= floor_key && (lv == 0 || (k >> (shift + 8)) == (prefix >> (shift + 8)))) {
         const int d = (k >> shift) & 255;
         atomicAdd(&sm.hmass[d], static_cast<double>(ex2((x - M) * c)));
         atomicAdd(&sm.hcnt[d], 1);
@@ -750,28 +757,61 @@ __device__ void block_topp_radix(const T* __restrict__ rp, int V, float tp, RowS
     });
     __syncthreads();
     if (threadIdx.x == 0) {
-      double running = sm.above;
+      double running = sm.above, counted = sm.cabove;
       int pick = -1;
       for (int d = 255; d >= 0; --d) {
         if (sm.hcnt[d] == 0) continue;
-        if (running + sm.hmass[d] >= target) { pick = d; break; }
+        if (BY_COUNT ? counted + sm.hcnt[d] >= goal : running + sm.hmass[d] >= goal) { pick = d; break; }
         running += sm.hmass[d];
+        counted += sm.hcnt[d];
       }
-      if (pick < 0) {  // rounding left the target unreached: keep the whole candidate range
+      if (pick < 0) {  // the goal is not reached (rounding, or fewer elements): the lowest bucket
         running = sm.above;
+        counted = sm.cabove;
         for (int d = 255; d >= 0; --d)
-          if (sm.hcnt[d] != 0) { pick = d; running += sm.hmass[d]; }
+          if (sm.hcnt[d] != 0) { pick = d; running += sm.hmass[d]; counted += sm.hcnt[d]; }
+        if (pick < 0) pick = 0;
         running -= sm.hmass[pick];
+        counted -= sm.hcnt[pick];
       }
       sm.prefix = prefix | (static_cast<uint32_t>(pick) << shift);
       sm.above = running;
+      sm.cabove = counted;
       sm.bucket = sm.hmass[pick];
     }
     __syncthreads();
   }
-  st.tau = sm.prefix;
-  st.s_kept = static_cast<float>(sm.above + sm.bucket);
+  const uint32_t key = sm.prefix;
+  *above = sm.above;
+  *bucket = sm.bucket;
   __syncthreads();
+  return key;
+}
+
+// General top-p select (any dtype and V): the largest key whose tail weight reaches top_p of
+// the row's total. Sets st.tau and st.s_kept in every thread.
+template <typename T>
+__device__ void block_topp_radix(const T* __restrict__ rp, int V, float tp, RowStat& st, RadixSmem& sm) {
+  double above, bucket;
+  st.tau = block_radix_pick<T, false>(rp, V, st, static_cast<double>(tp) * static_cast<double>(st.s), 0u, sm, &above,
+                                      &bucket);
+  st.s_kept = static_cast<float>(above + bucket);
+}
+
+// General top-k then top-p select (any dtype and V): the k-th largest key first (every
+// element at or above it kept), then, among those, the largest key whose tail weight reaches
+// top_p of their total. Sets st.tau and st.s_kept in every thread.
+template <typename T>
+__device__ void block_topk_topp_radix(const T* __restrict__ rp, int V, float tp, int k, RowStat& st, RadixSmem& sm) {
+  double above, bucket;
+  const uint32_t tau_k = block_radix_pick<T, true>(rp, V, st, static_cast<double>(k), 0u, sm, &above, &bucket);
+  const double s_k = above + bucket;
+  st.tau = tau_k;
+  st.s_kept = static_cast<float>(s_k);
+  if (tp < 1.0f) {
+    st.tau = block_radix_pick<T, false>(rp, V, st, static_cast<double>(tp) * s_k, tau_k, sm, &above, &bucket);
+    st.s_kept = static_cast<float>(above + bucket);
+  }
 }
 
 // Block-level top-p threshold of row rp under statistics st (m, c, s set); sets st.tau and

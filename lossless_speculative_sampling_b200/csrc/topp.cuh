@@ -465,11 +465,15 @@ __device__ RowStat tp_row_stats(const T* __restrict__ row, int V, float Tv, floa
 // Returns false (and leaves st alone) when the window holds less than that.
 constexpr int kTpWindow = 2048;
 
-// The logit value of a 16-bit order key of a bf16 number.
-__device__ __forceinline__ float key16_value(uint32_t k16) { return key_value(k16 << 16); }
+// The logit value of a 16-bit order key of a bf16 number (the inverse of fkey(x) >> 16 on
+// bf16 values: positive keys carry the bits with the sign set, negative keys their complement).
+__device__ __forceinline__ float key16_value(uint32_t k16) {
+  const uint32_t b16 = (k16 & 0x8000u) ? (k16 & 0x7FFFu) : (~k16 & 0xFFFFu);
+  return __uint_as_float(b16 << 16);
+}
 
 template <typename T>
-__device__ bool tp_window_select(const T* __restrict__ row, int V, float tp, RowStat& st, TpSmem& sm) {
+__device__ bool tp_window_select(const T* __restrict__ row, int V, float tp, int k, RowStat& st, TpSmem& sm) {
   static_assert(sizeof(T) == 2, "bf16 rows");
   static_assert(kTpWarps * kTpWindow <= kTpBins * kTpThreads, "window counts reuse the private counters");
   uint32_t* cnt = &sm.priv[0][0];  // [kTpWarps][kTpWindow]
@@ -517,21 +521,57 @@ __device__ bool tp_window_select(const T* __restrict__ row, int V, float tp, Row
   // masses of offsets [8t, 8t + 8) in thread t, scanned in thread order
   constexpr int kPer = kTpWindow / kTpThreads;
   double mass[kPer];
-  double tsum = 0.0;
+  uint32_t cnt8[kPer];
+  double tsum = 0.0, tcnt = 0.0;
 #pragma unroll
   for (int j = 0; j < kPer; ++j) {
     const int o = threadIdx.x * kPer + j;
     uint32_t c = 0u;
 #pragma unroll
     for (int w = 0; w < kTpWarps; ++w) c += cnt[w * kTpWindow + o];
+    cnt8[j] = km >= static_cast<uint32_t>(o) ? c : 0u;
     mass[j] = 0.0;
-    if (c != 0u && km >= static_cast<uint32_t>(o))
-      mass[j] = static_cast<double>(c) * static_cast<double>(ex2((key16_value(km - o) - st.m) * st.c));
+    if (cnt8[j] != 0u) mass[j] = static_cast<double>(c) * static_cast<double>(ex2((key16_value(km - o) - st.m) * st.c));
     tsum += mass[j];
+    tcnt += static_cast<double>(cnt8[j]);
   }
   double total;
   const double C0 = block_exclusive_scan(tsum, sm.mass, &total);
-  const double target = static_cast<double>(tp) * static_cast<double>(st.s);
+  // top-k: the offset of the k-th largest element (ties kept together) bounds the kept set;
+  // the top-p target is then top_p of the mass at or above it
+  int o_lim = kTpWindow - 1;
+  double s_k = static_cast<double>(st.s);
+  if (k > 0) {
+    double count_total;
+    const double K0 = block_exclusive_scan(tcnt, sm.mass, &count_total);
+    if (!(count_total >= static_cast<double>(k))) return false;  // the k-th value lies below the window
+    if (threadIdx.x == 0) sm.bin = -1;
+    __syncthreads();
+    if (K0 < static_cast<double>(k) && K0 + tcnt >= static_cast<double>(k)) {
+      double run = K0, runm = C0;
+#pragma unroll
+      for (int j = 0; j < kPer; ++j) {
+        run += static_cast<double>(cnt8[j]);
+        runm += mass[j];
+        if (run >= static_cast<double>(k)) {
+          sm.bin = threadIdx.x * kPer + j;
+          sm.tgt = runm;
+          break;
+        }
+      }
+    }
+    __syncthreads();
+    o_lim = sm.bin;
+    s_k = sm.tgt;
+    __syncthreads();
+    if (o_lim < 0) return false;  // uniform
+    if (!(tp < 1.0f)) {  // top-k alone
+      st.tau = (km - static_cast<uint32_t>(o_lim)) << 16;
+      st.s_kept = static_cast<float>(s_k);
+      return true;
+    }
+  }
+  const double target = static_cast<double>(tp) * s_k;
   if (!(total >= target)) return false;  // the threshold lies below the window (uniform)
   if (threadIdx.x == 0) sm.bin = -1;
   __syncthreads();
@@ -555,13 +595,14 @@ __device__ bool tp_window_select(const T* __restrict__ row, int V, float tp, Row
     if (threadIdx.x == 0) {
       double run = 0.0;
       int pick = -1;
-      for (int o = 0; o < kTpWindow && pick < 0; ++o) {
+      for (int o = 0; o <= o_lim && pick < 0; ++o) {
         uint32_t c = 0u;
         for (int w = 0; w < kTpWarps; ++w) c += cnt[w * kTpWindow + o];
         if (c == 0u || km < static_cast<uint32_t>(o)) continue;
         run += static_cast<double>(c) * static_cast<double>(ex2((key16_value(km - o) - st.m) * st.c));
         if (run >= target) pick = o;
       }
+      if (pick < 0 && k > 0) pick = o_lim;  // rounding: the whole top-k set
       sm.bin = pick;
       sm.base = run;
     }
@@ -569,16 +610,22 @@ __device__ bool tp_window_select(const T* __restrict__ row, int V, float tp, Row
     ostar = sm.bin;
     if (ostar < 0) return false;  // uniform
   }
+  if (ostar > o_lim) {  // rounding past the top-k bound: the whole top-k set
+    ostar = o_lim;
+    if (threadIdx.x == 0) sm.base = s_k;
+    __syncthreads();
+  }
   st.tau = (km - static_cast<uint32_t>(ostar)) << 16;
   st.s_kept = static_cast<float>(sm.base);
   __syncthreads();
   return true;
 }
 
-// Statistics of a row of a request with a top-p cut: maximum and normaliser from the row's
-// chunk partials, the threshold from the value window (bf16), else passes A-C over the row.
+// Statistics of a row of a request with a top-p or top-k cut: maximum and normaliser from the
+// row's chunk partials, the threshold from the value window (bf16), else passes A-C over the
+// row (top-p alone) or the general radix select (top-k). k is the request's top-k (0: off).
 template <typename T>
-__device__ RowStat tp_row_stats_partials(const T* __restrict__ row, int V, float Tv, float tp,
+__device__ RowStat tp_row_stats_partials(const T* __restrict__ row, int V, float Tv, float tp, int k,
                                          const Partial* __restrict__ pp, TpSmem& sm) {
   if (threadIdx.x < 32) {
     const RowStat s0 = warp_finalize_pick(pp, nchunks_for(V), Tv, 0.0f, false).st;
@@ -589,7 +636,11 @@ __device__ RowStat tp_row_stats_partials(const T* __restrict__ row, int V, float
   __syncthreads();
   if (st.status != 0) return st;
   if constexpr (sizeof(T) == 2) {
-    if (tp_window_select<T>(row, V, tp, st, sm)) return st;
+    if (tp_window_select<T>(row, V, tp, k, st, sm)) return st;
+  }
+  if (k > 0) {
+    block_topk_topp_radix<T>(row, V, tp, k, st, sm.radix);
+    return st;
   }
   return tp_row_stats(row, V, Tv, tp, sm);
 }
@@ -670,10 +721,16 @@ __device__ int tp_row_draw(const T* __restrict__ row, int V, const RowStat& st, 
   return y;
 }
 
-// Whether request r's rows carry a top-p cut.
+// Request r's top-k (0 when off: no array, k <= 0 or k >= V).
+__device__ __forceinline__ int request_k(const int32_t* __restrict__ top_k, int r, int V) {
+  const int k = top_k ? top_k[r] : 0;
+  return k > 0 && k < V ? k : 0;
+}
+
+// Whether request r's rows carry a cut (top-p below 1 or an active top-k, at T > 0).
 __device__ __forceinline__ bool request_cut(const float* __restrict__ temperature, const float* __restrict__ top_p,
-                                            int r) {
-  return top_p[r] < 1.0f && temp_scale(temperature[r]) != 0.0f;
+                                            const int32_t* __restrict__ top_k, int r, int V) {
+  return temp_scale(temperature[r]) != 0.0f && (top_p[r] < 1.0f || request_k(top_k, r, V) > 0);
 }
 
 // The row kernel of sample_draft. CTAs [0, warp_ctas) finish the rows without a top-p cut,
@@ -683,6 +740,7 @@ template <typename T>
 __global__ void __launch_bounds__(kTpThreads, 2) sample_rows_kernel(const T* __restrict__ draft, int K, int V,
                                                                    int rows, const float* __restrict__ temperature,
                                                                    const float* __restrict__ top_p,
+                                                                   const int32_t* __restrict__ top_k,
                                                                    const float* __restrict__ u,
                                                                    const Partial* __restrict__ parts,
                                                                    RowStat* __restrict__ stats,
@@ -690,7 +748,7 @@ __global__ void __launch_bounds__(kTpThreads, 2) sample_rows_kernel(const T* __r
                                                                    float* __restrict__ out_q, int warp_ctas) {
   if (static_cast<int>(blockIdx.x) < warp_ctas) {
     const int row = blockIdx.x * kTpWarps + (threadIdx.x >> 5);
-    if (row < rows && !request_cut(temperature, top_p, row / K))
+    if (row < rows && !request_cut(temperature, top_p, top_k, row / K, V))
       warp_sample_row(draft, row, K, V, temperature, u, parts, stats, out_tokens, out_q);
     return;
   }
@@ -699,10 +757,10 @@ __global__ void __launch_bounds__(kTpThreads, 2) sample_rows_kernel(const T* __r
   const int ctas = static_cast<int>(gridDim.x) - warp_ctas;
   for (int row = static_cast<int>(blockIdx.x) - warp_ctas; row < rows; row += ctas) {
     const int b = row / K;
-    if (!request_cut(temperature, top_p, b)) continue;
+    if (!request_cut(temperature, top_p, top_k, b, V)) continue;
     const T* rp = draft + static_cast<size_t>(row) * V;
-    const RowStat st =
-        tp_row_stats_partials(rp, V, temperature[b], top_p[b], parts + static_cast<size_t>(row) * nchunks_for(V), sm);
+    const RowStat st = tp_row_stats_partials(rp, V, temperature[b], top_p[b], request_k(top_k, b, V),
+                                             parts + static_cast<size_t>(row) * nchunks_for(V), sm);
     float q = -1.0f;
     const int y = st.status == 0 ? tp_row_draw(rp, V, st, u[row], sm, &q) : -1;
     if (threadIdx.x == 0) {
@@ -727,7 +785,7 @@ __global__ void __launch_bounds__(kTpThreads, 2) verify_rows_kernel(const T* __r
   const int rows = rows_t + (a.stream_draft ? a.B * K : 0);
   if (static_cast<int>(blockIdx.x) < warp_ctas) {
     const int g = blockIdx.x * kTpWarps + (threadIdx.x >> 5);
-    if (g < rows && !request_cut(a.temperature, a.top_p, g < rows_t ? g / (K + 1) : (g - rows_t) / K))
+    if (g < rows && !request_cut(a.temperature, a.top_p, a.top_k, g < rows_t ? g / (K + 1) : (g - rows_t) / K, V))
       warp_verify_row(tgt, drf, g, a);
     return;
   }
@@ -739,10 +797,10 @@ __global__ void __launch_bounds__(kTpThreads, 2) verify_rows_kernel(const T* __r
     const bool is_draft = g >= rows_t;
     const int row = is_draft ? g - rows_t : g;
     const int b = is_draft ? row / K : row / (K + 1);
-    if (!request_cut(a.temperature, a.top_p, b)) continue;
+    if (!request_cut(a.temperature, a.top_p, a.top_k, b, V)) continue;
     const T* rp = (is_draft ? drf : tgt) + static_cast<size_t>(row) * V;
     const Partial* pp = (is_draft ? a.parts_d : a.parts_t) + static_cast<size_t>(row) * nchunks_for(V);
-    const RowStat st = tp_row_stats_partials(rp, V, a.temperature[b], a.top_p[b], pp, sm);
+    const RowStat st = tp_row_stats_partials(rp, V, a.temperature[b], a.top_p[b], request_k(a.top_k, b, V), pp, sm);
     if (threadIdx.x == 0) (is_draft ? a.stats_d : a.stats_t)[row] = st;
     if (block_arrive_last(&a.cnt[b], per_req, &sm.flag) && threadIdx.x < 32)
       warp_decide_request<T>(b, tgt, drf, K, V, a.tokens, a.stats_t, a.stream_draft ? a.stats_d : a.dstats_in,

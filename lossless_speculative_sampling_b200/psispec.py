@@ -50,11 +50,14 @@ def lib():
         L.psispec_sample_draft.argtypes = [P, ctypes.c_int, I32, I32, I32, P, P, P, P, P, P, P, SZ, P]
         L.psispec_row_stats.argtypes = [P, ctypes.c_int, I32, I32, I32, P, P, P, P, SZ, P]
         L.psispec_verify_linear.argtypes = [P, P, ctypes.c_int, I32, I32, I32, P, P, P, P, P, P, P, P, P, P, P, SZ, P]
+        L.psispec_sample_draft_k.argtypes = [P, ctypes.c_int, I32, I32, I32, P, P, P, P, P, P, P, P, SZ, P]
+        L.psispec_verify_linear_k.argtypes = [P, P, ctypes.c_int, I32, I32, I32, P, P, P, P, P, P, P, P, P, P, P, P, SZ,
+                                              P]
         L.psispec_verify_tree.argtypes = [P, P, ctypes.c_int, I32, I32, I32, P, P, P, P, P, P, P, I32, P, P, P, P, SZ,
                                           P]
         L.psispec_verify_linear_static.argtypes = [P, P, ctypes.c_int, I32, I32, I32, P, P, P, P, P, P, P, P, P, P, P]
-        for f in ("psispec_sample_draft", "psispec_row_stats", "psispec_verify_linear", "psispec_verify_tree",
-                  "psispec_verify_linear_static"):
+        for f in ("psispec_sample_draft", "psispec_sample_draft_k", "psispec_row_stats", "psispec_verify_linear",
+                  "psispec_verify_linear_k", "psispec_verify_tree", "psispec_verify_linear_static"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -126,18 +129,22 @@ def _check(status: int, what: str):
         raise PsispecError(status, what)
 
 
-def sample_draft(draft, temperature, top_p, u, *, out_tokens=None, out_q=None, row_stats=None, ws=None, stream=None):
-    """Draw one token per drafted position from q = softmax(draft / T) after top-p.
+def sample_draft(draft, temperature, top_p, u, *, top_k=None, out_tokens=None, out_q=None, row_stats=None, ws=None,
+                 stream=None):
+    """Draw one token per drafted position from q = softmax(draft / T) after top-k and top-p.
 
-    draft [B, K, V] bf16/fp32; temperature, top_p [B] fp32; u [B, K] fp32 in [0, 1).
+    draft [B, K, V] bf16/fp32; temperature, top_p [B] fp32; u [B, K] fp32 in [0, 1); top_k
+    [B] int32 or None (off; k <= 0 or k >= V is off too).
     Returns (tokens [B, K] int32, q(token) [B, K] fp32, row_stats [B, K, 32] uint8), the last
-    reusable by verify_linear(draft_row_stats=...)."""
+    reusable by verify_linear(draft_row_stats=...) with the same top_k."""
     B, K, V = draft.shape
     dev = draft.device
     _req(draft, "draft")
     _req(temperature, "temperature", torch.float32, B, dev)
     _req(top_p, "top_p", torch.float32, B, dev)
     _req(u, "u", torch.float32, B * K, dev)
+    if top_k is not None:
+        _req(top_k, "top_k", torch.int32, B, dev)
     out_tokens = torch.empty((B, K), dtype=torch.int32, device=dev) if out_tokens is None else out_tokens
     out_q = torch.empty((B, K), dtype=torch.float32, device=dev) if out_q is None else out_q
     row_stats = torch.empty((B, K, ROW_STATS_BYTES), dtype=torch.uint8, device=dev) if row_stats is None else row_stats
@@ -146,8 +153,14 @@ def sample_draft(draft, temperature, top_p, u, *, out_tokens=None, out_q=None, r
     _req(row_stats, "row_stats", torch.uint8, B * K * ROW_STATS_BYTES, dev)
     need = workspace_size(OP_SAMPLE_DRAFT, B, K, V)
     ws = workspace(need, dev) if ws is None else ws
-    st = lib().psispec_sample_draft(_p(draft), _dtype(draft), B, K, V, _p(temperature), _p(top_p), _p(u),
-                                    _p(out_tokens), _p(out_q), _p(row_stats), _p(ws), ws.numel(), _stream(dev, stream))
+    if top_k is None:
+        st = lib().psispec_sample_draft(_p(draft), _dtype(draft), B, K, V, _p(temperature), _p(top_p), _p(u),
+                                        _p(out_tokens), _p(out_q), _p(row_stats), _p(ws), ws.numel(),
+                                        _stream(dev, stream))
+    else:
+        st = lib().psispec_sample_draft_k(_p(draft), _dtype(draft), B, K, V, _p(temperature), _p(top_p), _p(top_k),
+                                          _p(u), _p(out_tokens), _p(out_q), _p(row_stats), _p(ws), ws.numel(),
+                                          _stream(dev, stream))
     _check(st, "psispec_sample_draft")
     return out_tokens, out_q, row_stats
 
@@ -172,10 +185,12 @@ def row_stats(logits, temperature, top_p, *, out=None, ws=None, stream=None):
     return out
 
 
-def verify_linear(target, draft, draft_tokens, u_accept, u_resid, temperature, top_p, *, draft_row_stats=None,
-                  out_tokens=None, out_accept_len=None, out_p=None, out_q=None, want_pq=True, ws=None, stream=None):
+def verify_linear(target, draft, draft_tokens, u_accept, u_resid, temperature, top_p, *, top_k=None,
+                  draft_row_stats=None, out_tokens=None, out_accept_len=None, out_p=None, out_q=None, want_pq=True,
+                  ws=None, stream=None):
     """Psi-Spec linear verification. target [B, K+1, V], draft [B, K, V] (same dtype),
-    draft_tokens [B, K] int32, u_accept [B, K], u_resid [B, K+1], temperature/top_p [B].
+    draft_tokens [B, K] int32, u_accept [B, K], u_resid [B, K+1], temperature/top_p [B],
+    top_k [B] int32 or None (off).
     Returns dict(tokens [B, K+1], accept_len [B], p [B, K], q [B, K]) (p/q None if not wanted)."""
     B, K1, V = target.shape
     K = K1 - 1
@@ -187,6 +202,8 @@ def verify_linear(target, draft, draft_tokens, u_accept, u_resid, temperature, t
     _req(u_resid, "u_resid", torch.float32, B * (K + 1), dev)
     _req(temperature, "temperature", torch.float32, B, dev)
     _req(top_p, "top_p", torch.float32, B, dev)
+    if top_k is not None:
+        _req(top_k, "top_k", torch.int32, B, dev)
     if draft_row_stats is not None:
         _req(draft_row_stats, "draft_row_stats", torch.uint8, B * K * ROW_STATS_BYTES, dev)
     out_tokens = torch.empty((B, K + 1), dtype=torch.int32, device=dev) if out_tokens is None else out_tokens
@@ -196,10 +213,16 @@ def verify_linear(target, draft, draft_tokens, u_accept, u_resid, temperature, t
         out_q = torch.empty((B, K), dtype=torch.float32, device=dev) if out_q is None else out_q
     need = workspace_size(OP_VERIFY_LINEAR, B, K, V)
     ws = workspace(need, dev) if ws is None else ws
-    st = lib().psispec_verify_linear(_p(target), _p(draft), _dtype(target), B, K, V, _p(draft_tokens),
-                                     _p(draft_row_stats), _p(u_accept), _p(u_resid), _p(temperature), _p(top_p),
-                                     _p(out_tokens), _p(out_accept_len), _p(out_p), _p(out_q), _p(ws), ws.numel(),
-                                     _stream(dev, stream))
+    if top_k is None:
+        st = lib().psispec_verify_linear(_p(target), _p(draft), _dtype(target), B, K, V, _p(draft_tokens),
+                                         _p(draft_row_stats), _p(u_accept), _p(u_resid), _p(temperature), _p(top_p),
+                                         _p(out_tokens), _p(out_accept_len), _p(out_p), _p(out_q), _p(ws), ws.numel(),
+                                         _stream(dev, stream))
+    else:
+        st = lib().psispec_verify_linear_k(_p(target), _p(draft), _dtype(target), B, K, V, _p(draft_tokens),
+                                           _p(draft_row_stats), _p(u_accept), _p(u_resid), _p(temperature),
+                                           _p(top_p), _p(top_k), _p(out_tokens), _p(out_accept_len), _p(out_p),
+                                           _p(out_q), _p(ws), ws.numel(), _stream(dev, stream))
     _check(st, "psispec_verify_linear")
     return {"tokens": out_tokens, "accept_len": out_accept_len, "p": out_p, "q": out_q}
 

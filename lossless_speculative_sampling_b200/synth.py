@@ -45,6 +45,7 @@ class LinearCase:
     zipf_bias: float = 0.0  # amplitude of the rank bias; 0 disables it
     zipf_exponent: float = 1.1
     seed: int = 0
+    top_k: int = 0  # per-request top-k of every request (0: off)
 
 
 @dataclass
@@ -70,6 +71,8 @@ def linear_cases():
         "tiny": LinearCase("tiny", 1, 4, 1024, torch.float32, 2.0, 0.5, 1.0, 1.0, seed=0),
         "mid": LinearCase("mid", 64, 8, V_QWEN, bf, 3.0, 1.0, 1.0, 1.0, zipf_bias=8.0, seed=1001),
         "max": LinearCase("max", 512, 16, V_QWEN, bf, 2.0, (0.25, 2.0), 1.0, 0.95, seed=1002),
+        # the default workload's sizes and logits under top-k 50 and top-p 0.95
+        "mid_topk": LinearCase("mid_topk", 64, 8, V_QWEN, bf, 3.0, 1.0, 1.0, 0.95, zipf_bias=8.0, seed=1001, top_k=50),
     }
     for B in (1, 32, 256):
         for T in (0.0, 0.7, 1.0):

@@ -102,6 +102,31 @@ def test_verify_linear_host_checks(L):
     assert _linear(L, wsb=0) == psispec.ERR_WORKSPACE
 
 
+def test_topk_entries_host_checks(L):
+    """The top-k entry points validate like the plain ones (the top-k array itself may be null)."""
+    def sample_k(**kw):
+        a = dict(d=FAKE, B=2, K=3, V=100, u=FAKE, ws=FAKE, wsb=1 << 30)
+        a.update(kw)
+        return L.psispec_sample_draft_k(a["d"], psispec.BF16, a["B"], a["K"], a["V"], FAKE, FAKE, FAKE, a["u"], FAKE,
+                                        None, None, a["ws"], a["wsb"], None)
+
+    def linear_k(**kw):
+        a = dict(t=FAKE, K=4, V=64, ws=FAKE, wsb=1 << 30)
+        a.update(kw)
+        return L.psispec_verify_linear_k(a["t"], FAKE, psispec.F32, 2, a["K"], a["V"], FAKE, None, FAKE, FAKE, FAKE,
+                                         FAKE, None, FAKE, FAKE, None, None, a["ws"], a["wsb"], None)
+
+    assert sample_k(d=None) == psispec.ERR_INVALID_ARG
+    assert sample_k(u=None) == psispec.ERR_INVALID_ARG
+    assert sample_k(B=0) == psispec.ERR_INVALID_ARG
+    assert sample_k(V=(1 << 24) + 1) == psispec.ERR_UNSUPPORTED
+    assert sample_k(wsb=16) == psispec.ERR_WORKSPACE
+    assert linear_k(t=None) == psispec.ERR_INVALID_ARG
+    assert linear_k(K=65) == psispec.ERR_UNSUPPORTED
+    assert linear_k(t=ctypes.c_void_p(4098)) == psispec.ERR_INVALID_ARG
+    assert linear_k(ws=None) == psispec.ERR_WORKSPACE
+
+
 def _tree(L, **kw):
     a = dict(t=FAKE, d=FAKE, dtype=psispec.BF16, B=2, N=10, V=64, off=FAKE, par=FAKE, tok=FAKE, ua=FAKE, ur=FAKE,
              T=FAKE, P=FAKE, md=4, op=FAKE, ot=FAKE, ol=FAKE, ws=FAKE, wsb=1 << 30)

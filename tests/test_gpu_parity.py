@@ -210,6 +210,84 @@ def test_topp_fallback_paths(V, T, top_p):
     compare_linear(out, ora)
 
 
+TOPK_GRID = [
+    # B, K, V, dtype, T, top_p, top_k
+    (3, 4, 40000, torch.bfloat16, 1.0, 1.0, 50),       # value window, top-k alone
+    (3, 4, 50001, torch.bfloat16, 0.7, 0.9, 200),      # value window, top-k then top-p
+    (3, 4, 40000, torch.bfloat16, 1.0, 0.95, 30000),   # k-th value below the window: radix select
+    (3, 4, 40000, torch.float32, 1.3, 0.8, 1000),      # fp32: radix select, count then mass
+    (2, 3, 40000, torch.float32, 1.0, 1.0, 1),         # k = 1 (the maximum and its ties)
+    (4, 3, 7, torch.float32, 1.0, 0.9, 3),
+    (1, 2, 151936, torch.bfloat16, 1.0, 0.95, 20),
+]
+
+
+@pytest.mark.parametrize("use_stats", [False, True])
+@pytest.mark.parametrize("B,K,V,dtype,T,top_p,top_k", TOPK_GRID)
+def test_topk_parity(B, K, V, dtype, T, top_p, top_k, use_stats):
+    """Top-k (then top-p) in sampling and in verification against the oracle's reading: the
+    value-window select (bf16), the general radix select (fp32, or a k-th value below the
+    window), ties at the k-th value (bf16 rows hold many equal values), and the sampler's
+    records reused by verification."""
+    tgt, drf, ud, ua, ur, Ts, Ps = _linear_inputs(B, K, V, dtype, T, top_p, 0.6, seed=V + top_k)
+    Ks = torch.full((B,), top_k, dtype=torch.int32)
+    tok, q, rec = psispec.sample_draft(_cuda(drf), _cuda(Ts), _cuda(Ps), _cuda(ud), top_k=_cuda(Ks))
+    o_s = oracle.sample_draft(drf.reshape(B * K, V), Ts.numpy(), Ps.numpy(), ud.reshape(-1),
+                              row_req=np.arange(B * K) // K, top_k=Ks.numpy())
+    compare_sample(tok, q, o_s)
+    x = o_s["tokens"].reshape(B, K).astype(np.int32)
+    out = psispec.verify_linear(_cuda(tgt), _cuda(drf), _cuda(x), _cuda(ua), _cuda(ur), _cuda(Ts), _cuda(Ps),
+                                top_k=_cuda(Ks), draft_row_stats=rec if use_stats else None)
+    ora = oracle.verify_linear(tgt, drf, x, ua, ur, Ts.numpy(), Ps.numpy(), top_k=Ks.numpy())
+    compare_linear(out, ora)
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_topk_mixed_requests(dtype):
+    """Per-request top-k, off by k <= 0 and k >= V, beside greedy rows, top-p alone and both."""
+    B, K, V = 8, 4, 20011
+    tgt, drf, ud, ua, ur, _, _ = _linear_inputs(B, K, V, dtype, 1.0, 1.0, 0.7, seed=91, neg_inf_frac=0.1)
+    Ts = torch.tensor([1.0, 0.0, 0.8, 1.0, 1.5, 1.0, 0.7, 1.0])
+    Ps = torch.tensor([1.0, 1.0, 0.9, 0.5, 1.0, 1.0, 0.95, 0.9])
+    Ks = torch.tensor([0, 5, 100, 7, V, V - 1, -3, 2500], dtype=torch.int32)
+    tok, q, _ = psispec.sample_draft(_cuda(drf), _cuda(Ts), _cuda(Ps), _cuda(ud), top_k=_cuda(Ks))
+    o_s = oracle.sample_draft(drf.reshape(B * K, V), Ts.numpy(), Ps.numpy(), ud.reshape(-1),
+                              row_req=np.arange(B * K) // K, top_k=Ks.numpy())
+    compare_sample(tok, q, o_s)
+    x = o_s["tokens"].reshape(B, K).astype(np.int32)
+    out = psispec.verify_linear(_cuda(tgt), _cuda(drf), _cuda(x), _cuda(ua), _cuda(ur), _cuda(Ts), _cuda(Ps),
+                                top_k=_cuda(Ks))
+    ora = oracle.verify_linear(tgt, drf, x, ua, ur, Ts.numpy(), Ps.numpy(), top_k=Ks.numpy())
+    compare_linear(out, ora)
+    # a null top-k array and an all-off one agree with the entry points without top-k
+    off = torch.zeros(B, dtype=torch.int32)
+    a = psispec.verify_linear(_cuda(tgt), _cuda(drf), _cuda(x), _cuda(ua), _cuda(ur), _cuda(Ts), _cuda(Ps),
+                              top_k=_cuda(off))
+    b = psispec.verify_linear(_cuda(tgt), _cuda(drf), _cuda(x), _cuda(ua), _cuda(ur), _cuda(Ts), _cuda(Ps))
+    assert torch.equal(a["tokens"], b["tokens"]) and torch.equal(a["accept_len"], b["accept_len"])
+    assert torch.equal(a["p"], b["p"]) and torch.equal(a["q"], b["q"])
+
+
+@pytest.mark.parametrize("top_p,top_k", [(0.9, 0), (1.0, 100), (0.8, 500)])
+def test_negative_logit_rows(top_p, top_k):
+    """bf16 rows of log-probabilities (every logit negative): the top-p/top-k value window then
+    lies among negative values, whose weights come from the inverse of their 16-bit order keys."""
+    B, K, V = 3, 4, 40000
+    tgt, drf, ud, ua, ur, Ts, Ps = _linear_inputs(B, K, V, torch.float32, 1.0, top_p, 0.6, seed=404 + top_k)
+    tgt = torch.log_softmax(tgt, dim=-1).to(torch.bfloat16)
+    drf = torch.log_softmax(drf, dim=-1).to(torch.bfloat16)
+    Ks = torch.full((B,), top_k, dtype=torch.int32)
+    tok, q, _ = psispec.sample_draft(_cuda(drf), _cuda(Ts), _cuda(Ps), _cuda(ud), top_k=_cuda(Ks))
+    o_s = oracle.sample_draft(drf.reshape(B * K, V), Ts.numpy(), Ps.numpy(), ud.reshape(-1),
+                              row_req=np.arange(B * K) // K, top_k=Ks.numpy())
+    compare_sample(tok, q, o_s)
+    x = o_s["tokens"].reshape(B, K).astype(np.int32)
+    out = psispec.verify_linear(_cuda(tgt), _cuda(drf), _cuda(x), _cuda(ua), _cuda(ur), _cuda(Ts), _cuda(Ps),
+                                top_k=_cuda(Ks))
+    ora = oracle.verify_linear(tgt, drf, x, ua, ur, Ts.numpy(), Ps.numpy(), top_k=Ks.numpy())
+    compare_linear(out, ora)
+
+
 def test_q_equals_p_accepts_all_on_gpu():
     B, K, V = 16, 8, 30000
     g = torch.Generator().manual_seed(5)
@@ -365,26 +443,30 @@ def _sampled(B, n):
     return np.unique(np.linspace(0, B - 1, n).astype(int))
 
 
-@pytest.mark.parametrize("name", ["mid", "max", "sweep_b32_t0", "sweep_b32_t0.7", "sweep_b1_t1"])
+@pytest.mark.parametrize("name", ["mid", "max", "sweep_b32_t0", "sweep_b32_t0.7", "sweep_b1_t1", "mid_topk"])
 def test_full_size_linear_sampled(name):
     case = synth.linear_cases()[name]
     B, K, V = case.B, case.K, case.V
     tgt, drf = synth.linear_logits(case, device=DEV)
     ud, ua, ur = synth.linear_uniforms(case)
     Ts, Ps = torch.full((B,), case.temperature), torch.full((B,), case.top_p)
-    x, q, stats = psispec.sample_draft(drf, _cuda(Ts), _cuda(Ps), _cuda(ud))
+    Ks = torch.full((B,), case.top_k, dtype=torch.int32) if case.top_k else None
+    Kd = _cuda(Ks) if case.top_k else None
+    x, q, stats = psispec.sample_draft(drf, _cuda(Ts), _cuda(Ps), _cuda(ud), top_k=Kd)
     pick = _sampled(B, 4 if B >= 256 else 6)
     idx = torch.as_tensor(pick, device=DEV)
     d_host = drf[idx].cpu()
+    Kp = Ks[pick].numpy() if case.top_k else None
     o_s = oracle.sample_draft(d_host.reshape(-1, V), Ts[pick].numpy(), Ps[pick].numpy(), ud[pick].reshape(-1),
-                              row_req=np.arange(len(pick) * K) // K)
+                              row_req=np.arange(len(pick) * K) // K, top_k=Kp)
     compare_sample(x[idx], q[idx], o_s)
     # the oracle's draft tokens replace the sampled requests' rows
     x_in = x.clone()
     x_in[idx] = torch.from_numpy(o_s["tokens"].reshape(len(pick), K)).to(DEV)
-    out = psispec.verify_linear(tgt, drf, x_in, _cuda(ua), _cuda(ur), _cuda(Ts), _cuda(Ps), draft_row_stats=stats)
+    out = psispec.verify_linear(tgt, drf, x_in, _cuda(ua), _cuda(ur), _cuda(Ts), _cuda(Ps), top_k=Kd,
+                                draft_row_stats=stats)
     ora = oracle.verify_linear(tgt[idx].cpu(), d_host, o_s["tokens"].reshape(len(pick), K), ua[pick], ur[pick],
-                               Ts[pick].numpy(), Ps[pick].numpy())
+                               Ts[pick].numpy(), Ps[pick].numpy(), top_k=Kp)
     sub = {k: v[idx] for k, v in out.items()}
     stats_report = compare_linear(sub, ora)
     lens = out["accept_len"].cpu().numpy()
