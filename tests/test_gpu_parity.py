@@ -242,52 +242,6 @@ def test_topk_parity(B, K, V, dtype, T, top_p, top_k, use_stats):
     compare_linear(out, ora)
 
 
-@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
-def test_topk_mixed_requests(dtype):
-    """Per-request top-k, off by k <= 0 and k >= V, beside greedy rows, top-p alone and both."""
-    B, K, V = 8, 4, 20011
-    tgt, drf, ud, ua, ur, _, _ = _linear_inputs(B, K, V, dtype, 1.0, 1.0, 0.7, seed=91, neg_inf_frac=0.1)
-    Ts = torch.tensor([1.0, 0.0, 0.8, 1.0, 1.5, 1.0, 0.7, 1.0])
-    Ps = torch.tensor([1.0, 1.0, 0.9, 0.5, 1.0, 1.0, 0.95, 0.9])
-    Ks = torch.tensor([0, 5, 100, 7, V, V - 1, -3, 2500], dtype=torch.int32)
-    tok, q, _ = psispec.sample_draft(_cuda(drf), _cuda(Ts), _cuda(Ps), _cuda(ud), top_k=_cuda(Ks))
-    o_s = oracle.sample_draft(drf.reshape(B * K, V), Ts.numpy(), Ps.numpy(), ud.reshape(-1),
-                              row_req=np.arange(B * K) // K, top_k=Ks.numpy())
-    compare_sample(tok, q, o_s)
-    x = o_s["tokens"].reshape(B, K).astype(np.int32)
-    out = psispec.verify_linear(_cuda(tgt), _cuda(drf), _cuda(x), _cuda(ua), _cuda(ur), _cuda(Ts), _cuda(Ps),
-                                top_k=_cuda(Ks))
-    ora = oracle.verify_linear(tgt, drf, x, ua, ur, Ts.numpy(), Ps.numpy(), top_k=Ks.numpy())
-    compare_linear(out, ora)
-    # a null top-k array and an all-off one agree with the entry points without top-k
-    off = torch.zeros(B, dtype=torch.int32)
-    a = psispec.verify_linear(_cuda(tgt), _cuda(drf), _cuda(x), _cuda(ua), _cuda(ur), _cuda(Ts), _cuda(Ps),
-                              top_k=_cuda(off))
-    b = psispec.verify_linear(_cuda(tgt), _cuda(drf), _cuda(x), _cuda(ua), _cuda(ur), _cuda(Ts), _cuda(Ps))
-    assert torch.equal(a["tokens"], b["tokens"]) and torch.equal(a["accept_len"], b["accept_len"])
-    assert torch.equal(a["p"], b["p"]) and torch.equal(a["q"], b["q"])
-
-
-@pytest.mark.parametrize("top_p,top_k", [(0.9, 0), (1.0, 100), (0.8, 500)])
-def test_negative_logit_rows(top_p, top_k):
-    """bf16 rows of log-probabilities (every logit negative): the top-p/top-k value window then
-    lies among negative values, whose weights come from the inverse of their 16-bit order keys."""
-    B, K, V = 3, 4, 40000
-    tgt, drf, ud, ua, ur, Ts, Ps = _linear_inputs(B, K, V, torch.float32, 1.0, top_p, 0.6, seed=404 + top_k)
-    tgt = torch.log_softmax(tgt, dim=-1).to(torch.bfloat16)
-    drf = torch.log_softmax(drf, dim=-1).to(torch.bfloat16)
-    Ks = torch.full((B,), top_k, dtype=torch.int32)
-    tok, q, _ = psispec.sample_draft(_cuda(drf), _cuda(Ts), _cuda(Ps), _cuda(ud), top_k=_cuda(Ks))
-    o_s = oracle.sample_draft(drf.reshape(B * K, V), Ts.numpy(), Ps.numpy(), ud.reshape(-1),
-                              row_req=np.arange(B * K) // K, top_k=Ks.numpy())
-    compare_sample(tok, q, o_s)
-    x = o_s["tokens"].reshape(B, K).astype(np.int32)
-    out = psispec.verify_linear(_cuda(tgt), _cuda(drf), _cuda(x), _cuda(ua), _cuda(ur), _cuda(Ts), _cuda(Ps),
-                                top_k=_cuda(Ks))
-    ora = oracle.verify_linear(tgt, drf, x, ua, ur, Ts.numpy(), Ps.numpy(), top_k=Ks.numpy())
-    compare_linear(out, ora)
-
-
 def test_q_equals_p_accepts_all_on_gpu():
     B, K, V = 16, 8, 30000
     g = torch.Generator().manual_seed(5)
@@ -484,3 +438,52 @@ def test_full_size_tree():
     ora = oracle.verify_tree(tgt.cpu(), drf.cpu(), trie.node_offsets.numpy(), trie.parent.numpy(), toks.numpy(), ua, ur,
                              Ts.numpy(), Ps.numpy(), case.max_depth)
     print("tree", compare_tree(out, ora), "accept", out["accept_len"].tolist())
+
+
+# ------------------------------------------------------------------ top-k: mixed requests and negative rows
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_topk_mixed_requests(dtype):
+    """Per-request top-k, off by k <= 0 and k >= V, beside greedy rows, top-p alone and both."""
+    B, K, V = 8, 4, 20011
+    tgt, drf, ud, ua, ur, _, _ = _linear_inputs(B, K, V, dtype, 1.0, 1.0, 0.7, seed=91, neg_inf_frac=0.1)
+    Ts = torch.tensor([1.0, 0.0, 0.8, 1.0, 1.5, 1.0, 0.7, 1.0])
+    Ps = torch.tensor([1.0, 1.0, 0.9, 0.5, 1.0, 1.0, 0.95, 0.9])
+    Ks = torch.tensor([0, 5, 100, 7, V, V - 1, -3, 2500], dtype=torch.int32)
+    tok, q, _ = psispec.sample_draft(_cuda(drf), _cuda(Ts), _cuda(Ps), _cuda(ud), top_k=_cuda(Ks))
+    o_s = oracle.sample_draft(drf.reshape(B * K, V), Ts.numpy(), Ps.numpy(), ud.reshape(-1),
+                              row_req=np.arange(B * K) // K, top_k=Ks.numpy())
+    compare_sample(tok, q, o_s)
+    x = o_s["tokens"].reshape(B, K).astype(np.int32)
+    out = psispec.verify_linear(_cuda(tgt), _cuda(drf), _cuda(x), _cuda(ua), _cuda(ur), _cuda(Ts), _cuda(Ps),
+                                top_k=_cuda(Ks))
+    ora = oracle.verify_linear(tgt, drf, x, ua, ur, Ts.numpy(), Ps.numpy(), top_k=Ks.numpy())
+    compare_linear(out, ora)
+    # a null top-k array and an all-off one agree with the entry points without top-k
+    off = torch.zeros(B, dtype=torch.int32)
+    a = psispec.verify_linear(_cuda(tgt), _cuda(drf), _cuda(x), _cuda(ua), _cuda(ur), _cuda(Ts), _cuda(Ps),
+                              top_k=_cuda(off))
+    b = psispec.verify_linear(_cuda(tgt), _cuda(drf), _cuda(x), _cuda(ua), _cuda(ur), _cuda(Ts), _cuda(Ps))
+    assert torch.equal(a["tokens"], b["tokens"]) and torch.equal(a["accept_len"], b["accept_len"])
+    assert torch.equal(a["p"], b["p"]) and torch.equal(a["q"], b["q"])
+
+
+@pytest.mark.parametrize("top_p,top_k", [(0.9, 0), (1.0, 100), (0.8, 500)])
+def test_negative_logit_rows(top_p, top_k):
+    """bf16 rows of log-probabilities (every logit negative): the top-p/top-k value window then
+    lies among negative values, whose weights come from the inverse of their 16-bit order keys."""
+    B, K, V = 3, 4, 40000
+    tgt, drf, ud, ua, ur, Ts, Ps = _linear_inputs(B, K, V, torch.float32, 1.0, top_p, 0.6, seed=404 + top_k)
+    tgt = torch.log_softmax(tgt, dim=-1).to(torch.bfloat16)
+    drf = torch.log_softmax(drf, dim=-1).to(torch.bfloat16)
+    Ks = torch.full((B,), top_k, dtype=torch.int32)
+    tok, q, _ = psispec.sample_draft(_cuda(drf), _cuda(Ts), _cuda(Ps), _cuda(ud), top_k=_cuda(Ks))
+    o_s = oracle.sample_draft(drf.reshape(B * K, V), Ts.numpy(), Ps.numpy(), ud.reshape(-1),
+                              row_req=np.arange(B * K) // K, top_k=Ks.numpy())
+    compare_sample(tok, q, o_s)
+    x = o_s["tokens"].reshape(B, K).astype(np.int32)
+    out = psispec.verify_linear(_cuda(tgt), _cuda(drf), _cuda(x), _cuda(ua), _cuda(ur), _cuda(Ts), _cuda(Ps),
+                                top_k=_cuda(Ks))
+    ora = oracle.verify_linear(tgt, drf, x, ua, ur, Ts.numpy(), Ps.numpy(), top_k=Ks.numpy())
+    compare_linear(out, ora)
