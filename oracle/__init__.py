@@ -15,7 +15,8 @@ Pins (see tests/test_oracle_*.py): closed forms on hand-made rows, q == p accept
 position, disjoint one-hot drafts reject at position 0, temperature 0 is exact argmax
 matching, exhaustive uniform grids reproduce the exact rejection-sampling law, and
 Monte-Carlo chi-squared tests show the emitted tokens follow the verifier's law (linear and
-tree).
+tree, under each tree rule); the candidate trie equals a full enumeration of the candidate
+prefixes.
 """
 from __future__ import annotations
 
@@ -31,6 +32,9 @@ _LIB_PATH = os.path.join(_HERE, "libpsispec_oracle.so")
 _lib = None
 
 E_BAND = 1e-6  # decisions whose margin is below this may differ between correct implementations
+
+# candidate rules of tree verification (psispec_oracle.h)
+TREE_SAMPLED_WOR, TREE_DETERMINISTIC, TREE_SAMPLED_WR = 0, 1, 2
 
 
 def build(force: bool = False) -> str:
@@ -57,6 +61,10 @@ def _load():
                                              I, I, D, D, D, D]
         lib.oracle_verify_tree.argtypes = [D, D, ctypes.c_int, ctypes.c_int, I, I, I, D, D, D, D, I,
                                            ctypes.c_int, I, I, I, D]
+        lib.oracle_verify_tree_rule.argtypes = [D, D, ctypes.c_int, ctypes.c_int, I, I, I, D, D, D, D, I,
+                                                ctypes.c_int, ctypes.c_int, I, I, I, D]
+        lib.oracle_build_tree.argtypes = [D, ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_double,
+                                          ctypes.c_int, ctypes.c_int, ctypes.c_int, I, I, I, D, I]
         _lib = lib
     return _lib
 
@@ -153,9 +161,10 @@ def verify_linear(target, draft, draft_tokens, u_accept, u_resid, temperature, t
 
 
 def verify_tree(target, draft, node_offsets, parent, tokens, u_accept, u_resid, temperature, top_p,
-                max_depth: int, top_k=None):
+                max_depth: int, top_k=None, rule: int = TREE_SAMPLED_WOR):
     """target/draft [N, V]; node_offsets [B+1]; parent/tokens/u_accept/u_resid [N] (parent is
-    the request-local index, -1 at the root). Returns dict(path [B, max_depth],
+    the request-local index, -1 at the root); rule: how the children were produced
+    (TREE_SAMPLED_WOR, TREE_DETERMINISTIC, TREE_SAMPLED_WR). Returns dict(path [B, max_depth],
     tokens [B, max_depth+1], accept_len [B], band [B])."""
     t = _as_f64(target)
     N, V = t.shape
@@ -175,6 +184,36 @@ def verify_tree(target, draft, node_offsets, parent, tokens, u_accept, u_resid, 
     ln, lnp = _i32(np.zeros(B))
     band, bp = _f64(np.zeros(B))
     Kk, Kkp = _top_k(top_k, B)
-    _load().oracle_verify_tree(tp, dp, B, V, offp, parp, tkp, uap, urp, Tp, Pp, Kkp, int(max_depth), pathp,
-                               otkp, lnp, bp)
+    if rule == TREE_SAMPLED_WOR:
+        rc = _load().oracle_verify_tree(tp, dp, B, V, offp, parp, tkp, uap, urp, Tp, Pp, Kkp, int(max_depth), pathp,
+                                        otkp, lnp, bp)
+    else:
+        rc = _load().oracle_verify_tree_rule(tp, dp, B, V, offp, parp, tkp, uap, urp, Tp, Pp, Kkp, int(max_depth),
+                                             int(rule), pathp, otkp, lnp, bp)
+    if rc != 0:
+        raise ValueError("oracle_verify_tree: bad arguments (rule %r)" % (rule,))
     return {"path": path, "tokens": otk, "accept_len": ln, "band": band}
+
+
+def build_tree(draft_rows, temperature: float, top_p: float, cand_k: int, n_prefixes: int, top_k: int = 0):
+    """Candidate trie from the draft rows of K positions ([K, V] logits): the cand_k most probable
+    tokens per position, then the n_prefixes most probable prefixes. Returns dict(parent,
+    tokens, depth, score) over the trie's nodes (node 0 the empty prefix), or None when a
+    draft row is bad."""
+    d = _as_f64(draft_rows)
+    K, V = d.shape
+    d, dp = _f64(d)
+    cap = int(n_prefixes) + 1
+    par, parp = _i32(np.zeros(cap))
+    tok, tokp = _i32(np.zeros(cap))
+    dep, depp = _i32(np.zeros(cap))
+    sc, scp = _f64(np.zeros(cap))
+    nn, nnp = _i32(np.zeros(1))
+    rc = _load().oracle_build_tree(dp, K, V, float(temperature), float(top_p), int(top_k), int(cand_k),
+                                   int(n_prefixes), parp, tokp, depp, scp, nnp)
+    if rc == -1:
+        return None
+    if rc != 0:
+        raise ValueError("oracle_build_tree: bad arguments")
+    n = int(nn[0])
+    return {"parent": par[:n].copy(), "tokens": tok[:n].copy(), "depth": dep[:n].copy(), "score": sc[:n].copy()}

@@ -13,7 +13,10 @@
  * Temperature and top-p are the sampling controls listed by the project's README (inference
  * example, "--temperature --top-p"). Section 3.4 names the tree sampler; its acceptance rule
  * is not printed on the pages, and the reading implemented here is recursive rejection
- * sampling without replacement over the children of a node, in index order.
+ * sampling over the children of a node, in index order, with the proposal the children came
+ * from: drawn from q without replacement (the default), fixed in advance (the candidate trie
+ * of top-k tokens and best prefixes that section 3.4 describes, built by oracle_build_tree),
+ * or drawn from q independently.
  *
  * Readings where the pages are silent (each listed in the design notes):
  *   - top-p keeps every token whose logit is >= tau, where tau is the largest logit value
@@ -237,7 +240,34 @@ int oracle_verify_tree(const double* target, const double* draft, int B, int V,
                        const double* u_accept, const double* u_resid,
                        const double* temperature, const double* top_p, const int* top_k, int max_depth,
                        int* out_path, int* out_tokens, int* accept_len, double* band) {
+  return oracle_verify_tree_rule(target, draft, B, V, node_offsets, parent, tokens, u_accept, u_resid, temperature,
+                                 top_p, top_k, max_depth, ORACLE_TREE_SAMPLED_WOR, out_path, out_tokens, accept_len,
+                                 band);
+}
+
+/* Tree verification under one of three candidate rules, the same walk for each: at the
+ * current node the children are tested in index order with their own uniforms; an accepted
+ * child becomes the current node; when every child is rejected (or the node is a leaf) the
+ * final token is drawn from the node's current residual r with the node's u_resid.
+ *   ORACLE_TREE_SAMPLED_WOR    children drawn from q one after another without replacement:
+ *                              accept t iff u q~(t) < r(t); on rejection r <- norm([r - q~]_+)
+ *                              and q~ <- q~ without t, renormalised (R7);
+ *   ORACLE_TREE_DETERMINISTIC  children fixed in advance (a candidate tree from top-k and best
+ *                              prefixes): each is the point mass delta_t, so the same step with
+ *                              q~ = delta_t reads: accept t iff u < r(t); on rejection
+ *                              r <- [r - delta_t]_+ renormalised, i.e. r without t;
+ *   ORACLE_TREE_SAMPLED_WR     children drawn independently from q (with replacement): accept t
+ *                              iff u q(t) < r(t); on rejection r <- norm([r - q]_+), q unchanged.
+ * Each is recursive rejection sampling with the proposal its children were drawn from, so the
+ * emitted tokens follow the verifier's law whenever the children were produced that way. */
+int oracle_verify_tree_rule(const double* target, const double* draft, int B, int V,
+                            const int* node_offsets, const int* parent, const int* tokens,
+                            const double* u_accept, const double* u_resid,
+                            const double* temperature, const double* top_p, const int* top_k, int max_depth,
+                            int rule, int* out_path, int* out_tokens, int* accept_len, double* band) {
   if (B < 0 || V <= 0 || max_depth < 0) return ORACLE_BAD_ARG;
+  if (rule != ORACLE_TREE_SAMPLED_WOR && rule != ORACLE_TREE_DETERMINISTIC && rule != ORACLE_TREE_SAMPLED_WR)
+    return ORACLE_BAD_ARG;
   double* r = (double*)malloc(sizeof(double) * (size_t)V);
   double* qt = (double*)malloc(sizeof(double) * (size_t)V);
   double* res = (double*)malloc(sizeof(double) * (size_t)V);
@@ -272,7 +302,7 @@ int oracle_verify_tree(const double* target, const double* draft, int B, int V,
       path_band = dmin(path_band, b3);
       int has_child = 0;
       for (int c = cur + 1; c < n; ++c) has_child |= parent[n0 + c] == cur;
-      if (has_child && T > 0.0) {
+      if (has_child && T > 0.0 && rule != ORACLE_TREE_DETERMINISTIC) {
         if (oracle_row_dist_k(draft + (size_t)(n0 + cur) * V, V, T, tp, tk, qt, &b3) != 0) { bad = 1; break; }
         path_band = dmin(path_band, b3);
       }
@@ -282,6 +312,18 @@ int oracle_verify_tree(const double* target, const double* draft, int B, int V,
         int t = tokens[n0 + c];
         if (T == 0.0) { /* greedy: the child carrying the verifier's argmax is accepted */
           if (r[t] > 0.0) next = c;
+          continue;
+        }
+        if (rule == ORACLE_TREE_DETERMINISTIC) {
+          const double ud = u_accept[n0 + c];
+          path_band = dmin(path_band, fabs(ud - r[t]));
+          if (ud < r[t]) { next = c; break; }
+          /* rejected: [r - delta_t]_+ is r without t; renormalise */
+          r[t] = 0.0;
+          double Zr = 0.0;
+          for (int v = 0; v < V; ++v) Zr += r[v];
+          if (Zr > 0.0)
+            for (int v = 0; v < V; ++v) r[v] /= Zr;
           continue;
         }
         double qmass = 0.0;
@@ -298,11 +340,13 @@ int oracle_verify_tree(const double* target, const double* draft, int B, int V,
         }
         if (Z > 0.0)
           for (int v = 0; v < V; ++v) r[v] = res[v] / Z;
-        qt[t] = 0.0;
-        double Zq = 0.0;
-        for (int v = 0; v < V; ++v) Zq += qt[v];
-        if (Zq > 0.0)
-          for (int v = 0; v < V; ++v) qt[v] /= Zq;
+        if (rule == ORACLE_TREE_SAMPLED_WOR) {
+          qt[t] = 0.0;
+          double Zq = 0.0;
+          for (int v = 0; v < V; ++v) Zq += qt[v];
+          if (Zq > 0.0)
+            for (int v = 0; v < V; ++v) qt[v] /= Zq;
+        }
       }
       if (next >= 0) {
         path[len] = next;
@@ -328,5 +372,118 @@ int oracle_verify_tree(const double* target, const double* draft, int B, int V,
   free(r);
   free(qt);
   free(res);
+  return ORACLE_OK;
+}
+
+/* Candidate trie of the tree sampler. Review page, section 3.4 ("Tree Sampler"): at every
+ * position of the block take the top-K tokens, then keep the V most probable prefixes and
+ * verify them together with tree attention; the README's tree example sets the two sizes by
+ * flags (a tree candidate top-k and a tree verify size). Readings where the page is silent:
+ *   - the per-position distributions are the draft's q_i (after the sampling controls, as
+ *     everywhere); a prefix's probability is the product of q_i over its tokens;
+ *   - candidates at position i are the cand_k tokens of largest q_i with q_i > 0 (ties to the
+ *     lower token index); prefixes have length 1..K;
+ *   - "the V most probable prefixes" are taken in decreasing probability, ties to the shorter
+ *     prefix, then to the lexicographically smaller sequence of candidate ranks; a prefix is
+ *     never less probable than its parent, so the kept set is closed under taking prefixes and
+ *     forms a trie.
+ * They are found best-first: the frontier starts with the first position's candidates; the
+ * best frontier prefix is kept and its extensions by the next position's candidates join the
+ * frontier. Kept prefixes become nodes in the order kept (node 0 is the root, the empty
+ * prefix), so parents precede children and siblings are in decreasing probability.
+ * draft[K*V]: the draft rows of positions 0..K-1. Outputs (n_prefixes + 1 entries): parent,
+ * tokens (-1 at the root), depth (number of tokens of the prefix), score (its probability);
+ * *n_nodes = 1 + the number of kept prefixes (fewer than n_prefixes when the candidates run
+ * out). Returns ORACLE_OK, ORACLE_BAD_ARG, or -1 for a bad draft row. */
+int oracle_build_tree(const double* draft, int K, int V, double T, double top_p, int top_k, int cand_k,
+                      int n_prefixes, int* parent, int* tokens, int* depth, double* score, int* n_nodes) {
+  if (K < 0 || V <= 0 || cand_k < 0 || n_prefixes < 0) return ORACLE_BAD_ARG;
+  double* q = (double*)malloc(sizeof(double) * (size_t)(K > 0 ? K : 1) * V);
+  int* cand = (int*)malloc(sizeof(int) * (size_t)(K > 0 ? K : 1) * (cand_k > 0 ? cand_k : 1));
+  int* ncand = (int*)calloc((size_t)(K > 0 ? K : 1), sizeof(int));
+  int rc = ORACLE_OK;
+  for (int i = 0; i < K && rc == ORACLE_OK; ++i) {
+    double b3;
+    double* qi = q + (size_t)i * V;
+    if (oracle_row_dist_k(draft + (size_t)i * V, V, T, top_p, top_k, qi, &b3) != 0) { rc = -1; break; }
+    /* the cand_k most probable tokens, one selection pass each */
+    for (int r = 0; r < cand_k; ++r) {
+      int best = -1;
+      for (int v = 0; v < V; ++v) {
+        if (!(qi[v] > 0.0)) continue;
+        int taken = 0;
+        for (int j = 0; j < r && !taken; ++j) taken = cand[i * cand_k + j] == v;
+        if (taken) continue;
+        if (best < 0 || qi[v] > qi[best]) best = v;
+      }
+      if (best < 0) break;
+      cand[i * cand_k + r] = best;
+      ncand[i] = r + 1;
+    }
+  }
+  if (rc != ORACLE_OK) {
+    free(q);
+    free(cand);
+    free(ncand);
+    return rc;
+  }
+  /* kept prefixes: rank path of every node (its candidate rank at each position) */
+  const int cap = n_prefixes + 1;
+  int* ranks = (int*)calloc((size_t)cap * (K > 0 ? K : 1), sizeof(int));
+  /* frontier entries: (parent node, candidate rank at the parent's depth) */
+  const int fcap = cand_k * cap + 1;
+  int* f_par = (int*)malloc(sizeof(int) * (size_t)fcap);
+  int* f_rank = (int*)malloc(sizeof(int) * (size_t)fcap);
+  int nf = 0;
+  parent[0] = -1;
+  tokens[0] = -1;
+  depth[0] = 0;
+  score[0] = 1.0;
+  int nn = 1;
+  if (K > 0)
+    for (int r = 0; r < ncand[0]; ++r) { f_par[nf] = 0; f_rank[nf] = r; ++nf; }
+  while (nn < cap && nf > 0) {
+    /* the best frontier entry: highest probability, then shorter, then smaller rank path */
+    int bi = 0;
+    for (int e = 1; e < nf; ++e) {
+      const int pa = f_par[e], pb = f_par[bi];
+      const int da = depth[pa], db = depth[pb];
+      const double sa = score[pa] * q[(size_t)da * V + cand[da * cand_k + f_rank[e]]];
+      const double sb = score[pb] * q[(size_t)db * V + cand[db * cand_k + f_rank[bi]]];
+      int better = sa > sb;
+      if (sa == sb && !better) {
+        if (da != db) {
+          better = da < db;
+        } else {
+          int cmp = 0;
+          for (int j = 0; j < da && cmp == 0; ++j)
+            cmp = (ranks[(size_t)pa * K + j] > ranks[(size_t)pb * K + j]) -
+                  (ranks[(size_t)pa * K + j] < ranks[(size_t)pb * K + j]);
+          better = cmp < 0 || (cmp == 0 && f_rank[e] < f_rank[bi]);
+        }
+      }
+      if (better) bi = e;
+    }
+    const int pa = f_par[bi], ra = f_rank[bi], d = depth[pa];
+    f_par[bi] = f_par[nf - 1];
+    f_rank[bi] = f_rank[nf - 1];
+    --nf;
+    parent[nn] = pa;
+    tokens[nn] = cand[d * cand_k + ra];
+    depth[nn] = d + 1;
+    score[nn] = score[pa] * q[(size_t)d * V + tokens[nn]];
+    for (int j = 0; j < d; ++j) ranks[(size_t)nn * K + j] = ranks[(size_t)pa * K + j];
+    ranks[(size_t)nn * K + d] = ra;
+    if (d + 1 < K)
+      for (int r = 0; r < ncand[d + 1]; ++r) { f_par[nf] = nn; f_rank[nf] = r; ++nf; }
+    ++nn;
+  }
+  *n_nodes = nn;
+  free(q);
+  free(cand);
+  free(ncand);
+  free(ranks);
+  free(f_par);
+  free(f_rank);
   return ORACLE_OK;
 }

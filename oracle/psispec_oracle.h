@@ -89,6 +89,32 @@ int oracle_verify_tree(const double* target, const double* draft, int B, int V,
                        const double* temperature, const double* top_p, const int* top_k, int max_depth,
                        int* out_path, int* out_tokens, int* accept_len, double* band);
 
+/* Candidate rules of tree verification (oracle_verify_tree_rule). */
+#define ORACLE_TREE_SAMPLED_WOR 0    /* children drawn from q without replacement (R7) */
+#define ORACLE_TREE_DETERMINISTIC 1  /* children fixed in advance (top-k / best prefixes) */
+#define ORACLE_TREE_SAMPLED_WR 2     /* children drawn from q independently, with replacement */
+
+/* Tree verification under a candidate rule: ORACLE_TREE_SAMPLED_WOR is oracle_verify_tree;
+ * ORACLE_TREE_DETERMINISTIC tests child t with u < r(t) and on rejection removes t from r and
+ * renormalises (the draft rows are not read); ORACLE_TREE_SAMPLED_WR tests u q(t) < r(t) and
+ * on rejection sets r <- norm([r - q]_+) with q unchanged. Same arguments and outputs as
+ * oracle_verify_tree; an unknown rule is ORACLE_BAD_ARG. */
+int oracle_verify_tree_rule(const double* target, const double* draft, int B, int V,
+                            const int* node_offsets, const int* parent, const int* tokens,
+                            const double* u_accept, const double* u_resid,
+                            const double* temperature, const double* top_p, const int* top_k, int max_depth,
+                            int rule, int* out_path, int* out_tokens, int* accept_len, double* band);
+
+/* Candidate trie of the tree sampler from the draft rows of K positions (draft[K*V], after
+ * temperature/top-p/top-k): the cand_k most probable tokens per position, then the n_prefixes
+ * most probable prefixes (product of the q_i; ties to the shorter prefix, then to the smaller
+ * candidate ranks), as a trie whose node 0 is the empty prefix and whose nodes follow in the
+ * order kept. Outputs have room for n_prefixes + 1 nodes: parent (-1 at the root), tokens (-1
+ * at the root), depth, score (prefix probability); *n_nodes receives the node count. Returns
+ * ORACLE_OK, ORACLE_BAD_ARG, or -1 for a bad draft row. */
+int oracle_build_tree(const double* draft, int K, int V, double T, double top_p, int top_k, int cand_k,
+                      int n_prefixes, int* parent, int* tokens, int* depth, double* score, int* n_nodes);
+
 #ifdef __cplusplus
 }
 #endif

@@ -14,6 +14,9 @@ import pytest
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 SRC = os.path.join(ROOT, "oracle", "psispec_oracle.c")
 
+PINS = ("test_oracle_pins.py", "test_oracle_lossless.py")
+TREE_BUILD = ("test_oracle_tree_build.py",)
+
 MUTATIONS = {
     "accept_operands_swapped": ("if (u * q[x] < p[x]) continue;", "if (u * p[x] < q[x]) continue;"),
     "accept_not_strict": ("if (u * q[x] < p[x]) continue;", "if (u * q[x] <= p[x]) continue;"),
@@ -33,12 +36,26 @@ MUTATIONS = {
     "topk_off_by_one": ("tau = vals[top_k - 1];", "tau = vals[top_k];"),
     "topk_topp_over_whole_row": ("const double floor_v = tau, total = S_kept;",
                                  "const double floor_v = tau, total = S;"),
+    # the further tree rules and the candidate trie (pinned in test_oracle_tree_build.py)
+    "det_no_renormalise": ("for (int v = 0; v < V; ++v) r[v] /= Zr;", "(void)Zr;", TREE_BUILD),
+    "det_no_removal": ("          r[t] = 0.0;\n", "          (void)t;\n", TREE_BUILD),
+    "det_accept_not_by_r": ("if (ud < r[t]) { next = c; break; }", "if (ud < 0.5) { next = c; break; }", TREE_BUILD),
+    "wr_removes_token": ("if (rule == ORACLE_TREE_SAMPLED_WOR) {", "if (rule != ORACLE_TREE_DETERMINISTIC) {",
+                         TREE_BUILD),
+    "build_ties_to_deeper": ("better = da < db;", "better = da > db;", TREE_BUILD),
+    "build_ties_rank_reversed": ("(cmp == 0 && f_rank[e] < f_rank[bi])", "(cmp == 0 && f_rank[e] > f_rank[bi])",
+                                 TREE_BUILD),
+    "build_candidate_ties_high_index": ("if (best < 0 || qi[v] > qi[best]) best = v;",
+                                        "if (best < 0 || qi[v] >= qi[best]) best = v;", TREE_BUILD),
+    "build_score_sum": ("score[nn] = score[pa] * q[(size_t)d * V + tokens[nn]];",
+                        "score[nn] = score[pa] + q[(size_t)d * V + tokens[nn]];", TREE_BUILD),
 }
 
 
 @pytest.mark.parametrize("name", sorted(MUTATIONS))
 def test_mutant_is_caught(name, tmp_path):
-    old, new = MUTATIONS[name]
+    old, new = MUTATIONS[name][:2]
+    files = MUTATIONS[name][2] if len(MUTATIONS[name]) > 2 else PINS
     src = open(SRC).read()
     assert src.count(old) == 1, name
     mut = tmp_path / "mutant.c"
@@ -47,8 +64,7 @@ def test_mutant_is_caught(name, tmp_path):
     subprocess.check_call(["gcc", "-O2", "-std=c99", "-shared", "-fPIC", "-I", os.path.dirname(SRC),
                            "-o", str(lib), str(mut), "-lm"])
     env = dict(os.environ, ORACLE_LIB=str(lib))
-    r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
-                        os.path.join(ROOT, "tests", "test_oracle_pins.py"),
-                        os.path.join(ROOT, "tests", "test_oracle_lossless.py")],
+    r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider"] +
+                       [os.path.join(ROOT, "tests", f) for f in files],
                        cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
     assert r.returncode != 0, "mutation %s survived the pins" % name
