@@ -158,6 +158,15 @@ psispec_status psispec_row_stats(const void* logits, int dtype, int32_t B, int32
                                  void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * psispec_row_stats_k -- psispec_row_stats with a per-request top-k (see the conventions
+ * above): top_k [B] int32 device array, or NULL (off for every request). The records carry the
+ * top-k (then top-p) threshold and serve psispec_verify_linear_k with the same top_k.
+ */
+psispec_status psispec_row_stats_k(const void* logits, int dtype, int32_t B, int32_t K, int32_t V,
+                                   const float* temperature, const float* top_p, const int32_t* top_k,
+                                   void* out_row_stats, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * psispec_verify_linear -- Psi-Spec linear verification (review page, section 3.3; linear
  * sampler of section 3.4).
  *
@@ -241,6 +250,19 @@ psispec_status psispec_verify_tree(const void* target_logits, const void* draft_
                                    int32_t max_depth, int32_t* out_path, int32_t* out_tokens,
                                    int32_t* out_accept_len, void* workspace, size_t workspace_bytes,
                                    void* stream);
+
+/*
+ * psispec_verify_tree_k -- psispec_verify_tree with a per-request top-k applied to every
+ * node's verifier and draft rows: top_k [B] int32 device array, or NULL (off for every
+ * request). Same workspace size, limits and errors as psispec_verify_tree.
+ */
+psispec_status psispec_verify_tree_k(const void* target_logits, const void* draft_logits, int dtype,
+                                     int32_t B, int32_t N, int32_t V, const int32_t* node_offsets,
+                                     const int32_t* parent, const int32_t* tokens, const float* u_accept,
+                                     const float* u_resid, const float* temperature, const float* top_p,
+                                     const int32_t* top_k, int32_t max_depth, int32_t* out_path,
+                                     int32_t* out_tokens, int32_t* out_accept_len, void* workspace,
+                                     size_t workspace_bytes, void* stream);
 
 /*
  * psispec_verify_linear_static -- psispec_verify_linear without a caller workspace.

@@ -164,14 +164,15 @@ psispec_status launch_stream(RowSet<T> set, int64_t rows, int V, const float* te
 }
 
 // Row statistics of `rows` rows of a row set (the tree's statistics pass); with skip_uncut,
-// the rows of requests with T > 0 and no top-p cut are left out.
+// the rows of requests with T > 0 and no top-p cut are left out (callers with a top-k array
+// pass skip_uncut = 0: the streaming pass does not know top-k).
 template <typename T>
 psispec_status launch_stats(RowSet<T> set, int64_t rows, int V, const float* temperature, int nreq,
-                            const float* top_p, int skip_uncut, StatsWs ws, cudaStream_t st) {
+                            const float* top_p, const int32_t* top_k, int skip_uncut, StatsWs ws, cudaStream_t st) {
   psispec_status s = launch_stream<T>(set, rows, V, temperature, nreq, ws.parts, st, top_p, skip_uncut);
   if (s != PSISPEC_OK) return s;
   return launch(row_finalize_kernel<T>, static_cast<unsigned>((rows + kThreads / 32 - 1) / (kThreads / 32)), kThreads,
-                0, st, set, rows, V, temperature, top_p, ws.parts, ws.stats, skip_uncut);
+                0, st, set, rows, V, temperature, top_p, top_k, ws.parts, ws.stats, skip_uncut);
 }
 
 // Launch configuration of `nclusters` clusters of CL CTAs of `threads` threads; returns
@@ -356,8 +357,8 @@ psispec_status tree_cluster_config(int B, int V, cudaStream_t st, cudaLaunchConf
 template <typename T>
 psispec_status verify_tree_impl(const T* tgt, const T* drf, int B, int N, int V, const int32_t* offs,
                                 const int32_t* parent, const int32_t* tokens, const float* u_acc, const float* u_res,
-                                const float* temperature, const float* top_p, int max_depth, int32_t* out_path,
-                                int32_t* out_tokens, int32_t* out_len, void* ws, cudaStream_t st) {
+                                const float* temperature, const float* top_p, const int32_t* top_k, int max_depth,
+                                int32_t* out_path, int32_t* out_tokens, int32_t* out_len, void* ws, cudaStream_t st) {
   Carver c(ws);
   TreeWs w = carve_tree(c, N, V);
   // the walk: one cluster per trie, the node's rows staged across its CTAs' shared memory (16
@@ -372,10 +373,12 @@ psispec_status verify_tree_impl(const T* tgt, const T* drf, int B, int N, int V,
   }
   if (s == PSISPEC_ERR_UNSUPPORTED) CL = 0;
   else if (s != PSISPEC_OK) return s;
-  // the cluster walk finds the statistics of uncut requests' visited rows itself
-  const int lazy = CL != 0;
+  // the cluster walk finds the statistics of uncut requests' visited rows itself; with a top-k
+  // array every row goes through the statistics pass (its records carry the top-k threshold)
+  const int lazy = CL != 0 && top_k == nullptr;
   // one statistics pass over the rows of both tensors
-  s = launch_stats<T>(RowSet<T>{tgt, drf, N, 1, offs, B}, 2 * int64_t(N), V, temperature, B, top_p, lazy, w.st, st);
+  s = launch_stats<T>(RowSet<T>{tgt, drf, N, 1, offs, B}, 2 * int64_t(N), V, temperature, B, top_p, top_k, lazy, w.st,
+                      st);
   if (s != PSISPEC_OK) return s;
   const RowStat* ts = w.st.stats;
   const RowStat* ds = w.st.stats + N;
@@ -396,11 +399,12 @@ psispec_status verify_tree_impl(const T* tgt, const T* drf, int B, int N, int V,
 
 template <typename T>
 psispec_status row_stats_impl(const T* logits, int B, int K, int V, const float* temperature, const float* top_p,
-                              RowStat* out, void* ws, cudaStream_t st) {
+                              const int32_t* top_k, RowStat* out, void* ws, cudaStream_t st) {
   const int64_t rows = int64_t(B) * K;
   Carver c(ws);
   Partial* parts = carve_row_stats(c, rows, V);
-  return launch_stats<T>(one_tensor(logits, rows, K, B), rows, V, temperature, B, top_p, 0, StatsWs{parts, out}, st);
+  return launch_stats<T>(one_tensor(logits, rows, K, B), rows, V, temperature, B, top_p, top_k, 0,
+                         StatsWs{parts, out}, st);
 }
 
 bool bad_dtype(int dtype) { return dtype != PSISPEC_F32 && dtype != PSISPEC_BF16; }
@@ -518,12 +522,12 @@ psispec_status psispec_verify_linear(const void* target_logits, const void* draf
                                  workspace, workspace_bytes, stream);
 }
 
-psispec_status psispec_verify_tree(const void* target_logits, const void* draft_logits, int dtype, int32_t B,
-                                   int32_t N, int32_t V, const int32_t* node_offsets, const int32_t* parent,
-                                   const int32_t* tokens, const float* u_accept, const float* u_resid,
-                                   const float* temperature, const float* top_p, int32_t max_depth,
-                                   int32_t* out_path, int32_t* out_tokens, int32_t* out_accept_len, void* workspace,
-                                   size_t workspace_bytes, void* stream) {
+psispec_status psispec_verify_tree_k(const void* target_logits, const void* draft_logits, int dtype, int32_t B,
+                                     int32_t N, int32_t V, const int32_t* node_offsets, const int32_t* parent,
+                                     const int32_t* tokens, const float* u_accept, const float* u_resid,
+                                     const float* temperature, const float* top_p, const int32_t* top_k,
+                                     int32_t max_depth, int32_t* out_path, int32_t* out_tokens,
+                                     int32_t* out_accept_len, void* workspace, size_t workspace_bytes, void* stream) {
   if (!target_logits || !draft_logits || !node_offsets || !parent || !tokens || !u_accept || !u_resid ||
       !temperature || !top_p || !out_path || !out_tokens || !out_accept_len || bad_dtype(dtype))
     return PSISPEC_ERR_INVALID_ARG;
@@ -538,16 +542,27 @@ psispec_status psispec_verify_tree(const void* target_logits, const void* draft_
   if (dtype == PSISPEC_BF16)
     return verify_tree_impl(static_cast<const __nv_bfloat16*>(target_logits),
                             static_cast<const __nv_bfloat16*>(draft_logits), B, N, V, node_offsets, parent, tokens,
-                            u_accept, u_resid, temperature, top_p, max_depth, out_path, out_tokens, out_accept_len,
-                            workspace, st);
+                            u_accept, u_resid, temperature, top_p, top_k, max_depth, out_path, out_tokens,
+                            out_accept_len, workspace, st);
   return verify_tree_impl(static_cast<const float*>(target_logits), static_cast<const float*>(draft_logits), B, N, V,
-                          node_offsets, parent, tokens, u_accept, u_resid, temperature, top_p, max_depth, out_path,
-                          out_tokens, out_accept_len, workspace, st);
+                          node_offsets, parent, tokens, u_accept, u_resid, temperature, top_p, top_k, max_depth,
+                          out_path, out_tokens, out_accept_len, workspace, st);
 }
 
-psispec_status psispec_row_stats(const void* logits, int dtype, int32_t B, int32_t K, int32_t V,
-                                 const float* temperature, const float* top_p, void* out_row_stats,
-                                 void* workspace, size_t workspace_bytes, void* stream) {
+psispec_status psispec_verify_tree(const void* target_logits, const void* draft_logits, int dtype, int32_t B,
+                                   int32_t N, int32_t V, const int32_t* node_offsets, const int32_t* parent,
+                                   const int32_t* tokens, const float* u_accept, const float* u_resid,
+                                   const float* temperature, const float* top_p, int32_t max_depth,
+                                   int32_t* out_path, int32_t* out_tokens, int32_t* out_accept_len, void* workspace,
+                                   size_t workspace_bytes, void* stream) {
+  return psispec_verify_tree_k(target_logits, draft_logits, dtype, B, N, V, node_offsets, parent, tokens, u_accept,
+                               u_resid, temperature, top_p, nullptr, max_depth, out_path, out_tokens, out_accept_len,
+                               workspace, workspace_bytes, stream);
+}
+
+psispec_status psispec_row_stats_k(const void* logits, int dtype, int32_t B, int32_t K, int32_t V,
+                                   const float* temperature, const float* top_p, const int32_t* top_k,
+                                   void* out_row_stats, void* workspace, size_t workspace_bytes, void* stream) {
   if (!logits || !temperature || !top_p || !out_row_stats || bad_dtype(dtype)) return PSISPEC_ERR_INVALID_ARG;
   if (B <= 0 || K <= 0 || V <= 0) return PSISPEC_ERR_INVALID_ARG;
   if (!aligned_to(logits, esize(dtype)) || !aligned_to(out_row_stats, 16)) return PSISPEC_ERR_INVALID_ARG;
@@ -558,8 +573,16 @@ psispec_status psispec_row_stats(const void* logits, int dtype, int32_t B, int32
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   RowStat* rs = static_cast<RowStat*>(out_row_stats);
   if (dtype == PSISPEC_BF16)
-    return row_stats_impl(static_cast<const __nv_bfloat16*>(logits), B, K, V, temperature, top_p, rs, workspace, st);
-  return row_stats_impl(static_cast<const float*>(logits), B, K, V, temperature, top_p, rs, workspace, st);
+    return row_stats_impl(static_cast<const __nv_bfloat16*>(logits), B, K, V, temperature, top_p, top_k, rs,
+                          workspace, st);
+  return row_stats_impl(static_cast<const float*>(logits), B, K, V, temperature, top_p, top_k, rs, workspace, st);
+}
+
+psispec_status psispec_row_stats(const void* logits, int dtype, int32_t B, int32_t K, int32_t V,
+                                 const float* temperature, const float* top_p, void* out_row_stats,
+                                 void* workspace, size_t workspace_bytes, void* stream) {
+  return psispec_row_stats_k(logits, dtype, B, K, V, temperature, top_p, nullptr, out_row_stats, workspace,
+                             workspace_bytes, stream);
 }
 
 psispec_status psispec_verify_linear_static(const void* target_logits, const void* draft_logits, int dtype,

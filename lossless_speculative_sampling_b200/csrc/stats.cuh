@@ -33,6 +33,12 @@ __device__ __forceinline__ bool uncut_request(const float* __restrict__ temperat
   return temp_scale(temperature[req]) != 0.0f && !(top_p[req] < 1.0f);
 }
 
+// Request r's top-k (0 when off: no array, k <= 0 or k >= V).
+__device__ __forceinline__ int request_k(const int32_t* __restrict__ top_k, int r, int V) {
+  const int k = top_k ? top_k[r] : 0;
+  return k > 0 && k < V ? k : 0;
+}
+
 // Scale c of a request's rows for the streaming pass, or -1 for the rows it leaves alone: with
 // skip_uncut set, those of the requests uncut_request selects.
 __device__ __forceinline__ float stream_scale(const float* __restrict__ temperature, const float* __restrict__ top_p,
@@ -931,41 +937,52 @@ __device__ void block_topp_select(const T* __restrict__ rp, int V, float tp, Row
 
 // Row statistics from the chunk partials (the tree's statistics pass and psispec_row_stats):
 // kThreads / 32 rows per CTA, one warp finalizing each row; the CTA then runs the top-p
-// select for those of its rows that need one. Rows that stream_scale marks are skipped.
+// select (or, for a request with a top-k, the top-k then top-p select) for those of its rows
+// that need one. Rows that stream_scale marks are skipped. top_k may be null (off).
 template <typename T>
 __global__ void __launch_bounds__(kThreads) row_finalize_kernel(RowSet<T> rows, int64_t nrows, int V,
                                                                  const float* __restrict__ temperature,
                                                                  const float* __restrict__ top_p,
+                                                                 const int32_t* __restrict__ top_k,
                                                                  const Partial* __restrict__ parts,
                                                                  RowStat* __restrict__ stats, int skip_uncut) {
   constexpr int kRows = kThreads / 32;
   __shared__ ToppSmem sm;
   __shared__ RowStat sh_st[kRows];
   __shared__ int sh_topp[kRows];
+  __shared__ int sh_k[kRows];
   const int warp = threadIdx.x >> 5;
   const int64_t row = static_cast<int64_t>(blockIdx.x) * kRows + warp;
   const int nch = nchunks_for(V);
   if (row < nrows) {
     const int req = rows.request(row);
-    int topp = 0;
+    int topp = 0, k = 0;
     if (stream_scale(temperature, top_p, skip_uncut, req) >= 0.0f) {
       const RowStat st = warp_finalize_row(parts + static_cast<size_t>(row) * nch, nch, temperature[req]);
-      topp = needs_topp(st, top_p[req]);
+      k = st.status == 0 && st.c != 0.0f ? request_k(top_k, req, V) : 0;
+      topp = needs_topp(st, top_p[req]) || k > 0;
       if ((threadIdx.x & 31) == 0) {
         sh_st[warp] = st;
         if (!topp) stats[row] = st;
       }
     }
-    if ((threadIdx.x & 31) == 0) sh_topp[warp] = topp;
+    if ((threadIdx.x & 31) == 0) {
+      sh_topp[warp] = topp;
+      sh_k[warp] = k;
+    }
   } else if ((threadIdx.x & 31) == 0) {
     sh_topp[warp] = 0;
+    sh_k[warp] = 0;
   }
   __syncthreads();
   for (int w = 0; w < kRows; ++w) {
     if (!sh_topp[w]) continue;  // the same branch in every thread
     const int64_t r = static_cast<int64_t>(blockIdx.x) * kRows + w;
     RowStat st = sh_st[w];
-    block_topp_select<T>(rows.row(r, V), V, top_p[rows.request(r)], st, sm);
+    if (sh_k[w] > 0)  // the same branch in every thread
+      block_topk_topp_radix<T>(rows.row(r, V), V, top_p[rows.request(r)], sh_k[w], st, sm.radix);
+    else
+      block_topp_select<T>(rows.row(r, V), V, top_p[rows.request(r)], st, sm);
     if (threadIdx.x == 0) stats[r] = st;
   }
 }

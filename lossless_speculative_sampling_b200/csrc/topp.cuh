@@ -721,12 +721,6 @@ __device__ int tp_row_draw(const T* __restrict__ row, int V, const RowStat& st, 
   return y;
 }
 
-// Request r's top-k (0 when off: no array, k <= 0 or k >= V).
-__device__ __forceinline__ int request_k(const int32_t* __restrict__ top_k, int r, int V) {
-  const int k = top_k ? top_k[r] : 0;
-  return k > 0 && k < V ? k : 0;
-}
-
 // Whether request r's rows carry a cut (top-p below 1 or an active top-k, at T > 0).
 __device__ __forceinline__ bool request_cut(const float* __restrict__ temperature, const float* __restrict__ top_p,
                                             const int32_t* __restrict__ top_k, int r, int V) {

@@ -55,9 +55,13 @@ def lib():
                                               P]
         L.psispec_verify_tree.argtypes = [P, P, ctypes.c_int, I32, I32, I32, P, P, P, P, P, P, P, I32, P, P, P, P, SZ,
                                           P]
+        L.psispec_verify_tree_k.argtypes = [P, P, ctypes.c_int, I32, I32, I32, P, P, P, P, P, P, P, P, I32, P, P, P, P,
+                                            SZ, P]
+        L.psispec_row_stats_k.argtypes = [P, ctypes.c_int, I32, I32, I32, P, P, P, P, P, SZ, P]
         L.psispec_verify_linear_static.argtypes = [P, P, ctypes.c_int, I32, I32, I32, P, P, P, P, P, P, P, P, P, P, P]
-        for f in ("psispec_sample_draft", "psispec_sample_draft_k", "psispec_row_stats", "psispec_verify_linear",
-                  "psispec_verify_linear_k", "psispec_verify_tree", "psispec_verify_linear_static"):
+        for f in ("psispec_sample_draft", "psispec_sample_draft_k", "psispec_row_stats", "psispec_row_stats_k",
+                  "psispec_verify_linear", "psispec_verify_linear_k", "psispec_verify_tree", "psispec_verify_tree_k",
+                  "psispec_verify_linear_static"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -165,22 +169,29 @@ def sample_draft(draft, temperature, top_p, u, *, top_k=None, out_tokens=None, o
     return out_tokens, out_q, row_stats
 
 
-def row_stats(logits, temperature, top_p, *, out=None, ws=None, stream=None):
-    """Per-row statistics records of softmax(logits / T) after top-p.
+def row_stats(logits, temperature, top_p, *, top_k=None, out=None, ws=None, stream=None):
+    """Per-row statistics records of softmax(logits / T) after top-k and top-p.
 
-    logits [B, K, V] bf16/fp32; temperature, top_p [B] fp32. Returns [B, K, 32] uint8 records,
-    usable as verify_linear(draft_row_stats=...) for the same logits and controls."""
+    logits [B, K, V] bf16/fp32; temperature, top_p [B] fp32; top_k [B] int32 or None (off).
+    Returns [B, K, 32] uint8 records, usable as verify_linear(draft_row_stats=...) for the same
+    logits and controls."""
     B, K, V = logits.shape
     dev = logits.device
     _req(logits, "logits")
     _req(temperature, "temperature", torch.float32, B, dev)
     _req(top_p, "top_p", torch.float32, B, dev)
+    if top_k is not None:
+        _req(top_k, "top_k", torch.int32, B, dev)
     out = torch.empty((B, K, ROW_STATS_BYTES), dtype=torch.uint8, device=dev) if out is None else out
     _req(out, "out", torch.uint8, B * K * ROW_STATS_BYTES, dev)
     need = workspace_size(OP_ROW_STATS, B, K, V)
     ws = workspace(need, dev) if ws is None else ws
-    st = lib().psispec_row_stats(_p(logits), _dtype(logits), B, K, V, _p(temperature), _p(top_p), _p(out), _p(ws),
-                                 ws.numel(), _stream(dev, stream))
+    if top_k is None:
+        st = lib().psispec_row_stats(_p(logits), _dtype(logits), B, K, V, _p(temperature), _p(top_p), _p(out),
+                                     _p(ws), ws.numel(), _stream(dev, stream))
+    else:
+        st = lib().psispec_row_stats_k(_p(logits), _dtype(logits), B, K, V, _p(temperature), _p(top_p), _p(top_k),
+                                       _p(out), _p(ws), ws.numel(), _stream(dev, stream))
     _check(st, "psispec_row_stats")
     return out
 
@@ -228,11 +239,11 @@ def verify_linear(target, draft, draft_tokens, u_accept, u_resid, temperature, t
 
 
 def verify_tree(target, draft, node_offsets, parent, tokens, u_accept, u_resid, temperature, top_p, max_depth: int,
-                *, out_path=None, out_tokens=None, out_accept_len=None, ws=None, stream=None):
+                *, top_k=None, out_path=None, out_tokens=None, out_accept_len=None, ws=None, stream=None):
     """Psi-Spec tree verification. target/draft [N, V]; node_offsets [B+1] int32; parent,
     tokens [N] int32 (request-local parents, -1 at roots); u_accept, u_resid [N] fp32;
-    temperature/top_p [B]. Returns dict(path [B, max_depth], tokens [B, max_depth+1],
-    accept_len [B])."""
+    temperature/top_p [B]; top_k [B] int32 or None (off). Returns dict(path [B, max_depth],
+    tokens [B, max_depth+1], accept_len [B])."""
     N, V = target.shape
     B = node_offsets.numel() - 1
     dev = target.device
@@ -245,15 +256,23 @@ def verify_tree(target, draft, node_offsets, parent, tokens, u_accept, u_resid, 
         _req(t, name, torch.float32, N, dev)
     _req(temperature, "temperature", torch.float32, B, dev)
     _req(top_p, "top_p", torch.float32, B, dev)
+    if top_k is not None:
+        _req(top_k, "top_k", torch.int32, B, dev)
     out_path = torch.empty((B, max_depth), dtype=torch.int32, device=dev) if out_path is None else out_path
     out_tokens = torch.empty((B, max_depth + 1), dtype=torch.int32, device=dev) if out_tokens is None else out_tokens
     out_accept_len = torch.empty(B, dtype=torch.int32, device=dev) if out_accept_len is None else out_accept_len
     need = workspace_size(OP_VERIFY_TREE, B, N, V)
     ws = workspace(need, dev) if ws is None else ws
-    st = lib().psispec_verify_tree(_p(target), _p(draft), _dtype(target), B, N, V, _p(node_offsets), _p(parent),
-                                   _p(tokens), _p(u_accept), _p(u_resid), _p(temperature), _p(top_p), int(max_depth),
-                                   _p(out_path), _p(out_tokens), _p(out_accept_len), _p(ws), ws.numel(),
-                                   _stream(dev, stream))
+    if top_k is None:
+        st = lib().psispec_verify_tree(_p(target), _p(draft), _dtype(target), B, N, V, _p(node_offsets), _p(parent),
+                                       _p(tokens), _p(u_accept), _p(u_resid), _p(temperature), _p(top_p),
+                                       int(max_depth), _p(out_path), _p(out_tokens), _p(out_accept_len), _p(ws),
+                                       ws.numel(), _stream(dev, stream))
+    else:
+        st = lib().psispec_verify_tree_k(_p(target), _p(draft), _dtype(target), B, N, V, _p(node_offsets),
+                                         _p(parent), _p(tokens), _p(u_accept), _p(u_resid), _p(temperature),
+                                         _p(top_p), _p(top_k), int(max_depth), _p(out_path), _p(out_tokens),
+                                         _p(out_accept_len), _p(ws), ws.numel(), _stream(dev, stream))
     _check(st, "psispec_verify_tree")
     return {"path": out_path, "tokens": out_tokens, "accept_len": out_accept_len}
 

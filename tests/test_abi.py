@@ -126,6 +126,27 @@ def test_topk_entries_host_checks(L):
     assert linear_k(t=ctypes.c_void_p(4098)) == psispec.ERR_INVALID_ARG
     assert linear_k(ws=None) == psispec.ERR_WORKSPACE
 
+    def tree_k(**kw):
+        a = dict(par=FAKE, N=10, md=4, ws=FAKE, wsb=1 << 30)
+        a.update(kw)
+        return L.psispec_verify_tree_k(FAKE, FAKE, psispec.BF16, 2, a["N"], 64, FAKE, a["par"], FAKE, FAKE, FAKE, FAKE,
+                                       FAKE, None, a["md"], FAKE, FAKE, FAKE, a["ws"], a["wsb"], None)
+
+    def row_stats_k(**kw):
+        a = dict(l=FAKE, out=FAKE, K=3, ws=FAKE, wsb=1 << 30)
+        a.update(kw)
+        return L.psispec_row_stats_k(a["l"], psispec.BF16, 2, a["K"], 100, FAKE, FAKE, None, a["out"], a["ws"], a["wsb"],
+                                     None)
+
+    assert tree_k(par=None) == psispec.ERR_INVALID_ARG
+    assert tree_k(N=1) == psispec.ERR_INVALID_ARG
+    assert tree_k(md=65) == psispec.ERR_UNSUPPORTED
+    assert tree_k(ws=None) == psispec.ERR_WORKSPACE
+    assert row_stats_k(l=None) == psispec.ERR_INVALID_ARG
+    assert row_stats_k(K=0) == psispec.ERR_INVALID_ARG
+    assert row_stats_k(out=ctypes.c_void_p(4096 + 8)) == psispec.ERR_INVALID_ARG
+    assert row_stats_k(wsb=16) == psispec.ERR_WORKSPACE
+
 
 def _tree(L, **kw):
     a = dict(t=FAKE, d=FAKE, dtype=psispec.BF16, B=2, N=10, V=64, off=FAKE, par=FAKE, tok=FAKE, ua=FAKE, ur=FAKE,

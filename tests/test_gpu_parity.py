@@ -487,3 +487,45 @@ def test_negative_logit_rows(top_p, top_k):
                                 top_k=_cuda(Ks))
     ora = oracle.verify_linear(tgt, drf, x, ua, ur, Ts.numpy(), Ps.numpy(), top_k=Ks.numpy())
     compare_linear(out, ora)
+
+
+# ------------------------------------------------------------------ top-k: tree and row statistics
+
+
+@pytest.mark.parametrize("V,dtype,T,top_p", [(1000, torch.float32, 0.8, 1.0), (20011, torch.bfloat16, 1.0, 0.9),
+                                             (151936, torch.bfloat16, 1.0, 0.95)])
+def test_verify_tree_topk_parity(V, dtype, T, top_p):
+    """Per-request top-k in tree verification (off, k = 1, small and large k, k >= V)."""
+    B, nodes = 6, 24
+    trie, tgt, drf, toks, ua, ur = _tree_inputs(B, nodes, V, dtype, T, top_p, seed=V + 5)
+    Ts, Ps = torch.full((B,), T), torch.full((B,), top_p)
+    Ks = torch.tensor([5, 0, 100, V - 1, 1, V], dtype=torch.int32)
+    out = psispec.verify_tree(_cuda(tgt), _cuda(drf), _cuda(trie.node_offsets), _cuda(trie.parent), _cuda(toks),
+                              _cuda(ua), _cuda(ur), _cuda(Ts), _cuda(Ps), 6, top_k=_cuda(Ks))
+    ora = oracle.verify_tree(tgt, drf, trie.node_offsets.numpy(), trie.parent.numpy(), toks.numpy(), ua, ur,
+                             Ts.numpy(), Ps.numpy(), 6, top_k=Ks.numpy())
+    compare_tree(out, ora)
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_row_stats_topk_parity(dtype):
+    """psispec_row_stats_k records: the probability each record implies for every token within
+    1e-5 of the oracle's top-k (then top-p) distribution."""
+    B, K, V = 4, 3, 30011
+    tgt, drf, ud, ua, ur, _, _ = _linear_inputs(B, K, V, dtype, 1.0, 1.0, 0.6, seed=313, neg_inf_frac=0.05)
+    Ts = torch.tensor([1.0, 0.7, 1.3, 1.0])
+    Ps = torch.tensor([1.0, 0.9, 0.8, 1.0])
+    Ks = torch.tensor([40, 300, 5000, 0], dtype=torch.int32)
+    rec = psispec.row_stats(_cuda(drf), _cuda(Ts), _cuda(Ps), top_k=_cuda(Ks))
+    st = _decode_stats(rec)
+    rows = drf.reshape(B * K, V).float().numpy().astype(np.float64)
+    for r in range(B * K):
+        b = r // K
+        assert st["status"][r] == 0
+        probs, band = oracle.row_dist(rows[r], float(Ts[b]), float(Ps[b]), int(Ks[b]))
+        if band < 1e-6:
+            continue  # a threshold tie within the band: the kept set is not unique
+        l = rows[r].astype(np.float32)
+        kept = (_fkey(l) >= st["tau"][r]) if st["tau"][r] != 0 else np.ones(V, bool)
+        p = np.where(kept, np.exp2((l.astype(np.float64) - st["m"][r]) * st["c"][r]) / st["s_kept"][r], 0.0)
+        assert np.abs(p - probs).max() <= 1e-5, (r, np.abs(p - probs).max())
