@@ -2,10 +2,10 @@
 //
 // The streaming pass (stream_partials_kernel) reads every logits row once and leaves one
 // partial per kChunkElems-element chunk. The kernels here finish from those partials:
-//   warp_sample_row     one warp per draft row (no top-p cut): row statistics and the chunk
+//   warp_sample_row     one warp per draft row (no cut): row statistics and the chunk
 //                       holding u * Z (chunk partials are the prefix totals), then the draw
 //                       inside that chunk;
-//   warp_verify_row     one warp per verifier (and streamed draft) row (no top-p cut):
+//   warp_verify_row     one warp per verifier (and streamed draft) row (no cut):
 //                       statistics, then an arrival on the request's counter; the warp
 //                       completing a request runs the accept tests, finds the first rejection
 //                       and writes the draw job (both run inside the row kernels of topp.cuh);
@@ -251,7 +251,7 @@ __device__ __forceinline__ int warp_pick_resid(const double2* tot, int nchunks, 
   return warp_pick_totals(tot, nchunks, *use_p, u, base, target);
 }
 
-// Warp-level finish of one draft row without a top-p cut: statistics from the chunk
+// Warp-level finish of one draft row without a cut: statistics from the chunk
 // partials, the chunk holding u * Z (chunk partials are the prefix totals), and the draw
 // inside that chunk.
 template <typename T>
@@ -311,7 +311,7 @@ struct VerifyArgs {
 };
 
 // Warp-level finish of one row g (verifier rows, then streamed draft rows) of a request
-// without a top-p cut: statistics from the chunk partials, then the arrival on the request's
+// without a cut: statistics from the chunk partials, then the arrival on the request's
 // counter; the warp completing the request runs its accept tests, finds the first rejection
 // and writes the draw job.
 template <typename T>

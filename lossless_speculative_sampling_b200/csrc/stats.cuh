@@ -27,7 +27,7 @@ __device__ __forceinline__ float temp_scale(float T) {
 
 // Whether a request samples at a positive temperature with no top-p cut: its row statistics
 // are then the maximum and the sum alone, which the cluster tree walk computes itself on the
-// rows it visits.
+// rows it visits. (Calls with a top-k array do not use this: every row is finalized.)
 __device__ __forceinline__ bool uncut_request(const float* __restrict__ temperature, const float* __restrict__ top_p,
                                               int req) {
   return temp_scale(temperature[req]) != 0.0f && !(top_p[req] < 1.0f);

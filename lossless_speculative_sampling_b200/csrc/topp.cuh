@@ -1,9 +1,11 @@
-// topp.cuh -- rows of requests with a top-p cut: statistics, threshold and (draft rows) draw,
-// one CTA per row.
+// topp.cuh -- rows of requests with a cut (top-p below 1 or an active top-k, at T > 0):
+// statistics, threshold and (draft rows) draw, one CTA per row.
 //
 // The cut keeps every token whose logit is at least tau, the largest logit value t of the row
 // with mass(l >= t) >= top_p (review page of arXiv 2609.04010: the samplers take --top-p
-// with --temperature; ties are kept together), and renormalises over the kept set.
+// with --temperature; ties are kept together), and renormalises over the kept set. With a
+// top-k (the README's --top-k), the mass and the tail are those of the tokens at or above the
+// k-th largest logit, ties included.
 //
 // A CTA reads its row once from HBM and then, while the row is still in L2:
 //   A  maximum m (NaN-propagating; bf16 pairs compared packed);
@@ -727,7 +729,7 @@ __device__ __forceinline__ bool request_cut(const float* __restrict__ temperatur
   return temp_scale(temperature[r]) != 0.0f && (top_p[r] < 1.0f || request_k(top_k, r, V) > 0);
 }
 
-// The row kernel of sample_draft. CTAs [0, warp_ctas) finish the rows without a top-p cut,
+// The row kernel of sample_draft. CTAs [0, warp_ctas) finish the rows without a cut,
 // one warp per row; the remaining CTAs take the rows of requests with a cut, one row per CTA
 // at a time (statistics, threshold, draw). One launch serves both kinds of rows.
 template <typename T>
@@ -767,7 +769,7 @@ __global__ void __launch_bounds__(kTpThreads, 2) sample_rows_kernel(const T* __r
 }
 
 // The row kernel of verify_linear. CTAs [0, warp_ctas) finish the rows of requests without a
-// top-p cut, one warp per row; the remaining CTAs take the rows of requests with a cut, one
+// cut, one warp per row; the remaining CTAs take the rows of requests with a cut, one
 // row per CTA at a time (statistics and threshold). Every row then arrives on its request's
 // counter, and whoever completes a request runs its accept tests and writes the draw job.
 template <typename T>
