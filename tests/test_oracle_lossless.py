@@ -20,14 +20,19 @@ import scipy.stats
 import oracle
 
 
-def _dist(l, T, top_p):
-    """Verifier distribution computed independently of the oracle."""
+def _dist(l, T, top_p, top_k=0):
+    """Verifier distribution computed independently of the oracle (top-k by an explicit sort,
+    then top-p over the renormalised top-k set)."""
     l = np.asarray(l, dtype=np.float64)
     if T == 0:
         out = np.zeros_like(l)
         out[int(np.argmax(l))] = 1.0
         return out
     p = scipy.special.softmax(l / T)
+    if 0 < top_k < l.size:
+        kth = np.sort(l)[::-1][top_k - 1]
+        p = np.where(l >= kth, p, 0.0)
+        p = p / p.sum()
     if top_p >= 1:
         return p
     best = -np.inf
@@ -83,7 +88,7 @@ class TableLM:
     def extend(self, code, length, tok):
         return code + (np.asarray(tok) + 1) * self.base ** np.asarray(length)
 
-    def law(self, L, T, top_p):
+    def law(self, L, T, top_p, top_k=0):
         """Exact law of the first L tokens under the verifier."""
         out = {}
 
@@ -91,7 +96,7 @@ class TableLM:
             if len(prefix) == L:
                 out[tuple(prefix)] = prob
                 return
-            d = _dist(self.P[code], T, top_p)
+            d = _dist(self.P[code], T, top_p, top_k)
             for t in range(self.V):
                 if d[t] > 0:
                     rec(prefix + [t], int(self.extend(code, len(prefix), t)), prob * d[t])
@@ -117,11 +122,13 @@ def _chi2_check(samples, law, V, L):
     assert pval > 1e-3, (stat, pval)
 
 
-@pytest.mark.parametrize("K,T,top_p", [(1, 1.0, 1.0), (2, 1.0, 1.0), (3, 0.8, 0.8), (2, 1.3, 0.9)])
-def test_multiround_linear_matches_verifier_law(K, T, top_p):
+@pytest.mark.parametrize("K,T,top_p,top_k", [(1, 1.0, 1.0, 0), (2, 1.0, 1.0, 0), (3, 0.8, 0.8, 0), (2, 1.3, 0.9, 0),
+                                             (2, 1.0, 1.0, 2), (3, 1.2, 0.9, 2)])
+def test_multiround_linear_matches_verifier_law(K, T, top_p, top_k):
     V, L, N = 3, 4, 40000
-    lm = TableLM(V, seed=100 + K)
-    rng = np.random.default_rng(200 + K)
+    lm = TableLM(V, seed=100 + K + 10 * top_k)
+    rng = np.random.default_rng(200 + K + 10 * top_k)
+    kk = np.full(N, top_k, np.int32) if top_k else None
     seq = np.full((N, L + K + 1), -1, np.int64)
     length = np.zeros(N, np.int64)
     code = np.zeros(N, np.int64)
@@ -131,12 +138,13 @@ def test_multiround_linear_matches_verifier_law(K, T, top_p):
         c = [code[act]]
         x = np.zeros((n, K), np.int64)
         for i in range(K):
-            s = oracle.sample_draft(lm.Q[c[-1]], np.full(n, T), np.full(n, top_p), rng.random(n))
+            s = oracle.sample_draft(lm.Q[c[-1]], np.full(n, T), np.full(n, top_p), rng.random(n),
+                                    top_k=None if kk is None else kk[:n])
             x[:, i] = s["tokens"]
             c.append(lm.extend(c[-1], length[act] + i, x[:, i]))
         codes = np.stack(c, axis=1)  # [n, K+1]
         r = oracle.verify_linear(lm.P[codes], lm.Q[codes[:, :K]], x, rng.random((n, K)), rng.random((n, K + 1)),
-                                 np.full(n, T), np.full(n, top_p))
+                                 np.full(n, T), np.full(n, top_p), top_k=None if kk is None else kk[:n])
         assert (r["accept_len"] >= 0).all()
         for row, b in enumerate(act):
             j = r["accept_len"][row]
@@ -144,7 +152,7 @@ def test_multiround_linear_matches_verifier_law(K, T, top_p):
                 seq[b, length[b]] = t
                 code[b] = lm.extend(code[b], length[b], t)
                 length[b] += 1
-    _chi2_check(seq, lm.law(L, T, top_p), V, L)
+    _chi2_check(seq, lm.law(L, T, top_p, top_k), V, L)
 
 
 def test_multiround_tree_matches_verifier_law():
@@ -182,3 +190,44 @@ def test_multiround_tree_matches_verifier_law():
                 code[b] = lm.extend(code[b], length[b], t)
                 length[b] += 1
     _chi2_check(seq, lm.law(L, T, 1.0), V, L)
+
+
+def test_multiround_tree_with_top_k_matches_verifier_law():
+    """Binary trie of depth 2 per round under top-k 3 of V = 4: children drawn here (numpy,
+    from the independently computed top-k draft distribution) without replacement, verified by
+    the oracle with the same top-k; the emitted tokens follow the top-k verifier law."""
+    V, L, N, T, k = 4, 3, 30000, 1.0, 3
+    lm = TableLM(V, seed=700)
+    rng = np.random.default_rng(701)
+    parent = np.array([-1, 0, 0, 1, 1, 2, 2], np.int32)
+    seq = np.full((N, L + 4), -1, np.int64)
+    length = np.zeros(N, np.int64)
+    code = np.zeros(N, np.int64)
+    while (length < L).any():
+        act = np.nonzero(length < L)[0]
+        n = act.size
+        codes = np.zeros((n, 7), np.int64)
+        toks = np.zeros((n, 7), np.int64)
+        codes[:, 0] = code[act]
+        for node in range(1, 7):
+            pa = parent[node]
+            lq = lm.Q[codes[:, pa]] / T
+            kth = np.sort(lm.Q[codes[:, pa]], axis=1)[:, V - k][:, None]  # top-k by an explicit sort
+            q = np.where(lm.Q[codes[:, pa]] >= kth, np.exp(lq - lq.max(axis=1, keepdims=True)), 0.0)
+            for sib in range(1, node):  # earlier siblings' tokens are removed
+                if parent[sib] == pa:
+                    q[np.arange(n), toks[:, sib]] = 0.0
+            c = np.cumsum(q / q.sum(axis=1, keepdims=True), axis=1)
+            toks[:, node] = np.minimum((c <= rng.random(n)[:, None]).sum(axis=1), V - 1)
+            codes[:, node] = lm.extend(codes[:, pa], length[act] + (1 if pa == 0 else 2) - 1, toks[:, node])
+        r = oracle.verify_tree(lm.P[codes].reshape(-1, V), lm.Q[codes].reshape(-1, V), np.arange(0, 7 * n + 1, 7),
+                               np.tile(parent, n), toks.reshape(-1), rng.random(7 * n), rng.random(7 * n),
+                               np.full(n, T), np.ones(n), 2, top_k=np.full(n, k, np.int32))
+        assert (r["accept_len"] >= 0).all()
+        for row, b in enumerate(act):
+            j = r["accept_len"][row]
+            for t in r["tokens"][row, : j + 1]:
+                seq[b, length[b]] = t
+                code[b] = lm.extend(code[b], length[b], t)
+                length[b] += 1
+    _chi2_check(seq, lm.law(L, T, 1.0, k), V, L)
