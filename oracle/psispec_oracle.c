@@ -386,7 +386,12 @@ int oracle_verify_tree_rule(const double* target, const double* draft, int B, in
  *   - "the V most probable prefixes" are taken in decreasing probability, ties to the shorter
  *     prefix, then to the lexicographically smaller sequence of candidate ranks; a prefix is
  *     never less probable than its parent, so the kept set is closed under taking prefixes and
- *     forms a trie.
+ *     forms a trie;
+ *   - probabilities are compared exactly where that is possible: two prefixes of the same
+ *     length share their positions, hence their normalisers, so the more probable one is the
+ *     one with the larger sum of logits (exact in fp64 for bf16 and ordinary fp32 logits;
+ *     logits on the bf16 grid make equal sums, i.e. exact ties, common). Prefixes of different
+ *     lengths are compared by their fp64 probabilities.
  * They are found best-first: the frontier starts with the first position's candidates; the
  * best frontier prefix is kept and its extensions by the next position's candidates join the
  * frontier. Kept prefixes become nodes in the order kept (node 0 is the root, the empty
@@ -430,6 +435,7 @@ int oracle_build_tree(const double* draft, int K, int V, double T, double top_p,
   /* kept prefixes: rank path of every node (its candidate rank at each position) */
   const int cap = n_prefixes + 1;
   int* ranks = (int*)calloc((size_t)cap * (K > 0 ? K : 1), sizeof(int));
+  double* lsum = (double*)calloc((size_t)cap, sizeof(double)); /* sum of the prefix's logits */
   /* frontier entries: (parent node, candidate rank at the parent's depth) */
   const int fcap = cand_k * cap + 1;
   int* f_par = (int*)malloc(sizeof(int) * (size_t)fcap);
@@ -448,13 +454,17 @@ int oracle_build_tree(const double* draft, int K, int V, double T, double top_p,
     for (int e = 1; e < nf; ++e) {
       const int pa = f_par[e], pb = f_par[bi];
       const int da = depth[pa], db = depth[pb];
-      const double sa = score[pa] * q[(size_t)da * V + cand[da * cand_k + f_rank[e]]];
-      const double sb = score[pb] * q[(size_t)db * V + cand[db * cand_k + f_rank[bi]]];
-      int better = sa > sb;
-      if (sa == sb && !better) {
-        if (da != db) {
-          better = da < db;
-        } else {
+      const int ta = cand[da * cand_k + f_rank[e]], tb = cand[db * cand_k + f_rank[bi]];
+      int better;
+      if (da != db) {
+        const double sa = score[pa] * q[(size_t)da * V + ta];
+        const double sb = score[pb] * q[(size_t)db * V + tb];
+        better = sa > sb || (sa == sb && da < db);
+      } else {
+        const double la = lsum[pa] + draft[(size_t)da * V + ta];
+        const double lb = lsum[pb] + draft[(size_t)db * V + tb];
+        better = la > lb;
+        if (la == lb) {
           int cmp = 0;
           for (int j = 0; j < da && cmp == 0; ++j)
             cmp = (ranks[(size_t)pa * K + j] > ranks[(size_t)pb * K + j]) -
@@ -472,6 +482,7 @@ int oracle_build_tree(const double* draft, int K, int V, double T, double top_p,
     tokens[nn] = cand[d * cand_k + ra];
     depth[nn] = d + 1;
     score[nn] = score[pa] * q[(size_t)d * V + tokens[nn]];
+    lsum[nn] = lsum[pa] + draft[(size_t)d * V + tokens[nn]];
     for (int j = 0; j < d; ++j) ranks[(size_t)nn * K + j] = ranks[(size_t)pa * K + j];
     ranks[(size_t)nn * K + d] = ra;
     if (d + 1 < K)
@@ -483,6 +494,7 @@ int oracle_build_tree(const double* draft, int K, int V, double T, double top_p,
   free(cand);
   free(ncand);
   free(ranks);
+  free(lsum);
   free(f_par);
   free(f_rank);
   return ORACLE_OK;

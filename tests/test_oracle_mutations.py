@@ -42,7 +42,9 @@ MUTATIONS = {
     "det_accept_not_by_r": ("if (ud < r[t]) { next = c; break; }", "if (ud < 0.5) { next = c; break; }", TREE_BUILD),
     "wr_removes_token": ("if (rule == ORACLE_TREE_SAMPLED_WOR) {", "if (rule != ORACLE_TREE_DETERMINISTIC) {",
                          TREE_BUILD),
-    "build_ties_to_deeper": ("better = da < db;", "better = da > db;", TREE_BUILD),
+    "build_ties_to_deeper": ("(sa == sb && da < db)", "(sa == sb && da > db)", TREE_BUILD),
+    "build_logit_sum_not_accumulated": ("lsum[nn] = lsum[pa] + draft[(size_t)d * V + tokens[nn]];",
+                                        "lsum[nn] = draft[(size_t)d * V + tokens[nn]];", TREE_BUILD),
     "build_ties_rank_reversed": ("(cmp == 0 && f_rank[e] < f_rank[bi])", "(cmp == 0 && f_rank[e] > f_rank[bi])",
                                  TREE_BUILD),
     "build_candidate_ties_high_index": ("if (best < 0 || qi[v] > qi[best]) best = v;",
