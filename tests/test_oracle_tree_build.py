@@ -200,12 +200,14 @@ def _apply(seq, length, code, lm, act, r):
             length[b] += 1
 
 
-def test_multiround_deterministic_tree_matches_verifier_law():
+@pytest.mark.parametrize("top_k", [0, 2])
+def test_multiround_deterministic_tree_matches_verifier_law(top_k):
     """Per round: draft marginals for K positions (the draft's next-token row, then its row
-    after the draft's own argmax), the candidate trie over them, the deterministic rule."""
+    after the draft's own argmax), the candidate trie over them, the deterministic rule; with
+    top-k, the trie and the verification both use it and the law is the top-k verifier's."""
     V, L, N, T, K, ck, nv = 3, 4, 20000, 1.0, 2, 2, 4
-    lm = TableLM(V, seed=500)
-    rng = np.random.default_rng(501)
+    lm = TableLM(V, seed=500 + top_k)
+    rng = np.random.default_rng(501 + top_k)
     seq = np.full((N, L + K + 1), -1, np.int64)
     length = np.zeros(N, np.int64)
     code = np.zeros(N, np.int64)
@@ -216,7 +218,7 @@ def test_multiround_deterministic_tree_matches_verifier_law():
         c1 = lm.extend(c0, length[act], np.argmax(lm.Q[c0], axis=1))
         offs, pars, toks, codes = [0], [], [], []
         for row in range(n):
-            t = oracle.build_tree(np.stack([lm.Q[c0[row]], lm.Q[c1[row]]]), T, 1.0, ck, nv)
+            t = oracle.build_tree(np.stack([lm.Q[c0[row]], lm.Q[c1[row]]]), T, 1.0, ck, nv, top_k=top_k)
             m = len(t["parent"])
             nc = np.zeros(m, np.int64)
             nc[0] = c0[row]
@@ -231,18 +233,20 @@ def test_multiround_deterministic_tree_matches_verifier_law():
         tok[tok < 0] = 0
         r = oracle.verify_tree(lm.P[codes], lm.Q[codes], np.array(offs), np.concatenate(pars), tok,
                                rng.random(codes.size), rng.random(codes.size), np.full(n, T), np.ones(n), K,
-                               rule=oracle.TREE_DETERMINISTIC)
+                               top_k=np.full(n, top_k, np.int32), rule=oracle.TREE_DETERMINISTIC)
         assert (r["accept_len"] >= 0).all()
         _apply(seq, length, code, lm, act, r)
-    _chi2_check(seq, lm.law(L, T, 1.0), V, L)
+    _chi2_check(seq, lm.law(L, T, 1.0, top_k), V, L)
 
 
-def test_multiround_with_replacement_tree_matches_verifier_law():
+@pytest.mark.parametrize("top_k", [0, 2])
+def test_multiround_with_replacement_tree_matches_verifier_law(top_k):
     """Binary trie of depth 2; every child drawn from its parent's q independently (siblings
-    may repeat a token); the with-replacement rule."""
+    may repeat a token); the with-replacement rule, with and without top-k."""
     V, L, N, T = 3, 4, 20000, 1.0
-    lm = TableLM(V, seed=600, draft_noise=1.5)
-    rng = np.random.default_rng(601)
+    lm = TableLM(V, seed=600 + top_k, draft_noise=1.5)
+    rng = np.random.default_rng(601 + top_k)
+    kk = np.full(N, top_k, np.int32)
     parent = np.array([-1, 0, 0, 1, 1, 2, 2], np.int32)
     seq = np.full((N, L + 4), -1, np.int64)
     length = np.zeros(N, np.int64)
@@ -255,14 +259,15 @@ def test_multiround_with_replacement_tree_matches_verifier_law():
         codes[:, 0] = code[act]
         for node in range(1, 7):
             pa = parent[node]
-            toks[:, node] = oracle.sample_draft(lm.Q[codes[:, pa]], np.full(n, T), np.ones(n), rng.random(n))["tokens"]
+            toks[:, node] = oracle.sample_draft(lm.Q[codes[:, pa]], np.full(n, T), np.ones(n), rng.random(n),
+                                                top_k=kk[:n])["tokens"]
             codes[:, node] = lm.extend(codes[:, pa], length[act] + (1 if pa == 0 else 2) - 1, toks[:, node])
         r = oracle.verify_tree(lm.P[codes].reshape(-1, V), lm.Q[codes].reshape(-1, V), np.arange(0, 7 * n + 1, 7),
                                np.tile(parent, n), toks.reshape(-1), rng.random(7 * n), rng.random(7 * n),
-                               np.full(n, T), np.ones(n), 2, rule=oracle.TREE_SAMPLED_WR)
+                               np.full(n, T), np.ones(n), 2, top_k=kk[:n], rule=oracle.TREE_SAMPLED_WR)
         assert (r["accept_len"] >= 0).all()
         _apply(seq, length, code, lm, act, r)
-    _chi2_check(seq, lm.law(L, T, 1.0), V, L)
+    _chi2_check(seq, lm.law(L, T, 1.0, top_k), V, L)
 
 
 def test_rules_coincide_on_single_child_chains():
