@@ -25,7 +25,8 @@
  *  - Temperature T (per request): T == 0 means greedy (a point mass on the lowest-index
  *    maximum); T > 0 divides the logits by T before the softmax over the whole vocabulary.
  *    T < 0, NaN or inf is a per-request data error.
- *  - top_p (per request): in (0, 1); values >= 1 switch the filter off. The kept set is every
+ *  - top_p (per request): in (0, 1); values >= 1 (and NaN) switch the filter off, values <= 0
+ *    keep only the maximum's value (with its ties). The kept set is every
  *    token whose logit is >= tau, where tau is the largest logit value whose tie-inclusive
  *    upper-tail probability is >= top_p; the distribution is renormalised over the kept set.
  *    It is applied after the temperature, to the verifier row and to the draft row
