@@ -324,3 +324,16 @@ def test_branching_one_tree_equals_linear(T, tp):
     for b in range(B):
         j = lin["accept_len"][b]
         assert tr["path"][b, :j].tolist() == list(range(1, j + 1))
+
+
+def test_topp_at_or_below_zero_keeps_the_maximum_value():
+    """top_p <= 0 is met by the maximum's value alone (its ties kept), like a tiny top_p; NaN
+    and values >= 1 leave the row unfiltered."""
+    l = np.array([0.5, 2.0, -1.0, 2.0, 1.5])
+    for tp in (0.0, -0.5, 1e-9):
+        p, _ = oracle.row_dist(l, 1.0, tp)
+        assert np.array_equal(p, np.array([0.0, 0.5, 0.0, 0.5, 0.0]))
+    full, _ = oracle.row_dist(l, 1.0, 1.0)
+    assert np.allclose(full, np.exp(l - l.max()) / np.exp(l - l.max()).sum(), rtol=0, atol=1e-15)
+    for tp in (float("nan"), 1.0, 3.0):
+        assert np.array_equal(oracle.row_dist(l, 1.0, tp)[0], full)
