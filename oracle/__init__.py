@@ -35,6 +35,8 @@ E_BAND = 1e-6  # decisions whose margin is below this may differ between correct
 
 # candidate rules of tree verification (psispec_oracle.h)
 TREE_SAMPLED_WOR, TREE_DETERMINISTIC, TREE_SAMPLED_WR = 0, 1, 2
+# kinds of decision behind a band ("band_kind" outputs): none, accept test, draw edge, top-p tail
+BAND_NONE, BAND_E1, BAND_E2, BAND_E3 = 0, 1, 2, 3
 
 
 def build(force: bool = False) -> str:
@@ -56,13 +58,13 @@ def _load():
         lib.oracle_row_dist.argtypes = [D, ctypes.c_int, ctypes.c_double, ctypes.c_double, D, D]
         lib.oracle_row_dist_k.argtypes = [D, ctypes.c_int, ctypes.c_double, ctypes.c_double, ctypes.c_int, D, D]
         lib.oracle_inverse_cdf.argtypes = [D, ctypes.c_int, ctypes.c_double, D]
-        lib.oracle_sample_draft.argtypes = [D, ctypes.c_int, ctypes.c_int, I, D, D, I, D, I, D, D]
+        lib.oracle_sample_draft.argtypes = [D, ctypes.c_int, ctypes.c_int, I, D, D, I, D, I, D, D, I]
         lib.oracle_verify_linear.argtypes = [D, D, ctypes.c_int, ctypes.c_int, ctypes.c_int, I, D, D, D, D, I,
-                                             I, I, D, D, D, D]
+                                             I, I, D, D, D, D, I]
         lib.oracle_verify_tree.argtypes = [D, D, ctypes.c_int, ctypes.c_int, I, I, I, D, D, D, D, I,
-                                           ctypes.c_int, I, I, I, D]
+                                           ctypes.c_int, I, I, I, D, I]
         lib.oracle_verify_tree_rule.argtypes = [D, D, ctypes.c_int, ctypes.c_int, I, I, I, D, D, D, D, I,
-                                                ctypes.c_int, ctypes.c_int, I, I, I, D]
+                                                ctypes.c_int, ctypes.c_int, I, I, I, D, I]
         lib.oracle_build_tree.argtypes = [D, ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_double,
                                           ctypes.c_int, ctypes.c_int, ctypes.c_int, I, I, I, D, I]
         _lib = lib
@@ -118,7 +120,8 @@ def inverse_cdf(r, u: float):
 
 def sample_draft(draft_logits, temperature, top_p, u, row_req=None, top_k=None):
     """draft_logits [rows, V]; temperature/top_p (and top_k, None: off) per request; u [rows];
-    row_req maps rows to requests (default: row i -> request i). Returns dict(tokens, q, band)."""
+    row_req maps rows to requests (default: row i -> request i). Returns dict(tokens, q, band,
+    band_kind)."""
     d = _as_f64(draft_logits)
     rows, V = d.shape
     rr = np.arange(rows) if row_req is None else np.asarray(row_req)
@@ -130,15 +133,16 @@ def sample_draft(draft_logits, temperature, top_p, u, row_req=None, top_k=None):
     tok, tokp = _i32(np.zeros(rows))
     q, qp = _f64(np.zeros(rows))
     band, bp = _f64(np.zeros(rows))
+    kind, kp = _i32(np.zeros(rows))
     Kk, Kkp = _top_k(top_k, P.size)
-    _load().oracle_sample_draft(dp, rows, V, rrp, Tp, Pp, Kkp, up, tokp, qp, bp)
-    return {"tokens": tok, "q": q, "band": band}
+    _load().oracle_sample_draft(dp, rows, V, rrp, Tp, Pp, Kkp, up, tokp, qp, bp, kp)
+    return {"tokens": tok, "q": q, "band": band, "band_kind": kind}
 
 
 def verify_linear(target, draft, draft_tokens, u_accept, u_resid, temperature, top_p, top_k=None):
     """target [B, K+1, V], draft [B, K, V], draft_tokens [B, K], u_accept [B, K],
     u_resid [B, K+1], temperature [B], top_p [B], top_k [B] (None: off). Returns dict(tokens [B, K+1],
-    accept_len [B], p [B, K], q [B, K], band [B], pq_band [B, K])."""
+    accept_len [B], p [B, K], q [B, K], band [B], pq_band [B, K], band_kind [B])."""
     t = _as_f64(target)
     B, K1, V = t.shape
     K = K1 - 1
@@ -155,9 +159,10 @@ def verify_linear(target, draft, draft_tokens, u_accept, u_resid, temperature, t
     q, qp = _f64(np.zeros((B, K)))
     band, bp = _f64(np.zeros(B))
     pqb, pqbp = _f64(np.zeros((B, K)))
+    kind, kp = _i32(np.zeros(B))
     Kk, Kkp = _top_k(top_k, B)
-    _load().oracle_verify_linear(tp, dp, B, K, V, xp, uap, urp, Tp, Pp, Kkp, tokp, lnp, pp, qp, bp, pqbp)
-    return {"tokens": tok, "accept_len": ln, "p": p, "q": q, "band": band, "pq_band": pqb}
+    _load().oracle_verify_linear(tp, dp, B, K, V, xp, uap, urp, Tp, Pp, Kkp, tokp, lnp, pp, qp, bp, pqbp, kp)
+    return {"tokens": tok, "accept_len": ln, "p": p, "q": q, "band": band, "pq_band": pqb, "band_kind": kind}
 
 
 def verify_tree(target, draft, node_offsets, parent, tokens, u_accept, u_resid, temperature, top_p,
@@ -165,7 +170,7 @@ def verify_tree(target, draft, node_offsets, parent, tokens, u_accept, u_resid, 
     """target/draft [N, V]; node_offsets [B+1]; parent/tokens/u_accept/u_resid [N] (parent is
     the request-local index, -1 at the root); rule: how the children were produced
     (TREE_SAMPLED_WOR, TREE_DETERMINISTIC, TREE_SAMPLED_WR). Returns dict(path [B, max_depth],
-    tokens [B, max_depth+1], accept_len [B], band [B])."""
+    tokens [B, max_depth+1], accept_len [B], band [B], band_kind [B])."""
     t = _as_f64(target)
     N, V = t.shape
     off = np.asarray(node_offsets)
@@ -183,16 +188,17 @@ def verify_tree(target, draft, node_offsets, parent, tokens, u_accept, u_resid, 
     otk, otkp = _i32(np.zeros((B, max_depth + 1)))
     ln, lnp = _i32(np.zeros(B))
     band, bp = _f64(np.zeros(B))
+    kind, kp = _i32(np.zeros(B))
     Kk, Kkp = _top_k(top_k, B)
     if rule == TREE_SAMPLED_WOR:
         rc = _load().oracle_verify_tree(tp, dp, B, V, offp, parp, tkp, uap, urp, Tp, Pp, Kkp, int(max_depth), pathp,
-                                        otkp, lnp, bp)
+                                        otkp, lnp, bp, kp)
     else:
         rc = _load().oracle_verify_tree_rule(tp, dp, B, V, offp, parp, tkp, uap, urp, Tp, Pp, Kkp, int(max_depth),
-                                             int(rule), pathp, otkp, lnp, bp)
+                                             int(rule), pathp, otkp, lnp, bp, kp)
     if rc != 0:
         raise ValueError("oracle_verify_tree: bad arguments (rule %r)" % (rule,))
-    return {"path": path, "tokens": otk, "accept_len": ln, "band": band}
+    return {"path": path, "tokens": otk, "accept_len": ln, "band": band, "band_kind": kind}
 
 
 def build_tree(draft_rows, temperature: float, top_p: float, cand_k: int, n_prefixes: int, top_k: int = 0):

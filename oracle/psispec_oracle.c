@@ -43,6 +43,14 @@
 
 static double dmin(double a, double b) { return a < b ? a : b; }
 
+/* Keeps the smallest band of a path and the kind of decision (E1, E2, E3) it belongs to. */
+static void note_band(double* band, int* kind, double b, int k) {
+  if (b < *band) {
+    *band = b;
+    *kind = k;
+  }
+}
+
 static int cmp_desc(const void* a, const void* b) {
   double x = *(const double*)a, y = *(const double*)b;
   return (x < y) - (x > y);
@@ -144,7 +152,7 @@ int oracle_inverse_cdf(const double* r, int V, double u, double* band) {
 
 int oracle_sample_draft(const double* draft, int rows, int V, const int* row_req,
                         const double* temperature, const double* top_p, const int* top_k, const double* u,
-                        int* tokens, double* q_at, double* band) {
+                        int* tokens, double* q_at, double* band, int* band_kind) {
   if (rows < 0 || V <= 0) return ORACLE_BAD_ARG;
   double* q = (double*)malloc(sizeof(double) * (size_t)V);
   for (int i = 0; i < rows; ++i) {
@@ -153,12 +161,18 @@ int oracle_sample_draft(const double* draft, int rows, int V, const int* row_req
     tokens[i] = -1;
     q_at[i] = -1.0;
     band[i] = INFINITY;
+    if (band_kind) band_kind[i] = ORACLE_BAND_NONE;
     if (oracle_row_dist_k(draft + (size_t)i * V, V, temperature[b], top_p[b], top_k ? top_k[b] : 0, q, &b3) != 0)
       continue;
     int y = oracle_inverse_cdf(q, V, u[i], &b2);
     tokens[i] = y;
     q_at[i] = y >= 0 ? q[y] : -1.0;
-    band[i] = dmin(b2, b3);
+    int kind = ORACLE_BAND_NONE;
+    double bi = INFINITY;
+    note_band(&bi, &kind, b3, ORACLE_BAND_E3);
+    note_band(&bi, &kind, b2, ORACLE_BAND_E2);
+    band[i] = bi;
+    if (band_kind) band_kind[i] = kind;
   }
   free(q);
   return ORACLE_OK;
@@ -168,7 +182,7 @@ int oracle_verify_linear(const double* target, const double* draft, int B, int K
                          const int* draft_tokens, const double* u_accept, const double* u_resid,
                          const double* temperature, const double* top_p, const int* top_k,
                          int* out_tokens, int* accept_len, double* out_p, double* out_q,
-                         double* band, double* pq_band) {
+                         double* band, double* pq_band, int* band_kind) {
   if (B < 0 || K < 0 || V <= 0) return ORACLE_BAD_ARG;
   double* p = (double*)malloc(sizeof(double) * (size_t)V);
   double* q = (double*)malloc(sizeof(double) * (size_t)V);
@@ -179,7 +193,7 @@ int oracle_verify_linear(const double* target, const double* draft, int B, int K
     const double* tgt = target + (size_t)b * (K + 1) * V;
     const double* drf = draft + (size_t)b * K * V;
     int* toks = out_tokens + (size_t)b * (K + 1);
-    int bad = 0, j = K, y = -1;
+    int bad = 0, j = K, y = -1, path_kind = ORACLE_BAND_NONE;
     double path_band = INFINITY;
     for (int i = 0; i <= K; ++i) toks[i] = -1;
     for (int i = 0; i < K; ++i) pq_band[(size_t)b * K + i] = INFINITY;
@@ -195,8 +209,8 @@ int oracle_verify_linear(const double* target, const double* draft, int B, int K
       pq_band[(size_t)b * K + i] = dmin(bp, bq);
       if (i > j) continue; /* past the first rejection: probabilities only */
       double u = u_accept[(size_t)b * K + i];
-      path_band = dmin(path_band, dmin(bp, bq));
-      if (q[x] > 0.0) path_band = dmin(path_band, fabs(u - p[x] / q[x]));
+      note_band(&path_band, &path_kind, dmin(bp, bq), ORACLE_BAND_E3);
+      if (q[x] > 0.0) note_band(&path_band, &path_kind, fabs(u - p[x] / q[x]), ORACLE_BAND_E1);
       if (u * q[x] < p[x]) continue; /* accepted */
       /* first rejection: draw from the normalised residual [p - q]_+ */
       j = i;
@@ -207,7 +221,7 @@ int oracle_verify_linear(const double* target, const double* draft, int B, int K
       }
       double b2 = INFINITY;
       y = oracle_inverse_cdf(Z > 0.0 ? res : p, V, u_resid[(size_t)b * (K + 1) + i], &b2);
-      path_band = dmin(path_band, b2);
+      note_band(&path_band, &path_kind, b2, ORACLE_BAND_E2);
     }
     if (!bad) {
       double bp = INFINITY;
@@ -215,19 +229,22 @@ int oracle_verify_linear(const double* target, const double* draft, int B, int K
       if (!bad && j == K) { /* whole block accepted: bonus draw from the last verifier row */
         double b2 = INFINITY;
         y = oracle_inverse_cdf(p, V, u_resid[(size_t)b * (K + 1) + K], &b2);
-        path_band = dmin(path_band, dmin(bp, b2));
+        note_band(&path_band, &path_kind, bp, ORACLE_BAND_E3);
+        note_band(&path_band, &path_kind, b2, ORACLE_BAND_E2);
       }
     }
     if (bad) {
       accept_len[b] = -1;
       for (int i = 0; i < K; ++i) { out_p[(size_t)b * K + i] = -1.0; out_q[(size_t)b * K + i] = -1.0; }
       band[b] = INFINITY;
+      if (band_kind) band_kind[b] = ORACLE_BAND_NONE;
       continue;
     }
     accept_len[b] = j;
     for (int i = 0; i < j; ++i) toks[i] = draft_tokens[(size_t)b * K + i];
     toks[j] = y;
     band[b] = path_band;
+    if (band_kind) band_kind[b] = path_kind;
   }
   free(p);
   free(q);
@@ -239,10 +256,10 @@ int oracle_verify_tree(const double* target, const double* draft, int B, int V,
                        const int* node_offsets, const int* parent, const int* tokens,
                        const double* u_accept, const double* u_resid,
                        const double* temperature, const double* top_p, const int* top_k, int max_depth,
-                       int* out_path, int* out_tokens, int* accept_len, double* band) {
+                       int* out_path, int* out_tokens, int* accept_len, double* band, int* band_kind) {
   return oracle_verify_tree_rule(target, draft, B, V, node_offsets, parent, tokens, u_accept, u_resid, temperature,
                                  top_p, top_k, max_depth, ORACLE_TREE_SAMPLED_WOR, out_path, out_tokens, accept_len,
-                                 band);
+                                 band, band_kind);
 }
 
 /* Tree verification under one of three candidate rules, the same walk for each: at the
@@ -264,7 +281,8 @@ int oracle_verify_tree_rule(const double* target, const double* draft, int B, in
                             const int* node_offsets, const int* parent, const int* tokens,
                             const double* u_accept, const double* u_resid,
                             const double* temperature, const double* top_p, const int* top_k, int max_depth,
-                            int rule, int* out_path, int* out_tokens, int* accept_len, double* band) {
+                            int rule, int* out_path, int* out_tokens, int* accept_len, double* band,
+                            int* band_kind) {
   if (B < 0 || V <= 0 || max_depth < 0) return ORACLE_BAD_ARG;
   if (rule != ORACLE_TREE_SAMPLED_WOR && rule != ORACLE_TREE_DETERMINISTIC && rule != ORACLE_TREE_SAMPLED_WR)
     return ORACLE_BAD_ARG;
@@ -281,6 +299,7 @@ int oracle_verify_tree_rule(const double* target, const double* draft, int B, in
     for (int i = 0; i <= max_depth; ++i) toks[i] = -1;
     accept_len[b] = -1;
     band[b] = INFINITY;
+    if (band_kind) band_kind[b] = ORACLE_BAND_NONE;
 
     /* structure checks: root first, parents precede children, depth within max_depth */
     int bad = n <= 0 || parent[n0] != -1;
@@ -295,16 +314,16 @@ int oracle_verify_tree_rule(const double* target, const double* draft, int B, in
     if (bad) continue;
 
     double path_band = INFINITY;
-    int cur = 0, len = 0, y = -1;
+    int cur = 0, len = 0, y = -1, path_kind = ORACLE_BAND_NONE;
     for (;;) {
       double b3 = INFINITY;
       if (oracle_row_dist_k(target + (size_t)(n0 + cur) * V, V, T, tp, tk, r, &b3) != 0) { bad = 1; break; }
-      path_band = dmin(path_band, b3);
+      note_band(&path_band, &path_kind, b3, ORACLE_BAND_E3);
       int has_child = 0;
       for (int c = cur + 1; c < n; ++c) has_child |= parent[n0 + c] == cur;
       if (has_child && T > 0.0 && rule != ORACLE_TREE_DETERMINISTIC) {
         if (oracle_row_dist_k(draft + (size_t)(n0 + cur) * V, V, T, tp, tk, qt, &b3) != 0) { bad = 1; break; }
-        path_band = dmin(path_band, b3);
+        note_band(&path_band, &path_kind, b3, ORACLE_BAND_E3);
       }
       int next = -1;
       for (int c = cur + 1; c < n && next < 0; ++c) {
@@ -316,7 +335,7 @@ int oracle_verify_tree_rule(const double* target, const double* draft, int B, in
         }
         if (rule == ORACLE_TREE_DETERMINISTIC) {
           const double ud = u_accept[n0 + c];
-          path_band = dmin(path_band, fabs(ud - r[t]));
+          note_band(&path_band, &path_kind, fabs(ud - r[t]), ORACLE_BAND_E1);
           if (ud < r[t]) { next = c; break; }
           /* rejected: [r - delta_t]_+ is r without t; renormalise */
           r[t] = 0.0;
@@ -330,7 +349,7 @@ int oracle_verify_tree_rule(const double* target, const double* draft, int B, in
         for (int v = 0; v < V; ++v) qmass += qt[v];
         if (!(qmass > 0.0)) break; /* draft mass exhausted: remaining siblings skipped */
         double u = u_accept[n0 + c];
-        if (qt[t] > 0.0) path_band = dmin(path_band, fabs(u - r[t] / qt[t]));
+        if (qt[t] > 0.0) note_band(&path_band, &path_kind, fabs(u - r[t] / qt[t]), ORACLE_BAND_E1);
         if (u * qt[t] < r[t]) { next = c; break; }
         /* rejected: r <- norm([r - qt]_+), then remove t from the draft and renormalise */
         double Z = 0.0;
@@ -357,7 +376,7 @@ int oracle_verify_tree_rule(const double* target, const double* draft, int B, in
       }
       double b2 = INFINITY;
       y = oracle_inverse_cdf(r, V, u_resid[n0 + cur], &b2);
-      path_band = dmin(path_band, b2);
+      note_band(&path_band, &path_kind, b2, ORACLE_BAND_E2);
       break;
     }
     if (bad) {
@@ -368,6 +387,7 @@ int oracle_verify_tree_rule(const double* target, const double* draft, int B, in
     toks[len] = y;
     accept_len[b] = len;
     band[b] = path_band;
+    if (band_kind) band_kind[b] = path_kind;
   }
   free(r);
   free(qt);

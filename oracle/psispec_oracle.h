@@ -24,7 +24,9 @@
  *   E2 |C(y-1)/Z - u|, |C(y)/Z - u|   for each inverse-CDF draw,
  *   E3 |tail(tau)/S - top_p|, |tail(tau+)/S - top_p|   for each top-p threshold used.
  * A comparison whose band is below the agreed tolerance may legitimately differ between
- * two correct implementations with different rounding.
+ * two correct implementations with different rounding. The optional band_kind outputs (NULL:
+ * not wanted) name the kind of the decision that gives the band: ORACLE_BAND_E1, _E2 or _E3,
+ * or ORACLE_BAND_NONE when the path holds no decision (or on a data error).
  */
 #ifndef PSISPEC_ORACLE_H
 #define PSISPEC_ORACLE_H
@@ -36,6 +38,12 @@ extern "C" {
 /* Return codes. Per-request data errors are reported through accept_len = -1 instead. */
 #define ORACLE_OK 0
 #define ORACLE_BAD_ARG 1
+
+/* Kinds of decision behind a band (band_kind outputs). */
+#define ORACLE_BAND_NONE 0
+#define ORACLE_BAND_E1 1 /* accept test |u - p/q| */
+#define ORACLE_BAND_E2 2 /* inverse-CDF draw edge */
+#define ORACLE_BAND_E3 3 /* top-p tail against top_p */
 
 /* One row's distribution after temperature T and top-p.
  * l[V] logits; T == 0 means greedy (a point mass on the lowest-index maximum).
@@ -57,10 +65,11 @@ int oracle_inverse_cdf(const double* r, int V, double u, double* band);
 /* Draft sampling, one draw per row.
  * draft[rows*V]; row_req[rows] maps a row to its request for temperature[]/top_p[]/top_k[]
  * (top_k may be NULL: off for every request);
- * u[rows]. Outputs: tokens[rows] (-1 on a bad row), q_at[rows] = q(token), band[rows]. */
+ * u[rows]. Outputs: tokens[rows] (-1 on a bad row), q_at[rows] = q(token), band[rows],
+ * band_kind[rows] (nullable). */
 int oracle_sample_draft(const double* draft, int rows, int V, const int* row_req,
                         const double* temperature, const double* top_p, const int* top_k, const double* u,
-                        int* tokens, double* q_at, double* band);
+                        int* tokens, double* q_at, double* band, int* band_kind);
 
 /* Linear verification.
  * target[B*(K+1)*V], draft[B*K*V], draft_tokens[B*K], u_accept[B*K], u_resid[B*(K+1)],
@@ -68,12 +77,13 @@ int oracle_sample_draft(const double* draft, int rows, int V, const int* row_req
  * Outputs: out_tokens[B*(K+1)] (accepted prefix, then the resampled or bonus token, then -1),
  * accept_len[B] (-1 on a data error), out_p[B*K] = p_i(x_i), out_q[B*K] = q_i(x_i),
  * band[B] = smallest E1/E2/E3 margin on the request's path,
- * pq_band[B*K] = E3 margin of the two rows behind out_p/out_q at that position. */
+ * pq_band[B*K] = E3 margin of the two rows behind out_p/out_q at that position,
+ * band_kind[B] (nullable) = the kind of decision that gives band[b]. */
 int oracle_verify_linear(const double* target, const double* draft, int B, int K, int V,
                          const int* draft_tokens, const double* u_accept, const double* u_resid,
                          const double* temperature, const double* top_p, const int* top_k,
                          int* out_tokens, int* accept_len, double* out_p, double* out_q,
-                         double* band, double* pq_band);
+                         double* band, double* pq_band, int* band_kind);
 
 /* Tree verification (recursive rejection without replacement over siblings).
  * node_offsets[B+1]: request b owns nodes [node_offsets[b], node_offsets[b+1]); the first is
@@ -82,12 +92,13 @@ int oracle_verify_linear(const double* target, const double* draft, int B, int K
  * the next-token rows at each node. u_accept[N] is consumed when a node is tested as a
  * candidate child; u_resid[N] when the final draw happens at that node.
  * Outputs: out_path[B*max_depth] local node ids of the accepted path (-1 padded),
- * out_tokens[B*(max_depth+1)], accept_len[B] (-1 on a data error), band[B]. */
+ * out_tokens[B*(max_depth+1)], accept_len[B] (-1 on a data error), band[B], band_kind[B]
+ * (nullable). */
 int oracle_verify_tree(const double* target, const double* draft, int B, int V,
                        const int* node_offsets, const int* parent, const int* tokens,
                        const double* u_accept, const double* u_resid,
                        const double* temperature, const double* top_p, const int* top_k, int max_depth,
-                       int* out_path, int* out_tokens, int* accept_len, double* band);
+                       int* out_path, int* out_tokens, int* accept_len, double* band, int* band_kind);
 
 /* Candidate rules of tree verification (oracle_verify_tree_rule). */
 #define ORACLE_TREE_SAMPLED_WOR 0    /* children drawn from q without replacement (R7) */
@@ -103,7 +114,8 @@ int oracle_verify_tree_rule(const double* target, const double* draft, int B, in
                             const int* node_offsets, const int* parent, const int* tokens,
                             const double* u_accept, const double* u_resid,
                             const double* temperature, const double* top_p, const int* top_k, int max_depth,
-                            int rule, int* out_path, int* out_tokens, int* accept_len, double* band);
+                            int rule, int* out_path, int* out_tokens, int* accept_len, double* band,
+                            int* band_kind);
 
 /* Candidate trie of the tree sampler from the draft rows of K positions (draft[K*V], after
  * temperature/top-p/top-k): the cand_k most probable tokens per position, then the n_prefixes

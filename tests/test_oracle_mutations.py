@@ -16,6 +16,7 @@ SRC = os.path.join(ROOT, "oracle", "psispec_oracle.c")
 
 PINS = ("test_oracle_pins.py", "test_oracle_lossless.py")
 TREE_BUILD = ("test_oracle_tree_build.py",)
+BANDS = ("test_oracle_bands.py",)
 
 MUTATIONS = {
     "accept_operands_swapped": ("if (u * q[x] < p[x]) continue;", "if (u * p[x] < q[x]) continue;"),
@@ -51,6 +52,47 @@ MUTATIONS = {
                                         "if (best < 0 || qi[v] >= qi[best]) best = v;", TREE_BUILD),
     "build_score_sum": ("score[nn] = score[pa] * q[(size_t)d * V + tokens[nn]];",
                         "score[nn] = score[pa] + q[(size_t)d * V + tokens[nn]];", TREE_BUILD),
+    # the exception bands (pinned in test_oracle_bands.py): a wrong band would exempt requests
+    # from the parity comparison, or leave near-ties unreported
+    "cdf_band_zero": ("*band = dmin(fabs(before / Z - u), fabs(C / Z - u));", "*band = 0.0;", BANDS),
+    "cdf_band_unscaled": ("*band = dmin(fabs(before / Z - u), fabs(C / Z - u));",
+                          "*band = dmin(fabs(before - u), fabs(C - u));", BANDS),
+    "cdf_band_upper_edge_only": ("*band = dmin(fabs(before / Z - u), fabs(C / Z - u));", "*band = fabs(C / Z - u);",
+                                 BANDS),
+    "topp_band_dropped": ("*band = dmin(fabs(tail / total - top_p), fabs(above / total - top_p));",
+                          "*band = INFINITY;", BANDS),
+    "topp_band_zero": ("*band = dmin(fabs(tail / total - top_p), fabs(above / total - top_p));", "*band = 0.0;",
+                       BANDS),
+    "topp_band_one_tail": ("*band = dmin(fabs(tail / total - top_p), fabs(above / total - top_p));",
+                           "*band = fabs(tail / total - top_p);", BANDS),
+    "ratio_band_dropped": ("if (q[x] > 0.0) note_band(&path_band, &path_kind, fabs(u - p[x] / q[x]), ORACLE_BAND_E1);",
+                           "(void)u;", BANDS),
+    "ratio_band_inverted": ("fabs(u - p[x] / q[x])", "fabs(u - q[x] / p[x])", BANDS),
+    "resid_band_dropped": ("u_resid[(size_t)b * (K + 1) + i], &b2);\n      note_band(&path_band, &path_kind, b2, "
+                           "ORACLE_BAND_E2);", "u_resid[(size_t)b * (K + 1) + i], &b2);", BANDS),
+    "bonus_band_dropped": ("        note_band(&path_band, &path_kind, bp, ORACLE_BAND_E3);\n"
+                           "        note_band(&path_band, &path_kind, b2, ORACLE_BAND_E2);",
+                           "        note_band(&path_band, &path_kind, bp, ORACLE_BAND_E3);", BANDS),
+    "band_past_rejection": ("      if (i > j) continue; /* past the first rejection: probabilities only */\n"
+                            "      double u = u_accept[(size_t)b * K + i];\n"
+                            "      note_band(&path_band, &path_kind, dmin(bp, bq), ORACLE_BAND_E3);\n"
+                            "      if (q[x] > 0.0) note_band(&path_band, &path_kind, fabs(u - p[x] / q[x]), "
+                            "ORACLE_BAND_E1);\n",
+                            "      double u = u_accept[(size_t)b * K + i];\n"
+                            "      note_band(&path_band, &path_kind, dmin(bp, bq), ORACLE_BAND_E3);\n"
+                            "      if (q[x] > 0.0) note_band(&path_band, &path_kind, fabs(u - p[x] / q[x]), "
+                            "ORACLE_BAND_E1);\n"
+                            "      if (i > j) continue;\n", BANDS),
+    "linear_topp_band_mislabelled": ("note_band(&path_band, &path_kind, dmin(bp, bq), ORACLE_BAND_E3);",
+                                     "note_band(&path_band, &path_kind, dmin(bp, bq), ORACLE_BAND_E1);", BANDS),
+    "sample_band_without_draw": ("note_band(&bi, &kind, b2, ORACLE_BAND_E2);", "(void)b2;", BANDS),
+    "sample_band_without_topp": ("note_band(&bi, &kind, b3, ORACLE_BAND_E3);", "(void)b3;", BANDS),
+    "tree_ratio_band_dropped": ("if (qt[t] > 0.0) note_band(&path_band, &path_kind, fabs(u - r[t] / qt[t]), "
+                                "ORACLE_BAND_E1);", "(void)u;", BANDS),
+    "tree_det_band_dropped": ("note_band(&path_band, &path_kind, fabs(ud - r[t]), ORACLE_BAND_E1);", "(void)ud;",
+                              BANDS),
+    "tree_draw_band_dropped": ("u_resid[n0 + cur], &b2);\n      note_band(&path_band, &path_kind, b2, ORACLE_BAND_E2);",
+                               "u_resid[n0 + cur], &b2);", BANDS),
 }
 
 
