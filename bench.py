@@ -3,11 +3,12 @@
 One step = the whole hot path over one batch: psispec_sample_draft over the [B, K, V] draft
 logits (token draw, q(x), per-row statistics), then psispec_verify_linear over the
 [B, K+1, V] verifier logits reusing those statistics (accept tests, first rejection,
-residual or bonus draw). Default workload "mid": B=64 requests, K=8 drafted positions,
-V=151936, bf16, T=1, no top-p. Inputs are synthetic (seeded) and already resident in HBM;
-together they are 330 MB, larger than the 126 MB L2, so no flush is needed between steps.
+residual or bonus draw). Default workload "max", the largest linear configuration: B=512
+requests, K=16 drafted positions, V=151936, bf16, T=1, top-p 0.95 on both distributions. Inputs
+are synthetic (seeded) and already resident in HBM; together they are 5.1 GB, far larger than
+the 126 MB L2, so no flush is needed between steps.
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload mid] [--impl ours|reference]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload max] [--impl ours|reference]
 
 Prints one JSON line (rank 0). With N > 1 (torchrun), every rank verifies its own batch; no
 collective touches the data path (only the max-over-ranks timing reduction).
@@ -161,7 +162,7 @@ def _rank_seed(seed: int, rank: int) -> int:
 
 def _oracle_sample(case, tgt_h, drf_h, ud, ua, ur, reqs):
     """The oracle (fp64 C, one thread) on requests `reqs` of the workload: draft draws then
-    verification, exactly the step the GPU runs."""
+    verification, exactly the step the GPU runs. Returns (draws, verification)."""
     import oracle
 
     K, V = case.K, case.V
@@ -172,11 +173,66 @@ def _oracle_sample(case, tgt_h, drf_h, ud, ua, ur, reqs):
     s = oracle.sample_draft(d.reshape(n * K, V), T, P, ud[reqs].reshape(-1), row_req=np.arange(n * K) // K, top_k=Kk)
     r = oracle.verify_linear(tgt_h[reqs].to(torch.float64).numpy(), d, s["tokens"].reshape(n, K), ua[reqs], ur[reqs],
                              T, P, top_k=Kk)
-    return r
+    return s, r
+
+
+def _host_threads():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def _oracle_parallel(case, tgt_h, drf_h, ud, ua, ur, reqs, threads):
+    """The same oracle calls, one request per task on `threads` host threads (the C oracle
+    runs outside the interpreter lock). Returns per-request (draws, verification) pairs."""
+    from concurrent.futures import ThreadPoolExecutor
+
+    with ThreadPoolExecutor(max_workers=threads) as ex:
+        return list(ex.map(lambda b: _oracle_sample(case, tgt_h, drf_h, ud, ua, ur, np.array([b])), reqs))
+
+
+def _exceptions(case, results, reqs, gpu_x, gpu_tok, gpu_len):
+    """Counted exceptions of the GPU results against the oracle on the sampled requests: draws
+    and verifications whose path holds a decision within 1e-6 of its boundary, by kind (E1
+    accept test, E2 draw edge, E3 top-p tail), how many of those differ, and any difference
+    outside the bands (none is allowed)."""
+    import oracle
+
+    kinds = {oracle.BAND_E1: "e1", oracle.BAND_E2: "e2", oracle.BAND_E3: "e3"}
+    out = {"requests_checked": 0, "rows_checked": 0, "e1": 0, "e2": 0, "e3": 0, "differ_in_band": 0,
+           "differ_outside_band": 0, "verify_skipped_draft_differs": 0}
+    K = case.K
+    for b, (s, r) in zip(reqs, results):
+        out["rows_checked"] += K
+        same_x = True
+        for i in range(K):
+            band, kind = float(s["band"][i]), int(s["band_kind"][i])
+            differs = int(gpu_x[b, i]) != int(s["tokens"][i])
+            same_x &= not differs
+            if band < oracle.E_BAND:
+                out[kinds.get(kind, "e2")] += 1
+                out["differ_in_band"] += int(differs)
+            elif differs:
+                out["differ_outside_band"] += 1
+        if not same_x:
+            out["verify_skipped_draft_differs"] += 1
+            continue
+        out["requests_checked"] += 1
+        band, kind = float(r["band"][0]), int(r["band_kind"][0])
+        differs = int(gpu_len[b]) != int(r["accept_len"][0]) or list(map(int, gpu_tok[b])) != list(
+            map(int, r["tokens"][0]))
+        if band < oracle.E_BAND:
+            out[kinds.get(kind, "e2")] += 1
+            out["differ_in_band"] += int(differs)
+        elif differs:
+            out["differ_outside_band"] += 1
+    return out
 
 
 def run_reference(args):
-    """The reference arm: the oracle timed on the host cores (rank 0 only)."""
+    """The reference arm: the oracle timed on the host cores (rank 0 only), one request per
+    host thread."""
     if int(os.environ.get("RANK", "0")) != 0:
         return
     from lossless_speculative_sampling_b200 import synth
@@ -184,21 +240,26 @@ def run_reference(args):
     if args.workload in synth.tree_cases():
         return _run_reference_tree(args)
     case = synth.linear_cases()[args.workload]
-    # about 80 ms of oracle work per request at V = 151936: keep the whole run near two minutes
-    n_req = max(1, min(args.ref_requests, int(120.0 / (0.08 * (args.steps + args.warmup)))))
+    threads = _host_threads()
+    # one request per host thread per step, bounded so that the whole run stays near two
+    # minutes (a request of the top-p workloads takes about a second on one thread)
+    per_req = 1.0 if case.top_p < 1.0 or case.top_k else 0.1
+    n_req = max(1, min(case.B, threads * args.ref_requests,
+                       int(threads * 120.0 / (per_req * (args.steps + args.warmup)))))
     tgt, drf = synth.linear_logits(case, device="cpu", B=n_req)
     ud, ua, ur = synth.linear_uniforms(case, B=n_req)
     reqs = np.arange(n_req)
     for _ in range(args.warmup):
-        _oracle_sample(case, tgt, drf, ud, ua, ur, reqs[:1])
+        _oracle_parallel(case, tgt, drf, ud, ua, ur, reqs[:threads], threads)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        _oracle_sample(case, tgt, drf, ud, ua, ur, reqs)
+        _oracle_parallel(case, tgt, drf, ud, ua, ur, reqs, threads)
     dt = (time.perf_counter() - t0) / args.steps
     value = n_req * case.K / dt
-    sample = "%d of %d requests of workload %s per step (fp64 C oracle, 1 thread)" % (n_req, case.B, args.workload)
+    sample = "%d of %d requests of workload %s per step (fp64 C oracle, one request per host thread, %d threads)" % (
+        n_req, case.B, args.workload, threads)
     _print_reference(args, value, dt, "f64", {"workload": args.workload, "requests_per_step": n_req, "block": case.K,
-                                              "vocab": case.V}, sample)
+                                              "vocab": case.V}, sample, cores=threads)
 
 
 def _run_reference_tree(args):
@@ -229,11 +290,12 @@ def _run_reference_tree(args):
                                                "vocab": case.V}, sample)
 
 
-def _print_reference(args, value, dt, dtype, config, sample):
+def _print_reference(args, value, dt, dtype, config, sample, cores=1):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": dtype, "data": "synthetic", "config": config,
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample,
+                             "host_cores": os.cpu_count()},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -274,7 +336,7 @@ def _prepare_linear(case, dev):
 
     return {
         "inputs": (tgt, drf), "calls": [("sample_draft", sample), ("verify_linear", verify)],
-        "outputs": (o_tok, o_len), "positions": B * K, "esz": esz,
+        "outputs": (o_tok, o_len), "draft_tokens": x, "positions": B * K, "esz": esz,
         # algorithmic bytes: sample_draft reads the draft tensor once; verify_linear reads the
         # verifier tensor once plus, per request, the one draft row of the residual draw
         "bytes": {"sample_draft": B * K * V * esz, "verify_linear": B * (K + 1) * V * esz + B * V * esz},
@@ -478,9 +540,9 @@ def run_ours(args):
     d2h = sum(o.numel() * o.element_size() for o in P["outputs"])
     del hosts, devs
 
-    cpu = None
+    cpu, exc = None, None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and args.workload in _linear_names():
-        cpu = _cpu_baseline(args, case, P)
+        cpu, exc = _cpu_baseline(args, case, P)
 
     peak, peak_kind = _peaks()
     main_call = P["calls"][-1][0]
@@ -508,9 +570,12 @@ def run_ours(args):
             # both-tensors-once (the tree walk reads only the rows of the nodes it visits)
             "logit_bytes_read_per_step": P["read_bytes"]() if "read_bytes" in P else None,
             "step_gbs": P["bytes_step"] / (ms_step * 1e-3) / 1e9,
+            "step_frac": P["bytes_step"] / (ms_step * 1e-3) / 1e9 / peak,
             "calls": dict({k + "_ms": v for k, v in per.items()},
                           **{k + "_gbs": P["bytes"][k] / (v * 1e-3) / 1e9 for k, v in per.items()}),
             "mean_accept_len": mean_accept,
+            # the GPU's results on the requests the oracle leg computed (1e-6 bands by kind)
+            "exceptions": exc,
             "e2e": {"value": world * P["positions"] / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
             "gpu_launches": P["launches"] * args.steps,
@@ -529,21 +594,45 @@ def _linear_names():
 
 
 def _cpu_baseline(args, case, P):
-    """The oracle as it stands, on a bounded sample of the same workload (host cores)."""
+    """The oracle as it stands, on a bounded sample of the same workload (host cores): one
+    thread, then one request per host thread; its results on the sampled requests are also the
+    exception counts of the GPU's results (returned separately)."""
     from lossless_speculative_sampling_b200 import synth
 
     B, K = case.B, case.K
     tgt_c, drf_c = (t.cpu() for t in P["inputs"])
     udc, uac, urc = synth.linear_uniforms(synth.linear_cases()[args.workload])
-    n = 0
+    threads = _host_threads()
+    # single thread: requests spread over the batch until about half the time budget is spent
+    order = np.unique(np.linspace(0, B - 1, B).astype(int))[::max(1, B // 64)]
+    done, results = [], []
     t0 = time.perf_counter()
-    while time.perf_counter() - t0 < args.cpu_seconds and n < B:
-        _oracle_sample(case, tgt_c, drf_c, udc, uac, urc, np.arange(n, min(B, n + 4)))
-        n = min(B, n + 4)
-    dt = time.perf_counter() - t0
-    return {"value": n * K / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": "%d of %d requests of workload %s (sample_draft + verify_linear, fp64 C oracle, "
-                      "single thread, %.1f s)" % (n, B, args.workload, dt)}
+    for b in order:
+        if time.perf_counter() - t0 >= args.cpu_seconds / 2:
+            break
+        results.append(_oracle_sample(case, tgt_c, drf_c, udc, uac, urc, np.array([b])))
+        done.append(int(b))
+    dt1 = time.perf_counter() - t0
+    one = len(done) * K / dt1
+    # one request per host thread: as many requests as one thread did per thread, bounded by B
+    n_par = int(min(B, max(threads, len(done) * threads)))
+    par = np.linspace(0, B - 1, n_par).astype(int)
+    t0 = time.perf_counter()
+    res_par = _oracle_parallel(case, tgt_c, drf_c, udc, uac, urc, par, threads)
+    dtp = time.perf_counter() - t0
+    many = n_par * K / dtp
+    x = P["draft_tokens"].cpu().numpy()
+    tok, ln = (o.cpu().numpy() for o in P["outputs"])
+    seen = set(done)
+    all_reqs = done + [int(b) for b in par if int(b) not in seen]
+    all_res = results + [r for b, r in zip(par, res_par) if int(b) not in seen]
+    exc = _exceptions(case, all_res, all_reqs, x, tok, ln)
+    cpu = {"value": many, "unit": UNIT, "cores": threads, "kind": "oracle", "host_cores": os.cpu_count(),
+           "single_thread_value": one,
+           "sample": "workload %s (sample_draft + verify_linear, fp64 C oracle): %d requests on 1 thread in %.1f s, "
+                     "then %d requests spread over the batch, one per host thread on %d threads, in %.1f s" % (
+                         args.workload, len(done), dt1, n_par, threads, dtp)}
+    return cpu, exc
 
 
 def main():
@@ -551,12 +640,12 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=500)
     ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--workload", default="mid")
+    ap.add_argument("--workload", default="max")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="launch calls directly instead of replaying CUDA graphs")
-    ap.add_argument("--cpu-seconds", type=float, default=15.0)
-    ap.add_argument("--ref-requests", type=int, default=2)
+    ap.add_argument("--cpu-seconds", type=float, default=20.0)
+    ap.add_argument("--ref-requests", type=int, default=2, help="requests per host thread in a reference step")
     ap.add_argument("--all", action="store_true", help="one line per full-size workload instead of the bench line")
     args = ap.parse_args()
     if args.impl == "reference":

@@ -592,6 +592,9 @@ psispec_status psispec_verify_linear_static(const void* target_logits, const voi
                                             const float* top_p, int32_t* out_tokens, int32_t* out_accept_len,
                                             float* out_p, float* out_q, void* stream) {
   if (B <= 0 || K <= 0 || V <= 0) return PSISPEC_ERR_INVALID_ARG;
+  // the limits of psispec_verify_linear first, so that both calls report them alike
+  if (K > 64 || int64_t(B) * (K + 1) > kMaxRows || V > kMaxV || int64_t(B) * (K + 1) * nslices_for(V) > kMaxGrid)
+    return PSISPEC_ERR_UNSUPPORTED;
   const size_t need = psispec_workspace_size(PSISPEC_OP_VERIFY_LINEAR, B, K, V);
   if (need == 0) return PSISPEC_ERR_INVALID_ARG;
   if (need > static_cast<size_t>(PSISPEC_STATIC_WORKSPACE_BYTES)) return PSISPEC_ERR_UNSUPPORTED;

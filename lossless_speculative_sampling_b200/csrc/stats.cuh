@@ -429,6 +429,7 @@ __global__ void __launch_bounds__(kThreads) stream_partials_tma_kernel(RowSet<T>
     const int req = rows.request(r);
     return table ? scale[req] : stream_scale(temperature, top_p, skip_uncut, req);
   };
+  uint32_t pending = 0u;  // (lane 0) stages with a copy in flight
   auto issue = [&](int i) {  // copy of this warp's i-th chunk into stage i % kRing (lane 0)
     if (gi < total_chunks && scale_of(irow) >= 0.0f) {
       const int c0 = ichunk * kChunkElems, n = min(V - c0, kChunkElems);
@@ -436,6 +437,7 @@ __global__ void __launch_bounds__(kThreads) stream_partials_tma_kernel(RowSet<T>
       uint64_t* b = &bar[i % kRing];
       mbar_expect_tx(b, bytes);
       bulk_g2s(ring + (i % kRing) * kStageBytes<T>, rows.row(irow, V) + c0, bytes, b);
+      pending |= 1u << (i % kRing);
     }
     gi += nwarps;
     advance(irow, ichunk);
@@ -454,13 +456,25 @@ __global__ void __launch_bounds__(kThreads) stream_partials_tma_kernel(RowSet<T>
       continue;
     }
     const int st = i % kRing;
-    const bool landed = mbar_wait_bounded(&bar[st], (phase_bits >> st) & 1u);
-    phase_bits ^= 1u << st;
+    const uint32_t parity = (phase_bits >> st) & 1u;
+    const bool landed = mbar_wait_bounded(&bar[st], parity);
     if (!__all_sync(0xffffffffu, landed)) {
-      // a copy that never completed: report this chunk as a data error and stop streaming
-      if (lane == 0) parts[g] = Partial{0.0, NAN, 0, 1, 0};
+      // a copy that never completed: this chunk and every later chunk of this warp are reported
+      // as data errors (their rows end with status 1), nothing more is issued, and the copies
+      // still in flight get a bounded wait before the warp leaves (they write this CTA's
+      // shared memory)
+      if (lane == 0) {
+        for (int64_t h = g; h < total_chunks; h += nwarps) {
+          if (scale_of(row) >= 0.0f) parts[h] = Partial{0.0, NAN, 0, 1, 0};
+          advance(row, chunk);
+        }
+        for (int s = 0; s < kRing; ++s)
+          if ((pending >> s) & 1u) mbar_wait_bounded(&bar[s], s == st ? parity : (phase_bits >> s) & 1u);
+      }
       return;
     }
+    phase_bits ^= 1u << st;
+    pending &= ~(1u << st);
     const T* sp = reinterpret_cast<const T*>(ring + st * kStageBytes<T>);
     const Partial p = c == 0.0f ? warp_chunk_partial_smem<T, true>(sp, c0, n, c)
                                 : warp_chunk_partial_smem<T, false>(sp, c0, n, c);

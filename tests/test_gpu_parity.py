@@ -13,7 +13,8 @@ import torch
 
 import oracle
 from goldens import load, nums, rows
-from parity import compare_linear, compare_sample, compare_tree
+from parity import (band_limit, compare_linear, compare_sample, compare_tree, linear_recheck, sample_recheck,
+                    tree_recheck)
 from lossless_speculative_sampling_b200 import psispec, synth
 
 pytestmark = pytest.mark.gpu
@@ -30,6 +31,29 @@ def _rand_logits(g, shape, dtype, std=2.0, neg_inf_frac=0.0):
     if neg_inf_frac:
         x[torch.rand(shape, generator=g) < neg_inf_frac] = -float("inf")
     return x.to(dtype)
+
+
+def check_linear(out, ora, tgt, drf, x, ua, ur, Ts, Ps, Ks=None, label="", check_pq=True):
+    """compare_linear with the oracle recheck of in-band requests and the in-band bound."""
+    B, K1, V = tgt.shape
+    cut = bool((np.asarray(Ps) < 1).any()) or Ks is not None
+    return compare_linear(out, ora, check_pq=check_pq, recheck=linear_recheck(tgt, drf, x, ua, ur, Ts, Ps, Ks),
+                          limit=band_limit(B, V, 1.0, 2 * K1 - 1 if cut else 0), label=label)
+
+
+def check_sample(tok, q, ora, drf_rows, Ts, Ps, u, row_req, Ks=None, label=""):
+    n, V = drf_rows.shape
+    cut = bool((np.asarray(Ps) < 1).any()) or Ks is not None
+    return compare_sample(tok, q, ora, recheck=sample_recheck(drf_rows, Ts, Ps, u, row_req, Ks),
+                          limit=band_limit(n, V, 1.0, 1 if cut else 0), label=label)
+
+
+def check_tree(out, ora, tgt, drf, offs, parent, toks, ua, ur, Ts, Ps, D, Ks=None, label=""):
+    N, V = tgt.shape
+    B = len(offs) - 1
+    cut = bool((np.asarray(Ps) < 1).any()) or Ks is not None
+    return compare_tree(out, ora, recheck=tree_recheck(tgt, drf, offs, parent, toks, ua, ur, Ts, Ps, D, Ks),
+                        limit=band_limit(B, V, 1.0, 2 * N / B if cut else 0), label=label)
 
 
 # ------------------------------------------------------------------ worked examples
@@ -95,7 +119,8 @@ def test_sample_draft_parity(B, K, V, dtype, T, top_p, noise):
     tgt, drf, ud, ua, ur, Ts, Ps = _linear_inputs(B, K, V, dtype, T, top_p, noise, seed=V + K)
     tok, q, _ = psispec.sample_draft(_cuda(drf), _cuda(Ts), _cuda(Ps), _cuda(ud))
     ora = oracle.sample_draft(drf.reshape(B * K, V), Ts.numpy(), Ps.numpy(), ud.reshape(-1), row_req=np.arange(B * K) // K)
-    compare_sample(tok, q, ora)
+    check_sample(tok, q, ora, drf.reshape(B * K, V), Ts, Ps, ud, np.arange(B * K) // K,
+                 label="sample %s" % ((B, K, V, T, top_p),))
 
 
 def _decode_stats(rec):
@@ -149,7 +174,7 @@ def test_row_stats_parity(B, K, V, dtype, T, top_p):
     out = psispec.verify_linear(_cuda(tgt), _cuda(drf), _cuda(x), _cuda(ua), _cuda(ur), _cuda(Ts), _cuda(Ps),
                                 draft_row_stats=rec)
     ora = oracle.verify_linear(tgt, drf, x, ua, ur, Ts.numpy(), Ps.numpy())
-    compare_linear(out, ora)
+    check_linear(out, ora, tgt, drf, x, ua, ur, Ts, Ps, label="row-stats records %s" % ((B, K, V, T, top_p),))
 
 
 @pytest.mark.parametrize("use_stats", [False, True])
@@ -164,7 +189,7 @@ def test_verify_linear_parity(B, K, V, dtype, T, top_p, noise, use_stats):
     out = psispec.verify_linear(_cuda(tgt), _cuda(drf), _cuda(x), _cuda(ua), _cuda(ur), _cuda(Ts), _cuda(Ps),
                                 draft_row_stats=stats)
     ora = oracle.verify_linear(tgt, drf, x.numpy(), ua, ur, Ts.numpy(), Ps.numpy())
-    compare_linear(out, ora)
+    check_linear(out, ora, tgt, drf, x, ua, ur, Ts, Ps, label="verify %s" % ((B, K, V, T, top_p, use_stats),))
 
 
 def test_verify_linear_mixed_requests_and_data_errors():
@@ -181,7 +206,7 @@ def test_verify_linear_mixed_requests_and_data_errors():
     out = psispec.verify_linear(_cuda(tgt), _cuda(drf), _cuda(x), _cuda(ua), _cuda(ur), _cuda(Ts), _cuda(Ps))
     ora = oracle.verify_linear(tgt, drf, x, ua, ur, Ts.numpy(), Ps.numpy())
     assert ora["accept_len"][4] == ora["accept_len"][5] == ora["accept_len"][6] == -1
-    compare_linear(out, ora)
+    check_linear(out, ora, tgt, drf, x, ua, ur, Ts, Ps, label="mixed requests")
 
 
 @pytest.mark.parametrize("V,T,top_p", [(40000, 100.0, 0.9), (40000, 30.0, 0.5), ((1 << 19) + 1000, 1.0, 0.9)])
@@ -203,11 +228,12 @@ def test_topp_fallback_paths(V, T, top_p):
     tok, q, _ = psispec.sample_draft(_cuda(drf), _cuda(Ts), _cuda(Ps), _cuda(ud))
     o_s = oracle.sample_draft(drf.reshape(B * K, V), Ts.numpy(), Ps.numpy(), ud.reshape(-1),
                               row_req=np.arange(B * K) // K)
-    compare_sample(tok, q, o_s)
+    check_sample(tok, q, o_s, drf.reshape(B * K, V), Ts, Ps, ud, np.arange(B * K) // K,
+                 label="fallback sample %s" % ((V, T, top_p),))
     x = o_s["tokens"].reshape(B, K).astype(np.int32)
     out = psispec.verify_linear(_cuda(tgt), _cuda(drf), _cuda(x), _cuda(ua), _cuda(ur), _cuda(Ts), _cuda(Ps))
     ora = oracle.verify_linear(tgt, drf, x, ua, ur, Ts.numpy(), Ps.numpy())
-    compare_linear(out, ora)
+    check_linear(out, ora, tgt, drf, x, ua, ur, Ts, Ps, label="fallback verify %s" % ((V, T, top_p),))
 
 
 TOPK_GRID = [
@@ -234,12 +260,13 @@ def test_topk_parity(B, K, V, dtype, T, top_p, top_k, use_stats):
     tok, q, rec = psispec.sample_draft(_cuda(drf), _cuda(Ts), _cuda(Ps), _cuda(ud), top_k=_cuda(Ks))
     o_s = oracle.sample_draft(drf.reshape(B * K, V), Ts.numpy(), Ps.numpy(), ud.reshape(-1),
                               row_req=np.arange(B * K) // K, top_k=Ks.numpy())
-    compare_sample(tok, q, o_s)
+    check_sample(tok, q, o_s, drf.reshape(B * K, V), Ts, Ps, ud, np.arange(B * K) // K, Ks,
+                 label="top-k sample %s" % ((B, K, V, T, top_p, top_k),))
     x = o_s["tokens"].reshape(B, K).astype(np.int32)
     out = psispec.verify_linear(_cuda(tgt), _cuda(drf), _cuda(x), _cuda(ua), _cuda(ur), _cuda(Ts), _cuda(Ps),
                                 top_k=_cuda(Ks), draft_row_stats=rec if use_stats else None)
     ora = oracle.verify_linear(tgt, drf, x, ua, ur, Ts.numpy(), Ps.numpy(), top_k=Ks.numpy())
-    compare_linear(out, ora)
+    check_linear(out, ora, tgt, drf, x, ua, ur, Ts, Ps, Ks, label="top-k verify %s" % ((B, K, V, T, top_p, top_k),))
 
 
 def test_q_equals_p_accepts_all_on_gpu():
@@ -283,7 +310,8 @@ def test_verify_tree_parity(V, dtype, T, top_p):
                               _cuda(ua), _cuda(ur), _cuda(Ts), _cuda(Ps), 6)
     ora = oracle.verify_tree(tgt, drf, trie.node_offsets.numpy(), trie.parent.numpy(), toks.numpy(), ua, ur,
                              Ts.numpy(), Ps.numpy(), 6)
-    compare_tree(out, ora)
+    check_tree(out, ora, tgt, drf, trie.node_offsets, trie.parent, toks, ua, ur, Ts, Ps, 6,
+               label="tree %s" % ((V, T, top_p),))
 
 
 @pytest.mark.parametrize("V,dtype", [(20011, torch.bfloat16), (3001, torch.float32), (151936, torch.bfloat16)])
@@ -317,7 +345,7 @@ def test_verify_tree_mixed_requests_and_data_errors(V, dtype):
                              Ps.numpy(), 6)
     assert ora["accept_len"][4] == ora["accept_len"][5] == ora["accept_len"][6] == -1
     assert (ora["accept_len"][[0, 1, 2, 3]] >= 0).all()
-    compare_tree(out, ora)
+    check_tree(out, ora, tgt, drf, off, trie.parent, toks, ua, ur, Ts, Ps, 6, label="mixed tries V=%d" % V)
 
 
 def test_verify_tree_structure_errors():
@@ -368,7 +396,9 @@ def test_verify_tree_structure_errors():
     assert (ora["accept_len"][[1, 2, 3, 4, 6]] == -1).all(), ora["accept_len"]
     assert (g_len[[0, 7]] >= 0).all()
     keep = [0, 1, 2, 3, 4, 6, 7]  # request 5 is beyond the walk's limit only
-    compare_tree({k: v[keep] for k, v in out.items()}, {k: np.asarray(v)[keep] for k, v in ora.items()})
+    rep = compare_tree({k: v[keep] for k, v in out.items()}, {k: np.asarray(v)[keep] for k, v in ora.items()},
+                       label="malformed tries")
+    assert rep["differ_in_band"] == 0
 
 
 def test_branching_one_tree_equals_linear_gpu():
@@ -413,7 +443,9 @@ def test_full_size_linear_sampled(name):
     Kp = Ks[pick].numpy() if case.top_k else None
     o_s = oracle.sample_draft(d_host.reshape(-1, V), Ts[pick].numpy(), Ps[pick].numpy(), ud[pick].reshape(-1),
                               row_req=np.arange(len(pick) * K) // K, top_k=Kp)
-    compare_sample(x[idx], q[idx], o_s)
+    rows_req = np.arange(len(pick) * K) // K
+    check_sample(x[idx], q[idx], o_s, d_host.reshape(-1, V), Ts[pick], Ps[pick], ud[pick], rows_req, Kp,
+                 label="full-size sample %s" % name)
     # the oracle's draft tokens replace the sampled requests' rows
     x_in = x.clone()
     x_in[idx] = torch.from_numpy(o_s["tokens"].reshape(len(pick), K)).to(DEV)
@@ -422,7 +454,8 @@ def test_full_size_linear_sampled(name):
     ora = oracle.verify_linear(tgt[idx].cpu(), d_host, o_s["tokens"].reshape(len(pick), K), ua[pick], ur[pick],
                                Ts[pick].numpy(), Ps[pick].numpy(), top_k=Kp)
     sub = {k: v[idx] for k, v in out.items()}
-    stats_report = compare_linear(sub, ora)
+    stats_report = check_linear(sub, ora, tgt[idx].cpu(), d_host, o_s["tokens"].reshape(len(pick), K), ua[pick],
+                                ur[pick], Ts[pick], Ps[pick], Kp, label="full-size verify %s" % name)
     lens = out["accept_len"].cpu().numpy()
     assert (lens >= 0).all() and (lens <= K).all()
     print(name, stats_report, "gpu mean accept", lens.mean())
@@ -437,7 +470,9 @@ def test_full_size_tree():
                               _cuda(Ts), _cuda(Ps), case.max_depth)
     ora = oracle.verify_tree(tgt.cpu(), drf.cpu(), trie.node_offsets.numpy(), trie.parent.numpy(), toks.numpy(), ua, ur,
                              Ts.numpy(), Ps.numpy(), case.max_depth)
-    print("tree", compare_tree(out, ora), "accept", out["accept_len"].tolist())
+    rep = check_tree(out, ora, tgt.cpu(), drf.cpu(), trie.node_offsets, trie.parent, toks, ua, ur, Ts, Ps,
+                     case.max_depth, label="full-size tree")
+    print("tree", rep, "accept", out["accept_len"].tolist())
 
 
 # ------------------------------------------------------------------ top-k: mixed requests and negative rows
@@ -454,12 +489,13 @@ def test_topk_mixed_requests(dtype):
     tok, q, _ = psispec.sample_draft(_cuda(drf), _cuda(Ts), _cuda(Ps), _cuda(ud), top_k=_cuda(Ks))
     o_s = oracle.sample_draft(drf.reshape(B * K, V), Ts.numpy(), Ps.numpy(), ud.reshape(-1),
                               row_req=np.arange(B * K) // K, top_k=Ks.numpy())
-    compare_sample(tok, q, o_s)
+    check_sample(tok, q, o_s, drf.reshape(B * K, V), Ts, Ps, ud, np.arange(B * K) // K, Ks,
+                 label="top-k mixed sample %s" % dtype)
     x = o_s["tokens"].reshape(B, K).astype(np.int32)
     out = psispec.verify_linear(_cuda(tgt), _cuda(drf), _cuda(x), _cuda(ua), _cuda(ur), _cuda(Ts), _cuda(Ps),
                                 top_k=_cuda(Ks))
     ora = oracle.verify_linear(tgt, drf, x, ua, ur, Ts.numpy(), Ps.numpy(), top_k=Ks.numpy())
-    compare_linear(out, ora)
+    check_linear(out, ora, tgt, drf, x, ua, ur, Ts, Ps, Ks, label="top-k mixed verify %s" % dtype)
     # a null top-k array and an all-off one agree with the entry points without top-k
     off = torch.zeros(B, dtype=torch.int32)
     a = psispec.verify_linear(_cuda(tgt), _cuda(drf), _cuda(x), _cuda(ua), _cuda(ur), _cuda(Ts), _cuda(Ps),
@@ -481,12 +517,13 @@ def test_negative_logit_rows(top_p, top_k):
     tok, q, _ = psispec.sample_draft(_cuda(drf), _cuda(Ts), _cuda(Ps), _cuda(ud), top_k=_cuda(Ks))
     o_s = oracle.sample_draft(drf.reshape(B * K, V), Ts.numpy(), Ps.numpy(), ud.reshape(-1),
                               row_req=np.arange(B * K) // K, top_k=Ks.numpy())
-    compare_sample(tok, q, o_s)
+    check_sample(tok, q, o_s, drf.reshape(B * K, V), Ts, Ps, ud, np.arange(B * K) // K, Ks,
+                 label="negative rows sample %s" % ((top_p, top_k),))
     x = o_s["tokens"].reshape(B, K).astype(np.int32)
     out = psispec.verify_linear(_cuda(tgt), _cuda(drf), _cuda(x), _cuda(ua), _cuda(ur), _cuda(Ts), _cuda(Ps),
                                 top_k=_cuda(Ks))
     ora = oracle.verify_linear(tgt, drf, x, ua, ur, Ts.numpy(), Ps.numpy(), top_k=Ks.numpy())
-    compare_linear(out, ora)
+    check_linear(out, ora, tgt, drf, x, ua, ur, Ts, Ps, Ks, label="negative rows verify %s" % ((top_p, top_k),))
 
 
 # ------------------------------------------------------------------ top-k: tree and row statistics
@@ -504,7 +541,8 @@ def test_verify_tree_topk_parity(V, dtype, T, top_p):
                               _cuda(ua), _cuda(ur), _cuda(Ts), _cuda(Ps), 6, top_k=_cuda(Ks))
     ora = oracle.verify_tree(tgt, drf, trie.node_offsets.numpy(), trie.parent.numpy(), toks.numpy(), ua, ur,
                              Ts.numpy(), Ps.numpy(), 6, top_k=Ks.numpy())
-    compare_tree(out, ora)
+    check_tree(out, ora, tgt, drf, trie.node_offsets, trie.parent, toks, ua, ur, Ts, Ps, 6, Ks,
+               label="top-k tree %s" % ((V, T, top_p),))
 
 
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])

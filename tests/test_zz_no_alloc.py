@@ -27,6 +27,11 @@ def test_static_rejects_oversize_before_any_cuda_call():
                                           FAKE, FAKE, FAKE, None, None, None) == psispec.ERR_INVALID_ARG
     # the mid-size workload fits
     assert psispec.workspace_size(psispec.OP_VERIFY_LINEAR, 64, 8, 151936) <= psispec.STATIC_WORKSPACE_BYTES
+    # sizes beyond the limits of psispec_verify_linear are unsupported, as they are there
+    for B, K, V in ((1, 65, 1000), (1, 4, (1 << 24) + 1)):
+        st = L.psispec_verify_linear_static(FAKE, FAKE, psispec.BF16, B, K, V, FAKE, None, FAKE, FAKE, FAKE, FAKE,
+                                            FAKE, FAKE, None, None, None)
+        assert st == psispec.ERR_UNSUPPORTED, (B, K, V, st)
 
 
 @pytest.mark.gpu
@@ -52,10 +57,18 @@ def test_static_matches_workspace_call_twice(use_stats):
              "out_accept_len": torch.full((B,), -7, dtype=torch.int32, device=dev),
              "out_p": torch.full((B, K), -7.0, device=dev), "out_q": torch.full((B, K), -7.0, device=dev)}
         outs.append(o)
+    # a first call may load the module and look up the array's address; after it, the device's
+    # free memory must not move: the library allocates nothing (torch's allocator would not see
+    # a cudaMalloc made by the library, the driver's count does)
+    psispec.verify_linear_static(tgt, drf, tok, ua, ur, Ts, Ps, draft_row_stats=ds, **outs[0])
+    for t in outs[0].values():
+        t.fill_(-7)
     torch.cuda.synchronize()
+    free0 = torch.cuda.mem_get_info(dev)[0]
     for o in outs:  # two calls in a row, nothing allocated between them
         psispec.verify_linear_static(tgt, drf, tok, ua, ur, Ts, Ps, draft_row_stats=ds, **o)
     torch.cuda.synchronize()
+    assert torch.cuda.mem_get_info(dev)[0] == free0
     for o in outs:
         assert torch.equal(o["out_tokens"], ref["tokens"])
         assert torch.equal(o["out_accept_len"], ref["accept_len"])
