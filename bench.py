@@ -343,7 +343,11 @@ def _prepare_linear(case, dev):
         "bytes_step": (B * (K + 1) + B * K) * V * esz,
         # stream + sample rows; stream + verify rows + cluster draw
         "launches": 2 + 3,
-        "kernel_leg": ("stream_partials_tma_kernel (psispec_row_stats over the verifier tensor)", stream_leg,
+        # the dominant kernel: with a cut (top-p / top-k, bf16), the one-pass cut-row CTAs
+        # (cut_rows_kernel, the launch psispec_row_stats makes for them; the streaming pass and
+        # the finalize there find no rows and return at once); without one, the streaming pass
+        "kernel_leg": (("cut_rows_kernel" if (case.top_p < 1.0 or case.top_k) and esz == 2 else
+                        "stream_partials_tma_kernel") + " (psispec_row_stats over the verifier tensor)", stream_leg,
                        B * (K + 1) * V * esz),
         "describe": "linear verify B=%d K=%d V=%d %s, T=%g, top-p %g%s" % (
             B, K, V, "bf16" if esz == 2 else "fp32", case.temperature, case.top_p,

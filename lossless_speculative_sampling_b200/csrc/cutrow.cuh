@@ -1,0 +1,532 @@
+// cutrow.cuh -- rows of requests with a cut (top-p below 1 or an active top-k, at T > 0),
+// bf16, in one pass over HBM.
+//
+// The cut keeps every token whose logit is at least tau, the largest logit value t of the row
+// with mass(l >= t) >= top_p (review page of arXiv 2609.04010: the samplers take --top-p with
+// --temperature; ties are kept together), and renormalises over the kept set; with a top-k
+// (the README's --top-k), mass and tail are those of the tokens at or above the k-th largest
+// logit. Every element with one bf16 value has one weight, so counting the elements of each
+// value just below the row maximum gives the masses the cut is decided on (window_pick,
+// topp.cuh). The two-pass select counts them after a statistics pass has found the maximum;
+// here the counts are taken in the same pass that finds it.
+//
+// One CTA per row at a time, persistent over the rows. Warp w of the CTA streams a contiguous
+// range of the row once from HBM (16-byte loads, the next step's loads in flight while the
+// current step is reduced) and keeps, over its range:
+//   - the running maximum M (NaN-propagating, bf16 pairs compared packed) and, per lane, the
+//     fp64 sum of 2^((x - M) c), rescaled whenever M grows;
+//   - a ring of kCrRing counters in shared memory, counter d counting the elements whose
+//     16-bit order key is base - d. The base is set kCrHead keys above the warp's maximum at
+//     its first finite value and moved up (counters shifted) only when the maximum passes
+//     it, so the counters cover the kTpWindow keys below the warp's maximum at every moment,
+//     hence also the kTpWindow keys below the row's maximum at the end.
+// The CTA then combines its warps: the maximum m, the normaliser s (fp64), and the counts of
+// the window below m, from which window_pick finds tau and the kept mass. A draft row draws
+// its token at once: the warps' kept masses (counts x weights) give the warp whose range holds
+// u * Z, and only that range is read again (from L2) to find the token. A verifier row (or a
+// draft row that a verification reads) writes its record and arrives on its request's
+// counter; the last arrival runs the accept tests. A row whose cut lies outside the window is
+// finished in place by the general selects of topp.cuh and stats.cuh (the row is read again).
+// The same CTAs take fp32 rows with the general selects throughout.
+#pragma once
+
+#include "common.cuh"
+#include "finish.cuh"
+#include "linear.cuh"
+#include "sample.cuh"
+#include "stats.cuh"
+#include "topp.cuh"
+
+namespace psi {
+
+constexpr int kCrWarps = 8;                   // warps per CTA, each one contiguous range of the row
+constexpr int kCrThreads = kCrWarps * 32;
+constexpr int kCrHead = 256;                  // keys of headroom above a warp's maximum at its ring base
+constexpr int kCrRing = kTpWindow + kCrHead;  // counters per warp
+constexpr int kCrVec = 4;                     // 16-byte vectors per lane per step
+static_assert(kCrRing % 32 == 0, "ring shifts move 32 counters per step");
+
+enum CutMode : int { kCutSample = 0, kCutVerify = 1, kCutStats = 2 };
+
+// Rows of one cut-row launch: rows [0, rows_a) of tensor a (per_a rows per request), then
+// rows [0, rows_b) of tensor b (per_b rows per request). Sampling: a = the draft rows [B, K].
+// Verification: a = the verifier rows [B, K+1], b = the draft rows [B, K] when the call reads
+// them. Row statistics: a = the rows [B, K].
+struct CutArgs {
+  int mode;
+  int V;
+  int rows_a, per_a, rows_b, per_b;
+  const float* temperature;
+  const float* top_p;
+  const int32_t* top_k;  // per request, or null (off)
+  const float* u;        // kCutSample: one uniform per row
+  int32_t* out_tokens;   // kCutSample: the drawn token per row
+  float* out_q;          // kCutSample: its kept probability (nullable)
+  RowStat* stats_a;      // records of tensor a's rows
+  RowStat* stats_b;      // records of tensor b's rows
+};
+
+struct CrSmem {
+  uint32_t ring[kCrWarps][kCrRing];
+  float wm[kCrWarps];     // the warps' maxima (-inf: no finite value in the range)
+  double ws[kCrWarps];    // the warps' sums, relative to their own maxima
+  uint32_t wb[kCrWarps];  // the warps' ring bases
+  int wbad[kCrWarps];     // a NaN or +inf logit in the warp's range
+  double wk[kCrWarps];    // the warps' kept masses (draft rows)
+  double scan[40];
+  double tgt, base, dtarget, dbase;
+  int bin, flag, dwarp;
+  DrawSmem draw;
+};
+
+// One warp's running state over its range (uniform across the warp except s).
+struct CrLane {
+  float M;        // running maximum; -inf before the first finite value
+  float nmc;      // -M c
+  uint32_t base;  // ring base key; 0 before the first finite value
+  uint32_t kb;    // base - 0x8000: the raw-bit base of the positive-only path
+  bool fast;      // every key the ring covers belongs to a positive value
+  bool bad;       // a NaN or +inf logit
+  double s;       // this lane's sum of 2^((x - M) c)
+};
+
+// The 16-bit order key of a bf16 bit pattern (fkey(x) >> 16 of the widened value; -0 and +0
+// share the key of +0).
+__device__ __forceinline__ uint32_t key16_bits(uint32_t h) {
+  return (h & 0x8000u) ? (h == 0x8000u ? 0x8000u : (~h & 0xFFFFu)) : (h | 0x8000u);
+}
+
+// The warp's maximum grew to bm (finite): rescale the lane sums and, when bm's key passes the
+// ring base (or at the first finite value), move the base kCrHead keys above it. Counter d
+// then counts key base' - d = base - (d - delta): it takes old counter d - delta, or zero.
+__device__ __forceinline__ void cr_raise(CrLane& L, float bm, float c, uint32_t* ring) {
+  const int lane = threadIdx.x & 31;
+  if (L.M > -INFINITY) L.s *= static_cast<double>(ex2((L.M - bm) * c));
+  L.M = bm;
+  L.nmc = -bm * c;
+  const uint32_t kmax = fkey(bm) >> 16;
+  if (L.base != 0u && kmax <= L.base) return;
+  const uint32_t nb = min(kmax + static_cast<uint32_t>(kCrHead), 0xFFFFu);
+  const uint32_t delta = L.base == 0u ? static_cast<uint32_t>(kCrRing) : nb - L.base;
+  if (delta >= static_cast<uint32_t>(kCrRing)) {
+    for (int d = lane; d < kCrRing; d += 32) ring[d] = 0u;
+  } else {
+    // top down, 32 counters per step: a step reads below what earlier steps wrote
+    for (int top = kCrRing - 32; top >= 0; top -= 32) {
+      const int d = top + lane;
+      const uint32_t v = d >= static_cast<int>(delta) ? ring[d - static_cast<int>(delta)] : 0u;
+      __syncwarp();
+      ring[d] = v;
+      __syncwarp();
+    }
+  }
+  __syncwarp();
+  L.base = nb;
+  L.kb = nb - 0x8000u;
+  L.fast = nb >= 0x8000u + static_cast<uint32_t>(kCrRing);
+}
+
+// One step of a warp's range: nvalid of this lane's kCrVec vectors hold data (all when FULL).
+template <bool FULL>
+__device__ __forceinline__ void cr_absorb(CrLane& L, const uint4 (&raw)[kCrVec], int nvalid, float c,
+                                          uint32_t* ring) {
+  if (L.bad) return;
+  uint32_t pm = 0xFF80FF80u;  // packed bf16 pair (-inf, -inf)
+#pragma unroll
+  for (int j = 0; j < kCrVec; ++j)
+    if (FULL || j < nvalid) pm = bmax2(pm, bmax2(bmax2(raw[j].x, raw[j].y), bmax2(raw[j].z, raw[j].w)));
+  const float bm = warp_max(fmax_nan(__uint_as_float(pm << 16), __uint_as_float(pm & 0xFFFF0000u)));
+  if (!(bm <= L.M)) {  // a larger maximum, or a NaN (uniform)
+    if (!(bm < INFINITY)) {
+      L.bad = true;
+      return;
+    }
+    cr_raise(L, bm, c, ring);
+  }
+  if (L.base == 0u) return;  // every value so far is -inf: weight 0
+  const f32x2 cc = pack2(c, c), nn = pack2(L.nmc, L.nmc);
+  f32x2 a0 = pack2(0.0f, 0.0f), a1 = a0;
+#pragma unroll
+  for (int j = 0; j < kCrVec; ++j) {
+    if (!(FULL || j < nvalid)) continue;
+    const uint32_t w[4] = {raw[j].x, raw[j].y, raw[j].z, raw[j].w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      float e0, e1;
+      unpack2(fma2(pack2(__uint_as_float(w[q] << 16), __uint_as_float(w[q] & 0xFFFF0000u)), cc, nn), e0, e1);
+      if (q & 1) a1 = add2(a1, pack2(ex2(e0), ex2(e1)));
+      else a0 = add2(a0, pack2(ex2(e0), ex2(e1)));
+      if (L.fast) {
+        count_if_below(ring, L.kb - (w[q] & 0xFFFFu), kCrRing);
+        count_if_below(ring, L.kb - (w[q] >> 16), kCrRing);
+      } else {
+        count_if_below(ring, L.base - key16_bits(w[q] & 0xFFFFu), kCrRing);
+        count_if_below(ring, L.base - key16_bits(w[q] >> 16), kCrRing);
+      }
+    }
+  }
+  float x0, x1, y0, y1;
+  unpack2(a0, x0, x1);
+  unpack2(a1, y0, y1);
+  L.s += (static_cast<double>(x0) + static_cast<double>(x1)) + (static_cast<double>(y0) + static_cast<double>(y1));
+}
+
+// This warp's range of row rp: the aligned body [a0, a1) split into kCrWarps runs of whole
+// 16-byte vectors, warp 0 also owning the head [0, a0) and the last warp the tail [a1, V).
+struct CrRange {
+  int lo, hi;      // elements of the row this warp owns (in index order)
+  int v0, v1;      // its body vectors [v0, v1) (vector i = elements a0 + 8i .. a0 + 8i + 7)
+  int e0, e1;      // its scalar edge elements [e0, e1) (empty for middle warps)
+};
+
+template <typename T>
+__device__ __forceinline__ CrRange cr_range(const T* rp, int V, int w) {
+  int a0, a1;
+  vec_range(rp, 0, V, a0, a1);
+  const int nvec = (a1 - a0) / 8;
+  const int qv = (nvec + kCrWarps - 1) / kCrWarps;
+  CrRange r;
+  r.v0 = min(nvec, w * qv);
+  r.v1 = min(nvec, (w + 1) * qv);
+  r.lo = w == 0 ? 0 : a0 + 8 * r.v0;
+  r.hi = w == kCrWarps - 1 ? V : a0 + 8 * r.v1;
+  r.e0 = w == 0 ? 0 : (w == kCrWarps - 1 ? a1 : 0);
+  r.e1 = w == 0 ? a0 : (w == kCrWarps - 1 ? V : 0);
+  return r;
+}
+
+// Warp w streams its range of row rp (bf16) into L and its ring. Not inlined: the streaming
+// loop gets the registers to itself, apart from the row-end work of the caller.
+__device__ __noinline__ void cr_stream(const __nv_bfloat16* __restrict__ rp, int V, const CrRange r, float c,
+                                       CrLane& L, uint32_t* ring) {
+  const int lane = threadIdx.x & 31;
+  int a0, a1;
+  vec_range(rp, 0, V, a0, a1);
+  const uint4* body = reinterpret_cast<const uint4*>(rp + a0);
+  // scalar edges first (at most 7 elements): one element per lane, as a partial step
+  if (r.e1 > r.e0) {
+    uint4 raw[kCrVec];
+    const int e = r.e0 + lane;
+    const uint32_t h = e < r.e1 ? static_cast<uint32_t>(reinterpret_cast<const uint16_t*>(rp)[e]) : 0xFF80u;
+    raw[0] = make_uint4(h | 0xFF800000u, 0xFF80FF80u, 0xFF80FF80u, 0xFF80FF80u);
+    // the lanes past the edge hold -inf pairs, which neither weigh nor count (their keys lie
+    // far below any ring a finite maximum sets, except for rows of huge negative logits, which
+    // the caller sends to the general select)
+    cr_absorb<false>(L, raw, 1, c, ring);
+  }
+  constexpr int kStep = 32 * kCrVec;  // vectors per warp step
+  const int n = r.v1 - r.v0;
+  const int steps = (n + kStep - 1) / kStep;
+  auto load = [&](uint4 (&buf)[kCrVec], int s) {
+#pragma unroll
+    for (int j = 0; j < kCrVec; ++j) {
+      const int i = s * kStep + j * 32 + lane;
+      buf[j] = i < n ? __ldg(body + r.v0 + i) : make_uint4(0xFF80FF80u, 0xFF80FF80u, 0xFF80FF80u, 0xFF80FF80u);
+    }
+  };
+  auto absorb = [&](const uint4 (&buf)[kCrVec], int s) {
+    if ((s + 1) * kStep <= n) {
+      cr_absorb<true>(L, buf, kCrVec, c, ring);
+    } else {
+      // the last, partial step: this lane's valid vectors are the first nv of its kCrVec
+      const int left = n - s * kStep;
+      const int nv = left > lane ? (left - lane + 31) / 32 : 0;
+      cr_absorb<false>(L, buf, nv, c, ring);
+    }
+  };
+  uint4 A[kCrVec], B[kCrVec];
+  if (steps > 0) load(A, 0);
+  for (int s = 0; s < steps; s += 2) {
+    if (s + 1 < steps) load(B, s + 1);
+    absorb(A, s);
+    if (s + 1 >= steps || L.bad) break;
+    if (s + 2 < steps) load(A, s + 2);
+    absorb(B, s + 1);
+    if (L.bad) break;
+  }
+}
+
+// The count of window key `key` in the warps' rings (warps without a finite value add nothing;
+// a key above a warp's base has no element in its range).
+__device__ __forceinline__ uint32_t cr_count(const CrSmem& sm, uint32_t key) {
+  uint32_t c = 0u;
+#pragma unroll
+  for (int w = 0; w < kCrWarps; ++w) {
+    const uint32_t d = sm.wb[w] - key;
+    if (sm.wm[w] > -INFINITY && d < static_cast<uint32_t>(kCrRing)) c += sm.ring[w][d];
+  }
+  return c;
+}
+
+// Shared memory of a CTA of the row kernels: the one-pass cut rows, or the general selects
+// (the rows whose cut lies outside the window, and fp32 rows).
+union CutSmem {
+  CrSmem cr;
+  TpSmem tp;
+};
+
+// Finish a row once its record st is known: the draw (sampling), the arrival and, for the last
+// arrival of a request, the accept tests (verification), or the record alone (statistics).
+// For a draft row whose draw the caller has made, y and q are its token and probability.
+template <typename T>
+__device__ __forceinline__ void cut_row_finish(const T* __restrict__ A, const T* __restrict__ Bt, const CutArgs& a,
+                                               const VerifyArgs& va, RowStat* rec, const RowStat& st, int row,
+                                               int req, int y, float q, int* flag) {
+  if (a.mode == kCutSample) {
+    if (threadIdx.x == 0) {
+      *rec = st;
+      a.out_tokens[row] = y;
+      if (a.out_q) a.out_q[row] = q;
+    }
+  } else if (a.mode == kCutVerify) {
+    if (threadIdx.x == 0) *rec = st;
+    const int per_req = (va.K + 1) + (va.stream_draft ? va.K : 0);
+    if (block_arrive_last(&va.cnt[req], per_req, flag) && threadIdx.x < 32)
+      warp_decide_request<T>(req, A, Bt, va.K, a.V, va.tokens, va.stats_t, va.stream_draft ? va.stats_d : va.dstats_in,
+                             va.u_acc, va.u_res, va.out_tokens, va.out_len, va.out_p, va.out_q, va.jobs);
+  } else if (threadIdx.x == 0) {
+    *rec = st;
+  }
+}
+
+// A row's cut by the general selects: top-k by the count-then-mass radix select (m and c from
+// the one-pass statistics in st, or from the partials), top-p by tp_row_stats (which finds m and
+// s itself for bf16 rows; fp32 rows take them from the partials); then the draw, the arrival or
+// the record. Not inlined: a rare path, kept out of the streaming loop's registers.
+template <typename T>
+__device__ __noinline__ void cut_row_general(const T* __restrict__ A, const T* __restrict__ Bt, const CutArgs& a,
+                                             const VerifyArgs& va, const Partial* __restrict__ parts_a,
+                                             const Partial* __restrict__ parts_b, TpSmem& sm, const T* rp,
+                                             RowStat* rec, RowStat st, bool in_b, int row, int req, float Tv,
+                                             float tp, int k, float u) {
+  const int V = a.V;
+  if constexpr (sizeof(T) == 2) {
+    if (k > 0) block_topk_topp_radix<T>(rp, V, tp, k, st, sm.radix);
+    else st = tp_row_stats(rp, V, Tv, tp, sm);
+  } else {
+    const Partial* pp = (in_b ? parts_b : parts_a) + static_cast<size_t>(row) * nchunks_for(V);
+    st = tp_row_stats_partials(rp, V, Tv, tp, k, pp, sm);
+  }
+  int y = -1;
+  float q = -1.0f;
+  if (a.mode == kCutSample && st.status == 0) y = tp_row_draw(rp, V, st, u, sm, &q);
+  cut_row_finish<T>(A, Bt, a, va, rec, st, row, req, y, q, &sm.flag);
+  __syncthreads();
+}
+
+// The rows of cut requests of a launch, one CTA per row at a time: CTA `cta` of `nctas` takes
+// rows cta, cta + nctas, ... (rows of other requests are skipped). bf16 rows take the
+// one-pass path, with the general selects (tp_row_stats, block_topk_topp_radix) for a cut
+// outside the window; fp32 rows take the general selects throughout (their maximum and
+// normaliser come from the streaming pass's partials, parts_a / parts_b).
+template <typename T>
+__device__ void cut_rows_cta(const T* __restrict__ A, const T* __restrict__ Bt, const CutArgs& a,
+                             const VerifyArgs& va, const Partial* __restrict__ parts_a,
+                             const Partial* __restrict__ parts_b, int cta, int nctas, CutSmem& smu) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int V = a.V;
+  const int total = a.rows_a + a.rows_b;
+  for (int g = cta; g < total; g += nctas) {
+    const bool in_b = g >= a.rows_a;
+    const int row = in_b ? g - a.rows_a : g;
+    const int req = in_b ? row / a.per_b : row / a.per_a;
+    if (!request_cut(a.temperature, a.top_p, a.top_k, req, V)) continue;  // uniform
+    const T* rp = (in_b ? Bt : A) + static_cast<size_t>(row) * V;
+    RowStat* rec = (in_b ? a.stats_b : a.stats_a) + row;
+    const float Tv = a.temperature[req];
+    const float c = temp_scale(Tv);
+    const float tp = a.top_p[req];
+    const int k = request_k(a.top_k, req, V);
+    const float u = a.mode == kCutSample ? a.u[row] : 0.0f;
+    RowStat st{};
+    if constexpr (sizeof(T) == 2) {
+      CrSmem& sm = smu.cr;
+      uint32_t* ring = sm.ring[warp];
+      // every warp streams its range
+      const CrRange r = cr_range(rp, V, warp);
+      CrLane L{-INFINITY, 0.0f, 0u, 0u, false, false, 0.0};
+      cr_stream(reinterpret_cast<const __nv_bfloat16*>(rp), V, r, c, L, ring);
+      const double sw = warp_sum(L.s);
+      if (lane == 0) {
+        sm.wm[warp] = L.M;
+        sm.ws[warp] = sw;
+        sm.wb[warp] = L.base;
+        sm.wbad[warp] = L.bad ? 1 : 0;
+      }
+      __syncthreads();
+      // the row: maximum, normaliser, status (the same arithmetic in every thread)
+      float m = -INFINITY;
+      bool bad = !(Tv >= 0.0f && Tv < INFINITY);
+#pragma unroll
+      for (int w = 0; w < kCrWarps; ++w) {
+        bad |= sm.wbad[w] != 0;
+        m = fmax_nan(m, sm.wm[w]);
+      }
+      bad |= !(m > -INFINITY) || !(m < INFINITY);
+      double S = 0.0;
+      if (!bad) {
+#pragma unroll
+        for (int w = 0; w < kCrWarps; ++w)
+          if (sm.wm[w] > -INFINITY) S += sm.ws[w] * static_cast<double>(ex2((sm.wm[w] - m) * c));
+      }
+      st = RowStat{m, c, static_cast<float>(S), static_cast<float>(S), 0u, -1, bad ? 1 : 0, 0};
+      const uint32_t km = bad ? 0u : fkey(m) >> 16;
+      // a window reaching the keys of -inf (rows of huge negative logits) takes the general select
+      bool general = !bad && km < static_cast<uint32_t>(kTpWindow) + 0x80u;
+      if (!bad && !general)
+        general = !window_pick<kCrThreads>(
+            km, tp, k, st, [&](int o) { return cr_count(sm, km - static_cast<uint32_t>(o)); }, sm.scan, &sm.bin,
+            &sm.tgt, &sm.base);
+      if (!general) {
+        int y = -1;
+        float q = -1.0f;
+        if (a.mode == kCutSample && !bad) {
+          // kept mass of each warp's range from its counts (keys ktau .. km of the window)
+          const uint32_t ktau = st.tau >> 16;
+          double acc = 0.0;
+          if (sm.wm[warp] > -INFINITY) {
+            for (uint32_t key = km - static_cast<uint32_t>(lane); key >= ktau && key <= km; key -= 32u) {
+              const uint32_t d = sm.wb[warp] - key;
+              if (d < static_cast<uint32_t>(kCrRing) && ring[d] != 0u)
+                acc += static_cast<double>(ring[d]) * static_cast<double>(ex2((key16_value(key) - m) * c));
+              if (key < 32u) break;
+            }
+          }
+          acc = warp_sum(acc);
+          if (lane == 0) sm.wk[warp] = acc;
+          __syncthreads();
+          if (threadIdx.x == 0) {
+            // the warp whose range holds u * Z (else, by rounding, the last one with kept mass)
+            double Z = 0.0;
+            for (int w = 0; w < kCrWarps; ++w) Z += sm.wk[w];
+            const double target = static_cast<double>(u) * Z;
+            double C = 0.0, lastC = 0.0;
+            int pick = -1, last = -1;
+            for (int w = 0; w < kCrWarps; ++w) {
+              if (sm.wk[w] > 0.0) {
+                last = w;
+                lastC = C;
+                if (pick < 0 && C + sm.wk[w] > target) {
+                  pick = w;
+                  sm.dbase = C;
+                }
+              }
+              C += sm.wk[w];
+            }
+            if (pick < 0) {
+              pick = last;
+              sm.dbase = lastC;
+            }
+            sm.dwarp = pick;
+            sm.dtarget = target;
+          }
+          __syncthreads();
+          const int pw = sm.dwarp;
+          if (pw >= 0) {  // uniform
+            const CrRange pr = cr_range(rp, V, pw);
+            JobRows<T, false> J;
+            J.init(rp, st, nullptr, st);
+            y = block_draw_range(J, pr.lo, pr.hi, sm.dbase, sm.dtarget, u, sm.draw);
+            if (y >= 0) q = kept_weight(st, load_elem(rp + y)) / st.s_kept;
+          }
+        }
+        cut_row_finish<T>(A, Bt, a, va, rec, st, row, req, y, q, &sm.flag);
+        __syncthreads();
+        continue;
+      }
+      __syncthreads();  // the general select below reuses the shared memory
+      if (bad) {
+        cut_row_finish<T>(A, Bt, a, va, rec, st, row, req, -1, -1.0f, &smu.tp.flag);
+        __syncthreads();
+        continue;
+      }
+    }
+    cut_row_general<T>(A, Bt, a, va, parts_a, parts_b, smu.tp, rp, rec, st, in_b, row, req, Tv, tp, k, u);
+  }
+}
+
+// Row statistics of the cut requests' rows alone (psispec_row_stats): one CTA per row at a
+// time.
+template <typename T>
+__global__ void __launch_bounds__(kCrThreads, 2) cut_rows_kernel(const T* __restrict__ A, CutArgs a,
+                                                                const Partial* __restrict__ parts) {
+  extern __shared__ __align__(16) unsigned char cut_smem_raw[];
+  VerifyArgs none{};
+  cut_rows_cta<T>(A, nullptr, a, none, parts, nullptr, blockIdx.x, gridDim.x, *reinterpret_cast<CutSmem*>(cut_smem_raw));
+}
+
+// The row kernel of sample_draft. CTAs [0, warp_ctas) finish the rows without a cut, one
+// warp per row; the remaining CTAs take the rows of requests with a cut (cut_rows_cta). One
+// launch serves both kinds of rows.
+template <typename T>
+__global__ void __launch_bounds__(kTpThreads, 2) sample_rows_kernel(const T* __restrict__ draft, int K, int V,
+                                                                   int rows, const float* __restrict__ temperature,
+                                                                   const float* __restrict__ top_p,
+                                                                   const int32_t* __restrict__ top_k,
+                                                                   const float* __restrict__ u,
+                                                                   const Partial* __restrict__ parts,
+                                                                   RowStat* __restrict__ stats,
+                                                                   int32_t* __restrict__ out_tokens,
+                                                                   float* __restrict__ out_q, int warp_ctas) {
+  if (static_cast<int>(blockIdx.x) < warp_ctas) {
+    const int row = blockIdx.x * kTpWarps + (threadIdx.x >> 5);
+    if (row < rows && !request_cut(temperature, top_p, top_k, row / K, V))
+      warp_sample_row(draft, row, K, V, temperature, u, parts, stats, out_tokens, out_q);
+    return;
+  }
+  extern __shared__ __align__(16) unsigned char cut_smem_raw[];
+  CutArgs a{};
+  a.mode = kCutSample;
+  a.V = V;
+  a.rows_a = rows;
+  a.per_a = K;
+  a.rows_b = 0;
+  a.per_b = 1;
+  a.temperature = temperature;
+  a.top_p = top_p;
+  a.top_k = top_k;
+  a.u = u;
+  a.out_tokens = out_tokens;
+  a.out_q = out_q;
+  a.stats_a = stats;
+  a.stats_b = nullptr;
+  VerifyArgs none{};
+  cut_rows_cta<T>(draft, nullptr, a, none, parts, nullptr, static_cast<int>(blockIdx.x) - warp_ctas,
+                  static_cast<int>(gridDim.x) - warp_ctas, *reinterpret_cast<CutSmem*>(cut_smem_raw));
+}
+
+// The row kernel of verify_linear. CTAs [0, warp_ctas) finish the rows of requests without a
+// cut, one warp per row; the remaining CTAs take the rows of requests with a cut
+// (cut_rows_cta). Every row then arrives on its request's counter, and whoever completes a
+// request runs its accept tests and writes the draw job.
+template <typename T>
+__global__ void __launch_bounds__(kTpThreads, 2) verify_rows_kernel(const T* __restrict__ tgt,
+                                                                   const T* __restrict__ drf, VerifyArgs va,
+                                                                   int warp_ctas) {
+  const int K = va.K, V = va.V;
+  const int rows_t = va.B * (K + 1);
+  const int rows = rows_t + (va.stream_draft ? va.B * K : 0);
+  if (static_cast<int>(blockIdx.x) < warp_ctas) {
+    const int g = blockIdx.x * kTpWarps + (threadIdx.x >> 5);
+    if (g < rows && !request_cut(va.temperature, va.top_p, va.top_k, g < rows_t ? g / (K + 1) : (g - rows_t) / K, V))
+      warp_verify_row(tgt, drf, g, va);
+    return;
+  }
+  extern __shared__ __align__(16) unsigned char cut_smem_raw[];
+  CutArgs a{};
+  a.mode = kCutVerify;
+  a.V = V;
+  a.rows_a = rows_t;
+  a.per_a = K + 1;
+  a.rows_b = va.stream_draft ? va.B * K : 0;
+  a.per_b = K;
+  a.temperature = va.temperature;
+  a.top_p = va.top_p;
+  a.top_k = va.top_k;
+  a.stats_a = va.stats_t;
+  a.stats_b = va.stats_d;
+  cut_rows_cta<T>(tgt, drf, a, va, va.parts_t, va.parts_d, static_cast<int>(blockIdx.x) - warp_ctas,
+                  static_cast<int>(gridDim.x) - warp_ctas, *reinterpret_cast<CutSmem*>(cut_smem_raw));
+}
+
+}  // namespace psi

@@ -6,6 +6,7 @@
 #include <atomic>
 
 #include "common.cuh"
+#include "cutrow.cuh"
 #include "draw.cuh"
 #include "finish.cuh"
 #include "linear.cuh"
@@ -139,8 +140,8 @@ RowSet<T> one_tensor(const T* base, int64_t rows, int rows_per_req, int nreq) {
 // through the bulk-copy ring kernel, others through plain 16-byte loads.
 template <typename T>
 psispec_status launch_stream(RowSet<T> set, int64_t rows, int V, const float* temperature, int nreq, Partial* parts,
-                             cudaStream_t st, const float* top_p = nullptr, int skip_uncut = 0,
-                             int32_t* zero = nullptr, int nzero = 0) {
+                             cudaStream_t st, Skip skip = Skip{nullptr, nullptr, kSkipNone}, int32_t* zero = nullptr,
+                             int nzero = 0) {
   const int64_t chunks = rows * nchunks_for(V);
   const bool aligned = (reinterpret_cast<uintptr_t>(set.a) & 15u) == 0 &&
                        (reinterpret_cast<uintptr_t>(set.b) & 15u) == 0 && (int64_t(V) * sizeof(T)) % 16 == 0;
@@ -156,23 +157,29 @@ psispec_status launch_stream(RowSet<T> set, int64_t rows, int V, const float* te
     const int64_t want = (chunks + (kThreads / 32) - 1) / (kThreads / 32);
     const int64_t slots = static_cast<int64_t>(sms) * (occ > 0 ? occ : 1);
     const unsigned grid = static_cast<unsigned>(want < slots ? want : slots);
-    return launch(stream_partials_tma_kernel<T>, grid, kThreads, smem, st, set, V, chunks, temperature, top_p,
-                  skip_uncut, nreq, parts, zero, nzero);
+    return launch(stream_partials_tma_kernel<T>, grid, kThreads, smem, st, set, V, chunks, temperature, skip, nreq,
+                  parts, zero, nzero);
   }
   return launch(stream_partials_kernel<T>, persistent_grid(stream_partials_kernel<T>, chunks), kThreads, 0, st, set, V,
-                chunks, temperature, top_p, skip_uncut, parts, zero, nzero);
+                chunks, temperature, skip, parts, zero, nzero);
 }
 
-// Row statistics of `rows` rows of a row set (the tree's statistics pass); with skip_uncut,
-// the rows of requests with T > 0 and no top-p cut are left out (callers with a top-k array
-// pass skip_uncut = 0: the streaming pass does not know top-k).
+// Row statistics of `rows` rows of a row set (the tree's statistics pass, psispec_row_stats);
+// the rows of the requests that `skip` selects are left out.
 template <typename T>
 psispec_status launch_stats(RowSet<T> set, int64_t rows, int V, const float* temperature, int nreq,
-                            const float* top_p, const int32_t* top_k, int skip_uncut, StatsWs ws, cudaStream_t st) {
-  psispec_status s = launch_stream<T>(set, rows, V, temperature, nreq, ws.parts, st, top_p, skip_uncut);
+                            const float* top_p, const int32_t* top_k, Skip skip, StatsWs ws, cudaStream_t st) {
+  psispec_status s = launch_stream<T>(set, rows, V, temperature, nreq, ws.parts, st, skip);
   if (s != PSISPEC_OK) return s;
   return launch(row_finalize_kernel<T>, static_cast<unsigned>((rows + kThreads / 32 - 1) / (kThreads / 32)), kThreads,
-                0, st, set, rows, V, temperature, top_p, top_k, ws.parts, ws.stats, skip_uncut);
+                0, st, set, rows, V, temperature, top_p, top_k, ws.parts, ws.stats, skip);
+}
+
+// bf16 rows of cut requests go through the one-pass cut-row path; the streaming pass leaves
+// them alone. fp32 rows of such requests need the streaming pass's partials.
+template <typename T>
+Skip cut_skip(const float* top_p, const int32_t* top_k) {
+  return Skip{top_p, top_k, sizeof(T) == 2 ? kSkipCut : kSkipNone};
 }
 
 // Launch configuration of `nclusters` clusters of CL CTAs of `threads` threads; returns
@@ -254,10 +261,10 @@ psispec_status launch_draws(const T* A, const T* Bt, int V, int njobs, const Par
                 st, A, Bt, V, njobs, parts_a, jobs, tc, tg, out_tokens);
 }
 
-// The top-p CTAs of a row kernel: persistent (one per resident slot) over the call's rows.
+// The cut-row CTAs of a row kernel: persistent (one per resident slot) over the call's rows.
 template <typename Kern>
 psispec_status prepare_topp(Kern kernel, int64_t rows, unsigned* grid) {
-  const int smem = static_cast<int>(sizeof(TpSmem));
+  const int smem = static_cast<int>(sizeof(CutSmem));
   if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return PSISPEC_ERR_CUDA;
   *grid = static_cast<unsigned>(want_slots(rows, 1, kernel, kTpThreads, smem));
@@ -272,14 +279,15 @@ psispec_status sample_draft_impl(const T* draft, int B, int K, int V, const floa
   Carver c(ws);
   SampleWs w = carve_sample(c, rows, V);
   RowStat* stats = out_stats ? out_stats : w.st.stats;
-  // every row through the streaming pass (maximum and normaliser); the row kernel's top-p
-  // CTAs then find the thresholds
-  psispec_status s = launch_stream<T>(one_tensor(draft, rows, K, B), rows, V, temperature, B, w.st.parts, st);
+  // the rows of requests without a cut (and fp32 rows) through the streaming pass (maximum and
+  // normaliser); the row kernel's warps finish them, its cut-row CTAs take the others
+  psispec_status s = launch_stream<T>(one_tensor(draft, rows, K, B), rows, V, temperature, B, w.st.parts, st,
+                                      cut_skip<T>(top_p, top_k));
   if (s != PSISPEC_OK) return s;
   unsigned tgrid = 1;
   if ((s = prepare_topp(sample_rows_kernel<T>, rows, &tgrid)) != PSISPEC_OK) return s;
   const int warp_ctas = static_cast<int>((rows + kTpWarps - 1) / kTpWarps);
-  return launch(sample_rows_kernel<T>, warp_ctas + tgrid, kTpThreads, sizeof(TpSmem), st, draft, K, V,
+  return launch(sample_rows_kernel<T>, warp_ctas + tgrid, kTpThreads, sizeof(CutSmem), st, draft, K, V,
                 static_cast<int>(rows), temperature, top_p, top_k, u, w.st.parts, stats, out_tokens, out_q, warp_ctas);
 }
 
@@ -315,18 +323,19 @@ psispec_status verify_linear_impl(const T* tgt, const T* drf, int B, int K, int 
   a.out_q = out_q;
   a.jobs = w.jobs;
   // the first streaming pass also clears the request arrival counters
+  const Skip skip = cut_skip<T>(top_p, top_k);
   psispec_status s =
-      launch_stream<T>(one_tensor(tgt, rows_t, K + 1, B), rows_t, V, temperature, B, w.t.parts, st, nullptr, 0, w.cnt,
-                       B);
+      launch_stream<T>(one_tensor(tgt, rows_t, K + 1, B), rows_t, V, temperature, B, w.t.parts, st, skip, w.cnt, B);
   if (s != PSISPEC_OK) return s;
   if (rows_d > 0 &&
-      (s = launch_stream<T>(one_tensor(drf, rows_d, K, B), rows_d, V, temperature, B, w.d.parts, st)) != PSISPEC_OK)
+      (s = launch_stream<T>(one_tensor(drf, rows_d, K, B), rows_d, V, temperature, B, w.d.parts, st, skip)) !=
+          PSISPEC_OK)
     return s;
   // one row kernel: warps for the requests without a cut, whole CTAs for the others
   unsigned tgrid = 1;
   if ((s = prepare_topp(verify_rows_kernel<T>, rows_t + rows_d, &tgrid)) != PSISPEC_OK) return s;
   const int warp_ctas = static_cast<int>((rows_t + rows_d + kTpWarps - 1) / kTpWarps);
-  s = launch(verify_rows_kernel<T>, warp_ctas + tgrid, kTpThreads, sizeof(TpSmem), st, tgt, drf, a, warp_ctas);
+  s = launch(verify_rows_kernel<T>, warp_ctas + tgrid, kTpThreads, sizeof(CutSmem), st, tgt, drf, a, warp_ctas);
   if (s != PSISPEC_OK) return s;
   return launch_draws<T>(tgt, drf, V, B, w.t.parts, w.jobs, w.draw_tc, w.draw_tg, out_tokens, st);
 }
@@ -377,8 +386,8 @@ psispec_status verify_tree_impl(const T* tgt, const T* drf, int B, int N, int V,
   // array every row goes through the statistics pass (its records carry the top-k threshold)
   const int lazy = CL != 0 && top_k == nullptr;
   // one statistics pass over the rows of both tensors
-  s = launch_stats<T>(RowSet<T>{tgt, drf, N, 1, offs, B}, 2 * int64_t(N), V, temperature, B, top_p, top_k, lazy, w.st,
-                      st);
+  s = launch_stats<T>(RowSet<T>{tgt, drf, N, 1, offs, B}, 2 * int64_t(N), V, temperature, B, top_p, top_k,
+                      Skip{top_p, top_k, lazy ? kSkipUncut : kSkipNone}, w.st, st);
   if (s != PSISPEC_OK) return s;
   const RowStat* ts = w.st.stats;
   const RowStat* ds = w.st.stats + N;
@@ -403,8 +412,27 @@ psispec_status row_stats_impl(const T* logits, int B, int K, int V, const float*
   const int64_t rows = int64_t(B) * K;
   Carver c(ws);
   Partial* parts = carve_row_stats(c, rows, V);
-  return launch_stats<T>(one_tensor(logits, rows, K, B), rows, V, temperature, B, top_p, top_k, 0,
-                         StatsWs{parts, out}, st);
+  const Skip skip = cut_skip<T>(top_p, top_k);
+  psispec_status s =
+      launch_stats<T>(one_tensor(logits, rows, K, B), rows, V, temperature, B, top_p, top_k, skip, StatsWs{parts, out}, st);
+  if (s != PSISPEC_OK || skip.mode != kSkipCut) return s;
+  // the cut requests' rows: one CTA per row at a time
+  const int smem = static_cast<int>(sizeof(CutSmem));
+  if (cudaFuncSetAttribute(cut_rows_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return PSISPEC_ERR_CUDA;
+  CutArgs a{};
+  a.mode = kCutStats;
+  a.V = V;
+  a.rows_a = static_cast<int>(rows);
+  a.per_a = K;
+  a.rows_b = 0;
+  a.per_b = 1;
+  a.temperature = temperature;
+  a.top_p = top_p;
+  a.top_k = top_k;
+  a.stats_a = out;
+  return launch(cut_rows_kernel<T>, static_cast<unsigned>(want_slots(rows, 1, cut_rows_kernel<T>, kCrThreads, smem)),
+                kCrThreads, smem, st, logits, a, static_cast<const Partial*>(parts));
 }
 
 bool bad_dtype(int dtype) { return dtype != PSISPEC_F32 && dtype != PSISPEC_BF16; }

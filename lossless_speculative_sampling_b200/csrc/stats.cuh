@@ -39,12 +39,23 @@ __device__ __forceinline__ int request_k(const int32_t* __restrict__ top_k, int 
   return k > 0 && k < V ? k : 0;
 }
 
-// Scale c of a request's rows for the streaming pass, or -1 for the rows it leaves alone: with
-// skip_uncut set, those of the requests uncut_request selects.
-__device__ __forceinline__ float stream_scale(const float* __restrict__ temperature, const float* __restrict__ top_p,
-                                              int skip_uncut, int req) {
+// Which requests' rows a statistics pass leaves to another kernel: none; those sampling at a
+// positive temperature without a cut (the cluster tree walk finds their statistics itself); or
+// those with a cut, top-p below 1 or an active top-k at a positive temperature (the one-pass
+// cut-row kernel of cutrow.cuh takes them).
+enum SkipMode : int { kSkipNone = 0, kSkipUncut = 1, kSkipCut = 2 };
+struct Skip {
+  const float* top_p;    // per request (read unless mode is kSkipNone)
+  const int32_t* top_k;  // per request, or null (off)
+  int mode;
+};
+
+// Scale c of a request's rows for the streaming pass, or -1 for the rows it leaves alone.
+__device__ __forceinline__ float stream_scale(const float* __restrict__ temperature, const Skip& sk, int req, int V) {
   const float c = temp_scale(temperature[req]);
-  return skip_uncut && c != 0.0f && !(top_p[req] < 1.0f) ? -1.0f : c;
+  if (sk.mode == kSkipNone || c == 0.0f) return c;
+  const bool cut = sk.top_p[req] < 1.0f || request_k(sk.top_k, req, V) > 0;
+  return (sk.mode == kSkipUncut ? !cut : cut) ? -1.0f : c;
 }
 
 // The rows a statistics pass reads: rows [0, rows_a) of tensor a, then the rows of tensor b
@@ -196,8 +207,7 @@ __device__ __forceinline__ Partial warp_chunk_partial(const T* __restrict__ row,
 template <typename T>
 __global__ void __launch_bounds__(kThreads, 4) stream_partials_kernel(RowSet<T> rows, int V,
                                                                     int64_t total_chunks,
-                                                                    const float* __restrict__ temperature,
-                                                                    const float* __restrict__ top_p, int skip_uncut,
+                                                                    const float* __restrict__ temperature, Skip skip,
                                                                     Partial* __restrict__ parts,
                                                                     int32_t* __restrict__ zero, int nzero) {
   if (blockIdx.x == 0)
@@ -211,7 +221,7 @@ __global__ void __launch_bounds__(kThreads, 4) stream_partials_kernel(RowSet<T> 
   const int drow = static_cast<int>(nwarps / nch), dchunk = static_cast<int>(nwarps - static_cast<int64_t>(drow) * nch);
 #pragma unroll 1
   for (; g < total_chunks; g += nwarps) {
-    const float c = stream_scale(temperature, top_p, skip_uncut, rows.request(row));
+    const float c = stream_scale(temperature, skip, rows.request(row), V);
     if (c >= 0.0f) {
       const T* rp = rows.row(row, V);
       const int c0 = chunk * kChunkElems, c1 = min(V, c0 + kChunkElems);
@@ -382,8 +392,7 @@ constexpr int kScaleTable = 1024;
 template <typename T>
 __global__ void __launch_bounds__(kThreads) stream_partials_tma_kernel(RowSet<T> rows, int V,
                                                                         int64_t total_chunks,
-                                                                        const float* __restrict__ temperature,
-                                                                        const float* __restrict__ top_p, int skip_uncut,
+                                                                        const float* __restrict__ temperature, Skip skip,
                                                                         int nreq,
                                                                         Partial* __restrict__ parts,
                                                                         int32_t* __restrict__ zero, int nzero) {
@@ -396,7 +405,7 @@ __global__ void __launch_bounds__(kThreads) stream_partials_tma_kernel(RowSet<T>
   bool some = !table;  // whether any request's rows are read
   if (table)
     for (int i = threadIdx.x; i < nreq; i += kThreads) {
-      scale[i] = stream_scale(temperature, top_p, skip_uncut, i);
+      scale[i] = stream_scale(temperature, skip, i, V);
       some |= scale[i] >= 0.0f;
     }
   if (!__syncthreads_or(some)) return;  // every row left alone
@@ -427,7 +436,7 @@ __global__ void __launch_bounds__(kThreads) stream_partials_tma_kernel(RowSet<T>
   int64_t gi = g0;
   auto scale_of = [&](int r) {
     const int req = rows.request(r);
-    return table ? scale[req] : stream_scale(temperature, top_p, skip_uncut, req);
+    return table ? scale[req] : stream_scale(temperature, skip, req, V);
   };
   uint32_t pending = 0u;  // (lane 0) stages with a copy in flight
   auto issue = [&](int i) {  // copy of this warp's i-th chunk into stage i % kRing (lane 0)
@@ -959,7 +968,7 @@ __global__ void __launch_bounds__(kThreads) row_finalize_kernel(RowSet<T> rows, 
                                                                  const float* __restrict__ top_p,
                                                                  const int32_t* __restrict__ top_k,
                                                                  const Partial* __restrict__ parts,
-                                                                 RowStat* __restrict__ stats, int skip_uncut) {
+                                                                 RowStat* __restrict__ stats, Skip skip) {
   constexpr int kRows = kThreads / 32;
   __shared__ ToppSmem sm;
   __shared__ RowStat sh_st[kRows];
@@ -971,7 +980,7 @@ __global__ void __launch_bounds__(kThreads) row_finalize_kernel(RowSet<T> rows, 
   if (row < nrows) {
     const int req = rows.request(row);
     int topp = 0, k = 0;
-    if (stream_scale(temperature, top_p, skip_uncut, req) >= 0.0f) {
+    if (stream_scale(temperature, skip, req, V) >= 0.0f) {
       const RowStat st = warp_finalize_row(parts + static_cast<size_t>(row) * nch, nch, temperature[req]);
       k = st.status == 0 && st.c != 0.0f ? request_k(top_k, req, V) : 0;
       topp = needs_topp(st, top_p[req]) || k > 0;

@@ -474,6 +474,120 @@ __device__ __forceinline__ float key16_value(uint32_t k16) {
   return __uint_as_float(b16 << 16);
 }
 
+// The cut from the counts of the kTpWindow values just below the row maximum (key16 km): the
+// value of offset o is the bf16 whose 16-bit order key is km - o, and count(o) how many
+// elements of the row carry it. Every element with one value has one weight, so the masses
+// are count x weight, exact up to the weight's rounding. Top-k: the first offset whose
+// cumulative count reaches k bounds the kept set (ties kept together) and its cumulative mass
+// is the top-k total s_k; top-p: the first offset (up to that bound) whose cumulative mass
+// reaches top_p x s_k (s_k = st.s without top-k). Sets st.tau and st.s_kept and returns true;
+// returns false (st untouched) when the window holds less than the goal. Called by every
+// thread of an NT-thread block: count(o) is evaluated for offsets [kPer t, kPer t + kPer) by
+// thread t (and by thread 0 for the rounding fallback); scan holds 33 doubles of scratch;
+// *bin, *tgt and *base are shared scalars.
+template <int NT, typename CountAt>
+__device__ bool window_pick(uint32_t km, float tp, int k, RowStat& st, CountAt&& count_at, double* scan, int* bin,
+                            double* tgt, double* base) {
+  constexpr int kPer = kTpWindow / NT;
+  static_assert(kPer * NT == kTpWindow, "the window splits evenly over the block");
+  double mass[kPer];
+  uint32_t cnt8[kPer];
+  double tsum = 0.0, tcnt = 0.0;
+#pragma unroll
+  for (int j = 0; j < kPer; ++j) {
+    const int o = threadIdx.x * kPer + j;
+    const uint32_t c = km >= static_cast<uint32_t>(o) ? count_at(o) : 0u;
+    cnt8[j] = c;
+    mass[j] = 0.0;
+    if (c != 0u) mass[j] = static_cast<double>(c) * static_cast<double>(ex2((key16_value(km - o) - st.m) * st.c));
+    tsum += mass[j];
+    tcnt += static_cast<double>(c);
+  }
+  double total;
+  const double C0 = block_exclusive_scan(tsum, scan, &total);
+  // top-k: the offset of the k-th largest element (ties kept together) bounds the kept set;
+  // the top-p target is then top_p of the mass at or above it
+  int o_lim = kTpWindow - 1;
+  double s_k = static_cast<double>(st.s);
+  if (k > 0) {
+    double count_total;
+    const double K0 = block_exclusive_scan(tcnt, scan, &count_total);
+    if (!(count_total >= static_cast<double>(k))) return false;  // the k-th value lies below the window
+    if (threadIdx.x == 0) *bin = -1;
+    __syncthreads();
+    if (K0 < static_cast<double>(k) && K0 + tcnt >= static_cast<double>(k)) {
+      double run = K0, runm = C0;
+#pragma unroll
+      for (int j = 0; j < kPer; ++j) {
+        run += static_cast<double>(cnt8[j]);
+        runm += mass[j];
+        if (run >= static_cast<double>(k)) {
+          *bin = threadIdx.x * kPer + j;
+          *tgt = runm;
+          break;
+        }
+      }
+    }
+    __syncthreads();
+    o_lim = *bin;
+    s_k = *tgt;
+    __syncthreads();
+    if (o_lim < 0) return false;  // uniform
+    if (!(tp < 1.0f)) {  // top-k alone
+      st.tau = (km - static_cast<uint32_t>(o_lim)) << 16;
+      st.s_kept = static_cast<float>(s_k);
+      return true;
+    }
+  }
+  const double target = static_cast<double>(tp) * s_k;
+  if (!(total >= target)) return false;  // the threshold lies below the window (uniform)
+  if (threadIdx.x == 0) *bin = -1;
+  __syncthreads();
+  if (C0 < target && C0 + tsum >= target) {  // the thread whose offsets cross the target
+    double run = C0;
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      if (mass[j] > 0.0 && run + mass[j] >= target) {
+        *bin = threadIdx.x * kPer + j;
+        *base = run + mass[j];
+        break;
+      }
+      run += mass[j];
+    }
+  }
+  __syncthreads();
+  int ostar = *bin;
+  if (ostar < 0) {
+    // a target of zero (the maximum's value alone), or rounding at a thread boundary: the
+    // first offset whose cumulative mass reaches the target, by thread 0
+    if (threadIdx.x == 0) {
+      double run = 0.0;
+      int pick = -1;
+      for (int o = 0; o <= o_lim && pick < 0; ++o) {
+        const uint32_t c = km >= static_cast<uint32_t>(o) ? count_at(o) : 0u;
+        if (c == 0u) continue;
+        run += static_cast<double>(c) * static_cast<double>(ex2((key16_value(km - o) - st.m) * st.c));
+        if (run >= target) pick = o;
+      }
+      if (pick < 0 && k > 0) pick = o_lim;  // rounding: the whole top-k set
+      *bin = pick;
+      *base = run;
+    }
+    __syncthreads();
+    ostar = *bin;
+    if (ostar < 0) return false;  // uniform
+  }
+  if (ostar > o_lim) {  // rounding past the top-k bound: the whole top-k set
+    ostar = o_lim;
+    if (threadIdx.x == 0) *base = s_k;
+    __syncthreads();
+  }
+  st.tau = (km - static_cast<uint32_t>(ostar)) << 16;
+  st.s_kept = static_cast<float>(*base);
+  __syncthreads();
+  return true;
+}
+
 template <typename T>
 __device__ bool tp_window_select(const T* __restrict__ row, int V, float tp, int k, RowStat& st, TpSmem& sm) {
   static_assert(sizeof(T) == 2, "bf16 rows");
@@ -520,107 +634,14 @@ __device__ bool tp_window_select(const T* __restrict__ row, int V, float tp, int
     });
   }
   __syncthreads();
-  // masses of offsets [8t, 8t + 8) in thread t, scanned in thread order
-  constexpr int kPer = kTpWindow / kTpThreads;
-  double mass[kPer];
-  uint32_t cnt8[kPer];
-  double tsum = 0.0, tcnt = 0.0;
-#pragma unroll
-  for (int j = 0; j < kPer; ++j) {
-    const int o = threadIdx.x * kPer + j;
-    uint32_t c = 0u;
-#pragma unroll
-    for (int w = 0; w < kTpWarps; ++w) c += cnt[w * kTpWindow + o];
-    cnt8[j] = km >= static_cast<uint32_t>(o) ? c : 0u;
-    mass[j] = 0.0;
-    if (cnt8[j] != 0u) mass[j] = static_cast<double>(c) * static_cast<double>(ex2((key16_value(km - o) - st.m) * st.c));
-    tsum += mass[j];
-    tcnt += static_cast<double>(cnt8[j]);
-  }
-  double total;
-  const double C0 = block_exclusive_scan(tsum, sm.mass, &total);
-  // top-k: the offset of the k-th largest element (ties kept together) bounds the kept set;
-  // the top-p target is then top_p of the mass at or above it
-  int o_lim = kTpWindow - 1;
-  double s_k = static_cast<double>(st.s);
-  if (k > 0) {
-    double count_total;
-    const double K0 = block_exclusive_scan(tcnt, sm.mass, &count_total);
-    if (!(count_total >= static_cast<double>(k))) return false;  // the k-th value lies below the window
-    if (threadIdx.x == 0) sm.bin = -1;
-    __syncthreads();
-    if (K0 < static_cast<double>(k) && K0 + tcnt >= static_cast<double>(k)) {
-      double run = K0, runm = C0;
-#pragma unroll
-      for (int j = 0; j < kPer; ++j) {
-        run += static_cast<double>(cnt8[j]);
-        runm += mass[j];
-        if (run >= static_cast<double>(k)) {
-          sm.bin = threadIdx.x * kPer + j;
-          sm.tgt = runm;
-          break;
-        }
-      }
-    }
-    __syncthreads();
-    o_lim = sm.bin;
-    s_k = sm.tgt;
-    __syncthreads();
-    if (o_lim < 0) return false;  // uniform
-    if (!(tp < 1.0f)) {  // top-k alone
-      st.tau = (km - static_cast<uint32_t>(o_lim)) << 16;
-      st.s_kept = static_cast<float>(s_k);
-      return true;
-    }
-  }
-  const double target = static_cast<double>(tp) * s_k;
-  if (!(total >= target)) return false;  // the threshold lies below the window (uniform)
-  if (threadIdx.x == 0) sm.bin = -1;
-  __syncthreads();
-  if (C0 < target && C0 + tsum >= target) {  // the thread whose offsets cross the target
-    double run = C0;
-#pragma unroll
-    for (int j = 0; j < kPer; ++j) {
-      if (mass[j] > 0.0 && run + mass[j] >= target) {
-        sm.bin = threadIdx.x * kPer + j;
-        sm.base = run + mass[j];
-        break;
-      }
-      run += mass[j];
-    }
-  }
-  __syncthreads();
-  int ostar = sm.bin;
-  if (ostar < 0) {
-    // a target of zero (the maximum's value alone), or rounding at a thread boundary: the
-    // first offset whose cumulative mass reaches the target, by thread 0
-    if (threadIdx.x == 0) {
-      double run = 0.0;
-      int pick = -1;
-      for (int o = 0; o <= o_lim && pick < 0; ++o) {
+  return window_pick<kTpThreads>(
+      km, tp, k, st, [&](int o) {
         uint32_t c = 0u;
+#pragma unroll
         for (int w = 0; w < kTpWarps; ++w) c += cnt[w * kTpWindow + o];
-        if (c == 0u || km < static_cast<uint32_t>(o)) continue;
-        run += static_cast<double>(c) * static_cast<double>(ex2((key16_value(km - o) - st.m) * st.c));
-        if (run >= target) pick = o;
-      }
-      if (pick < 0 && k > 0) pick = o_lim;  // rounding: the whole top-k set
-      sm.bin = pick;
-      sm.base = run;
-    }
-    __syncthreads();
-    ostar = sm.bin;
-    if (ostar < 0) return false;  // uniform
-  }
-  if (ostar > o_lim) {  // rounding past the top-k bound: the whole top-k set
-    ostar = o_lim;
-    if (threadIdx.x == 0) sm.base = s_k;
-    __syncthreads();
-  }
-  st.tau = (km - static_cast<uint32_t>(ostar)) << 16;
-  st.s_kept = static_cast<float>(sm.base);
-  __syncthreads();
-  return true;
+        return c;
+      },
+      sm.mass, &sm.bin, &sm.tgt, &sm.base);
 }
 
 // Statistics of a row of a request with a top-p or top-k cut: maximum and normaliser from the
@@ -727,82 +748,6 @@ __device__ int tp_row_draw(const T* __restrict__ row, int V, const RowStat& st, 
 __device__ __forceinline__ bool request_cut(const float* __restrict__ temperature, const float* __restrict__ top_p,
                                             const int32_t* __restrict__ top_k, int r, int V) {
   return temp_scale(temperature[r]) != 0.0f && (top_p[r] < 1.0f || request_k(top_k, r, V) > 0);
-}
-
-// The row kernel of sample_draft. CTAs [0, warp_ctas) finish the rows without a cut,
-// one warp per row; the remaining CTAs take the rows of requests with a cut, one row per CTA
-// at a time (statistics, threshold, draw). One launch serves both kinds of rows.
-template <typename T>
-__global__ void __launch_bounds__(kTpThreads, 2) sample_rows_kernel(const T* __restrict__ draft, int K, int V,
-                                                                   int rows, const float* __restrict__ temperature,
-                                                                   const float* __restrict__ top_p,
-                                                                   const int32_t* __restrict__ top_k,
-                                                                   const float* __restrict__ u,
-                                                                   const Partial* __restrict__ parts,
-                                                                   RowStat* __restrict__ stats,
-                                                                   int32_t* __restrict__ out_tokens,
-                                                                   float* __restrict__ out_q, int warp_ctas) {
-  if (static_cast<int>(blockIdx.x) < warp_ctas) {
-    const int row = blockIdx.x * kTpWarps + (threadIdx.x >> 5);
-    if (row < rows && !request_cut(temperature, top_p, top_k, row / K, V))
-      warp_sample_row(draft, row, K, V, temperature, u, parts, stats, out_tokens, out_q);
-    return;
-  }
-  extern __shared__ __align__(16) unsigned char tp_smem_raw[];
-  TpSmem& sm = *reinterpret_cast<TpSmem*>(tp_smem_raw);
-  const int ctas = static_cast<int>(gridDim.x) - warp_ctas;
-  for (int row = static_cast<int>(blockIdx.x) - warp_ctas; row < rows; row += ctas) {
-    const int b = row / K;
-    if (!request_cut(temperature, top_p, top_k, b, V)) continue;
-    const T* rp = draft + static_cast<size_t>(row) * V;
-    const RowStat st = tp_row_stats_partials(rp, V, temperature[b], top_p[b], request_k(top_k, b, V),
-                                             parts + static_cast<size_t>(row) * nchunks_for(V), sm);
-    float q = -1.0f;
-    const int y = st.status == 0 ? tp_row_draw(rp, V, st, u[row], sm, &q) : -1;
-    if (threadIdx.x == 0) {
-      stats[row] = st;
-      out_tokens[row] = y;
-      if (out_q) out_q[row] = q;
-    }
-    __syncthreads();
-  }
-}
-
-// The row kernel of verify_linear. CTAs [0, warp_ctas) finish the rows of requests without a
-// cut, one warp per row; the remaining CTAs take the rows of requests with a cut, one
-// row per CTA at a time (statistics and threshold). Every row then arrives on its request's
-// counter, and whoever completes a request runs its accept tests and writes the draw job.
-template <typename T>
-__global__ void __launch_bounds__(kTpThreads, 2) verify_rows_kernel(const T* __restrict__ tgt,
-                                                                   const T* __restrict__ drf, VerifyArgs a,
-                                                                   int warp_ctas) {
-  const int K = a.K, V = a.V;
-  const int rows_t = a.B * (K + 1);
-  const int rows = rows_t + (a.stream_draft ? a.B * K : 0);
-  if (static_cast<int>(blockIdx.x) < warp_ctas) {
-    const int g = blockIdx.x * kTpWarps + (threadIdx.x >> 5);
-    if (g < rows && !request_cut(a.temperature, a.top_p, a.top_k, g < rows_t ? g / (K + 1) : (g - rows_t) / K, V))
-      warp_verify_row(tgt, drf, g, a);
-    return;
-  }
-  extern __shared__ __align__(16) unsigned char tp_smem_raw[];
-  TpSmem& sm = *reinterpret_cast<TpSmem*>(tp_smem_raw);
-  const int per_req = (K + 1) + (a.stream_draft ? K : 0);
-  const int ctas = static_cast<int>(gridDim.x) - warp_ctas;
-  for (int g = static_cast<int>(blockIdx.x) - warp_ctas; g < rows; g += ctas) {
-    const bool is_draft = g >= rows_t;
-    const int row = is_draft ? g - rows_t : g;
-    const int b = is_draft ? row / K : row / (K + 1);
-    if (!request_cut(a.temperature, a.top_p, a.top_k, b, V)) continue;
-    const T* rp = (is_draft ? drf : tgt) + static_cast<size_t>(row) * V;
-    const Partial* pp = (is_draft ? a.parts_d : a.parts_t) + static_cast<size_t>(row) * nchunks_for(V);
-    const RowStat st = tp_row_stats_partials(rp, V, a.temperature[b], a.top_p[b], request_k(a.top_k, b, V), pp, sm);
-    if (threadIdx.x == 0) (is_draft ? a.stats_d : a.stats_t)[row] = st;
-    if (block_arrive_last(&a.cnt[b], per_req, &sm.flag) && threadIdx.x < 32)
-      warp_decide_request<T>(b, tgt, drf, K, V, a.tokens, a.stats_t, a.stream_draft ? a.stats_d : a.dstats_in,
-                             a.u_acc, a.u_res, a.out_tokens, a.out_len, a.out_p, a.out_q, a.jobs);
-    __syncthreads();
-  }
 }
 
 }  // namespace psi

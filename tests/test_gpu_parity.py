@@ -567,3 +567,69 @@ def test_row_stats_topk_parity(dtype):
         kept = (_fkey(l) >= st["tau"][r]) if st["tau"][r] != 0 else np.ones(V, bool)
         p = np.where(kept, np.exp2((l.astype(np.float64) - st["m"][r]) * st["c"][r]) / st["s_kept"][r], 0.0)
         assert np.abs(p - probs).max() <= 1e-5, (r, np.abs(p - probs).max())
+
+
+# ------------------------------------------------------------------ one-pass cut rows: edge rows
+
+
+def _edge_rows(V, n_rows, g):
+    """bf16 draft-like rows that stress the one-pass cut path: the row maximum arriving last
+    (far above, and just above, what the first values set), spikes in several warps' ranges,
+    rows of huge negative logits (the window reaches the keys of -inf), a row of -inf with one
+    finite value, a NaN row, and plain rows."""
+    x = torch.randn((n_rows, V), generator=g) * 2.0
+    x[0, V - 3] = 60.0                    # the maximum last, many binades above the rest
+    x[1, V - 1] = 9.0                     # just above the usual maximum, at the very end
+    x[2, ::V // 7 + 1] = torch.linspace(5.0, 40.0, len(range(0, V, V // 7 + 1)))  # rising spikes
+    x[3] = -3.0e38 + x[3].abs() * 1.0e36  # huge negative logits
+    x[4] = -float("inf")
+    x[4, V // 2] = 1.0                    # one finite value
+    x[5, min(17, V - 1)] = float("nan")   # a data error
+    x[6, :V // 2] = -float("inf")         # the first half -inf: the first warps see no finite value
+    return x.to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("V", [7, 300, 16384 * 2 + 37, 151936])
+@pytest.mark.parametrize("top_p,top_k", [(0.9, 0), (1.0, 40), (0.95, 500)])
+def test_cut_rows_edge_rows(V, top_p, top_k):
+    """The one-pass cut-row path on edge rows, for sampling, verification (streaming the draft
+    rows, and reusing the sampler's records) and row statistics, against the oracle."""
+    B, K = 4, 2
+    g = torch.Generator().manual_seed(V + 7 * top_k)
+    drf = _edge_rows(V, B * K, g).reshape(B, K, V)
+    tgt = torch.cat([_edge_rows(V, B * K, g).reshape(B, K, V)[:, torch.randperm(K, generator=g)],
+                     (torch.randn((B, 1, V), generator=g) * 2.0).to(torch.bfloat16)], dim=1)
+    Ts = torch.tensor([1.0, 0.7, 1.3, 1.0])
+    Ps = torch.full((B,), top_p)
+    Ks = torch.full((B,), top_k, dtype=torch.int32) if top_k else None
+    Kd = _cuda(Ks) if top_k else None
+    ud, ua, ur = synth.uniforms((B, K), V + 1), synth.uniforms((B, K), V + 2), synth.uniforms((B, K + 1), V + 3)
+    tok, q, rec = psispec.sample_draft(_cuda(drf), _cuda(Ts), _cuda(Ps), _cuda(ud), top_k=Kd)
+    rr = np.arange(B * K) // K
+    o_s = oracle.sample_draft(drf.reshape(B * K, V), Ts.numpy(), Ps.numpy(), ud.reshape(-1), row_req=rr,
+                              top_k=None if Ks is None else Ks.numpy())
+    assert (o_s["tokens"].reshape(B, K)[:, :] >= -1).all()
+    check_sample(tok, q, o_s, drf.reshape(B * K, V), Ts, Ps, ud, rr, Ks, label="edge rows sample V=%d" % V)
+    x = o_s["tokens"].reshape(B, K).astype(np.int32)
+    x[x < 0] = 0
+    ora = oracle.verify_linear(tgt, drf, x, ua, ur, Ts.numpy(), Ps.numpy(), top_k=None if Ks is None else Ks.numpy())
+    for stats in (None, rec):
+        out = psispec.verify_linear(_cuda(tgt), _cuda(drf), _cuda(x), _cuda(ua), _cuda(ur), _cuda(Ts), _cuda(Ps),
+                                    top_k=Kd, draft_row_stats=stats)
+        check_linear(out, ora, tgt, drf, x, ua, ur, Ts, Ps, Ks, label="edge rows verify V=%d" % V)
+    # the records the statistics entry writes imply the oracle's distributions
+    recs = _decode_stats(psispec.row_stats(_cuda(drf), _cuda(Ts), _cuda(Ps), top_k=Kd))
+    rows = drf.reshape(B * K, V).float().numpy().astype(np.float64)
+    for r in range(B * K):
+        b = r // K
+        probs, band = oracle.row_dist(rows[r], float(Ts[b]), float(Ps[b]), top_k)
+        if probs is None:
+            assert recs["status"][r] != 0, r
+            continue
+        assert recs["status"][r] == 0, r
+        if band < 1e-6:
+            continue
+        l = rows[r].astype(np.float32)
+        kept = (_fkey(l) >= recs["tau"][r]) if recs["tau"][r] != 0 else np.ones(V, bool)
+        p = np.where(kept, np.exp2((l.astype(np.float64) - recs["m"][r]) * recs["c"][r]) / recs["s_kept"][r], 0.0)
+        assert np.abs(p - probs).max() <= 1e-5, (r, np.abs(p - probs).max())
