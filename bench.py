@@ -239,6 +239,8 @@ def run_reference(args):
 
     if args.workload in synth.tree_cases():
         return _run_reference_tree(args)
+    if args.workload in synth.trie_cases():
+        return _run_reference_trie(args)
     case = synth.linear_cases()[args.workload]
     threads = _host_threads()
     # one request per host thread per step, bounded so that the whole run stays near two
@@ -288,6 +290,49 @@ def _run_reference_tree(args):
                                                                                               args.workload)
     _print_reference(args, n / dt, dt, "f64", {"workload": args.workload, "tries_per_step": n_req, "nodes": n,
                                                "vocab": case.V}, sample)
+
+
+def _run_reference_trie(args):
+    """The oracle's candidate trie and its deterministic-rule verification, one request per host
+    thread, on a bounded number of the workload's requests."""
+    from concurrent.futures import ThreadPoolExecutor
+
+    import oracle
+    from lossless_speculative_sampling_b200 import synth
+
+    case = synth.trie_cases()[args.workload]
+    K, V, n = case.K, case.V, case.n_prefixes
+    threads = _host_threads()
+    n_req = max(1, min(case.B, threads))
+    drf = synth.trie_draft(case, device="cpu")[:n_req].to(torch.float64)
+    ua, ur = synth.trie_uniforms(case)
+
+    def one(b):
+        t = oracle.build_tree(drf[b].numpy(), case.temperature, case.top_p, case.cand_k, n)
+        dep = torch.from_numpy(t["depth"]).view(1, -1)
+        rows = synth.trie_verifier_rows(case, drf[b:b + 1].to(case.dtype), dep).to(torch.float64).numpy()
+        tk = t["tokens"].copy()
+        tk[0] = 0
+        m = len(tk)
+        s0 = b * (n + 1)
+        return oracle.verify_tree(rows, rows, [0, m], t["parent"], tk, ua[s0:s0 + m], ur[s0:s0 + m],
+                                  [case.temperature], [case.top_p], K, rule=oracle.TREE_DETERMINISTIC)
+
+    def step():
+        with ThreadPoolExecutor(max_workers=threads) as ex:
+            list(ex.map(one, range(n_req)))
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = (time.perf_counter() - t0) / args.steps
+    sample = "%d of %d requests of workload %s per step (fp64 C oracle, one request per host thread, %d threads)" % (
+        n_req, case.B, args.workload, threads)
+    _print_reference(args, n_req * n / dt, dt, "f64", {"workload": args.workload, "requests_per_step": n_req,
+                                                       "block": K, "vocab": V, "cand_k": case.cand_k,
+                                                       "n_prefixes": n}, sample, cores=threads)
 
 
 def _print_reference(args, value, dt, dtype, config, sample, cores=1):
@@ -397,14 +442,65 @@ def _prepare_tree(case, dev):
     }
 
 
+def _prepare_trie(case, dev):
+    """The tree sampler's step: the candidate trie from the draft rows (psispec_build_tree),
+    then its verification with the deterministic-candidate rule (psispec_verify_tree_det) on
+    the verifier rows of its nodes."""
+    from lossless_speculative_sampling_b200 import psispec, synth
+
+    B, K, V, n = case.B, case.K, case.V, case.n_prefixes
+    cap = n + 1
+    drf = synth.trie_draft(case, device=dev)
+    Ts = torch.full((B,), case.temperature, device=dev)
+    Ps = torch.full((B,), case.top_p, device=dev)
+    trie = {"parent": torch.empty((B, cap), dtype=torch.int32, device=dev),
+            "tokens": torch.empty((B, cap), dtype=torch.int32, device=dev),
+            "depth": torch.empty((B, cap), dtype=torch.int32, device=dev),
+            "score": torch.empty((B, cap), dtype=torch.float64, device=dev),
+            "nodes": torch.empty(B, dtype=torch.int32, device=dev)}
+    ws_b = torch.empty(psispec.workspace_size(psispec.OP_BUILD_TREE, B, K, V), dtype=torch.uint8, device=dev)
+    psispec.build_tree(drf, Ts, Ps, case.cand_k, n, out=trie, ws=ws_b)
+    assert bool((trie["nodes"] == cap).all()), "every request keeps n_prefixes prefixes"
+    tgt = synth.trie_verifier_rows(case, drf, trie["depth"])  # the verifier rows of the built trie's nodes
+    ua, ur = (t.to(dev) for t in synth.trie_uniforms(case))
+    offs = torch.arange(0, B * cap + 1, cap, dtype=torch.int32, device=dev)
+    o_path = torch.empty((B, K), dtype=torch.int32, device=dev)
+    o_tok = torch.empty((B, K + 1), dtype=torch.int32, device=dev)
+    o_len = torch.empty(B, dtype=torch.int32, device=dev)
+    ws_v = torch.empty(psispec.workspace_size(psispec.OP_VERIFY_TREE, B, B * cap, V), dtype=torch.uint8, device=dev)
+    esz = tgt.element_size()
+
+    def build(t_in=tgt, d_in=drf):
+        psispec.build_tree(d_in, Ts, Ps, case.cand_k, n, out=trie, ws=ws_b)
+
+    def verify(t_in=tgt, d_in=drf):
+        psispec.verify_tree_det(t_in, offs, trie["parent"].view(-1), trie["tokens"].view(-1), ua, ur, Ts, Ps, K,
+                                out_path=o_path, out_tokens=o_tok, out_accept_len=o_len, ws=ws_v)
+
+    return {
+        "inputs": (tgt, drf), "calls": [("build_tree", build), ("verify_tree_det", verify)],
+        "outputs": (o_tok, o_len), "positions": B * n, "esz": esz,
+        "bytes": {"build_tree": B * K * V * esz, "verify_tree_det": B * cap * V * esz},
+        "bytes_step": (B * K + B * cap) * V * esz, "launches": 4 + 3,
+        "describe": "candidate trie B=%d K=%d V=%d %s, %d candidates per position, %d prefixes, T=%g, top-p %g" % (
+            B, K, V, "bf16" if esz == 2 else "fp32", case.cand_k, n, case.temperature, case.top_p),
+        "config": {"global_batch": B, "block": K, "vocab": V, "cand_k": case.cand_k, "n_prefixes": n},
+        "accept": lambda: float(o_len.float().mean()),
+    }
+
+
 def _prepare(name, dev, rank=0):
     from lossless_speculative_sampling_b200 import synth
 
-    lin, tre = synth.linear_cases(), synth.tree_cases()
+    lin, tre, tri = synth.linear_cases(), synth.tree_cases(), synth.trie_cases()
     if name in lin:
         case = lin[name]
         case.seed = _rank_seed(case.seed, rank)
         return _prepare_linear(case, dev), case
+    if name in tri:
+        case = tri[name]
+        case.seed = _rank_seed(case.seed, rank)
+        return _prepare_trie(case, dev), case
     case = tre[name]
     case.seed = _rank_seed(case.seed, rank)
     return _prepare_tree(case, dev), case
@@ -478,7 +574,7 @@ def _all_workloads(args, dev):
     from lossless_speculative_sampling_b200 import synth
 
     peak, peak_kind = _peaks()
-    names = [n for n in synth.linear_cases() if n != "tiny"] + list(synth.tree_cases())
+    names = [n for n in synth.linear_cases() if n != "tiny"] + list(synth.tree_cases()) + list(synth.trie_cases())
     for name in names:
         P, case = _prepare(name, dev)
         calls = _graphs(P["calls"], dev, 3) if not args.no_graph else P["calls"]

@@ -74,7 +74,8 @@ typedef enum {
   PSISPEC_OP_SAMPLE_DRAFT = 0,
   PSISPEC_OP_VERIFY_LINEAR = 1,
   PSISPEC_OP_VERIFY_TREE = 2,
-  PSISPEC_OP_ROW_STATS = 3
+  PSISPEC_OP_ROW_STATS = 3,
+  PSISPEC_OP_BUILD_TREE = 4 /* a = B, b = K, c = V */
 } psispec_op;
 
 /* Bytes of one per-row statistics record (psispec_sample_draft's out_row_stats,
@@ -264,6 +265,50 @@ psispec_status psispec_verify_tree_k(const void* target_logits, const void* draf
                                      const int32_t* top_k, int32_t max_depth, int32_t* out_path,
                                      int32_t* out_tokens, int32_t* out_accept_len, void* workspace,
                                      size_t workspace_bytes, void* stream);
+
+/*
+ * psispec_build_tree -- candidate trie of the tree sampler (review page, section 3.4: at every
+ * position the top-K tokens, then the V most probable prefixes; the README's tree flags set
+ * the two sizes). Readings: position i's distribution is draft row i's q after temperature,
+ * top-k and top-p; its candidates are the cand_k kept tokens of largest q (ties to the lower
+ * index, q > 0); a prefix's probability is the product of its tokens' q (fp64); the
+ * n_prefixes most probable prefixes are kept, ties to the shorter prefix and then to the
+ * smaller sequence of candidate ranks, numbered in the order kept (node 0 = the empty prefix,
+ * so parents precede children and siblings follow in decreasing probability).
+ *
+ *   draft_logits  [B, K, V] dtype   draft rows of the K drafted positions of each request
+ *   temperature [B] float, top_p [B] float, top_k [B] int32 or NULL
+ *   out_parent, out_tokens, out_depth  [B, n_prefixes + 1] int32 (root: -1, -1, 0; slots
+ *                 beyond the node count: -1)
+ *   out_score     [B, n_prefixes + 1] double, prefix probabilities; may be NULL
+ *   out_nodes     [B] int32 node count (1 + kept prefixes), or -1 when a draft row of the
+ *                 request has a data error
+ * Workspace: psispec_workspace_size(PSISPEC_OP_BUILD_TREE, B, K, V) bytes.
+ * Limits: 1 <= K <= 16, 1 <= cand_k <= 32, 1 <= n_prefixes <= 64, B*K <= 2^26, V <= 2^24.
+ * The trie's node arrays plug into psispec_verify_tree (node_offsets b*(n_prefixes+1) with
+ * the unused slots trimmed by the caller).
+ */
+psispec_status psispec_build_tree(const void* draft_logits, int dtype, int32_t B, int32_t K, int32_t V,
+                                  const float* temperature, const float* top_p, const int32_t* top_k,
+                                  int32_t cand_k, int32_t n_prefixes, int32_t* out_parent, int32_t* out_tokens,
+                                  int32_t* out_depth, double* out_score, int32_t* out_nodes, void* workspace,
+                                  size_t workspace_bytes, void* stream);
+
+/*
+ * psispec_verify_tree_det -- tree verification of a trie whose children were fixed in advance
+ * (the candidate trie of psispec_build_tree): rejection sampling with point-mass proposals.
+ * At a node with verifier distribution p (after temperature, top-k, top-p), child t (in node
+ * order) is accepted iff u_accept[t] < r(t), r = p without the siblings rejected before it,
+ * renormalised; where the walk stops the final token is drawn from that r with the node's
+ * u_resid (-1 if the rejected siblings held all of p's mass). No draft rows are read.
+ * Arguments, outputs, limits and errors as psispec_verify_tree (top_k may be NULL).
+ */
+psispec_status psispec_verify_tree_det(const void* target_logits, int dtype, int32_t B, int32_t N, int32_t V,
+                                       const int32_t* node_offsets, const int32_t* parent, const int32_t* tokens,
+                                       const float* u_accept, const float* u_resid, const float* temperature,
+                                       const float* top_p, const int32_t* top_k, int32_t max_depth,
+                                       int32_t* out_path, int32_t* out_tokens, int32_t* out_accept_len,
+                                       void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * psispec_verify_linear_static -- psispec_verify_linear without a caller workspace.

@@ -16,10 +16,11 @@
 //   - the running maximum M (NaN-propagating, bf16 pairs compared packed) and, per lane, the
 //     fp64 sum of 2^((x - M) c), rescaled whenever M grows;
 //   - a ring of kCrRing counters in shared memory, counter d counting the elements whose
-//     16-bit order key is base - d. The base is set kCrHead keys above the warp's maximum at
-//     its first finite value and moved up (counters shifted) only when the maximum passes
-//     it, so the counters cover the kTpWindow keys below the warp's maximum at every moment,
-//     hence also the kTpWindow keys below the row's maximum at the end.
+//     16-bit order key is lower + d. The ring's top key, lower + kCrRing - 1, is set kCrHead
+//     keys above the warp's maximum at its first finite value and moved up (counters shifted)
+//     only when the maximum passes it, so the counters cover the kTpWindow keys below the
+//     warp's maximum at every moment, hence also the kTpWindow keys below the row's maximum at
+//     the end.
 // The CTA then combines its warps: the maximum m, the normaliser s (fp64), and the counts of
 // the window below m, from which window_pick finds tau and the kept mass. A draft row draws
 // its token at once: the warps' kept masses (counts x weights) give the warp whose range holds
@@ -67,10 +68,10 @@ struct CutArgs {
 };
 
 struct CrSmem {
-  uint32_t ring[kCrWarps][kCrRing];
+  uint32_t ring[kCrWarps][kCrRing + 32];  // the counters, then one discard counter per lane
   float wm[kCrWarps];     // the warps' maxima (-inf: no finite value in the range)
   double ws[kCrWarps];    // the warps' sums, relative to their own maxima
-  uint32_t wb[kCrWarps];  // the warps' ring bases
+  uint32_t wl[kCrWarps];  // the warps' ring lower keys (0: no finite value)
   int wbad[kCrWarps];     // a NaN or +inf logit in the warp's range
   double wk[kCrWarps];    // the warps' kept masses (draft rows)
   double scan[40];
@@ -79,15 +80,20 @@ struct CrSmem {
   DrawSmem draw;
 };
 
-// One warp's running state over its range (uniform across the warp except s).
+// One warp's running state over its range. Per lane: the running maximum M of the lane's own
+// values and the fp64 sum of 2^((x - M) c) over them (rescaled when M grows), and whether a NaN
+// or +inf logit was seen. Uniform across the warp: the ring's keys.
 struct CrLane {
-  float M;        // running maximum; -inf before the first finite value
-  float nmc;      // -M c
-  uint32_t base;  // ring base key; 0 before the first finite value
-  uint32_t kb;    // base - 0x8000: the raw-bit base of the positive-only path
-  bool fast;      // every key the ring covers belongs to a positive value
-  bool bad;       // a NaN or +inf logit
-  double s;       // this lane's sum of 2^((x - M) c)
+  float M;         // this lane's running maximum; -inf before its first finite value
+  float nmc;       // -M c (0 while M is -inf, so that -inf values weigh exp2(-inf) = 0)
+  double s;        // this lane's sum of 2^((x - M) c)
+  bool bad;        // this lane saw a NaN or +inf logit
+  uint32_t top;    // the ring's top key (uniform); 0 before the warp's first finite value
+  uint32_t lower;  // its lowest key, top - kCrRing + 1
+  uint32_t nl16;   // -((lower - 0x8000) << 16): the positive-only path's offset of raw value bits
+  bool fast;       // every key the ring covers belongs to a positive value
+  uint32_t dl;     // (kCrRing + lane) << 16: this lane's discard counter, as a clamp
+  uint32_t ra;     // shared address of the warp's ring
 };
 
 // The 16-bit order key of a bf16 bit pattern (fkey(x) >> 16 of the widened value; -0 and +0
@@ -96,79 +102,129 @@ __device__ __forceinline__ uint32_t key16_bits(uint32_t h) {
   return (h & 0x8000u) ? (h == 0x8000u ? 0x8000u : (~h & 0xFFFFu)) : (h | 0x8000u);
 }
 
-// The warp's maximum grew to bm (finite): rescale the lane sums and, when bm's key passes the
-// ring base (or at the first finite value), move the base kCrHead keys above it. Counter d
-// then counts key base' - d = base - (d - delta): it takes old counter d - delta, or zero.
-__device__ __forceinline__ void cr_raise(CrLane& L, float bm, float c, uint32_t* ring) {
+// Some lane's maximum passed the ring's top key (or the warp's first finite value arrived): the
+// top moves kCrHead keys above the warp's maximum key kmax; returns the new top. With the top
+// (and the lower key) up by delta, counter d counts key lower + delta + d: it takes old counter
+// d + delta, or zero. Warp-uniform; rare, but inlined: a call inside the streaming loop would
+// make the loop keep its values in memory across it.
+__device__ __forceinline__ uint32_t cr_rebase(uint32_t top, uint32_t kmax, uint32_t* ring) {
   const int lane = threadIdx.x & 31;
-  if (L.M > -INFINITY) L.s *= static_cast<double>(ex2((L.M - bm) * c));
-  L.M = bm;
-  L.nmc = -bm * c;
-  const uint32_t kmax = fkey(bm) >> 16;
-  if (L.base != 0u && kmax <= L.base) return;
-  const uint32_t nb = min(kmax + static_cast<uint32_t>(kCrHead), 0xFFFFu);
-  const uint32_t delta = L.base == 0u ? static_cast<uint32_t>(kCrRing) : nb - L.base;
+  const uint32_t nt = min(kmax + static_cast<uint32_t>(kCrHead), 0xFFFFu);
+  const uint32_t delta = top == 0u ? static_cast<uint32_t>(kCrRing) : nt - top;
+  __syncwarp();  // the reductions of earlier steps are visible to every lane
   if (delta >= static_cast<uint32_t>(kCrRing)) {
     for (int d = lane; d < kCrRing; d += 32) ring[d] = 0u;
   } else {
-    // top down, 32 counters per step: a step reads below what earlier steps wrote
-    for (int top = kCrRing - 32; top >= 0; top -= 32) {
-      const int d = top + lane;
-      const uint32_t v = d >= static_cast<int>(delta) ? ring[d - static_cast<int>(delta)] : 0u;
+    // bottom up, 32 counters per step: a step reads above what earlier steps wrote
+    for (int b = 0; b < kCrRing; b += 32) {
+      const int d = b + lane;
+      const uint32_t v = d + static_cast<int>(delta) < kCrRing ? ring[d + static_cast<int>(delta)] : 0u;
       __syncwarp();
       ring[d] = v;
       __syncwarp();
     }
   }
   __syncwarp();
-  L.base = nb;
-  L.kb = nb - 0x8000u;
-  L.fast = nb >= 0x8000u + static_cast<uint32_t>(kCrRing);
+  return nt;
 }
 
-// One step of a warp's range: nvalid of this lane's kCrVec vectors hold data (all when FULL).
-template <bool FULL>
-__device__ __forceinline__ void cr_absorb(CrLane& L, const uint4 (&raw)[kCrVec], int nvalid, float c,
-                                          uint32_t* ring) {
-  if (L.bad) return;
-  uint32_t pm = 0xFF80FF80u;  // packed bf16 pair (-inf, -inf)
-#pragma unroll
-  for (int j = 0; j < kCrVec; ++j)
-    if (FULL || j < nvalid) pm = bmax2(pm, bmax2(bmax2(raw[j].x, raw[j].y), bmax2(raw[j].z, raw[j].w)));
-  const float bm = warp_max(fmax_nan(__uint_as_float(pm << 16), __uint_as_float(pm & 0xFFFF0000u)));
-  if (!(bm <= L.M)) {  // a larger maximum, or a NaN (uniform)
-    if (!(bm < INFINITY)) {
-      L.bad = true;
-      return;
-    }
-    cr_raise(L, bm, c, ring);
-  }
-  if (L.base == 0u) return;  // every value so far is -inf: weight 0
-  const f32x2 cc = pack2(c, c), nn = pack2(L.nmc, L.nmc);
-  f32x2 a0 = pack2(0.0f, 0.0f), a1 = a0;
+// One to ring counter d = h - lb of a positive bf16 value h (the ring holds positive values
+// only; lb = lower - 0x8000 is the raw bits of its lowest value), taken from the value's bits
+// xf = h << 16 as a float's upper half: t = xf - (lb << 16) = d << 16, one add of nl16 =
+// -(lb << 16). A value below the ring wraps to a large t; a negative value (xf >= 2^31) gives
+// t >= 2^31 - (lb << 16) >= kCrRing << 16, as lb <= 0xFFFF - (kCrRing - 1) - 0x8000 = 0x7700.
+// Either lands on a discard counter: t is clamped to this lane's dl =
+// (kCrRing + lane) << 16, so that every value takes one unconditional reduction (a predicated
+// one costs a branch around it). The counter's shared address is ra + 4 d = ra + (t >> 14).
+// No memory effect is declared (see count_if_below).
+__device__ __forceinline__ void cr_count_pos(uint32_t xf, uint32_t nl16, uint32_t dl, uint32_t ra) {
+  asm volatile(
+      "{\n"
+      " .reg .u32 t;\n"
+      " add.u32 t, %0, %1;\n"
+      " min.u32 t, t, %2;\n"
+      " shr.u32 t, t, 14;\n"
+      " add.u32 t, t, %3;\n"
+      " red.shared.add.u32 [t], 1;\n"
+      "}" ::"r"(xf),
+      "r"(nl16), "r"(dl), "r"(ra));
+}
+
+// One step of a warp's range: kCrVec 16-byte vectors per lane (a range's last step and its
+// scalar edges padded with -inf, which weighs nothing and, on the positive-only path, lands on a
+// discard counter; rows whose window could reach -inf's key take the general select).
+struct CrStep {
+  uint4 v[kCrVec];
+};
+
+// Sums and counts of one step. FAST: the ring holds positive values only (counted from the raw
+// bits); otherwise every value is mapped to its 16-bit order key first.
+template <bool FAST>
+__device__ __forceinline__ void cr_absorb_sum(CrLane& L, const CrStep& raw, float c, uint32_t* ring) {
+  const uint32_t nl16 = L.nl16, dl = L.dl, ra = L.ra;
+  float a0 = 0.0f, a1 = 0.0f, a2 = 0.0f, a3 = 0.0f;
 #pragma unroll
   for (int j = 0; j < kCrVec; ++j) {
-    if (!(FULL || j < nvalid)) continue;
-    const uint32_t w[4] = {raw[j].x, raw[j].y, raw[j].z, raw[j].w};
+    const uint32_t w[4] = {raw.v[j].x, raw.v[j].y, raw.v[j].z, raw.v[j].w};
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      float e0, e1;
-      unpack2(fma2(pack2(__uint_as_float(w[q] << 16), __uint_as_float(w[q] & 0xFFFF0000u)), cc, nn), e0, e1);
-      if (q & 1) a1 = add2(a1, pack2(ex2(e0), ex2(e1)));
-      else a0 = add2(a0, pack2(ex2(e0), ex2(e1)));
-      if (L.fast) {
-        count_if_below(ring, L.kb - (w[q] & 0xFFFFu), kCrRing);
-        count_if_below(ring, L.kb - (w[q] >> 16), kCrRing);
+      const uint32_t lo = w[q] << 16, hi = w[q] & 0xFFFF0000u;  // the two values as float bits
+      const float e0 = ex2(fmaf(__uint_as_float(lo), c, L.nmc));
+      const float e1 = ex2(fmaf(__uint_as_float(hi), c, L.nmc));
+      if (q & 1) {
+        a2 += e0;
+        a3 += e1;
       } else {
-        count_if_below(ring, L.base - key16_bits(w[q] & 0xFFFFu), kCrRing);
-        count_if_below(ring, L.base - key16_bits(w[q] >> 16), kCrRing);
+        a0 += e0;
+        a1 += e1;
+      }
+      if (FAST) {
+        cr_count_pos(lo, nl16, dl, ra);
+        cr_count_pos(hi, nl16, dl, ra);
+      } else {
+        count_if_below(ring, key16_bits(lo >> 16) - L.lower, kCrRing);
+        count_if_below(ring, key16_bits(hi >> 16) - L.lower, kCrRing);
       }
     }
   }
-  float x0, x1, y0, y1;
-  unpack2(a0, x0, x1);
-  unpack2(a1, y0, y1);
-  L.s += (static_cast<double>(x0) + static_cast<double>(x1)) + (static_cast<double>(y0) + static_cast<double>(y1));
+  L.s += (static_cast<double>(a0) + static_cast<double>(a1)) + (static_cast<double>(a2) + static_cast<double>(a3));
+}
+
+// The per-step bookkeeping: this lane's maximum of the step (NaN and +inf flagged), the ring's
+// top following the warp's maximum (a vote per step; the move itself is rare), the lane's sum
+// rescaled when its maximum grows.
+__device__ __forceinline__ void cr_step_max(CrLane& L, const CrStep& raw, float c, uint32_t* ring) {
+  uint32_t pm = 0xFF80FF80u;  // packed bf16 pair (-inf, -inf)
+#pragma unroll
+  for (int j = 0; j < kCrVec; ++j)
+    pm = bmax2(pm, bmax2(bmax2(raw.v[j].x, raw.v[j].y), bmax2(raw.v[j].z, raw.v[j].w)));
+  const float lm = fmax_nan(__uint_as_float(pm << 16), __uint_as_float(pm & 0xFFFF0000u));
+  const bool finite = lm > -INFINITY && lm < INFINITY;
+  L.bad |= !(lm < INFINITY);  // NaN or +inf
+  const uint32_t lk = finite ? fkey(lm) >> 16 : 0u;
+  if (__any_sync(0xffffffffu, lk > L.top)) {
+    uint32_t wk = lk;
+#pragma unroll
+    for (int o = 16; o; o >>= 1) wk = max(wk, __shfl_xor_sync(0xffffffffu, wk, o));
+    L.top = cr_rebase(L.top, wk, ring);
+    L.lower = L.top - static_cast<uint32_t>(kCrRing - 1);
+    L.fast = L.lower > 0x8000u;
+    L.nl16 = (0x8000u - L.lower) << 16;
+  }
+  if (finite && lm > L.M) {  // this lane's maximum grows
+    if (L.M > -INFINITY) L.s *= static_cast<double>(ex2((L.M - lm) * c));
+    L.M = lm;
+    L.nmc = -lm * c;
+  }
+}
+
+// One step: bookkeeping, then sums and counts on the path the ring's keys allow (uniform).
+// Everything is inlined: a call inside the streaming loop would make the loop keep its values
+// in memory across it.
+__device__ __forceinline__ void cr_absorb(CrLane& L, const CrStep& raw, float c, uint32_t* ring) {
+  cr_step_max(L, raw, c, ring);
+  if (L.fast) cr_absorb_sum<true>(L, raw, c, ring);
+  else cr_absorb_sum<false>(L, raw, c, ring);
 }
 
 // This warp's range of row rp: the aligned body [a0, a1) split into kCrWarps runs of whole
@@ -198,52 +254,50 @@ __device__ __forceinline__ CrRange cr_range(const T* rp, int V, int w) {
 // Warp w streams its range of row rp (bf16) into L and its ring. Not inlined: the streaming
 // loop gets the registers to itself, apart from the row-end work of the caller.
 __device__ __noinline__ void cr_stream(const __nv_bfloat16* __restrict__ rp, int V, const CrRange r, float c,
-                                       CrLane& L, uint32_t* ring) {
+                                       CrLane& Lout, uint32_t* ring) {
   const int lane = threadIdx.x & 31;
+  CrLane L = Lout;  // in registers for the loop
+  L.dl = static_cast<uint32_t>(kCrRing + lane) << 16;
+  L.ra = smem_u32(ring);
+  constexpr uint32_t kNegInf2 = 0xFF80FF80u;  // packed bf16 pair (-inf, -inf)
   int a0, a1;
   vec_range(rp, 0, V, a0, a1);
   const uint4* body = reinterpret_cast<const uint4*>(rp + a0);
-  // scalar edges first (at most 7 elements): one element per lane, as a partial step
+  // scalar edges first (at most 7 elements): one element per lane, the rest -inf
   if (r.e1 > r.e0) {
-    uint4 raw[kCrVec];
+    CrStep raw;
     const int e = r.e0 + lane;
     const uint32_t h = e < r.e1 ? static_cast<uint32_t>(reinterpret_cast<const uint16_t*>(rp)[e]) : 0xFF80u;
-    raw[0] = make_uint4(h | 0xFF800000u, 0xFF80FF80u, 0xFF80FF80u, 0xFF80FF80u);
-    // the lanes past the edge hold -inf pairs, which neither weigh nor count (their keys lie
-    // far below any ring a finite maximum sets, except for rows of huge negative logits, which
-    // the caller sends to the general select)
-    cr_absorb<false>(L, raw, 1, c, ring);
+    raw.v[0] = make_uint4(h | 0xFF800000u, kNegInf2, kNegInf2, kNegInf2);
+#pragma unroll
+    for (int j = 1; j < kCrVec; ++j) raw.v[j] = make_uint4(kNegInf2, kNegInf2, kNegInf2, kNegInf2);
+    cr_absorb(L, raw, c, ring);
   }
   constexpr int kStep = 32 * kCrVec;  // vectors per warp step
   const int n = r.v1 - r.v0;
   const int steps = (n + kStep - 1) / kStep;
-  auto load = [&](uint4 (&buf)[kCrVec], int s) {
+  auto load = [&](CrStep& buf, int s) {
+    const uint4* p = body + r.v0 + s * kStep + lane;
+    if ((s + 1) * kStep <= n) {  // a full step (warp-uniform)
 #pragma unroll
-    for (int j = 0; j < kCrVec; ++j) {
-      const int i = s * kStep + j * 32 + lane;
-      buf[j] = i < n ? __ldg(body + r.v0 + i) : make_uint4(0xFF80FF80u, 0xFF80FF80u, 0xFF80FF80u, 0xFF80FF80u);
+      for (int j = 0; j < kCrVec; ++j) buf.v[j] = __ldg(p + j * 32);
+    } else {  // the range's last step: -inf past its end
+#pragma unroll
+      for (int j = 0; j < kCrVec; ++j)
+        buf.v[j] = s * kStep + j * 32 + lane < n ? __ldg(p + j * 32) : make_uint4(kNegInf2, kNegInf2, kNegInf2, kNegInf2);
     }
   };
-  auto absorb = [&](const uint4 (&buf)[kCrVec], int s) {
-    if ((s + 1) * kStep <= n) {
-      cr_absorb<true>(L, buf, kCrVec, c, ring);
-    } else {
-      // the last, partial step: this lane's valid vectors are the first nv of its kCrVec
-      const int left = n - s * kStep;
-      const int nv = left > lane ? (left - lane + 31) / 32 : 0;
-      cr_absorb<false>(L, buf, nv, c, ring);
-    }
-  };
-  uint4 A[kCrVec], B[kCrVec];
+  CrStep A, B;
   if (steps > 0) load(A, 0);
   for (int s = 0; s < steps; s += 2) {
     if (s + 1 < steps) load(B, s + 1);
-    absorb(A, s);
-    if (s + 1 >= steps || L.bad) break;
+    cr_absorb(L, A, c, ring);
+    if (s + 1 >= steps) break;
     if (s + 2 < steps) load(A, s + 2);
-    absorb(B, s + 1);
-    if (L.bad) break;
+    cr_absorb(L, B, c, ring);
   }
+  __syncwarp();  // the ring's reductions are complete before the caller's barrier
+  Lout = L;
 }
 
 // The count of window key `key` in the warps' rings (warps without a finite value add nothing;
@@ -252,7 +306,7 @@ __device__ __forceinline__ uint32_t cr_count(const CrSmem& sm, uint32_t key) {
   uint32_t c = 0u;
 #pragma unroll
   for (int w = 0; w < kCrWarps; ++w) {
-    const uint32_t d = sm.wb[w] - key;
+    const uint32_t d = key - sm.wl[w];
     if (sm.wm[w] > -INFINITY && d < static_cast<uint32_t>(kCrRing)) c += sm.ring[w][d];
   }
   return c;
@@ -344,14 +398,17 @@ __device__ void cut_rows_cta(const T* __restrict__ A, const T* __restrict__ Bt, 
       uint32_t* ring = sm.ring[warp];
       // every warp streams its range
       const CrRange r = cr_range(rp, V, warp);
-      CrLane L{-INFINITY, 0.0f, 0u, 0u, false, false, 0.0};
+      CrLane L{-INFINITY, 0.0f, 0.0, false, 0u, 0u, 0u, false, 0u, 0u};
       cr_stream(reinterpret_cast<const __nv_bfloat16*>(rp), V, r, c, L, ring);
-      const double sw = warp_sum(L.s);
+      // the warp: its maximum, and the lanes' sums brought to it
+      const float mw = warp_max(L.M);
+      const double sw = warp_sum(L.M > -INFINITY ? L.s * static_cast<double>(ex2((L.M - mw) * c)) : 0.0);
+      const bool badw = __any_sync(0xffffffffu, L.bad);
       if (lane == 0) {
-        sm.wm[warp] = L.M;
+        sm.wm[warp] = mw;
         sm.ws[warp] = sw;
-        sm.wb[warp] = L.base;
-        sm.wbad[warp] = L.bad ? 1 : 0;
+        sm.wl[warp] = L.top != 0u ? L.lower : 0u;
+        sm.wbad[warp] = badw ? 1 : 0;
       }
       __syncthreads();
       // the row: maximum, normaliser, status (the same arithmetic in every thread)
@@ -386,7 +443,7 @@ __device__ void cut_rows_cta(const T* __restrict__ A, const T* __restrict__ Bt, 
           double acc = 0.0;
           if (sm.wm[warp] > -INFINITY) {
             for (uint32_t key = km - static_cast<uint32_t>(lane); key >= ktau && key <= km; key -= 32u) {
-              const uint32_t d = sm.wb[warp] - key;
+              const uint32_t d = key - sm.wl[warp];
               if (d < static_cast<uint32_t>(kCrRing) && ring[d] != 0u)
                 acc += static_cast<double>(ring[d]) * static_cast<double>(ex2((key16_value(key) - m) * c));
               if (key < 32u) break;

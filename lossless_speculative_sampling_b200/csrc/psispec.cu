@@ -14,6 +14,7 @@
 #include "stats.cuh"
 #include "topp.cuh"
 #include "tree.cuh"
+#include "trie.cuh"
 
 namespace psi {
 namespace {
@@ -435,6 +436,62 @@ psispec_status row_stats_impl(const T* logits, int B, int K, int V, const float*
                 kCrThreads, smem, st, logits, a, static_cast<const Partial*>(parts));
 }
 
+struct TrieWs {
+  StatsWs st;
+  int32_t* cand_tok;
+  double* cand_q;
+  double* cand_l;
+  int32_t* ncand;
+};
+TrieWs carve_trie(Carver& c, int64_t rows, int64_t V) {
+  TrieWs w;
+  w.st = carve_stats(c, rows, nchunks_for(V));
+  w.cand_tok = c.take<int32_t>(rows * kTrieMaxCand);
+  w.cand_q = c.take<double>(rows * kTrieMaxCand);
+  w.cand_l = c.take<double>(rows * kTrieMaxCand);
+  w.ncand = c.take<int32_t>(rows);
+  return w;
+}
+
+// Candidate trie: row statistics of the B*K draft rows (with the sampling controls), the
+// candidates of every row, then the best-first choice per request.
+template <typename T>
+psispec_status build_tree_impl(const T* draft, int B, int K, int V, const float* temperature, const float* top_p,
+                               const int32_t* top_k, int cand_k, int n_prefixes, int32_t* out_parent,
+                               int32_t* out_tokens, int32_t* out_depth, double* out_score, int32_t* out_nodes,
+                               void* ws, cudaStream_t st) {
+  const int64_t rows = int64_t(B) * K;
+  Carver c(ws);
+  TrieWs w = carve_trie(c, rows, V);
+  psispec_status s = launch_stats<T>(one_tensor(draft, rows, K, B), rows, V, temperature, B, top_p, top_k,
+                                     Skip{top_p, top_k, kSkipNone}, w.st, st);
+  if (s != PSISPEC_OK) return s;
+  s = launch(trie_candidates_kernel<T>, static_cast<unsigned>(rows), kTrieThreads, 0, st, draft, V,
+             static_cast<const RowStat*>(w.st.stats), cand_k, w.cand_tok, w.cand_q, w.cand_l, w.ncand);
+  if (s != PSISPEC_OK) return s;
+  return launch(trie_select_kernel, static_cast<unsigned>(B), 32, 0, st, K, n_prefixes,
+                static_cast<const int32_t*>(w.cand_tok), static_cast<const double*>(w.cand_q),
+                static_cast<const double*>(w.cand_l), static_cast<const int32_t*>(w.ncand), out_parent, out_tokens,
+                out_depth, out_score, out_nodes);
+}
+
+// Tree verification of a trie whose children were fixed in advance: statistics of the
+// verifier rows, then one CTA per trie (no draft rows).
+template <typename T>
+psispec_status verify_tree_det_impl(const T* tgt, int B, int N, int V, const int32_t* offs, const int32_t* parent,
+                                    const int32_t* tokens, const float* u_acc, const float* u_res,
+                                    const float* temperature, const float* top_p, const int32_t* top_k,
+                                    int max_depth, int32_t* out_path, int32_t* out_tokens, int32_t* out_len, void* ws,
+                                    cudaStream_t st) {
+  Carver c(ws);
+  TreeWs w = carve_tree(c, N, V);
+  psispec_status s = launch_stats<T>(RowSet<T>{tgt, tgt, N, 1, offs, B}, int64_t(N), V, temperature, B, top_p, top_k,
+                                     Skip{top_p, top_k, kSkipNone}, w.st, st);
+  if (s != PSISPEC_OK) return s;
+  return launch(tree_walk_det_kernel<T>, static_cast<unsigned>(B), kTreeThreads, 0, st, tgt, V, offs, parent, tokens,
+                static_cast<const RowStat*>(w.st.stats), u_acc, u_res, max_depth, out_path, out_tokens, out_len);
+}
+
 bool bad_dtype(int dtype) { return dtype != PSISPEC_F32 && dtype != PSISPEC_BF16; }
 size_t esize(int dtype) { return dtype == PSISPEC_BF16 ? 2 : 4; }
 
@@ -476,6 +533,7 @@ size_t psispec_workspace_size(int op, int64_t a, int64_t b, int64_t c) {
     case PSISPEC_OP_VERIFY_LINEAR: carve_linear(m, a, b, c); break;
     case PSISPEC_OP_VERIFY_TREE: carve_tree(m, b, c); break;
     case PSISPEC_OP_ROW_STATS: carve_row_stats(m, a * b, c); break;
+    case PSISPEC_OP_BUILD_TREE: carve_trie(m, a * b, c); break;
     default: return 0;
   }
   return m.used;
@@ -636,6 +694,55 @@ psispec_status psispec_verify_linear_static(const void* target_logits, const voi
   return psispec_verify_linear(target_logits, draft_logits, dtype, B, K, V, draft_tokens, draft_row_stats, u_accept,
                                u_resid, temperature, top_p, out_tokens, out_accept_len, out_p, out_q, ws,
                                static_cast<size_t>(PSISPEC_STATIC_WORKSPACE_BYTES), stream);
+}
+
+psispec_status psispec_build_tree(const void* draft_logits, int dtype, int32_t B, int32_t K, int32_t V,
+                                  const float* temperature, const float* top_p, const int32_t* top_k, int32_t cand_k,
+                                  int32_t n_prefixes, int32_t* out_parent, int32_t* out_tokens, int32_t* out_depth,
+                                  double* out_score, int32_t* out_nodes, void* workspace, size_t workspace_bytes,
+                                  void* stream) {
+  if (!draft_logits || !temperature || !top_p || !out_parent || !out_tokens || !out_depth || !out_nodes ||
+      bad_dtype(dtype))
+    return PSISPEC_ERR_INVALID_ARG;
+  if (B <= 0 || K <= 0 || V <= 0 || cand_k <= 0 || n_prefixes <= 0) return PSISPEC_ERR_INVALID_ARG;
+  if (!aligned_to(draft_logits, esize(dtype))) return PSISPEC_ERR_INVALID_ARG;
+  const int64_t rows = int64_t(B) * K;
+  if (K > kTrieMaxK || cand_k > kTrieMaxCand || n_prefixes > kTrieMaxPrefixes || rows > kMaxRows || V > kMaxV ||
+      rows * nslices_for(V) > kMaxGrid)
+    return PSISPEC_ERR_UNSUPPORTED;
+  psispec_status s = check_ws(workspace, workspace_bytes, psispec_workspace_size(PSISPEC_OP_BUILD_TREE, B, K, V));
+  if (s != PSISPEC_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dtype == PSISPEC_BF16)
+    return build_tree_impl(static_cast<const __nv_bfloat16*>(draft_logits), B, K, V, temperature, top_p, top_k, cand_k,
+                           n_prefixes, out_parent, out_tokens, out_depth, out_score, out_nodes, workspace, st);
+  return build_tree_impl(static_cast<const float*>(draft_logits), B, K, V, temperature, top_p, top_k, cand_k,
+                         n_prefixes, out_parent, out_tokens, out_depth, out_score, out_nodes, workspace, st);
+}
+
+psispec_status psispec_verify_tree_det(const void* target_logits, int dtype, int32_t B, int32_t N, int32_t V,
+                                       const int32_t* node_offsets, const int32_t* parent, const int32_t* tokens,
+                                       const float* u_accept, const float* u_resid, const float* temperature,
+                                       const float* top_p, const int32_t* top_k, int32_t max_depth, int32_t* out_path,
+                                       int32_t* out_tokens, int32_t* out_accept_len, void* workspace,
+                                       size_t workspace_bytes, void* stream) {
+  if (!target_logits || !node_offsets || !parent || !tokens || !u_accept || !u_resid || !temperature || !top_p ||
+      !out_path || !out_tokens || !out_accept_len || bad_dtype(dtype))
+    return PSISPEC_ERR_INVALID_ARG;
+  if (B <= 0 || N < B || V <= 0 || max_depth < 1) return PSISPEC_ERR_INVALID_ARG;
+  if (!aligned_to(target_logits, esize(dtype))) return PSISPEC_ERR_INVALID_ARG;
+  if (max_depth > 64 || N > kMaxRows || V > kMaxV || int64_t(N) * nslices_for(V) > kMaxGrid)
+    return PSISPEC_ERR_UNSUPPORTED;
+  psispec_status s = check_ws(workspace, workspace_bytes, psispec_workspace_size(PSISPEC_OP_VERIFY_TREE, B, N, V));
+  if (s != PSISPEC_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dtype == PSISPEC_BF16)
+    return verify_tree_det_impl(static_cast<const __nv_bfloat16*>(target_logits), B, N, V, node_offsets, parent,
+                                tokens, u_accept, u_resid, temperature, top_p, top_k, max_depth, out_path, out_tokens,
+                                out_accept_len, workspace, st);
+  return verify_tree_det_impl(static_cast<const float*>(target_logits), B, N, V, node_offsets, parent, tokens, u_accept,
+                              u_resid, temperature, top_p, top_k, max_depth, out_path, out_tokens, out_accept_len,
+                              workspace, st);
 }
 
 }  // extern "C"

@@ -32,7 +32,9 @@
 namespace psi {
 
 // One to the shared-memory counter p[o] when o < n, as a predicated reduction (no branch;
-// p + o is not formed into an access otherwise).
+// p + o is not formed into an access otherwise). It declares no memory effect, so that the
+// compiler can schedule loads and arithmetic around it: callers order every other access to
+// the counters with a barrier (__syncthreads or __syncwarp) between them and the reductions.
 __device__ __forceinline__ void count_if_below(uint32_t* p, uint32_t o, uint32_t n) {
   asm volatile(
       "{\n"
@@ -40,8 +42,7 @@ __device__ __forceinline__ void count_if_below(uint32_t* p, uint32_t o, uint32_t
       " setp.lt.u32 q, %1, %2;\n"
       " @q red.shared.add.u32 [%0], 1;\n"
       "}" ::"r"(smem_u32(p) + 4u * o),
-      "r"(o), "r"(n)
-      : "memory");
+      "r"(o), "r"(n));
 }
 
 constexpr int kTpThreads = 256;
@@ -459,12 +460,10 @@ __device__ RowStat tp_row_stats(const T* __restrict__ row, int V, float Tv, floa
   return st;
 }
 
-// Top-p threshold of a bf16 row whose maximum m and normaliser s are already known (from the
-// streaming pass): every element with the same logit has the same weight, so counting the
-// elements of each of the kTpWindow representable values just below m gives their masses
-// exactly (count times one weight). One pass over the row, no exponential per element; the
-// threshold is the first value, from m down, at which the cumulative mass reaches top_p * s.
-// Returns false (and leaves st alone) when the window holds less than that.
+// The value window of a bf16 row: every element with the same logit has the same weight, so
+// counting the elements of each of the kTpWindow representable values just below the row
+// maximum m gives their masses exactly (count times one weight), and the cut is the first value,
+// from m down, at which the cumulative mass reaches top_p * s (window_pick).
 constexpr int kTpWindow = 2048;
 
 // The logit value of a 16-bit order key of a bf16 number (the inverse of fkey(x) >> 16 on
@@ -588,65 +587,10 @@ __device__ bool window_pick(uint32_t km, float tp, int k, RowStat& st, CountAt&&
   return true;
 }
 
-template <typename T>
-__device__ bool tp_window_select(const T* __restrict__ row, int V, float tp, int k, RowStat& st, TpSmem& sm) {
-  static_assert(sizeof(T) == 2, "bf16 rows");
-  static_assert(kTpWarps * kTpWindow <= kTpBins * kTpThreads, "window counts reuse the private counters");
-  uint32_t* cnt = &sm.priv[0][0];  // [kTpWarps][kTpWindow]
-  const int warp = threadIdx.x >> 5;
-  for (int i = threadIdx.x; i < kTpWarps * kTpWindow; i += kTpThreads) cnt[i] = 0u;
-  __syncthreads();
-  const uint32_t km = fkey(st.m) >> 16;
-  uint32_t* mine = cnt + warp * kTpWindow;
-  if (km >= 0x8000u + kTpWindow) {
-    // the window holds positive values only: a positive bf16 with bits h has the key
-    // h + 0x8000, so its offset is kb - h; negative values (h >= 0x8000) wrap to offsets far
-    // outside the window, so the raw bits are counted without any conversion
-    const uint32_t kb = km - 0x8000u;
-    const uint16_t* r16 = reinterpret_cast<const uint16_t*>(row);
-    auto count = [&](uint32_t h) { count_if_below(mine, kb - h, kTpWindow); };
-    int a0, a1;
-    vec_range(row, 0, V, a0, a1);
-    for (int v = threadIdx.x; v < a0; v += kTpThreads) count(r16[v]);
-    for (int v = a1 + threadIdx.x; v < V; v += kTpThreads) count(r16[v]);
-    constexpr int kLoads = 4, kStep = kTpThreads * 8;
-    for (int v = a0 + threadIdx.x * 8; v < a1; v += kLoads * kStep) {
-      uint4 raw[kLoads];
-#pragma unroll
-      for (int i = 0; i < kLoads; ++i)
-        if (v + i * kStep < a1) raw[i] = __ldcg(reinterpret_cast<const uint4*>(row + v + i * kStep));
-#pragma unroll
-      for (int i = 0; i < kLoads; ++i) {
-        if (v + i * kStep < a1) {
-          const uint32_t w[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            count(w[k] & 0xFFFFu);
-            count(w[k] >> 16);
-          }
-        }
-      }
-    }
-  } else {
-    tp_for_each8<T, 4>(row, V, [&](const float (&x)[8]) {
-#pragma unroll
-      for (int k = 0; k < 8; ++k) count_if_below(mine, km - (fkey(x[k]) >> 16), kTpWindow);
-    });
-  }
-  __syncthreads();
-  return window_pick<kTpThreads>(
-      km, tp, k, st, [&](int o) {
-        uint32_t c = 0u;
-#pragma unroll
-        for (int w = 0; w < kTpWarps; ++w) c += cnt[w * kTpWindow + o];
-        return c;
-      },
-      sm.mass, &sm.bin, &sm.tgt, &sm.base);
-}
-
-// Statistics of a row of a request with a top-p or top-k cut: maximum and normaliser from the
-// row's chunk partials, the threshold from the value window (bf16), else passes A-C over the
-// row (top-p alone) or the general radix select (top-k). k is the request's top-k (0: off).
+// Statistics of a row of a request with a top-p or top-k cut from the row's chunk partials
+// (the fp32 rows; bf16 rows take the one-pass path of cutrow.cuh): the general top-k then top-p
+// radix select from the partials' maximum and normaliser, or passes A-C over the row (top-p
+// alone). k is the request's top-k (0: off).
 template <typename T>
 __device__ RowStat tp_row_stats_partials(const T* __restrict__ row, int V, float Tv, float tp, int k,
                                          const Partial* __restrict__ pp, TpSmem& sm) {
@@ -658,9 +602,6 @@ __device__ RowStat tp_row_stats_partials(const T* __restrict__ row, int V, float
   RowStat st = sm.st;
   __syncthreads();
   if (st.status != 0) return st;
-  if constexpr (sizeof(T) == 2) {
-    if (tp_window_select<T>(row, V, tp, k, st, sm)) return st;
-  }
   if (k > 0) {
     block_topk_topp_radix<T>(row, V, tp, k, st, sm.radix);
     return st;

@@ -23,7 +23,7 @@ HEADER = os.path.join(os.path.dirname(_HERE), "include", "psispec.h")
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_WORKSPACE = 0, 1, 2, 3, 4
 STATIC_WORKSPACE_BYTES = 16 << 20  # PSISPEC_STATIC_WORKSPACE_BYTES
 F32, BF16 = 0, 1
-OP_SAMPLE_DRAFT, OP_VERIFY_LINEAR, OP_VERIFY_TREE, OP_ROW_STATS = 0, 1, 2, 3
+OP_SAMPLE_DRAFT, OP_VERIFY_LINEAR, OP_VERIFY_TREE, OP_ROW_STATS, OP_BUILD_TREE = 0, 1, 2, 3, 4
 ROW_STATS_BYTES = 32
 
 _lib = None
@@ -58,10 +58,13 @@ def lib():
         L.psispec_verify_tree_k.argtypes = [P, P, ctypes.c_int, I32, I32, I32, P, P, P, P, P, P, P, P, I32, P, P, P, P,
                                             SZ, P]
         L.psispec_row_stats_k.argtypes = [P, ctypes.c_int, I32, I32, I32, P, P, P, P, P, SZ, P]
+        L.psispec_build_tree.argtypes = [P, ctypes.c_int, I32, I32, I32, P, P, P, I32, I32, P, P, P, P, P, P, SZ, P]
+        L.psispec_verify_tree_det.argtypes = [P, ctypes.c_int, I32, I32, I32, P, P, P, P, P, P, P, P, I32, P, P, P, P,
+                                              SZ, P]
         L.psispec_verify_linear_static.argtypes = [P, P, ctypes.c_int, I32, I32, I32, P, P, P, P, P, P, P, P, P, P, P]
         for f in ("psispec_sample_draft", "psispec_sample_draft_k", "psispec_row_stats", "psispec_row_stats_k",
                   "psispec_verify_linear", "psispec_verify_linear_k", "psispec_verify_tree", "psispec_verify_tree_k",
-                  "psispec_verify_linear_static"):
+                  "psispec_verify_linear_static", "psispec_build_tree", "psispec_verify_tree_det"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -305,3 +308,70 @@ def verify_linear_static(target, draft, draft_tokens, u_accept, u_resid, tempera
                                             _stream(dev, stream))
     _check(st, "psispec_verify_linear_static")
     return {"tokens": out_tokens, "accept_len": out_accept_len, "p": out_p, "q": out_q}
+
+def build_tree(draft, temperature, top_p, cand_k: int, n_prefixes: int, *, top_k=None, out=None, ws=None,
+               stream=None):
+    """Candidate trie of the tree sampler from draft rows [B, K, V] (bf16/fp32): the cand_k
+    most probable tokens per position, then the n_prefixes most probable prefixes.
+    Returns dict(parent, tokens, depth [B, n_prefixes+1] int32, score [B, n_prefixes+1] fp64,
+    nodes [B] int32); `out` may hold those tensors to write into."""
+    B, K, V = draft.shape
+    dev = draft.device
+    _req(draft, "draft")
+    _req(temperature, "temperature", torch.float32, B, dev)
+    _req(top_p, "top_p", torch.float32, B, dev)
+    if top_k is not None:
+        _req(top_k, "top_k", torch.int32, B, dev)
+    cap = int(n_prefixes) + 1
+    out = {} if out is None else out
+    par = out.get("parent") if out.get("parent") is not None else torch.empty((B, cap), dtype=torch.int32, device=dev)
+    tok = out.get("tokens") if out.get("tokens") is not None else torch.empty((B, cap), dtype=torch.int32, device=dev)
+    dep = out.get("depth") if out.get("depth") is not None else torch.empty((B, cap), dtype=torch.int32, device=dev)
+    score = out.get("score") if out.get("score") is not None else torch.empty((B, cap), dtype=torch.float64,
+                                                                              device=dev)
+    nodes = out.get("nodes") if out.get("nodes") is not None else torch.empty(B, dtype=torch.int32, device=dev)
+    for name, t, dt in (("parent", par, torch.int32), ("tokens", tok, torch.int32), ("depth", dep, torch.int32),
+                        ("score", score, torch.float64)):
+        _req(t, name, dt, B * cap, dev)
+    _req(nodes, "nodes", torch.int32, B, dev)
+    need = workspace_size(OP_BUILD_TREE, B, K, V)
+    ws = workspace(need, dev) if ws is None else ws
+    st = lib().psispec_build_tree(_p(draft), _dtype(draft), B, K, V, _p(temperature), _p(top_p), _p(top_k),
+                                  int(cand_k), int(n_prefixes), _p(par), _p(tok), _p(dep), _p(score), _p(nodes),
+                                  _p(ws), ws.numel(), _stream(dev, stream))
+    _check(st, "psispec_build_tree")
+    return {"parent": par, "tokens": tok, "depth": dep, "score": score, "nodes": nodes}
+
+
+def verify_tree_det(target, node_offsets, parent, tokens, u_accept, u_resid, temperature, top_p, max_depth: int, *,
+                    top_k=None, out_path=None, out_tokens=None, out_accept_len=None, ws=None, stream=None):
+    """Tree verification of a trie whose children were fixed in advance (the candidate trie):
+    target [N, V]; node_offsets [B+1]; parent, tokens [N] int32; u_accept, u_resid [N] fp32;
+    temperature/top_p [B]; top_k [B] int32 or None. Returns dict(path, tokens, accept_len)."""
+    N, V = target.shape
+    B = node_offsets.numel() - 1
+    dev = target.device
+    _req(target, "target")
+    _req(node_offsets, "node_offsets", torch.int32, B + 1, dev)
+    for name, t in (("parent", parent), ("tokens", tokens)):
+        _req(t, name, torch.int32, N, dev)
+    for name, t in (("u_accept", u_accept), ("u_resid", u_resid)):
+        _req(t, name, torch.float32, N, dev)
+    _req(temperature, "temperature", torch.float32, B, dev)
+    _req(top_p, "top_p", torch.float32, B, dev)
+    if top_k is not None:
+        _req(top_k, "top_k", torch.int32, B, dev)
+    out_path = torch.empty((B, max_depth), dtype=torch.int32, device=dev) if out_path is None else out_path
+    out_tokens = torch.empty((B, max_depth + 1), dtype=torch.int32, device=dev) if out_tokens is None else out_tokens
+    out_len = torch.empty(B, dtype=torch.int32, device=dev) if out_accept_len is None else out_accept_len
+    _req(out_path, "out_path", torch.int32, B * max_depth, dev)
+    _req(out_tokens, "out_tokens", torch.int32, B * (max_depth + 1), dev)
+    _req(out_len, "out_accept_len", torch.int32, B, dev)
+    need = workspace_size(OP_VERIFY_TREE, B, N, V)
+    ws = workspace(need, dev) if ws is None else ws
+    st = lib().psispec_verify_tree_det(_p(target), _dtype(target), B, N, V, _p(node_offsets), _p(parent), _p(tokens),
+                                       _p(u_accept), _p(u_resid), _p(temperature), _p(top_p), _p(top_k),
+                                       int(max_depth), _p(out_path), _p(out_tokens), _p(out_len), _p(ws), ws.numel(),
+                                       _stream(dev, stream))
+    _check(st, "psispec_verify_tree_det")
+    return {"path": out_path, "tokens": out_tokens, "accept_len": out_len}

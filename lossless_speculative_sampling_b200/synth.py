@@ -17,6 +17,11 @@ section 5.1; these synthetic rows stand in for the verifier and drafter heads):
                                   N(0, 2^2), draft noise 0.5), child tokens drawn without
                                   replacement from the parent's draft distribution
   sweep    B in {1, 32, 256}, K=32, V=151936, bf16, draft std 0.5, T in {0, 0.7, 1}, top-p 0.9
+  trie     the tree sampler's candidate trie: B=16 requests, K=15 drafted positions (a block of
+           16 whose first token is the verifier's), V=151936, bf16, draft rows N(0, 2^2), T=1;
+           cand_k=32 candidates per position, 32 kept prefixes (review page section 3.4's
+           single-request optimum) or 60 (the README's tree example); the verifier row of a
+           node at depth d is the draft row of position d plus N(0, 0.5^2)
 
 Uniforms are fp32 values k * 2^-24 (k a uniform 24-bit integer from numpy's PCG64), so fp32
 and fp64 consumers see the same numbers.
@@ -104,6 +109,60 @@ def _draft_std(case, B, seed):
         rng = np.random.Generator(np.random.PCG64(seed + 7))
         return torch.from_numpy(rng.uniform(lo, hi, size=B).astype(np.float32))
     return torch.full((B,), float(case.draft_std))
+
+
+@dataclass
+class TrieCase:
+    name: str
+    B: int
+    K: int
+    V: int
+    dtype: torch.dtype
+    draft_std: float
+    target_noise: float
+    temperature: float
+    top_p: float
+    cand_k: int
+    n_prefixes: int
+    seed: int = 0
+
+
+def trie_cases():
+    bf = torch.bfloat16
+    return {
+        "trie_32": TrieCase("trie_32", 16, 15, V_QWEN, bf, 2.0, 0.5, 1.0, 1.0, 32, 32, seed=1005),
+        "trie_60": TrieCase("trie_60", 16, 15, V_QWEN, bf, 2.0, 0.5, 1.0, 1.0, 32, 60, seed=1006),
+    }
+
+
+def trie_draft(case: TrieCase, device="cpu"):
+    """Draft rows [B, K, V] of the candidate-trie workload."""
+    dev = torch.device(device)
+    g = _gen(dev, case.seed)
+    d = torch.randn((case.B, case.K, case.V), generator=g, device=dev, dtype=torch.float32) * case.draft_std
+    return d.to(case.dtype)
+
+
+def trie_verifier_rows(case: TrieCase, draft: torch.Tensor, depth: torch.Tensor):
+    """Verifier rows of the trie's nodes: [B * (n_prefixes + 1), V] for depth [B, n_prefixes + 1]
+    (a node at depth d < K gets draft row d plus noise; depth K or an unused slot, noise alone)."""
+    B, K, V = draft.shape
+    dev = draft.device
+    g = _gen(dev, case.seed + 1)
+    dep = depth.to(dev).long().clamp(min=0)
+    base = torch.zeros((B, dep.shape[1], V), dtype=torch.float32, device=dev)
+    has = dep < K
+    idx = dep.clamp(max=K - 1)
+    rows = torch.gather(draft.float(), 1, idx.unsqueeze(-1).expand(-1, -1, V))
+    base = torch.where(has.unsqueeze(-1), rows, base)
+    noise = torch.randn(base.shape, generator=g, device=dev, dtype=torch.float32) * case.target_noise
+    return (base + noise).to(case.dtype).reshape(-1, V)
+
+
+def trie_uniforms(case: TrieCase):
+    n = case.B * (case.n_prefixes + 1)
+    s = case.seed * 16
+    return uniforms((n,), s + 2), uniforms((n,), s + 3)
 
 
 def linear_logits(case: LinearCase, device="cpu", B: int | None = None, chunk_rows: int = 2048):

@@ -148,6 +148,24 @@ def test_topk_entries_host_checks(L):
     assert row_stats_k(wsb=16) == psispec.ERR_WORKSPACE
 
 
+def test_build_tree_host_checks(L):
+    def bt(**kw):
+        a = dict(d=FAKE, B=2, K=3, V=100, ck=4, n=10, par=FAKE, ws=FAKE, wsb=1 << 30)
+        a.update(kw)
+        return L.psispec_build_tree(a["d"], psispec.BF16, a["B"], a["K"], a["V"], FAKE, FAKE, None, a["ck"], a["n"],
+                                    a["par"], FAKE, FAKE, None, FAKE, a["ws"], a["wsb"], None)
+
+    assert bt(d=None) == psispec.ERR_INVALID_ARG
+    assert bt(par=None) == psispec.ERR_INVALID_ARG
+    assert bt(ck=0) == psispec.ERR_INVALID_ARG
+    assert bt(n=0) == psispec.ERR_INVALID_ARG
+    assert bt(K=17) == psispec.ERR_UNSUPPORTED
+    assert bt(ck=33) == psispec.ERR_UNSUPPORTED
+    assert bt(n=65) == psispec.ERR_UNSUPPORTED
+    assert bt(ws=None) == psispec.ERR_WORKSPACE
+    assert psispec.workspace_size(psispec.OP_BUILD_TREE, 4, 16, 151936) > 0
+
+
 def _tree(L, **kw):
     a = dict(t=FAKE, d=FAKE, dtype=psispec.BF16, B=2, N=10, V=64, off=FAKE, par=FAKE, tok=FAKE, ua=FAKE, ur=FAKE,
              T=FAKE, P=FAKE, md=4, op=FAKE, ot=FAKE, ol=FAKE, ws=FAKE, wsb=1 << 30)
