@@ -42,7 +42,7 @@ namespace psi {
 
 constexpr int kCrWarps = 8;                   // warps per CTA, each one contiguous range of the row
 constexpr int kCrThreads = kCrWarps * 32;
-constexpr int kCrHead = 256;                  // keys of headroom above a warp's maximum at its ring base
+constexpr int kCrHead = 256;                  // keys of headroom above a warp's maximum at its ring's top
 constexpr int kCrRing = kTpWindow + kCrHead;  // counters per warp
 constexpr int kCrVec = 4;                     // 16-byte vectors per lane per step
 static_assert(kCrRing % 32 == 0, "ring shifts move 32 counters per step");
@@ -85,7 +85,7 @@ struct CrSmem {
 // or +inf logit was seen. Uniform across the warp: the ring's keys.
 struct CrLane {
   float M;         // this lane's running maximum; -inf before its first finite value
-  float nmc;       // -M c (0 while M is -inf, so that -inf values weigh exp2(-inf) = 0)
+  float mref;      // M, or 0 while M is -inf (so that -inf values weigh exp2(-inf) = 0)
   double s;        // this lane's sum of 2^((x - M) c)
   bool bad;        // this lane saw a NaN or +inf logit
   uint32_t top;    // the ring's top key (uniform); 0 before the warp's first finite value
@@ -132,7 +132,7 @@ __device__ __forceinline__ uint32_t cr_rebase(uint32_t top, uint32_t kmax, uint3
 // only; lb = lower - 0x8000 is the raw bits of its lowest value), taken from the value's bits
 // xf = h << 16 as a float's upper half: t = xf - (lb << 16) = d << 16, one add of nl16 =
 // -(lb << 16). A value below the ring wraps to a large t; a negative value (xf >= 2^31) gives
-// t >= 2^31 - (lb << 16) >= kCrRing << 16, as lb <= 0xFFFF - (kCrRing - 1) - 0x8000 = 0x7700.
+// t >= 2^31 - (lb << 16) >= kCrRing << 16, as lb <= 0xFFFF - (kCrRing - 1) - 0x8000.
 // Either lands on a discard counter: t is clamped to this lane's dl =
 // (kCrRing + lane) << 16, so that every value takes one unconditional reduction (a predicated
 // one costs a branch around it). The counter's shared address is ra + 4 d = ra + (t >> 14).
@@ -162,22 +162,21 @@ struct CrStep {
 template <bool FAST>
 __device__ __forceinline__ void cr_absorb_sum(CrLane& L, const CrStep& raw, float c, uint32_t* ring) {
   const uint32_t nl16 = L.nl16, dl = L.dl, ra = L.ra;
-  float a0 = 0.0f, a1 = 0.0f, a2 = 0.0f, a3 = 0.0f;
+  // weights 2^((x - M) c) with the difference and the product each rounded, the arithmetic of
+  // every other weight in the library (x c - M c in one fused step would round M c once, off by
+  // up to half an ulp of M c for every weight alike, and overflow for |M| near the float range)
+  const f32x2 mm = pack2(L.mref, L.mref), cc = pack2(c, c);
+  f32x2 p0 = pack2(0.0f, 0.0f), p1 = p0;
 #pragma unroll
   for (int j = 0; j < kCrVec; ++j) {
     const uint32_t w[4] = {raw.v[j].x, raw.v[j].y, raw.v[j].z, raw.v[j].w};
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       const uint32_t lo = w[q] << 16, hi = w[q] & 0xFFFF0000u;  // the two values as float bits
-      const float e0 = ex2(fmaf(__uint_as_float(lo), c, L.nmc));
-      const float e1 = ex2(fmaf(__uint_as_float(hi), c, L.nmc));
-      if (q & 1) {
-        a2 += e0;
-        a3 += e1;
-      } else {
-        a0 += e0;
-        a1 += e1;
-      }
+      float d0, d1;
+      unpack2(mul2(sub2(pack2(__uint_as_float(lo), __uint_as_float(hi)), mm), cc), d0, d1);
+      if (q & 1) p1 = add2(p1, pack2(ex2(d0), ex2(d1)));
+      else p0 = add2(p0, pack2(ex2(d0), ex2(d1)));
       if (FAST) {
         cr_count_pos(lo, nl16, dl, ra);
         cr_count_pos(hi, nl16, dl, ra);
@@ -187,6 +186,9 @@ __device__ __forceinline__ void cr_absorb_sum(CrLane& L, const CrStep& raw, floa
       }
     }
   }
+  float a0, a1, a2, a3;
+  unpack2(p0, a0, a1);
+  unpack2(p1, a2, a3);
   L.s += (static_cast<double>(a0) + static_cast<double>(a1)) + (static_cast<double>(a2) + static_cast<double>(a3));
 }
 
@@ -214,7 +216,7 @@ __device__ __forceinline__ void cr_step_max(CrLane& L, const CrStep& raw, float 
   if (finite && lm > L.M) {  // this lane's maximum grows
     if (L.M > -INFINITY) L.s *= static_cast<double>(ex2((L.M - lm) * c));
     L.M = lm;
-    L.nmc = -lm * c;
+    L.mref = lm;
   }
 }
 
@@ -312,12 +314,32 @@ __device__ __forceinline__ uint32_t cr_count(const CrSmem& sm, uint32_t key) {
   return c;
 }
 
-// Shared memory of a CTA of the row kernels: the one-pass cut rows, or the general selects
-// (the rows whose cut lies outside the window, and fp32 rows).
-union CutSmem {
+// Shared memory of the general selects of a bf16 row whose cut lies outside the window: the
+// block histogram select (and the radix selects inside it), the block draw.
+struct GenSmem {
+  ToppSmem topp;
+  DrawSmem draw;
+  int flag;
+};
+
+// Shared memory of a CTA of the row kernels: bf16, the one-pass cut rows or the general
+// selects; fp32, the general selects from the streaming pass's partials.
+template <typename T>
+union CutSmem;
+template <>
+union CutSmem<__nv_bfloat16> {
   CrSmem cr;
+  GenSmem gen;
+};
+template <>
+union CutSmem<float> {
   TpSmem tp;
 };
+
+// CTAs per SM of the row kernels (their registers: a third CTA per SM would cap them at 80,
+// where the streaming loop spills).
+template <typename T>
+constexpr int kRowCtas = 2;
 
 // Finish a row once its record st is known: the draw (sampling), the arrival and, for the last
 // arrival of a request, the accept tests (verification), or the record alone (statistics).
@@ -350,21 +372,32 @@ __device__ __forceinline__ void cut_row_finish(const T* __restrict__ A, const T*
 template <typename T>
 __device__ __noinline__ void cut_row_general(const T* __restrict__ A, const T* __restrict__ Bt, const CutArgs& a,
                                              const VerifyArgs& va, const Partial* __restrict__ parts_a,
-                                             const Partial* __restrict__ parts_b, TpSmem& sm, const T* rp,
+                                             const Partial* __restrict__ parts_b, CutSmem<T>& smu, const T* rp,
                                              RowStat* rec, RowStat st, bool in_b, int row, int req, float Tv,
                                              float tp, int k, float u) {
   const int V = a.V;
-  if constexpr (sizeof(T) == 2) {
-    if (k > 0) block_topk_topp_radix<T>(rp, V, tp, k, st, sm.radix);
-    else st = tp_row_stats(rp, V, Tv, tp, sm);
-  } else {
-    const Partial* pp = (in_b ? parts_b : parts_a) + static_cast<size_t>(row) * nchunks_for(V);
-    st = tp_row_stats_partials(rp, V, Tv, tp, k, pp, sm);
-  }
   int y = -1;
   float q = -1.0f;
-  if (a.mode == kCutSample && st.status == 0) y = tp_row_draw(rp, V, st, u, sm, &q);
-  cut_row_finish<T>(A, Bt, a, va, rec, st, row, req, y, q, &sm.flag);
+  if constexpr (sizeof(T) == 2) {
+    // m, c and s from the one pass; the threshold by the block selects, the draw over the row
+    GenSmem& sm = smu.gen;
+    if (k > 0) block_topk_topp_radix<T>(rp, V, tp, k, st, sm.topp.radix);
+    else block_topp_select<T>(rp, V, tp, st, sm.topp);
+    if (a.mode == kCutSample && st.status == 0) {
+      JobRows<T, false> J;
+      J.init(rp, st, nullptr, st);
+      y = block_draw_range(J, 0, V, 0.0, -1.0, u, sm.draw);
+      if (y >= 0) q = kept_weight(st, load_elem(rp + y)) / st.s_kept;
+    }
+    cut_row_finish<T>(A, Bt, a, va, rec, st, row, req, y, q, &sm.flag);
+  } else {
+    (void)Tv;
+    TpSmem& sm = smu.tp;
+    const Partial* pp = (in_b ? parts_b : parts_a) + static_cast<size_t>(row) * nchunks_for(V);
+    st = tp_row_stats_partials(rp, V, Tv, tp, k, pp, sm);
+    if (a.mode == kCutSample && st.status == 0) y = tp_row_draw(rp, V, st, u, sm, &q);
+    cut_row_finish<T>(A, Bt, a, va, rec, st, row, req, y, q, &sm.flag);
+  }
   __syncthreads();
 }
 
@@ -376,7 +409,7 @@ __device__ __noinline__ void cut_row_general(const T* __restrict__ A, const T* _
 template <typename T>
 __device__ void cut_rows_cta(const T* __restrict__ A, const T* __restrict__ Bt, const CutArgs& a,
                              const VerifyArgs& va, const Partial* __restrict__ parts_a,
-                             const Partial* __restrict__ parts_b, int cta, int nctas, CutSmem& smu) {
+                             const Partial* __restrict__ parts_b, int cta, int nctas, CutSmem<T>& smu) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int V = a.V;
   const int total = a.rows_a + a.rows_b;
@@ -493,30 +526,30 @@ __device__ void cut_rows_cta(const T* __restrict__ A, const T* __restrict__ Bt, 
       }
       __syncthreads();  // the general select below reuses the shared memory
       if (bad) {
-        cut_row_finish<T>(A, Bt, a, va, rec, st, row, req, -1, -1.0f, &smu.tp.flag);
+        cut_row_finish<T>(A, Bt, a, va, rec, st, row, req, -1, -1.0f, &smu.gen.flag);
         __syncthreads();
         continue;
       }
     }
-    cut_row_general<T>(A, Bt, a, va, parts_a, parts_b, smu.tp, rp, rec, st, in_b, row, req, Tv, tp, k, u);
+    cut_row_general<T>(A, Bt, a, va, parts_a, parts_b, smu, rp, rec, st, in_b, row, req, Tv, tp, k, u);
   }
 }
 
 // Row statistics of the cut requests' rows alone (psispec_row_stats): one CTA per row at a
 // time.
 template <typename T>
-__global__ void __launch_bounds__(kCrThreads, 2) cut_rows_kernel(const T* __restrict__ A, CutArgs a,
+__global__ void __launch_bounds__(kCrThreads, kRowCtas<T>) cut_rows_kernel(const T* __restrict__ A, CutArgs a,
                                                                 const Partial* __restrict__ parts) {
   extern __shared__ __align__(16) unsigned char cut_smem_raw[];
   VerifyArgs none{};
-  cut_rows_cta<T>(A, nullptr, a, none, parts, nullptr, blockIdx.x, gridDim.x, *reinterpret_cast<CutSmem*>(cut_smem_raw));
+  cut_rows_cta<T>(A, nullptr, a, none, parts, nullptr, blockIdx.x, gridDim.x, *reinterpret_cast<CutSmem<T>*>(cut_smem_raw));
 }
 
 // The row kernel of sample_draft. CTAs [0, warp_ctas) finish the rows without a cut, one
 // warp per row; the remaining CTAs take the rows of requests with a cut (cut_rows_cta). One
 // launch serves both kinds of rows.
 template <typename T>
-__global__ void __launch_bounds__(kTpThreads, 2) sample_rows_kernel(const T* __restrict__ draft, int K, int V,
+__global__ void __launch_bounds__(kTpThreads, kRowCtas<T>) sample_rows_kernel(const T* __restrict__ draft, int K, int V,
                                                                    int rows, const float* __restrict__ temperature,
                                                                    const float* __restrict__ top_p,
                                                                    const int32_t* __restrict__ top_k,
@@ -549,7 +582,7 @@ __global__ void __launch_bounds__(kTpThreads, 2) sample_rows_kernel(const T* __r
   a.stats_b = nullptr;
   VerifyArgs none{};
   cut_rows_cta<T>(draft, nullptr, a, none, parts, nullptr, static_cast<int>(blockIdx.x) - warp_ctas,
-                  static_cast<int>(gridDim.x) - warp_ctas, *reinterpret_cast<CutSmem*>(cut_smem_raw));
+                  static_cast<int>(gridDim.x) - warp_ctas, *reinterpret_cast<CutSmem<T>*>(cut_smem_raw));
 }
 
 // The row kernel of verify_linear. CTAs [0, warp_ctas) finish the rows of requests without a
@@ -557,7 +590,7 @@ __global__ void __launch_bounds__(kTpThreads, 2) sample_rows_kernel(const T* __r
 // (cut_rows_cta). Every row then arrives on its request's counter, and whoever completes a
 // request runs its accept tests and writes the draw job.
 template <typename T>
-__global__ void __launch_bounds__(kTpThreads, 2) verify_rows_kernel(const T* __restrict__ tgt,
+__global__ void __launch_bounds__(kTpThreads, kRowCtas<T>) verify_rows_kernel(const T* __restrict__ tgt,
                                                                    const T* __restrict__ drf, VerifyArgs va,
                                                                    int warp_ctas) {
   const int K = va.K, V = va.V;
@@ -583,7 +616,7 @@ __global__ void __launch_bounds__(kTpThreads, 2) verify_rows_kernel(const T* __r
   a.stats_a = va.stats_t;
   a.stats_b = va.stats_d;
   cut_rows_cta<T>(tgt, drf, a, va, va.parts_t, va.parts_d, static_cast<int>(blockIdx.x) - warp_ctas,
-                  static_cast<int>(gridDim.x) - warp_ctas, *reinterpret_cast<CutSmem*>(cut_smem_raw));
+                  static_cast<int>(gridDim.x) - warp_ctas, *reinterpret_cast<CutSmem<T>*>(cut_smem_raw));
 }
 
 }  // namespace psi

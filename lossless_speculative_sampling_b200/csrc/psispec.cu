@@ -263,9 +263,9 @@ psispec_status launch_draws(const T* A, const T* Bt, int V, int njobs, const Par
 }
 
 // The cut-row CTAs of a row kernel: persistent (one per resident slot) over the call's rows.
-template <typename Kern>
+template <typename T, typename Kern>
 psispec_status prepare_topp(Kern kernel, int64_t rows, unsigned* grid) {
-  const int smem = static_cast<int>(sizeof(CutSmem));
+  const int smem = static_cast<int>(sizeof(CutSmem<T>));
   if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return PSISPEC_ERR_CUDA;
   *grid = static_cast<unsigned>(want_slots(rows, 1, kernel, kTpThreads, smem));
@@ -286,9 +286,9 @@ psispec_status sample_draft_impl(const T* draft, int B, int K, int V, const floa
                                       cut_skip<T>(top_p, top_k));
   if (s != PSISPEC_OK) return s;
   unsigned tgrid = 1;
-  if ((s = prepare_topp(sample_rows_kernel<T>, rows, &tgrid)) != PSISPEC_OK) return s;
+  if ((s = prepare_topp<T>(sample_rows_kernel<T>, rows, &tgrid)) != PSISPEC_OK) return s;
   const int warp_ctas = static_cast<int>((rows + kTpWarps - 1) / kTpWarps);
-  return launch(sample_rows_kernel<T>, warp_ctas + tgrid, kTpThreads, sizeof(CutSmem), st, draft, K, V,
+  return launch(sample_rows_kernel<T>, warp_ctas + tgrid, kTpThreads, sizeof(CutSmem<T>), st, draft, K, V,
                 static_cast<int>(rows), temperature, top_p, top_k, u, w.st.parts, stats, out_tokens, out_q, warp_ctas);
 }
 
@@ -334,9 +334,9 @@ psispec_status verify_linear_impl(const T* tgt, const T* drf, int B, int K, int 
     return s;
   // one row kernel: warps for the requests without a cut, whole CTAs for the others
   unsigned tgrid = 1;
-  if ((s = prepare_topp(verify_rows_kernel<T>, rows_t + rows_d, &tgrid)) != PSISPEC_OK) return s;
+  if ((s = prepare_topp<T>(verify_rows_kernel<T>, rows_t + rows_d, &tgrid)) != PSISPEC_OK) return s;
   const int warp_ctas = static_cast<int>((rows_t + rows_d + kTpWarps - 1) / kTpWarps);
-  s = launch(verify_rows_kernel<T>, warp_ctas + tgrid, kTpThreads, sizeof(CutSmem), st, tgt, drf, a, warp_ctas);
+  s = launch(verify_rows_kernel<T>, warp_ctas + tgrid, kTpThreads, sizeof(CutSmem<T>), st, tgt, drf, a, warp_ctas);
   if (s != PSISPEC_OK) return s;
   return launch_draws<T>(tgt, drf, V, B, w.t.parts, w.jobs, w.draw_tc, w.draw_tg, out_tokens, st);
 }
@@ -418,7 +418,7 @@ psispec_status row_stats_impl(const T* logits, int B, int K, int V, const float*
       launch_stats<T>(one_tensor(logits, rows, K, B), rows, V, temperature, B, top_p, top_k, skip, StatsWs{parts, out}, st);
   if (s != PSISPEC_OK || skip.mode != kSkipCut) return s;
   // the cut requests' rows: one CTA per row at a time
-  const int smem = static_cast<int>(sizeof(CutSmem));
+  const int smem = static_cast<int>(sizeof(CutSmem<T>));
   if (cudaFuncSetAttribute(cut_rows_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return PSISPEC_ERR_CUDA;
   CutArgs a{};

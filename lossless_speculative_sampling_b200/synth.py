@@ -15,7 +15,8 @@ section 5.1; these synthetic rows stand in for the verifier and drafter heads):
                                   request, T=1, top-p 0.95
   tree     B=4 tries x 64 nodes, depth <= 8, branching <= 4, bf16, rows as "tiny" (target
                                   N(0, 2^2), draft noise 0.5), child tokens drawn without
-                                  replacement from the parent's draft distribution
+                                  replacement from the parent's draft distribution; tree_deep the
+                                  same with draft = target (walks to full depth)
   sweep    B in {1, 32, 256}, K=32, V=151936, bf16, draft std 0.5, T in {0, 0.7, 1}, top-p 0.9
   trie     the tree sampler's candidate trie: B=16 requests, K=15 drafted positions (a block of
            16 whose first token is the verifier's), V=151936, bf16, draft rows N(0, 2^2), T=1;
@@ -87,7 +88,11 @@ def linear_cases():
 
 
 def tree_cases():
-    return {"tree": TreeCase("tree", 4, 64, 8, 4, V_QWEN, torch.bfloat16, 2.0, 0.5, 1.0, 1.0, seed=1003)}
+    return {
+        "tree": TreeCase("tree", 4, 64, 8, 4, V_QWEN, torch.bfloat16, 2.0, 0.5, 1.0, 1.0, seed=1003),
+        # the drafter equal to the verifier: every first child is accepted, walks reach full depth
+        "tree_deep": TreeCase("tree_deep", 4, 64, 8, 4, V_QWEN, torch.bfloat16, 2.0, 0.0, 1.0, 1.0, seed=1007),
+    }
 
 
 def uniforms(shape, seed: int) -> torch.Tensor:

@@ -427,7 +427,9 @@ def _sampled(B, n):
     return np.unique(np.linspace(0, B - 1, n).astype(int))
 
 
-@pytest.mark.parametrize("name", ["mid", "max", "sweep_b32_t0", "sweep_b32_t0.7", "sweep_b1_t1", "mid_topk"])
+@pytest.mark.parametrize("name", ["mid", "max", "sweep_b32_t0", "sweep_b32_t0.7", "sweep_b32_t1", "sweep_b1_t0",
+                                  "sweep_b1_t0.7", "sweep_b1_t1", "sweep_b256_t0", "sweep_b256_t0.7", "sweep_b256_t1",
+                                  "mid_topk"])
 def test_full_size_linear_sampled(name):
     case = synth.linear_cases()[name]
     B, K, V = case.B, case.K, case.V
@@ -461,8 +463,9 @@ def test_full_size_linear_sampled(name):
     print(name, stats_report, "gpu mean accept", lens.mean())
 
 
-def test_full_size_tree():
-    case = synth.tree_cases()["tree"]
+@pytest.mark.parametrize("name", ["tree", "tree_deep"])
+def test_full_size_tree(name):
+    case = synth.tree_cases()[name]
     trie, tgt, drf, toks, ua, ur = synth.tree_inputs(case, device=DEV)
     B = case.B
     Ts, Ps = torch.full((B,), case.temperature), torch.full((B,), case.top_p)
@@ -472,7 +475,25 @@ def test_full_size_tree():
                              Ts.numpy(), Ps.numpy(), case.max_depth)
     rep = check_tree(out, ora, tgt.cpu(), drf.cpu(), trie.node_offsets, trie.parent, toks, ua, ur, Ts, Ps,
                      case.max_depth, label="full-size tree")
-    print("tree", rep, "accept", out["accept_len"].tolist())
+    print(name, rep, "accept", out["accept_len"].tolist())
+    if name == "tree_deep":  # q == p: every first child is accepted down to a leaf
+        assert (out["accept_len"].cpu() >= 1).all()
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_tree_walk_single_cta_fallback(dtype):
+    """V too large for the cluster walk's shared-memory slices (16 or 8 CTAs): the walk runs
+    one CTA per trie (tree_walk_kernel) on the statistics pass's records."""
+    B, nodes, V = 2, 8, 500_000
+    trie, tgt, drf, toks, ua, ur = _tree_inputs(B, nodes, V, dtype, 1.0, 1.0, seed=77)
+    for T, P in ((1.0, 1.0), (0.8, 0.9)):
+        Ts, Ps = torch.full((B,), T), torch.full((B,), P)
+        out = psispec.verify_tree(_cuda(tgt), _cuda(drf), _cuda(trie.node_offsets), _cuda(trie.parent), _cuda(toks),
+                                  _cuda(ua), _cuda(ur), _cuda(Ts), _cuda(Ps), 6)
+        ora = oracle.verify_tree(tgt, drf, trie.node_offsets.numpy(), trie.parent.numpy(), toks.numpy(), ua, ur,
+                                 Ts.numpy(), Ps.numpy(), 6)
+        check_tree(out, ora, tgt, drf, trie.node_offsets, trie.parent, toks, ua, ur, Ts, Ps, 6,
+                   label="single-CTA walk V=%d %s T=%g P=%g" % (V, dtype, T, P))
 
 
 # ------------------------------------------------------------------ top-k: mixed requests and negative rows
@@ -575,8 +596,8 @@ def test_row_stats_topk_parity(dtype):
 def _edge_rows(V, n_rows, g):
     """bf16 draft-like rows that stress the one-pass cut path: the row maximum arriving last
     (far above, and just above, what the first values set), spikes in several warps' ranges,
-    rows of huge negative logits (the window reaches the keys of -inf), a row of -inf with one
-    finite value, a NaN row, and plain rows."""
+    rows of huge negative logits (the window reaches the keys of -inf) and of huge positive ones,
+    a row of -inf with one finite value, a NaN row, and a row whose first half is -inf."""
     x = torch.randn((n_rows, V), generator=g) * 2.0
     x[0, V - 3] = 60.0                    # the maximum last, many binades above the rest
     x[1, V - 1] = 9.0                     # just above the usual maximum, at the very end
@@ -586,6 +607,7 @@ def _edge_rows(V, n_rows, g):
     x[4, V // 2] = 1.0                    # one finite value
     x[5, min(17, V - 1)] = float("nan")   # a data error
     x[6, :V // 2] = -float("inf")         # the first half -inf: the first warps see no finite value
+    x[7] = 3.0e38 - x[7].abs() * 1.0e36   # huge positive logits (their products with log2(e)/T overflow)
     return x.to(torch.bfloat16)
 
 
