@@ -255,10 +255,10 @@ __device__ __forceinline__ CrRange cr_range(const T* rp, int V, int w) {
 
 // Warp w streams its range of row rp (bf16) into L and its ring. Not inlined: the streaming
 // loop gets the registers to itself, apart from the row-end work of the caller.
-__device__ __noinline__ void cr_stream(const __nv_bfloat16* __restrict__ rp, int V, const CrRange r, float c,
-                                       CrLane& Lout, uint32_t* ring) {
+__device__ __noinline__ CrLane cr_stream(const __nv_bfloat16* __restrict__ rp, int V, const CrRange r, float c,
+                                         uint32_t* ring) {
   const int lane = threadIdx.x & 31;
-  CrLane L = Lout;  // in registers for the loop
+  CrLane L{-INFINITY, 0.0f, 0.0, false, 0u, 0u, 0u, false, 0u, 0u};
   L.dl = static_cast<uint32_t>(kCrRing + lane) << 16;
   L.ra = smem_u32(ring);
   constexpr uint32_t kNegInf2 = 0xFF80FF80u;  // packed bf16 pair (-inf, -inf)
@@ -299,7 +299,7 @@ __device__ __noinline__ void cr_stream(const __nv_bfloat16* __restrict__ rp, int
     cr_absorb(L, B, c, ring);
   }
   __syncwarp();  // the ring's reductions are complete before the caller's barrier
-  Lout = L;
+  return L;
 }
 
 // The count of window key `key` in the warps' rings (warps without a finite value add nothing;
@@ -431,8 +431,7 @@ __device__ void cut_rows_cta(const T* __restrict__ A, const T* __restrict__ Bt, 
       uint32_t* ring = sm.ring[warp];
       // every warp streams its range
       const CrRange r = cr_range(rp, V, warp);
-      CrLane L{-INFINITY, 0.0f, 0.0, false, 0u, 0u, 0u, false, 0u, 0u};
-      cr_stream(reinterpret_cast<const __nv_bfloat16*>(rp), V, r, c, L, ring);
+      const CrLane L = cr_stream(reinterpret_cast<const __nv_bfloat16*>(rp), V, r, c, ring);
       // the warp: its maximum, and the lanes' sums brought to it
       const float mw = warp_max(L.M);
       const double sw = warp_sum(L.M > -INFINITY ? L.s * static_cast<double>(ex2((L.M - mw) * c)) : 0.0);
@@ -537,12 +536,15 @@ __device__ void cut_rows_cta(const T* __restrict__ A, const T* __restrict__ Bt, 
 
 // Row statistics of the cut requests' rows alone (psispec_row_stats): one CTA per row at a
 // time.
+// (The argument structs are grid constants: the helpers take them by reference without a
+// per-thread copy in local memory.)
 template <typename T>
-__global__ void __launch_bounds__(kCrThreads, kRowCtas<T>) cut_rows_kernel(const T* __restrict__ A, CutArgs a,
+__global__ void __launch_bounds__(kCrThreads, kRowCtas<T>) cut_rows_kernel(const T* __restrict__ A,
+                                                                const __grid_constant__ CutArgs a,
+                                                                const __grid_constant__ VerifyArgs va,
                                                                 const Partial* __restrict__ parts) {
   extern __shared__ __align__(16) unsigned char cut_smem_raw[];
-  VerifyArgs none{};
-  cut_rows_cta<T>(A, nullptr, a, none, parts, nullptr, blockIdx.x, gridDim.x, *reinterpret_cast<CutSmem<T>*>(cut_smem_raw));
+  cut_rows_cta<T>(A, nullptr, a, va, parts, nullptr, blockIdx.x, gridDim.x, *reinterpret_cast<CutSmem<T>*>(cut_smem_raw));
 }
 
 // The row kernel of sample_draft. CTAs [0, warp_ctas) finish the rows without a cut, one
@@ -557,7 +559,9 @@ __global__ void __launch_bounds__(kTpThreads, kRowCtas<T>) sample_rows_kernel(co
                                                                    const Partial* __restrict__ parts,
                                                                    RowStat* __restrict__ stats,
                                                                    int32_t* __restrict__ out_tokens,
-                                                                   float* __restrict__ out_q, int warp_ctas) {
+                                                                   float* __restrict__ out_q, int warp_ctas,
+                                                                   const __grid_constant__ CutArgs a,
+                                                                   const __grid_constant__ VerifyArgs va) {
   if (static_cast<int>(blockIdx.x) < warp_ctas) {
     const int row = blockIdx.x * kTpWarps + (threadIdx.x >> 5);
     if (row < rows && !request_cut(temperature, top_p, top_k, row / K, V))
@@ -565,23 +569,7 @@ __global__ void __launch_bounds__(kTpThreads, kRowCtas<T>) sample_rows_kernel(co
     return;
   }
   extern __shared__ __align__(16) unsigned char cut_smem_raw[];
-  CutArgs a{};
-  a.mode = kCutSample;
-  a.V = V;
-  a.rows_a = rows;
-  a.per_a = K;
-  a.rows_b = 0;
-  a.per_b = 1;
-  a.temperature = temperature;
-  a.top_p = top_p;
-  a.top_k = top_k;
-  a.u = u;
-  a.out_tokens = out_tokens;
-  a.out_q = out_q;
-  a.stats_a = stats;
-  a.stats_b = nullptr;
-  VerifyArgs none{};
-  cut_rows_cta<T>(draft, nullptr, a, none, parts, nullptr, static_cast<int>(blockIdx.x) - warp_ctas,
+  cut_rows_cta<T>(draft, nullptr, a, va, parts, nullptr, static_cast<int>(blockIdx.x) - warp_ctas,
                   static_cast<int>(gridDim.x) - warp_ctas, *reinterpret_cast<CutSmem<T>*>(cut_smem_raw));
 }
 
@@ -591,8 +579,9 @@ __global__ void __launch_bounds__(kTpThreads, kRowCtas<T>) sample_rows_kernel(co
 // request runs its accept tests and writes the draw job.
 template <typename T>
 __global__ void __launch_bounds__(kTpThreads, kRowCtas<T>) verify_rows_kernel(const T* __restrict__ tgt,
-                                                                   const T* __restrict__ drf, VerifyArgs va,
-                                                                   int warp_ctas) {
+                                                                   const T* __restrict__ drf,
+                                                                   const __grid_constant__ VerifyArgs va,
+                                                                   const __grid_constant__ CutArgs a, int warp_ctas) {
   const int K = va.K, V = va.V;
   const int rows_t = va.B * (K + 1);
   const int rows = rows_t + (va.stream_draft ? va.B * K : 0);
@@ -603,18 +592,6 @@ __global__ void __launch_bounds__(kTpThreads, kRowCtas<T>) verify_rows_kernel(co
     return;
   }
   extern __shared__ __align__(16) unsigned char cut_smem_raw[];
-  CutArgs a{};
-  a.mode = kCutVerify;
-  a.V = V;
-  a.rows_a = rows_t;
-  a.per_a = K + 1;
-  a.rows_b = va.stream_draft ? va.B * K : 0;
-  a.per_b = K;
-  a.temperature = va.temperature;
-  a.top_p = va.top_p;
-  a.top_k = va.top_k;
-  a.stats_a = va.stats_t;
-  a.stats_b = va.stats_d;
   cut_rows_cta<T>(tgt, drf, a, va, va.parts_t, va.parts_d, static_cast<int>(blockIdx.x) - warp_ctas,
                   static_cast<int>(gridDim.x) - warp_ctas, *reinterpret_cast<CutSmem<T>*>(cut_smem_raw));
 }

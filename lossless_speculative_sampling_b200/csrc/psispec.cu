@@ -288,8 +288,23 @@ psispec_status sample_draft_impl(const T* draft, int B, int K, int V, const floa
   unsigned tgrid = 1;
   if ((s = prepare_topp<T>(sample_rows_kernel<T>, rows, &tgrid)) != PSISPEC_OK) return s;
   const int warp_ctas = static_cast<int>((rows + kTpWarps - 1) / kTpWarps);
+  CutArgs ca{};
+  ca.mode = kCutSample;
+  ca.V = V;
+  ca.rows_a = static_cast<int>(rows);
+  ca.per_a = K;
+  ca.rows_b = 0;
+  ca.per_b = 1;
+  ca.temperature = temperature;
+  ca.top_p = top_p;
+  ca.top_k = top_k;
+  ca.u = u;
+  ca.out_tokens = out_tokens;
+  ca.out_q = out_q;
+  ca.stats_a = stats;
   return launch(sample_rows_kernel<T>, warp_ctas + tgrid, kTpThreads, sizeof(CutSmem<T>), st, draft, K, V,
-                static_cast<int>(rows), temperature, top_p, top_k, u, w.st.parts, stats, out_tokens, out_q, warp_ctas);
+                static_cast<int>(rows), temperature, top_p, top_k, u, w.st.parts, stats, out_tokens, out_q, warp_ctas,
+                ca, VerifyArgs{});
 }
 
 template <typename T>
@@ -336,7 +351,19 @@ psispec_status verify_linear_impl(const T* tgt, const T* drf, int B, int K, int 
   unsigned tgrid = 1;
   if ((s = prepare_topp<T>(verify_rows_kernel<T>, rows_t + rows_d, &tgrid)) != PSISPEC_OK) return s;
   const int warp_ctas = static_cast<int>((rows_t + rows_d + kTpWarps - 1) / kTpWarps);
-  s = launch(verify_rows_kernel<T>, warp_ctas + tgrid, kTpThreads, sizeof(CutSmem<T>), st, tgt, drf, a, warp_ctas);
+  CutArgs ca{};
+  ca.mode = kCutVerify;
+  ca.V = V;
+  ca.rows_a = static_cast<int>(rows_t);
+  ca.per_a = K + 1;
+  ca.rows_b = static_cast<int>(rows_d);
+  ca.per_b = K;
+  ca.temperature = temperature;
+  ca.top_p = top_p;
+  ca.top_k = top_k;
+  ca.stats_a = a.stats_t;
+  ca.stats_b = a.stats_d;
+  s = launch(verify_rows_kernel<T>, warp_ctas + tgrid, kTpThreads, sizeof(CutSmem<T>), st, tgt, drf, a, ca, warp_ctas);
   if (s != PSISPEC_OK) return s;
   return launch_draws<T>(tgt, drf, V, B, w.t.parts, w.jobs, w.draw_tc, w.draw_tg, out_tokens, st);
 }
@@ -433,7 +460,7 @@ psispec_status row_stats_impl(const T* logits, int B, int K, int V, const float*
   a.top_k = top_k;
   a.stats_a = out;
   return launch(cut_rows_kernel<T>, static_cast<unsigned>(want_slots(rows, 1, cut_rows_kernel<T>, kCrThreads, smem)),
-                kCrThreads, smem, st, logits, a, static_cast<const Partial*>(parts));
+                kCrThreads, smem, st, logits, a, VerifyArgs{}, static_cast<const Partial*>(parts));
 }
 
 struct TrieWs {
