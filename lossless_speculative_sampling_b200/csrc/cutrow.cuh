@@ -44,7 +44,7 @@ constexpr int kCrWarps = 8;                   // warps per CTA, each one contigu
 constexpr int kCrThreads = kCrWarps * 32;
 constexpr int kCrHead = 256;                  // keys of headroom above a warp's maximum at its ring's top
 constexpr int kCrRing = kTpWindow + kCrHead;  // counters per warp
-constexpr int kCrVec = 4;                     // 16-byte vectors per lane per step
+constexpr int kCrVec = 6;                     // 16-byte vectors per lane per step
 static_assert(kCrRing % 32 == 0, "ring shifts move 32 counters per step");
 
 enum CutMode : int { kCutSample = 0, kCutVerify = 1, kCutStats = 2 };
