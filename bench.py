@@ -45,12 +45,13 @@ def _peaks():
         return 6650.0, "fallback"
 
 
-def _kernel_source_hash():
-    """Hash of the kernel sources with their comments removed (a comment edit leaves the
-    captured traffic valid; any code change invalidates it)."""
+def _kernel_source_hash(files=None):
+    """Hash of the kernel sources (all of them, or the named files that define one kernel)
+    with their comments removed: a comment edit leaves the captured traffic valid; any code
+    change invalidates it."""
     h = hashlib.sha256()
     d = os.path.join(ROOT, "lossless_speculative_sampling_b200", "csrc")
-    for f in sorted(os.listdir(d)):
+    for f in sorted(files or os.listdir(d)):
         with open(os.path.join(d, f)) as fh:
             src = fh.read()
         src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
@@ -66,7 +67,7 @@ def _traffic(workload):
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
             t = json.load(f)
         e = t.get(workload)
-        if e and e.get("source_hash") == _kernel_source_hash():
+        if e and e.get("source_hash") == _kernel_source_hash(e.get("source_files")):
             return e.get("bytes_per_call")
     except Exception:
         pass
