@@ -18,11 +18,13 @@ section 5.1; these synthetic rows stand in for the verifier and drafter heads):
                                   replacement from the parent's draft distribution; tree_deep the
                                   same with draft = target (walks to full depth)
   sweep    B in {1, 32, 256}, K=32, V=151936, bf16, draft std 0.5, T in {0, 0.7, 1}, top-p 0.9
-  trie     the tree sampler's candidate trie: B=16 requests, K=15 drafted positions (a block of
-           16 whose first token is the verifier's), V=151936, bf16, draft rows N(0, 2^2), T=1;
-           cand_k=32 candidates per position, 32 kept prefixes (review page section 3.4's
-           single-request optimum) or 60 (the README's tree example); the verifier row of a
-           node at depth d is the draft row of position d plus N(0, 0.5^2)
+  trie     the tree sampler's candidate trie: B=16 requests (trie_32_b1: one, the operating
+           point's own batch), K=15 drafted positions (a block of 16 whose first token is the
+           verifier's), V=151936, bf16, draft rows N(0, 1) plus 14 * r^-1.1 on the token of rank r
+           of a seeded per-row ranking (peaked: the rank-1 token holds about 0.8 of a row's
+           mass), T=1; cand_k=32 candidates per position, 32 kept prefixes (review page section
+           3.4's single-request optimum) or 60 (the README's tree example); the verifier row of
+           a node at depth d is the draft row of position d plus N(0, 0.5^2)
 
 Uniforms are fp32 values k * 2^-24 (k a uniform 24-bit integer from numpy's PCG64), so fp32
 and fp64 consumers see the same numbers.
@@ -130,21 +132,34 @@ class TrieCase:
     cand_k: int
     n_prefixes: int
     seed: int = 0
+    zipf_bias: float = 0.0  # amplitude of a per-row rank bias; 0 disables it
+    zipf_exponent: float = 1.1
 
 
 def trie_cases():
     bf = torch.bfloat16
+    # peaked rows: the rank-1 token of a row holds about 0.8 of its mass (bias 14 over
+    # N(0, 1) logits of 151936 tokens), the next ranks fall off as r^-1.1
     return {
-        "trie_32": TrieCase("trie_32", 16, 15, V_QWEN, bf, 2.0, 0.5, 1.0, 1.0, 32, 32, seed=1005),
-        "trie_60": TrieCase("trie_60", 16, 15, V_QWEN, bf, 2.0, 0.5, 1.0, 1.0, 32, 60, seed=1006),
+        "trie_32": TrieCase("trie_32", 16, 15, V_QWEN, bf, 1.0, 0.5, 1.0, 1.0, 32, 32, seed=1005, zipf_bias=14.0),
+        "trie_60": TrieCase("trie_60", 16, 15, V_QWEN, bf, 1.0, 0.5, 1.0, 1.0, 32, 60, seed=1006, zipf_bias=14.0),
+        # the single-request operating point itself (batch 1)
+        "trie_32_b1": TrieCase("trie_32_b1", 1, 15, V_QWEN, bf, 1.0, 0.5, 1.0, 1.0, 32, 32, seed=1008, zipf_bias=14.0),
     }
 
 
 def trie_draft(case: TrieCase, device="cpu"):
-    """Draft rows [B, K, V] of the candidate-trie workload."""
+    """Draft rows [B, K, V] of the candidate-trie workload: N(0, draft_std^2) logits plus, with
+    zipf_bias, bias * r^-exponent on the token of rank r of a seeded per-row ranking."""
     dev = torch.device(device)
     g = _gen(dev, case.seed)
     d = torch.randn((case.B, case.K, case.V), generator=g, device=dev, dtype=torch.float32) * case.draft_std
+    if case.zipf_bias:
+        bias = case.zipf_bias * torch.arange(1, case.V + 1, device=dev, dtype=torch.float32).pow(-case.zipf_exponent)
+        for b in range(case.B):
+            for k in range(case.K):
+                perm = torch.randperm(case.V, generator=g, device=dev)
+                d[b, k, perm] += bias
     return d.to(case.dtype)
 
 
