@@ -490,11 +490,13 @@ psispec_status build_tree_impl(const T* draft, int B, int K, int V, const float*
   const int64_t rows = int64_t(B) * K;
   Carver c(ws);
   TrieWs w = carve_trie(c, rows, V);
+  // rows of requests with T > 0 and no cut: the candidate kernel finds their statistics itself
   psispec_status s = launch_stats<T>(one_tensor(draft, rows, K, B), rows, V, temperature, B, top_p, top_k,
-                                     Skip{top_p, top_k, kSkipNone}, w.st, st);
+                                     Skip{top_p, top_k, kSkipUncut}, w.st, st);
   if (s != PSISPEC_OK) return s;
-  s = launch(trie_candidates_kernel<T>, static_cast<unsigned>(rows), kTrieThreads, 0, st, draft, V,
-             static_cast<const RowStat*>(w.st.stats), cand_k, w.cand_tok, w.cand_q, w.cand_l, w.ncand);
+  s = launch(trie_candidates_kernel<T>, static_cast<unsigned>(rows), kTrieThreads, 0, st, draft, K, V,
+             static_cast<const RowStat*>(w.st.stats), 1, temperature, top_p, top_k, cand_k, w.cand_tok, w.cand_q,
+             w.cand_l, w.ncand);
   if (s != PSISPEC_OK) return s;
   return launch(trie_select_kernel, static_cast<unsigned>(B), 32, 0, st, K, n_prefixes,
                 static_cast<const int32_t*>(w.cand_tok), static_cast<const double*>(w.cand_q),

@@ -87,20 +87,53 @@ __device__ __forceinline__ TrieGeom trie_geom(const T* rp, int V) {
   return g;
 }
 
-// Maximum of the 8 (bf16) or 4 (fp32) values of one 16-byte vector, folded into m.
+// Maximum of the 8 (bf16) or 4 (fp32) values of one 16-byte vector, folded into m. NaN
+// propagates (a row that reaches this pass with one is a data error: rows with statistics
+// from the statistics pass have none, and the rows found here check).
 __device__ __forceinline__ void vmax_fold(const uint4& v, __nv_bfloat162& m, const __nv_bfloat16*) {
-  m = __hmax2(m, *reinterpret_cast<const __nv_bfloat162*>(&v.x));
-  m = __hmax2(m, *reinterpret_cast<const __nv_bfloat162*>(&v.y));
-  m = __hmax2(m, *reinterpret_cast<const __nv_bfloat162*>(&v.z));
-  m = __hmax2(m, *reinterpret_cast<const __nv_bfloat162*>(&v.w));
+  m = __hmax2_nan(m, *reinterpret_cast<const __nv_bfloat162*>(&v.x));
+  m = __hmax2_nan(m, *reinterpret_cast<const __nv_bfloat162*>(&v.y));
+  m = __hmax2_nan(m, *reinterpret_cast<const __nv_bfloat162*>(&v.z));
+  m = __hmax2_nan(m, *reinterpret_cast<const __nv_bfloat162*>(&v.w));
 }
 __device__ __forceinline__ void vmax_fold(const uint4& v, float& m, const float*) {
-  m = fmaxf(m, fmaxf(fmaxf(__uint_as_float(v.x), __uint_as_float(v.y)), fmaxf(__uint_as_float(v.z), __uint_as_float(v.w))));
+  m = fmax_nan(m, fmax_nan(fmax_nan(__uint_as_float(v.x), __uint_as_float(v.y)),
+                           fmax_nan(__uint_as_float(v.z), __uint_as_float(v.w))));
 }
 __device__ __forceinline__ float vmax_value(const __nv_bfloat162& m) {
-  return fmaxf(__low2float(m), __high2float(m));
+  return fmax_nan(__low2float(m), __high2float(m));
 }
 __device__ __forceinline__ float vmax_value(float m) { return m; }
+__device__ __forceinline__ void vmax_merge(__nv_bfloat162& m, const __nv_bfloat162& x) { m = __hmax2_nan(m, x); }
+__device__ __forceinline__ void vmax_merge(float& m, float x) { m = fmax_nan(m, x); }
+
+// Sum of the weights 2^((x - M) c) of one 16-byte vector (8 bf16 or 4 fp32 values), each the
+// arithmetic of kept_weight, summed in fp32.
+__device__ __forceinline__ float vweight_sum(const uint4& v, float M, float c, const __nv_bfloat16*) {
+  float x[8], w[8];
+  Vec<__nv_bfloat16>::unpack(v, x);
+  exp8(x, M, c, w);
+  return sum8(w);
+}
+__device__ __forceinline__ float vweight_sum(const uint4& v, float M, float c, const float*) {
+  return ex2((__uint_as_float(v.x) - M) * c) + ex2((__uint_as_float(v.y) - M) * c) +
+         (ex2((__uint_as_float(v.z) - M) * c) + ex2((__uint_as_float(v.w) - M) * c));
+}
+
+// A lane's running maximum M of the values it has seen and its fp64 sum of 2^((x - M) c),
+// rescaled when M grows.
+struct TrieLaneSum {
+  float M;
+  double s;
+  bool bad;  // a NaN or +inf seen
+  __device__ __forceinline__ void grow(float mx, float c) {
+    bad |= !(mx < INFINITY) && !(mx == -INFINITY);
+    if (mx > M && mx < INFINITY) {
+      if (M > -INFINITY) s *= static_cast<double>(ex2((M - mx) * c));
+      M = mx;
+    }
+  }
+};
 
 template <typename T>
 struct VmaxAcc;
@@ -226,31 +259,38 @@ __device__ int trie_general_select(const T* __restrict__ rp, int V, const RowSta
 }
 
 // Candidates of draft row `row`: cand_tok[row, r], cand_q[row, r] and their logits cand_l[row,
-// r] for r < ncand[row] in rank order; ncand = -1 for a row with a data error.
+// r] for r < ncand[row] in rank order; ncand = -1 for a row with a data error. With `lazy`,
+// the rows of requests with T > 0 and no cut (no top-p, no top-k) take their statistics from
+// the kernel's own pass: every lane keeps its running maximum and sum of weights while it
+// finds its block maxima, and the block combines them (a NaN or +inf anywhere, or no finite
+// value, is a data error; every element is kept). The other rows read `stats`.
 template <typename T>
-__global__ void __launch_bounds__(kTrieThreads, 2) trie_candidates_kernel(const T* __restrict__ draft, int V,
-                                                                          const RowStat* __restrict__ stats,
-                                                                          int cand_k, int32_t* __restrict__ cand_tok,
-                                                                          double* __restrict__ cand_q,
-                                                                          double* __restrict__ cand_l,
-                                                                          int32_t* __restrict__ ncand) {
+__global__ void __launch_bounds__(kTrieThreads, 2) trie_candidates_kernel(
+    const T* __restrict__ draft, int K, int V, const RowStat* __restrict__ stats, int lazy,
+    const float* __restrict__ temperature, const float* __restrict__ top_p, const int32_t* __restrict__ top_k,
+    int cand_k, int32_t* __restrict__ cand_tok, double* __restrict__ cand_q, double* __restrict__ cand_l,
+    int32_t* __restrict__ ncand) {
   constexpr int N = Vec<T>::N;
   using Acc = VmaxAcc<T>;
   __shared__ TrieCandSmem smu;
   __shared__ int sel_idx[kTrieMaxCand];
+  __shared__ double red_s[32];
+  __shared__ float red_m[32];
   TrieFastSmem& sm = smu.fast;
   const int64_t row = blockIdx.x;
+  const int req = static_cast<int>(row / K);
   const T* rp = draft + row * static_cast<int64_t>(V);
-  const RowStat st = stats[row];
+  const bool own = lazy && uncut_request(temperature, top_p, req) && request_k(top_k, req, V) == 0;
+  RowStat st = own ? RowStat{} : stats[row];
   int32_t* tok = cand_tok + row * kTrieMaxCand;
   double* qo = cand_q + row * kTrieMaxCand;
   double* lo = cand_l + row * kTrieMaxCand;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  if (st.status != 0) {
+  if (!own && st.status != 0) {
     if (threadIdx.x == 0) ncand[row] = -1;
     return;
   }
-  if (st.c == 0.0f) {  // greedy: a point mass on the argmax
+  if (!own && st.c == 0.0f) {  // greedy: a point mass on the argmax
     if (threadIdx.x == 0) {
       tok[0] = st.amax;
       qo[0] = 1.0;
@@ -259,12 +299,13 @@ __global__ void __launch_bounds__(kTrieThreads, 2) trie_candidates_kernel(const 
     }
     return;
   }
-  // eligible: kept by the row's threshold and above -inf
-  const uint32_t floor_key = max(st.tau, 0x00800000u);
   const TrieGeom g = trie_geom(rp, V);
   const uint4 ninf = make_uint4(Acc::kNegInfWord, Acc::kNegInfWord, Acc::kNegInfWord, Acc::kNegInfWord);
 
-  // pass 1: the maximum of every lane block
+  // pass 1: the maximum of every lane block (and, for a row whose statistics are found here,
+  // the lane's running maximum and sum of weights)
+  const float c_own = own ? temp_scale(temperature[req]) : 0.0f;
+  TrieLaneSum ls{-INFINITY, 0.0, false};
   for (int i = 0; i < g.bpl; ++i) {
     typename Acc::type m = Acc::init();
     const int s0 = warp * g.spw + i * g.r, s1 = warp * g.spw + min((i + 1) * g.r, g.spw);
@@ -275,21 +316,63 @@ __global__ void __launch_bounds__(kTrieThreads, 2) trie_candidates_kernel(const 
         const int vi = (s * kTrieVec + j) * 32 + lane;
         w[j] = vi < g.nv ? __ldg(reinterpret_cast<const uint4*>(rp + g.a0 + vi * N)) : ninf;
       }
+      typename Acc::type ms = Acc::init();
 #pragma unroll
-      for (int j = 0; j < kTrieVec; ++j) vmax_fold(w[j], m, rp);
+      for (int j = 0; j < kTrieVec; ++j) vmax_fold(w[j], ms, rp);
+      vmax_merge(m, ms);
+      if (own) {  // uniform
+        ls.grow(vmax_value(ms), c_own);
+        if (ls.M > -INFINITY) {
+          float acc = 0.0f;
+#pragma unroll
+          for (int j = 0; j < kTrieVec; ++j) acc += vweight_sum(w[j], ls.M, c_own, rp);
+          ls.s += static_cast<double>(acc);
+        }
+      }
     }
     sm.bkey[(warp * g.bpl + i) * 32 + lane] = fkey(vmax_value(m));
   }
   if (warp == 0) {  // the edge block: [0, a0) to lanes 0..15, [a1, V) to lanes 16..31
     const int v = lane < 16 ? lane : g.a1 + lane - 16;
     const bool in = lane < 16 ? v < g.a0 : v < V;
-    float x = in ? load_elem(rp + v) : -INFINITY;
+    const float xe = in ? load_elem(rp + v) : -INFINITY;
+    if (own && in) {
+      ls.grow(xe, c_own);
+      if (ls.M > -INFINITY) ls.s += static_cast<double>(ex2((xe - ls.M) * c_own));
+    }
+    float x = xe;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+    for (int o = 16; o > 0; o >>= 1) x = fmax_nan(x, __shfl_xor_sync(0xffffffffu, x, o));
     if (lane == 0) sm.bkey[g.nb] = fkey(x);
+  }
+  if (own) {  // the row's statistics from the lanes' (the same order in every thread)
+    const float mw = warp_max(ls.M);
+    const double sw = warp_sum(ls.M > -INFINITY ? ls.s * static_cast<double>(ex2((ls.M - mw) * c_own)) : 0.0);
+    const bool bw = __any_sync(0xffffffffu, ls.bad);
+    if (lane == 0) {
+      red_m[warp] = bw ? NAN : mw;
+      red_s[warp] = sw;
+    }
   }
   if (threadIdx.x == 0) sm.ncand = 0;
   __syncthreads();
+  if (own) {
+    const int nw = blockDim.x >> 5;
+    float M = -INFINITY;
+    for (int w = 0; w < nw; ++w) M = fmax_nan(M, red_m[w]);
+    double S = 0.0;
+    if (M > -INFINITY && M < INFINITY)
+      for (int w = 0; w < nw; ++w)
+        if (red_m[w] > -INFINITY) S += red_s[w] * static_cast<double>(ex2((red_m[w] - M) * c_own));
+    st = RowStat{M, c_own, static_cast<float>(S), static_cast<float>(S), 0u, -1,
+                 (M > -INFINITY && M < INFINITY && S > 0.0 && S < INFINITY) ? 0 : 1, 0};
+    if (st.status != 0) {
+      if (threadIdx.x == 0) ncand[row] = -1;
+      return;
+    }
+  }
+  // eligible: kept by the row's threshold and above -inf
+  const uint32_t floor_key = max(st.tau, 0x00800000u);
 
   // the pivot: at most the cand_k-th largest eligible element (a bf16 value fixes the top 16
   // bits of its key, so two digits find it)
@@ -515,12 +598,32 @@ __global__ void __launch_bounds__(32) trie_select_kernel(int K, int n_prefixes, 
 #pragma unroll
     for (int k = 1; k < kTrieSlots; ++k)
       if (trie_before(sm, of[k], best)) best = of[k];
+    // the lanes' best offers by the top 32 bits of their probabilities (positive doubles order
+    // as their bits): a lead of two or more in those bits is a relative gap of at least 2^-20,
+    // far above rounding, so it decides in the order trie_before gives (of one length,
+    // probability and logit-sum order agree then: the prefixes share their normalisers);
+    // offers within one of the lead go to the full comparison
+    const uint32_t key =
+        best.d == 0 ? 0u : max(1u, static_cast<uint32_t>(__double_as_longlong(best.s) >> 32));
+    const uint32_t kmax = __reduce_max_sync(0xffffffffu, key);
+    if (kmax == 0u) break;  // no offer left
+    const unsigned tied = __ballot_sync(0xffffffffu, key != 0u && key + 1u >= kmax);
+    if (__popc(tied) == 1) {
+      const int src = __ffs(tied) - 1;
+      best.s = __shfl_sync(0xffffffffu, best.s, src);
+      best.l = __shfl_sync(0xffffffffu, best.l, src);
+      const int packed = __shfl_sync(0xffffffffu, best.d | (best.r << 8) | (best.n << 16), src);
+      best.d = packed & 0xFF;
+      best.r = (packed >> 8) & 0xFF;
+      best.n = packed >> 16;
+    } else {
+      if (!(key != 0u && key + 1u >= kmax)) best.d = 0;
 #pragma unroll
-    for (int m = 16; m > 0; m >>= 1) {
-      const TrieOffer other = trie_shfl_xor(best, m);
-      if (trie_before(sm, other, best)) best = other;
+      for (int m = 16; m > 0; m >>= 1) {
+        const TrieOffer other = trie_shfl_xor(best, m);
+        if (trie_before(sm, other, best)) best = other;
+      }
     }
-    if (best.d == 0) break;  // no offer left
     const int p = best.n, d = best.d, r = best.r;
     // the new node nn: its rank path, record, and first offer
     if (lane + 1 < d) sm.node_rank[nn][lane] = sm.node_rank[p][lane];
@@ -735,9 +838,10 @@ __device__ int block_draw_without(const JobRows<T, false>& J, int V, const int* 
 // the final token is drawn from that r with u_resid of the node. No draft row is read, and a
 // rejection needs no pass over the vocabulary. One CTA per trie; ts = statistics records of
 // the verifier rows (every row's, found in parallel beforehand: a walk can be as deep as the
-// block, so no per-node pass sits on its chain). The children are listed by warp ballots,
-// their probabilities and uniforms read in parallel; the accept test runs in child order on
-// one thread from shared memory; the final draw is one coalesced block draw.
+// block, so no per-node pass sits on its chain). Every node's p(token) under its parent's row
+// and its uniform are read by the whole CTA before the walk; the walk itself is one warp
+// (children listed by ballots, the accept tests in child order on one lane, all from shared
+// memory); the final draw is one coalesced block draw.
 template <typename T>
 __global__ void __launch_bounds__(kTreeThreads, 1) tree_walk_det_kernel(
     const T* __restrict__ tgt, int V, const int32_t* __restrict__ offs, const int32_t* __restrict__ parent,
@@ -747,12 +851,13 @@ __global__ void __launch_bounds__(kTreeThreads, 1) tree_walk_det_kernel(
   __shared__ int depth[kMaxNodes];
   __shared__ int spar[kMaxNodes];
   __shared__ int stok[kMaxNodes];
+  __shared__ double pn[kMaxNodes];  // node c's p(token) under its parent's verifier row
+  __shared__ float un[kMaxNodes];   // node c's u_accept
+  __shared__ int rowf[kMaxNodes];   // node c's own row: -2 data error, -1 sampling, else the greedy argmax
   __shared__ int ch[kMaxChildren];
-  __shared__ float chw[kMaxChildren];
-  __shared__ float chu[kMaxChildren];
   __shared__ int removed[kMaxChildren];
   __shared__ DrawSmem dsm;
-  __shared__ int sh_bad, sh_nch, sh_next, sh_y, sh_nrem;
+  __shared__ int sh_bad, sh_cur, sh_len, sh_draw, sh_y, sh_nrem;
   const int b = blockIdx.x;
   const int n0 = offs[b], n = offs[b + 1] - n0;
   int32_t* path = out_path + static_cast<size_t>(b) * max_depth;
@@ -775,16 +880,30 @@ __global__ void __launch_bounds__(kTreeThreads, 1) tree_walk_det_kernel(
       if (depth[c] > max_depth) bad = 1;
     }
     sh_bad = bad;
-    sh_y = -1;
   }
   __syncthreads();
+  if (!sh_bad)
+    for (int c = threadIdx.x; c < n; c += blockDim.x) {
+      const RowStat own = ts[n0 + c];
+      rowf[c] = own.status != 0 ? -2 : (own.c == 0.0f ? own.amax : -1);
+      if (c > 0) {
+        const int pa = spar[c];
+        const RowStat sp = ts[n0 + pa];
+        pn[c] = sp.status == 0 && sp.c != 0.0f
+                    ? static_cast<double>(kept_weight(sp, load_elem(tgt + static_cast<size_t>(n0 + pa) * V + stok[c]))) /
+                          static_cast<double>(sp.s_kept)
+                    : 0.0;
+        un[c] = u_acc[n0 + c];
+      }
+    }
+  __syncthreads();
 
-  int cur = 0, len = 0;
-  while (!sh_bad) {
-    const T* rp = tgt + static_cast<size_t>(n0 + cur) * V;
-    const RowStat sp = ts[n0 + cur];
-    if (threadIdx.x < 32) {  // children of cur in index order (warp ballots)
-      const int lane = threadIdx.x;
+  if (threadIdx.x < 32 && !sh_bad) {  // the walk: one warp
+    const int lane = threadIdx.x;
+    int cur = 0, len = 0, bad = 0, draw = 0, y = -1, nrem = 0;
+    while (true) {
+      const int f = rowf[cur];
+      if (f == -2) { bad = 1; break; }
       int nch = 0;
       for (int c0 = cur + 1; c0 < n; c0 += 32) {
         const int c = c0 + lane;
@@ -794,69 +913,69 @@ __global__ void __launch_bounds__(kTreeThreads, 1) tree_walk_det_kernel(
         if (is && pos < kMaxChildren) ch[pos] = c;
         nch += __popc(m);
       }
+      if (nch > kMaxChildren) { bad = 1; break; }
+      __syncwarp();
+      int next = -1;
       if (lane == 0) {
-        sh_nch = min(nch, kMaxChildren);
-        sh_next = -1;
-        sh_nrem = 0;
-        if (nch > kMaxChildren || sp.status != 0) sh_bad = 1;
-      }
-    }
-    __syncthreads();
-    if (sh_bad) break;
-    const int nch = sh_nch;
-    if (sp.c != 0.0f && static_cast<int>(threadIdx.x) < nch) {
-      const int c = ch[threadIdx.x];
-      chw[threadIdx.x] = kept_weight(sp, load_elem(rp + stok[c]));
-      chu[threadIdx.x] = u_acc[n0 + c];
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      if (sp.c == 0.0f) {  // greedy: follow the child carrying the verifier argmax
-        for (int k = 0; k < nch; ++k)
-          if (stok[ch[k]] == sp.amax) { sh_next = ch[k]; break; }
-        sh_y = sp.amax;
-      } else {
-        double R = 1.0;  // mass of p left
-        int nrem = 0;
-        for (int k = 0; k < nch; ++k) {
-          const int c = ch[k], t = stok[c];
-          bool gone = false;
-          for (int i = 0; i < nrem; ++i) gone |= removed[i] == t;
-          const double pt = gone ? 0.0 : static_cast<double>(chw[k]) / static_cast<double>(sp.s_kept);
-          if (R > 0.0 && static_cast<double>(chu[k]) * R < pt) { sh_next = c; break; }
-          if (!gone) {
-            removed[nrem++] = t;
-            R -= pt;
+        if (f >= 0) {  // greedy: follow the child carrying the verifier argmax
+          for (int k = 0; k < nch; ++k)
+            if (stok[ch[k]] == f) { next = ch[k]; break; }
+          y = f;
+        } else {
+          double R = 1.0;  // mass of p left
+          nrem = 0;
+          for (int k = 0; k < nch; ++k) {
+            const int c = ch[k], t = stok[c];
+            bool gone = false;
+            for (int i = 0; i < nrem; ++i) gone |= removed[i] == t;
+            const double pt = gone ? 0.0 : pn[c];
+            if (R > 0.0 && static_cast<double>(un[c]) * R < pt) { next = c; break; }
+            if (!gone) {
+              removed[nrem++] = t;
+              R -= pt;
+            }
           }
         }
-        // ascending order for the draw
+        if (next >= 0) {
+          path[len] = next;
+          toks[len] = stok[next];
+        }
+      }
+      next = __shfl_sync(0xffffffffu, next, 0);
+      if (next < 0) {
+        draw = f == -1;
+        break;
+      }
+      cur = next;
+      ++len;
+    }
+    if (lane == 0) {
+      if (draw)  // ascending order for the draw
         for (int i = 1; i < nrem; ++i) {
           const int t = removed[i];
           int k = i - 1;
           while (k >= 0 && removed[k] > t) { removed[k + 1] = removed[k]; --k; }
           removed[k + 1] = t;
         }
-        sh_nrem = nrem;
-      }
+      sh_bad = bad;
+      sh_cur = cur;
+      sh_len = len;
+      sh_draw = draw;
+      sh_y = y;
+      sh_nrem = nrem;
     }
-    __syncthreads();
-    if (sh_next >= 0) {
-      if (threadIdx.x == 0) { path[len] = sh_next; toks[len] = stok[sh_next]; }
-      cur = sh_next;
-      ++len;
-      __syncthreads();
-      continue;
-    }
-    if (sp.c == 0.0f) break;  // greedy: final token sh_y
-
-    // final draw from p without the removed tokens
+  }
+  __syncthreads();
+  if (!sh_bad && sh_draw) {  // final draw from p without the removed tokens
+    const int cur = sh_cur;
+    const T* rp = tgt + static_cast<size_t>(n0 + cur) * V;
+    const RowStat sp = ts[n0 + cur];
     JobRows<T, false> J;
     J.init(rp, sp, nullptr, sp);
     const int y = block_draw_without(J, V, removed, sh_nrem, u_res[n0 + cur], dsm);
     if (threadIdx.x == 0) sh_y = y;
-    __syncthreads();
-    break;
   }
+  __syncthreads();
 
   if (threadIdx.x == 0) {
     if (sh_bad) {
@@ -864,6 +983,7 @@ __global__ void __launch_bounds__(kTreeThreads, 1) tree_walk_det_kernel(
       for (int i = 0; i <= max_depth; ++i) toks[i] = -1;
       out_len[b] = -1;
     } else {
+      const int len = sh_len;
       for (int i = len; i < max_depth; ++i) path[i] = -1;
       toks[len] = sh_y;
       for (int i = len + 1; i <= max_depth; ++i) toks[i] = -1;

@@ -248,3 +248,26 @@ def test_verify_tree_det_mixed_requests_and_data_errors(V, dtype):
                       rule=oracle.TREE_DETERMINISTIC)
     compare_tree(out, ora, recheck=rc, limit=band_limit(B, V, 1.0, 2 * trie.N / B),
                  label="deterministic mixed tries V=%d" % V)
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_build_tree_uncut_data_errors(dtype):
+    """Requests sampling with no cut take their row statistics from the candidate kernel's own
+    pass: a NaN, a +inf, or a row without a finite value is a data error of its request only."""
+    B, K, V, n = 4, 3, 5003, 12
+    g = torch.Generator().manual_seed(17)
+    d = torch.randn((B, K, V), generator=g) * 2.0
+    d[0, 1, 4000] = float("nan")
+    d[1, 2, 17] = float("inf")
+    d[2, 0] = -float("inf")
+    d = d.to(dtype)
+    Ts, Ps = torch.ones(B), torch.ones(B)
+    out = psispec.build_tree(d.to(DEV), Ts.to(DEV), Ps.to(DEV), 4, n)
+    got = {k: v.cpu().numpy() for k, v in out.items()}
+    assert list(got["nodes"][:3]) == [-1, -1, -1]
+    assert (got["parent"][:3] == -1).all()
+    ora = oracle.build_tree(d[3].float().numpy().astype(np.float64), 1.0, 1.0, 4, n)
+    m = len(ora["parent"])
+    assert got["nodes"][3] == m
+    assert np.array_equal(got["tokens"][3, :m], ora["tokens"])
+    assert np.array_equal(got["parent"][3, :m], ora["parent"])
