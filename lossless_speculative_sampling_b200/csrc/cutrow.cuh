@@ -292,6 +292,14 @@ __device__ __noinline__ CrLane cr_stream(const __nv_bfloat16* __restrict__ rp, i
   CrStep A;
   for (int s = 0; s < steps; ++s) {
     load(A, s);
+    // the warp's next step (2 KB contiguous) brought into L2 while this one is reduced: its
+    // loads then wait on L2 rather than HBM (measured: 2.03 against 2.10 ms per step of
+    // B=512, K=16, top-p 0.95)
+    if (lane == 0 && s + 1 < steps) {
+      const uint4* pf = body + r.v0 + (s + 1) * kStep;
+      const uint32_t bytes = static_cast<uint32_t>(min(kStep, n - (s + 1) * kStep)) * 16u;
+      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(pf), "r"(bytes) : "memory");
+    }
     cr_absorb(L, A, c, ring);
   }
   __syncwarp();  // the ring's reductions are complete before the caller's barrier
