@@ -11,7 +11,7 @@
 // here the counts are taken in the same pass that finds it.
 //
 // One CTA per row at a time, persistent over the rows, three CTAs per SM. Warp w of the CTA
-// streams a contiguous range of the row once from HBM (four 16-byte loads per lane per step;
+// streams a contiguous range of the row once from HBM (five 16-byte loads per lane per step;
 // the 24 warps of an SM keep the loads in flight) and keeps, over its range:
 //   - the running maximum M (NaN-propagating, bf16 pairs compared packed) and, per lane, the
 //     fp64 sum of 2^((x - M) c), rescaled whenever M grows;
@@ -44,7 +44,7 @@ constexpr int kCrWarps = 8;                   // warps per CTA, each one contigu
 constexpr int kCrThreads = kCrWarps * 32;
 constexpr int kCrHead = 224;                  // keys of headroom above a warp's maximum at its ring's top
 constexpr int kCrRing = kTpWindow + kCrHead;  // counters per warp
-constexpr int kCrVec = 4;                     // 16-byte vectors per lane per step
+constexpr int kCrVec = 5;                     // 16-byte vectors per lane per step
 static_assert(kCrRing % 32 == 0, "ring shifts move 32 counters per step");
 
 enum CutMode : int { kCutSample = 0, kCutVerify = 1, kCutStats = 2 };
@@ -292,7 +292,7 @@ __device__ __noinline__ CrLane cr_stream(const __nv_bfloat16* __restrict__ rp, i
   CrStep A;
   for (int s = 0; s < steps; ++s) {
     load(A, s);
-    // the warp's next step (2 KB contiguous) brought into L2 while this one is reduced: its
+    // the warp's next step (2.5 KB contiguous) brought into L2 while this one is reduced: its
     // loads then wait on L2 rather than HBM (measured: 2.03 against 2.10 ms per step of
     // B=512, K=16, top-p 0.95)
     if (lane == 0 && s + 1 < steps) {
