@@ -10,19 +10,22 @@
 // their normalisers, so they compare exactly by their logit sums (fp64 sums of the input
 // values); prefixes of different lengths compare by their fp64 probabilities.
 //
-// Two kernels after the row statistics of the B*K draft rows:
+// Two kernels after the row statistics of the B*K draft rows (rows of requests with a cut;
+// the others get theirs in the first kernel's pass):
 //   trie_candidates_kernel  one CTA per row: one coalesced pass keeps the maximum of every lane
-//                           block (a lane's elements of a few steps) in shared memory; the
-//                           cand_k-th largest block maximum (an exact radix select over the
-//                           block keys) is a pivot at or below the cand_k-th largest element;
-//                           only the blocks at or above it are read again, their elements at or
-//                           above it are ranked exactly (key, then the lower index) and the
-//                           first cand_k kept. Rows with more elements at the pivot than the
-//                           ranking holds (long runs of equal values) take a general radix
-//                           select instead;
+//                           block (a lane's elements of a few steps) in shared memory (and,
+//                           for a row without a cut, each lane's running maximum and sum of
+//                           weights); the cand_k-th largest block maximum (an exact radix
+//                           select over the block keys) is a pivot at or below the cand_k-th
+//                           largest element; only the blocks at or above it are read again,
+//                           their elements at or above it are ranked exactly (key, then the
+//                           lower index) and the first cand_k kept. Rows with more elements at
+//                           the pivot than the ranking holds (long runs of equal values) take a
+//                           general radix select instead;
 //   trie_select_kernel      one warp per request: best-first choice of the prefixes, one
-//                           offer per kept node (its best child not kept yet) in shared
-//                           memory, the products in fp64.
+//                           offer per kept node (its best child not kept yet) held in lane
+//                           registers, the products in fp64.
+// Then tree_walk_det_kernel verifies such a trie (the deterministic-candidate rule).
 #pragma once
 
 #include <cuda_bf16.h>
