@@ -169,9 +169,10 @@ def trie_verifier_rows(case: TrieCase, draft: torch.Tensor, depth: torch.Tensor)
     B, K, V = draft.shape
     dev = draft.device
     g = _gen(dev, case.seed + 1)
-    dep = depth.to(dev).long().clamp(min=0)
+    dep = depth.to(dev).long()
     base = torch.zeros((B, dep.shape[1], V), dtype=torch.float32, device=dev)
-    has = dep < K
+    has = (dep >= 0) & (dep < K)
+    dep = dep.clamp(min=0)
     idx = dep.clamp(max=K - 1)
     rows = torch.gather(draft.float(), 1, idx.unsqueeze(-1).expand(-1, -1, V))
     base = torch.where(has.unsqueeze(-1), rows, base)
